@@ -1,0 +1,226 @@
+"""CPU oracle for the FP8 training-GEMM path (test infrastructure only).
+
+Only tests/, ``__graft_entry__.smoke()`` and bench.py's ``cpu_baseline`` and
+``--impl reference`` legs may import this package.  It shares no code with the
+CUDA path: the arithmetic lives in ``fp8_oracle.c`` (plain C, fp64); this
+module only marshals numpy arrays into it and composes the relu^2 MLP chain in
+the order the method runs it.
+
+Tensors cross this interface as numpy arrays of raw bits: bf16 as uint16,
+FP8 codes as uint8, all row-major.
+
+The chain (``mlp_fwd`` / ``mlp_bwd``) follows the method described on
+decomputer.nl, "Het trainen van een 3.8B LLM tot 0.384 CORE voor $998":
+section "Vroege experimenten" item 4 and section "Doorvoer (Throughput)
+verhogen" (FP8 with dynamic tensorwise scaling on the forward GEMM and both
+backward GEMMs), with the non-gated relu^2 MLP of the "Niet-gated MLPs" bullet
+and of "Appendix: De configuratie".  Every tensor is quantised once per call
+with one tensorwise scale; the backward reuses the forward's quantised X,
+W_up, W_down and h and their scales.
+
+Parity status: no page prints a numeric value for any cast or GEMM of this
+path, so every value check rests on pins against the format definitions,
+closed forms, brute force and finite differences (tests/test_oracle_*.py).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+E4M3, E5M2 = 0, 1
+EPI_NONE, EPI_RELU2_FWD, EPI_RELU2_BWD = 0, 1, 2
+FP8_MAX = {E4M3: 448.0, E5M2: 57344.0}
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        L.orc_num_threads.restype = ctypes.c_int
+        L.orc_fp8_decode.argtypes = [ctypes.c_uint8, ctypes.c_int]
+        L.orc_fp8_decode.restype = ctypes.c_double
+        L.orc_fp8_encode.argtypes = [ctypes.c_float, ctypes.c_int]
+        L.orc_fp8_encode.restype = ctypes.c_uint8
+        L.orc_bf16_to_double.argtypes = [ctypes.c_uint16]
+        L.orc_bf16_to_double.restype = ctypes.c_double
+        L.orc_bf16_from_double.argtypes = [ctypes.c_double]
+        L.orc_bf16_from_double.restype = ctypes.c_uint16
+        L.orc_amax.argtypes = [P, i64, i64, i64, ctypes.c_int]
+        L.orc_amax.restype = ctypes.c_float
+        L.orc_scale.argtypes = [ctypes.c_float, ctypes.c_int, P, P]
+        L.orc_scale.restype = None
+        L.orc_cast.argtypes = [P, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_float, P, P]
+        L.orc_cast.restype = None
+        L.orc_gemm_acc.argtypes = [P, ctypes.c_int, P, ctypes.c_int, i64, i64, i64, P, i64, P]
+        L.orc_gemm_acc.restype = None
+        L.orc_gemm.argtypes = [P, ctypes.c_int, P, ctypes.c_int, i64, i64, i64, ctypes.c_float,
+                               ctypes.c_float, ctypes.c_int, P, P, i64, P, P]
+        L.orc_gemm.restype = None
+        L.orc_mlp_f64.argtypes = [P, P, P, P, i64, i64, i64, P, P, P, P]
+        L.orc_mlp_f64.restype = None
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == dtype, (a.dtype, dtype)
+    return a
+
+
+def num_threads() -> int:
+    return lib().orc_num_threads()
+
+
+# ------------------------------------------------------------------ codecs
+def fp8_decode(code: int, fmt: int) -> float:
+    return lib().orc_fp8_decode(code, fmt)
+
+
+def fp8_encode(x: float, fmt: int) -> int:
+    return lib().orc_fp8_encode(x, fmt)
+
+
+def fp8_decode_array(codes, fmt):
+    table = np.array([fp8_decode(c, fmt) for c in range(256)], dtype=np.float64)
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+def bf16_to_double(b: int) -> float:
+    return lib().orc_bf16_to_double(b)
+
+
+def bf16_from_double(v: float) -> int:
+    return lib().orc_bf16_from_double(v)
+
+
+def bf16_bits_to_f64(bits):
+    bits = np.asarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# ------------------------------------------------------ amax / scale / cast
+def amax(x, relu2_input=False) -> np.float32:
+    x = _c(x, np.uint16)
+    rows, cols = x.shape
+    return np.float32(lib().orc_amax(_ptr(x), rows, cols, cols, int(relu2_input)))
+
+
+def scale(amax_value, fmt):
+    s = np.zeros(1, np.float32)
+    inv = np.zeros(1, np.float32)
+    lib().orc_scale(float(np.float32(amax_value)), fmt, _ptr(s), _ptr(inv))
+    return s[0], inv[0]
+
+
+def cast(x, fmt, scale_value, relu2_input=False, want_q=True, want_qT=True):
+    """Return (q, qT) codes of a rows x cols bf16 tensor at a given scale."""
+    x = _c(x, np.uint16)
+    rows, cols = x.shape
+    q = np.zeros((rows, cols), np.uint8) if want_q else None
+    qT = np.zeros((cols, rows), np.uint8) if want_qT else None
+    lib().orc_cast(_ptr(x), rows, cols, cols, fmt, int(relu2_input),
+                   float(np.float32(scale_value)), _ptr(q), _ptr(qT))
+    return q, qT
+
+
+def amax_scale_cast(x, fmt, relu2_input=False, amax_in=None):
+    """The full dynamic-scaling cast: amax -> scale -> codes (+ transpose)."""
+    a = amax(x, relu2_input) if amax_in is None else np.float32(amax_in)
+    s, inv = scale(a, fmt)
+    q, qT = cast(x, fmt, s, relu2_input)
+    return dict(amax=a, scale=s, inv_scale=inv, q=q, qT=qT)
+
+
+# ------------------------------------------------------------------- GEMM
+def gemm_acc(A, fa, B, fb, rows=None):
+    """fp64 C = dec(A) dec(B)^T over the listed rows of A (all if None)."""
+    A = _c(A, np.uint8)
+    B = _c(B, np.uint8)
+    M, K = A.shape
+    N, K2 = B.shape
+    assert K == K2
+    r = None if rows is None else _c(np.asarray(rows, dtype=np.int64), np.int64)
+    nr = M if r is None else len(r)
+    C = np.zeros((nr, N), np.float64)
+    lib().orc_gemm_acc(_ptr(A), fa, _ptr(B), fb, M, N, K, _ptr(r), nr, _ptr(C))
+    return C
+
+
+def gemm(A, fa, B, fb, inv_sa, inv_sb, epi=EPI_NONE, aux=None, rows=None):
+    """bf16 D = epi((dec(A) dec(B)^T) inv_sa inv_sb) and the amax of what the
+    next cast consumes.  Returns (D bits, amax)."""
+    A = _c(A, np.uint8)
+    B = _c(B, np.uint8)
+    M, K = A.shape
+    N, K2 = B.shape
+    assert K == K2
+    if epi == EPI_RELU2_BWD:
+        aux = _c(aux, np.uint16)
+        assert aux.shape == (M, N)
+    r = None if rows is None else _c(np.asarray(rows, dtype=np.int64), np.int64)
+    nr = M if r is None else len(r)
+    D = np.zeros((nr, N), np.uint16)
+    am = np.zeros(1, np.float32)
+    lib().orc_gemm(_ptr(A), fa, _ptr(B), fb, M, N, K, float(np.float32(inv_sa)),
+                   float(np.float32(inv_sb)), epi, _ptr(aux), _ptr(r), nr, _ptr(D), _ptr(am))
+    return D, am[0]
+
+
+# -------------------------------------------------------------- MLP chain
+def mlp_fwd(X, W_up, W_down):
+    """relu^2 MLP forward with dynamic tensorwise FP8 scaling.
+
+    X: M x d, W_up: f x d, W_down: d x f (bf16 bits).  Returns a dict holding
+    Y and every intermediate the backward reuses.
+    """
+    cx = amax_scale_cast(X, E4M3)
+    cu = amax_scale_cast(W_up, E4M3)
+    cd = amax_scale_cast(W_down, E4M3)
+    H, amax_h = gemm(cx["q"], E4M3, cu["q"], E4M3, cx["inv_scale"], cu["inv_scale"],
+                     EPI_RELU2_FWD)
+    ch = amax_scale_cast(H, E4M3, relu2_input=True, amax_in=amax_h)
+    Y, amax_y = gemm(ch["q"], E4M3, cd["q"], E4M3, ch["inv_scale"], cd["inv_scale"])
+    return dict(Y=Y, X=cx, W_up=cu, W_down=cd, H=H, h=ch, amax_y=amax_y)
+
+
+def mlp_bwd(dY, saved):
+    """relu^2 MLP backward: dgrad and wgrad of both linears in FP8, e5m2
+    gradients against e4m3 saved operands."""
+    cg = amax_scale_cast(dY, E5M2)
+    cx, cu, cd, ch = saved["X"], saved["W_up"], saved["W_down"], saved["h"]
+    dH, amax_dh = gemm(cg["q"], E5M2, cd["qT"], E4M3, cg["inv_scale"], cd["inv_scale"],
+                       EPI_RELU2_BWD, aux=saved["H"])
+    dW_down, _ = gemm(cg["qT"], E5M2, ch["qT"], E4M3, cg["inv_scale"], ch["inv_scale"])
+    cdh = amax_scale_cast(dH, E5M2, amax_in=amax_dh)
+    dX, _ = gemm(cdh["q"], E5M2, cu["qT"], E4M3, cdh["inv_scale"], cu["inv_scale"])
+    dW_up, _ = gemm(cdh["qT"], E5M2, cx["qT"], E4M3, cdh["inv_scale"], cx["inv_scale"])
+    return dict(dX=dX, dW_up=dW_up, dW_down=dW_down, dY=cg, dH=dH, dh=cdh)
+
+
+def mlp_f64(X, W_up, W_down, dY=None):
+    """Unquantised fp64 relu^2 MLP forward and backward (float64 arrays)."""
+    X = _c(X, np.float64)
+    W_up = _c(W_up, np.float64)
+    W_down = _c(W_down, np.float64)
+    M, d = X.shape
+    f = W_up.shape[0]
+    Y = np.zeros((M, d))
+    out = dict(Y=Y)
+    if dY is not None:
+        dY = _c(dY, np.float64)
+        out.update(dX=np.zeros((M, d)), dW_up=np.zeros((f, d)), dW_down=np.zeros((d, f)))
+    lib().orc_mlp_f64(_ptr(X), _ptr(W_up), _ptr(W_down), _ptr(dY), M, d, f, _ptr(Y),
+                      _ptr(out.get("dX")), _ptr(out.get("dW_up")), _ptr(out.get("dW_down")))
+    return out
