@@ -1,0 +1,157 @@
+"""ctypes binding of libfp8lm.so (include/lm_fp8.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  If the
+library is missing the import fails loudly -- there is no fallback.
+"""
+import ctypes
+import os
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libfp8lm.so")
+
+E4M3, E5M2 = 0, 1
+EPI_NONE, EPI_RELU2_FWD, EPI_RELU2_BWD = 0, 1, 2
+
+STATUS = {0: "LM_OK", 1: "LM_ERR_INVALID_ARG", 2: "LM_ERR_ALIGNMENT",
+          3: "LM_ERR_UNSUPPORTED_SHAPE", 4: "LM_ERR_UNSUPPORTED_FORMAT", 5: "LM_ERR_CUDA",
+          6: "LM_ERR_TIMEOUT", 7: "LM_ERR_NONFINITE"}
+
+EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
+            "lm_relu2_mlp_saved_carve", "lm_relu2_mlp_workspace_size", "lm_relu2_mlp_fwd",
+            "lm_relu2_mlp_bwd", "lm_get_error", "lm_status_string", "lm_version"]
+
+
+class LmError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+class MlpSaved(ctypes.Structure):
+    """Mirror of lm_mlp_saved."""
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("Xq", "XqT", "Wuq", "WuqT", "Wdq", "WdqT", "H", "hq", "hqT", "scales")]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m fp8_gemms_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i64, i32, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int
+    L.lm_fp8_amax_scale_cast.argtypes = [P, i64, i64, i64, i32, i32, P, P, P, P, P, P, P]
+    L.lm_fp8_amax_scale_cast.restype = st
+    L.lm_fp8_gemm.argtypes = [P, i32, P, i32, i64, i64, i64, P, P, i32, P, P, P, P]
+    L.lm_fp8_gemm.restype = st
+    L.lm_relu2_mlp_saved_bytes.argtypes = [i64, i64, i64]
+    L.lm_relu2_mlp_saved_bytes.restype = ctypes.c_size_t
+    L.lm_relu2_mlp_saved_carve.argtypes = [P, ctypes.c_size_t, i64, i64, i64,
+                                           ctypes.POINTER(MlpSaved)]
+    L.lm_relu2_mlp_saved_carve.restype = st
+    L.lm_relu2_mlp_workspace_size.argtypes = [i64, i64, i64]
+    L.lm_relu2_mlp_workspace_size.restype = ctypes.c_size_t
+    L.lm_relu2_mlp_fwd.argtypes = [P, P, P, i64, i64, i64, P, ctypes.POINTER(MlpSaved), P,
+                                   ctypes.c_size_t, P]
+    L.lm_relu2_mlp_fwd.restype = st
+    L.lm_relu2_mlp_bwd.argtypes = [P, ctypes.POINTER(MlpSaved), i64, i64, i64, P, P, P, P,
+                                   ctypes.c_size_t, P]
+    L.lm_relu2_mlp_bwd.restype = st
+    L.lm_get_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    L.lm_get_error.restype = st
+    L.lm_status_string.argtypes = [st]
+    L.lm_status_string.restype = ctypes.c_char_p
+    L.lm_version.restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _check(status, what):
+    if status != 0:
+        raise LmError(status, what)
+
+
+# ------------------------------------------------------- C-ABI mirrors
+def lm_fp8_amax_scale_cast(x, fmt, amax_out, scale_out, inv_scale_out, q=None, qT=None,
+                           relu2_input=False, amax_in=None, stream=None):
+    """x: 2-D bf16 CUDA tensor (row stride = ld).  Scales are 1-element (or
+    sliced) fp32 CUDA tensors.  Raises LmError on a non-zero status."""
+    rows, cols = x.shape
+    ld = x.stride(0) if rows > 1 else cols
+    assert x.dtype == torch.bfloat16 and x.stride(-1) == 1
+    _check(lib.lm_fp8_amax_scale_cast(_p(x), rows, cols, ld, fmt, int(relu2_input), _p(amax_in),
+                                      _p(amax_out), _p(scale_out), _p(inv_scale_out), _p(q),
+                                      _p(qT), _stream(stream)), "lm_fp8_amax_scale_cast")
+
+
+def lm_fp8_gemm(A, fa, B, fb, inv_scale_a, inv_scale_b, D, epi=EPI_NONE, aux=None,
+                amax_out=None, stream=None):
+    """D[M x N] (bf16) = epi(A[M x K] B[N x K]^T * inv_a * inv_b); A, B uint8 codes."""
+    M, K = A.shape
+    N, K2 = B.shape
+    assert K == K2 and tuple(D.shape) == (M, N)
+    _check(lib.lm_fp8_gemm(_p(A), fa, _p(B), fb, M, N, K, _p(inv_scale_a), _p(inv_scale_b), epi,
+                           _p(aux), _p(D), _p(amax_out), _stream(stream)), "lm_fp8_gemm")
+
+
+def lm_relu2_mlp_saved_bytes(M, d, f):
+    return lib.lm_relu2_mlp_saved_bytes(M, d, f)
+
+
+def lm_relu2_mlp_workspace_size(M, d, f):
+    return lib.lm_relu2_mlp_workspace_size(M, d, f)
+
+
+def lm_relu2_mlp_saved_carve(buf, M, d, f):
+    s = MlpSaved()
+    _check(lib.lm_relu2_mlp_saved_carve(_p(buf), buf.numel() * buf.element_size(), M, d, f,
+                                        ctypes.byref(s)), "lm_relu2_mlp_saved_carve")
+    return s
+
+
+def lm_relu2_mlp_fwd(X, W_up, W_down, Y, saved, stream=None):
+    M, d = X.shape
+    f = W_up.shape[0]
+    _check(lib.lm_relu2_mlp_fwd(_p(X), _p(W_up), _p(W_down), M, d, f, _p(Y),
+                                ctypes.byref(saved), None, 0, _stream(stream)),
+           "lm_relu2_mlp_fwd")
+
+
+def lm_relu2_mlp_bwd(dY, saved, dX, dW_up, dW_down, workspace, stream=None):
+    M, d = dY.shape
+    f = dW_up.shape[0]
+    _check(lib.lm_relu2_mlp_bwd(_p(dY), ctypes.byref(saved), M, d, f, _p(dX), _p(dW_up),
+                                _p(dW_down), _p(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream)),
+           "lm_relu2_mlp_bwd")
+
+
+def lm_get_error(stream=None):
+    where = ctypes.c_uint32(0)
+    st = lib.lm_get_error(_stream(stream), ctypes.byref(where))
+    return st, where.value
+
+
+def lm_status_string(status):
+    return lib.lm_status_string(status).decode()
+
+
+def lm_version():
+    return lib.lm_version()

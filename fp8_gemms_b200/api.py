@@ -1,0 +1,128 @@
+"""Allocation helpers over the C ABI: PyTorch provides the device buffers,
+libfp8lm.so does every step of the computation.
+
+    from fp8_gemms_b200 import api
+    mlp = api.Relu2Mlp(M, d, f)          # caller-owned saved tensors + workspace
+    Y = mlp.forward(X, W_up, W_down)
+    dX, dW_up, dW_down = mlp.backward(dY)
+"""
+import torch
+
+from . import _lib
+from ._lib import E4M3, E5M2, EPI_NONE, EPI_RELU2_BWD, EPI_RELU2_FWD, LmError  # noqa: F401
+
+
+def _dev(t):
+    return t.device
+
+
+def new_scales(device, n=1):
+    """n blocks of 4 fp32 {amax, scale, inv_scale, unused}, zeroed."""
+    return torch.zeros(n, 4, dtype=torch.float32, device=device)
+
+
+def cast(x, fmt, relu2_input=False, amax_in=None, want_q=True, want_qT=True, scales=None,
+         stream=None):
+    """Dynamic tensorwise cast of a bf16 [rows x cols] tensor.  Returns
+    (q, qT, scales) with scales = [amax, scale, inv_scale, 0] on the device."""
+    rows, cols = x.shape
+    dev = _dev(x)
+    q = torch.empty(rows, cols, dtype=torch.uint8, device=dev) if want_q else None
+    qT = torch.empty(cols, rows, dtype=torch.uint8, device=dev) if want_qT else None
+    sc = new_scales(dev)[0] if scales is None else scales
+    _lib.lm_fp8_amax_scale_cast(x, fmt, sc[0:1], sc[1:2], sc[2:3], q, qT,
+                                relu2_input=relu2_input, amax_in=amax_in, stream=stream)
+    return q, qT, sc
+
+
+def gemm(A, fa, B, fb, inv_a, inv_b, epi=EPI_NONE, aux=None, amax_out=None, out=None,
+         stream=None):
+    """bf16 D[M x N] = epi(A B^T inv_a inv_b) for K-major FP8 codes A, B."""
+    M, N = A.shape[0], B.shape[0]
+    D = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=_dev(A))
+    _lib.lm_fp8_gemm(A, fa, B, fb, inv_a, inv_b, D, epi=epi, aux=aux, amax_out=amax_out,
+                     stream=stream)
+    return D
+
+
+class Relu2Mlp:
+    """Buffers for one relu^2 MLP block of shape (M, d, f): the forward's saved
+    tensors (one device allocation carved by the library) and the backward's
+    workspace.  forward()/backward() are single C-ABI calls."""
+
+    def __init__(self, M, d, f, device="cuda"):
+        self.M, self.d, self.f = M, d, f
+        nbytes = _lib.lm_relu2_mlp_saved_bytes(M, d, f)
+        if nbytes == 0:
+            raise LmError(3, "lm_relu2_mlp_saved_bytes")
+        self.saved_buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.saved = _lib.lm_relu2_mlp_saved_carve(self.saved_buf, M, d, f)
+        self.workspace = torch.empty(_lib.lm_relu2_mlp_workspace_size(M, d, f),
+                                     dtype=torch.uint8, device=device)
+        self.device = device
+
+    def forward(self, X, W_up, W_down, Y=None, stream=None):
+        if Y is None:
+            Y = torch.empty(self.M, self.d, dtype=torch.bfloat16, device=self.device)
+        _lib.lm_relu2_mlp_fwd(X, W_up, W_down, Y, self.saved, stream=stream)
+        return Y
+
+    def backward(self, dY, dX=None, dW_up=None, dW_down=None, stream=None):
+        dev = self.device
+        dX = dX if dX is not None else torch.empty(self.M, self.d, dtype=torch.bfloat16, device=dev)
+        dW_up = dW_up if dW_up is not None else torch.empty(self.f, self.d, dtype=torch.bfloat16,
+                                                            device=dev)
+        dW_down = dW_down if dW_down is not None else torch.empty(self.d, self.f,
+                                                                  dtype=torch.bfloat16, device=dev)
+        _lib.lm_relu2_mlp_bwd(dY, self.saved, dX, dW_up, dW_down, self.workspace, stream=stream)
+        return dX, dW_up, dW_down
+
+    # views of the saved tensors (for inspection and stagewise checks)
+    def view(self, name):
+        M, d, f = self.M, self.d, self.f
+        shapes = {"Xq": (M, d), "XqT": (d, M), "Wuq": (f, d), "WuqT": (d, f), "Wdq": (d, f),
+                  "WdqT": (f, d), "hq": (M, f), "hqT": (f, M)}
+        base = self.saved_buf.data_ptr()
+        if name == "H":
+            off = self.saved.H - base
+            return self.saved_buf[off:off + M * f * 2].view(torch.bfloat16).view(M, f)
+        if name == "scales":
+            off = self.saved.scales - base
+            return self.saved_buf[off:off + 64].view(torch.float32).view(4, 4)
+        r, c = shapes[name]
+        off = getattr(self.saved, name) - base
+        return self.saved_buf[off:off + r * c].view(r, c)
+
+    def workspace_view(self, name):
+        """Backward scratch: dYq, dYqT, dH, dHq, dHqT, scales (library layout:
+        each buffer rounded up to 256 bytes, in that order)."""
+        M, d, f = self.M, self.d, self.f
+        r256 = lambda n: (n + 255) // 256 * 256
+        sizes = [("dYq", M * d), ("dYqT", M * d), ("dH", M * f * 2), ("dHq", M * f),
+                 ("dHqT", M * f), ("scales", 32)]
+        off = 0
+        for n, sz in sizes:
+            if n == name:
+                v = self.workspace[off:off + sz]
+                if n == "dH":
+                    return v.view(torch.bfloat16).view(M, f)
+                if n == "scales":
+                    return v.view(torch.float32).view(2, 4)
+                return v.view(*{"dYq": (M, d), "dYqT": (d, M), "dHq": (M, f),
+                                "dHqT": (f, M)}[n])
+            off += r256(sz)
+        raise KeyError(name)
+
+
+def linear_fwd_bwd(X, W, dY, stream=None):
+    """Plain linear Y = X W^T with its dgrad and wgrad, all in FP8: X, W cast
+    to e4m3 and dY to e5m2 (each with its K-major transposed copy), then
+    Y = Xq Wq^T, dX = dYq (Wq^T)^T, dW = (dYq^T)(Xq^T)^T.  Returns (Y, dX, dW)."""
+    sc = new_scales(X.device, 3)
+    Xq, XqT, _ = cast(X, E4M3, scales=sc[0], stream=stream)
+    Wq, WqT, _ = cast(W, E4M3, scales=sc[1], stream=stream)
+    dYq, dYqT, _ = cast(dY, E5M2, scales=sc[2], stream=stream)
+    Y = gemm(Xq, E4M3, Wq, E4M3, sc[0, 2:3], sc[1, 2:3], stream=stream)
+    dX = gemm(dYq, E5M2, WqT, E4M3, sc[2, 2:3], sc[1, 2:3], stream=stream)
+    dW = gemm(dYqT, E5M2, XqT, E4M3, sc[2, 2:3], sc[0, 2:3], stream=stream)
+    return Y, dX, dW, dict(Xq=Xq, XqT=XqT, Wq=Wq, WqT=WqT, dYq=dYq, dYqT=dYqT, scales=sc)

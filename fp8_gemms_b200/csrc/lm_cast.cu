@@ -1,0 +1,276 @@
+// lm_cast.cu -- dynamic tensorwise FP8 scaling: amax reduction, scale, and
+// the saturating round-to-nearest-even cast with its K-major transposed copy.
+//
+// Method: one fp32 scale per tensor per cast, computed from that tensor's
+// current amax (decomputer.nl, "Het trainen van een 3.8B LLM tot 0.384 CORE
+// voor $998", section "Vroege experimenten" item 4 -- FP8 with dynamic
+// tensorwise scaling on all three GEMMs).  e4m3 (max 448) for activations and
+// weights, e5m2 (max 57344) for gradients.
+//
+// Both kernels are HBM-bound: 16-byte vector loads of bf16, codes written
+// with 8-byte (row-major) and 16-byte (transposed) stores; the transpose goes
+// through a 32 KB shared-memory tile and 4x4 byte permutes.
+#include <cuda_bf16.h>
+
+#include "lm_internal.h"
+
+namespace lm {
+namespace {
+
+constexpr int kCastRows = 256;  // tile rows (the qT segment written per column)
+constexpr int kCastCols = 128;  // tile columns (bytes of codes per smem row)
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// h = bf16(relu(x)^2): the square of a bf16 value is exact in fp32, then
+// rounded once to bf16.  relu(NaN) stays NaN.
+__device__ __forceinline__ float relu2_bf16(float x) {
+    float r = x > 0.f ? x : (x != x ? x : 0.f);
+    return __bfloat162float(__float2bfloat16_rn(r * r));
+}
+
+// Two fp32 values -> two saturated RNE FP8 codes (lo in the low byte).
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt_pair(float lo, float hi) {
+    uint16_t r;
+    if (FMT == LM_FP8_E4M3)
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    else
+        asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// 8 bf16 (16 bytes) -> 8 codes (8 bytes), code = fp8(fp32(v * scale)).
+template <int FMT, bool RELU2>
+__device__ __forceinline__ uint2 convert8(uint4 v, float scale) {
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t p[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
+        if (RELU2) {
+            lo = relu2_bf16(lo);
+            hi = relu2_bf16(hi);
+        }
+        p[i] = cvt_pair<FMT>(__fmul_rn(lo, scale), __fmul_rn(hi, scale));
+    }
+    return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+}
+
+// max over the 8 bf16 of v of |x| (or of h = bf16(relu(x)^2)), as bf16 bits.
+// Non-negative bf16 values order like their bits; NaN sorts above infinity.
+template <bool RELU2>
+__device__ __forceinline__ uint32_t absmax8(uint4 v, uint32_t m) {
+    if (!RELU2) {
+        m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+        return m;
+    }
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t lo = __float_as_uint(relu2_bf16(bf16_lo(w[i]))) >> 16;
+        uint32_t hi = __float_as_uint(relu2_bf16(bf16_hi(w[i]))) & 0xFFFF0000u;
+        m = __vmaxu2(m, (lo | hi) & 0x7FFF7FFFu);
+    }
+    return m;
+}
+
+// Pass 1: amax over the tensor into *amax_bits (fp32 bit pattern of a
+// non-negative value, max-reduced with atomicMax; zeroed by the caller).
+template <bool RELU2>
+__global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restrict__ x,
+                                                        int64_t rows, int64_t cols, int64_t ld,
+                                                        unsigned int* __restrict__ amax_bits) {
+    uint32_t m = 0;
+    const int64_t vpr = cols >> 3;  // 16-byte vectors per row
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    if (ld == cols) {
+        const int64_t nvec = rows * vpr;
+        const uint4* xv = reinterpret_cast<const uint4*>(x);
+        for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nvec; i += stride)
+            m = absmax8<RELU2>(ld_stream_v4(xv + i), m);
+    } else {
+        const int64_t nvec = rows * vpr;
+        for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nvec; i += stride) {
+            int64_t r = i / vpr, c = (i - r * vpr) << 3;
+            m = absmax8<RELU2>(ld_stream_v4(x + r * ld + c), m);
+        }
+    }
+    m = max(m & 0xFFFFu, m >> 16);
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    __shared__ uint32_t warp_max[kThreads / 32];
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+#pragma unroll
+        for (int i = 0; i < kThreads / 32; ++i) b = max(b, warp_max[i]);
+        if (b) atomicMax(amax_bits, b << 16);
+    }
+}
+
+__device__ __forceinline__ void write_scales(float amax, float fmax, float* amax_out,
+                                             float* scale_out, float* inv_out, float* scale_reg) {
+    const float a = amax < 1e-12f ? 1e-12f : amax;
+    const float scale = __fdiv_rn(fmax, a);
+    *scale_reg = scale;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *amax_out = amax;
+        *scale_out = scale;
+        *inv_out = __fdiv_rn(1.0f, scale);
+    }
+}
+
+__global__ void scales_only_kernel(const float* amax_src, float fmax, float* amax_out,
+                                   float* scale_out, float* inv_out) {
+    float s;
+    write_scales(*amax_src, fmax, amax_out, scale_out, inv_out, &s);
+}
+
+// Pass 2: scale, cast and transpose one 256 x 128 tile per block.  Tiles are
+// taken in reverse memory order so the first blocks re-read the tail of the
+// tensor, the part pass 1 left in L2.
+template <int FMT, bool RELU2>
+__global__ void __launch_bounds__(kThreads) cast_kernel(
+    const uint16_t* __restrict__ x, int rows, int cols, int64_t ld, const float* amax_src,
+    float* amax_out, float* scale_out, float* inv_out, uint8_t* __restrict__ q,
+    uint8_t* __restrict__ qT, int tiles_c, int num_tiles) {
+    __shared__ __align__(16) uint32_t tile[kCastRows][kCastCols / 4];
+    const float fmax = FMT == LM_FP8_E4M3 ? 448.0f : 57344.0f;
+    float scale;
+    write_scales(*amax_src, fmax, amax_out, scale_out, inv_out, &scale);
+
+    const int t = num_tiles - 1 - (int)blockIdx.x;
+    const int r0 = (t / tiles_c) * kCastRows;
+    const int c0 = (t % tiles_c) * kCastCols;
+    const int tid = threadIdx.x;
+
+    // load 16 bytes of bf16 -> 8 codes; row-major codes straight to q
+#pragma unroll 4
+    for (int it = 0; it < (kCastRows * kCastCols / 8) / kThreads; ++it) {
+        const int idx = it * kThreads + tid;
+        const int rr = idx >> 4, ch = idx & 15;
+        const int r = r0 + rr, c = c0 + ch * 8;
+        uint2 codes = make_uint2(0u, 0u);
+        if (r < rows && c < cols) {
+            codes = convert8<FMT, RELU2>(ld_stream_v4(x + (int64_t)r * ld + c), scale);
+            if (q) *reinterpret_cast<uint2*>(q + (int64_t)r * cols + c) = codes;
+        }
+        *reinterpret_cast<uint2*>(&tile[rr][ch * 2]) = codes;
+    }
+    if (!qT) return;
+    __syncthreads();
+
+    // warp w owns tile rows [32w, 32w+32), lane l owns tile columns [4l, 4l+4)
+    const int w = tid >> 5, l = tid & 31;
+    uint32_t v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = tile[w * 32 + i][l];
+    uint32_t o[4][8];  // o[j][k]: column 4l+j, tile rows 32w+4k .. +3
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t t0 = __byte_perm(v[4 * k], v[4 * k + 1], 0x5140);
+        const uint32_t t1 = __byte_perm(v[4 * k + 2], v[4 * k + 3], 0x5140);
+        const uint32_t t2 = __byte_perm(v[4 * k], v[4 * k + 1], 0x7362);
+        const uint32_t t3 = __byte_perm(v[4 * k + 2], v[4 * k + 3], 0x7362);
+        o[0][k] = __byte_perm(t0, t1, 0x5410);
+        o[1][k] = __byte_perm(t0, t1, 0x7632);
+        o[2][k] = __byte_perm(t2, t3, 0x5410);
+        o[3][k] = __byte_perm(t2, t3, 0x7632);
+    }
+    const int rb = r0 + w * 32;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int c = c0 + 4 * l + j;
+        if (c >= cols) continue;
+        uint8_t* dst = qT + (int64_t)c * rows + rb;
+        if (rb + 16 <= rows)
+            *reinterpret_cast<uint4*>(dst) = make_uint4(o[j][0], o[j][1], o[j][2], o[j][3]);
+        if (rb + 32 <= rows)
+            *reinterpret_cast<uint4*>(dst + 16) = make_uint4(o[j][4], o[j][5], o[j][6], o[j][7]);
+    }
+}
+
+template <int FMT, bool RELU2>
+void launch_cast(const uint16_t* x, int rows, int cols, int64_t ld, const float* amax_src,
+                 float* amax_out, float* scale_out, float* inv_out, uint8_t* q, uint8_t* qT,
+                 cudaStream_t s) {
+    const int tiles_r = (rows + kCastRows - 1) / kCastRows;
+    const int tiles_c = (cols + kCastCols - 1) / kCastCols;
+    const int n = tiles_r * tiles_c;
+    cast_kernel<FMT, RELU2><<<n, kThreads, 0, s>>>(x, rows, cols, ld, amax_src, amax_out,
+                                                  scale_out, inv_out, q, qT, tiles_c, n);
+}
+
+}  // namespace
+}  // namespace lm
+
+extern "C" lm_status lm_fp8_amax_scale_cast(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                            lm_fp8_format fmt, int relu2_input,
+                                            const float* amax_in, float* amax_out,
+                                            float* scale_out, float* inv_scale_out, uint8_t* q,
+                                            uint8_t* qT, lm_stream_t stream) {
+    using namespace lm;
+    if (fmt != LM_FP8_E4M3 && fmt != LM_FP8_E5M2) return LM_ERR_UNSUPPORTED_FORMAT;
+    if (rows < 0 || cols < 0 || ld < cols) return LM_ERR_INVALID_ARG;
+    if (!amax_out || !scale_out || !inv_scale_out) return LM_ERR_INVALID_ARG;
+    const bool empty = rows == 0 || cols == 0;
+    if (!empty && !x) return LM_ERR_INVALID_ARG;
+    if (cols % 16 != 0 || ld % 8 != 0) return LM_ERR_UNSUPPORTED_SHAPE;
+    if (qT && rows % 16 != 0) return LM_ERR_UNSUPPORTED_SHAPE;
+    if (rows >= (int64_t(1) << 31) || cols >= (int64_t(1) << 31)) return LM_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(qT)) return LM_ERR_ALIGNMENT;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const float fmax = fmt == LM_FP8_E4M3 ? 448.0f : 57344.0f;
+    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    const float* amax_src = amax_in;
+    if (!amax_in) {
+        if (cudaMemsetAsync(amax_out, 0, sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
+        if (!empty) {
+            int grid = sm_count() * 4;
+            if (grid <= 0) return LM_ERR_CUDA;
+            if (relu2_input)
+                amax_kernel<true><<<grid, kThreads, 0, s>>>(xb, rows, cols, ld,
+                                                             reinterpret_cast<unsigned*>(amax_out));
+            else
+                amax_kernel<false><<<grid, kThreads, 0, s>>>(xb, rows, cols, ld,
+                                                              reinterpret_cast<unsigned*>(amax_out));
+        }
+        amax_src = amax_out;
+    }
+    if (empty || (!q && !qT)) {
+        scales_only_kernel<<<1, 1, 0, s>>>(amax_src, fmax, amax_out, scale_out, inv_scale_out);
+        return launch_status();
+    }
+    const int r = (int)rows, c = (int)cols;
+    if (fmt == LM_FP8_E4M3) {
+        if (relu2_input)
+            launch_cast<LM_FP8_E4M3, true>(xb, r, c, ld, amax_src, amax_out, scale_out,
+                                           inv_scale_out, q, qT, s);
+        else
+            launch_cast<LM_FP8_E4M3, false>(xb, r, c, ld, amax_src, amax_out, scale_out,
+                                            inv_scale_out, q, qT, s);
+    } else {
+        if (relu2_input)
+            launch_cast<LM_FP8_E5M2, true>(xb, r, c, ld, amax_src, amax_out, scale_out,
+                                           inv_scale_out, q, qT, s);
+        else
+            launch_cast<LM_FP8_E5M2, false>(xb, r, c, ld, amax_src, amax_out, scale_out,
+                                            inv_scale_out, q, qT, s);
+    }
+    return launch_status();
+}

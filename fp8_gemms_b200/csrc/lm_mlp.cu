@@ -1,0 +1,166 @@
+// lm_mlp.cu -- the non-gated relu^2 MLP, forward and backward, composed from
+// the cast and GEMM kernels on one stream with no host synchronisation.
+//
+// Model: hidden_act relu2, gated_mlp false, intermediate 4x (decomputer.nl,
+// "Het trainen van een 3.8B LLM tot 0.384 CORE voor $998", "Appendix: De
+// configuratie", and section "Doorvoer (Throughput) verhogen", bullet
+// "Niet-gated MLPs": two matmuls instead of three).  All six GEMMs (forward,
+// dgrad and wgrad of both linears) run in FP8 with dynamic tensorwise scaling
+// (same page, section "Vroege experimenten" item 4).  Each tensor is
+// quantised once per call; the backward reuses the forward's codes and scales.
+#include "lm_internal.h"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool mlp_shape_ok(int64_t M, int64_t d, int64_t f) {
+    return M >= 0 && d > 0 && f > 0 && M % 16 == 0 && d % 16 == 0 && f % 16 == 0;
+}
+
+// scale block layout: 4 floats per tensor {amax, scale, inv_scale, unused}
+enum { S_X = 0, S_WU = 4, S_WD = 8, S_H = 12 };  // in lm_mlp_saved::scales
+enum { S_DY = 0, S_DH = 4 };                      // in the backward workspace
+
+struct BwdWorkspace {
+    uint8_t *dYq, *dYqT, *dHq, *dHqT;
+    void* dH;
+    float* scales;
+};
+
+size_t bwd_layout(int64_t M, int64_t d, int64_t f, uint8_t* base, BwdWorkspace* w) {
+    const size_t Md = (size_t)M * (size_t)d, Mf = (size_t)M * (size_t)f;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* p = base ? base + off : nullptr;
+        off += round_up(bytes);
+        return p;
+    };
+    uint8_t* dYq = take(Md);
+    uint8_t* dYqT = take(Md);
+    uint8_t* dH = take(Mf * 2);
+    uint8_t* dHq = take(Mf);
+    uint8_t* dHqT = take(Mf);
+    uint8_t* sc = take(8 * sizeof(float));
+    if (w) *w = BwdWorkspace{dYq, dYqT, dHq, dHqT, dH, reinterpret_cast<float*>(sc)};
+    return off;
+}
+
+size_t saved_layout(int64_t M, int64_t d, int64_t f, uint8_t* base, lm_mlp_saved* s) {
+    const size_t Md = (size_t)M * (size_t)d, Mf = (size_t)M * (size_t)f,
+                 fd = (size_t)f * (size_t)d;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* p = base ? base + off : nullptr;
+        off += round_up(bytes);
+        return p;
+    };
+    lm_mlp_saved o;
+    o.Xq = take(Md);
+    o.XqT = take(Md);
+    o.Wuq = take(fd);
+    o.WuqT = take(fd);
+    o.Wdq = take(fd);
+    o.WdqT = take(fd);
+    o.H = take(Mf * 2);
+    o.hq = take(Mf);
+    o.hqT = take(Mf);
+    o.scales = reinterpret_cast<float*>(take(16 * sizeof(float)));
+    if (s) *s = o;
+    return off;
+}
+
+#define LM_TRY(expr)                       \
+    do {                                   \
+        lm_status _st = (expr);            \
+        if (_st != LM_OK) return _st;      \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t lm_relu2_mlp_saved_bytes(int64_t M, int64_t d, int64_t f) {
+    if (!mlp_shape_ok(M, d, f)) return 0;
+    return saved_layout(M, d, f, nullptr, nullptr);
+}
+
+lm_status lm_relu2_mlp_saved_carve(void* base, size_t bytes, int64_t M, int64_t d, int64_t f,
+                                   lm_mlp_saved* out) {
+    if (!base || !out) return LM_ERR_INVALID_ARG;
+    if (!mlp_shape_ok(M, d, f)) return LM_ERR_UNSUPPORTED_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(base) % kAlign) != 0) return LM_ERR_ALIGNMENT;
+    if (bytes < saved_layout(M, d, f, nullptr, nullptr)) return LM_ERR_INVALID_ARG;
+    saved_layout(M, d, f, static_cast<uint8_t*>(base), out);
+    return LM_OK;
+}
+
+size_t lm_relu2_mlp_workspace_size(int64_t M, int64_t d, int64_t f) {
+    if (!mlp_shape_ok(M, d, f)) return 0;
+    return bwd_layout(M, d, f, nullptr, nullptr);
+}
+
+lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W_down, int64_t M,
+                           int64_t d, int64_t f, void* Y, lm_mlp_saved* sv, void* workspace,
+                           size_t ws_bytes, lm_stream_t stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    if (!mlp_shape_ok(M, d, f)) return LM_ERR_UNSUPPORTED_SHAPE;
+    if (!X || !W_up || !W_down || !Y || !sv) return LM_ERR_INVALID_ARG;
+    if (!sv->Xq || !sv->XqT || !sv->Wuq || !sv->WuqT || !sv->Wdq || !sv->WdqT || !sv->H ||
+        !sv->hq || !sv->hqT || !sv->scales)
+        return LM_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float* S = sv->scales;
+    if (cudaMemsetAsync(S, 0, 16 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
+    LM_TRY(lm_fp8_amax_scale_cast(X, M, d, d, LM_FP8_E4M3, 0, nullptr, S + S_X, S + S_X + 1,
+                                  S + S_X + 2, sv->Xq, sv->XqT, stream));
+    LM_TRY(lm_fp8_amax_scale_cast(W_up, f, d, d, LM_FP8_E4M3, 0, nullptr, S + S_WU, S + S_WU + 1,
+                                  S + S_WU + 2, sv->Wuq, sv->WuqT, stream));
+    LM_TRY(lm_fp8_amax_scale_cast(W_down, d, f, f, LM_FP8_E4M3, 0, nullptr, S + S_WD,
+                                  S + S_WD + 1, S + S_WD + 2, sv->Wdq, sv->WdqT, stream));
+    // H = X W_up^T (bf16) and amax of h = bf16(relu(H)^2)
+    LM_TRY(lm_fp8_gemm(sv->Xq, LM_FP8_E4M3, sv->Wuq, LM_FP8_E4M3, M, f, d, S + S_X + 2,
+                       S + S_WU + 2, LM_EPI_RELU2_FWD, nullptr, sv->H, S + S_H, stream));
+    LM_TRY(lm_fp8_amax_scale_cast(sv->H, M, f, f, LM_FP8_E4M3, 1, S + S_H, S + S_H, S + S_H + 1,
+                                  S + S_H + 2, sv->hq, sv->hqT, stream));
+    // Y = h W_down^T
+    LM_TRY(lm_fp8_gemm(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, S + S_H + 2,
+                       S + S_WD + 2, LM_EPI_NONE, nullptr, Y, nullptr, stream));
+    return LM_OK;
+}
+
+lm_status lm_relu2_mlp_bwd(const void* dY, const lm_mlp_saved* sv, int64_t M, int64_t d,
+                           int64_t f, void* dX, void* dW_up, void* dW_down, void* workspace,
+                           size_t ws_bytes, lm_stream_t stream) {
+    if (!mlp_shape_ok(M, d, f)) return LM_ERR_UNSUPPORTED_SHAPE;
+    if (!dY || !sv || !dX || !dW_up || !dW_down || !workspace) return LM_ERR_INVALID_ARG;
+    if (ws_bytes < bwd_layout(M, d, f, nullptr, nullptr)) return LM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return LM_ERR_ALIGNMENT;
+    BwdWorkspace w;
+    bwd_layout(M, d, f, static_cast<uint8_t*>(workspace), &w);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const float* S = sv->scales;
+    float* G = w.scales;
+    if (cudaMemsetAsync(G, 0, 8 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
+    LM_TRY(lm_fp8_amax_scale_cast(dY, M, d, d, LM_FP8_E5M2, 0, nullptr, G + S_DY, G + S_DY + 1,
+                                  G + S_DY + 2, w.dYq, w.dYqT, stream));
+    // dH = bf16(bf16(dY W_down) * 2 relu(H)), and its amax
+    LM_TRY(lm_fp8_gemm(w.dYq, LM_FP8_E5M2, sv->WdqT, LM_FP8_E4M3, M, f, d, G + S_DY + 2,
+                       S + S_WD + 2, LM_EPI_RELU2_BWD, sv->H, w.dH, G + S_DH, stream));
+    // dW_down = dY^T h (K = M)
+    LM_TRY(lm_fp8_gemm(w.dYqT, LM_FP8_E5M2, sv->hqT, LM_FP8_E4M3, d, f, M, G + S_DY + 2,
+                       S + S_H + 2, LM_EPI_NONE, nullptr, dW_down, nullptr, stream));
+    LM_TRY(lm_fp8_amax_scale_cast(w.dH, M, f, f, LM_FP8_E5M2, 0, G + S_DH, G + S_DH,
+                                  G + S_DH + 1, G + S_DH + 2, w.dHq, w.dHqT, stream));
+    // dX = dH W_up;  dW_up = dH^T X (K = M)
+    LM_TRY(lm_fp8_gemm(w.dHq, LM_FP8_E5M2, sv->WuqT, LM_FP8_E4M3, M, d, f, G + S_DH + 2,
+                       S + S_WU + 2, LM_EPI_NONE, nullptr, dX, nullptr, stream));
+    LM_TRY(lm_fp8_gemm(w.dHqT, LM_FP8_E5M2, sv->XqT, LM_FP8_E4M3, f, d, M, G + S_DH + 2,
+                       S + S_X + 2, LM_EPI_NONE, nullptr, dW_up, nullptr, stream));
+    return LM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,198 @@
+/*
+ * lm_fp8.h -- C ABI of libfp8lm.so: FP8 training GEMMs with dynamic
+ * tensorwise scaling for a non-gated relu^2 MLP and plain linears, written for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (little-lm write-up, decomputer.nl, "Het trainen van een 3.8B
+ * LLM tot 0.384 CORE voor $998", section "Vroege experimenten" item 4 and
+ * section "Doorvoer (Throughput) verhogen", FP8 bullet; simpleprog.com,
+ * "Training a 3.8B LLM to 0.384 CORE for $998", "Five Changes That Mattered"):
+ * all three GEMMs of every linear layer -- forward Y = X W^T, dgrad
+ * dX = dY W, wgrad dW = dY^T X -- run in FP8, each operand quantised with one
+ * fp32 scale computed from that tensor's current amax.  The MLP is the
+ * non-gated relu^2 MLP at 4x ("Niet-gated MLPs" bullet; "Appendix: De
+ * configuratie": hidden 3072, intermediate 12288, hidden_act relu2).
+ *
+ * Formats: e4m3 (OCP E4M3, max 448, no infinities) for activations and
+ * weights, e5m2 (OCP E5M2, max 57344) for gradients.  Codes are raw bytes.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    allocates no device memory.  bf16 tensors are passed as `const void*` /
+ *    `void*` holding IEEE bfloat16 bits.  Scales are device fp32.
+ *  - Matrices are row-major.  "K-major" means the reduction dimension is the
+ *    contiguous one: A [M x K] and B [N x K] for D = A B^T.
+ *  - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).  No entry point synchronises the host, and
+ *    no scale ever travels to the host.
+ *  - Argument, alignment and shape checks run on the host before any launch
+ *    and return a non-zero status without enqueuing anything.  A failed launch
+ *    returns LM_ERR_CUDA.  Device-side failures (a bounded wait that ran out)
+ *    are recorded in a per-device error word read by lm_get_error().
+ *  - No C++ exception crosses this interface.
+ */
+#ifndef LM_FP8_H
+#define LM_FP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LM_API __attribute__((visibility("default")))
+#else
+#define LM_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* lm_stream_t;
+
+typedef enum {
+    LM_OK = 0,
+    LM_ERR_INVALID_ARG = 1,        /* null pointer, negative size, workspace too small */
+    LM_ERR_ALIGNMENT = 2,          /* a pointer or row pitch not 16-byte aligned */
+    LM_ERR_UNSUPPORTED_SHAPE = 3,  /* a dimension violates the documented multiple */
+    LM_ERR_UNSUPPORTED_FORMAT = 4, /* e5m2 x e5m2, or an unknown format/epilogue */
+    LM_ERR_CUDA = 5,               /* a CUDA runtime/driver call or launch failed */
+    LM_ERR_TIMEOUT = 6,            /* a device-side bounded wait ran out */
+    LM_ERR_NONFINITE = 7           /* reserved: non-finite amax reported by a check */
+} lm_status;
+
+typedef enum { LM_FP8_E4M3 = 0, LM_FP8_E5M2 = 1 } lm_fp8_format;
+
+typedef enum {
+    LM_EPI_NONE = 0,      /* D = bf16(acc * s) */
+    LM_EPI_RELU2_FWD = 1, /* D = H = bf16(acc * s); amax of h = bf16(relu(H)^2) */
+    LM_EPI_RELU2_BWD = 2  /* g = bf16(acc * s); D = dH = bf16(g * 2 * relu(aux)) */
+} lm_epilogue;
+
+/*
+ * Dynamic tensorwise scaling cast (amax -> scale -> saturating RNE cast).
+ *
+ *   amax  = max |x|                      (relu2_input: max h, h = bf16(relu(x)^2))
+ *   scale = fp32(fmax / max(amax, 1e-12)),  fmax = 448 (e4m3) or 57344 (e5m2)
+ *   inv   = fp32(1 / scale)
+ *   q[r][c] = sat_rne_fp8(fp32(x_or_h[r][c] * scale)),  qT[c][r] = q[r][c]
+ *
+ * x: bf16 [rows x cols] with leading dimension ld (elements).
+ * amax_in: if non-NULL, a device fp32 already holding the amax of the tensor
+ *   to be cast (for example written by lm_fp8_gemm's epilogue); no reduction
+ *   pass runs.  If NULL, a reduction pass computes it.
+ * amax_out, scale_out, inv_scale_out: device fp32, written (amax_out may
+ *   alias amax_in).  When amax_in is NULL, amax_out is also the reduction's
+ *   accumulator and is overwritten.
+ * q: [rows x cols] codes, qT: [cols x rows] codes (the K-major copy that
+ *   dgrad/wgrad consume); either may be NULL to skip it.
+ * Requirements: cols % 16 == 0, ld % 8 == 0, ld >= cols; rows % 16 == 0 when
+ *   qT != NULL; x, q, qT 16-byte aligned.  rows == 0 or cols == 0 writes the
+ *   amax (0) and scales only.
+ */
+LM_API lm_status lm_fp8_amax_scale_cast(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                 lm_fp8_format fmt, int relu2_input, const float* amax_in,
+                                 float* amax_out, float* scale_out, float* inv_scale_out,
+                                 uint8_t* q, uint8_t* qT, lm_stream_t stream);
+
+/*
+ * FP8 GEMM on the 5th-generation tensor cores (tcgen05, TMEM accumulators):
+ *
+ *   acc[m][n] = sum_k A[m][k] * B[n][k]      (fp32 accumulation of the FP8 products)
+ *   s = inv_scale_a * inv_scale_b
+ *   D[m][n] = epilogue(acc * s) as bf16     (see lm_epilogue)
+ *
+ * A: [M x K] codes of format fa, B: [N x K] codes of format fb, both K-major.
+ * inv_scale_a / inv_scale_b: device fp32 dequantisation factors (1/scale).
+ * aux: bf16 [M x N], the saved pre-activation H, required for
+ *   LM_EPI_RELU2_BWD, ignored otherwise.
+ * D: bf16 [M x N], row-major.
+ * amax_out: device fp32 or NULL.  If non-NULL it is max-reduced (atomically,
+ *   order independent) with the amax of the tensor the next cast consumes:
+ *   max|D| (NONE), max bf16(relu(D)^2) (RELU2_FWD), max|D| (RELU2_BWD).  The
+ *   caller zeroes it before the first GEMM that feeds it.
+ * Formats: (e4m3, e4m3), (e5m2, e4m3), (e4m3, e5m2); e5m2 x e5m2 returns
+ *   LM_ERR_UNSUPPORTED_FORMAT.
+ * Requirements: K % 16 == 0, N % 8 == 0; A, B, D, aux 16-byte aligned.
+ *   M and N need not be multiples of the tile; K == 0 writes D = 0.
+ */
+LM_API lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8_t* B, lm_fp8_format fb,
+                      int64_t M, int64_t N, int64_t K, const float* inv_scale_a,
+                      const float* inv_scale_b, lm_epilogue epi, const void* aux, void* D,
+                      float* amax_out, lm_stream_t stream);
+
+/*
+ * Tensors the relu^2 MLP forward saves for its backward.  Every pointer is a
+ * caller-owned device buffer (see lm_relu2_mlp_saved_carve).  Shapes for
+ * X [M x d], W_up [f x d], W_down [d x f]:
+ */
+typedef struct lm_mlp_saved {
+    uint8_t* Xq;   /* [M x d] e4m3 */
+    uint8_t* XqT;  /* [d x M] e4m3, for wgrad of W_up */
+    uint8_t* Wuq;  /* [f x d] e4m3, forward B operand of the up GEMM */
+    uint8_t* WuqT; /* [d x f] e4m3, dgrad B operand */
+    uint8_t* Wdq;  /* [d x f] e4m3, forward B operand of the down GEMM */
+    uint8_t* WdqT; /* [f x d] e4m3, dgrad B operand */
+    void* H;       /* [M x f] bf16 pre-activation X W_up^T */
+    uint8_t* hq;   /* [M x f] e4m3 codes of h = bf16(relu(H)^2) */
+    uint8_t* hqT;  /* [f x M] e4m3, for wgrad of W_down */
+    float* scales; /* 16 device floats: {amax, scale, inv_scale, unused} for X, W_up, W_down, h */
+} lm_mlp_saved;
+
+/* Bytes needed to hold every buffer of lm_mlp_saved (each 256-byte aligned). */
+LM_API size_t lm_relu2_mlp_saved_bytes(int64_t M, int64_t d, int64_t f);
+
+/* Host-only pointer arithmetic: carve a caller-allocated device buffer `base`
+ * of `bytes` (>= lm_relu2_mlp_saved_bytes) into `out`.  Launches nothing. */
+LM_API lm_status lm_relu2_mlp_saved_carve(void* base, size_t bytes, int64_t M, int64_t d, int64_t f,
+                                   lm_mlp_saved* out);
+
+/* Bytes of scratch lm_relu2_mlp_bwd needs (lm_relu2_mlp_fwd needs none). */
+LM_API size_t lm_relu2_mlp_workspace_size(int64_t M, int64_t d, int64_t f);
+
+/*
+ * relu^2 MLP forward, Y = relu(X W_up^T)^2 W_down^T, every GEMM in FP8:
+ *   cast X, W_up, W_down to e4m3 (+ K-major transposes)
+ *   H = up GEMM with the RELU2_FWD epilogue (bf16 H + amax of h)
+ *   cast h = bf16(relu(H)^2) to e4m3 (+ transpose) using that amax
+ *   Y = down GEMM (bf16)
+ * X: bf16 [M x d], W_up: bf16 [f x d], W_down: bf16 [d x f], Y: bf16 [M x d].
+ * workspace may be NULL (ws_bytes 0).  Requirements: M, d, f multiples of 16.
+ */
+LM_API lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W_down, int64_t M,
+                           int64_t d, int64_t f, void* Y, lm_mlp_saved* saved, void* workspace,
+                           size_t ws_bytes, lm_stream_t stream);
+
+/*
+ * relu^2 MLP backward from the forward's saved tensors:
+ *   cast dY to e5m2 (+ transpose)
+ *   dH = dgrad of W_down with the RELU2_BWD epilogue: bf16(bf16(dY W_down) * 2 relu(H))
+ *   dW_down = dY^T h   (wgrad, K = M)
+ *   cast dH to e5m2 (+ transpose) using the epilogue's amax
+ *   dX = dH W_up;  dW_up = dH^T X
+ * dY: bf16 [M x d]; outputs bf16 dX [M x d], dW_up [f x d], dW_down [d x f].
+ * workspace: device scratch of >= lm_relu2_mlp_workspace_size bytes,
+ * 256-byte aligned.  Requirements as for the forward.
+ */
+LM_API lm_status lm_relu2_mlp_bwd(const void* dY, const lm_mlp_saved* saved, int64_t M, int64_t d,
+                           int64_t f, void* dX, void* dW_up, void* dW_down, void* workspace,
+                           size_t ws_bytes, lm_stream_t stream);
+
+/* Synchronises `stream`, then returns and clears the current device's error
+ * word: LM_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
+ * LM_ERR_CUDA if the synchronisation itself failed, else LM_OK.  If
+ * where_out is non-NULL it receives the code of the wait that ran out (0 if
+ * none). */
+LM_API lm_status lm_get_error(lm_stream_t stream, uint32_t* where_out);
+
+/* Static, human-readable name of a status. */
+LM_API const char* lm_status_string(lm_status status);
+
+/* Library version, as major*10000 + minor*100 + patch. */
+LM_API int lm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LM_FP8_H */

@@ -1,0 +1,92 @@
+"""The C-ABI library loads on a CPU-only host, exports every symbol that
+include/*.h declares, and its host-side argument checks reject bad calls
+before any launch (no GPU needed for any of this)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names += re.findall(r"^LM_API\s+[\w\s\*]+?\b(lm_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    from fp8_gemms_b200 import build
+    build.build()
+    from fp8_gemms_b200 import _lib
+    return _lib
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for fn in ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_fwd", "lm_relu2_mlp_bwd"]:
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    lib = ctypes.CDLL(L.LIB_PATH)
+    for fn in declared_functions():
+        assert hasattr(lib, fn), fn
+    assert sorted(declared_functions()) == sorted(L.EXPORTED)
+
+
+def test_status_strings_and_version(L):
+    assert L.lm_version() >= 100
+    for code, name in L.STATUS.items():
+        assert L.lm_status_string(code).startswith(name)
+
+
+def test_gemm_host_checks_reject_before_launch(L):
+    g = L.lib.lm_fp8_gemm
+    fake = 0x10000  # never dereferenced: every call below fails a host check first
+    E4, E5 = L.E4M3, L.E5M2
+    assert g(fake, E5, fake, E5, 16, 16, 16, fake, fake, 0, None, fake, None, None) == 4
+    assert g(fake, 7, fake, E4, 16, 16, 16, fake, fake, 0, None, fake, None, None) == 4
+    assert g(fake, E4, fake, E4, 16, 16, 16, fake, fake, 9, None, fake, None, None) == 4
+    assert g(fake, E4, fake, E4, -1, 16, 16, fake, fake, 0, None, fake, None, None) == 1
+    assert g(fake, E4, fake, E4, 16, 16, 16, None, fake, 0, None, fake, None, None) == 1
+    assert g(fake, E4, fake, E4, 16, 16, 16, fake, fake, 2, None, fake, None, None) == 1
+    assert g(fake, E4, fake, E4, 16, 16, 24, fake, fake, 0, None, fake, None, None) == 3
+    assert g(fake, E4, fake, E4, 16, 12, 16, fake, fake, 0, None, fake, None, None) == 3
+    assert g(fake + 8, E4, fake, E4, 16, 16, 16, fake, fake, 0, None, fake, None, None) == 2
+    assert g(fake, E4, fake, E4, 16, 16, 16, fake, fake, 0, None, fake + 4, None, None) == 2
+    # empty output: nothing to do, nothing launched
+    assert g(fake, E4, fake, E4, 0, 16, 16, fake, fake, 0, None, fake, None, None) == 0
+
+
+def test_cast_host_checks_reject_before_launch(L):
+    c = L.lib.lm_fp8_amax_scale_cast
+    fake = 0x10000
+    assert c(fake, 32, 32, 32, 5, 0, None, fake, fake, fake, fake, fake, None) == 4
+    assert c(fake, 32, 24, 24, 0, 0, None, fake, fake, fake, fake, None, None) == 3
+    assert c(fake, 24, 32, 32, 0, 0, None, fake, fake, fake, None, fake, None) == 3
+    assert c(fake, 32, 32, 16, 0, 0, None, fake, fake, fake, fake, fake, None) == 1
+    assert c(fake, 32, 32, 32, 0, 0, None, None, fake, fake, fake, fake, None) == 1
+    assert c(fake + 2, 32, 32, 32, 0, 0, None, fake, fake, fake, fake, fake, None) == 2
+
+
+def test_mlp_sizes_and_carve(L):
+    M, d, f = 256, 256, 1024
+    r = lambda n: (n + 255) // 256 * 256
+    assert L.lm_relu2_mlp_saved_bytes(M, d, f) == (2 * r(M * d) + 4 * r(f * d) + r(2 * M * f)
+                                                   + 2 * r(M * f) + r(64))
+    assert L.lm_relu2_mlp_workspace_size(M, d, f) == (2 * r(M * d) + r(2 * M * f)
+                                                      + 2 * r(M * f) + r(32))
+    assert L.lm_relu2_mlp_saved_bytes(M, d, 1000) == 0      # f not a multiple of 16
+    s = L.MlpSaved()
+    base = 0x100000
+    n = L.lm_relu2_mlp_saved_bytes(M, d, f)
+    assert L.lib.lm_relu2_mlp_saved_carve(base, n, M, d, f, ctypes.byref(s)) == 0
+    assert s.Xq == base and s.XqT == base + r(M * d) and s.scales == base + n - r(64)
+    assert L.lib.lm_relu2_mlp_saved_carve(base, n - 1, M, d, f, ctypes.byref(s)) == 1
+    assert L.lib.lm_relu2_mlp_saved_carve(base + 16, n, M, d, f, ctypes.byref(s)) == 2

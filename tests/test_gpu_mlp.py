@@ -1,0 +1,149 @@
+"""GPU parity of the relu^2 MLP forward and backward (single C-ABI calls)
+against the oracle's chain.
+
+Two kinds of check:
+  * end to end: the same bf16 inputs go to lm_relu2_mlp_fwd/bwd and to the
+    oracle chain; Y, dX, dW_up, dW_down within the stated tolerance;
+  * stagewise: every cast the library runs is checked bit-exact against the
+    oracle's cast of the GPU's own input to that cast (its H, its dH, its
+    amax), and every GEMM within tolerance against the oracle's GEMM of the
+    GPU's own codes and scales.
+"""
+import numpy as np
+import pytest
+import torch
+
+from fp8_gemms_b200 import synthetic
+from gpu_util import assert_close, f32, u8, u16
+
+pytestmark = pytest.mark.gpu
+
+E4M3, E5M2 = 0, 1
+
+
+@pytest.fixture(scope="module")
+def api():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from fp8_gemms_b200 import api as a
+    return a
+
+
+def run_chain(api, w):
+    t = w.tensors()
+    dev = {k: v.cuda() for k, v in t.items()}
+    mlp = api.Relu2Mlp(w.M, w.d, w.f)
+    Y = mlp.forward(dev["X"], dev["W_up"], dev["W_down"])
+    dX, dWu, dWd = mlp.backward(dev["dY"]) if w.backward else (None, None, None)
+    torch.cuda.synchronize()
+    from fp8_gemms_b200 import _lib
+    assert _lib.lm_get_error()[0] == 0
+    return t, mlp, Y, dX, dWu, dWd
+
+
+def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None):
+    """rows: sample of output rows to check for the M x * GEMMs (None = all)."""
+    sc = mlp.view("scales").cpu().numpy()
+    # casts of the inputs: bit-exact
+    for name, key, si in [("X", "Xq", 0), ("W_up", "Wuq", 1), ("W_down", "Wdq", 2)]:
+        ref = orc.amax_scale_cast(synthetic.bits_u16(t[name]), E4M3)
+        assert sc[si, 0] == ref["amax"] and sc[si, 1] == ref["scale"] and sc[si, 2] == ref["inv_scale"], name
+        assert np.array_equal(u8(mlp.view(key)), ref["q"]), name
+        assert np.array_equal(u8(mlp.view(key + "T")), ref["qT"]), name + "T"
+    Xq, Wuq, Wdq = u8(mlp.view("Xq")), u8(mlp.view("Wuq")), u8(mlp.view("Wdq"))
+    H = u16(mlp.view("H"))
+    # up GEMM (RELU2_FWD) from the GPU's codes and scales
+    Href, _ = orc.gemm(Xq, E4M3, Wuq, E4M3, sc[0, 2], sc[1, 2], orc.EPI_RELU2_FWD, rows=rows)
+    assert_close(H if rows is None else H[rows], Href, "H")
+    # amax of h from the epilogue == amax of the GPU's own H, bit-exact
+    assert sc[3, 0] == orc.amax(H, relu2_input=True)
+    # cast of h from the GPU's H and amax: bit-exact
+    s_h, inv_h = orc.scale(sc[3, 0], E4M3)
+    assert sc[3, 1] == s_h and sc[3, 2] == inv_h
+    hq_ref, hqT_ref = orc.cast(H, E4M3, s_h, relu2_input=True)
+    hq, hqT = u8(mlp.view("hq")), u8(mlp.view("hqT"))
+    assert np.array_equal(hq, hq_ref) and np.array_equal(hqT, hqT_ref)
+    # down GEMM
+    Yref, _ = orc.gemm(hq, E4M3, Wdq, E4M3, sc[3, 2], sc[2, 2], rows=rows)
+    assert_close(u16(Y) if rows is None else u16(Y)[rows], Yref, "Y")
+    if dX is None:
+        return
+    g = mlp.workspace_view("scales").cpu().numpy()
+    ref = orc.amax_scale_cast(synthetic.bits_u16(t["dY"]), E5M2)
+    assert g[0, 0] == ref["amax"] and g[0, 1] == ref["scale"] and g[0, 2] == ref["inv_scale"]
+    dYq, dYqT = u8(mlp.workspace_view("dYq")), u8(mlp.workspace_view("dYqT"))
+    assert np.array_equal(dYq, ref["q"]) and np.array_equal(dYqT, ref["qT"])
+    dH = u16(mlp.workspace_view("dH"))
+    dHref, _ = orc.gemm(dYq, E5M2, u8(mlp.view("WdqT")), E4M3, g[0, 2], sc[2, 2],
+                        orc.EPI_RELU2_BWD, aux=H, rows=rows)
+    assert_close(dH if rows is None else dH[rows], dHref, "dH")
+    assert g[1, 0] == orc.amax(dH)
+    s_dh, inv_dh = orc.scale(g[1, 0], E5M2)
+    assert g[1, 1] == s_dh and g[1, 2] == inv_dh
+    dHq_ref, dHqT_ref = orc.cast(dH, E5M2, s_dh)
+    dHq, dHqT = u8(mlp.workspace_view("dHq")), u8(mlp.workspace_view("dHqT"))
+    assert np.array_equal(dHq, dHq_ref) and np.array_equal(dHqT, dHqT_ref)
+    wrows = None if rows is None else np.arange(0, dWd.shape[0], max(1, dWd.shape[0] // 24))
+    ref_dWd, _ = orc.gemm(dYqT, E5M2, hqT, E4M3, g[0, 2], sc[3, 2], rows=wrows)
+    assert_close(u16(dWd) if wrows is None else u16(dWd)[wrows], ref_dWd, "dW_down")
+    ref_dX, _ = orc.gemm(dHq, E5M2, u8(mlp.view("WuqT")), E4M3, g[1, 2], sc[1, 2], rows=rows)
+    assert_close(u16(dX) if rows is None else u16(dX)[rows], ref_dX, "dX")
+    urows = None if rows is None else np.arange(0, dWu.shape[0], max(1, dWu.shape[0] // 24))
+    ref_dWu, _ = orc.gemm(dHqT, E5M2, u8(mlp.view("XqT")), E4M3, g[1, 2], sc[0, 2], rows=urows)
+    assert_close(u16(dWu) if urows is None else u16(dWu)[urows], ref_dWu, "dW_up")
+
+
+def test_tiny_mlp_end_to_end(orc, api):
+    """Tiny relu^2 MLP block fwd+bwd: X [256x256], W_up [1024x256],
+    W_down [256x1024], dY [256x256]; GPU chain vs oracle chain."""
+    w = synthetic.TINY_MLP
+    t, mlp, Y, dX, dWu, dWd = run_chain(api, w)
+    b = {k: synthetic.bits_u16(v) for k, v in t.items()}
+    fwd = orc.mlp_fwd(b["X"], b["W_up"], b["W_down"])
+    bwd = orc.mlp_bwd(b["dY"], fwd)
+    assert_close(u16(Y), fwd["Y"], "Y")
+    assert_close(u16(dX), bwd["dX"], "dX")
+    assert_close(u16(dWu), bwd["dW_up"], "dW_up")
+    assert_close(u16(dWd), bwd["dW_down"], "dW_down")
+
+
+def test_tiny_mlp_stagewise(orc, api):
+    w = synthetic.TINY_MLP
+    t, mlp, Y, dX, dWu, dWd = run_chain(api, w)
+    check_stagewise(orc, mlp, t, Y, dX, dWu, dWd)
+
+
+def test_mlp_ragged_shapes(orc, api):
+    """M, d, f multiples of 16 but not of any tile: every GEMM and cast has a
+    ragged tail."""
+    w = synthetic.MlpWorkload("ragged", 272, 208, 848, True)
+    t, mlp, Y, dX, dWu, dWd = run_chain(api, w)
+    check_stagewise(orc, mlp, t, Y, dX, dWu, dWd)
+
+
+def test_mlp_student_t_inputs(orc, api):
+    w = synthetic.MlpWorkload("t3", 512, 256, 1024, True, ("t3", None), 5)
+    t, mlp, Y, dX, dWu, dWd = run_chain(api, w)
+    check_stagewise(orc, mlp, t, Y, dX, dWu, dWd)
+
+
+def test_mlp_repeated_calls_are_deterministic(orc, api):
+    w = synthetic.TINY_MLP
+    t, mlp, Y, dX, dWu, dWd = run_chain(api, w)
+    dev = {k: v.cuda() for k, v in t.items()}
+    Y2 = mlp.forward(dev["X"], dev["W_up"], dev["W_down"])
+    dX2, dWu2, dWd2 = mlp.backward(dev["dY"])
+    torch.cuda.synchronize()
+    for a, b in [(Y, Y2), (dX, dX2), (dWu, dWu2), (dWd, dWd2)]:
+        assert torch.equal(a, b)
+
+
+@pytest.mark.slow
+def test_full_size_mlp_sampled(orc, api):
+    """The 3.8B-shape block (M=16384, d=3072, f=12288) fwd+bwd in the launch
+    configuration bench.py times: casts bit-exact over whole tensors, GEMM
+    outputs on sampled rows."""
+    w = synthetic.MLP_FWD_BWD
+    t, mlp, Y, dX, dWu, dWd = run_chain(api, w)
+    rows = np.concatenate([np.arange(0, 16), np.arange(w.M - 16, w.M),
+                           np.random.default_rng(0).choice(w.M, 16, replace=False)])
+    check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=np.sort(rows))
