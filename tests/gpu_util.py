@@ -6,6 +6,12 @@ import torch
 # GEMM / MLP outputs (bf16): elementwise |d| <= 1e-2 |ref| + 1e-3 rms(ref),
 # and normwise ||d||_F / ||ref||_F <= 5e-3.
 ELEM_REL, ELEM_RMS, NORM_REL = 1e-2, 1e-3, 5e-3
+# The relu^2-backward epilogue rounds twice: g = bf16(acc s), then
+# dH = bf16(g * 2 relu(H)).  fp32 tensor-core accumulation and the oracle's
+# fp64 sum can put g one bf16 ulp apart; the second rounding can then leave
+# dH two ulps apart, i.e. up to 2 * 2^-7 = 2^-6 of |dH|.  Elementwise bound for
+# that epilogue's output: 2^-6 |ref| + 1e-3 rms(ref) (normwise bound unchanged).
+ELEM_REL_RELU2_BWD = 2.0 ** -6
 
 
 def u16(t):
@@ -34,7 +40,7 @@ def f32(t):
     return np.float32(t.detach().cpu().numpy().reshape(-1)[0])
 
 
-def assert_close(got_bits, ref_bits, what=""):
+def assert_close(got_bits, ref_bits, what="", elem_rel=ELEM_REL):
     g = bf16_to_f64(got_bits)
     r = bf16_to_f64(ref_bits)
     assert g.shape == r.shape, (what, g.shape, r.shape)
@@ -43,7 +49,7 @@ def assert_close(got_bits, ref_bits, what=""):
         return
     rms = float(np.sqrt(np.mean(r * r)))
     d = np.abs(g - r)
-    bound = ELEM_REL * np.abs(r) + ELEM_RMS * rms
+    bound = elem_rel * np.abs(r) + ELEM_RMS * rms
     bad = d > bound
     assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} elements out of tolerance; "
                            f"worst |d|={d.max():.3e} at {np.unravel_index(d.argmax(), d.shape)}, "
@@ -51,3 +57,15 @@ def assert_close(got_bits, ref_bits, what=""):
     nr = np.linalg.norm(r)
     if nr > 0:
         assert np.linalg.norm(g - r) / nr <= NORM_REL, f"{what}: normwise {np.linalg.norm(g - r) / nr:.3e}"
+
+
+def bf16_neighbours(bits):
+    """The bf16 values one ulp below and above each value (bits, same shape)."""
+    b = np.asarray(bits, np.uint16).astype(np.int32)
+    mag, neg = b & 0x7FFF, (b & 0x8000) != 0
+    up_mag = np.minimum(mag + 1, 0x7F7F)
+    dn_mag = np.where(mag == 0, 1, mag - 1)       # below +-0 is the smallest subnormal
+    dn_neg = np.where(mag == 0, ~neg, neg)
+    toward_big = np.where(neg, up_mag | 0x8000, up_mag)
+    toward_small = np.where(dn_neg, dn_mag | 0x8000, dn_mag)
+    return toward_small.astype(np.uint16), toward_big.astype(np.uint16)

@@ -8,7 +8,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import assert_close, bf16_to_f64, f32, from_u8, from_u16, u16
+from gpu_util import (ELEM_REL, ELEM_REL_RELU2_BWD, assert_close, bf16_neighbours, bf16_to_f64,
+                      f32, from_u8, from_u16, u16)
 
 pytestmark = pytest.mark.gpu
 
@@ -49,7 +50,19 @@ def run(lib, orc, M, N, K, fa=E4M3, fb=E4M3, epi=EPI_NONE, inv_a=0.02, inv_b=0.5
     assert lib.lm_get_error()[0] == 0
     ref, ref_amax = orc.gemm(A, fa, B, fb, np.float32(inv_a), np.float32(inv_b), epi=epi, aux=aux)
     got = u16(D)
-    assert_close(got, ref, f"gemm M={M} N={N} K={K} fa={fa} fb={fb} epi={epi}")
+    assert_close(got, ref, f"gemm M={M} N={N} K={K} fa={fa} fb={fb} epi={epi}",
+                 ELEM_REL_RELU2_BWD if epi == EPI_RELU2_BWD else ELEM_REL)
+    if epi == EPI_RELU2_BWD:
+        # exact epilogue arithmetic: dH = bf16(g' * 2 relu(H)) for a g' equal to,
+        # or one bf16 ulp from, the oracle's g = bf16(acc s)
+        g, _ = orc.gemm(A, fa, B, fb, np.float32(inv_a), np.float32(inv_b))
+        h = torch.from_numpy(aux.view(np.int16)).view(torch.bfloat16).float()
+        ok = np.zeros(got.shape, bool)
+        for cand in (g, *bf16_neighbours(g)):
+            gc = torch.from_numpy(cand.view(np.int16)).view(torch.bfloat16).float()
+            dh = u16((gc * 2.0 * torch.relu(h)).to(torch.bfloat16))  # exact product, one rounding
+            ok |= dh == got
+        assert ok.all(), f"{int((~ok).sum())} dH elements not explained by g within 1 ulp"
     # the amax written by the epilogue is exactly the amax of the GPU's own D
     own = orc.amax(got, relu2_input=(epi == EPI_RELU2_FWD))
     assert f32(am) == own

@@ -14,7 +14,7 @@ import pytest
 import torch
 
 from fp8_gemms_b200 import synthetic
-from gpu_util import assert_close, f32, u8, u16
+from gpu_util import ELEM_REL_RELU2_BWD, assert_close, f32, u8, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -75,7 +75,7 @@ def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None):
     dH = u16(mlp.workspace_view("dH"))
     dHref, _ = orc.gemm(dYq, E5M2, u8(mlp.view("WdqT")), E4M3, g[0, 2], sc[2, 2],
                         orc.EPI_RELU2_BWD, aux=H, rows=rows)
-    assert_close(dH if rows is None else dH[rows], dHref, "dH")
+    assert_close(dH if rows is None else dH[rows], dHref, "dH", ELEM_REL_RELU2_BWD)
     assert g[1, 0] == orc.amax(dH)
     s_dh, inv_dh = orc.scale(g[1, 0], E5M2)
     assert g[1, 1] == s_dh and g[1, 2] == inv_dh
