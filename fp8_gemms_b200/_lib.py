@@ -21,7 +21,8 @@ STATUS = {0: "LM_OK", 1: "LM_ERR_INVALID_ARG", 2: "LM_ERR_ALIGNMENT",
 
 EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
             "lm_relu2_mlp_saved_carve", "lm_relu2_mlp_workspace_size", "lm_relu2_mlp_fwd",
-            "lm_relu2_mlp_bwd", "lm_get_error", "lm_status_string", "lm_version"]
+            "lm_relu2_mlp_bwd", "lm_get_error", "lm_status_string", "lm_version",
+            "lm_timing_attach", "lm_timing_detach", "lm_timing_kinds"]
 
 
 class LmError(RuntimeError):
@@ -63,6 +64,12 @@ def _load():
     L.lm_status_string.argtypes = [st]
     L.lm_status_string.restype = ctypes.c_char_p
     L.lm_version.restype = ctypes.c_int
+    L.lm_timing_attach.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
+    L.lm_timing_attach.restype = None
+    L.lm_timing_detach.argtypes = []
+    L.lm_timing_detach.restype = i32
+    L.lm_timing_kinds.argtypes = [ctypes.c_char_p, i32]
+    L.lm_timing_kinds.restype = i32
     return L
 
 
@@ -155,3 +162,32 @@ def lm_status_string(status):
 
 def lm_version():
     return lib.lm_version()
+
+
+class KernelTimer:
+    """Context manager over lm_timing_attach/detach: records a CUDA event before
+    every library kernel launched on this host thread (at most `capacity`).
+    After exit, `.kinds` labels each launch and `.durations_ms(end_event)`
+    gives per-launch times, the last one ending at `end_event`."""
+
+    def __init__(self, capacity=64):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(capacity)]
+        for e in self.events:       # torch creates the CUDA event on first record
+            e.record()
+        self._arr = (ctypes.c_void_p * capacity)(*[e.cuda_event for e in self.events])
+        self.n = 0
+        self.kinds = ""
+
+    def __enter__(self):
+        lib.lm_timing_attach(self._arr, len(self.events))
+        return self
+
+    def __exit__(self, *exc):
+        self.n = lib.lm_timing_detach()
+        buf = ctypes.create_string_buffer(self.n + 1)
+        k = lib.lm_timing_kinds(buf, self.n)
+        self.kinds = buf.raw[:k].decode()
+
+    def durations_ms(self, end_event):
+        marks = self.events[:self.n] + [end_event]
+        return [a.elapsed_time(b) for a, b in zip(marks[:-1], marks[1:])]

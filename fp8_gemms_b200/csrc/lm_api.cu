@@ -38,7 +38,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     });
     return fn;
 }
+struct TimingState {
+    void* const* events = nullptr;
+    int capacity = 0;
+    int count = 0;
+    char kinds[512];
+};
+thread_local TimingState t_timing;
 }  // namespace
+
+void timing_mark(cudaStream_t s, char kind) {
+    TimingState& t = t_timing;
+    if (!t.events || t.count >= t.capacity) return;
+    cudaEventRecord(static_cast<cudaEvent_t>(t.events[t.count]), s);
+    if (t.count < (int)sizeof(t.kinds)) t.kinds[t.count] = kind;
+    ++t.count;
+}
 
 unsigned int* device_error_word() {
     int dev = current_device();
@@ -79,6 +94,20 @@ bool encode_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
     return r == CUDA_SUCCESS;
 }
 
+bool encode_tmap_bf16_sw64(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                           uint32_t box_rows, uint32_t box_cols) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace lm
 
 extern "C" {
@@ -112,5 +141,25 @@ const char* lm_status_string(lm_status s) {
 }
 
 int lm_version(void) { return 100; }
+
+void lm_timing_attach(void* const* events, int capacity) {
+    lm::t_timing.events = events;
+    lm::t_timing.capacity = events ? capacity : 0;
+    lm::t_timing.count = 0;
+}
+
+int lm_timing_detach(void) {
+    lm::t_timing.events = nullptr;
+    lm::t_timing.capacity = 0;
+    return lm::t_timing.count;
+}
+
+int lm_timing_kinds(char* out, int cap) {
+    const int n = lm::t_timing.count < (int)sizeof(lm::t_timing.kinds) ? lm::t_timing.count
+                                                                        : (int)sizeof(lm::t_timing.kinds);
+    const int m = n < cap ? n : cap;
+    for (int i = 0; i < m; ++i) out[i] = lm::t_timing.kinds[i];
+    return m;
+}
 
 }  // extern "C"

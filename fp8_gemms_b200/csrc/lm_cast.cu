@@ -96,16 +96,23 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
                                                         unsigned int* __restrict__ amax_bits) {
     uint32_t m = 0;
     const int64_t vpr = cols >> 3;  // 16-byte vectors per row
+    const int64_t nvec = rows * vpr;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
+    int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     if (ld == cols) {
-        const int64_t nvec = rows * vpr;
         const uint4* xv = reinterpret_cast<const uint4*>(x);
-        for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nvec; i += stride)
-            m = absmax8<RELU2>(ld_stream_v4(xv + i), m);
+        // eight independent 16-byte loads in flight per thread
+        for (; i + 7 * stride < nvec; i += 8 * stride) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = ld_stream_v4(xv + i + u * stride);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) m = absmax8<RELU2>(v[u], m);
+        }
+        for (; i < nvec; i += stride) m = absmax8<RELU2>(ld_stream_v4(xv + i), m);
     } else {
-        const int64_t nvec = rows * vpr;
-        for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nvec; i += stride) {
-            int64_t r = i / vpr, c = (i - r * vpr) << 3;
+        for (; i < nvec; i += stride) {
+            const int64_t r = i / vpr, c = (i - r * vpr) << 3;
             m = absmax8<RELU2>(ld_stream_v4(x + r * ld + c), m);
         }
     }
@@ -158,17 +165,24 @@ __global__ void __launch_bounds__(kThreads) cast_kernel(
     const int c0 = (t % tiles_c) * kCastCols;
     const int tid = threadIdx.x;
 
-    // load 16 bytes of bf16 -> 8 codes; row-major codes straight to q
-#pragma unroll 4
-    for (int it = 0; it < (kCastRows * kCastCols / 8) / kThreads; ++it) {
+    // all sixteen 16-byte loads of this thread in flight, then convert:
+    // 8 bf16 -> 8 codes per load; row-major codes straight to q
+    constexpr int kIters = (kCastRows * kCastCols / 8) / kThreads;
+    uint4 xin[kIters];
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+        const int idx = it * kThreads + tid;
+        const int r = r0 + (idx >> 4), c = c0 + (idx & 15) * 8;
+        xin[it] = (r < rows && c < cols) ? ld_stream_v4(x + (int64_t)r * ld + c)
+                                       : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
         const int idx = it * kThreads + tid;
         const int rr = idx >> 4, ch = idx & 15;
         const int r = r0 + rr, c = c0 + ch * 8;
-        uint2 codes = make_uint2(0u, 0u);
-        if (r < rows && c < cols) {
-            codes = convert8<FMT, RELU2>(ld_stream_v4(x + (int64_t)r * ld + c), scale);
-            if (q) *reinterpret_cast<uint2*>(q + (int64_t)r * cols + c) = codes;
-        }
+        const uint2 codes = convert8<FMT, RELU2>(xin[it], scale);
+        if (q && r < rows && c < cols) *reinterpret_cast<uint2*>(q + (int64_t)r * cols + c) = codes;
         *reinterpret_cast<uint2*>(&tile[rr][ch * 2]) = codes;
     }
     if (!qT) return;
@@ -211,6 +225,7 @@ void launch_cast(const uint16_t* x, int rows, int cols, int64_t ld, const float*
     const int tiles_r = (rows + kCastRows - 1) / kCastRows;
     const int tiles_c = (cols + kCastCols - 1) / kCastCols;
     const int n = tiles_r * tiles_c;
+    timing_mark(s, 'c');
     cast_kernel<FMT, RELU2><<<n, kThreads, 0, s>>>(x, rows, cols, ld, amax_src, amax_out,
                                                   scale_out, inv_out, q, qT, tiles_c, n);
 }
@@ -239,6 +254,7 @@ extern "C" lm_status lm_fp8_amax_scale_cast(const void* x, int64_t rows, int64_t
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     const float* amax_src = amax_in;
     if (!amax_in) {
+        if (!empty) timing_mark(s, 'a');
         if (cudaMemsetAsync(amax_out, 0, sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
         if (!empty) {
             int grid = sm_count() * 4;
@@ -253,6 +269,7 @@ extern "C" lm_status lm_fp8_amax_scale_cast(const void* x, int64_t rows, int64_t
         amax_src = amax_out;
     }
     if (empty || (!q && !qT)) {
+        timing_mark(s, 's');
         scales_only_kernel<<<1, 1, 0, s>>>(amax_src, fmax, amax_out, scale_out, inv_scale_out);
         return launch_status();
     }

@@ -3,21 +3,26 @@
 // The pages run all three GEMMs of each linear in FP8 with one fp32 scale
 // per operand, bf16 out (decomputer.nl, "Het trainen van een 3.8B LLM tot
 // 0.384 CORE voor $998", section "Doorvoer (Throughput) verhogen", FP8
-// bullet; manulx.blog names the library call, torch._scaled_mm).  This is
-// a kernel of our own for B200 instead of that library call:
+// bullet; manulx.blog names the library call, torch._scaled_mm).  These are
+// kernels of our own for B200 in place of that library call.
 //
-//  * persistent grid, one CTA per SM, tiles of 128 x 256 outputs visited in
-//    groups of 16 M-blocks so that concurrently running CTAs share A and B
-//    panels in L2;
-//  * warp 0: one thread issues TMA tile loads (128-byte swizzle, K-major) into
-//    a 4-stage shared-memory ring guarded by full/empty mbarriers;
-//  * warp 1: one thread issues tcgen05.mma kind::f8f6f4 (128 x 256 x 32 per
-//    instruction) into a TMEM fp32 accumulator; two accumulators of 256
-//    columns (all 512 TMEM columns) let the epilogue of one tile overlap the
-//    main loop of the next;
-//  * warps 2-5: epilogue -- tcgen05.ld of 32 columns at a time, dequant scale,
-//    relu^2 (forward) or 2 relu(H) g (backward), bf16 stores, and the amax of
-//    what the next cast consumes (atomicMax on fp32 bits, order independent).
+// Main kernel (M > 128): a CTA pair (cluster of 2, cta_group::2) computes a
+// 256 x 256 output tile.  Each CTA TMA-loads its own 128 rows of A and its
+// own 128 rows (N) of B into a 6-stage shared-memory ring; both loads count
+// on the leader CTA's "full" mbarrier; the leader issues tcgen05.mma
+// kind::f8f6f4 with M = 256, N = 256, K = 32, reading both CTAs' shared
+// memory, so each SM streams half of B instead of all of it.  Accumulators
+// live in TMEM (2 x 256 fp32 columns per CTA, double-buffered so the
+// epilogue of one tile overlaps the main loop of the next).  The epilogue
+// warps of each CTA drain their own 128 rows: tcgen05.ld -> dequant scale ->
+// relu^2 / relu^2' -> bf16 -> 64B-swizzled shared staging -> TMA store, and
+// reduce the amax of what the next cast consumes.  No TMA load uses cluster
+// multicast; only the MMA-completion commits are multicast to the pair.
+//
+// Thin kernel (M <= 128): one CTA per 128 x 256 tile (cta_group::1), same
+// ring and TMEM double buffer, per-thread global stores.
+//
+// Every mbarrier wait is bounded (see lm_ptx.cuh).
 #include <cuda_bf16.h>
 
 #include "lm_internal.h"
@@ -26,21 +31,16 @@
 namespace lm {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128;  // BK in bytes = FP8 elements
-constexpr int UMMA_K = 32;                   // K per tcgen05.mma for 8-bit inputs
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK;
-constexpr int B_BYTES = BN * BK;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 192;
-constexpr int NUM_EPI_THREADS = 128;
-constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr int GROUP_M = 16;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int BK = 128;     // K bytes (= FP8 elements) per pipeline stage
+constexpr int UMMA_K = 32;  // K per tcgen05.mma for 8-bit inputs
+constexpr int NUM_THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int NUM_EPI_WARPS = 4;
 
 // codes recorded in the device error word when a bounded wait runs out
-enum : unsigned { W_EMPTY = 0x101, W_TEMPTY = 0x102, W_FULL = 0x103, W_DRAIN = 0x104,
-                  W_TFULL = 0x105, W_LOADS = 0x106 };
+enum : unsigned {
+    W_EMPTY = 0x101, W_TEMPTY = 0x102, W_FULL = 0x103, W_DRAIN = 0x104, W_TFULL = 0x105,
+    W_LOADS = 0x106, W_AUX = 0x107
+};
 
 struct GemmArgs {
     int M, N, num_mb, num_nb, num_kb, num_tiles;
@@ -53,6 +53,9 @@ struct GemmArgs {
     uint32_t idesc;
 };
 
+// Tile visiting order: groups of GROUP_M row-blocks, column-blocks within a
+// group, so the tiles in flight at once share A and B panels in L2.
+template <int GROUP_M>
 __device__ __forceinline__ void tile_coords(int t, int num_mb, int num_nb, int& mb, int& nb) {
     const int per_group = GROUP_M * num_nb;
     const int g = t / per_group;
@@ -66,6 +69,318 @@ __device__ __forceinline__ void tile_coords(int t, int num_mb, int num_nb, int& 
 __device__ __forceinline__ uint32_t bf16_bits(float v) {
     return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
+
+// One accumulator value -> bf16 output bits under the epilogue, updating the
+// running amax (bf16 bits) of what the next cast consumes.
+template <int EPI>
+__device__ __forceinline__ uint32_t epi_value(uint32_t acc_bits, float s, uint32_t h_bits,
+                                              uint32_t& amax) {
+    uint32_t b = bf16_bits(__fmul_rn(__uint_as_float(acc_bits), s));
+    if (EPI == LM_EPI_RELU2_BWD) {
+        const float g = __uint_as_float(b << 16);
+        const float h = __uint_as_float(h_bits << 16);
+        const float rh = h > 0.f ? h : 0.f;
+        b = bf16_bits(__fmul_rn(__fmul_rn(g, 2.0f), rh));
+    }
+    if (EPI == LM_EPI_RELU2_FWD)
+        amax = (b & 0x8000u) ? amax : max(amax, b);  // max of relu(H)
+    else
+        amax = max(amax, b & 0x7FFFu);
+    return b;
+}
+
+// Final per-warp amax reduction into the fp32 bits at amax_out.
+template <int EPI>
+__device__ __forceinline__ void reduce_amax(uint32_t amax, float* amax_out, int lane) {
+    if (!amax_out) return;
+    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, amax);
+    if (lane == 0 && m) {
+        uint32_t bits = m << 16;
+        if (EPI == LM_EPI_RELU2_FWD) {
+            // max h = bf16(max(relu H)^2): squaring and rounding are monotone
+            const float r = __uint_as_float(bits);
+            bits = bf16_bits(__fmul_rn(r, r)) << 16;
+        }
+        atomicMax(reinterpret_cast<unsigned int*>(amax_out), bits);
+    }
+}
+
+// =====================================================================
+// CTA-pair kernel: 256 x 256 tiles, cta_group::2
+// =====================================================================
+namespace pair {
+
+constexpr int TILE_M = 256, TILE_N = 256;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = 128 * BK;  // this CTA's 128 rows of A
+constexpr int B_BYTES = 128 * BK;  // this CTA's 128 rows (N) of B
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int EPI_COLS = 32;                   // columns per epilogue chunk
+constexpr int BOX_BYTES = 32 * EPI_COLS * 2;   // one warp's 32 x 32 bf16 box
+constexpr int STORE_BYTES = NUM_EPI_WARPS * 2 * BOX_BYTES;
+constexpr int AUX_BYTES = NUM_EPI_WARPS * 2 * BOX_BYTES;
+constexpr uint32_t TMEM_COLS = 2 * TILE_N;
+constexpr int GROUP_M = 8;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + AUX_BYTES + 1024 + 512;
+
+// Offset of 16-byte chunk j of row r in a 32-row x 64-byte box written or
+// read by a TMA with CU_TENSOR_MAP_SWIZZLE_64B: chunk bits [4,6) are XORed
+// with address bits [7,9), i.e. with (r >> 1) & 3.
+__device__ __forceinline__ uint32_t sw64(int r, int j) {
+    return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    gemm_fp8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmD,
+                         const __grid_constant__ CUtensorMap tmAux, const GemmArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + STAGES * A_BYTES;
+    uint8_t* sStore = sB + STAGES * B_BYTES;
+    uint8_t* sAux = sStore + STORE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sAux + AUX_BYTES);
+    uint64_t* full = bars;                  // [STAGES], used in the leader only
+    uint64_t* empty = full + STAGES;        // [STAGES], both CTAs
+    uint64_t* tfull = empty + STAGES;       // [2], both CTAs
+    uint64_t* tempty = tfull + 2;           // [2], leader only
+    uint64_t* drain = tempty + 2;           // leader only
+    uint64_t* auxbar = drain + 1;           // [4 warps][2 buffers]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + 2 * NUM_EPI_WARPS);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 2 * NUM_EPI_WARPS);
+        }
+        mbar_init(drain, 1);
+        for (int i = 0; i < 2 * NUM_EPI_WARPS; ++i) mbar_init(&auxbar[i], 1);
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmD);
+        if (EPI == LM_EPI_RELU2_BWD) tma_prefetch_desc(&tmAux);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------- TMA producer (both CTAs)
+            const uint32_t full_leader = map_to_rank(smem_addr(full), 0);
+            int stage = 0;
+            uint32_t phase = 0, issued = 0;
+            bool ok = true;
+            for (int t = cluster; t < args.num_tiles && ok; t += nclusters) {
+                int mb, nb;
+                tile_coords<GROUP_M>(t, args.num_mb, args.num_nb, mb, nb);
+                const int arow = mb * TILE_M + (int)rank * 128;
+                const int brow = nb * TILE_N + (int)rank * 128;
+                for (int kb = 0; kb < args.num_kb; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, args.err, W_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+                    const uint32_t bar = full_leader + (uint32_t)(stage * 8);
+                    tma_load_2d_pair(smem_addr(sA + stage * A_BYTES), &tmA, bar, kb * BK, arow);
+                    tma_load_2d_pair(smem_addr(sB + stage * B_BYTES), &tmB, bar, kb * BK, brow);
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (leader) {
+                // both CTAs' loads of every armed phase have landed before exit
+                for (int s = 0; s < STAGES; ++s) {
+                    const uint32_t n = issued / STAGES + ((uint32_t)s < issued % STAGES ? 1u : 0u);
+                    if (n) mbar_wait(&full[s], (n - 1) & 1u, args.err, W_LOADS);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ------------------------------------------- MMA issuer (leader)
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = cluster; t < args.num_tiles && ok; t += nclusters) {
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.err, W_TEMPTY)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TILE_N);
+                for (int kb = 0; kb < args.num_kb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, args.err, W_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc_k128(smem_addr(sA + stage * A_BYTES));
+                    const uint64_t bd = smem_desc_k128(smem_addr(sB + stage * B_BYTES));
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk)
+                        mma_fp8_pair(d_tmem, ad + (uint64_t)(kk * UMMA_K / 16),
+                                     bd + (uint64_t)(kk * UMMA_K / 16), args.idesc,
+                                     (kb | kk) != 0 ? 1u : 0u);
+                    mma_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit_pair(&tfull[acc], 0x3);  // accumulator ready in both CTAs
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            mma_commit_pair(drain, 0x1);  // all MMAs retired before teardown
+            mbar_wait(drain, 0, args.err, W_DRAIN);
+        }
+    } else {
+        // ------------------------------------------- epilogue (both CTAs)
+        const int wi = warp - 2;       // staging slot
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        uint8_t* st_buf = sStore + wi * 2 * BOX_BYTES;
+        uint8_t* ax_buf = sAux + wi * 2 * BOX_BYTES;
+        uint64_t* ax_bar = auxbar + wi * 2;
+        const uint32_t tempty_leader = map_to_rank(smem_addr(tempty), 0);
+        const float s = __fmul_rn(*args.inv_a, *args.inv_b);
+        uint32_t amax = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        uint32_t ax_phase = 0;  // bit b: parity of the next wait on aux buffer b
+        uint32_t n_stores = 0;
+        bool ok = true;
+        for (int t = cluster; t < args.num_tiles && ok; t += nclusters) {
+            int mb, nb;
+            tile_coords<GROUP_M>(t, args.num_mb, args.num_nb, mb, nb);
+            const int grow = mb * TILE_M + (int)rank * 128 + quarter * 32;  // row of lane 0
+            const int gcol = nb * TILE_N;
+            const int left = args.N - gcol;
+            const int n_chunks = left >= TILE_N ? TILE_N / EPI_COLS : (left + EPI_COLS - 1) / EPI_COLS;
+            if (EPI == LM_EPI_RELU2_BWD && lane == 0) {
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(&ax_bar[0], BOX_BYTES);
+                tma_load_2d(smem_addr(ax_buf), &tmAux, &ax_bar[0], gcol, grow);
+            }
+            if (!mbar_wait(&tfull[acc], acc_phase, args.err, W_TFULL)) break;
+            tc_fence_after();
+            const uint32_t tbase =
+                tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * TILE_N);
+            for (int c = 0; c < n_chunks; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tbase + (uint32_t)(c * EPI_COLS), r);
+                tmem_ld_wait();
+                uint32_t hb[32];
+                if (EPI == LM_EPI_RELU2_BWD) {
+                    const int b = c & 1;
+                    if (lane == 0 && c + 1 < n_chunks) {
+                        fence_proxy_async_smem();
+                        mbar_arrive_expect_tx(&ax_bar[b ^ 1], BOX_BYTES);
+                        tma_load_2d(smem_addr(ax_buf + (b ^ 1) * BOX_BYTES), &tmAux, &ax_bar[b ^ 1],
+                                    gcol + (c + 1) * EPI_COLS, grow);
+                    }
+                    if (!mbar_wait(&ax_bar[b], (ax_phase >> b) & 1u, args.err, W_AUX)) {
+                        ok = false;
+                        break;
+                    }
+                    ax_phase ^= 1u << b;
+                    const uint8_t* src = ax_buf + b * BOX_BYTES;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(src + sw64(lane, j));
+                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            hb[8 * j + 2 * i] = w[i] & 0xFFFFu;
+                            hb[8 * j + 2 * i + 1] = w[i] >> 16;
+                        }
+                    }
+                }
+                uint32_t packed[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t lo = epi_value<EPI>(r[2 * i], s, hb[2 * i], amax);
+                    const uint32_t hi = epi_value<EPI>(r[2 * i + 1], s, hb[2 * i + 1], amax);
+                    packed[i] = lo | (hi << 16);
+                }
+                // staging buffer n_stores & 1: the store that last used it must
+                // have finished reading shared memory
+                uint8_t* dst = st_buf + (n_stores & 1u) * BOX_BYTES;
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    *reinterpret_cast<uint4*>(dst + sw64(lane, j)) =
+                        make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                                   packed[4 * j + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmD, smem_addr(dst), gcol + c * EPI_COLS, grow);
+                    bulk_commit_group();
+                }
+                ++n_stores;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(tempty_leader + (uint32_t)(acc * 8));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+        if (lane == 0) bulk_wait_group<0>();
+        reduce_amax<EPI>(amax, args.amax_out, lane);
+    }
+
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync();  // peer shared memory and TMEM no longer in use
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace pair
+
+// =====================================================================
+// Single-CTA kernel for thin problems (M <= 128): 128 x 256 tiles
+// =====================================================================
+namespace one {
+
+constexpr int BM = 128, BN = 256;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK;
+constexpr int B_BYTES = BN * BK;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_EPI_THREADS = 128;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int GROUP_M = 16;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -112,14 +427,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------------------------------------- TMA producer
             int stage = 0;
-            uint32_t phase = 0;
-            uint32_t issued = 0;
+            uint32_t phase = 0, issued = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
                 int mb, nb;
-                tile_coords(t, args.num_mb, args.num_nb, mb, nb);
+                tile_coords<GROUP_M>(t, args.num_mb, args.num_nb, mb, nb);
                 for (int kb = 0; kb < args.num_kb; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, args.err, W_EMPTY)) {
                         ok = false;
@@ -137,8 +450,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
             }
-            // every load this CTA issued has landed before shared memory is
-            // released (already true on the normal path: the MMA waited)
             for (int s = 0; s < STAGES; ++s) {
                 const uint32_t n = issued / STAGES + ((uint32_t)s < issued % STAGES ? 1u : 0u);
                 if (n) mbar_wait(&full[s], (n - 1) & 1u, args.err, W_LOADS);
@@ -146,7 +457,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // ------------------------------------------------ MMA issuer
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -180,20 +490,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
             }
-            // all MMAs retired before TMEM is deallocated
             mma_commit(drain);
             mbar_wait(drain, 0, args.err, W_DRAIN);
         }
     } else {
-        // ---------------------------------------------------- epilogue
-        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int quarter = warp & 3;
         const float s = __fmul_rn(*args.inv_a, *args.inv_b);
-        uint32_t amax = 0;  // bf16 bits of the running max
+        uint32_t amax = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
             int mb, nb;
-            tile_coords(t, args.num_mb, args.num_nb, mb, nb);
+            tile_coords<GROUP_M>(t, args.num_mb, args.num_nb, mb, nb);
             if (!mbar_wait(&tfull[acc], acc_phase, args.err, W_TFULL)) break;
             tc_fence_after();
             const int row = mb * BM + quarter * 32 + lane;
@@ -211,7 +519,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                     if (col0 + v * 8 >= args.N) break;
-                    uint32_t hb[8];
+                    uint32_t hb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
                     if (EPI == LM_EPI_RELU2_BWD) {
                         const uint4 a4 = *reinterpret_cast<const uint4*>(args.aux + off + v * 8);
                         const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w};
@@ -223,21 +531,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                     uint32_t ob[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float y = __fmul_rn(__uint_as_float(r[v * 8 + i]), s);
-                        uint32_t b = bf16_bits(y);
-                        if (EPI == LM_EPI_RELU2_BWD) {
-                            const float g = __uint_as_float(b << 16);
-                            const float h = __uint_as_float(hb[i] << 16);
-                            const float rh = h > 0.f ? h : 0.f;
-                            b = bf16_bits(__fmul_rn(__fmul_rn(g, 2.0f), rh));
-                        }
-                        ob[i] = b;
-                        if (EPI == LM_EPI_RELU2_FWD)
-                            amax = (b & 0x8000u) ? amax : max(amax, b);
-                        else
-                            amax = max(amax, b & 0x7FFFu);
-                    }
+                    for (int i = 0; i < 8; ++i) ob[i] = epi_value<EPI>(r[v * 8 + i], s, hb[i], amax);
                     *reinterpret_cast<uint4*>(args.D + off + v * 8) =
                         make_uint4(ob[0] | (ob[1] << 16), ob[2] | (ob[3] << 16),
                                    ob[4] | (ob[5] << 16), ob[6] | (ob[7] << 16));
@@ -248,18 +542,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
-        if (args.amax_out) {
-            uint32_t m = __reduce_max_sync(0xFFFFFFFFu, amax);
-            if (lane == 0 && m) {
-                uint32_t bits = m << 16;
-                if (EPI == LM_EPI_RELU2_FWD) {
-                    // max h = bf16(max(relu H)^2): squaring and rounding are monotone
-                    const float r = __uint_as_float(bits);
-                    bits = bf16_bits(__fmul_rn(r, r)) << 16;
-                }
-                atomicMax(reinterpret_cast<unsigned int*>(args.amax_out), bits);
-            }
-        }
+        reduce_amax<EPI>(amax, args.amax_out, lane);
     }
 
     tc_fence_before();
@@ -270,20 +553,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 }
 
-template <int EPI>
-lm_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
-                      cudaStream_t s) {
-    static bool configured = false;  // the attribute is per kernel, not per call
-    if (!configured) {
-        if (cudaFuncSetAttribute(gemm_fp8_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SMEM_BYTES) != cudaSuccess)
-            return LM_ERR_CUDA;
-        configured = true;
+}  // namespace one
+
+// cudaFuncSetAttribute once per kernel and device
+template <typename F>
+bool ensure_smem(F* kernel, int bytes, bool (&done)[64]) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (!done[dev]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+            cudaSuccess)
+            return false;
+        done[dev] = true;
     }
+    return true;
+}
+
+template <int EPI>
+lm_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                      const CUtensorMap& tx, const GemmArgs& a, cudaStream_t s) {
+    static bool done[64] = {};
+    if (!ensure_smem(pair::gemm_fp8_pair_kernel<EPI>, pair::SMEM_BYTES, done)) return LM_ERR_CUDA;
+    const int sms = sm_count();
+    if (sms < 2) return LM_ERR_CUDA;
+    const int clusters = a.num_tiles < sms / 2 ? a.num_tiles : sms / 2;
+    timing_mark(s, 'g');
+    pair::gemm_fp8_pair_kernel<EPI><<<2 * clusters, NUM_THREADS, pair::SMEM_BYTES, s>>>(ta, tb, td,
+                                                                                      tx, a);
+    return launch_status();
+}
+
+template <int EPI>
+lm_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
+                     cudaStream_t s) {
+    static bool done[64] = {};
+    if (!ensure_smem(one::gemm_fp8_kernel<EPI>, one::SMEM_BYTES, done)) return LM_ERR_CUDA;
     const int sms = sm_count();
     if (sms <= 0) return LM_ERR_CUDA;
     const int grid = a.num_tiles < sms ? a.num_tiles : sms;
-    gemm_fp8_kernel<EPI><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, a);
+    timing_mark(s, 'g');
+    one::gemm_fp8_kernel<EPI><<<grid, NUM_THREADS, one::SMEM_BYTES, s>>>(ta, tb, a);
     return launch_status();
 }
 
@@ -318,30 +627,53 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
             return LM_ERR_CUDA;
         return LM_OK;
     }
-    CUtensorMap ta, tb;
-    if (!encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, BM, BK) ||
-        !encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, BN, BK))
-        return LM_ERR_CUDA;
     unsigned int* err = device_error_word();
     if (!err) return LM_ERR_CUDA;
 
     GemmArgs a;
     a.M = (int)M;
     a.N = (int)N;
-    a.num_mb = (int)((M + BM - 1) / BM);
-    a.num_nb = (int)((N + BN - 1) / BN);
     a.num_kb = (int)((K + BK - 1) / BK);
-    a.num_tiles = a.num_mb * a.num_nb;
     a.inv_a = inv_scale_a;
     a.inv_b = inv_scale_b;
     a.aux = static_cast<const uint16_t*>(aux);
     a.D = static_cast<uint16_t*>(D);
     a.amax_out = amax_out;
     a.err = err;
-    a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, BM, BN);
+
+    CUtensorMap ta, tb;
+    if (M > 128) {
+        a.num_mb = (int)((M + pair::TILE_M - 1) / pair::TILE_M);
+        a.num_nb = (int)((N + pair::TILE_N - 1) / pair::TILE_N);
+        a.num_tiles = a.num_mb * a.num_nb;
+        a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, pair::TILE_M, pair::TILE_N);
+        CUtensorMap td, tx;
+        if (!encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, 128, BK) ||
+            !encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, 128, BK) ||
+            !encode_tmap_bf16_sw64(&td, D, (uint64_t)M, (uint64_t)N, 32, pair::EPI_COLS))
+            return LM_ERR_CUDA;
+        if (epi == LM_EPI_RELU2_BWD) {
+            if (!encode_tmap_bf16_sw64(&tx, aux, (uint64_t)M, (uint64_t)N, 32, pair::EPI_COLS))
+                return LM_ERR_CUDA;
+        } else {
+            tx = td;  // unused
+        }
+        switch (epi) {
+            case LM_EPI_NONE: return launch_pair<LM_EPI_NONE>(ta, tb, td, tx, a, s);
+            case LM_EPI_RELU2_FWD: return launch_pair<LM_EPI_RELU2_FWD>(ta, tb, td, tx, a, s);
+            default: return launch_pair<LM_EPI_RELU2_BWD>(ta, tb, td, tx, a, s);
+        }
+    }
+    a.num_mb = (int)((M + one::BM - 1) / one::BM);
+    a.num_nb = (int)((N + one::BN - 1) / one::BN);
+    a.num_tiles = a.num_mb * a.num_nb;
+    a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, one::BM, one::BN);
+    if (!encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, one::BM, BK) ||
+        !encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, one::BN, BK))
+        return LM_ERR_CUDA;
     switch (epi) {
-        case LM_EPI_NONE: return launch_gemm<LM_EPI_NONE>(ta, tb, a, s);
-        case LM_EPI_RELU2_FWD: return launch_gemm<LM_EPI_RELU2_FWD>(ta, tb, a, s);
-        default: return launch_gemm<LM_EPI_RELU2_BWD>(ta, tb, a, s);
+        case LM_EPI_NONE: return launch_one<LM_EPI_NONE>(ta, tb, a, s);
+        case LM_EPI_RELU2_FWD: return launch_one<LM_EPI_RELU2_FWD>(ta, tb, a, s);
+        default: return launch_one<LM_EPI_RELU2_BWD>(ta, tb, a, s);
     }
 }

@@ -23,6 +23,16 @@ int sm_count();
 bool encode_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint64_t pitch, uint32_t box_rows, uint32_t box_cols);
 
+// 2-D bf16 tensor map for a row-major [rows x cols] matrix, box
+// [box_rows x box_cols] with the 64-byte swizzle (box_cols * 2 must be 64);
+// used for the epilogue's TMA stores of D and loads of the saved H.
+bool encode_tmap_bf16_sw64(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                           uint32_t box_rows, uint32_t box_cols);
+
+// If the calling thread attached timing events, record the next one on `s`
+// (call right before a kernel launch); `kind` labels the launch.
+void timing_mark(cudaStream_t s, char kind);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline lm_status launch_status() {

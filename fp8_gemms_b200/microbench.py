@@ -1,0 +1,101 @@
+"""Time one C-ABI call on synthetic data (CUDA events, L2 flushed between
+iterations).  Also the small, self-contained command to run under ncu.
+
+    python -m fp8_gemms_b200.microbench gemm --M 16384 --N 12288 --K 3072 --epi relu2_fwd
+    python -m fp8_gemms_b200.microbench cast --rows 16384 --cols 3072 --fmt e4m3
+    python -m fp8_gemms_b200.microbench cast --rows 16384 --cols 12288 --relu2 --amax-in
+"""
+import argparse
+import json
+
+import torch
+
+from . import _lib
+from ._lib import E4M3, E5M2, EPI_NONE, EPI_RELU2_BWD, EPI_RELU2_FWD
+
+FMT = {"e4m3": E4M3, "e5m2": E5M2}
+EPI = {"none": EPI_NONE, "relu2_fwd": EPI_RELU2_FWD, "relu2_bwd": EPI_RELU2_BWD}
+TDT = {E4M3: torch.float8_e4m3fn, E5M2: torch.float8_e5m2}
+
+
+def random_codes(fmt, rows, cols, gen):
+    v = torch.randn(rows, cols, device="cuda", generator=gen)
+    return v.to(TDT[fmt]).view(torch.uint8)
+
+
+def time_it(fn, iters, warmup, flush):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ms = []
+    for i in range(iters):
+        flush.fill_(i & 0xFF)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        e.synchronize()
+        ms.append(s.elapsed_time(e))
+    return ms
+
+
+def main():
+    p = argparse.ArgumentParser()
+    p.add_argument("op", choices=["gemm", "cast"])
+    p.add_argument("--M", type=int, default=16384)
+    p.add_argument("--N", type=int, default=12288)
+    p.add_argument("--K", type=int, default=3072)
+    p.add_argument("--fa", default="e4m3")
+    p.add_argument("--fb", default="e4m3")
+    p.add_argument("--epi", default="none", choices=list(EPI))
+    p.add_argument("--rows", type=int, default=16384)
+    p.add_argument("--cols", type=int, default=3072)
+    p.add_argument("--fmt", default="e4m3")
+    p.add_argument("--relu2", action="store_true")
+    p.add_argument("--amax-in", action="store_true")
+    p.add_argument("--iters", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    a = p.parse_args()
+    gen = torch.Generator(device="cuda").manual_seed(0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    if a.op == "gemm":
+        fa, fb, epi = FMT[a.fa], FMT[a.fb], EPI[a.epi]
+        A = random_codes(fa, a.M, a.K, gen)
+        B = random_codes(fb, a.N, a.K, gen)
+        ia = torch.full((1,), 1e-2, device="cuda")
+        ib = torch.full((1,), 1e-2, device="cuda")
+        D = torch.empty(a.M, a.N, dtype=torch.bfloat16, device="cuda")
+        aux = torch.randn(a.M, a.N, device="cuda", generator=gen).to(torch.bfloat16) \
+            if epi == EPI_RELU2_BWD else None
+        am = torch.zeros(1, device="cuda")
+        fn = lambda: _lib.lm_fp8_gemm(A, fa, B, fb, ia, ib, D, epi=epi, aux=aux, amax_out=am)
+        ms = time_it(fn, a.iters, a.warmup, flush)
+        flops = 2 * a.M * a.N * a.K
+        byts = a.M * a.K + a.N * a.K + 2 * a.M * a.N * (2 if epi == EPI_RELU2_BWD else 1)
+        avg = sum(ms) / len(ms)
+        out = dict(op="gemm", M=a.M, N=a.N, K=a.K, fa=a.fa, fb=a.fb, epi=a.epi,
+                   avg_ms=round(avg, 4), min_ms=round(min(ms), 4),
+                   tflops=round(flops / avg / 1e9, 1), algorithmic_bytes=byts)
+    else:
+        fmt = FMT[a.fmt]
+        x = (torch.randn(a.rows, a.cols, device="cuda", generator=gen)).to(torch.bfloat16)
+        q = torch.empty(a.rows, a.cols, dtype=torch.uint8, device="cuda")
+        qT = torch.empty(a.cols, a.rows, dtype=torch.uint8, device="cuda")
+        sc = torch.zeros(4, device="cuda")
+        amax_in = torch.full((1,), 4.0, device="cuda") if a.amax_in else None
+        fn = lambda: _lib.lm_fp8_amax_scale_cast(x, fmt, sc[0:1], sc[1:2], sc[2:3], q, qT,
+                                                 relu2_input=a.relu2, amax_in=amax_in)
+        ms = time_it(fn, a.iters, a.warmup, flush)
+        n = a.rows * a.cols
+        byts = n * (4 if a.amax_in else 6)
+        avg = sum(ms) / len(ms)
+        out = dict(op="cast", rows=a.rows, cols=a.cols, fmt=a.fmt, relu2=a.relu2,
+                   amax_in=a.amax_in, avg_ms=round(avg, 4), min_ms=round(min(ms), 4),
+                   gbs=round(byts / avg / 1e6, 1), algorithmic_bytes=byts)
+    st, where = _lib.lm_get_error()
+    out["device_error"] = st
+    print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()

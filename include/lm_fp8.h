@@ -185,6 +185,22 @@ LM_API lm_status lm_relu2_mlp_bwd(const void* dY, const lm_mlp_saved* saved, int
  * none). */
 LM_API lm_status lm_get_error(lm_stream_t stream, uint32_t* where_out);
 
+/*
+ * Kernel-boundary timing, for benchmarks (no counterpart on the pages).
+ * lm_timing_attach(events, capacity) makes every kernel launch that the
+ * calling host thread enqueues through this library first record
+ * events[i] (each a cudaEvent_t created by the caller) on the launch's
+ * stream, i = 0, 1, ... up to capacity; the interval from events[i] to the
+ * next recorded event therefore brackets launch i.  lm_timing_detach()
+ * stops recording and returns the number of events recorded.
+ * lm_timing_kinds() copies one character per recorded launch ('a' amax
+ * reduction, 'c' cast, 's' scales only, 'g' GEMM) into out[0..cap) and
+ * returns how many it wrote.  State is per host thread.
+ */
+LM_API void lm_timing_attach(void* const* events, int capacity);
+LM_API int lm_timing_detach(void);
+LM_API int lm_timing_kinds(char* out, int cap);
+
 /* Static, human-readable name of a status. */
 LM_API const char* lm_status_string(lm_status status);
 
