@@ -22,7 +22,8 @@ STATUS = {0: "LM_OK", 1: "LM_ERR_INVALID_ARG", 2: "LM_ERR_ALIGNMENT",
 EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
             "lm_relu2_mlp_saved_carve", "lm_relu2_mlp_workspace_size", "lm_relu2_mlp_fwd",
             "lm_relu2_mlp_bwd", "lm_get_error", "lm_status_string", "lm_version",
-            "lm_timing_attach", "lm_timing_detach", "lm_timing_kinds"]
+            "lm_timing_attach", "lm_timing_detach", "lm_timing_kinds",
+            "lm_relu2_mlp_bwd_noalloc", "lm_relu2_mlp_bwd_noalloc_max_bytes"]
 
 
 class LmError(RuntimeError):
@@ -70,6 +71,10 @@ def _load():
     L.lm_timing_detach.restype = i32
     L.lm_timing_kinds.argtypes = [ctypes.c_char_p, i32]
     L.lm_timing_kinds.restype = i32
+    L.lm_relu2_mlp_bwd_noalloc.argtypes = [P, ctypes.POINTER(MlpSaved), i64, i64, i64, P, P, P, P]
+    L.lm_relu2_mlp_bwd_noalloc.restype = st
+    L.lm_relu2_mlp_bwd_noalloc_max_bytes.argtypes = []
+    L.lm_relu2_mlp_bwd_noalloc_max_bytes.restype = ctypes.c_size_t
     return L
 
 
@@ -148,6 +153,16 @@ def lm_relu2_mlp_bwd(dY, saved, dX, dW_up, dW_down, workspace, stream=None):
                                 _p(dW_down), _p(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(stream)),
            "lm_relu2_mlp_bwd")
+
+
+def lm_relu2_mlp_bwd_noalloc(dY, saved, dX, dW_up, dW_down, stream=None):
+    """The relu^2 MLP backward with the library's own fixed scratch (no workspace
+    argument); see include/lm_fp8.h for its size limit and sharing rules."""
+    M, d = dY.shape
+    f = dW_up.shape[0]
+    _check(lib.lm_relu2_mlp_bwd_noalloc(_p(dY), ctypes.byref(saved), M, d, f, _p(dX), _p(dW_up),
+                                        _p(dW_down), _stream(stream)),
+           "lm_relu2_mlp_bwd_noalloc")
 
 
 def lm_get_error(stream=None):

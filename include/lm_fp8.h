@@ -178,6 +178,33 @@ LM_API lm_status lm_relu2_mlp_bwd(const void* dY, const lm_mlp_saved* saved, int
                            int64_t f, void* dX, void* dW_up, void* dW_down, void* workspace,
                            size_t ws_bytes, lm_stream_t stream);
 
+/*
+ * relu^2 MLP backward that allocates nothing (no counterpart on the pages:
+ * the method itself says nothing about memory ownership).  For callers that
+ * cannot hand the library a workspace -- code running during CUDA graph
+ * capture, where cudaMalloc is not allowed; plugins whose host framework owns
+ * all device memory and forbids allocation in its execute callback; loops that
+ * cannot absorb the device-wide synchronisation of cudaMalloc/cudaFree.
+ * Computes exactly what lm_relu2_mlp_bwd computes, using as its workspace a
+ * 64 MiB device array owned by the library (lm_relu2_mlp_bwd_noalloc_max_bytes).
+ *  - Shapes whose lm_relu2_mlp_workspace_size exceeds that size return
+ *    LM_ERR_UNSUPPORTED_SHAPE with nothing enqueued.
+ *  - The first call on a device looks up the array's device address with that
+ *    device current; make that first call before any stream capture begins.
+ *    Every GPU that loads the array keeps it until the process exits.
+ *  - All calls on a device share the array, which keeps the previous call's
+ *    contents (the backward re-zeroes what must start at zero).  Calls whose
+ *    work overlaps on the GPU (e.g. on two unordered streams) race; calls on
+ *    one stream are safe.
+ * Other arguments, layouts and errors as lm_relu2_mlp_bwd.
+ */
+LM_API lm_status lm_relu2_mlp_bwd_noalloc(const void* dY, const lm_mlp_saved* saved, int64_t M,
+                                          int64_t d, int64_t f, void* dX, void* dW_up,
+                                          void* dW_down, lm_stream_t stream);
+
+/* Size in bytes of the array lm_relu2_mlp_bwd_noalloc uses as its workspace. */
+LM_API size_t lm_relu2_mlp_bwd_noalloc_max_bytes(void);
+
 /* Synchronises `stream`, then returns and clears the current device's error
  * word: LM_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
  * LM_ERR_CUDA if the synchronisation itself failed, else LM_OK.  If
