@@ -13,6 +13,7 @@
 #include <cuda_bf16.h>
 
 #include "lm_internal.h"
+#include "lm_ptx.cuh"
 
 namespace lm {
 namespace {
@@ -218,16 +219,179 @@ __global__ void __launch_bounds__(kThreads) cast_kernel(
     }
 }
 
+
+// Pass 2, TMA-fed: a persistent kernel, two CTAs per SM.  Warp 8 streams
+// 128 x 128 bf16 tiles (32 KB) into a 3-stage shared ring with TMA; warps
+// 0-7 convert each tile (16-byte shared loads, 8-byte stores of row-major
+// codes to q), stage the codes in shared memory and write the transposed
+// codes to qT (4 x 4 byte permutes, one 16-byte store per column and warp).
+// Tiles are taken in reverse memory order so the first ones re-read what the
+// amax pass left in L2.  Waits are bounded; after a timeout a thread stops
+// waiting but keeps the loop's barrier sequence, so no barrier can hang.
+namespace tmac {
+constexpr int TR = 128, TC = 128;
+constexpr int STAGES = 3;
+constexpr int IN_BYTES = TR * TC * 2;
+constexpr int CODE_BYTES = TR * TC;
+constexpr int CONSUMERS = 256;
+constexpr int THREADS = CONSUMERS + 32;
+constexpr int SMEM = STAGES * IN_BYTES + CODE_BYTES + 128 + 128;
+enum : unsigned { W_CAST_EMPTY = 0x201, W_CAST_FULL = 0x202, W_CAST_LOADS = 0x203 };
+}  // namespace tmac
+
+__device__ __forceinline__ void consumers_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(tmac::CONSUMERS) : "memory");
+}
+
 template <int FMT, bool RELU2>
-void launch_cast(const uint16_t* x, int rows, int cols, int64_t ld, const float* amax_src,
-                 float* amax_out, float* scale_out, float* inv_out, uint8_t* q, uint8_t* qT,
-                 cudaStream_t s) {
+__global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
+    const __grid_constant__ CUtensorMap tmX, int rows, int cols, const float* amax_src,
+    float* amax_out, float* scale_out, float* inv_out, uint8_t* __restrict__ q,
+    uint8_t* __restrict__ qT, int tiles_c, int num_tiles, unsigned int* err) {
+    using namespace tmac;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + ((128u - (raw & 127u)) & 127u);
+    uint8_t* sIn = smem;
+    uint32_t* sCode = reinterpret_cast<uint32_t*>(smem + STAGES * IN_BYTES);  // [TR][TC/4]
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * IN_BYTES + CODE_BYTES);
+    uint64_t* empty = full + STAGES;
+
+    const float fmax = FMT == LM_FP8_E4M3 ? 448.0f : 57344.0f;
+    float scale;
+    write_scales(*amax_src, fmax, amax_out, scale_out, inv_out, &scale);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], CONSUMERS / 32);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == CONSUMERS / 32) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0, issued = 0;
+            for (int i = blockIdx.x; i < num_tiles; i += gridDim.x) {
+                const int t = num_tiles - 1 - i;
+                if (!mbar_wait(&empty[s], ph ^ 1u, err, W_CAST_EMPTY)) break;
+                mbar_arrive_expect_tx(&full[s], IN_BYTES);
+                tma_load_2d(smem_addr(sIn + s * IN_BYTES), &tmX, &full[s], (t % tiles_c) * TC,
+                            (t / tiles_c) * TR);
+                ++issued;
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            for (int st = 0; st < STAGES; ++st) {  // every issued load has landed
+                const uint32_t n = issued / STAGES + ((uint32_t)st < issued % STAGES ? 1u : 0u);
+                if (n) mbar_wait(&full[st], (n - 1) & 1u, err, W_CAST_LOADS);
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------- consumers
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; i < num_tiles; i += gridDim.x) {
+        const int t = num_tiles - 1 - i;
+        const int r0 = (t / tiles_c) * TR, c0 = (t % tiles_c) * TC;
+        if (ok) ok = mbar_wait(&full[s], ph, err, W_CAST_FULL);
+        const uint8_t* in = sIn + s * IN_BYTES;
+#pragma unroll
+        for (int it = 0; it < (TR * TC / 8) / CONSUMERS; ++it) {
+            const int idx = it * CONSUMERS + tid;
+            const int rr = idx >> 4, ch = idx & 15;
+            const uint4 v = *reinterpret_cast<const uint4*>(in + rr * (TC * 2) + ch * 16);
+            const uint2 codes = convert8<FMT, RELU2>(v, scale);
+            const int r = r0 + rr, c = c0 + ch * 8;
+            if (q && r < rows && c < cols)
+                *reinterpret_cast<uint2*>(q + (int64_t)r * cols + c) = codes;
+            *reinterpret_cast<uint2*>(&sCode[rr * (TC / 4) + ch * 2]) = codes;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
+        if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+        }
+        if (!qT) continue;
+        consumers_sync();  // the codes tile is complete
+        // warp w: tile rows [16w, 16w+16); lane l: tile columns [4l, 4l+4)
+        uint32_t v[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = sCode[(warp * 16 + k) * (TC / 4) + lane];
+        uint32_t o[4][4];  // o[j][k]: column 4l+j, rows 16w+4k .. +3
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t t0 = __byte_perm(v[4 * k], v[4 * k + 1], 0x5140);
+            const uint32_t t1 = __byte_perm(v[4 * k + 2], v[4 * k + 3], 0x5140);
+            const uint32_t t2 = __byte_perm(v[4 * k], v[4 * k + 1], 0x7362);
+            const uint32_t t3 = __byte_perm(v[4 * k + 2], v[4 * k + 3], 0x7362);
+            o[0][k] = __byte_perm(t0, t1, 0x5410);
+            o[1][k] = __byte_perm(t0, t1, 0x7632);
+            o[2][k] = __byte_perm(t2, t3, 0x5410);
+            o[3][k] = __byte_perm(t2, t3, 0x7632);
+        }
+        const int rb = r0 + warp * 16;
+        if (rb < rows) {  // rows % 16 == 0: a 16-row group is all in or all out
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int c = c0 + 4 * lane + j;
+                if (c < cols)
+                    *reinterpret_cast<uint4*>(qT + (int64_t)c * rows + rb) =
+                        make_uint4(o[j][0], o[j][1], o[j][2], o[j][3]);
+            }
+        }
+        consumers_sync();  // before the next tile overwrites the codes
+    }
+}
+
+template <int FMT, bool RELU2>
+lm_status launch_cast(const uint16_t* x, int rows, int cols, int64_t ld, const float* amax_src,
+                      float* amax_out, float* scale_out, float* inv_out, uint8_t* q, uint8_t* qT,
+                      cudaStream_t s) {
+    if (rows % 16 == 0) {
+        // TMA-fed persistent kernel (its transposed stores need 16-row groups)
+        static bool configured[64] = {};
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LM_ERR_CUDA;
+        if (!configured[dev]) {
+            if (cudaFuncSetAttribute(cast_tma_kernel<FMT, RELU2>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     tmac::SMEM) != cudaSuccess)
+                return LM_ERR_CUDA;
+            configured[dev] = true;
+        }
+        CUtensorMap tm;
+        if (!encode_tmap_bf16_plain(&tm, x, (uint64_t)rows, (uint64_t)cols, (uint64_t)ld * 2,
+                                    tmac::TR, tmac::TC))
+            return LM_ERR_CUDA;
+        unsigned int* err = device_error_word();
+        if (!err) return LM_ERR_CUDA;
+        const int tiles_c = (cols + tmac::TC - 1) / tmac::TC;
+        const int n = ((rows + tmac::TR - 1) / tmac::TR) * tiles_c;
+        int grid = 2 * sm_count();
+        if (grid <= 0) return LM_ERR_CUDA;
+        if (grid > n) grid = n;
+        timing_mark(s, 'c');
+        cast_tma_kernel<FMT, RELU2><<<grid, tmac::THREADS, tmac::SMEM, s>>>(
+            tm, rows, cols, amax_src, amax_out, scale_out, inv_out, q, qT, tiles_c, n, err);
+        return launch_status();
+    }
     const int tiles_r = (rows + kCastRows - 1) / kCastRows;
     const int tiles_c = (cols + kCastCols - 1) / kCastCols;
     const int n = tiles_r * tiles_c;
     timing_mark(s, 'c');
     cast_kernel<FMT, RELU2><<<n, kThreads, 0, s>>>(x, rows, cols, ld, amax_src, amax_out,
                                                   scale_out, inv_out, q, qT, tiles_c, n);
+    return launch_status();
 }
 
 }  // namespace
@@ -274,20 +438,14 @@ extern "C" lm_status lm_fp8_amax_scale_cast(const void* x, int64_t rows, int64_t
         return launch_status();
     }
     const int r = (int)rows, c = (int)cols;
-    if (fmt == LM_FP8_E4M3) {
-        if (relu2_input)
-            launch_cast<LM_FP8_E4M3, true>(xb, r, c, ld, amax_src, amax_out, scale_out,
-                                           inv_scale_out, q, qT, s);
-        else
-            launch_cast<LM_FP8_E4M3, false>(xb, r, c, ld, amax_src, amax_out, scale_out,
-                                            inv_scale_out, q, qT, s);
-    } else {
-        if (relu2_input)
-            launch_cast<LM_FP8_E5M2, true>(xb, r, c, ld, amax_src, amax_out, scale_out,
-                                           inv_scale_out, q, qT, s);
-        else
-            launch_cast<LM_FP8_E5M2, false>(xb, r, c, ld, amax_src, amax_out, scale_out,
-                                            inv_scale_out, q, qT, s);
-    }
-    return launch_status();
+    if (launch_status() != LM_OK) return LM_ERR_CUDA;  // the amax pass launched cleanly
+    if (fmt == LM_FP8_E4M3)
+        return relu2_input ? launch_cast<LM_FP8_E4M3, true>(xb, r, c, ld, amax_src, amax_out,
+                                                            scale_out, inv_scale_out, q, qT, s)
+                           : launch_cast<LM_FP8_E4M3, false>(xb, r, c, ld, amax_src, amax_out,
+                                                             scale_out, inv_scale_out, q, qT, s);
+    return relu2_input ? launch_cast<LM_FP8_E5M2, true>(xb, r, c, ld, amax_src, amax_out,
+                                                        scale_out, inv_scale_out, q, qT, s)
+                       : launch_cast<LM_FP8_E5M2, false>(xb, r, c, ld, amax_src, amax_out,
+                                                         scale_out, inv_scale_out, q, qT, s);
 }

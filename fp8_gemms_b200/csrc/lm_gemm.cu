@@ -43,7 +43,7 @@ enum : unsigned {
 };
 
 struct GemmArgs {
-    int M, N, num_mb, num_nb, num_kb, num_tiles;
+    int M, N, num_mb, num_nb, num_kb, num_tiles, group_m;
     const float* inv_a;
     const float* inv_b;
     const uint16_t* aux;
@@ -53,14 +53,14 @@ struct GemmArgs {
     uint32_t idesc;
 };
 
-// Tile visiting order: groups of GROUP_M row-blocks, column-blocks within a
+// Tile visiting order: groups of group_m row-blocks, column-blocks within a
 // group, so the tiles in flight at once share A and B panels in L2.
-template <int GROUP_M>
-__device__ __forceinline__ void tile_coords(int t, int num_mb, int num_nb, int& mb, int& nb) {
-    const int per_group = GROUP_M * num_nb;
+__device__ __forceinline__ void tile_coords(int t, int group_m, int num_mb, int num_nb, int& mb,
+                                            int& nb) {
+    const int per_group = group_m * num_nb;
     const int g = t / per_group;
-    const int first = g * GROUP_M;
-    const int gsize = min(GROUP_M, num_mb - first);
+    const int first = g * group_m;
+    const int gsize = min(group_m, num_mb - first);
     const int local = t - g * per_group;
     mb = first + local % gsize;
     nb = local / gsize;
@@ -120,7 +120,6 @@ constexpr int BOX_BYTES = 32 * EPI_COLS * 2;   // one warp's 32 x 32 bf16 box
 constexpr int STORE_BYTES = NUM_EPI_WARPS * 2 * BOX_BYTES;
 constexpr int AUX_BYTES = NUM_EPI_WARPS * 2 * BOX_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * TILE_N;
-constexpr int GROUP_M = 8;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + AUX_BYTES + 1024 + 512;
 
 // Offset of 16-byte chunk j of row r in a 32-row x 64-byte box written or
@@ -194,7 +193,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             bool ok = true;
             for (int t = cluster; t < args.num_tiles && ok; t += nclusters) {
                 int mb, nb;
-                tile_coords<GROUP_M>(t, args.num_mb, args.num_nb, mb, nb);
+                tile_coords(t, args.group_m, args.num_mb, args.num_nb, mb, nb);
                 const int arow = mb * TILE_M + (int)rank * 128;
                 const int brow = nb * TILE_N + (int)rank * 128;
                 for (int kb = 0; kb < args.num_kb; ++kb) {
@@ -268,6 +267,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         uint8_t* ax_buf = sAux + wi * 2 * BOX_BYTES;
         uint64_t* ax_bar = auxbar + wi * 2;
         const uint32_t tempty_leader = map_to_rank(smem_addr(tempty), 0);
+        const uint64_t stream_policy = l2_policy_evict_first();  // D and H are touched once
         const float s = __fmul_rn(*args.inv_a, *args.inv_b);
         uint32_t amax = 0;
         int acc = 0;
@@ -277,7 +277,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         bool ok = true;
         for (int t = cluster; t < args.num_tiles && ok; t += nclusters) {
             int mb, nb;
-            tile_coords<GROUP_M>(t, args.num_mb, args.num_nb, mb, nb);
+            tile_coords(t, args.group_m, args.num_mb, args.num_nb, mb, nb);
             const int grow = mb * TILE_M + (int)rank * 128 + quarter * 32;  // row of lane 0
             const int gcol = nb * TILE_N;
             const int left = args.N - gcol;
@@ -285,7 +285,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if (EPI == LM_EPI_RELU2_BWD && lane == 0) {
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(&ax_bar[0], BOX_BYTES);
-                tma_load_2d(smem_addr(ax_buf), &tmAux, &ax_bar[0], gcol, grow);
+                tma_load_2d_hint(smem_addr(ax_buf), &tmAux, &ax_bar[0], gcol, grow, stream_policy);
             }
             if (!mbar_wait(&tfull[acc], acc_phase, args.err, W_TFULL)) break;
             tc_fence_after();
@@ -301,8 +301,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     if (lane == 0 && c + 1 < n_chunks) {
                         fence_proxy_async_smem();
                         mbar_arrive_expect_tx(&ax_bar[b ^ 1], BOX_BYTES);
-                        tma_load_2d(smem_addr(ax_buf + (b ^ 1) * BOX_BYTES), &tmAux, &ax_bar[b ^ 1],
-                                    gcol + (c + 1) * EPI_COLS, grow);
+                        tma_load_2d_hint(smem_addr(ax_buf + (b ^ 1) * BOX_BYTES), &tmAux,
+                                         &ax_bar[b ^ 1], gcol + (c + 1) * EPI_COLS, grow,
+                                         stream_policy);
                     }
                     if (!mbar_wait(&ax_bar[b], (ax_phase >> b) & 1u, args.err, W_AUX)) {
                         ok = false;
@@ -341,7 +342,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(&tmD, smem_addr(dst), gcol + c * EPI_COLS, grow);
+                    tma_store_2d_hint(&tmD, smem_addr(dst), gcol + c * EPI_COLS, grow,
+                                      stream_policy);
                     bulk_commit_group();
                 }
                 ++n_stores;
@@ -379,7 +381,6 @@ constexpr int B_BYTES = BN * BK;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_EPI_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr int GROUP_M = 16;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 
 template <int EPI>
@@ -432,7 +433,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             bool ok = true;
             for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
                 int mb, nb;
-                tile_coords<GROUP_M>(t, args.num_mb, args.num_nb, mb, nb);
+                tile_coords(t, args.group_m, args.num_mb, args.num_nb, mb, nb);
                 for (int kb = 0; kb < args.num_kb; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, args.err, W_EMPTY)) {
                         ok = false;
@@ -501,7 +502,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
             int mb, nb;
-            tile_coords<GROUP_M>(t, args.num_mb, args.num_nb, mb, nb);
+            tile_coords(t, args.group_m, args.num_mb, args.num_nb, mb, nb);
             if (!mbar_wait(&tfull[acc], acc_phase, args.err, W_TFULL)) break;
             tc_fence_after();
             const int row = mb * BM + quarter * 32 + lane;
@@ -646,6 +647,9 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
         a.num_mb = (int)((M + pair::TILE_M - 1) / pair::TILE_M);
         a.num_nb = (int)((N + pair::TILE_N - 1) / pair::TILE_N);
         a.num_tiles = a.num_mb * a.num_nb;
+        // up to 16 row-blocks: one group spans all of M, so every B panel is
+        // fetched once; otherwise groups of 8
+        a.group_m = a.num_mb <= 16 ? a.num_mb : 8;
         a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, pair::TILE_M, pair::TILE_N);
         CUtensorMap td, tx;
         if (!encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, 128, BK) ||
@@ -667,6 +671,7 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
     a.num_mb = (int)((M + one::BM - 1) / one::BM);
     a.num_nb = (int)((N + one::BN - 1) / one::BN);
     a.num_tiles = a.num_mb * a.num_nb;
+    a.group_m = 16;
     a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, one::BM, one::BN);
     if (!encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, one::BM, BK) ||
         !encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, one::BN, BK))

@@ -29,6 +29,11 @@ bool encode_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 bool encode_tmap_bf16_sw64(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                            uint32_t box_rows, uint32_t box_cols);
 
+// 2-D bf16 tensor map, no swizzle, row pitch `pitch` bytes (a multiple of
+// 16), box [box_rows x box_cols]; out-of-bounds elements read as zero.
+bool encode_tmap_bf16_plain(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                            uint64_t pitch, uint32_t box_rows, uint32_t box_cols);
+
 // If the calling thread attached timing events, record the next one on `s`
 // (call right before a kernel launch); `kind` labels the launch.
 void timing_mark(cudaStream_t s, char kind);

@@ -78,7 +78,8 @@ SHAPES = [
     (200, 328, 208),    # ragged M, N (N % 256 != 0) and K (K % 128 != 0)
     (16, 8, 16),        # smaller than one tile in every dimension
     (1, 264, 48),       # a single row
-    (2304, 256, 256),   # more M-blocks than one raster group (16)
+    (2304, 256, 256),   # 9 row-blocks of 256: one raster group spans M
+    (4608, 512, 128),   # 18 row-blocks: groups of 8 plus a ragged last group
     (300, 1032, 1040),  # ragged everywhere, many tiles
 ]
 
