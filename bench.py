@@ -133,6 +133,23 @@ def make_inputs(torch, device):
     return t, {k: v.to(device) for k, v in t.items()}
 
 
+def max_over_ranks(x, world, device):
+    """Max of a per-rank float over all ranks (the job's time is its slowest
+    rank's).  Every rank must call it, in the same order."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world, steps, flops_per_step, total_ms):
+    """Whole-job throughput: the units all ranks processed over the job's time."""
+    return world * steps * flops_per_step / (total_ms * 1e-3) / 1e12
+
+
 # algorithmic bytes of the cast launches of one step, in launch order:
 # full cast (amax pass + cast pass) = 2 B amax read + 2 B read + 1 B q + 1 B qT
 # per element; fused-amax cast = 2 B read + 1 B q + 1 B qT per element.
@@ -202,11 +219,7 @@ def run_gpu(args):
         barrier()
     clocks = clk.summary()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, device)
     st, where = lib.lm_get_error()
     if st != 0:
         raise RuntimeError(f"device error {st} at wait {where:#x}")
@@ -243,15 +256,11 @@ def run_gpu(args):
             v.copy_(dev[n], non_blocking=True)
     e_e.record()
     barrier()
-    e2e_ms = e_s.elapsed_time(e_e)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), world, device)
 
     peaks = read_peaks()
-    value = world * K * STEP_FLOPS / (total_ms * 1e-3) / 1e12
-    e2e_value = world * Ke * STEP_FLOPS / (e2e_ms * 1e-3) / 1e12
+    value = job_tflops(world, K, STEP_FLOPS, total_ms)
+    e2e_value = job_tflops(world, Ke, STEP_FLOPS, e2e_ms)
     fp8_peak = peaks["bf16_sus"] * NOMINAL_FP8_OVER_BF16
     achieved = GEMM_FLOPS / (gemm_avg_ms * 1e-3) / 1e12
     traffic = None

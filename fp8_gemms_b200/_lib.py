@@ -23,7 +23,8 @@ EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
             "lm_relu2_mlp_saved_carve", "lm_relu2_mlp_workspace_size", "lm_relu2_mlp_fwd",
             "lm_relu2_mlp_bwd", "lm_get_error", "lm_status_string", "lm_version",
             "lm_timing_attach", "lm_timing_detach", "lm_timing_kinds",
-            "lm_relu2_mlp_bwd_noalloc", "lm_relu2_mlp_bwd_noalloc_max_bytes"]
+            "lm_relu2_mlp_bwd_noalloc", "lm_relu2_mlp_bwd_noalloc_max_bytes",
+            "lm_selftest_bounded_wait"]
 
 
 class LmError(RuntimeError):
@@ -75,6 +76,8 @@ def _load():
     L.lm_relu2_mlp_bwd_noalloc.restype = st
     L.lm_relu2_mlp_bwd_noalloc_max_bytes.argtypes = []
     L.lm_relu2_mlp_bwd_noalloc_max_bytes.restype = ctypes.c_size_t
+    L.lm_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
+    L.lm_selftest_bounded_wait.restype = st
     return L
 
 
@@ -169,6 +172,10 @@ def lm_get_error(stream=None):
     where = ctypes.c_uint32(0)
     st = lib.lm_get_error(_stream(stream), ctypes.byref(where))
     return st, where.value
+
+
+def lm_selftest_bounded_wait(limit_ms, stream=None):
+    _check(lib.lm_selftest_bounded_wait(limit_ms, _stream(stream)), "lm_selftest_bounded_wait")
 
 
 def lm_status_string(status):

@@ -5,6 +5,7 @@
 #include <mutex>
 
 #include "lm_internal.h"
+#include "lm_ptx.cuh"
 
 namespace lm {
 
@@ -122,9 +123,31 @@ bool encode_tmap_bf16_plain(CUtensorMap* map, const void* base, uint64_t rows, u
     return r == CUDA_SUCCESS;
 }
 
+namespace {
+// A wait that nothing satisfies: exercises the bounded-wait expiry path.
+__global__ void selftest_wait_kernel(unsigned int* err, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_limit(&bar, 0, err, 0x301u, limit_ns);
+}
+}  // namespace
+
 }  // namespace lm
 
 extern "C" {
+
+lm_status lm_selftest_bounded_wait(uint32_t limit_ms, lm_stream_t stream) {
+    if (limit_ms < 1 || limit_ms > 5000) return LM_ERR_INVALID_ARG;
+    unsigned int* err = lm::device_error_word();
+    if (!err) return LM_ERR_CUDA;
+    lm::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        err, (uint64_t)limit_ms * 1000000ull);
+    return lm::launch_status();
+}
 
 lm_status lm_get_error(lm_stream_t stream, uint32_t* where_out) {
     if (where_out) *where_out = 0;

@@ -44,6 +44,7 @@ enum : unsigned {
 
 struct GemmArgs {
     int M, N, num_mb, num_nb, num_kb, num_tiles, group_m;
+    int stream_a;  // 1: A is the streamed operand (evict-first loads), 0: B is
     const float* inv_a;
     const float* inv_b;
     const uint16_t* aux;
@@ -103,6 +104,33 @@ __device__ __forceinline__ void reduce_amax(uint32_t amax, float* amax_out, int 
         }
         atomicMax(reinterpret_cast<unsigned int*>(amax_out), bits);
     }
+}
+
+// Two accumulator values -> two bf16 output values packed in one word (lo =
+// even column), and the running packed amax (bf16 bits, two halves) of what
+// the next cast consumes.  bf16x2 arithmetic: for the relu^2 backward,
+// dH = g * (2 relu(H)) where 2 relu(H) is exact and the product of two bf16
+// values is exact before its single rounding -- the same value as
+// bf16(g * 2 * relu(H)).  relu of a NaN H gives 0, as max(h, 0) does.
+template <int EPI>
+__device__ __forceinline__ uint32_t epi_pair(uint32_t acc0, uint32_t acc1, float s,
+                                             uint32_t h_pair, uint32_t& amax2) {
+    const __nv_bfloat162 g2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(acc0), s),
+                                                    __fmul_rn(__uint_as_float(acc1), s));
+    uint32_t w = *reinterpret_cast<const uint32_t*>(&g2);
+    if (EPI == LM_EPI_RELU2_BWD) {
+        const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&h_pair);
+        __nv_bfloat162 r2 = __hmax2(h2, __float2bfloat162_rn(0.0f));
+        r2 = __hadd2(r2, r2);
+        const __nv_bfloat162 d2 = __hmul2(g2, r2);
+        w = *reinterpret_cast<const uint32_t*>(&d2);
+        amax2 = __vmaxu2(amax2, w & 0x7FFF7FFFu);
+    } else if (EPI == LM_EPI_RELU2_FWD) {
+        amax2 = __vmaxu2(amax2, __vmaxs2(w, 0u));  // negative halves -> 0: max of relu(H)
+    } else {
+        amax2 = __vmaxu2(amax2, w & 0x7FFF7FFFu);
+    }
+    return w;
 }
 
 // =====================================================================
@@ -188,6 +216,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
             // ---------------------------------------- TMA producer (both CTAs)
             const uint32_t full_leader = map_to_rank(smem_addr(full), 0);
+            // the operand that every tile wave re-reads stays at normal L2
+            // priority; the one streamed through once is evicted first
+            const uint64_t pol_first = l2_policy_evict_first();
+            const uint64_t pol_a = args.stream_a ? pol_first : 0ull;
+            const uint64_t pol_b = args.stream_a ? 0ull : pol_first;
             int stage = 0;
             uint32_t phase = 0, issued = 0;
             bool ok = true;
@@ -203,8 +236,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     }
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
                     const uint32_t bar = full_leader + (uint32_t)(stage * 8);
-                    tma_load_2d_pair(smem_addr(sA + stage * A_BYTES), &tmA, bar, kb * BK, arow);
-                    tma_load_2d_pair(smem_addr(sB + stage * B_BYTES), &tmB, bar, kb * BK, brow);
+                    if (args.stream_a) {
+                        tma_load_2d_pair_hint(smem_addr(sA + stage * A_BYTES), &tmA, bar, kb * BK,
+                                              arow, pol_a);
+                        tma_load_2d_pair(smem_addr(sB + stage * B_BYTES), &tmB, bar, kb * BK, brow);
+                    } else {
+                        tma_load_2d_pair(smem_addr(sA + stage * A_BYTES), &tmA, bar, kb * BK, arow);
+                        tma_load_2d_pair_hint(smem_addr(sB + stage * B_BYTES), &tmB, bar, kb * BK,
+                                              brow, pol_b);
+                    }
                     ++issued;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -269,7 +309,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const uint32_t tempty_leader = map_to_rank(smem_addr(tempty), 0);
         const uint64_t stream_policy = l2_policy_evict_first();  // D and H are touched once
         const float s = __fmul_rn(*args.inv_a, *args.inv_b);
-        uint32_t amax = 0;
+        uint32_t amax2 = 0;  // two bf16-bit halves of the running max
         int acc = 0;
         uint32_t acc_phase = 0;
         uint32_t ax_phase = 0;  // bit b: parity of the next wait on aux buffer b
@@ -283,6 +323,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int left = args.N - gcol;
             const int n_chunks = left >= TILE_N ? TILE_N / EPI_COLS : (left + EPI_COLS - 1) / EPI_COLS;
             if (EPI == LM_EPI_RELU2_BWD && lane == 0) {
+                // this warp's 32 rows of H for the tile after this one go to L2 now
+                const int tn = t + nclusters;
+                if (tn < args.num_tiles) {
+                    int mb2, nb2;
+                    tile_coords(tn, args.group_m, args.num_mb, args.num_nb, mb2, nb2);
+                    const int grow2 = mb2 * TILE_M + (int)rank * 128 + quarter * 32;
+                    for (int c = 0; c < TILE_N / EPI_COLS; ++c)
+                        tma_prefetch_l2_2d(&tmAux, nb2 * TILE_N + c * EPI_COLS, grow2);
+                }
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(&ax_bar[0], BOX_BYTES);
                 tma_load_2d_hint(smem_addr(ax_buf), &tmAux, &ax_bar[0], gcol, grow, stream_policy);
@@ -295,7 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tbase + (uint32_t)(c * EPI_COLS), r);
                 tmem_ld_wait();
-                uint32_t hb[32];
+                uint32_t hw[16];  // saved H, two bf16 per word, columns 2i and 2i+1
                 if (EPI == LM_EPI_RELU2_BWD) {
                     const int b = c & 1;
                     if (lane == 0 && c + 1 < n_chunks) {
@@ -314,21 +363,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint4 v = *reinterpret_cast<const uint4*>(src + sw64(lane, j));
-                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            hb[8 * j + 2 * i] = w[i] & 0xFFFFu;
-                            hb[8 * j + 2 * i + 1] = w[i] >> 16;
-                        }
+                        hw[4 * j] = v.x;
+                        hw[4 * j + 1] = v.y;
+                        hw[4 * j + 2] = v.z;
+                        hw[4 * j + 3] = v.w;
                     }
                 }
                 uint32_t packed[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t lo = epi_value<EPI>(r[2 * i], s, hb[2 * i], amax);
-                    const uint32_t hi = epi_value<EPI>(r[2 * i + 1], s, hb[2 * i + 1], amax);
-                    packed[i] = lo | (hi << 16);
-                }
+                for (int i = 0; i < 16; ++i)
+                    packed[i] = epi_pair<EPI>(r[2 * i], r[2 * i + 1], s,
+                                              EPI == LM_EPI_RELU2_BWD ? hw[i] : 0u, amax2);
                 // staging buffer n_stores & 1: the store that last used it must
                 // have finished reading shared memory
                 uint8_t* dst = st_buf + (n_stores & 1u) * BOX_BYTES;
@@ -355,7 +400,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if (acc == 0) acc_phase ^= 1u;
         }
         if (lane == 0) bulk_wait_group<0>();
-        reduce_amax<EPI>(amax, args.amax_out, lane);
+        reduce_amax<EPI>(max(amax2 & 0xFFFFu, amax2 >> 16), args.amax_out, lane);
     }
 
     tc_fence_before();
@@ -647,9 +692,13 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
         a.num_mb = (int)((M + pair::TILE_M - 1) / pair::TILE_M);
         a.num_nb = (int)((N + pair::TILE_N - 1) / pair::TILE_N);
         a.num_tiles = a.num_mb * a.num_nb;
-        // up to 16 row-blocks: one group spans all of M, so every B panel is
-        // fetched once; otherwise groups of 8
-        a.group_m = a.num_mb <= 16 ? a.num_mb : 8;
+        // Sweep the smaller operand's dimension fastest: every wave of tiles
+        // then re-reads all of the smaller operand, which stays in L2, while
+        // the larger one streams through once.  N <= M: column-blocks fastest
+        // (groups of one row-block); otherwise row-blocks fastest (one group
+        // spanning M).
+        a.stream_a = N <= M ? 1 : 0;
+        a.group_m = a.stream_a ? 1 : a.num_mb;
         a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, pair::TILE_M, pair::TILE_N);
         CUtensorMap td, tx;
         if (!encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, 128, BK) ||
@@ -672,6 +721,7 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
     a.num_nb = (int)((N + one::BN - 1) / one::BN);
     a.num_tiles = a.num_mb * a.num_nb;
     a.group_m = 16;
+    a.stream_a = 0;
     a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, one::BM, one::BN);
     if (!encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, one::BM, BK) ||
         !encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, one::BN, BK))

@@ -228,6 +228,17 @@ LM_API void lm_timing_attach(void* const* events, int capacity);
 LM_API int lm_timing_detach(void);
 LM_API int lm_timing_kinds(char* out, int cap);
 
+/*
+ * Self-test of the device-side failure path (no counterpart on the pages).
+ * Enqueues one small kernel whose single thread waits, for at most limit_ms
+ * milliseconds (1..5000), on a shared-memory barrier that nothing ever
+ * arrives at.  The wait runs out, the kernel records code 0x301 in the
+ * device error word and exits normally, so the next lm_get_error() returns
+ * LM_ERR_TIMEOUT with where = 0x301 and the CUDA context stays usable.  Every
+ * wait in the GEMM and cast kernels takes this same bounded path.
+ */
+LM_API lm_status lm_selftest_bounded_wait(uint32_t limit_ms, lm_stream_t stream);
+
 /* Static, human-readable name of a status. */
 LM_API const char* lm_status_string(lm_status status);
 
