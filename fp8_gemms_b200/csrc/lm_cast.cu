@@ -221,21 +221,27 @@ __global__ void __launch_bounds__(kThreads) cast_kernel(
 
 
 // Pass 2, TMA-fed: a persistent kernel, two CTAs per SM.  Warp 8 streams
-// 128 x 128 bf16 tiles (32 KB) into a 3-stage shared ring with TMA; warps
-// 0-7 convert each tile (16-byte shared loads, 8-byte stores of row-major
-// codes to q), stage the codes in shared memory and write the transposed
-// codes to qT (4 x 4 byte permutes, one 16-byte store per column and warp).
+// 128 x 128 bf16 tiles (32 KB) into a 2-stage shared ring with TMA; warps
+// 0-7 convert each tile (16-byte shared loads; 8-byte stores of the
+// row-major codes straight to q) and build its transpose in shared memory,
+// which one thread writes to qT with a single TMA store per tile.
+//  - codes tile: word w of tile row r sits at r*32 + (w ^ 4*((r >> 4) & 7)),
+//    so both the row-major writes and the column-quad reads of the
+//    transpose are free of bank conflicts;
+//  - transposed tile: tile column c is a 128-byte row, its 16-byte chunk k
+//    at ((k ^ (c & 7)) * 16) -- the 128-byte swizzle the qT tensor map
+//    uses -- so the 16-byte writes are conflict-free too.
 // Tiles are taken in reverse memory order so the first ones re-read what the
 // amax pass left in L2.  Waits are bounded; after a timeout a thread stops
 // waiting but keeps the loop's barrier sequence, so no barrier can hang.
 namespace tmac {
 constexpr int TR = 128, TC = 128;
-constexpr int STAGES = 3;
+constexpr int STAGES = 2;
 constexpr int IN_BYTES = TR * TC * 2;
 constexpr int CODE_BYTES = TR * TC;
 constexpr int CONSUMERS = 256;
 constexpr int THREADS = CONSUMERS + 32;
-constexpr int SMEM = STAGES * IN_BYTES + CODE_BYTES + 128 + 128;
+constexpr int SMEM = 1024 + CODE_BYTES + STAGES * IN_BYTES + CODE_BYTES + 64;
 enum : unsigned { W_CAST_EMPTY = 0x201, W_CAST_FULL = 0x202, W_CAST_LOADS = 0x203 };
 }  // namespace tmac
 
@@ -245,16 +251,17 @@ __device__ __forceinline__ void consumers_sync() {
 
 template <int FMT, bool RELU2>
 __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
-    const __grid_constant__ CUtensorMap tmX, int rows, int cols, const float* amax_src,
-    float* amax_out, float* scale_out, float* inv_out, uint8_t* __restrict__ q,
-    uint8_t* __restrict__ qT, int tiles_c, int num_tiles, unsigned int* err) {
+    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQT, int rows,
+    int cols, const float* amax_src, float* amax_out, float* scale_out, float* inv_out,
+    uint8_t* __restrict__ q, int want_qT, int tiles_c, int num_tiles, unsigned int* err) {
     using namespace tmac;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
-    uint8_t* smem = smem_raw + ((128u - (raw & 127u)) & 127u);
-    uint8_t* sIn = smem;
-    uint32_t* sCode = reinterpret_cast<uint32_t*>(smem + STAGES * IN_BYTES);  // [TR][TC/4]
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * IN_BYTES + CODE_BYTES);
+    uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    uint8_t* sT = smem;                         // transposed codes, 1024-aligned
+    uint8_t* sIn = smem + CODE_BYTES;           // STAGES x 32 KB
+    uint32_t* sCode = reinterpret_cast<uint32_t*>(sIn + STAGES * IN_BYTES);  // [TR][TC/4]
+    uint64_t* full = reinterpret_cast<uint64_t*>(sIn + STAGES * IN_BYTES + CODE_BYTES);
     uint64_t* empty = full + STAGES;
 
     const float fmax = FMT == LM_FP8_E4M3 ? 448.0f : 57344.0f;
@@ -313,7 +320,8 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
             const int r = r0 + rr, c = c0 + ch * 8;
             if (q && r < rows && c < cols)
                 *reinterpret_cast<uint2*>(q + (int64_t)r * cols + c) = codes;
-            *reinterpret_cast<uint2*>(&sCode[rr * (TC / 4) + ch * 2]) = codes;
+            const int wpos = (2 * ch) ^ (4 * ((rr >> 4) & 7));
+            *reinterpret_cast<uint2*>(&sCode[rr * (TC / 4) + wpos]) = codes;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
@@ -321,36 +329,41 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
             s = 0;
             ph ^= 1u;
         }
-        if (!qT) continue;
-        consumers_sync();  // the codes tile is complete
-        // warp w: tile rows [16w, 16w+16); lane l: tile columns [4l, 4l+4)
+        if (!want_qT) continue;
+        if (tid == 0) bulk_wait_group_read<0>();  // the previous tile's store has read sT
+        consumers_sync();                           // codes tile complete, sT free
+        // lane: tile rows [16k, 16k+16) with k = lane % 8; tile columns
+        // [4q, 4q+4) with q = 4 * warp + lane / 8
+        const int k = lane & 7, qd = 4 * warp + (lane >> 3);
         uint32_t v[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = sCode[(warp * 16 + k) * (TC / 4) + lane];
-        uint32_t o[4][4];  // o[j][k]: column 4l+j, rows 16w+4k .. +3
+        for (int i2 = 0; i2 < 16; ++i2) v[i2] = sCode[(16 * k + i2) * (TC / 4) + (qd ^ (4 * k))];
+        uint32_t o[4][4];  // o[j][m]: column 4q+j, rows 16k+4m .. +3
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t t0 = __byte_perm(v[4 * k], v[4 * k + 1], 0x5140);
-            const uint32_t t1 = __byte_perm(v[4 * k + 2], v[4 * k + 3], 0x5140);
-            const uint32_t t2 = __byte_perm(v[4 * k], v[4 * k + 1], 0x7362);
-            const uint32_t t3 = __byte_perm(v[4 * k + 2], v[4 * k + 3], 0x7362);
-            o[0][k] = __byte_perm(t0, t1, 0x5410);
-            o[1][k] = __byte_perm(t0, t1, 0x7632);
-            o[2][k] = __byte_perm(t2, t3, 0x5410);
-            o[3][k] = __byte_perm(t2, t3, 0x7632);
+        for (int m = 0; m < 4; ++m) {
+            const uint32_t t0 = __byte_perm(v[4 * m], v[4 * m + 1], 0x5140);
+            const uint32_t t1 = __byte_perm(v[4 * m + 2], v[4 * m + 3], 0x5140);
+            const uint32_t t2 = __byte_perm(v[4 * m], v[4 * m + 1], 0x7362);
+            const uint32_t t3 = __byte_perm(v[4 * m + 2], v[4 * m + 3], 0x7362);
+            o[0][m] = __byte_perm(t0, t1, 0x5410);
+            o[1][m] = __byte_perm(t0, t1, 0x7632);
+            o[2][m] = __byte_perm(t2, t3, 0x5410);
+            o[3][m] = __byte_perm(t2, t3, 0x7632);
         }
-        const int rb = r0 + warp * 16;
-        if (rb < rows) {  // rows % 16 == 0: a 16-row group is all in or all out
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int c = c0 + 4 * lane + j;
-                if (c < cols)
-                    *reinterpret_cast<uint4*>(qT + (int64_t)c * rows + rb) =
-                        make_uint4(o[j][0], o[j][1], o[j][2], o[j][3]);
-            }
+        for (int j = 0; j < 4; ++j) {
+            const int c = 4 * qd + j;
+            *reinterpret_cast<uint4*>(sT + c * 128 + ((k ^ (c & 7)) << 4)) =
+                make_uint4(o[j][0], o[j][1], o[j][2], o[j][3]);
         }
-        consumers_sync();  // before the next tile overwrites the codes
+        fence_proxy_async_smem();
+        consumers_sync();  // transposed tile complete; codes tile fully read
+        if (tid == 0) {
+            tma_store_2d(&tmQT, smem_addr(sT), r0, c0);
+            bulk_commit_group();
+        }
     }
+    if (tid == 0) bulk_wait_group<0>();
 }
 
 template <int FMT, bool RELU2>
@@ -369,10 +382,17 @@ lm_status launch_cast(const uint16_t* x, int rows, int cols, int64_t ld, const f
                 return LM_ERR_CUDA;
             configured[dev] = true;
         }
-        CUtensorMap tm;
+        CUtensorMap tm, tq;
         if (!encode_tmap_bf16_plain(&tm, x, (uint64_t)rows, (uint64_t)cols, (uint64_t)ld * 2,
                                     tmac::TR, tmac::TC))
             return LM_ERR_CUDA;
+        if (qT) {  // qT is [cols x rows]: tile rows become 128-byte rows of codes
+            if (!encode_tmap_u8(&tq, qT, (uint64_t)cols, (uint64_t)rows, (uint64_t)rows, tmac::TC,
+                                tmac::TR))
+                return LM_ERR_CUDA;
+        } else {
+            tq = tm;  // unused
+        }
         unsigned int* err = device_error_word();
         if (!err) return LM_ERR_CUDA;
         const int tiles_c = (cols + tmac::TC - 1) / tmac::TC;
@@ -382,7 +402,8 @@ lm_status launch_cast(const uint16_t* x, int rows, int cols, int64_t ld, const f
         if (grid > n) grid = n;
         timing_mark(s, 'c');
         cast_tma_kernel<FMT, RELU2><<<grid, tmac::THREADS, tmac::SMEM, s>>>(
-            tm, rows, cols, amax_src, amax_out, scale_out, inv_out, q, qT, tiles_c, n, err);
+            tm, tq, rows, cols, amax_src, amax_out, scale_out, inv_out, q, qT ? 1 : 0, tiles_c, n,
+            err);
         return launch_status();
     }
     const int tiles_r = (rows + kCastRows - 1) / kCastRows;
