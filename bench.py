@@ -42,7 +42,10 @@ LAUNCHES_PER_STEP = 16                         # kernels of ours per fwd+bwd: "a
 # DRAM traffic of one GEMM launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum), valid only for the kernel source it was taken on;
 # the summary and the command are in profiles/.
-GEMM_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None}
+GEMM_TRAFFIC = {
+    "source_sha256": "34d6339b86646053ba2ea7ebcb7ed88a1a8c2bcd5f7e26a686682d971c6b454c",
+    "bytes_per_launch": 585130197,  # mean of the step's six GEMMs, profiles/gemm_fp8_pair_relu2_mlp_shapes.md
+}
 
 
 def parse_args():
@@ -287,7 +290,7 @@ def run_gpu(args):
                    "gemms_per_step": 6, "flops_per_step": STEP_FLOPS,
                    "l2": "flushed before every timed step (256 MiB write)",
                    "parallelism": f"{world} independent replica(s), no collective"},
-        "roofline": {"bound": "tensor", "kernel": "gemm_fp8_kernel (tcgen05)",
+        "roofline": {"bound": "tensor", "kernel": "gemm_fp8_pair_kernel (tcgen05, CTA pairs)",
                      "achieved": round(achieved, 2), "peak": round(fp8_peak, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
                      "peak_source": f"{peaks['src']} bf16 sustained {peaks['bf16_sus']} x "
