@@ -13,7 +13,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libfp8lm.so")
 
 E4M3, E5M2 = 0, 1
-EPI_NONE, EPI_RELU2_FWD, EPI_RELU2_BWD = 0, 1, 2
+EPI_NONE, EPI_RELU2_FWD, EPI_RELU2_BWD, EPI_ACCUM_F32 = 0, 1, 2, 3
+MLP_REUSE_WEIGHT_CASTS, MLP_ACCUMULATE_WGRAD = 1, 2
 
 STATUS = {0: "LM_OK", 1: "LM_ERR_INVALID_ARG", 2: "LM_ERR_ALIGNMENT",
           3: "LM_ERR_UNSUPPORTED_SHAPE", 4: "LM_ERR_UNSUPPORTED_FORMAT", 5: "LM_ERR_CUDA",
@@ -24,7 +25,7 @@ EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
             "lm_relu2_mlp_bwd", "lm_get_error", "lm_status_string", "lm_version",
             "lm_timing_attach", "lm_timing_detach", "lm_timing_kinds",
             "lm_relu2_mlp_bwd_noalloc", "lm_relu2_mlp_bwd_noalloc_max_bytes",
-            "lm_selftest_bounded_wait"]
+            "lm_selftest_bounded_wait", "lm_relu2_mlp_fwd_ex", "lm_relu2_mlp_bwd_ex"]
 
 
 class LmError(RuntimeError):
@@ -76,6 +77,12 @@ def _load():
     L.lm_relu2_mlp_bwd_noalloc.restype = st
     L.lm_relu2_mlp_bwd_noalloc_max_bytes.argtypes = []
     L.lm_relu2_mlp_bwd_noalloc_max_bytes.restype = ctypes.c_size_t
+    L.lm_relu2_mlp_fwd_ex.argtypes = [P, P, P, i64, i64, i64, P, ctypes.POINTER(MlpSaved),
+                                      ctypes.c_uint32, P]
+    L.lm_relu2_mlp_fwd_ex.restype = st
+    L.lm_relu2_mlp_bwd_ex.argtypes = [P, ctypes.POINTER(MlpSaved), i64, i64, i64, P, P, P, P,
+                                      ctypes.c_size_t, ctypes.c_uint32, P]
+    L.lm_relu2_mlp_bwd_ex.restype = st
     L.lm_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
     L.lm_selftest_bounded_wait.restype = st
     return L
@@ -156,6 +163,23 @@ def lm_relu2_mlp_bwd(dY, saved, dX, dW_up, dW_down, workspace, stream=None):
                                 _p(dW_down), _p(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(stream)),
            "lm_relu2_mlp_bwd")
+
+
+def lm_relu2_mlp_fwd_ex(X, W_up, W_down, Y, saved, f, flags=0, stream=None):
+    """f: hidden size (W_up may be None when its cast is reused)."""
+    M, d = X.shape
+    _check(lib.lm_relu2_mlp_fwd_ex(_p(X), _p(W_up), _p(W_down), M, d, f, _p(Y),
+                                   ctypes.byref(saved), flags, _stream(stream)),
+           "lm_relu2_mlp_fwd_ex")
+
+
+def lm_relu2_mlp_bwd_ex(dY, saved, dX, dW_up, dW_down, workspace, flags=0, stream=None):
+    M, d = dY.shape
+    f = dW_up.shape[0]
+    _check(lib.lm_relu2_mlp_bwd_ex(_p(dY), ctypes.byref(saved), M, d, f, _p(dX), _p(dW_up),
+                                   _p(dW_down), _p(workspace),
+                                   workspace.numel() * workspace.element_size(), flags,
+                                   _stream(stream)), "lm_relu2_mlp_bwd_ex")
 
 
 def lm_relu2_mlp_bwd_noalloc(dY, saved, dX, dW_up, dW_down, stream=None):

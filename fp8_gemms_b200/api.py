@@ -9,7 +9,8 @@ libfp8lm.so does every step of the computation.
 import torch
 
 from . import _lib
-from ._lib import E4M3, E5M2, EPI_NONE, EPI_RELU2_BWD, EPI_RELU2_FWD, LmError  # noqa: F401
+from ._lib import (E4M3, E5M2, EPI_ACCUM_F32, EPI_NONE, EPI_RELU2_BWD,  # noqa: F401
+                   EPI_RELU2_FWD, MLP_ACCUMULATE_WGRAD, MLP_REUSE_WEIGHT_CASTS, LmError)
 
 
 def _dev(t):
@@ -61,11 +62,27 @@ class Relu2Mlp:
                                      dtype=torch.uint8, device=device)
         self.device = device
 
-    def forward(self, X, W_up, W_down, Y=None, stream=None):
+    def forward(self, X, W_up, W_down, Y=None, stream=None, reuse_weight_casts=False):
+        """reuse_weight_casts: W_up/W_down were cast by an earlier forward of
+        the same weights (gradient accumulation); their casts are skipped."""
         if Y is None:
             Y = torch.empty(self.M, self.d, dtype=torch.bfloat16, device=self.device)
-        _lib.lm_relu2_mlp_fwd(X, W_up, W_down, Y, self.saved, stream=stream)
+        if reuse_weight_casts:
+            _lib.lm_relu2_mlp_fwd_ex(X, None, None, Y, self.saved, self.f,
+                                     flags=MLP_REUSE_WEIGHT_CASTS, stream=stream)
+        else:
+            _lib.lm_relu2_mlp_fwd(X, W_up, W_down, Y, self.saved, stream=stream)
         return Y
+
+    def backward_accumulate(self, dY, dW_up_f32, dW_down_f32, dX=None, stream=None):
+        """Backward that adds this micro-batch's weight gradients into fp32
+        accumulators dW_up_f32 [f x d] and dW_down_f32 [d x f]; returns dX."""
+        dX = dX if dX is not None else torch.empty(self.M, self.d, dtype=torch.bfloat16,
+                                                   device=self.device)
+        assert dW_up_f32.dtype == torch.float32 and dW_down_f32.dtype == torch.float32
+        _lib.lm_relu2_mlp_bwd_ex(dY, self.saved, dX, dW_up_f32, dW_down_f32, self.workspace,
+                                 flags=MLP_ACCUMULATE_WGRAD, stream=stream)
+        return dX
 
     def backward(self, dY, dX=None, dW_up=None, dW_down=None, stream=None):
         dev = self.device

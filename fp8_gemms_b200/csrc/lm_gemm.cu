@@ -48,7 +48,7 @@ struct GemmArgs {
     const float* inv_a;
     const float* inv_b;
     const uint16_t* aux;
-    uint16_t* D;
+    void* D;
     float* amax_out;
     unsigned int* err;
     uint32_t idesc;
@@ -147,6 +147,10 @@ constexpr int EPI_COLS = 32;                   // columns per epilogue chunk
 constexpr int BOX_BYTES = 32 * EPI_COLS * 2;   // one warp's 32 x 32 bf16 box
 constexpr int STORE_BYTES = NUM_EPI_WARPS * 2 * BOX_BYTES;
 constexpr int AUX_BYTES = NUM_EPI_WARPS * 2 * BOX_BYTES;
+// the accumulating epilogue stages 32 x 32 fp32 boxes (4 KB, two per warp) in
+// the store and aux areas together (contiguous, 32 KB)
+constexpr int ACC_BOX_BYTES = 32 * EPI_COLS * 4;
+static_assert(NUM_EPI_WARPS * 2 * ACC_BOX_BYTES == STORE_BYTES + AUX_BYTES, "staging layout");
 constexpr uint32_t TMEM_COLS = 2 * TILE_N;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + AUX_BYTES + 1024 + 512;
 
@@ -369,6 +373,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         hw[4 * j + 3] = v.w;
                     }
                 }
+                if (EPI == LM_EPI_ACCUM_F32) {
+                    // fp32 partial -> 128B-swizzled 32 x 32 fp32 box -> TMA reduce-add
+                    uint8_t* dst = sStore + wi * 2 * ACC_BOX_BYTES + (n_stores & 1u) * ACC_BOX_BYTES;
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<float4*>(dst + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                            make_float4(__fmul_rn(__uint_as_float(r[4 * j]), s),
+                                        __fmul_rn(__uint_as_float(r[4 * j + 1]), s),
+                                        __fmul_rn(__uint_as_float(r[4 * j + 2]), s),
+                                        __fmul_rn(__uint_as_float(r[4 * j + 3]), s));
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_reduce_add_2d(&tmD, smem_addr(dst), gcol + c * EPI_COLS, grow);
+                        bulk_commit_group();
+                    }
+                    ++n_stores;
+                    continue;
+                }
                 uint32_t packed[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
@@ -562,6 +587,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tmem_ld_wait();
                 if (!row_ok) continue;
                 const int64_t off = (int64_t)row * args.N + col0;
+                if (EPI == LM_EPI_ACCUM_F32) {
+                    // each element has one owner thread: a plain read-modify-write
+                    float* Df = static_cast<float*>(args.D) + off;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        if (col0 + v * 4 >= args.N) break;
+                        float4 d4 = *reinterpret_cast<float4*>(Df + v * 4);
+                        d4.x = __fadd_rn(d4.x, __fmul_rn(__uint_as_float(r[4 * v]), s));
+                        d4.y = __fadd_rn(d4.y, __fmul_rn(__uint_as_float(r[4 * v + 1]), s));
+                        d4.z = __fadd_rn(d4.z, __fmul_rn(__uint_as_float(r[4 * v + 2]), s));
+                        d4.w = __fadd_rn(d4.w, __fmul_rn(__uint_as_float(r[4 * v + 3]), s));
+                        *reinterpret_cast<float4*>(Df + v * 4) = d4;
+                    }
+                    continue;
+                }
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                     if (col0 + v * 8 >= args.N) break;
@@ -578,7 +618,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     uint32_t ob[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) ob[i] = epi_value<EPI>(r[v * 8 + i], s, hb[i], amax);
-                    *reinterpret_cast<uint4*>(args.D + off + v * 8) =
+                    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(args.D) + off + v * 8) =
                         make_uint4(ob[0] | (ob[1] << 16), ob[2] | (ob[3] << 16),
                                    ob[4] | (ob[5] << 16), ob[6] | (ob[7] << 16));
                 }
@@ -654,7 +694,8 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
     if ((fa != LM_FP8_E4M3 && fa != LM_FP8_E5M2) || (fb != LM_FP8_E4M3 && fb != LM_FP8_E5M2))
         return LM_ERR_UNSUPPORTED_FORMAT;
     if (fa == LM_FP8_E5M2 && fb == LM_FP8_E5M2) return LM_ERR_UNSUPPORTED_FORMAT;
-    if (epi != LM_EPI_NONE && epi != LM_EPI_RELU2_FWD && epi != LM_EPI_RELU2_BWD)
+    if (epi != LM_EPI_NONE && epi != LM_EPI_RELU2_FWD && epi != LM_EPI_RELU2_BWD &&
+        epi != LM_EPI_ACCUM_F32)
         return LM_ERR_UNSUPPORTED_FORMAT;
     if (M < 0 || N < 0 || K < 0) return LM_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return LM_OK;
@@ -668,7 +709,8 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
         return LM_ERR_ALIGNMENT;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (K == 0) {  // empty reduction: D = epi(0) = 0, amax unchanged
+    if (K == 0) {  // empty reduction: D = epi(0) = 0 (accumulating: D += 0), amax unchanged
+        if (epi == LM_EPI_ACCUM_F32) return LM_OK;
         if (cudaMemsetAsync(D, 0, (size_t)M * (size_t)N * 2, s) != cudaSuccess)
             return LM_ERR_CUDA;
         return LM_OK;
@@ -683,7 +725,8 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
     a.inv_a = inv_scale_a;
     a.inv_b = inv_scale_b;
     a.aux = static_cast<const uint16_t*>(aux);
-    a.D = static_cast<uint16_t*>(D);
+    a.D = D;
+    if (epi == LM_EPI_ACCUM_F32) a.amax_out = nullptr;
     a.amax_out = amax_out;
     a.err = err;
 
@@ -702,9 +745,14 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
         a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, pair::TILE_M, pair::TILE_N);
         CUtensorMap td, tx;
         if (!encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, 128, BK) ||
-            !encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, 128, BK) ||
-            !encode_tmap_bf16_sw64(&td, D, (uint64_t)M, (uint64_t)N, 32, pair::EPI_COLS))
+            !encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, 128, BK))
             return LM_ERR_CUDA;
+        const bool dok = epi == LM_EPI_ACCUM_F32
+                             ? encode_tmap_f32_sw128(&td, D, (uint64_t)M, (uint64_t)N, 32,
+                                                     pair::EPI_COLS)
+                             : encode_tmap_bf16_sw64(&td, D, (uint64_t)M, (uint64_t)N, 32,
+                                                     pair::EPI_COLS);
+        if (!dok) return LM_ERR_CUDA;
         if (epi == LM_EPI_RELU2_BWD) {
             if (!encode_tmap_bf16_sw64(&tx, aux, (uint64_t)M, (uint64_t)N, 32, pair::EPI_COLS))
                 return LM_ERR_CUDA;
@@ -714,7 +762,8 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
         switch (epi) {
             case LM_EPI_NONE: return launch_pair<LM_EPI_NONE>(ta, tb, td, tx, a, s);
             case LM_EPI_RELU2_FWD: return launch_pair<LM_EPI_RELU2_FWD>(ta, tb, td, tx, a, s);
-            default: return launch_pair<LM_EPI_RELU2_BWD>(ta, tb, td, tx, a, s);
+            case LM_EPI_RELU2_BWD: return launch_pair<LM_EPI_RELU2_BWD>(ta, tb, td, tx, a, s);
+            default: return launch_pair<LM_EPI_ACCUM_F32>(ta, tb, td, tx, a, s);
         }
     }
     a.num_mb = (int)((M + one::BM - 1) / one::BM);
@@ -729,6 +778,7 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
     switch (epi) {
         case LM_EPI_NONE: return launch_one<LM_EPI_NONE>(ta, tb, a, s);
         case LM_EPI_RELU2_FWD: return launch_one<LM_EPI_RELU2_FWD>(ta, tb, a, s);
-        default: return launch_one<LM_EPI_RELU2_BWD>(ta, tb, a, s);
+        case LM_EPI_RELU2_BWD: return launch_one<LM_EPI_RELU2_BWD>(ta, tb, a, s);
+        default: return launch_one<LM_EPI_ACCUM_F32>(ta, tb, a, s);
     }
 }

@@ -29,6 +29,12 @@ bool encode_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 bool encode_tmap_bf16_sw64(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                            uint32_t box_rows, uint32_t box_cols);
 
+// 2-D fp32 tensor map for a row-major [rows x cols] matrix, box
+// [box_rows x box_cols] with the 128-byte swizzle (box_cols * 4 must be 128);
+// used for the accumulating epilogue's TMA reduce-adds.
+bool encode_tmap_f32_sw128(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                           uint32_t box_rows, uint32_t box_cols);
+
 // 2-D bf16 tensor map, no swizzle, row pitch `pitch` bytes (a multiple of
 // 16), box [box_rows x box_cols]; out-of-bounds elements read as zero.
 bool encode_tmap_bf16_plain(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,

@@ -102,25 +102,33 @@ size_t lm_relu2_mlp_workspace_size(int64_t M, int64_t d, int64_t f) {
     return bwd_layout(M, d, f, nullptr, nullptr);
 }
 
-lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W_down, int64_t M,
-                           int64_t d, int64_t f, void* Y, lm_mlp_saved* sv, void* workspace,
-                           size_t ws_bytes, lm_stream_t stream) {
-    (void)workspace;
-    (void)ws_bytes;
+lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_down, int64_t M,
+                              int64_t d, int64_t f, void* Y, lm_mlp_saved* sv, uint32_t flags,
+                              lm_stream_t stream) {
     if (!mlp_shape_ok(M, d, f)) return LM_ERR_UNSUPPORTED_SHAPE;
-    if (!X || !W_up || !W_down || !Y || !sv) return LM_ERR_INVALID_ARG;
+    if (flags & ~LM_MLP_REUSE_WEIGHT_CASTS) return LM_ERR_INVALID_ARG;
+    const bool reuse = (flags & LM_MLP_REUSE_WEIGHT_CASTS) != 0;
+    if (!X || !Y || !sv || (!reuse && (!W_up || !W_down))) return LM_ERR_INVALID_ARG;
     if (!sv->Xq || !sv->XqT || !sv->Wuq || !sv->WuqT || !sv->Wdq || !sv->WdqT || !sv->H ||
         !sv->hq || !sv->hqT || !sv->scales)
         return LM_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     float* S = sv->scales;
-    if (cudaMemsetAsync(S, 0, 16 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
+    if (reuse) {  // keep the weights' scale blocks; reset X's and h's
+        if (cudaMemsetAsync(S + S_X, 0, 4 * sizeof(float), s) != cudaSuccess ||
+            cudaMemsetAsync(S + S_H, 0, 4 * sizeof(float), s) != cudaSuccess)
+            return LM_ERR_CUDA;
+    } else if (cudaMemsetAsync(S, 0, 16 * sizeof(float), s) != cudaSuccess) {
+        return LM_ERR_CUDA;
+    }
     LM_TRY(lm_fp8_amax_scale_cast(X, M, d, d, LM_FP8_E4M3, 0, nullptr, S + S_X, S + S_X + 1,
                                   S + S_X + 2, sv->Xq, sv->XqT, stream));
-    LM_TRY(lm_fp8_amax_scale_cast(W_up, f, d, d, LM_FP8_E4M3, 0, nullptr, S + S_WU, S + S_WU + 1,
-                                  S + S_WU + 2, sv->Wuq, sv->WuqT, stream));
-    LM_TRY(lm_fp8_amax_scale_cast(W_down, d, f, f, LM_FP8_E4M3, 0, nullptr, S + S_WD,
-                                  S + S_WD + 1, S + S_WD + 2, sv->Wdq, sv->WdqT, stream));
+    if (!reuse) {
+        LM_TRY(lm_fp8_amax_scale_cast(W_up, f, d, d, LM_FP8_E4M3, 0, nullptr, S + S_WU,
+                                      S + S_WU + 1, S + S_WU + 2, sv->Wuq, sv->WuqT, stream));
+        LM_TRY(lm_fp8_amax_scale_cast(W_down, d, f, f, LM_FP8_E4M3, 0, nullptr, S + S_WD,
+                                      S + S_WD + 1, S + S_WD + 2, sv->Wdq, sv->WdqT, stream));
+    }
     // H = X W_up^T (bf16) and amax of h = bf16(relu(H)^2)
     LM_TRY(lm_fp8_gemm(sv->Xq, LM_FP8_E4M3, sv->Wuq, LM_FP8_E4M3, M, f, d, S + S_X + 2,
                        S + S_WU + 2, LM_EPI_RELU2_FWD, nullptr, sv->H, S + S_H, stream));
@@ -132,13 +140,24 @@ lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W_down, 
     return LM_OK;
 }
 
-lm_status lm_relu2_mlp_bwd(const void* dY, const lm_mlp_saved* sv, int64_t M, int64_t d,
-                           int64_t f, void* dX, void* dW_up, void* dW_down, void* workspace,
+lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W_down, int64_t M,
+                           int64_t d, int64_t f, void* Y, lm_mlp_saved* sv, void* workspace,
                            size_t ws_bytes, lm_stream_t stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    return lm_relu2_mlp_fwd_ex(X, W_up, W_down, M, d, f, Y, sv, 0u, stream);
+}
+
+lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* sv, int64_t M, int64_t d,
+                              int64_t f, void* dX, void* dW_up, void* dW_down, void* workspace,
+                              size_t ws_bytes, uint32_t flags, lm_stream_t stream) {
     if (!mlp_shape_ok(M, d, f)) return LM_ERR_UNSUPPORTED_SHAPE;
+    if (flags & ~LM_MLP_ACCUMULATE_WGRAD) return LM_ERR_INVALID_ARG;
     if (!dY || !sv || !dX || !dW_up || !dW_down || !workspace) return LM_ERR_INVALID_ARG;
     if (ws_bytes < bwd_layout(M, d, f, nullptr, nullptr)) return LM_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return LM_ERR_ALIGNMENT;
+    const lm_epilogue wgrad_epi =
+        (flags & LM_MLP_ACCUMULATE_WGRAD) ? LM_EPI_ACCUM_F32 : LM_EPI_NONE;
     BwdWorkspace w;
     bwd_layout(M, d, f, static_cast<uint8_t*>(workspace), &w);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -152,15 +171,22 @@ lm_status lm_relu2_mlp_bwd(const void* dY, const lm_mlp_saved* sv, int64_t M, in
                        S + S_WD + 2, LM_EPI_RELU2_BWD, sv->H, w.dH, G + S_DH, stream));
     // dW_down = dY^T h (K = M)
     LM_TRY(lm_fp8_gemm(w.dYqT, LM_FP8_E5M2, sv->hqT, LM_FP8_E4M3, d, f, M, G + S_DY + 2,
-                       S + S_H + 2, LM_EPI_NONE, nullptr, dW_down, nullptr, stream));
+                       S + S_H + 2, wgrad_epi, nullptr, dW_down, nullptr, stream));
     LM_TRY(lm_fp8_amax_scale_cast(w.dH, M, f, f, LM_FP8_E5M2, 0, G + S_DH, G + S_DH,
                                   G + S_DH + 1, G + S_DH + 2, w.dHq, w.dHqT, stream));
     // dX = dH W_up;  dW_up = dH^T X (K = M)
     LM_TRY(lm_fp8_gemm(w.dHq, LM_FP8_E5M2, sv->WuqT, LM_FP8_E4M3, M, d, f, G + S_DH + 2,
                        S + S_WU + 2, LM_EPI_NONE, nullptr, dX, nullptr, stream));
     LM_TRY(lm_fp8_gemm(w.dHqT, LM_FP8_E5M2, sv->XqT, LM_FP8_E4M3, f, d, M, G + S_DH + 2,
-                       S + S_X + 2, LM_EPI_NONE, nullptr, dW_up, nullptr, stream));
+                       S + S_X + 2, wgrad_epi, nullptr, dW_up, nullptr, stream));
     return LM_OK;
+}
+
+lm_status lm_relu2_mlp_bwd(const void* dY, const lm_mlp_saved* sv, int64_t M, int64_t d,
+                           int64_t f, void* dX, void* dW_up, void* dW_down, void* workspace,
+                           size_t ws_bytes, lm_stream_t stream) {
+    return lm_relu2_mlp_bwd_ex(dY, sv, M, d, f, dX, dW_up, dW_down, workspace, ws_bytes, 0u,
+                               stream);
 }
 
 }  // extern "C"

@@ -4,6 +4,10 @@ iterations).  Also the small, self-contained command to run under ncu.
     python -m fp8_gemms_b200.microbench gemm --M 16384 --N 12288 --K 3072 --epi relu2_fwd
     python -m fp8_gemms_b200.microbench cast --rows 16384 --cols 3072 --fmt e4m3
     python -m fp8_gemms_b200.microbench cast --rows 16384 --cols 12288 --relu2 --amax-in
+    python -m fp8_gemms_b200.microbench mlp-accum --M 16384 --micro 7
+        (one optimizer step of gradient accumulation: the weights are cast by the
+        first micro-batch's forward and reused by the others; every backward adds
+        its weight gradients into fp32 accumulators)
 """
 import argparse
 import json
@@ -41,7 +45,10 @@ def time_it(fn, iters, warmup, flush):
 
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("op", choices=["gemm", "cast"])
+    p.add_argument("op", choices=["gemm", "cast", "mlp-accum"])
+    p.add_argument("--micro", type=int, default=7)
+    p.add_argument("--d", type=int, default=3072)
+    p.add_argument("--f", type=int, default=12288)
     p.add_argument("--M", type=int, default=16384)
     p.add_argument("--N", type=int, default=12288)
     p.add_argument("--K", type=int, default=3072)
@@ -58,7 +65,9 @@ def main():
     a = p.parse_args()
     gen = torch.Generator(device="cuda").manual_seed(0)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    if a.op == "gemm":
+    if a.op == "mlp-accum":
+        pass
+    elif a.op == "gemm":
         fa, fb, epi = FMT[a.fa], FMT[a.fb], EPI[a.epi]
         A = random_codes(fa, a.M, a.K, gen)
         B = random_codes(fb, a.N, a.K, gen)
@@ -92,6 +101,34 @@ def main():
         out = dict(op="cast", rows=a.rows, cols=a.cols, fmt=a.fmt, relu2=a.relu2,
                    amax_in=a.amax_in, avg_ms=round(avg, 4), min_ms=round(min(ms), 4),
                    gbs=round(byts / avg / 1e6, 1), algorithmic_bytes=byts)
+    if a.op == "mlp-accum":
+        from . import api
+        M, d, f = a.M, a.d, a.f
+        mlp = api.Relu2Mlp(M, d, f)
+        Wu = (torch.randn(f, d, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)
+        Wd = (torch.randn(d, f, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)
+        Xs = [torch.randn(M, d, device="cuda", generator=gen).to(torch.bfloat16)
+              for _ in range(a.micro)]
+        dYs = [(torch.randn(M, d, device="cuda", generator=gen) * 1e-3).to(torch.bfloat16)
+               for _ in range(a.micro)]
+        dWu = torch.zeros(f, d, dtype=torch.float32, device="cuda")
+        dWd = torch.zeros(d, f, dtype=torch.float32, device="cuda")
+        Y = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+        dX = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+
+        def opt_step():
+            dWu.zero_()
+            dWd.zero_()
+            for i in range(a.micro):
+                mlp.forward(Xs[i], Wu, Wd, Y=Y, reuse_weight_casts=i > 0)
+                mlp.backward_accumulate(dYs[i], dWu, dWd, dX=dX)
+
+        ms = time_it(opt_step, a.iters, a.warmup, flush)
+        avg = sum(ms) / len(ms)
+        flops = a.micro * 6 * 2 * M * d * f
+        out = dict(op="mlp-accum", M=M, d=d, f=f, micro_batches=a.micro, avg_ms=round(avg, 4),
+                   ms_per_micro_batch=round(avg / a.micro, 4),
+                   tflops=round(flops / avg / 1e9, 1))
     st, where = _lib.lm_get_error()
     out["device_error"] = st
     print(json.dumps(out))

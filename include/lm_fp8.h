@@ -66,8 +66,18 @@ typedef enum { LM_FP8_E4M3 = 0, LM_FP8_E5M2 = 1 } lm_fp8_format;
 typedef enum {
     LM_EPI_NONE = 0,      /* D = bf16(acc * s) */
     LM_EPI_RELU2_FWD = 1, /* D = H = bf16(acc * s); amax of h = bf16(relu(H)^2) */
-    LM_EPI_RELU2_BWD = 2  /* g = bf16(acc * s); D = dH = bf16(g * 2 * relu(aux)) */
+    LM_EPI_RELU2_BWD = 2, /* g = bf16(acc * s); D = dH = bf16(g * 2 * relu(aux)) */
+    LM_EPI_ACCUM_F32 = 3  /* D is fp32: D += fp32(acc * s) (gradient accumulation) */
 } lm_epilogue;
+
+/* Flags of lm_relu2_mlp_fwd_ex / lm_relu2_mlp_bwd_ex (gradient accumulation
+ * over micro-batches: decomputer.nl, "Het trainen van een 3.8B LLM tot 0.384
+ * CORE voor $998", section "Vroege experimenten" item 2 and "Appendix: De
+ * configuratie", total_batch_size = 20 x 2048 x 7 grad_accum x 8 GPUs). */
+#define LM_MLP_REUSE_WEIGHT_CASTS 1u /* fwd: the W_up/W_down codes and scales already in
+                                        `saved` are current; their casts are skipped */
+#define LM_MLP_ACCUMULATE_WGRAD 2u   /* bwd: dW_up and dW_down are fp32 accumulators;
+                                        this micro-batch's weight gradients are added */
 
 /*
  * Dynamic tensorwise scaling cast (amax -> scale -> saturating RNE cast).
@@ -106,11 +116,13 @@ LM_API lm_status lm_fp8_amax_scale_cast(const void* x, int64_t rows, int64_t col
  * inv_scale_a / inv_scale_b: device fp32 dequantisation factors (1/scale).
  * aux: bf16 [M x N], the saved pre-activation H, required for
  *   LM_EPI_RELU2_BWD, ignored otherwise.
- * D: bf16 [M x N], row-major.
+ * D: bf16 [M x N], row-major; for LM_EPI_ACCUM_F32 an fp32 [M x N] accumulator
+ *   that is added to (each element receives exactly one add per call, so the
+ *   result does not depend on scheduling).
  * amax_out: device fp32 or NULL.  If non-NULL it is max-reduced (atomically,
  *   order independent) with the amax of the tensor the next cast consumes:
- *   max|D| (NONE), max bf16(relu(D)^2) (RELU2_FWD), max|D| (RELU2_BWD).  The
- *   caller zeroes it before the first GEMM that feeds it.
+ *   max|D| (NONE), max bf16(relu(D)^2) (RELU2_FWD), max|D| (RELU2_BWD); unused
+ *   for ACCUM_F32.  The caller zeroes it before the first GEMM that feeds it.
  * Formats: (e4m3, e4m3), (e5m2, e4m3), (e4m3, e5m2); e5m2 x e5m2 returns
  *   LM_ERR_UNSUPPORTED_FORMAT.
  * Requirements: K % 16 == 0, N % 8 == 0; A, B, D, aux 16-byte aligned.
@@ -204,6 +216,24 @@ LM_API lm_status lm_relu2_mlp_bwd_noalloc(const void* dY, const lm_mlp_saved* sa
 
 /* Size in bytes of the array lm_relu2_mlp_bwd_noalloc uses as its workspace. */
 LM_API size_t lm_relu2_mlp_bwd_noalloc_max_bytes(void);
+
+/*
+ * Gradient-accumulation forms of the MLP forward and backward (flags above).
+ * With flags == 0 they are lm_relu2_mlp_fwd / lm_relu2_mlp_bwd.
+ *  - LM_MLP_REUSE_WEIGHT_CASTS (fwd): skip the casts of W_up and W_down and
+ *    use the codes, transposes and scales `saved` holds from an earlier
+ *    forward of the same weights (once per optimizer step is enough).
+ *  - LM_MLP_ACCUMULATE_WGRAD (bwd): dW_up [f x d] and dW_down [d x f] are fp32;
+ *    each wgrad GEMM adds fp32(acc * s) into them (LM_EPI_ACCUM_F32); dX stays
+ *    bf16.  The caller zeroes the accumulators at the start of an optimizer step.
+ */
+LM_API lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_down,
+                                     int64_t M, int64_t d, int64_t f, void* Y, lm_mlp_saved* saved,
+                                     uint32_t flags, lm_stream_t stream);
+LM_API lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* saved, int64_t M,
+                                     int64_t d, int64_t f, void* dX, void* dW_up, void* dW_down,
+                                     void* workspace, size_t ws_bytes, uint32_t flags,
+                                     lm_stream_t stream);
 
 /* Synchronises `stream`, then returns and clears the current device's error
  * word: LM_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,

@@ -63,6 +63,9 @@ def lib():
         L.orc_gemm.argtypes = [P, ctypes.c_int, P, ctypes.c_int, i64, i64, i64, ctypes.c_float,
                                ctypes.c_float, ctypes.c_int, P, P, i64, P, P]
         L.orc_gemm.restype = None
+        L.orc_gemm_accum_f32.argtypes = [P, ctypes.c_int, P, ctypes.c_int, i64, i64, i64,
+                                         ctypes.c_float, ctypes.c_float, P, i64, P]
+        L.orc_gemm_accum_f32.restype = None
         L.orc_mlp_f64.argtypes = [P, P, P, P, i64, i64, i64, P, P, P, P]
         L.orc_mlp_f64.restype = None
         _lib = L
@@ -178,6 +181,23 @@ def gemm(A, fa, B, fb, inv_sa, inv_sb, epi=EPI_NONE, aux=None, rows=None):
     return D, am[0]
 
 
+def gemm_accum_f32(A, fa, B, fb, inv_sa, inv_sb, D, rows=None):
+    """In place: D (fp32, rows x N) += fp32(dec(A) dec(B)^T inv_sa inv_sb) for the
+    listed rows of A (all if None); D holds those rows in order."""
+    A = _c(A, np.uint8)
+    B = _c(B, np.uint8)
+    assert D.dtype == np.float32 and D.flags.c_contiguous
+    M, K = A.shape
+    N, K2 = B.shape
+    assert K == K2
+    r = None if rows is None else _c(np.asarray(rows, dtype=np.int64), np.int64)
+    nr = M if r is None else len(r)
+    assert D.shape == (nr, N)
+    lib().orc_gemm_accum_f32(_ptr(A), fa, _ptr(B), fb, M, N, K, float(np.float32(inv_sa)),
+                             float(np.float32(inv_sb)), _ptr(r), nr, _ptr(D))
+    return D
+
+
 # -------------------------------------------------------------- MLP chain
 def mlp_fwd(X, W_up, W_down):
     """relu^2 MLP forward with dynamic tensorwise FP8 scaling.
@@ -207,6 +227,34 @@ def mlp_bwd(dY, saved):
     dX, _ = gemm(cdh["q"], E5M2, cu["qT"], E4M3, cdh["inv_scale"], cu["inv_scale"])
     dW_up, _ = gemm(cdh["qT"], E5M2, cx["qT"], E4M3, cdh["inv_scale"], cx["inv_scale"])
     return dict(dX=dX, dW_up=dW_up, dW_down=dW_down, dY=cg, dH=dH, dh=cdh)
+
+
+def mlp_grad_accum(micro_batches, W_up, W_down):
+    """One optimizer step of gradient accumulation over micro-batches
+    [(X, dY), ...]: the weights are cast once (first micro-batch) and their
+    codes reused; each backward adds its weight gradients into fp32
+    accumulators.  Returns per-micro-batch (Y, dX) and the fp32 dW_up, dW_down."""
+    f, d = W_up.shape
+    dWu = np.zeros((f, d), np.float32)
+    dWd = np.zeros((d, f), np.float32)
+    outs = []
+    cu = amax_scale_cast(W_up, E4M3)
+    cd = amax_scale_cast(W_down, E4M3)
+    for X, dY in micro_batches:
+        cx = amax_scale_cast(X, E4M3)
+        H, amax_h = gemm(cx["q"], E4M3, cu["q"], E4M3, cx["inv_scale"], cu["inv_scale"],
+                         EPI_RELU2_FWD)
+        ch = amax_scale_cast(H, E4M3, relu2_input=True, amax_in=amax_h)
+        Y, _ = gemm(ch["q"], E4M3, cd["q"], E4M3, ch["inv_scale"], cd["inv_scale"])
+        cg = amax_scale_cast(dY, E5M2)
+        dH, amax_dh = gemm(cg["q"], E5M2, cd["qT"], E4M3, cg["inv_scale"], cd["inv_scale"],
+                           EPI_RELU2_BWD, aux=H)
+        gemm_accum_f32(cg["qT"], E5M2, ch["qT"], E4M3, cg["inv_scale"], ch["inv_scale"], dWd)
+        cdh = amax_scale_cast(dH, E5M2, amax_in=amax_dh)
+        dX, _ = gemm(cdh["q"], E5M2, cu["qT"], E4M3, cdh["inv_scale"], cu["inv_scale"])
+        gemm_accum_f32(cdh["qT"], E5M2, cx["qT"], E4M3, cdh["inv_scale"], cx["inv_scale"], dWu)
+        outs.append((Y, dX))
+    return outs, dWu, dWd
 
 
 def mlp_f64(X, W_up, W_down, dY=None):

@@ -273,6 +273,27 @@ void orc_gemm(const uint8_t* A, int fa, const uint8_t* B, int fb, int64_t M, int
     if (amax_out) *amax_out = orc_amax(D, nr, N, N, epi == ORC_EPI_RELU2_FWD);
 }
 
+/* Gradient accumulation into an fp32 buffer: for the listed rows (or all),
+ * D[i, n] = fp32(D[i, n] + fp32(C * inv_sa * inv_sb)): the scaled fp64 sum is
+ * rounded once to fp32, then added to the accumulator with one fp32 addition.
+ * (Micro-batches, grad_accum 7: decomputer.nl, "Appendix: De configuratie",
+ * total_batch_size; section "Vroege experimenten" item 2.) */
+void orc_gemm_accum_f32(const uint8_t* A, int fa, const uint8_t* B, int fb, int64_t M,
+                        int64_t N, int64_t K, float inv_sa, float inv_sb, const int64_t* rows,
+                        int64_t nrows, float* D) {
+    int64_t nr = rows ? nrows : M;
+    double* C = (double*)malloc(sizeof(double) * (size_t)(nr * N > 0 ? nr * N : 1));
+    orc_gemm_acc(A, fa, B, fb, M, N, K, rows, nrows, C);
+    const double s_a = (double)inv_sa, s_b = (double)inv_sb;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nr; ++i)
+        for (int64_t n = 0; n < N; ++n) {
+            float part = (float)(C[i * N + n] * s_a * s_b);
+            D[i * N + n] = D[i * N + n] + part; /* one fp32 add */
+        }
+    free(C);
+}
+
 /* ---------------------------------------------- unquantised fp64 MLP chain */
 
 /* Plain fp64 relu^2 MLP, no quantisation: the sanity reference that the FP8

@@ -69,3 +69,19 @@ def bf16_neighbours(bits):
     toward_big = np.where(neg, up_mag | 0x8000, up_mag)
     toward_small = np.where(dn_neg, dn_mag | 0x8000, dn_mag)
     return toward_small.astype(np.uint16), toward_big.astype(np.uint16)
+
+
+def assert_close_f32(got, ref, what=""):
+    """The same tolerance for fp32 results (numpy arrays)."""
+    g = np.asarray(got, np.float64)
+    r = np.asarray(ref, np.float64)
+    assert g.shape == r.shape, (what, g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    rms = float(np.sqrt(np.mean(r * r)))
+    d = np.abs(g - r)
+    bad = d > ELEM_REL * np.abs(r) + ELEM_RMS * rms
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} out of tolerance, "
+                           f"worst {d.max():.3e}, rms {rms:.3e}")
+    nr = np.linalg.norm(r)
+    if nr > 0:
+        assert np.linalg.norm(g - r) / nr <= NORM_REL, what

@@ -194,3 +194,49 @@ def test_fp8_chain_within_fp8_error_of_f64_chain(orc):
     assert fwd["h"]["amax"] == np.float32(
         torch.relu(torch.from_numpy(fwd["H"].view(np.int16)).view(torch.bfloat16).float())
         .pow(2).to(torch.bfloat16).float().max().item())
+
+
+def test_accumulating_gemm_adds_one_fp32_rounding_per_call(orc):
+    """Gradient accumulation: D += fp32(C * inv_sa * inv_sb), one fp32 addition
+    per call.  Pinned against exact products rounded by numpy's float32."""
+    rng = np.random.default_rng(29)
+    M, N, K = 7, 9, 48
+    A = finite_codes(E5M2, rng, (M, K))
+    B = finite_codes(E4M3, rng, (N, K))
+    inv_a, inv_b = np.float32(2.0 ** -10), np.float32(0.25)   # powers of two: exact in fp64
+    exact = tdecode(A, E5M2) @ tdecode(B, E4M3).T * float(inv_a) * float(inv_b)
+    D = np.zeros((M, N), np.float32)
+    orc.gemm_accum_f32(A, E5M2, B, E4M3, inv_a, inv_b, D)
+    assert np.array_equal(D, exact.astype(np.float32))       # 0 + x = x: one rounding
+    D0 = rng.standard_normal((M, N)).astype(np.float32)
+    D = D0.copy()
+    orc.gemm_accum_f32(A, E5M2, B, E4M3, inv_a, inv_b, D)
+    assert np.array_equal(D, D0 + exact.astype(np.float32))   # numpy float32 add
+    # a row subset touches only its own rows
+    rows = [6, 1]
+    Dr = D0[rows].copy()
+    orc.gemm_accum_f32(A, E5M2, B, E4M3, inv_a, inv_b, Dr, rows=rows)
+    assert np.array_equal(Dr, D0[rows] + exact[rows].astype(np.float32))
+
+
+def test_grad_accum_chain_matches_sum_of_per_micro_batch_gradients(orc):
+    """Accumulating two micro-batches equals the float32 sum of the two
+    single-micro-batch wgrads computed with the same (reused) weight casts."""
+    from fp8_gemms_b200 import synthetic
+    w = synthetic.MlpWorkload("ga", 64, 64, 256, True)
+    t = w.tensors()
+    b = {k: synthetic.bits_u16(v) for k, v in t.items()}
+    X2 = synthetic.bits_u16(synthetic.normal_bf16((64, 64), 1.0, 77, 0))
+    dY2 = synthetic.bits_u16(synthetic.normal_bf16((64, 64), 1e-3, 77, 1))
+    outs, dWu, dWd = orc.mlp_grad_accum([(b["X"], b["dY"]), (X2, dY2)], b["W_up"], b["W_down"])
+    singles = [orc.mlp_grad_accum([mb], b["W_up"], b["W_down"]) for mb in
+               [(b["X"], b["dY"]), (X2, dY2)]]
+    assert np.array_equal(dWu, singles[0][1] + singles[1][1])
+    assert np.array_equal(dWd, singles[0][2] + singles[1][2])
+    # and each micro-batch's Y and dX equal the plain chain's
+    fwd = orc.mlp_fwd(b["X"], b["W_up"], b["W_down"])
+    bwd = orc.mlp_bwd(b["dY"], fwd)
+    assert np.array_equal(outs[0][0], fwd["Y"]) and np.array_equal(outs[0][1], bwd["dX"])
+    # the fp32 accumulator of one micro-batch equals the bf16 chain's wgrad to bf16 rounding
+    dWu_bf = bf16_vals(bwd["dW_up"])
+    assert np.all(np.abs(singles[0][1] - dWu_bf) <= 2.0 ** -8 * np.abs(dWu_bf) + 1e-30)
