@@ -25,7 +25,8 @@ EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
             "lm_relu2_mlp_bwd", "lm_get_error", "lm_status_string", "lm_version",
             "lm_timing_attach", "lm_timing_detach", "lm_timing_kinds",
             "lm_relu2_mlp_bwd_noalloc", "lm_relu2_mlp_bwd_noalloc_max_bytes",
-            "lm_selftest_bounded_wait", "lm_relu2_mlp_fwd_ex", "lm_relu2_mlp_bwd_ex"]
+            "lm_selftest_bounded_wait", "lm_relu2_mlp_fwd_ex", "lm_relu2_mlp_bwd_ex",
+            "lm_rmsnorm_fp8_cast"]
 
 
 class LmError(RuntimeError):
@@ -83,6 +84,8 @@ def _load():
     L.lm_relu2_mlp_bwd_ex.argtypes = [P, ctypes.POINTER(MlpSaved), i64, i64, i64, P, P, P, P,
                                       ctypes.c_size_t, ctypes.c_uint32, P]
     L.lm_relu2_mlp_bwd_ex.restype = st
+    L.lm_rmsnorm_fp8_cast.argtypes = [P, P, i64, i64, ctypes.c_float, i32, P, P, P, P, P, P, P]
+    L.lm_rmsnorm_fp8_cast.restype = st
     L.lm_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
     L.lm_selftest_bounded_wait.restype = st
     return L
@@ -131,6 +134,15 @@ def lm_fp8_gemm(A, fa, B, fb, inv_scale_a, inv_scale_b, D, epi=EPI_NONE, aux=Non
     assert K == K2 and tuple(D.shape) == (M, N)
     _check(lib.lm_fp8_gemm(_p(A), fa, _p(B), fb, M, N, K, _p(inv_scale_a), _p(inv_scale_b), epi,
                            _p(aux), _p(D), _p(amax_out), _stream(stream)), "lm_fp8_gemm")
+
+
+def lm_rmsnorm_fp8_cast(R, weight, X, fmt, amax_out, scale_out, inv_scale_out, q=None, qT=None,
+                        eps=1e-6, stream=None):
+    rows, cols = R.shape
+    assert R.is_contiguous() and X.is_contiguous()
+    _check(lib.lm_rmsnorm_fp8_cast(_p(R), _p(weight), rows, cols, eps, fmt, _p(X), _p(amax_out),
+                                   _p(scale_out), _p(inv_scale_out), _p(q), _p(qT),
+                                   _stream(stream)), "lm_rmsnorm_fp8_cast")
 
 
 def lm_relu2_mlp_saved_bytes(M, d, f):

@@ -45,7 +45,7 @@ def time_it(fn, iters, warmup, flush):
 
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("op", choices=["gemm", "cast", "mlp-accum"])
+    p.add_argument("op", choices=["gemm", "cast", "mlp-accum", "rmsnorm-cast"])
     p.add_argument("--micro", type=int, default=7)
     p.add_argument("--d", type=int, default=3072)
     p.add_argument("--f", type=int, default=12288)
@@ -67,6 +67,20 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     if a.op == "mlp-accum":
         pass
+    elif a.op == "rmsnorm-cast":
+        R = torch.randn(a.rows, a.cols, device="cuda", generator=gen).to(torch.bfloat16)
+        w = torch.randn(a.cols, device="cuda", generator=gen).to(torch.bfloat16)
+        X = torch.empty_like(R)
+        q = torch.empty(a.rows, a.cols, dtype=torch.uint8, device="cuda")
+        qT = torch.empty(a.cols, a.rows, dtype=torch.uint8, device="cuda")
+        sc = torch.zeros(4, device="cuda")
+        fn = lambda: _lib.lm_rmsnorm_fp8_cast(R, w, X, FMT[a.fmt], sc[0:1], sc[1:2], sc[2:3], q, qT)
+        ms = time_it(fn, a.iters, a.warmup, flush)
+        n = a.rows * a.cols
+        avg = sum(ms) / len(ms)
+        # R read, X write, X read, q, qT: 8 bytes per element
+        out = dict(op="rmsnorm-cast", rows=a.rows, cols=a.cols, fmt=a.fmt, avg_ms=round(avg, 4),
+                   gbs=round(8 * n / avg / 1e6, 1), algorithmic_bytes=8 * n)
     elif a.op == "gemm":
         fa, fb, epi = FMT[a.fa], FMT[a.fb], EPI[a.epi]
         A = random_codes(fa, a.M, a.K, gen)

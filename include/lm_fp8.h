@@ -134,6 +134,27 @@ LM_API lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8_t* 
                       float* amax_out, lm_stream_t stream);
 
 /*
+ * The producer of a GEMM input: RMSNorm, then the dynamic FP8 cast of its
+ * output (the model's pre-norm; decomputer.nl, "Het trainen van een 3.8B
+ * LLM tot 0.384 CORE voor $998", "Appendix: De configuratie", rms_norm_eps
+ * 1e-6, PyTorch's F.rms_norm):
+ *
+ *   X[r][c] = bf16( R[r][c] / sqrt(mean_c R[r][c]^2 + eps) * weight[c] )
+ *   then amax / scale / q / qT of X exactly as lm_fp8_amax_scale_cast.
+ *
+ * The normalising pass also max-reduces |X|, so the cast needs no reduction
+ * pass of its own.  R: bf16 [rows x cols] (contiguous); weight: bf16 [cols] or
+ * NULL (no weight); X: bf16 [rows x cols] output; amax_out, scale_out,
+ * inv_scale_out, q, qT as in lm_fp8_amax_scale_cast.  The norm accumulates in
+ * fp32 (sum of squares, one IEEE sqrt and division).  Requirements as for
+ * the cast, plus R, weight, X 16-byte aligned and eps >= 0.
+ */
+LM_API lm_status lm_rmsnorm_fp8_cast(const void* R, const void* weight, int64_t rows,
+                                     int64_t cols, float eps, lm_fp8_format fmt, void* X,
+                                     float* amax_out, float* scale_out, float* inv_scale_out,
+                                     uint8_t* q, uint8_t* qT, lm_stream_t stream);
+
+/*
  * Tensors the relu^2 MLP forward saves for its backward.  Every pointer is a
  * caller-owned device buffer (see lm_relu2_mlp_saved_carve).  Shapes for
  * X [M x d], W_up [f x d], W_down [d x f]:
@@ -251,7 +272,7 @@ LM_API lm_status lm_get_error(lm_stream_t stream, uint32_t* where_out);
  * next recorded event therefore brackets launch i.  lm_timing_detach()
  * stops recording and returns the number of events recorded.
  * lm_timing_kinds() copies one character per recorded launch ('a' amax
- * reduction, 'c' cast, 's' scales only, 'g' GEMM) into out[0..cap) and
+ * reduction, 'c' cast, 's' scales only, 'g' GEMM, 'n' RMSNorm) into out[0..cap) and
  * returns how many it wrote.  State is per host thread.
  */
 LM_API void lm_timing_attach(void* const* events, int capacity);

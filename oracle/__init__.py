@@ -66,6 +66,8 @@ def lib():
         L.orc_gemm_accum_f32.argtypes = [P, ctypes.c_int, P, ctypes.c_int, i64, i64, i64,
                                          ctypes.c_float, ctypes.c_float, P, i64, P]
         L.orc_gemm_accum_f32.restype = None
+        L.orc_rmsnorm.argtypes = [P, P, i64, i64, ctypes.c_double, P]
+        L.orc_rmsnorm.restype = None
         L.orc_mlp_f64.argtypes = [P, P, P, P, i64, i64, i64, P, P, P, P]
         L.orc_mlp_f64.restype = None
         _lib = L
@@ -196,6 +198,26 @@ def gemm_accum_f32(A, fa, B, fb, inv_sa, inv_sb, D, rows=None):
     lib().orc_gemm_accum_f32(_ptr(A), fa, _ptr(B), fb, M, N, K, float(np.float32(inv_sa)),
                              float(np.float32(inv_sb)), _ptr(r), nr, _ptr(D))
     return D
+
+
+def rmsnorm(R, w=None, eps=1e-6):
+    """bf16 X = RMSNorm(R) * w, fp64 then one rounding (bits in, bits out)."""
+    R = _c(R, np.uint16)
+    rows, cols = R.shape
+    if w is not None:
+        w = _c(w, np.uint16)
+        assert w.shape == (cols,)
+    X = np.zeros((rows, cols), np.uint16)
+    lib().orc_rmsnorm(_ptr(R), _ptr(w), rows, cols, float(eps), _ptr(X))
+    return X
+
+
+def rmsnorm_fp8_cast(R, w=None, eps=1e-6, fmt=E4M3):
+    """The fused producer: X = RMSNorm(R) * w, then X's dynamic cast."""
+    X = rmsnorm(R, w, eps)
+    out = amax_scale_cast(X, fmt)
+    out["X"] = X
+    return out
 
 
 # -------------------------------------------------------------- MLP chain

@@ -294,6 +294,30 @@ void orc_gemm_accum_f32(const uint8_t* A, int fa, const uint8_t* B, int fb, int6
     free(C);
 }
 
+/* RMSNorm producer of the FP8 GEMM input: for each row,
+ *   X[r, c] = bf16( R[r, c] / sqrt(mean_c R[r, c]^2 + eps) * w[c] )
+ * in fp64, rounded once to bf16 (w == NULL means w = 1).  The model's norm is
+ * RMSNorm with rms_norm_eps 1e-6 computed by PyTorch's F.rms_norm
+ * (decomputer.nl, "Appendix: De configuratie"; section "Wat niet werkte",
+ * Liger RMSNorm bullet). */
+void orc_rmsnorm(const uint16_t* R, const uint16_t* w, int64_t rows, int64_t cols, double eps,
+                 uint16_t* X) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        double ss = 0.0;
+        for (int64_t c = 0; c < cols; ++c) {
+            double v = orc_bf16_to_double(R[r * cols + c]);
+            ss += v * v;
+        }
+        double inv = 1.0 / sqrt(ss / (double)cols + eps);
+        for (int64_t c = 0; c < cols; ++c) {
+            double v = orc_bf16_to_double(R[r * cols + c]) * inv;
+            if (w) v *= orc_bf16_to_double(w[c]);
+            X[r * cols + c] = orc_bf16_from_double(v);
+        }
+    }
+}
+
 /* ---------------------------------------------- unquantised fp64 MLP chain */
 
 /* Plain fp64 relu^2 MLP, no quantisation: the sanity reference that the FP8
