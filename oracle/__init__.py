@@ -68,6 +68,12 @@ def lib():
         L.orc_gemm_accum_f32.restype = None
         L.orc_rmsnorm.argtypes = [P, P, i64, i64, ctypes.c_double, P]
         L.orc_rmsnorm.restype = None
+        L.orc_swiglu_h.argtypes = [P, i64, i64, P]
+        L.orc_swiglu_h.restype = ctypes.c_float
+        L.orc_swiglu_bwd.argtypes = [P, P, i64, i64, P]
+        L.orc_swiglu_bwd.restype = ctypes.c_float
+        L.orc_swiglu_f64.argtypes = [P, P, P, P, P, i64, i64, i64, P, P, P, P, P]
+        L.orc_swiglu_f64.restype = None
         L.orc_mlp_f64.argtypes = [P, P, P, P, i64, i64, i64, P, P, P, P]
         L.orc_mlp_f64.restype = None
         _lib = L
@@ -293,4 +299,80 @@ def mlp_f64(X, W_up, W_down, dY=None):
         out.update(dX=np.zeros((M, d)), dW_up=np.zeros((f, d)), dW_down=np.zeros((d, f)))
     lib().orc_mlp_f64(_ptr(X), _ptr(W_up), _ptr(W_down), _ptr(dY), M, d, f, _ptr(Y),
                       _ptr(out.get("dX")), _ptr(out.get("dW_up")), _ptr(out.get("dW_down")))
+    return out
+
+
+# ------------------------------------------------ gated (SwiGLU) variant
+def interleave_gate_up(Wg, Wu):
+    """Rows of W_gate and W_up (each f x d) interleaved in blocks of 128:
+    [Wg[0:128]; Wu[0:128]; Wg[128:256]; Wu[128:256]; ...] (f % 128 == 0)."""
+    f, d = Wg.shape
+    assert f % 128 == 0 and Wu.shape == (f, d)
+    out = np.empty((2 * f, d), Wg.dtype)
+    for b in range(f // 128):
+        out[256 * b:256 * b + 128] = Wg[128 * b:128 * b + 128]
+        out[256 * b + 128:256 * b + 256] = Wu[128 * b:128 * b + 128]
+    return out
+
+
+def deinterleave_gate_up(Wgu):
+    f = Wgu.shape[0] // 2
+    Wg = np.concatenate([Wgu[256 * b:256 * b + 128] for b in range(f // 128)])
+    Wu = np.concatenate([Wgu[256 * b + 128:256 * b + 256] for b in range(f // 128)])
+    return Wg, Wu
+
+
+def swiglu_h(GU):
+    GU = _c(GU, np.uint16)
+    M, f2 = GU.shape
+    h = np.zeros((M, f2 // 2), np.uint16)
+    a = lib().orc_swiglu_h(_ptr(GU), M, f2 // 2, _ptr(h))
+    return h, np.float32(a)
+
+
+def swiglu_bwd(g, GU):
+    g = _c(g, np.uint16)
+    GU = _c(GU, np.uint16)
+    M, f = g.shape
+    dGU = np.zeros((M, 2 * f), np.uint16)
+    a = lib().orc_swiglu_bwd(_ptr(g), _ptr(GU), M, f, _ptr(dGU))
+    return dGU, np.float32(a)
+
+
+def swiglu_fwd(X, W_gu, W_down):
+    """Gated MLP forward in FP8: W_gu is the interleaved [2f x d] gate/up weight."""
+    cx = amax_scale_cast(X, E4M3)
+    cgu = amax_scale_cast(W_gu, E4M3)
+    cd = amax_scale_cast(W_down, E4M3)
+    GU, _ = gemm(cx["q"], E4M3, cgu["q"], E4M3, cx["inv_scale"], cgu["inv_scale"])
+    h, amax_h = swiglu_h(GU)
+    ch = amax_scale_cast(h, E4M3, amax_in=amax_h)
+    Y, _ = gemm(ch["q"], E4M3, cd["q"], E4M3, ch["inv_scale"], cd["inv_scale"])
+    return dict(Y=Y, X=cx, W_gu=cgu, W_down=cd, GU=GU, h_bf16=h, h=ch)
+
+
+def swiglu_bwd_chain(dY, saved):
+    cg = amax_scale_cast(dY, E5M2)
+    cx, cgu, cd, ch = saved["X"], saved["W_gu"], saved["W_down"], saved["h"]
+    g, _ = gemm(cg["q"], E5M2, cd["qT"], E4M3, cg["inv_scale"], cd["inv_scale"])
+    dW_down, _ = gemm(cg["qT"], E5M2, ch["qT"], E4M3, cg["inv_scale"], ch["inv_scale"])
+    dGU, amax_d = swiglu_bwd(g, saved["GU"])
+    cdg = amax_scale_cast(dGU, E5M2, amax_in=amax_d)
+    dX, _ = gemm(cdg["q"], E5M2, cgu["qT"], E4M3, cdg["inv_scale"], cgu["inv_scale"])
+    dW_gu, _ = gemm(cdg["qT"], E5M2, cx["qT"], E4M3, cdg["inv_scale"], cx["inv_scale"])
+    return dict(dX=dX, dW_gu=dW_gu, dW_down=dW_down, dY=cg, g=g, dGU=dGU, dgu=cdg)
+
+
+def swiglu_f64(X, Wg, Wu, Wd, dY=None):
+    X, Wg, Wu, Wd = (_c(a, np.float64) for a in (X, Wg, Wu, Wd))
+    M, d = X.shape
+    f = Wg.shape[0]
+    out = dict(Y=np.zeros((M, d)))
+    if dY is not None:
+        dY = _c(dY, np.float64)
+        out.update(dX=np.zeros((M, d)), dWg=np.zeros((f, d)), dWu=np.zeros((f, d)),
+                   dWd=np.zeros((d, f)))
+    lib().orc_swiglu_f64(_ptr(X), _ptr(Wg), _ptr(Wu), _ptr(Wd), _ptr(dY), M, d, f,
+                         _ptr(out["Y"]), _ptr(out.get("dX")), _ptr(out.get("dWg")),
+                         _ptr(out.get("dWu")), _ptr(out.get("dWd")))
     return out

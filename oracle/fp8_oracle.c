@@ -318,7 +318,125 @@ void orc_rmsnorm(const uint16_t* R, const uint16_t* w, int64_t rows, int64_t col
     }
 }
 
+/* ------------------------------------------ gated (SwiGLU) MLP variant */
+/* The comparison workload of the "Niet-gated MLPs" bullet (decomputer.nl,
+ * section "Doorvoer (Throughput) verhogen"): h = silu(G) * U with
+ * G = X W_gate^T, U = X W_up^T, silu(x) = x / (1 + exp(-x)).
+ * Layout used by the GEMM path: gate and up are interleaved in blocks of 128
+ * columns, GU[:, 256 b + j] = G[:, 128 b + j] and GU[:, 256 b + 128 + j] =
+ * U[:, 128 b + j] (j < 128); the same order holds for the interleaved weight
+ * rows and for dGU.  Readings: h and dG, dU are each rounded once to bf16
+ * from the exact (fp64) value of the product. */
+static double silu(double x) { return x / (1.0 + exp(-x)); }
+static double dsilu(double x) {
+    double sg = 1.0 / (1.0 + exp(-x));
+    return sg * (1.0 + x * (1.0 - sg));
+}
+
+/* h [M x f] from GU [M x 2f] (bf16 bits), amax of h returned. */
+float orc_swiglu_h(const uint16_t* GU, int64_t M, int64_t f, uint16_t* h) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t j = 0; j < f; ++j) {
+            int64_t b = j / 128, o = j % 128;
+            double g = orc_bf16_to_double(GU[m * 2 * f + 256 * b + o]);
+            double u = orc_bf16_to_double(GU[m * 2 * f + 256 * b + 128 + o]);
+            h[m * f + j] = orc_bf16_from_double(silu(g) * u);
+        }
+    return orc_amax(h, M, f, f, 0);
+}
+
+/* dGU [M x 2f] from g = dh [M x f] and GU: dG = g U silu'(G), dU = g silu(G). */
+float orc_swiglu_bwd(const uint16_t* g_, const uint16_t* GU, int64_t M, int64_t f,
+                     uint16_t* dGU) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t j = 0; j < f; ++j) {
+            int64_t b = j / 128, o = j % 128;
+            int64_t ig = m * 2 * f + 256 * b + o, iu = ig + 128;
+            double g = orc_bf16_to_double(g_[m * f + j]);
+            double G = orc_bf16_to_double(GU[ig]), U = orc_bf16_to_double(GU[iu]);
+            dGU[ig] = orc_bf16_from_double(g * U * dsilu(G));
+            dGU[iu] = orc_bf16_from_double(g * silu(G));
+        }
+    return orc_amax(dGU, M, 2 * f, 2 * f, 0);
+}
+
 /* ---------------------------------------------- unquantised fp64 MLP chain */
+
+/* Plain fp64 SwiGLU MLP, no quantisation (same role as orc_mlp_f64):
+ *   G = X Wg^T, U = X Wu^T, h = silu(G) U, Y = h Wd^T
+ *   dh = dY Wd, dG = dh U silu'(G), dU = dh silu(G)
+ *   dX = dG Wg + dU Wu, dWg = dG^T X, dWu = dU^T X, dWd = dY^T h
+ * Wg, Wu: f x d; Wd: d x f.  Output pointers may be NULL. */
+void orc_swiglu_f64(const double* X, const double* Wg, const double* Wu, const double* Wd,
+                    const double* dY, int64_t M, int64_t d, int64_t f, double* Y, double* dX,
+                    double* dWg, double* dWu, double* dWd) {
+    size_t Mf = (size_t)(M * f > 0 ? M * f : 1);
+    double* G = (double*)calloc(Mf, sizeof(double));
+    double* U = (double*)calloc(Mf, sizeof(double));
+    double* h = (double*)calloc(Mf, sizeof(double));
+    double* dG = (double*)calloc(Mf, sizeof(double));
+    double* dU = (double*)calloc(Mf, sizeof(double));
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t j = 0; j < f; ++j) {
+            double a = 0.0, b = 0.0;
+            for (int64_t k = 0; k < d; ++k) {
+                a += X[m * d + k] * Wg[j * d + k];
+                b += X[m * d + k] * Wu[j * d + k];
+            }
+            G[m * f + j] = a;
+            U[m * f + j] = b;
+            h[m * f + j] = silu(a) * b;
+        }
+    if (Y)
+        for (int64_t m = 0; m < M; ++m)
+            for (int64_t i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < f; ++j) acc += h[m * f + j] * Wd[i * f + j];
+                Y[m * d + i] = acc;
+            }
+    if (dY) {
+        for (int64_t m = 0; m < M; ++m)
+            for (int64_t j = 0; j < f; ++j) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < d; ++i) acc += dY[m * d + i] * Wd[i * f + j];
+                dG[m * f + j] = acc * U[m * f + j] * dsilu(G[m * f + j]);
+                dU[m * f + j] = acc * silu(G[m * f + j]);
+            }
+        if (dX)
+            for (int64_t m = 0; m < M; ++m)
+                for (int64_t k = 0; k < d; ++k) {
+                    double acc = 0.0;
+                    for (int64_t j = 0; j < f; ++j)
+                        acc += dG[m * f + j] * Wg[j * d + k] + dU[m * f + j] * Wu[j * d + k];
+                    dX[m * d + k] = acc;
+                }
+        if (dWg || dWu)
+            for (int64_t j = 0; j < f; ++j)
+                for (int64_t k = 0; k < d; ++k) {
+                    double a = 0.0, b = 0.0;
+                    for (int64_t m = 0; m < M; ++m) {
+                        a += dG[m * f + j] * X[m * d + k];
+                        b += dU[m * f + j] * X[m * d + k];
+                    }
+                    if (dWg) dWg[j * d + k] = a;
+                    if (dWu) dWu[j * d + k] = b;
+                }
+        if (dWd)
+            for (int64_t i = 0; i < d; ++i)
+                for (int64_t j = 0; j < f; ++j) {
+                    double acc = 0.0;
+                    for (int64_t m = 0; m < M; ++m) acc += dY[m * d + i] * h[m * f + j];
+                    dWd[i * f + j] = acc;
+                }
+    }
+    free(G);
+    free(U);
+    free(h);
+    free(dG);
+    free(dU);
+}
 
 /* Plain fp64 relu^2 MLP, no quantisation: the sanity reference that the FP8
  * chain must approach within FP8 error, and whose backward is pinned by
