@@ -26,7 +26,8 @@ EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
             "lm_timing_attach", "lm_timing_detach", "lm_timing_kinds",
             "lm_relu2_mlp_bwd_noalloc", "lm_relu2_mlp_bwd_noalloc_max_bytes",
             "lm_selftest_bounded_wait", "lm_relu2_mlp_fwd_ex", "lm_relu2_mlp_bwd_ex",
-            "lm_rmsnorm_fp8_cast"]
+            "lm_rmsnorm_fp8_cast", "lm_swiglu_mlp_saved_bytes", "lm_swiglu_mlp_saved_carve",
+            "lm_swiglu_mlp_workspace_size", "lm_swiglu_mlp_fwd", "lm_swiglu_mlp_bwd"]
 
 
 class LmError(RuntimeError):
@@ -39,6 +40,12 @@ class MlpSaved(ctypes.Structure):
     """Mirror of lm_mlp_saved."""
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("Xq", "XqT", "Wuq", "WuqT", "Wdq", "WdqT", "H", "hq", "hqT", "scales")]
+
+
+class SwigluSaved(ctypes.Structure):
+    """Mirror of lm_swiglu_saved."""
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("Xq", "XqT", "Wguq", "WguqT", "Wdq", "WdqT", "GU", "h", "hq", "hqT", "scales")]
 
 
 def _load():
@@ -86,6 +93,18 @@ def _load():
     L.lm_relu2_mlp_bwd_ex.restype = st
     L.lm_rmsnorm_fp8_cast.argtypes = [P, P, i64, i64, ctypes.c_float, i32, P, P, P, P, P, P, P]
     L.lm_rmsnorm_fp8_cast.restype = st
+    L.lm_swiglu_mlp_saved_bytes.argtypes = [i64, i64, i64]
+    L.lm_swiglu_mlp_saved_bytes.restype = ctypes.c_size_t
+    L.lm_swiglu_mlp_saved_carve.argtypes = [P, ctypes.c_size_t, i64, i64, i64,
+                                            ctypes.POINTER(SwigluSaved)]
+    L.lm_swiglu_mlp_saved_carve.restype = st
+    L.lm_swiglu_mlp_workspace_size.argtypes = [i64, i64, i64]
+    L.lm_swiglu_mlp_workspace_size.restype = ctypes.c_size_t
+    L.lm_swiglu_mlp_fwd.argtypes = [P, P, P, i64, i64, i64, P, ctypes.POINTER(SwigluSaved), P]
+    L.lm_swiglu_mlp_fwd.restype = st
+    L.lm_swiglu_mlp_bwd.argtypes = [P, ctypes.POINTER(SwigluSaved), i64, i64, i64, P, P, P, P,
+                                    ctypes.c_size_t, P]
+    L.lm_swiglu_mlp_bwd.restype = st
     L.lm_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
     L.lm_selftest_bounded_wait.restype = st
     return L
@@ -202,6 +221,29 @@ def lm_relu2_mlp_bwd_noalloc(dY, saved, dX, dW_up, dW_down, stream=None):
     _check(lib.lm_relu2_mlp_bwd_noalloc(_p(dY), ctypes.byref(saved), M, d, f, _p(dX), _p(dW_up),
                                         _p(dW_down), _stream(stream)),
            "lm_relu2_mlp_bwd_noalloc")
+
+
+def lm_swiglu_mlp_saved_carve(buf, M, d, f):
+    s = SwigluSaved()
+    _check(lib.lm_swiglu_mlp_saved_carve(_p(buf), buf.numel() * buf.element_size(), M, d, f,
+                                         ctypes.byref(s)), "lm_swiglu_mlp_saved_carve")
+    return s
+
+
+def lm_swiglu_mlp_fwd(X, W_gu, W_down, Y, saved, stream=None):
+    M, d = X.shape
+    f = W_gu.shape[0] // 2
+    _check(lib.lm_swiglu_mlp_fwd(_p(X), _p(W_gu), _p(W_down), M, d, f, _p(Y),
+                                 ctypes.byref(saved), _stream(stream)), "lm_swiglu_mlp_fwd")
+
+
+def lm_swiglu_mlp_bwd(dY, saved, dX, dW_gu, dW_down, workspace, stream=None):
+    M, d = dY.shape
+    f = dW_gu.shape[0] // 2
+    _check(lib.lm_swiglu_mlp_bwd(_p(dY), ctypes.byref(saved), M, d, f, _p(dX), _p(dW_gu),
+                                 _p(dW_down), _p(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "lm_swiglu_mlp_bwd")
 
 
 def lm_get_error(stream=None):

@@ -131,6 +131,66 @@ class Relu2Mlp:
         raise KeyError(name)
 
 
+def interleave_gate_up(W_gate, W_up):
+    """[2f x d] weight whose rows alternate 128-row blocks of W_gate and W_up
+    (the layout the gated MLP's single up GEMM reads)."""
+    f, d = W_gate.shape
+    assert f % 128 == 0 and W_up.shape == (f, d)
+    return torch.stack([W_gate.view(f // 128, 128, d), W_up.view(f // 128, 128, d)],
+                       dim=1).reshape(2 * f, d)
+
+
+def deinterleave_gate_up(W_gu):
+    f2, d = W_gu.shape
+    v = W_gu.view(f2 // 256, 2, 128, d)
+    return v[:, 0].reshape(f2 // 2, d), v[:, 1].reshape(f2 // 2, d)
+
+
+class SwigluMlp:
+    """Buffers of one gated (SwiGLU) MLP block (M, d, f) over the C ABI."""
+
+    def __init__(self, M, d, f, device="cuda"):
+        self.M, self.d, self.f = M, d, f
+        nbytes = _lib.lib.lm_swiglu_mlp_saved_bytes(M, d, f)
+        if nbytes == 0:
+            raise LmError(3, "lm_swiglu_mlp_saved_bytes")
+        self.saved_buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.saved = _lib.lm_swiglu_mlp_saved_carve(self.saved_buf, M, d, f)
+        self.workspace = torch.empty(_lib.lib.lm_swiglu_mlp_workspace_size(M, d, f),
+                                     dtype=torch.uint8, device=device)
+        self.device = device
+
+    def forward(self, X, W_gu, W_down, Y=None, stream=None):
+        Y = Y if Y is not None else torch.empty(self.M, self.d, dtype=torch.bfloat16,
+                                                device=self.device)
+        _lib.lm_swiglu_mlp_fwd(X, W_gu, W_down, Y, self.saved, stream=stream)
+        return Y
+
+    def backward(self, dY, dX=None, dW_gu=None, dW_down=None, stream=None):
+        dev, M, d, f = self.device, self.M, self.d, self.f
+        dX = dX if dX is not None else torch.empty(M, d, dtype=torch.bfloat16, device=dev)
+        dW_gu = dW_gu if dW_gu is not None else torch.empty(2 * f, d, dtype=torch.bfloat16,
+                                                            device=dev)
+        dW_down = dW_down if dW_down is not None else torch.empty(d, f, dtype=torch.bfloat16,
+                                                                  device=dev)
+        _lib.lm_swiglu_mlp_bwd(dY, self.saved, dX, dW_gu, dW_down, self.workspace, stream=stream)
+        return dX, dW_gu, dW_down
+
+    def view(self, name):
+        """Saved tensors: Xq, Wguq, GU, h, hq, hqT, scales (library layout)."""
+        M, d, f = self.M, self.d, self.f
+        base = self.saved_buf.data_ptr()
+        off = getattr(self.saved, name) - base
+        if name in ("GU", "h"):
+            cols = 2 * f if name == "GU" else f
+            return self.saved_buf[off:off + M * cols * 2].view(torch.bfloat16).view(M, cols)
+        if name == "scales":
+            return self.saved_buf[off:off + 64].view(torch.float32).view(4, 4)
+        shape = {"Xq": (M, d), "XqT": (d, M), "Wguq": (2 * f, d), "WguqT": (d, 2 * f),
+                 "Wdq": (d, f), "WdqT": (f, d), "hq": (M, f), "hqT": (f, M)}[name]
+        return self.saved_buf[off:off + shape[0] * shape[1]].view(*shape)
+
+
 def linear_fwd_bwd(X, W, dY, stream=None):
     """Plain linear Y = X W^T with its dgrad and wgrad, all in FP8: X, W cast
     to e4m3 and dY to e5m2 (each with its K-major transposed copy), then

@@ -49,6 +49,7 @@ struct GemmArgs {
     const float* inv_b;
     const uint16_t* aux;
     void* D;
+    void* D2;
     float* amax_out;
     unsigned int* err;
     uint32_t idesc;
@@ -133,6 +134,33 @@ __device__ __forceinline__ uint32_t epi_pair(uint32_t acc0, uint32_t acc1, float
     return w;
 }
 
+// silu(x) = x / (1 + exp(-x)) in fp32 (expf, one IEEE division)
+__device__ __forceinline__ float silu_f32(float x) {
+    return __fdiv_rn(x, __fadd_rn(1.0f, expf(-x)));
+}
+
+// Stage one 32 x 32 bf16 box (this lane's row: 16 packed words) in a ring of
+// four 2 KB boxes at `ring` (64B-swizzled, as the tensor map expects) and
+// TMA-store it at (x, y).  The box reused is the one stored four stores ago.
+__device__ __forceinline__ void stage_box_store(uint8_t* ring, uint32_t& n_stores,
+                                                const uint32_t (&w)[16], const CUtensorMap* map,
+                                                int x, int y, uint64_t policy, int lane) {
+    uint8_t* dst = ring + (n_stores & 3u) * 2048;
+    if (lane == 0) bulk_wait_group_read<3>();
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(dst + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+            make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d_hint(map, smem_addr(dst), x, y, policy);
+        bulk_commit_group();
+    }
+    ++n_stores;
+}
+
 // =====================================================================
 // CTA-pair kernel: 256 x 256 tiles, cta_group::2
 // =====================================================================
@@ -166,7 +194,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_fp8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmD,
-                         const __grid_constant__ CUtensorMap tmAux, const GemmArgs args) {
+                         const __grid_constant__ CUtensorMap tmAux,
+                         const __grid_constant__ CUtensorMap tmD2, const GemmArgs args) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -206,6 +235,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmD);
         if (EPI == LM_EPI_RELU2_BWD) tma_prefetch_desc(&tmAux);
+        if (EPI == kEpiSwigluFwd) tma_prefetch_desc(&tmD2);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -344,6 +374,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const uint32_t tbase =
                 tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * TILE_N);
+            if (EPI == kEpiSwigluFwd) {
+                // gate columns [0,128) and up columns [128,256) of the tile: store
+                // G, U (bf16, interleaved as computed) and h = bf16(silu(G) U)
+                for (int c = 0; c < TILE_N / 2 / EPI_COLS; ++c) {
+                    uint32_t rg[32], ru[32];
+                    tmem_ld_32x32b_x32(tbase + (uint32_t)(c * EPI_COLS), rg);
+                    tmem_ld_32x32b_x32(tbase + (uint32_t)(TILE_N / 2 + c * EPI_COLS), ru);
+                    tmem_ld_wait();
+                    uint32_t pg[16], pu[16], ph[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const __nv_bfloat162 g2 =
+                            __floats2bfloat162_rn(__fmul_rn(__uint_as_float(rg[2 * i]), s),
+                                                  __fmul_rn(__uint_as_float(rg[2 * i + 1]), s));
+                        const __nv_bfloat162 u2 =
+                            __floats2bfloat162_rn(__fmul_rn(__uint_as_float(ru[2 * i]), s),
+                                                  __fmul_rn(__uint_as_float(ru[2 * i + 1]), s));
+                        const float2 gf = __bfloat1622float2(g2), uf = __bfloat1622float2(u2);
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(
+                            __fmul_rn(silu_f32(gf.x), uf.x), __fmul_rn(silu_f32(gf.y), uf.y));
+                        pg[i] = *reinterpret_cast<const uint32_t*>(&g2);
+                        pu[i] = *reinterpret_cast<const uint32_t*>(&u2);
+                        ph[i] = *reinterpret_cast<const uint32_t*>(&h2);
+                        amax2 = __vmaxu2(amax2, ph[i] & 0x7FFF7FFFu);
+                    }
+                    const int hcol = nb * (TILE_N / 2) + c * EPI_COLS;
+                    stage_box_store(sStore + wi * 2 * ACC_BOX_BYTES, n_stores, pg, &tmD,
+                                    gcol + c * EPI_COLS, grow, stream_policy, lane);
+                    stage_box_store(sStore + wi * 2 * ACC_BOX_BYTES, n_stores, pu, &tmD,
+                                    gcol + TILE_N / 2 + c * EPI_COLS, grow, stream_policy, lane);
+                    stage_box_store(sStore + wi * 2 * ACC_BOX_BYTES, n_stores, ph, &tmD2, hcol, grow,
+                                    stream_policy, lane);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(tempty_leader + (uint32_t)(acc * 8));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+                continue;
+            }
             for (int c = 0; c < n_chunks; ++c) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tbase + (uint32_t)(c * EPI_COLS), r);
@@ -657,7 +727,8 @@ bool ensure_smem(F* kernel, int bytes, bool (&done)[64]) {
 
 template <int EPI>
 lm_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
-                      const CUtensorMap& tx, const GemmArgs& a, cudaStream_t s) {
+                      const CUtensorMap& tx, const CUtensorMap& td2, const GemmArgs& a,
+                      cudaStream_t s) {
     static bool done[64] = {};
     if (!ensure_smem(pair::gemm_fp8_pair_kernel<EPI>, pair::SMEM_BYTES, done)) return LM_ERR_CUDA;
     const int sms = sm_count();
@@ -665,7 +736,7 @@ lm_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
     const int clusters = a.num_tiles < sms / 2 ? a.num_tiles : sms / 2;
     timing_mark(s, 'g');
     pair::gemm_fp8_pair_kernel<EPI><<<2 * clusters, NUM_THREADS, pair::SMEM_BYTES, s>>>(ta, tb, td,
-                                                                                      tx, a);
+                                                                                      tx, td2, a);
     return launch_status();
 }
 
@@ -685,27 +756,28 @@ lm_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArg
 }  // namespace
 }  // namespace lm
 
-extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
-                                 lm_fp8_format fb, int64_t M, int64_t N, int64_t K,
-                                 const float* inv_scale_a, const float* inv_scale_b,
-                                 lm_epilogue epi, const void* aux, void* D, float* amax_out,
-                                 lm_stream_t stream) {
+lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
+                            lm_fp8_format fb, int64_t M, int64_t N, int64_t K,
+                            const float* inv_scale_a, const float* inv_scale_b, int epi,
+                            const void* aux, void* D, void* D2, float* amax_out,
+                            lm_stream_t stream) {
     using namespace lm;
     if ((fa != LM_FP8_E4M3 && fa != LM_FP8_E5M2) || (fb != LM_FP8_E4M3 && fb != LM_FP8_E5M2))
         return LM_ERR_UNSUPPORTED_FORMAT;
     if (fa == LM_FP8_E5M2 && fb == LM_FP8_E5M2) return LM_ERR_UNSUPPORTED_FORMAT;
     if (epi != LM_EPI_NONE && epi != LM_EPI_RELU2_FWD && epi != LM_EPI_RELU2_BWD &&
-        epi != LM_EPI_ACCUM_F32)
+        epi != LM_EPI_ACCUM_F32 && epi != kEpiSwigluFwd)
         return LM_ERR_UNSUPPORTED_FORMAT;
     if (M < 0 || N < 0 || K < 0) return LM_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return LM_OK;
     if (!D || !inv_scale_a || !inv_scale_b) return LM_ERR_INVALID_ARG;
     if (K > 0 && (!A || !B)) return LM_ERR_INVALID_ARG;
     if (epi == LM_EPI_RELU2_BWD && !aux) return LM_ERR_INVALID_ARG;
+    if (epi == kEpiSwigluFwd && (!D2 || N % 256 != 0 || K == 0)) return LM_ERR_INVALID_ARG;
     if (K % 16 != 0 || N % 8 != 0) return LM_ERR_UNSUPPORTED_SHAPE;
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
         return LM_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(aux))
+    if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(aux) || !aligned16(D2))
         return LM_ERR_ALIGNMENT;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -726,12 +798,13 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
     a.inv_b = inv_scale_b;
     a.aux = static_cast<const uint16_t*>(aux);
     a.D = D;
+    a.D2 = D2;
     if (epi == LM_EPI_ACCUM_F32) a.amax_out = nullptr;
     a.amax_out = amax_out;
     a.err = err;
 
     CUtensorMap ta, tb;
-    if (M > 128) {
+    if (M > 128 || epi == kEpiSwigluFwd) {
         a.num_mb = (int)((M + pair::TILE_M - 1) / pair::TILE_M);
         a.num_nb = (int)((N + pair::TILE_N - 1) / pair::TILE_N);
         a.num_tiles = a.num_mb * a.num_nb;
@@ -759,11 +832,19 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
         } else {
             tx = td;  // unused
         }
+        CUtensorMap td2 = td;  // unused unless the gated epilogue writes h
+        if (epi == kEpiSwigluFwd &&
+            !encode_tmap_bf16_sw64(&td2, D2, (uint64_t)M, (uint64_t)(N / 2), 32, pair::EPI_COLS))
+            return LM_ERR_CUDA;
         switch (epi) {
-            case LM_EPI_NONE: return launch_pair<LM_EPI_NONE>(ta, tb, td, tx, a, s);
-            case LM_EPI_RELU2_FWD: return launch_pair<LM_EPI_RELU2_FWD>(ta, tb, td, tx, a, s);
-            case LM_EPI_RELU2_BWD: return launch_pair<LM_EPI_RELU2_BWD>(ta, tb, td, tx, a, s);
-            default: return launch_pair<LM_EPI_ACCUM_F32>(ta, tb, td, tx, a, s);
+            case LM_EPI_NONE: return launch_pair<LM_EPI_NONE>(ta, tb, td, tx, td2, a, s);
+            case LM_EPI_RELU2_FWD:
+                return launch_pair<LM_EPI_RELU2_FWD>(ta, tb, td, tx, td2, a, s);
+            case LM_EPI_RELU2_BWD:
+                return launch_pair<LM_EPI_RELU2_BWD>(ta, tb, td, tx, td2, a, s);
+            case LM_EPI_ACCUM_F32:
+                return launch_pair<LM_EPI_ACCUM_F32>(ta, tb, td, tx, td2, a, s);
+            default: return launch_pair<kEpiSwigluFwd>(ta, tb, td, tx, td2, a, s);
         }
     }
     a.num_mb = (int)((M + one::BM - 1) / one::BM);
@@ -781,4 +862,16 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
         case LM_EPI_RELU2_BWD: return launch_one<LM_EPI_RELU2_BWD>(ta, tb, a, s);
         default: return launch_one<LM_EPI_ACCUM_F32>(ta, tb, a, s);
     }
+}
+
+extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
+                                 lm_fp8_format fb, int64_t M, int64_t N, int64_t K,
+                                 const float* inv_scale_a, const float* inv_scale_b,
+                                 lm_epilogue epi, const void* aux, void* D, float* amax_out,
+                                 lm_stream_t stream) {
+    if (epi != LM_EPI_NONE && epi != LM_EPI_RELU2_FWD && epi != LM_EPI_RELU2_BWD &&
+        epi != LM_EPI_ACCUM_F32)
+        return LM_ERR_UNSUPPORTED_FORMAT;
+    return lm::gemm_dispatch(A, fa, B, fb, M, N, K, inv_scale_a, inv_scale_b, (int)epi, aux, D,
+                             nullptr, amax_out, stream);
 }

@@ -40,6 +40,18 @@ bool encode_tmap_f32_sw128(CUtensorMap* map, const void* base, uint64_t rows, ui
 bool encode_tmap_bf16_plain(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                             uint64_t pitch, uint32_t box_rows, uint32_t box_cols);
 
+// Epilogue used only inside the library (the gated MLP's up GEMM): D is the
+// interleaved G|U pre-activation (plain bf16 epilogue on a GEMM whose N is
+// 2f, gate and up alternating in 128-column blocks) and D2 receives
+// h = bf16(silu(G) U) [M x N/2]; amax_out gets max |h|.
+constexpr int kEpiSwigluFwd = 4;
+
+// lm_fp8_gemm with the internal epilogues and a second output.
+lm_status gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B, lm_fp8_format fb,
+                        int64_t M, int64_t N, int64_t K, const float* inv_scale_a,
+                        const float* inv_scale_b, int epi, const void* aux, void* D, void* D2,
+                        float* amax_out, lm_stream_t stream);
+
 // If the calling thread attached timing events, record the next one on `s`
 // (call right before a kernel launch); `kind` labels the launch.
 void timing_mark(cudaStream_t s, char kind);

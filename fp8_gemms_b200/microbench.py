@@ -4,6 +4,9 @@ iterations).  Also the small, self-contained command to run under ncu.
     python -m fp8_gemms_b200.microbench gemm --M 16384 --N 12288 --K 3072 --epi relu2_fwd
     python -m fp8_gemms_b200.microbench cast --rows 16384 --cols 3072 --fmt e4m3
     python -m fp8_gemms_b200.microbench cast --rows 16384 --cols 12288 --relu2 --amax-in
+    python -m fp8_gemms_b200.microbench mlp-compare --M 16384
+        (the non-gated relu^2 block, f = 4d, against the gated SwiGLU block,
+        f = 2.75d, both fwd + bwd in FP8: ms per step and tokens per second)
     python -m fp8_gemms_b200.microbench mlp-accum --M 16384 --micro 7
         (one optimizer step of gradient accumulation: the weights are cast by the
         first micro-batch's forward and reused by the others; every backward adds
@@ -45,7 +48,7 @@ def time_it(fn, iters, warmup, flush):
 
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("op", choices=["gemm", "cast", "mlp-accum", "rmsnorm-cast"])
+    p.add_argument("op", choices=["gemm", "cast", "mlp-accum", "rmsnorm-cast", "mlp-compare"])
     p.add_argument("--micro", type=int, default=7)
     p.add_argument("--d", type=int, default=3072)
     p.add_argument("--f", type=int, default=12288)
@@ -67,6 +70,31 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     if a.op == "mlp-accum":
         pass
+    elif a.op == "mlp-compare":
+        from . import api
+        M, d = a.M, a.d
+        res = {}
+        for name, f in (("relu2", 4 * d), ("swiglu", (11 * d) // 4)):
+            mk = lambda *sh, s=1.0: (torch.randn(*sh, device="cuda", generator=gen) * s).to(
+                torch.bfloat16)
+            X, dY = mk(M, d), mk(M, d, s=1e-3)
+            Wd = mk(d, f, s=0.02)
+            if name == "relu2":
+                mlp, W1 = api.Relu2Mlp(M, d, f), mk(f, d, s=0.02)
+                flops = 6 * 2 * M * d * f
+            else:
+                mlp, W1 = api.SwigluMlp(M, d, f), mk(2 * f, d, s=0.02)
+                flops = 9 * 2 * M * d * f
+            step = lambda: (mlp.forward(X, W1, Wd), mlp.backward(dY))
+            ms = time_it(step, a.iters, a.warmup, flush)
+            avg = sum(ms) / len(ms)
+            res[name] = dict(f=f, ms_per_step=round(avg, 4),
+                             tokens_per_s=round(M / avg * 1e3), tflops=round(flops / avg / 1e9, 1))
+            del mlp
+            torch.cuda.empty_cache()
+        out = dict(op="mlp-compare", M=M, d=d, **res,
+                   relu2_over_swiglu_tokens=round(res["relu2"]["tokens_per_s"] /
+                                                  res["swiglu"]["tokens_per_s"], 4))
     elif a.op == "rmsnorm-cast":
         R = torch.randn(a.rows, a.cols, device="cuda", generator=gen).to(torch.bfloat16)
         w = torch.randn(a.cols, device="cuda", generator=gen).to(torch.bfloat16)
@@ -116,7 +144,7 @@ def main():
                    amax_in=a.amax_in, avg_ms=round(avg, 4), min_ms=round(min(ms), 4),
                    gbs=round(byts / avg / 1e6, 1), algorithmic_bytes=byts)
     if a.op == "mlp-accum":
-        from . import api
+        from . import api  # noqa: F811
         M, d, f = a.M, a.d, a.f
         mlp = api.Relu2Mlp(M, d, f)
         Wu = (torch.randn(f, d, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)

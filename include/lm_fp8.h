@@ -256,6 +256,44 @@ LM_API lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* saved, 
                                      void* workspace, size_t ws_bytes, uint32_t flags,
                                      lm_stream_t stream);
 
+/*
+ * Gated (SwiGLU) MLP, the comparison workload of the non-gated relu^2 MLP
+ * (decomputer.nl, "Het trainen van een 3.8B LLM tot 0.384 CORE voor $998",
+ * section "Doorvoer (Throughput) verhogen", bullet "Niet-gated MLPs": three
+ * matmuls instead of two; intermediate ratio 2.75).  Same FP8 tensorwise
+ * scaling, e4m3 activations and weights, e5m2 gradients.
+ *
+ *   G = X W_gate^T, U = X W_up^T, h = bf16(silu(G) U), Y = h W_down^T
+ *   backward: g = dY W_down; dG = bf16(g U silu'(G)); dU = bf16(g silu(G));
+ *   dX = dG W_gate + dU W_up; dW_gate = dG^T X; dW_up = dU^T X; dW_down = dY^T h
+ *
+ * Layout: W_gu is [2f x d] with the rows of W_gate and W_up interleaved in
+ * blocks of 128 (rows 256b..256b+127 = W_gate rows 128b.., the next 128 =
+ * W_up rows 128b..); dW_gu comes back in the same order.  f % 128 == 0,
+ * d % 16 == 0, M % 16 == 0.  Buffers, workspace and errors as for the relu^2
+ * MLP; the saved GU holds G and U in the same interleaved column order.
+ */
+typedef struct lm_swiglu_saved {
+    uint8_t *Xq, *XqT;     /* [M x d], [d x M] e4m3 */
+    uint8_t *Wguq, *WguqT; /* [2f x d], [d x 2f] e4m3, interleaved gate/up */
+    uint8_t *Wdq, *WdqT;   /* [d x f], [f x d] e4m3 */
+    void* GU;              /* [M x 2f] bf16 pre-activations, interleaved */
+    void* h;               /* [M x f] bf16 silu(G) U */
+    uint8_t *hq, *hqT;     /* [M x f], [f x M] e4m3 */
+    float* scales;         /* 16 floats: {amax, scale, inv_scale, 0} for X, W_gu, W_down, h */
+} lm_swiglu_saved;
+
+LM_API size_t lm_swiglu_mlp_saved_bytes(int64_t M, int64_t d, int64_t f);
+LM_API lm_status lm_swiglu_mlp_saved_carve(void* base, size_t bytes, int64_t M, int64_t d,
+                                           int64_t f, lm_swiglu_saved* out);
+LM_API size_t lm_swiglu_mlp_workspace_size(int64_t M, int64_t d, int64_t f);
+LM_API lm_status lm_swiglu_mlp_fwd(const void* X, const void* W_gu, const void* W_down,
+                                   int64_t M, int64_t d, int64_t f, void* Y, lm_swiglu_saved* saved,
+                                   lm_stream_t stream);
+LM_API lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* saved, int64_t M,
+                                   int64_t d, int64_t f, void* dX, void* dW_gu, void* dW_down,
+                                   void* workspace, size_t ws_bytes, lm_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the current device's error
  * word: LM_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
  * LM_ERR_CUDA if the synchronisation itself failed, else LM_OK.  If
@@ -272,7 +310,8 @@ LM_API lm_status lm_get_error(lm_stream_t stream, uint32_t* where_out);
  * next recorded event therefore brackets launch i.  lm_timing_detach()
  * stops recording and returns the number of events recorded.
  * lm_timing_kinds() copies one character per recorded launch ('a' amax
- * reduction, 'c' cast, 's' scales only, 'g' GEMM, 'n' RMSNorm) into out[0..cap) and
+ * reduction, 'c' cast, 's' scales only, 'g' GEMM, 'n' RMSNorm, 'w'
+ * SwiGLU backward elementwise) into out[0..cap) and
  * returns how many it wrote.  State is per host thread.
  */
 LM_API void lm_timing_attach(void* const* events, int capacity);

@@ -1,0 +1,99 @@
+"""GPU parity of the gated (SwiGLU) MLP comparison workload against the
+oracle: end to end on a small block, stagewise (the GPU's own G|U, h and
+scales fed to the oracle), and at the 2.75x shape on sampled rows."""
+import numpy as np
+import pytest
+import torch
+
+from fp8_gemms_b200 import synthetic
+from gpu_util import ELEM_REL, assert_close, f32, u8, u16
+
+pytestmark = pytest.mark.gpu
+
+E4M3, E5M2 = 0, 1
+
+
+def make(M, d, f, seed):
+    X = synthetic.normal_bf16((M, d), 1.0, seed, 0)
+    Wg = synthetic.normal_bf16((f, d), 0.02, seed, 1)
+    Wu = synthetic.normal_bf16((f, d), 0.02, seed, 2)
+    Wd = synthetic.normal_bf16((d, f), 0.02, seed, 3)
+    dY = synthetic.normal_bf16((M, d), 1e-3, seed, 4)
+    return X, Wg, Wu, Wd, dY
+
+
+def run_gpu(M, d, f, X, Wg, Wu, Wd, dY):
+    from fp8_gemms_b200 import _lib, api
+    Wgu = api.interleave_gate_up(Wg.cuda(), Wu.cuda())
+    mlp = api.SwigluMlp(M, d, f)
+    Y = mlp.forward(X.cuda(), Wgu, Wd.cuda())
+    dX, dWgu, dWd = mlp.backward(dY.cuda())
+    torch.cuda.synchronize()
+    assert _lib.lm_get_error()[0] == 0
+    return mlp, Wgu, Y, dX, dWgu, dWd
+
+
+def test_swiglu_end_to_end_small(orc):
+    M, d, f = 256, 256, 768
+    X, Wg, Wu, Wd, dY = make(M, d, f, 80)
+    mlp, Wgu, Y, dX, dWgu, dWd = run_gpu(M, d, f, X, Wg, Wu, Wd, dY)
+    b = synthetic.bits_u16
+    fwd = orc.swiglu_fwd(b(X), orc.interleave_gate_up(b(Wg), b(Wu)), b(Wd))
+    bwd = orc.swiglu_bwd_chain(b(dY), fwd)
+    assert np.array_equal(u16(Wgu), orc.interleave_gate_up(b(Wg), b(Wu)))
+    assert_close(u16(Y), fwd["Y"], "Y")
+    assert_close(u16(dX), bwd["dX"], "dX")
+    assert_close(u16(dWgu), bwd["dW_gu"], "dW_gu")
+    assert_close(u16(dWd), bwd["dW_down"], "dW_down")
+
+
+def check_stagewise(orc, mlp, X, Wgu, rows=None):
+    sc = mlp.view("scales").cpu().numpy()
+    Xq, Wguq = u8(mlp.view("Xq")), u8(mlp.view("Wguq"))
+    ref = orc.amax_scale_cast(synthetic.bits_u16(X), E4M3)
+    assert np.array_equal(Xq, ref["q"]) and sc[0, 0] == ref["amax"]
+    refw = orc.amax_scale_cast(u16(Wgu), E4M3)
+    assert np.array_equal(Wguq, refw["q"]) and sc[1, 1] == refw["scale"]
+    GU = u16(mlp.view("GU"))
+    GUref, _ = orc.gemm(Xq, E4M3, Wguq, E4M3, sc[0, 2], sc[1, 2], rows=rows)
+    assert_close(GU if rows is None else GU[rows], GUref, "GU")
+    h = u16(mlp.view("h"))
+    # h from the GPU's own G|U: within one bf16 step of bf16(silu(G) U)
+    href, _ = orc.swiglu_h(GU if rows is None else GU[rows])
+    hv = (h if rows is None else h[rows]).astype(np.uint32) << 16
+    rv = href.astype(np.uint32) << 16
+    g, r = hv.view(np.float32).astype(np.float64), rv.view(np.float32).astype(np.float64)
+    assert np.all(np.abs(g - r) <= 2.0 ** -7 * np.abs(r) + 1e-30)
+    # amax of h reported by the epilogue = max |GPU h|; the cast of h bit-exact
+    assert sc[3, 0] == orc.amax(h)
+    s_h, _ = orc.scale(sc[3, 0], E4M3)
+    hq, hqT = orc.cast(h, E4M3, s_h)
+    assert np.array_equal(u8(mlp.view("hq")), hq) and np.array_equal(u8(mlp.view("hqT")), hqT)
+
+
+def test_swiglu_stagewise_ragged(orc):
+    M, d, f = 272, 208, 640
+    X, Wg, Wu, Wd, dY = make(M, d, f, 81)
+    mlp, Wgu, *_ = run_gpu(M, d, f, X, Wg, Wu, Wd, dY)
+    check_stagewise(orc, mlp, X, Wgu)
+
+
+def test_swiglu_thin_batch(orc):
+    """M <= 128 still runs the gated epilogue (CTA-pair kernel, half-empty tiles)."""
+    M, d, f = 64, 128, 256
+    X, Wg, Wu, Wd, dY = make(M, d, f, 82)
+    mlp, Wgu, Y, dX, dWgu, dWd = run_gpu(M, d, f, X, Wg, Wu, Wd, dY)
+    b = synthetic.bits_u16
+    fwd = orc.swiglu_fwd(b(X), orc.interleave_gate_up(b(Wg), b(Wu)), b(Wd))
+    bwd = orc.swiglu_bwd_chain(b(dY), fwd)
+    assert_close(u16(Y), fwd["Y"], "Y")
+    assert_close(u16(dX), bwd["dX"], "dX")
+
+
+def test_swiglu_full_shape_sampled(orc):
+    """d = 3072, f = 2.75 d = 8448, M = 4096 tokens; GEMMs on sampled rows."""
+    M, d, f = 4096, 3072, 8448
+    X, Wg, Wu, Wd, dY = make(M, d, f, 83)
+    mlp, Wgu, *_ = run_gpu(M, d, f, X, Wg, Wu, Wd, dY)
+    rows = np.sort(np.random.default_rng(0).choice(M, 24, replace=False))
+    check_stagewise(orc, mlp, X, Wgu, rows=rows)
