@@ -74,6 +74,8 @@ def lib():
         L.orc_swiglu_bwd.restype = ctypes.c_float
         L.orc_swiglu_f64.argtypes = [P, P, P, P, P, i64, i64, i64, P, P, P, P, P]
         L.orc_swiglu_f64.restype = None
+        L.orc_softcap_ce.argtypes = [P, P, i64, i64, ctypes.c_double, ctypes.c_double, P, P]
+        L.orc_softcap_ce.restype = None
         L.orc_mlp_f64.argtypes = [P, P, P, P, i64, i64, i64, P, P, P, P]
         L.orc_mlp_f64.restype = None
         _lib = L
@@ -376,3 +378,43 @@ def swiglu_f64(X, Wg, Wu, Wd, dY=None):
                          _ptr(out["Y"]), _ptr(out.get("dX")), _ptr(out.get("dWg")),
                          _ptr(out.get("dWu")), _ptr(out.get("dWd")))
     return out
+
+
+# ------------------------------------- LM head with softcapped cross-entropy
+def softcap_ce(logits, labels, softcap=15.0, inv_count=None, want_grad=True):
+    """Row losses (fp64) and bf16 dlogits of the softcapped CE over bf16 logits."""
+    logits = _c(logits, np.uint16)
+    labels = _c(np.asarray(labels, dtype=np.int32), np.int32)
+    rows, V = logits.shape
+    inv = 1.0 / rows if inv_count is None else inv_count
+    dl = np.zeros((rows, V), np.uint16) if want_grad else None
+    loss = np.zeros(rows, np.float64)
+    lib().orc_softcap_ce(_ptr(logits), _ptr(labels), rows, V, float(softcap), float(inv),
+                         _ptr(dl), _ptr(loss))
+    return loss, dl
+
+
+def lmhead_ce(X, W, labels, chunk, softcap=15.0):
+    """FP8 LM head inside a chunked, softcapped fused linear cross-entropy:
+    X and W are quantised once (X's per-chunk codes use the whole tensor's
+    scale); per chunk of rows: bf16 logits = Xq_c Wq^T, CE -> dlogits,
+    dlogits cast to e5m2 (its own tensorwise scale), dX_c = dL_c W,
+    dW += fp32(dL_c^T X_c).  Returns mean loss, dX (bf16 bits), dW (fp32)."""
+    M, d = X.shape
+    V = W.shape[0]
+    cw = amax_scale_cast(W, E4M3)
+    ax = amax(X)
+    sx, isx = scale(ax, E4M3)
+    dX = np.zeros((M, d), np.uint16)
+    dW = np.zeros((V, d), np.float32)
+    losses = np.zeros(M, np.float64)
+    for c0 in range(0, M, chunk):
+        c1 = min(M, c0 + chunk)
+        Xq, XqT = cast(X[c0:c1], E4M3, sx)
+        logits, _ = gemm(Xq, E4M3, cw["q"], E4M3, isx, cw["inv_scale"])
+        loss, dl = softcap_ce(logits, labels[c0:c1], softcap, inv_count=1.0 / M)
+        losses[c0:c1] = loss
+        cdl = amax_scale_cast(dl, E5M2)
+        dX[c0:c1], _ = gemm(cdl["q"], E5M2, cw["qT"], E4M3, cdl["inv_scale"], cw["inv_scale"])
+        gemm_accum_f32(cdl["qT"], E5M2, XqT, E4M3, cdl["inv_scale"], isx, dW)
+    return losses.mean(), dX, dW, losses

@@ -362,6 +362,40 @@ float orc_swiglu_bwd(const uint16_t* g_, const uint16_t* GU, int64_t M, int64_t 
     return orc_amax(dGU, M, 2 * f, 2 * f, 0);
 }
 
+/* ----------------------------- softcapped cross-entropy of the LM head */
+/* Loss of the run: Liger's fused linear cross-entropy with softcap 15
+ * (decomputer.nl, "Het trainen van een 3.8B LLM tot 0.384 CORE voor $998",
+ * "Appendix: De configuratie", loss; section "Doorvoer verhogen", fused CE
+ * bullet).  For each row r of bf16 logits l (V entries):
+ *   z = c tanh(l / c),  lse = log sum_v exp(z_v),  loss_r = lse - z[label_r]
+ *   dlogits_v = bf16( (exp(z_v - lse) - [v == label_r]) (1 - (z_v / c)^2) * inv_count )
+ * in fp64; inv_count is 1 / (number of tokens) for the mean reduction.  All V
+ * columns take part in the softmax (the padded vocabulary rows are ordinary
+ * rows of the weight).  Returns the row losses in loss_rows. */
+void orc_softcap_ce(const uint16_t* logits, const int32_t* labels, int64_t rows, int64_t V,
+                    double c, double inv_count, uint16_t* dlogits, double* loss_rows) {
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* l = logits + r * V;
+        double m = -INFINITY;
+        for (int64_t v = 0; v < V; ++v) {
+            double z = c * tanh(orc_bf16_to_double(l[v]) / c);
+            if (z > m) m = z;
+        }
+        double sum = 0.0;
+        for (int64_t v = 0; v < V; ++v) sum += exp(c * tanh(orc_bf16_to_double(l[v]) / c) - m);
+        double lse = m + log(sum);
+        double zl = c * tanh(orc_bf16_to_double(l[labels[r]]) / c);
+        loss_rows[r] = lse - zl;
+        if (dlogits)
+            for (int64_t v = 0; v < V; ++v) {
+                double z = c * tanh(orc_bf16_to_double(l[v]) / c);
+                double p = exp(z - lse) - (v == labels[r] ? 1.0 : 0.0);
+                dlogits[r * V + v] = orc_bf16_from_double(p * (1.0 - (z / c) * (z / c)) * inv_count);
+            }
+    }
+}
+
 /* ---------------------------------------------- unquantised fp64 MLP chain */
 
 /* Plain fp64 SwiGLU MLP, no quantisation (same role as orc_mlp_f64):
