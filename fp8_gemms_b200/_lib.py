@@ -27,7 +27,8 @@ EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
             "lm_relu2_mlp_bwd_noalloc", "lm_relu2_mlp_bwd_noalloc_max_bytes",
             "lm_selftest_bounded_wait", "lm_relu2_mlp_fwd_ex", "lm_relu2_mlp_bwd_ex",
             "lm_rmsnorm_fp8_cast", "lm_swiglu_mlp_saved_bytes", "lm_swiglu_mlp_saved_carve",
-            "lm_swiglu_mlp_workspace_size", "lm_swiglu_mlp_fwd", "lm_swiglu_mlp_bwd"]
+            "lm_swiglu_mlp_workspace_size", "lm_swiglu_mlp_fwd", "lm_swiglu_mlp_bwd",
+            "lm_fp8_lmhead_ce_workspace_size", "lm_fp8_lmhead_ce"]
 
 
 class LmError(RuntimeError):
@@ -105,6 +106,11 @@ def _load():
     L.lm_swiglu_mlp_bwd.argtypes = [P, ctypes.POINTER(SwigluSaved), i64, i64, i64, P, P, P, P,
                                     ctypes.c_size_t, P]
     L.lm_swiglu_mlp_bwd.restype = st
+    L.lm_fp8_lmhead_ce_workspace_size.argtypes = [i64, i64, i64, i64]
+    L.lm_fp8_lmhead_ce_workspace_size.restype = ctypes.c_size_t
+    L.lm_fp8_lmhead_ce.argtypes = [P, P, P, i64, i64, i64, i64, ctypes.c_float, P, P, P, P,
+                                   ctypes.c_size_t, P]
+    L.lm_fp8_lmhead_ce.restype = st
     L.lm_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
     L.lm_selftest_bounded_wait.restype = st
     return L
@@ -244,6 +250,17 @@ def lm_swiglu_mlp_bwd(dY, saved, dX, dW_gu, dW_down, workspace, stream=None):
                                  _p(dW_down), _p(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)),
            "lm_swiglu_mlp_bwd")
+
+
+def lm_fp8_lmhead_ce(X, W, labels, loss_out, dX, dW, workspace, chunk, softcap=15.0,
+                     stream=None):
+    M, d = X.shape
+    V = W.shape[0]
+    assert labels.dtype == torch.int32 and dW.dtype == torch.float32
+    _check(lib.lm_fp8_lmhead_ce(_p(X), _p(W), _p(labels), M, d, V, chunk, softcap, _p(loss_out),
+                                _p(dX), _p(dW), _p(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream)),
+           "lm_fp8_lmhead_ce")
 
 
 def lm_get_error(stream=None):

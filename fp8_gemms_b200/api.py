@@ -191,6 +191,34 @@ class SwigluMlp:
         return self.saved_buf[off:off + shape[0] * shape[1]].view(*shape)
 
 
+class LmHeadCE:
+    """Workspace of the chunked FP8 LM head with softcapped cross-entropy."""
+
+    def __init__(self, M, d, V, chunk, device="cuda"):
+        self.M, self.d, self.V, self.chunk = M, d, V, chunk
+        n = _lib.lib.lm_fp8_lmhead_ce_workspace_size(M, d, V, chunk)
+        if n == 0:
+            raise LmError(3, "lm_fp8_lmhead_ce_workspace_size")
+        self.workspace = torch.empty(n, dtype=torch.uint8, device=device)
+        self.loss = torch.zeros(1, dtype=torch.float32, device=device)
+        self.device = device
+
+    def __call__(self, X, W, labels, dW=None, dX=None, softcap=15.0, stream=None):
+        """Mean loss (device scalar), dX (bf16) and dW (fp32, accumulated)."""
+        dX = dX if dX is not None else torch.empty_like(X)
+        dW = dW if dW is not None else torch.zeros(self.V, self.d, dtype=torch.float32,
+                                                   device=self.device)
+        _lib.lm_fp8_lmhead_ce(X, W, labels, self.loss, dX, dW, self.workspace, self.chunk,
+                              softcap=softcap, stream=stream)
+        return self.loss, dX, dW
+
+    def row_losses(self):
+        """Per-token losses of the last call (the workspace's tail)."""
+        n = self.M * 4
+        tail = (n + 255) // 256 * 256
+        return self.workspace[-tail:][:n].view(torch.float32)
+
+
 def linear_fwd_bwd(X, W, dY, stream=None):
     """Plain linear Y = X W^T with its dgrad and wgrad, all in FP8: X, W cast
     to e4m3 and dY to e5m2 (each with its K-major transposed copy), then

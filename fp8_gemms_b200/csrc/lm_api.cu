@@ -174,7 +174,8 @@ lm_status lm_get_error(lm_stream_t stream, uint32_t* where_out) {
     if (v != 0 && cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
         return LM_ERR_CUDA;
     if (where_out) *where_out = v;
-    return v ? LM_ERR_TIMEOUT : LM_OK;
+    if (!v) return LM_OK;
+    return (v & 0xF00u) == 0x400u ? LM_ERR_INVALID_ARG : LM_ERR_TIMEOUT;
 }
 
 const char* lm_status_string(lm_status s) {

@@ -1,0 +1,252 @@
+// lm_lmhead_ce.cu -- the LM head in FP8 inside a chunked, softcapped fused
+// linear cross-entropy: the B*T x V logits never exist in full.
+//
+// The run's loss is Liger's fused linear cross-entropy with softcap 15,
+// which chunks the head matmul so the logits are never materialised
+// (decomputer.nl, "Het trainen van een 3.8B LLM tot 0.384 CORE voor $998",
+// section "Doorvoer (Throughput) verhogen", fused linear cross-entropy
+// bullet; "Appendix: De configuratie", loss).  Here the head's three GEMMs
+// run in FP8 with dynamic tensorwise scaling like every other linear:
+//
+//   once:      W -> e4m3 (+ transpose); amax/scale of X (whole tensor)
+//   per chunk: X_c -> e4m3 (+ transpose) at X's scale
+//              logits_c = X_c W^T (bf16)
+//              CE: z = c tanh(l / c), row loss, dlogits (bf16, in place) + amax
+//              dlogits_c -> e5m2 (+ transpose), no reduction pass
+//              dX_c = dlogits_c W        (K = V)
+//              dW  += fp32(dlogits_c^T X_c)   (TMA reduce-add epilogue)
+//   end:       mean loss = deterministic fp64 sum of the row losses / M
+#include <cuda_bf16.h>
+
+#include "lm_internal.h"
+
+namespace lm {
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+constexpr int kCeThreads = 512;
+
+struct Ws {
+    float* scales;  // {amax, scale, inv, 0} for X, W, dlogits
+    uint8_t *Wq, *WqT, *Xq, *XqT, *dLq, *dLqT;
+    uint16_t* logits;
+    float* loss_rows;
+};
+
+size_t layout(int64_t M, int64_t d, int64_t V, int64_t C, uint8_t* base, Ws* w) {
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* p = base ? base + off : nullptr;
+        off += round_up(bytes);
+        return p;
+    };
+    Ws o;
+    o.scales = reinterpret_cast<float*>(take(16 * sizeof(float)));
+    o.Wq = take((size_t)V * d);
+    o.WqT = take((size_t)V * d);
+    o.Xq = take((size_t)C * d);
+    o.XqT = take((size_t)C * d);
+    o.logits = reinterpret_cast<uint16_t*>(take((size_t)C * V * 2));
+    o.dLq = take((size_t)C * V);
+    o.dLqT = take((size_t)C * V);
+    o.loss_rows = reinterpret_cast<float*>(take((size_t)M * sizeof(float)));
+    if (w) *w = o;
+    return off;
+}
+
+bool shapes_ok(int64_t M, int64_t d, int64_t V, int64_t C) {
+    return M >= 0 && d > 0 && V > 0 && C > 0 && M % 16 == 0 && d % 16 == 0 && V % 16 == 0 &&
+           C % 16 == 0 && V < (int64_t(1) << 31) && C < (int64_t(1) << 31);
+}
+
+__device__ __forceinline__ float softcap_f(float l, float c) {
+    return __fmul_rn(c, tanhf(__fdiv_rn(l, c)));
+}
+
+// combine two (max, sum of exp(z - max)) pairs
+__device__ __forceinline__ void lse_combine(float& m, float& s, float m2, float s2) {
+    const float mm = fmaxf(m, m2);
+    if (mm == -INFINITY) return;
+    s = __fadd_rn(__fmul_rn(s, expf(m - mm)), __fmul_rn(s2, expf(m2 - mm)));
+    m = mm;
+}
+
+// One block per row of bf16 logits (V entries, V % 8 == 0).  Writes the row
+// loss and, in place, dlogits = bf16((p - onehot) (1 - (z/c)^2) inv_count);
+// max |dlogits| is max-reduced into amax_bits.
+__global__ void __launch_bounds__(kCeThreads)
+    softcap_ce_kernel(uint16_t* __restrict__ logits, const int32_t* __restrict__ labels, int V,
+                      float c, float inv_count, float* __restrict__ loss_rows,
+                      unsigned int* __restrict__ amax_bits, unsigned int* err) {
+    const int64_t row = blockIdx.x;
+    uint4* lv = reinterpret_cast<uint4*>(logits + row * (int64_t)V);
+    const int nv = V >> 3;
+    int label = labels[row];
+    const bool label_ok = (unsigned)label < (unsigned)V;  // never read outside the row
+    if (!label_ok) {
+        if (threadIdx.x == 0) atomicCAS(err, 0u, 0x401u);
+        label = -1;  // no target: loss = lse, no one-hot term
+    }
+    float m = -INFINITY, s = 0.f;
+    for (int v = threadIdx.x; v < nv; v += kCeThreads) {
+        const uint4 x = lv[v];
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        float z[8], zm = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            z[2 * i] = softcap_f(__uint_as_float(w[i] << 16), c);
+            z[2 * i + 1] = softcap_f(__uint_as_float(w[i] & 0xFFFF0000u), c);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) zm = fmaxf(zm, z[i]);
+        float zs = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) zs = __fadd_rn(zs, expf(z[i] - zm));
+        lse_combine(m, s, zm, zs);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xFFFFFFFFu, m, o);
+        const float s2 = __shfl_xor_sync(0xFFFFFFFFu, s, o);
+        lse_combine(m, s, m2, s2);
+    }
+    __shared__ float sm[kCeThreads / 32], ss[kCeThreads / 32];
+    __shared__ float s_lse;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        sm[warp] = m;
+        ss[warp] = s;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float M0 = sm[0], S0 = ss[0];
+        for (int i = 1; i < kCeThreads / 32; ++i) lse_combine(M0, S0, sm[i], ss[i]);
+        const float lse = __fadd_rn(M0, logf(S0));
+        s_lse = lse;
+        const float zl =
+            label_ok ? softcap_f(__uint_as_float((uint32_t)logits[row * (int64_t)V + label] << 16), c)
+                     : 0.0f;
+        loss_rows[row] = __fsub_rn(lse, zl);
+    }
+    __syncthreads();
+    const float lse = s_lse;
+    const float inv_c = __fdiv_rn(1.0f, c);
+    uint32_t m2 = 0;
+    for (int v = threadIdx.x; v < nv; v += kCeThreads) {
+        const uint4 x = lv[v];
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float r[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float l = __uint_as_float(h ? (w[i] & 0xFFFF0000u) : (w[i] << 16));
+                const float z = softcap_f(l, c);
+                float p = expf(z - lse);
+                if (8 * v + 2 * i + h == label) p = __fsub_rn(p, 1.0f);
+                const float t = __fmul_rn(z, inv_c);
+                r[h] = __fmul_rn(__fmul_rn(p, __fsub_rn(1.0f, __fmul_rn(t, t))), inv_count);
+            }
+            const __nv_bfloat162 b = __floats2bfloat162_rn(r[0], r[1]);
+            o[i] = *reinterpret_cast<const uint32_t*>(&b);
+            m2 = __vmaxu2(m2, o[i] & 0x7FFF7FFFu);
+        }
+        lv[v] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    uint32_t mm = max(m2 & 0xFFFFu, m2 >> 16);
+    mm = __reduce_max_sync(0xFFFFFFFFu, mm);
+    __shared__ uint32_t wm[kCeThreads / 32];
+    if (lane == 0) wm[warp] = mm;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int i = 0; i < kCeThreads / 32; ++i) b = max(b, wm[i]);
+        if (b) atomicMax(amax_bits, b << 16);
+    }
+}
+
+// mean of the row losses: fixed-order fp64 sum in one block (deterministic)
+__global__ void __launch_bounds__(1024) mean_loss_kernel(const float* __restrict__ rows, int64_t n,
+                                                         float* __restrict__ out) {
+    __shared__ double part[1024];
+    double acc = 0.0;
+    for (int64_t i = threadIdx.x; i < n; i += 1024) acc += (double)rows[i];
+    part[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = 512; w > 0; w >>= 1) {
+        if ((int)threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) *out = n ? (float)(part[0] / (double)n) : 0.0f;
+}
+
+#define LM_TRY(expr)                  \
+    do {                              \
+        lm_status _st = (expr);       \
+        if (_st != LM_OK) return _st; \
+    } while (0)
+
+}  // namespace
+}  // namespace lm
+
+extern "C" {
+
+size_t lm_fp8_lmhead_ce_workspace_size(int64_t M, int64_t d, int64_t V, int64_t chunk) {
+    if (!lm::shapes_ok(M, d, V, chunk)) return 0;
+    return lm::layout(M, d, V, chunk, nullptr, nullptr);
+}
+
+lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* labels, int64_t M,
+                           int64_t d, int64_t V, int64_t chunk, float softcap, float* loss_out,
+                           void* dX, float* dW, void* workspace, size_t ws_bytes,
+                           lm_stream_t stream) {
+    using namespace lm;
+    if (!shapes_ok(M, d, V, chunk)) return LM_ERR_UNSUPPORTED_SHAPE;
+    if (!X || !W || !labels || !loss_out || !dX || !dW || !workspace) return LM_ERR_INVALID_ARG;
+    if (!(softcap > 0.f)) return LM_ERR_INVALID_ARG;
+    if (ws_bytes < layout(M, d, V, chunk, nullptr, nullptr)) return LM_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return LM_ERR_ALIGNMENT;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(dX) || !aligned16(dW)) return LM_ERR_ALIGNMENT;
+    unsigned int* err = device_error_word();
+    if (!err) return LM_ERR_CUDA;
+    Ws w;
+    layout(M, d, V, chunk, static_cast<uint8_t*>(workspace), &w);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float* SX = w.scales;
+    float* SW = w.scales + 4;
+    float* SL = w.scales + 8;
+    if (cudaMemsetAsync(w.scales, 0, 16 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
+    LM_TRY(lm_fp8_amax_scale_cast(W, V, d, d, LM_FP8_E4M3, 0, nullptr, SW, SW + 1, SW + 2, w.Wq,
+                                  w.WqT, stream));
+    // X's amax and scale over the whole tensor (no codes yet)
+    LM_TRY(lm_fp8_amax_scale_cast(X, M, d, d, LM_FP8_E4M3, 0, nullptr, SX, SX + 1, SX + 2,
+                                  nullptr, nullptr, stream));
+    const uint16_t* Xb = static_cast<const uint16_t*>(X);
+    uint16_t* dXb = static_cast<uint16_t*>(dX);
+    for (int64_t c0 = 0; c0 < M; c0 += chunk) {
+        const int64_t rows = (M - c0) < chunk ? (M - c0) : chunk;
+        LM_TRY(lm_fp8_amax_scale_cast(Xb + c0 * d, rows, d, d, LM_FP8_E4M3, 0, SX, SX, SX + 1,
+                                      SX + 2, w.Xq, w.XqT, stream));
+        LM_TRY(lm_fp8_gemm(w.Xq, LM_FP8_E4M3, w.Wq, LM_FP8_E4M3, rows, V, d, SX + 2, SW + 2,
+                           LM_EPI_NONE, nullptr, w.logits, nullptr, stream));
+        if (cudaMemsetAsync(SL, 0, 4 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
+        timing_mark(s, 'e');
+        softcap_ce_kernel<<<(unsigned)rows, kCeThreads, 0, s>>>(
+            w.logits, labels + c0, (int)V, softcap, (float)(1.0 / (double)M), w.loss_rows + c0,
+            reinterpret_cast<unsigned int*>(SL), err);
+        if (launch_status() != LM_OK) return LM_ERR_CUDA;
+        LM_TRY(lm_fp8_amax_scale_cast(w.logits, rows, V, V, LM_FP8_E5M2, 0, SL, SL, SL + 1,
+                                      SL + 2, w.dLq, w.dLqT, stream));
+        LM_TRY(lm_fp8_gemm(w.dLq, LM_FP8_E5M2, w.WqT, LM_FP8_E4M3, rows, d, V, SL + 2, SW + 2,
+                           LM_EPI_NONE, nullptr, dXb + c0 * d, nullptr, stream));
+        LM_TRY(lm_fp8_gemm(w.dLqT, LM_FP8_E5M2, w.XqT, LM_FP8_E4M3, V, d, rows, SL + 2, SX + 2,
+                           LM_EPI_ACCUM_F32, nullptr, dW, nullptr, stream));
+    }
+    timing_mark(s, 'l');
+    mean_loss_kernel<<<1, 1024, 0, s>>>(w.loss_rows, M, loss_out);
+    return launch_status();
+}
+
+}  // extern "C"

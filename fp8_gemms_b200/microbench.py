@@ -48,7 +48,10 @@ def time_it(fn, iters, warmup, flush):
 
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("op", choices=["gemm", "cast", "mlp-accum", "rmsnorm-cast", "mlp-compare"])
+    p.add_argument("op", choices=["gemm", "cast", "mlp-accum", "rmsnorm-cast", "mlp-compare",
+                                  "lmhead-ce"])
+    p.add_argument("--V", type=int, default=50304)
+    p.add_argument("--chunk", type=int, default=4096)
     p.add_argument("--micro", type=int, default=7)
     p.add_argument("--d", type=int, default=3072)
     p.add_argument("--f", type=int, default=12288)
@@ -95,6 +98,23 @@ def main():
         out = dict(op="mlp-compare", M=M, d=d, **res,
                    relu2_over_swiglu_tokens=round(res["relu2"]["tokens_per_s"] /
                                                   res["swiglu"]["tokens_per_s"], 4))
+    elif a.op == "lmhead-ce":
+        from . import api
+        M, d, V = a.M, a.d, a.V
+        head = api.LmHeadCE(M, d, V, a.chunk)
+        X = torch.randn(M, d, device="cuda", generator=gen).to(torch.bfloat16)
+        W = (torch.randn(V, d, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)
+        labels = torch.randint(0, 50257, (M,), device="cuda", generator=gen, dtype=torch.int32)
+        dW = torch.zeros(V, d, dtype=torch.float32, device="cuda")
+        dX = torch.empty_like(X)
+        fn = lambda: head(X, W, labels, dW=dW, dX=dX)
+        ms = time_it(fn, a.iters, a.warmup, flush)
+        avg = sum(ms) / len(ms)
+        flops = 3 * 2 * M * d * V
+        out = dict(op="lmhead-ce", M=M, d=d, V=V, chunk=a.chunk, avg_ms=round(avg, 4),
+                   tokens_per_s=round(M / avg * 1e3), tflops=round(flops / avg / 1e9, 1),
+                   workspace_bytes=head.workspace.numel(), full_logits_bytes=2 * M * V,
+                   loss=round(float(head.loss.item()), 5))
     elif a.op == "rmsnorm-cast":
         R = torch.randn(a.rows, a.cols, device="cuda", generator=gen).to(torch.bfloat16)
         w = torch.randn(a.cols, device="cuda", generator=gen).to(torch.bfloat16)

@@ -294,8 +294,37 @@ LM_API lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* saved,
                                    int64_t d, int64_t f, void* dX, void* dW_gu, void* dW_down,
                                    void* workspace, size_t ws_bytes, lm_stream_t stream);
 
+/*
+ * The LM head in FP8 inside a chunked, softcapped fused linear cross-entropy
+ * (decomputer.nl, "Het trainen van een 3.8B LLM tot 0.384 CORE voor $998",
+ * section "Doorvoer (Throughput) verhogen", fused linear cross-entropy
+ * bullet, and "Appendix: De configuratie": loss with softcap 15.0).  Forward
+ * and backward in one call; the M x V logits are never held in full:
+ *
+ *   z = softcap * tanh(logits / softcap),  logits = X W^T (FP8 GEMM, bf16)
+ *   loss_out = mean over the M tokens of (logsumexp(z) - z[label])
+ *   dX  = dlogits W              (FP8 dgrad, e5m2 x e4m3, bf16 out)
+ *   dW += fp32(dlogits^T X)      (FP8 wgrad accumulated into the caller's fp32 dW)
+ *   dlogits = (softmax(z) - onehot(label)) (1 - (z/softcap)^2) / M
+ *
+ * X and W are quantised once (X's per-chunk codes use X's whole-tensor
+ * scale); each chunk's dlogits gets its own tensorwise e5m2 scale.  All V
+ * columns take part in the softmax.
+ * X: bf16 [M x d]; W: bf16 [V x d]; labels: device int32 [M], each in [0, V);
+ * loss_out: device fp32 scalar; dX: bf16 [M x d]; dW: fp32 [V x d] (added to);
+ * chunk: tokens per chunk; workspace: >= lm_fp8_lmhead_ce_workspace_size bytes,
+ * 256-byte aligned.  M, d, V, chunk multiples of 16.
+ */
+LM_API size_t lm_fp8_lmhead_ce_workspace_size(int64_t M, int64_t d, int64_t V, int64_t chunk);
+LM_API lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* labels, int64_t M,
+                                  int64_t d, int64_t V, int64_t chunk, float softcap,
+                                  float* loss_out, void* dX, float* dW, void* workspace,
+                                  size_t ws_bytes, lm_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the current device's error
  * word: LM_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
+ * LM_ERR_INVALID_ARG if a kernel met invalid device-side data (code 0x401: a
+ * label outside [0, V) in lm_fp8_lmhead_ce, treated as having no target),
  * LM_ERR_CUDA if the synchronisation itself failed, else LM_OK.  If
  * where_out is non-NULL it receives the code of the wait that ran out (0 if
  * none). */
@@ -311,7 +340,7 @@ LM_API lm_status lm_get_error(lm_stream_t stream, uint32_t* where_out);
  * stops recording and returns the number of events recorded.
  * lm_timing_kinds() copies one character per recorded launch ('a' amax
  * reduction, 'c' cast, 's' scales only, 'g' GEMM, 'n' RMSNorm, 'w'
- * SwiGLU backward elementwise) into out[0..cap) and
+ * SwiGLU backward elementwise, 'e' softcapped CE, 'l' mean loss) into out[0..cap) and
  * returns how many it wrote.  State is per host thread.
  */
 LM_API void lm_timing_attach(void* const* events, int capacity);
