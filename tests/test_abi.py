@@ -90,3 +90,40 @@ def test_mlp_sizes_and_carve(L):
     assert s.Xq == base and s.XqT == base + r(M * d) and s.scales == base + n - r(64)
     assert L.lib.lm_relu2_mlp_saved_carve(base, n - 1, M, d, f, ctypes.byref(s)) == 1
     assert L.lib.lm_relu2_mlp_saved_carve(base + 16, n, M, d, f, ctypes.byref(s)) == 2
+
+
+def test_newer_entry_points_reject_before_launch(L):
+    import ctypes as C
+    fake = 0x10000
+    lib = L.lib
+    s = L.MlpSaved()
+    # unknown flags
+    assert lib.lm_relu2_mlp_fwd_ex(fake, fake, fake, 256, 256, 1024, fake, C.byref(s), 4, None) == 1
+    assert lib.lm_relu2_mlp_bwd_ex(fake, C.byref(s), 256, 256, 1024, fake, fake, fake, fake,
+                                   1 << 30, 1, None) == 1
+    # rmsnorm: eps < 0, cols not a multiple of 16, misaligned weight
+    f32 = C.c_float
+    assert lib.lm_rmsnorm_fp8_cast(fake, None, 32, 64, f32(-1.0), 0, fake, fake, fake, fake,
+                                   fake, fake, None) == 1
+    assert lib.lm_rmsnorm_fp8_cast(fake, None, 32, 40, f32(1e-6), 0, fake, fake, fake, fake,
+                                   fake, fake, None) == 3
+    assert lib.lm_rmsnorm_fp8_cast(fake, fake + 2, 32, 64, f32(1e-6), 0, fake, fake, fake,
+                                   fake, fake, fake, None) == 2
+    # swiglu: f must be a multiple of 128
+    assert L.lib.lm_swiglu_mlp_saved_bytes(256, 256, 200) == 0
+    sw = L.SwigluSaved()
+    assert lib.lm_swiglu_mlp_fwd(fake, fake, fake, 256, 256, 200, fake, C.byref(sw), None) == 3
+    # lm head: chunk not a multiple of 16, softcap <= 0, workspace too small
+    assert lib.lm_fp8_lmhead_ce_workspace_size(64, 64, 128, 24) == 0
+    n = lib.lm_fp8_lmhead_ce_workspace_size(64, 64, 128, 32)
+    assert n > 0
+    assert lib.lm_fp8_lmhead_ce(fake, fake, fake, 64, 64, 128, 32, f32(0.0), fake, fake, fake,
+                                fake, n, None) == 1
+    assert lib.lm_fp8_lmhead_ce(fake, fake, fake, 64, 64, 128, 32, f32(15.0), fake, fake, fake,
+                                fake, n - 1, None) == 1
+    # the internal gated epilogue is not reachable through the public GEMM
+    assert lib.lm_fp8_gemm(fake, 0, fake, 0, 256, 256, 64, fake, fake, 4, None, fake, None,
+                           None) == 4
+    # no-alloc backward: shape beyond its array
+    assert lib.lm_relu2_mlp_bwd_noalloc(None, C.byref(s), 16384, 3072, 12288, None, None, None,
+                                        None) == 3
