@@ -37,7 +37,7 @@ STEP_FLOPS = 6 * GEMM_FLOPS
 DENSE_FP8_PEAK_TFLOPS = 4500.0                 # public B200 dense FP8 figure
 NOMINAL_FP8_OVER_BF16 = 2.0                    # 4.5 / 2.25 PFLOP/s dense
 WORKLOAD = "relu2 MLP fwd+dgrad+wgrad M=16384 d=3072 f=12288"
-LAUNCHES_PER_STEP = 16                         # kernels of ours per fwd+bwd: "acacacgcgacggcgg"
+LAUNCHES_PER_STEP = 12                         # kernels of ours per fwd+bwd: "acgcgacggcgg"
 
 # DRAM traffic of one GEMM launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum), valid only for the kernel source it was taken on;

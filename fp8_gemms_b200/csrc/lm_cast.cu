@@ -89,17 +89,42 @@ __device__ __forceinline__ uint32_t absmax8(uint4 v, uint32_t m) {
     return m;
 }
 
-// Pass 1: amax over the tensor into *amax_bits (fp32 bit pattern of a
-// non-negative value, max-reduced with atomicMax; zeroed by the caller).
+// Up to kMaxSet tensors handled by one launch of a pass.  Per-tensor values
+// are picked with compile-time indices (no dynamic indexing of a kernel
+// parameter, which would copy it to local memory).
+constexpr int kMaxSet = kMaxCastSet;
+
+template <typename T>
+__device__ __forceinline__ T pick(int j, T a, T b, T c) {
+    return j == 0 ? a : (j == 1 ? b : c);
+}
+
+struct AmaxSet {
+    int n;
+    const uint16_t* x[kMaxSet];
+    int64_t rows[kMaxSet], cols[kMaxSet], ld[kMaxSet];
+    unsigned int* out[kMaxSet];  // fp32 bits of the amax, zeroed beforehand
+    int block_end[kMaxSet];      // blocks [block_end[j-1], block_end[j]) reduce tensor j
+};
+
+// Pass 1: amax of each tensor of the set into its *out (fp32 bit pattern of
+// a non-negative value, max-reduced with atomicMax).  Each block reduces one
+// tensor; blocks are shared out in proportion to the tensors' sizes.
 template <bool RELU2>
-__global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restrict__ x,
-                                                        int64_t rows, int64_t cols, int64_t ld,
-                                                        unsigned int* __restrict__ amax_bits) {
+__global__ void __launch_bounds__(kThreads) amax_kernel(const AmaxSet set) {
+    const int b = (int)blockIdx.x;
+    const int j = b < set.block_end[0] ? 0 : (b < set.block_end[1] ? 1 : 2);
+    const int b0 = pick(j, 0, set.block_end[0], set.block_end[1]);
+    const int nblocks = pick(j, set.block_end[0], set.block_end[1], set.block_end[2]) - b0;
+    const uint16_t* x = pick(j, set.x[0], set.x[1], set.x[2]);
+    const int64_t rows = pick(j, set.rows[0], set.rows[1], set.rows[2]);
+    const int64_t cols = pick(j, set.cols[0], set.cols[1], set.cols[2]);
+    const int64_t ld = pick(j, set.ld[0], set.ld[1], set.ld[2]);
     uint32_t m = 0;
     const int64_t vpr = cols >> 3;  // 16-byte vectors per row
     const int64_t nvec = rows * vpr;
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    const int64_t stride = (int64_t)nblocks * kThreads;
+    int64_t i = (int64_t)(b - b0) * kThreads + threadIdx.x;
     if (ld == cols) {
         const uint4* xv = reinterpret_cast<const uint4*>(x);
         // eight independent 16-byte loads in flight per thread
@@ -123,10 +148,10 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
     if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
     __syncthreads();
     if (threadIdx.x == 0) {
-        uint32_t b = 0;
+        uint32_t bm = 0;
 #pragma unroll
-        for (int i = 0; i < kThreads / 32; ++i) b = max(b, warp_max[i]);
-        if (b) atomicMax(amax_bits, b << 16);
+        for (int w = 0; w < kThreads / 32; ++w) bm = max(bm, warp_max[w]);
+        if (bm) atomicMax(pick(j, set.out[0], set.out[1], set.out[2]), bm << 16);
     }
 }
 
@@ -249,11 +274,32 @@ __device__ __forceinline__ void consumers_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(tmac::CONSUMERS) : "memory");
 }
 
+// The tensors of one launch of the TMA-fed cast.  Global tile indices
+// [tile_end[j-1], tile_end[j]) belong to tensor j; unused entries repeat the
+// total.  Each tensor has its own tensor maps (kernel parameters tmX<j>,
+// tmQT<j>), scale and outputs.
+struct CastSet {
+    int n, num_tiles;
+    int want_qT;  // bit j: write tensor j's transposed codes
+    int tile_end[kMaxSet];
+    int rows[kMaxSet], cols[kMaxSet], tiles_c[kMaxSet];
+    const float* amax_src[kMaxSet];
+    float* amax_out[kMaxSet];
+    float* scale_out[kMaxSet];
+    float* inv_out[kMaxSet];
+    uint8_t* q[kMaxSet];
+};
+
+__device__ __forceinline__ int set_member(const CastSet& set, int t) {
+    return t < set.tile_end[0] ? 0 : (t < set.tile_end[1] ? 1 : 2);
+}
+
 template <int FMT, bool RELU2>
 __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
-    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQT, int rows,
-    int cols, const float* amax_src, float* amax_out, float* scale_out, float* inv_out,
-    uint8_t* __restrict__ q, int want_qT, int tiles_c, int num_tiles, unsigned int* err) {
+    const __grid_constant__ CUtensorMap tmX0, const __grid_constant__ CUtensorMap tmX1,
+    const __grid_constant__ CUtensorMap tmX2, const __grid_constant__ CUtensorMap tmQT0,
+    const __grid_constant__ CUtensorMap tmQT1, const __grid_constant__ CUtensorMap tmQT2,
+    const CastSet set, unsigned int* err) {
     using namespace tmac;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -265,8 +311,12 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
     uint64_t* empty = full + STAGES;
 
     const float fmax = FMT == LM_FP8_E4M3 ? 448.0f : 57344.0f;
-    float scale;
-    write_scales(*amax_src, fmax, amax_out, scale_out, inv_out, &scale);
+    float sc[kMaxSet] = {0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < kMaxSet; ++j)
+        if (j < set.n)
+            write_scales(*set.amax_src[j], fmax, set.amax_out[j], set.scale_out[j], set.inv_out[j],
+                         &sc[j]);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -276,6 +326,7 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
         fence_barrier_init();
     }
     __syncthreads();
+    const int num_tiles = set.num_tiles;
 
     if (warp == CONSUMERS / 32) {
         // ------------------------------------------------ TMA producer
@@ -284,10 +335,13 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
             uint32_t ph = 0, issued = 0;
             for (int i = blockIdx.x; i < num_tiles; i += gridDim.x) {
                 const int t = num_tiles - 1 - i;
+                const int j = set_member(set, t);
+                const int lt = t - pick(j, 0, set.tile_end[0], set.tile_end[1]);
+                const int tc = pick(j, set.tiles_c[0], set.tiles_c[1], set.tiles_c[2]);
                 if (!mbar_wait(&empty[s], ph ^ 1u, err, W_CAST_EMPTY)) break;
                 mbar_arrive_expect_tx(&full[s], IN_BYTES);
-                tma_load_2d(smem_addr(sIn + s * IN_BYTES), &tmX, &full[s], (t % tiles_c) * TC,
-                            (t / tiles_c) * TR);
+                tma_load_2d(smem_addr(sIn + s * IN_BYTES), pick(j, &tmX0, &tmX1, &tmX2), &full[s],
+                            (lt % tc) * TC, (lt / tc) * TR);
                 ++issued;
                 if (++s == STAGES) {
                     s = 0;
@@ -308,7 +362,14 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
     bool ok = true;
     for (int i = blockIdx.x; i < num_tiles; i += gridDim.x) {
         const int t = num_tiles - 1 - i;
-        const int r0 = (t / tiles_c) * TR, c0 = (t % tiles_c) * TC;
+        const int j = set_member(set, t);
+        const int lt = t - pick(j, 0, set.tile_end[0], set.tile_end[1]);
+        const int tc = pick(j, set.tiles_c[0], set.tiles_c[1], set.tiles_c[2]);
+        const int rows = pick(j, set.rows[0], set.rows[1], set.rows[2]);
+        const int cols = pick(j, set.cols[0], set.cols[1], set.cols[2]);
+        uint8_t* q = pick(j, set.q[0], set.q[1], set.q[2]);
+        const float scale = pick(j, sc[0], sc[1], sc[2]);
+        const int r0 = (lt / tc) * TR, c0 = (lt % tc) * TC;
         if (ok) ok = mbar_wait(&full[s], ph, err, W_CAST_FULL);
         const uint8_t* in = sIn + s * IN_BYTES;
 #pragma unroll
@@ -329,7 +390,7 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
             s = 0;
             ph ^= 1u;
         }
-        if (!want_qT) continue;
+        if (!((set.want_qT >> j) & 1)) continue;
         if (tid == 0) bulk_wait_group_read<0>();  // the previous tile's store has read sT
         consumers_sync();                           // codes tile complete, sT free
         // lane: tile rows [16k, 16k+16) with k = lane % 8; tile columns
@@ -351,122 +412,206 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
             o[3][m] = __byte_perm(t2, t3, 0x7632);
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c = 4 * qd + j;
+        for (int jj = 0; jj < 4; ++jj) {
+            const int c = 4 * qd + jj;
             *reinterpret_cast<uint4*>(sT + c * 128 + ((k ^ (c & 7)) << 4)) =
-                make_uint4(o[j][0], o[j][1], o[j][2], o[j][3]);
+                make_uint4(o[jj][0], o[jj][1], o[jj][2], o[jj][3]);
         }
         fence_proxy_async_smem();
         consumers_sync();  // transposed tile complete; codes tile fully read
         if (tid == 0) {
-            tma_store_2d(&tmQT, smem_addr(sT), r0, c0);
+            tma_store_2d(pick(j, &tmQT0, &tmQT1, &tmQT2), smem_addr(sT), r0, c0);
             bulk_commit_group();
         }
     }
     if (tid == 0) bulk_wait_group<0>();
 }
 
+// TMA-fed cast of the items (each with rows % 16 == 0) in one launch.
 template <int FMT, bool RELU2>
-lm_status launch_cast(const uint16_t* x, int rows, int cols, int64_t ld, const float* amax_src,
-                      float* amax_out, float* scale_out, float* inv_out, uint8_t* q, uint8_t* qT,
-                      cudaStream_t s) {
-    if (rows % 16 == 0) {
-        // TMA-fed persistent kernel (its transposed stores need 16-row groups)
-        static bool configured[64] = {};
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LM_ERR_CUDA;
-        if (!configured[dev]) {
-            if (cudaFuncSetAttribute(cast_tma_kernel<FMT, RELU2>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     tmac::SMEM) != cudaSuccess)
-                return LM_ERR_CUDA;
-            configured[dev] = true;
-        }
-        CUtensorMap tm, tq;
-        if (!encode_tmap_bf16_plain(&tm, x, (uint64_t)rows, (uint64_t)cols, (uint64_t)ld * 2,
-                                    tmac::TR, tmac::TC))
+lm_status launch_cast_tma(const CastItem* const* items, const float* const* amax_src, int n,
+                          cudaStream_t s) {
+    static bool configured[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LM_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(cast_tma_kernel<FMT, RELU2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tmac::SMEM) != cudaSuccess)
             return LM_ERR_CUDA;
-        if (qT) {  // qT is [cols x rows]: tile rows become 128-byte rows of codes
-            if (!encode_tmap_u8(&tq, qT, (uint64_t)cols, (uint64_t)rows, (uint64_t)rows, tmac::TC,
-                                tmac::TR))
-                return LM_ERR_CUDA;
-        } else {
-            tq = tm;  // unused
-        }
-        unsigned int* err = device_error_word();
-        if (!err) return LM_ERR_CUDA;
-        const int tiles_c = (cols + tmac::TC - 1) / tmac::TC;
-        const int n = ((rows + tmac::TR - 1) / tmac::TR) * tiles_c;
-        int grid = 2 * sm_count();
-        if (grid <= 0) return LM_ERR_CUDA;
-        if (grid > n) grid = n;
-        timing_mark(s, 'c');
-        cast_tma_kernel<FMT, RELU2><<<grid, tmac::THREADS, tmac::SMEM, s>>>(
-            tm, tq, rows, cols, amax_src, amax_out, scale_out, inv_out, q, qT ? 1 : 0, tiles_c, n,
-            err);
-        return launch_status();
+        configured[dev] = true;
     }
-    const int tiles_r = (rows + kCastRows - 1) / kCastRows;
-    const int tiles_c = (cols + kCastCols - 1) / kCastCols;
-    const int n = tiles_r * tiles_c;
+    CUtensorMap tx[kMaxSet], tq[kMaxSet];
+    CastSet set = {};
+    set.n = n;
+    int total = 0;
+    for (int j = 0; j < n; ++j) {
+        const CastItem& it = *items[j];
+        const int rows = (int)it.rows, cols = (int)it.cols;
+        if (!encode_tmap_bf16_plain(&tx[j], it.x, (uint64_t)rows, (uint64_t)cols,
+                                    (uint64_t)it.ld * 2, tmac::TR, tmac::TC))
+            return LM_ERR_CUDA;
+        if (it.qT) {  // qT is [cols x rows]: tile rows become 128-byte rows of codes
+            if (!encode_tmap_u8(&tq[j], it.qT, (uint64_t)cols, (uint64_t)rows, (uint64_t)rows,
+                                tmac::TC, tmac::TR))
+                return LM_ERR_CUDA;
+            set.want_qT |= 1 << j;
+        } else {
+            tq[j] = tx[j];  // unused
+        }
+        const int tiles_c = (cols + tmac::TC - 1) / tmac::TC;
+        total += ((rows + tmac::TR - 1) / tmac::TR) * tiles_c;
+        set.tile_end[j] = total;
+        set.rows[j] = rows;
+        set.cols[j] = cols;
+        set.tiles_c[j] = tiles_c;
+        set.amax_src[j] = amax_src[j];
+        set.amax_out[j] = it.amax_out;
+        set.scale_out[j] = it.scale_out;
+        set.inv_out[j] = it.inv_scale_out;
+        set.q[j] = it.q;
+    }
+    for (int j = n; j < kMaxSet; ++j) {
+        set.tile_end[j] = total;
+        tx[j] = tx[0];
+        tq[j] = tq[0];
+    }
+    set.num_tiles = total;
+    unsigned int* err = device_error_word();
+    if (!err) return LM_ERR_CUDA;
+    int grid = 2 * sm_count();
+    if (grid <= 0) return LM_ERR_CUDA;
+    if (grid > total) grid = total;
     timing_mark(s, 'c');
-    cast_kernel<FMT, RELU2><<<n, kThreads, 0, s>>>(x, rows, cols, ld, amax_src, amax_out,
-                                                  scale_out, inv_out, q, qT, tiles_c, n);
+    cast_tma_kernel<FMT, RELU2><<<grid, tmac::THREADS, tmac::SMEM, s>>>(tx[0], tx[1], tx[2], tq[0],
+                                                                        tq[1], tq[2], set, err);
     return launch_status();
+}
+
+// One tensor with rows % 16 != 0 (row-major codes only): one block per tile.
+template <int FMT, bool RELU2>
+lm_status launch_cast_rows(const CastItem& it, const float* amax_src, cudaStream_t s) {
+    const int rows = (int)it.rows, cols = (int)it.cols;
+    const int tiles_c = (cols + kCastCols - 1) / kCastCols;
+    const int n = ((rows + kCastRows - 1) / kCastRows) * tiles_c;
+    timing_mark(s, 'c');
+    cast_kernel<FMT, RELU2><<<n, kThreads, 0, s>>>(static_cast<const uint16_t*>(it.x), rows, cols,
+                                                  it.ld, amax_src, it.amax_out, it.scale_out,
+                                                  it.inv_scale_out, it.q, it.qT, tiles_c, n);
+    return launch_status();
+}
+
+template <int FMT, bool RELU2>
+lm_status launch_casts(const CastItem* items, const float* const* amax_src, int n,
+                       cudaStream_t s) {
+    const CastItem* tma[kMaxSet];
+    const float* tma_src[kMaxSet];
+    int nt = 0;
+    for (int j = 0; j < n; ++j) {
+        const CastItem& it = items[j];
+        if (it.rows == 0 || it.cols == 0 || (!it.q && !it.qT)) continue;
+        if (it.rows % 16 == 0) {
+            tma[nt] = &it;
+            tma_src[nt++] = amax_src[j];
+        } else if (launch_cast_rows<FMT, RELU2>(it, amax_src[j], s) != LM_OK) {
+            return LM_ERR_CUDA;
+        }
+    }
+    return nt ? launch_cast_tma<FMT, RELU2>(tma, tma_src, nt, s) : LM_OK;
+}
+
+lm_status check_item(const CastItem& it) {
+    if (it.rows < 0 || it.cols < 0 || it.ld < it.cols) return LM_ERR_INVALID_ARG;
+    if (!it.amax_out || !it.scale_out || !it.inv_scale_out) return LM_ERR_INVALID_ARG;
+    const bool empty = it.rows == 0 || it.cols == 0;
+    if (!empty && !it.x) return LM_ERR_INVALID_ARG;
+    if (it.cols % 16 != 0 || it.ld % 8 != 0) return LM_ERR_UNSUPPORTED_SHAPE;
+    if (it.qT && it.rows % 16 != 0) return LM_ERR_UNSUPPORTED_SHAPE;
+    if (it.rows >= (int64_t(1) << 31) || it.cols >= (int64_t(1) << 31))
+        return LM_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(it.x) || !aligned16(it.q) || !aligned16(it.qT)) return LM_ERR_ALIGNMENT;
+    return LM_OK;
 }
 
 }  // namespace
 }  // namespace lm
+
+lm_status lm::cast_set(const CastItem* items, int n, lm_fp8_format fmt, int relu2_input,
+                       bool amax_zeroed, cudaStream_t s) {
+    using namespace lm;
+    if (fmt != LM_FP8_E4M3 && fmt != LM_FP8_E5M2) return LM_ERR_UNSUPPORTED_FORMAT;
+    if (!items || n < 1 || n > kMaxSet) return LM_ERR_INVALID_ARG;
+    for (int j = 0; j < n; ++j)
+        if (lm_status st = check_item(items[j])) return st;
+
+    // pass 1: one launch reduces every tensor whose amax is not supplied
+    const float* src[kMaxSet];
+    AmaxSet aset = {};
+    int64_t nvec[kMaxSet], total_vec = 0;
+    int need_zero = 0;
+    for (int j = 0; j < n; ++j) {
+        const CastItem& it = items[j];
+        src[j] = it.amax_in ? it.amax_in : it.amax_out;
+        if (it.amax_in) continue;
+        ++need_zero;
+        if (it.rows == 0 || it.cols == 0) continue;
+        const int k = aset.n++;
+        aset.x[k] = static_cast<const uint16_t*>(it.x);
+        aset.rows[k] = it.rows;
+        aset.cols[k] = it.cols;
+        aset.ld[k] = it.ld;
+        aset.out[k] = reinterpret_cast<unsigned int*>(it.amax_out);
+        nvec[k] = it.rows * (it.cols >> 3);
+        total_vec += nvec[k];
+    }
+    if (aset.n) timing_mark(s, 'a');
+    if (!amax_zeroed && need_zero)
+        for (int j = 0; j < n; ++j)
+            if (!items[j].amax_in &&
+                cudaMemsetAsync(items[j].amax_out, 0, sizeof(float), s) != cudaSuccess)
+                return LM_ERR_CUDA;
+    if (aset.n) {
+        const int sms = sm_count();
+        if (sms <= 0) return LM_ERR_CUDA;
+        // blocks shared out in proportion to size, at least one per tensor
+        const int budget = 4 * sms;
+        int end = 0;
+        for (int k = 0; k < aset.n; ++k) {
+            int b = (int)((double)budget * (double)nvec[k] / (double)total_vec);
+            end += b < 1 ? 1 : b;
+            aset.block_end[k] = end;
+        }
+        for (int k = aset.n; k < kMaxSet; ++k) aset.block_end[k] = end;
+        if (relu2_input)
+            amax_kernel<true><<<end, kThreads, 0, s>>>(aset);
+        else
+            amax_kernel<false><<<end, kThreads, 0, s>>>(aset);
+        if (launch_status() != LM_OK) return LM_ERR_CUDA;
+    }
+
+    // scales alone for tensors with nothing to cast
+    const float fmax = fmt == LM_FP8_E4M3 ? 448.0f : 57344.0f;
+    for (int j = 0; j < n; ++j) {
+        const CastItem& it = items[j];
+        if (it.rows == 0 || it.cols == 0 || (!it.q && !it.qT)) {
+            timing_mark(s, 's');
+            scales_only_kernel<<<1, 1, 0, s>>>(src[j], fmax, it.amax_out, it.scale_out,
+                                               it.inv_scale_out);
+            if (launch_status() != LM_OK) return LM_ERR_CUDA;
+        }
+    }
+    if (fmt == LM_FP8_E4M3)
+        return relu2_input ? launch_casts<LM_FP8_E4M3, true>(items, src, n, s)
+                           : launch_casts<LM_FP8_E4M3, false>(items, src, n, s);
+    return relu2_input ? launch_casts<LM_FP8_E5M2, true>(items, src, n, s)
+                       : launch_casts<LM_FP8_E5M2, false>(items, src, n, s);
+}
 
 extern "C" lm_status lm_fp8_amax_scale_cast(const void* x, int64_t rows, int64_t cols, int64_t ld,
                                             lm_fp8_format fmt, int relu2_input,
                                             const float* amax_in, float* amax_out,
                                             float* scale_out, float* inv_scale_out, uint8_t* q,
                                             uint8_t* qT, lm_stream_t stream) {
-    using namespace lm;
-    if (fmt != LM_FP8_E4M3 && fmt != LM_FP8_E5M2) return LM_ERR_UNSUPPORTED_FORMAT;
-    if (rows < 0 || cols < 0 || ld < cols) return LM_ERR_INVALID_ARG;
-    if (!amax_out || !scale_out || !inv_scale_out) return LM_ERR_INVALID_ARG;
-    const bool empty = rows == 0 || cols == 0;
-    if (!empty && !x) return LM_ERR_INVALID_ARG;
-    if (cols % 16 != 0 || ld % 8 != 0) return LM_ERR_UNSUPPORTED_SHAPE;
-    if (qT && rows % 16 != 0) return LM_ERR_UNSUPPORTED_SHAPE;
-    if (rows >= (int64_t(1) << 31) || cols >= (int64_t(1) << 31)) return LM_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(x) || !aligned16(q) || !aligned16(qT)) return LM_ERR_ALIGNMENT;
-
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const float fmax = fmt == LM_FP8_E4M3 ? 448.0f : 57344.0f;
-    const uint16_t* xb = static_cast<const uint16_t*>(x);
-    const float* amax_src = amax_in;
-    if (!amax_in) {
-        if (!empty) timing_mark(s, 'a');
-        if (cudaMemsetAsync(amax_out, 0, sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
-        if (!empty) {
-            int grid = sm_count() * 4;
-            if (grid <= 0) return LM_ERR_CUDA;
-            if (relu2_input)
-                amax_kernel<true><<<grid, kThreads, 0, s>>>(xb, rows, cols, ld,
-                                                             reinterpret_cast<unsigned*>(amax_out));
-            else
-                amax_kernel<false><<<grid, kThreads, 0, s>>>(xb, rows, cols, ld,
-                                                              reinterpret_cast<unsigned*>(amax_out));
-        }
-        amax_src = amax_out;
-    }
-    if (empty || (!q && !qT)) {
-        timing_mark(s, 's');
-        scales_only_kernel<<<1, 1, 0, s>>>(amax_src, fmax, amax_out, scale_out, inv_scale_out);
-        return launch_status();
-    }
-    const int r = (int)rows, c = (int)cols;
-    if (launch_status() != LM_OK) return LM_ERR_CUDA;  // the amax pass launched cleanly
-    if (fmt == LM_FP8_E4M3)
-        return relu2_input ? launch_cast<LM_FP8_E4M3, true>(xb, r, c, ld, amax_src, amax_out,
-                                                            scale_out, inv_scale_out, q, qT, s)
-                           : launch_cast<LM_FP8_E4M3, false>(xb, r, c, ld, amax_src, amax_out,
-                                                             scale_out, inv_scale_out, q, qT, s);
-    return relu2_input ? launch_cast<LM_FP8_E5M2, true>(xb, r, c, ld, amax_src, amax_out,
-                                                        scale_out, inv_scale_out, q, qT, s)
-                       : launch_cast<LM_FP8_E5M2, false>(xb, r, c, ld, amax_src, amax_out,
-                                                         scale_out, inv_scale_out, q, qT, s);
+    const lm::CastItem it = {x, rows, cols, ld, amax_in, amax_out, scale_out, inv_scale_out, q, qT};
+    return lm::cast_set(&it, 1, fmt, relu2_input, false, reinterpret_cast<cudaStream_t>(stream));
 }

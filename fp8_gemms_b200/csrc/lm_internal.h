@@ -52,6 +52,23 @@ lm_status gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B, lm
                         const float* inv_scale_b, int epi, const void* aux, void* D, void* D2,
                         float* amax_out, lm_stream_t stream);
 
+// One tensor of lm::cast_set: the arguments of lm_fp8_amax_scale_cast.
+struct CastItem {
+    const void* x;
+    int64_t rows, cols, ld;
+    const float* amax_in;
+    float *amax_out, *scale_out, *inv_scale_out;
+    uint8_t *q, *qT;
+};
+constexpr int kMaxCastSet = 3;
+
+// lm_fp8_amax_scale_cast of up to kMaxCastSet tensors that share the format
+// and relu2_input, with one launch for all their amax reductions and one for
+// all their TMA-fed casts.  amax_zeroed: the caller has already zeroed, on
+// this stream, every amax_out whose amax_in is NULL, so no memset is issued.
+lm_status cast_set(const CastItem* items, int n, lm_fp8_format fmt, int relu2_input,
+                   bool amax_zeroed, cudaStream_t s);
+
 // If the calling thread attached timing events, record the next one on `s`
 // (call right before a kernel launch); `kind` labels the launch.
 void timing_mark(cudaStream_t s, char kind);

@@ -218,11 +218,11 @@ lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* labels, 
     float* SW = w.scales + 4;
     float* SL = w.scales + 8;
     if (cudaMemsetAsync(w.scales, 0, 16 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
-    LM_TRY(lm_fp8_amax_scale_cast(W, V, d, d, LM_FP8_E4M3, 0, nullptr, SW, SW + 1, SW + 2, w.Wq,
-                                  w.WqT, stream));
-    // X's amax and scale over the whole tensor (no codes yet)
-    LM_TRY(lm_fp8_amax_scale_cast(X, M, d, d, LM_FP8_E4M3, 0, nullptr, SX, SX + 1, SX + 2,
-                                  nullptr, nullptr, stream));
+    // W cast, and X's amax and scale over the whole tensor (no codes yet), with
+    // one amax launch for both (slots zeroed above)
+    const CastItem in[2] = {{W, V, d, d, nullptr, SW, SW + 1, SW + 2, w.Wq, w.WqT},
+                            {X, M, d, d, nullptr, SX, SX + 1, SX + 2, nullptr, nullptr}};
+    LM_TRY(cast_set(in, 2, LM_FP8_E4M3, 0, true, s));
     const uint16_t* Xb = static_cast<const uint16_t*>(X);
     uint16_t* dXb = static_cast<uint16_t*>(dX);
     for (int64_t c0 = 0; c0 < M; c0 += chunk) {

@@ -121,14 +121,13 @@ lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_dow
     } else if (cudaMemsetAsync(S, 0, 16 * sizeof(float), s) != cudaSuccess) {
         return LM_ERR_CUDA;
     }
-    LM_TRY(lm_fp8_amax_scale_cast(X, M, d, d, LM_FP8_E4M3, 0, nullptr, S + S_X, S + S_X + 1,
-                                  S + S_X + 2, sv->Xq, sv->XqT, stream));
-    if (!reuse) {
-        LM_TRY(lm_fp8_amax_scale_cast(W_up, f, d, d, LM_FP8_E4M3, 0, nullptr, S + S_WU,
-                                      S + S_WU + 1, S + S_WU + 2, sv->Wuq, sv->WuqT, stream));
-        LM_TRY(lm_fp8_amax_scale_cast(W_down, d, f, f, LM_FP8_E4M3, 0, nullptr, S + S_WD,
-                                      S + S_WD + 1, S + S_WD + 2, sv->Wdq, sv->WdqT, stream));
-    }
+    // X, W_up and W_down (or X alone): one amax launch and one cast launch;
+    // their amax slots were zeroed above
+    const lm::CastItem in[3] = {
+        {X, M, d, d, nullptr, S + S_X, S + S_X + 1, S + S_X + 2, sv->Xq, sv->XqT},
+        {W_up, f, d, d, nullptr, S + S_WU, S + S_WU + 1, S + S_WU + 2, sv->Wuq, sv->WuqT},
+        {W_down, d, f, f, nullptr, S + S_WD, S + S_WD + 1, S + S_WD + 2, sv->Wdq, sv->WdqT}};
+    LM_TRY(lm::cast_set(in, reuse ? 1 : 3, LM_FP8_E4M3, 0, true, s));
     // H = X W_up^T (bf16) and amax of h = bf16(relu(H)^2)
     LM_TRY(lm_fp8_gemm(sv->Xq, LM_FP8_E4M3, sv->Wuq, LM_FP8_E4M3, M, f, d, S + S_X + 2,
                        S + S_WU + 2, LM_EPI_RELU2_FWD, nullptr, sv->H, S + S_H, stream));
@@ -164,8 +163,9 @@ lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* sv, int64_t M,
     const float* S = sv->scales;
     float* G = w.scales;
     if (cudaMemsetAsync(G, 0, 8 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
-    LM_TRY(lm_fp8_amax_scale_cast(dY, M, d, d, LM_FP8_E5M2, 0, nullptr, G + S_DY, G + S_DY + 1,
-                                  G + S_DY + 2, w.dYq, w.dYqT, stream));
+    const lm::CastItem dy = {dY, M, d, d, nullptr, G + S_DY, G + S_DY + 1, G + S_DY + 2,
+                             w.dYq, w.dYqT};
+    LM_TRY(lm::cast_set(&dy, 1, LM_FP8_E5M2, 0, true, s));  // slot zeroed above
     // dH = bf16(bf16(dY W_down) * 2 relu(H)), and its amax
     LM_TRY(lm_fp8_gemm(w.dYq, LM_FP8_E5M2, sv->WdqT, LM_FP8_E4M3, M, f, d, G + S_DY + 2,
                        S + S_WD + 2, LM_EPI_RELU2_BWD, sv->H, w.dH, G + S_DH, stream));

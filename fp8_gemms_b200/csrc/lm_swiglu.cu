@@ -178,12 +178,13 @@ lm_status lm_swiglu_mlp_fwd(const void* X, const void* W_gu, const void* W_down,
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     float* S = sv->scales;
     if (cudaMemsetAsync(S, 0, 16 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
-    LM_TRY(lm_fp8_amax_scale_cast(X, M, d, d, LM_FP8_E4M3, 0, nullptr, S + S_X, S + S_X + 1,
-                                  S + S_X + 2, sv->Xq, sv->XqT, stream));
-    LM_TRY(lm_fp8_amax_scale_cast(W_gu, 2 * f, d, d, LM_FP8_E4M3, 0, nullptr, S + S_WGU,
-                                  S + S_WGU + 1, S + S_WGU + 2, sv->Wguq, sv->WguqT, stream));
-    LM_TRY(lm_fp8_amax_scale_cast(W_down, d, f, f, LM_FP8_E4M3, 0, nullptr, S + S_WD,
-                                  S + S_WD + 1, S + S_WD + 2, sv->Wdq, sv->WdqT, stream));
+    // X, W_gu, W_down: one amax launch, one cast launch (slots zeroed above)
+    const CastItem in[3] = {
+        {X, M, d, d, nullptr, S + S_X, S + S_X + 1, S + S_X + 2, sv->Xq, sv->XqT},
+        {W_gu, 2 * f, d, d, nullptr, S + S_WGU, S + S_WGU + 1, S + S_WGU + 2, sv->Wguq,
+         sv->WguqT},
+        {W_down, d, f, f, nullptr, S + S_WD, S + S_WD + 1, S + S_WD + 2, sv->Wdq, sv->WdqT}};
+    LM_TRY(cast_set(in, 3, LM_FP8_E4M3, 0, true, s));
     if (M > 0)
         LM_TRY(gemm_dispatch(sv->Xq, LM_FP8_E4M3, sv->Wguq, LM_FP8_E4M3, M, 2 * f, d, S + S_X + 2,
                              S + S_WGU + 2, kEpiSwigluFwd, nullptr, sv->GU, sv->h, S + S_H,
@@ -209,8 +210,9 @@ lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* sv, int64_t M
     const float* S = sv->scales;
     float* G = w.scales;
     if (cudaMemsetAsync(G, 0, 8 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
-    LM_TRY(lm_fp8_amax_scale_cast(dY, M, d, d, LM_FP8_E5M2, 0, nullptr, G + S_DY, G + S_DY + 1,
-                                  G + S_DY + 2, w.dYq, w.dYqT, stream));
+    const CastItem dy = {dY, M, d, d, nullptr, G + S_DY, G + S_DY + 1, G + S_DY + 2, w.dYq,
+                         w.dYqT};
+    LM_TRY(cast_set(&dy, 1, LM_FP8_E5M2, 0, true, s));  // slot zeroed above
     // g = dY W_down (plain bf16), dW_down = dY^T h
     LM_TRY(lm_fp8_gemm(w.dYq, LM_FP8_E5M2, sv->WdqT, LM_FP8_E4M3, M, f, d, G + S_DY + 2,
                        S + S_WD + 2, LM_EPI_NONE, nullptr, w.g, nullptr, stream));
