@@ -153,12 +153,13 @@ def job_tflops(world, steps, flops_per_step, total_ms):
     return world * steps * flops_per_step / (total_ms * 1e-3) / 1e12
 
 
-# algorithmic bytes of the cast launches of one step, in launch order:
-# full cast (amax pass + cast pass) = 2 B amax read + 2 B read + 1 B q + 1 B qT
-# per element; fused-amax cast = 2 B read + 1 B q + 1 B qT per element.
+# algorithmic bytes of the casts of one step (X, W_up, W_down, h, dY, dH):
+# full cast (amax pass + cast pass) = 2 B amax read + 2 B read + 1 B codes per
+# element; a cast whose amax came from a GEMM epilogue = 2 B read + 1 B codes.
+# Only row-major codes are written: the backward's GEMMs read them MN-major.
 def cast_bytes():
     Md, fd, Mf = M_TOK * D_MODEL, D_FF * D_MODEL, M_TOK * D_FF
-    return [6 * Md, 6 * fd, 6 * fd, 4 * Mf, 6 * Md, 4 * Mf]
+    return [5 * Md, 5 * fd, 5 * fd, 3 * Mf, 5 * Md, 3 * Mf]
 
 
 def src_sha(path):

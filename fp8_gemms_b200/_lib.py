@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(PKG, "libfp8lm.so")
 
 E4M3, E5M2 = 0, 1
 EPI_NONE, EPI_RELU2_FWD, EPI_RELU2_BWD, EPI_ACCUM_F32 = 0, 1, 2, 3
+GEMM_A_MN_MAJOR, GEMM_B_MN_MAJOR = 1, 2
 MLP_REUSE_WEIGHT_CASTS, MLP_ACCUMULATE_WGRAD = 1, 2
 
 STATUS = {0: "LM_OK", 1: "LM_ERR_INVALID_ARG", 2: "LM_ERR_ALIGNMENT",
@@ -28,7 +29,7 @@ EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
             "lm_selftest_bounded_wait", "lm_relu2_mlp_fwd_ex", "lm_relu2_mlp_bwd_ex",
             "lm_rmsnorm_fp8_cast", "lm_swiglu_mlp_saved_bytes", "lm_swiglu_mlp_saved_carve",
             "lm_swiglu_mlp_workspace_size", "lm_swiglu_mlp_fwd", "lm_swiglu_mlp_bwd",
-            "lm_fp8_lmhead_ce_workspace_size", "lm_fp8_lmhead_ce"]
+            "lm_fp8_lmhead_ce_workspace_size", "lm_fp8_lmhead_ce", "lm_fp8_gemm_ex"]
 
 
 class LmError(RuntimeError):
@@ -40,13 +41,13 @@ class LmError(RuntimeError):
 class MlpSaved(ctypes.Structure):
     """Mirror of lm_mlp_saved."""
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("Xq", "XqT", "Wuq", "WuqT", "Wdq", "WdqT", "H", "hq", "hqT", "scales")]
+                ("Xq", "Wuq", "Wdq", "H", "hq", "scales")]
 
 
 class SwigluSaved(ctypes.Structure):
     """Mirror of lm_swiglu_saved."""
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("Xq", "XqT", "Wguq", "WguqT", "Wdq", "WdqT", "GU", "h", "hq", "hqT", "scales")]
+                ("Xq", "Wguq", "Wdq", "GU", "h", "hq", "scales")]
 
 
 def _load():
@@ -58,6 +59,9 @@ def _load():
     L.lm_fp8_amax_scale_cast.restype = st
     L.lm_fp8_gemm.argtypes = [P, i32, P, i32, i64, i64, i64, P, P, i32, P, P, P, P]
     L.lm_fp8_gemm.restype = st
+    L.lm_fp8_gemm_ex.argtypes = [P, i32, P, i32, i64, i64, i64, ctypes.c_uint32, P, P, i32, P, P,
+                                 P, P]
+    L.lm_fp8_gemm_ex.restype = st
     L.lm_relu2_mlp_saved_bytes.argtypes = [i64, i64, i64]
     L.lm_relu2_mlp_saved_bytes.restype = ctypes.c_size_t
     L.lm_relu2_mlp_saved_carve.argtypes = [P, ctypes.c_size_t, i64, i64, i64,
@@ -159,6 +163,18 @@ def lm_fp8_gemm(A, fa, B, fb, inv_scale_a, inv_scale_b, D, epi=EPI_NONE, aux=Non
     assert K == K2 and tuple(D.shape) == (M, N)
     _check(lib.lm_fp8_gemm(_p(A), fa, _p(B), fb, M, N, K, _p(inv_scale_a), _p(inv_scale_b), epi,
                            _p(aux), _p(D), _p(amax_out), _stream(stream)), "lm_fp8_gemm")
+
+
+def lm_fp8_gemm_ex(A, fa, B, fb, inv_scale_a, inv_scale_b, D, flags=0, epi=EPI_NONE, aux=None,
+                   amax_out=None, stream=None):
+    """lm_fp8_gemm with per-operand storage: with GEMM_A_MN_MAJOR, A is given as
+    its [K x M] transpose (row-major); with GEMM_B_MN_MAJOR, B as [K x N]."""
+    M, K = (A.shape[1], A.shape[0]) if flags & GEMM_A_MN_MAJOR else tuple(A.shape)
+    N, K2 = (B.shape[1], B.shape[0]) if flags & GEMM_B_MN_MAJOR else tuple(B.shape)
+    assert K == K2 and tuple(D.shape) == (M, N)
+    _check(lib.lm_fp8_gemm_ex(_p(A), fa, _p(B), fb, M, N, K, flags, _p(inv_scale_a),
+                              _p(inv_scale_b), epi, _p(aux), _p(D), _p(amax_out), _stream(stream)),
+           "lm_fp8_gemm_ex")
 
 
 def lm_rmsnorm_fp8_cast(R, weight, X, fmt, amax_out, scale_out, inv_scale_out, q=None, qT=None,

@@ -10,7 +10,8 @@ import torch
 
 from . import _lib
 from ._lib import (E4M3, E5M2, EPI_ACCUM_F32, EPI_NONE, EPI_RELU2_BWD,  # noqa: F401
-                   EPI_RELU2_FWD, MLP_ACCUMULATE_WGRAD, MLP_REUSE_WEIGHT_CASTS, LmError)
+                   EPI_RELU2_FWD, GEMM_A_MN_MAJOR, GEMM_B_MN_MAJOR, MLP_ACCUMULATE_WGRAD,
+                   MLP_REUSE_WEIGHT_CASTS, LmError)
 
 
 def _dev(t):
@@ -37,12 +38,15 @@ def cast(x, fmt, relu2_input=False, amax_in=None, want_q=True, want_qT=True, sca
 
 
 def gemm(A, fa, B, fb, inv_a, inv_b, epi=EPI_NONE, aux=None, amax_out=None, out=None,
-         stream=None):
-    """bf16 D[M x N] = epi(A B^T inv_a inv_b) for K-major FP8 codes A, B."""
-    M, N = A.shape[0], B.shape[0]
+         flags=0, stream=None):
+    """bf16 D[M x N] = epi(A B^T inv_a inv_b) for FP8 codes A [M x K], B [N x K];
+    with GEMM_A_MN_MAJOR / GEMM_B_MN_MAJOR in flags, A is given as [K x M] /
+    B as [K x N] (the row-major codes of the transpose)."""
+    M = A.shape[1] if flags & GEMM_A_MN_MAJOR else A.shape[0]
+    N = B.shape[1] if flags & GEMM_B_MN_MAJOR else B.shape[0]
     D = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=_dev(A))
-    _lib.lm_fp8_gemm(A, fa, B, fb, inv_a, inv_b, D, epi=epi, aux=aux, amax_out=amax_out,
-                     stream=stream)
+    _lib.lm_fp8_gemm_ex(A, fa, B, fb, inv_a, inv_b, D, flags=flags, epi=epi, aux=aux,
+                        amax_out=amax_out, stream=stream)
     return D
 
 
@@ -97,8 +101,7 @@ class Relu2Mlp:
     # views of the saved tensors (for inspection and stagewise checks)
     def view(self, name):
         M, d, f = self.M, self.d, self.f
-        shapes = {"Xq": (M, d), "XqT": (d, M), "Wuq": (f, d), "WuqT": (d, f), "Wdq": (d, f),
-                  "WdqT": (f, d), "hq": (M, f), "hqT": (f, M)}
+        shapes = {"Xq": (M, d), "Wuq": (f, d), "Wdq": (d, f), "hq": (M, f)}
         base = self.saved_buf.data_ptr()
         if name == "H":
             off = self.saved.H - base
@@ -111,12 +114,11 @@ class Relu2Mlp:
         return self.saved_buf[off:off + r * c].view(r, c)
 
     def workspace_view(self, name):
-        """Backward scratch: dYq, dYqT, dH, dHq, dHqT, scales (library layout:
-        each buffer rounded up to 256 bytes, in that order)."""
+        """Backward scratch: dYq, dH, dHq, scales (library layout: each buffer
+        rounded up to 256 bytes, in that order)."""
         M, d, f = self.M, self.d, self.f
         r256 = lambda n: (n + 255) // 256 * 256
-        sizes = [("dYq", M * d), ("dYqT", M * d), ("dH", M * f * 2), ("dHq", M * f),
-                 ("dHqT", M * f), ("scales", 32)]
+        sizes = [("dYq", M * d), ("dH", M * f * 2), ("dHq", M * f), ("scales", 32)]
         off = 0
         for n, sz in sizes:
             if n == name:
@@ -125,8 +127,7 @@ class Relu2Mlp:
                     return v.view(torch.bfloat16).view(M, f)
                 if n == "scales":
                     return v.view(torch.float32).view(2, 4)
-                return v.view(*{"dYq": (M, d), "dYqT": (d, M), "dHq": (M, f),
-                                "dHqT": (f, M)}[n])
+                return v.view(*{"dYq": (M, d), "dHq": (M, f)}[n])
             off += r256(sz)
         raise KeyError(name)
 
@@ -177,7 +178,7 @@ class SwigluMlp:
         return dX, dW_gu, dW_down
 
     def view(self, name):
-        """Saved tensors: Xq, Wguq, GU, h, hq, hqT, scales (library layout)."""
+        """Saved tensors: Xq, Wguq, Wdq, GU, h, hq, scales (library layout)."""
         M, d, f = self.M, self.d, self.f
         base = self.saved_buf.data_ptr()
         off = getattr(self.saved, name) - base
@@ -186,8 +187,7 @@ class SwigluMlp:
             return self.saved_buf[off:off + M * cols * 2].view(torch.bfloat16).view(M, cols)
         if name == "scales":
             return self.saved_buf[off:off + 64].view(torch.float32).view(4, 4)
-        shape = {"Xq": (M, d), "XqT": (d, M), "Wguq": (2 * f, d), "WguqT": (d, 2 * f),
-                 "Wdq": (d, f), "WdqT": (f, d), "hq": (M, f), "hqT": (f, M)}[name]
+        shape = {"Xq": (M, d), "Wguq": (2 * f, d), "Wdq": (d, f), "hq": (M, f)}[name]
         return self.saved_buf[off:off + shape[0] * shape[1]].view(*shape)
 
 
@@ -221,13 +221,15 @@ class LmHeadCE:
 
 def linear_fwd_bwd(X, W, dY, stream=None):
     """Plain linear Y = X W^T with its dgrad and wgrad, all in FP8: X, W cast
-    to e4m3 and dY to e5m2 (each with its K-major transposed copy), then
-    Y = Xq Wq^T, dX = dYq (Wq^T)^T, dW = (dYq^T)(Xq^T)^T.  Returns (Y, dX, dW)."""
+    to e4m3 and dY to e5m2 (row-major codes only), then Y = Xq Wq^T,
+    dX = dYq W (Wq read MN-major), dW = dY^T X (dYq and Xq read MN-major).
+    Returns (Y, dX, dW, intermediates)."""
     sc = new_scales(X.device, 3)
-    Xq, XqT, _ = cast(X, E4M3, scales=sc[0], stream=stream)
-    Wq, WqT, _ = cast(W, E4M3, scales=sc[1], stream=stream)
-    dYq, dYqT, _ = cast(dY, E5M2, scales=sc[2], stream=stream)
+    Xq, _, _ = cast(X, E4M3, want_qT=False, scales=sc[0], stream=stream)
+    Wq, _, _ = cast(W, E4M3, want_qT=False, scales=sc[1], stream=stream)
+    dYq, _, _ = cast(dY, E5M2, want_qT=False, scales=sc[2], stream=stream)
     Y = gemm(Xq, E4M3, Wq, E4M3, sc[0, 2:3], sc[1, 2:3], stream=stream)
-    dX = gemm(dYq, E5M2, WqT, E4M3, sc[2, 2:3], sc[1, 2:3], stream=stream)
-    dW = gemm(dYqT, E5M2, XqT, E4M3, sc[2, 2:3], sc[0, 2:3], stream=stream)
-    return Y, dX, dW, dict(Xq=Xq, XqT=XqT, Wq=Wq, WqT=WqT, dYq=dYq, dYqT=dYqT, scales=sc)
+    dX = gemm(dYq, E5M2, Wq, E4M3, sc[2, 2:3], sc[1, 2:3], flags=GEMM_B_MN_MAJOR, stream=stream)
+    dW = gemm(dYq, E5M2, Xq, E4M3, sc[2, 2:3], sc[0, 2:3],
+              flags=GEMM_A_MN_MAJOR | GEMM_B_MN_MAJOR, stream=stream)
+    return Y, dX, dW, dict(Xq=Xq, Wq=Wq, dYq=dYq, scales=sc)

@@ -246,10 +246,11 @@ __global__ void __launch_bounds__(kThreads) cast_kernel(
 
 
 // Pass 2, TMA-fed: a persistent kernel, two CTAs per SM.  Warp 8 streams
-// 128 x 128 bf16 tiles (32 KB) into a 2-stage shared ring with TMA; warps
-// 0-7 convert each tile (16-byte shared loads; 8-byte stores of the
-// row-major codes straight to q) and build its transpose in shared memory,
-// which one thread writes to qT with a single TMA store per tile.
+// 128 x 128 bf16 tiles (32 KB) into a shared ring with TMA; warps 0-7 convert
+// each tile (16-byte shared loads; 8-byte stores of the row-major codes
+// straight to q).  The TRANS instantiation (2 stages) also builds each
+// tile's transpose in shared memory, which one thread writes to qT with a
+// single TMA store; without it the ring has 3 stages.
 //  - codes tile: word w of tile row r sits at r*32 + (w ^ 4*((r >> 4) & 7)),
 //    so both the row-major writes and the column-quad reads of the
 //    transpose are free of bank conflicts;
@@ -261,12 +262,17 @@ __global__ void __launch_bounds__(kThreads) cast_kernel(
 // waiting but keeps the loop's barrier sequence, so no barrier can hang.
 namespace tmac {
 constexpr int TR = 128, TC = 128;
-constexpr int STAGES = 2;
 constexpr int IN_BYTES = TR * TC * 2;
 constexpr int CODE_BYTES = TR * TC;
 constexpr int CONSUMERS = 256;
 constexpr int THREADS = CONSUMERS + 32;
-constexpr int SMEM = 1024 + CODE_BYTES + STAGES * IN_BYTES + CODE_BYTES + 64;
+// With transposes: 2 input stages plus the codes and transposed tiles.
+// Without (row-major codes only): the same shared memory holds 3 stages.
+// Either way two CTAs fit on an SM.
+__host__ __device__ constexpr int stages(bool trans) { return trans ? 2 : 3; }
+__host__ __device__ constexpr int smem_bytes(bool trans) {
+    return 1024 + (trans ? 2 * CODE_BYTES : 0) + stages(trans) * IN_BYTES + 64;
+}
 enum : unsigned { W_CAST_EMPTY = 0x201, W_CAST_FULL = 0x202, W_CAST_LOADS = 0x203 };
 }  // namespace tmac
 
@@ -294,20 +300,22 @@ __device__ __forceinline__ int set_member(const CastSet& set, int t) {
     return t < set.tile_end[0] ? 0 : (t < set.tile_end[1] ? 1 : 2);
 }
 
-template <int FMT, bool RELU2>
+template <int FMT, bool RELU2, bool TRANS>
 __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
     const __grid_constant__ CUtensorMap tmX0, const __grid_constant__ CUtensorMap tmX1,
     const __grid_constant__ CUtensorMap tmX2, const __grid_constant__ CUtensorMap tmQT0,
     const __grid_constant__ CUtensorMap tmQT1, const __grid_constant__ CUtensorMap tmQT2,
     const CastSet set, unsigned int* err) {
     using namespace tmac;
+    constexpr int STAGES = stages(TRANS);
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-    uint8_t* sT = smem;                         // transposed codes, 1024-aligned
-    uint8_t* sIn = smem + CODE_BYTES;           // STAGES x 32 KB
+    uint8_t* sT = smem;                                   // transposed codes, 1024-aligned
+    uint8_t* sIn = smem + (TRANS ? CODE_BYTES : 0);       // STAGES x 32 KB
     uint32_t* sCode = reinterpret_cast<uint32_t*>(sIn + STAGES * IN_BYTES);  // [TR][TC/4]
-    uint64_t* full = reinterpret_cast<uint64_t*>(sIn + STAGES * IN_BYTES + CODE_BYTES);
+    uint64_t* full =
+        reinterpret_cast<uint64_t*>(sIn + STAGES * IN_BYTES + (TRANS ? CODE_BYTES : 0));
     uint64_t* empty = full + STAGES;
 
     const float fmax = FMT == LM_FP8_E4M3 ? 448.0f : 57344.0f;
@@ -381,8 +389,10 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
             const int r = r0 + rr, c = c0 + ch * 8;
             if (q && r < rows && c < cols)
                 *reinterpret_cast<uint2*>(q + (int64_t)r * cols + c) = codes;
-            const int wpos = (2 * ch) ^ (4 * ((rr >> 4) & 7));
-            *reinterpret_cast<uint2*>(&sCode[rr * (TC / 4) + wpos]) = codes;
+            if (TRANS) {
+                const int wpos = (2 * ch) ^ (4 * ((rr >> 4) & 7));
+                *reinterpret_cast<uint2*>(&sCode[rr * (TC / 4) + wpos]) = codes;
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
@@ -390,7 +400,7 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
             s = 0;
             ph ^= 1u;
         }
-        if (!((set.want_qT >> j) & 1)) continue;
+        if (!TRANS || !((set.want_qT >> j) & 1)) continue;
         if (tid == 0) bulk_wait_group_read<0>();  // the previous tile's store has read sT
         consumers_sync();                           // codes tile complete, sT free
         // lane: tile rows [16k, 16k+16) with k = lane % 8; tile columns
@@ -427,20 +437,32 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
     if (tid == 0) bulk_wait_group<0>();
 }
 
-// TMA-fed cast of the items (each with rows % 16 == 0) in one launch.
-template <int FMT, bool RELU2>
-lm_status launch_cast_tma(const CastItem* const* items, const float* const* amax_src, int n,
-                          cudaStream_t s) {
+// One launch of the TMA-fed cast kernel (with or without its transpose stage).
+template <int FMT, bool RELU2, bool TRANS>
+lm_status launch_cast_tma_kernel(const CUtensorMap (&tx)[kMaxSet],
+                                 const CUtensorMap (&tq)[kMaxSet], const CastSet& set, int grid,
+                                 unsigned int* err, cudaStream_t s) {
     static bool configured[64] = {};
+    constexpr int smem = tmac::smem_bytes(TRANS);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LM_ERR_CUDA;
     if (!configured[dev]) {
-        if (cudaFuncSetAttribute(cast_tma_kernel<FMT, RELU2>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tmac::SMEM) != cudaSuccess)
+        if (cudaFuncSetAttribute(cast_tma_kernel<FMT, RELU2, TRANS>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return LM_ERR_CUDA;
         configured[dev] = true;
     }
+    timing_mark(s, 'c');
+    cast_tma_kernel<FMT, RELU2, TRANS><<<grid, tmac::THREADS, smem, s>>>(
+        tx[0], tx[1], tx[2], tq[0], tq[1], tq[2], set, err);
+    return launch_status();
+}
+
+// TMA-fed cast of the items (each with rows % 16 == 0) in one launch; the
+// kernel without the transpose stage when no item wants qT.
+template <int FMT, bool RELU2>
+lm_status launch_cast_tma(const CastItem* const* items, const float* const* amax_src, int n,
+                          cudaStream_t s) {
     CUtensorMap tx[kMaxSet], tq[kMaxSet];
     CastSet set = {};
     set.n = n;
@@ -482,10 +504,8 @@ lm_status launch_cast_tma(const CastItem* const* items, const float* const* amax
     int grid = 2 * sm_count();
     if (grid <= 0) return LM_ERR_CUDA;
     if (grid > total) grid = total;
-    timing_mark(s, 'c');
-    cast_tma_kernel<FMT, RELU2><<<grid, tmac::THREADS, tmac::SMEM, s>>>(tx[0], tx[1], tx[2], tq[0],
-                                                                        tq[1], tq[2], set, err);
-    return launch_status();
+    return set.want_qT ? launch_cast_tma_kernel<FMT, RELU2, true>(tx, tq, set, grid, err, s)
+                       : launch_cast_tma_kernel<FMT, RELU2, false>(tx, tq, set, grid, err, s);
 }
 
 // One tensor with rows % 16 != 0 (row-major codes only): one block per tile.

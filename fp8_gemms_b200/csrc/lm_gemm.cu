@@ -44,6 +44,7 @@ enum : unsigned {
 
 struct GemmArgs {
     int M, N, num_mb, num_nb, num_kb, num_tiles, group_m;
+    int a_mn, b_mn;  // 1: the operand is stored MN-major ([K x M] / [K x N], M or N contiguous)
     int stream_a;  // 1: A is the streamed operand (evict-first loads), 0: B is
     const float* inv_a;
     const float* inv_b;
@@ -264,6 +265,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const int arow = mb * TILE_M + (int)rank * 128;
                 const int brow = nb * TILE_N + (int)rank * 128;
                 for (int kb = 0; kb < args.num_kb; ++kb) {
+                    // box coordinates (x innermost): K-major (k, m|n), MN-major (m|n, k)
+                    const int ax = args.a_mn ? arow : kb * BK, ay = args.a_mn ? kb * BK : arow;
+                    const int bx = args.b_mn ? brow : kb * BK, by = args.b_mn ? kb * BK : brow;
                     if (!mbar_wait(&empty[stage], phase ^ 1u, args.err, W_EMPTY)) {
                         ok = false;
                         break;
@@ -271,13 +275,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
                     const uint32_t bar = full_leader + (uint32_t)(stage * 8);
                     if (args.stream_a) {
-                        tma_load_2d_pair_hint(smem_addr(sA + stage * A_BYTES), &tmA, bar, kb * BK,
-                                              arow, pol_a);
-                        tma_load_2d_pair(smem_addr(sB + stage * B_BYTES), &tmB, bar, kb * BK, brow);
+                        tma_load_2d_pair_hint(smem_addr(sA + stage * A_BYTES), &tmA, bar, ax, ay,
+                                              pol_a);
+                        tma_load_2d_pair(smem_addr(sB + stage * B_BYTES), &tmB, bar, bx, by);
                     } else {
-                        tma_load_2d_pair(smem_addr(sA + stage * A_BYTES), &tmA, bar, kb * BK, arow);
-                        tma_load_2d_pair_hint(smem_addr(sB + stage * B_BYTES), &tmB, bar, kb * BK,
-                                              brow, pol_b);
+                        tma_load_2d_pair(smem_addr(sA + stage * A_BYTES), &tmA, bar, ax, ay);
+                        tma_load_2d_pair_hint(smem_addr(sB + stage * B_BYTES), &tmB, bar, bx, by,
+                                              pol_b);
                     }
                     ++issued;
                     if (++stage == STAGES) {
@@ -302,6 +306,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
+            // descriptor advance (16-byte units) per UMMA_K: 32 bytes along a
+            // K-major row, or 32 rows of an MN-major tile
+            const uint64_t a_step = args.a_mn ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
+            const uint64_t b_step = args.b_mn ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
             for (int t = cluster; t < args.num_tiles && ok; t += nclusters) {
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.err, W_TEMPTY)) break;
                 tc_fence_after();
@@ -316,9 +324,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     const uint64_t bd = smem_desc_k128(smem_addr(sB + stage * B_BYTES));
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk)
-                        mma_fp8_pair(d_tmem, ad + (uint64_t)(kk * UMMA_K / 16),
-                                     bd + (uint64_t)(kk * UMMA_K / 16), args.idesc,
-                                     (kb | kk) != 0 ? 1u : 0u);
+                        mma_fp8_pair(d_tmem, ad + (uint64_t)kk * a_step, bd + (uint64_t)kk * b_step,
+                                     args.idesc, (kb | kk) != 0 ? 1u : 0u);
                     mma_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
                     if (++stage == STAGES) {
                         stage = 0;
@@ -519,6 +526,7 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK;
 constexpr int B_BYTES = BN * BK;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int B_MN_BLOCK = 128 * BK;  // one 128-wide block of an MN-major B tile
 constexpr int NUM_EPI_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
@@ -580,10 +588,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-                    tma_load_2d(smem_addr(sA + stage * A_BYTES), &tmA, &full[stage], kb * BK,
-                                mb * BM);
-                    tma_load_2d(smem_addr(sB + stage * B_BYTES), &tmB, &full[stage], kb * BK,
-                                nb * BN);
+                    if (args.a_mn)
+                        tma_load_2d(smem_addr(sA + stage * A_BYTES), &tmA, &full[stage], mb * BM,
+                                    kb * BK);
+                    else
+                        tma_load_2d(smem_addr(sA + stage * A_BYTES), &tmA, &full[stage], kb * BK,
+                                    mb * BM);
+                    if (args.b_mn) {
+                        // two 128-wide MN blocks, B_MN_BLOCK bytes apart
+                        for (int h = 0; h < BN / 128; ++h)
+                            tma_load_2d(smem_addr(sB + stage * B_BYTES + h * B_MN_BLOCK), &tmB,
+                                        &full[stage], nb * BN + h * 128, kb * BK);
+                    } else {
+                        tma_load_2d(smem_addr(sB + stage * B_BYTES), &tmB, &full[stage], kb * BK,
+                                    nb * BN);
+                    }
                     ++issued;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -603,6 +622,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
+            const uint64_t a_step = args.a_mn ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
+            const uint64_t b_step = args.b_mn ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
+            const uint32_t b_lbo = args.b_mn ? (uint32_t)B_MN_BLOCK : 16u;
             for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.err, W_TEMPTY)) break;
                 tc_fence_after();
@@ -614,12 +636,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                     tc_fence_after();
                     const uint64_t ad = smem_desc_k128(smem_addr(sA + stage * A_BYTES));
-                    const uint64_t bd = smem_desc_k128(smem_addr(sB + stage * B_BYTES));
+                    const uint64_t bd = smem_desc_sw128(smem_addr(sB + stage * B_BYTES), b_lbo);
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk)
-                        mma_fp8(d_tmem, ad + (uint64_t)(kk * UMMA_K / 16),
-                                bd + (uint64_t)(kk * UMMA_K / 16), args.idesc,
-                                (kb | kk) != 0 ? 1u : 0u);
+                        mma_fp8(d_tmem, ad + (uint64_t)kk * a_step, bd + (uint64_t)kk * b_step,
+                                args.idesc, (kb | kk) != 0 ? 1u : 0u);
                     mma_commit(&empty[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
@@ -757,7 +778,7 @@ lm_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArg
 }  // namespace lm
 
 lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
-                            lm_fp8_format fb, int64_t M, int64_t N, int64_t K,
+                            lm_fp8_format fb, int64_t M, int64_t N, int64_t K, uint32_t flags,
                             const float* inv_scale_a, const float* inv_scale_b, int epi,
                             const void* aux, void* D, void* D2, float* amax_out,
                             lm_stream_t stream) {
@@ -774,7 +795,11 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
     if (K > 0 && (!A || !B)) return LM_ERR_INVALID_ARG;
     if (epi == LM_EPI_RELU2_BWD && !aux) return LM_ERR_INVALID_ARG;
     if (epi == kEpiSwigluFwd && (!D2 || N % 256 != 0 || K == 0)) return LM_ERR_INVALID_ARG;
+    if (flags & ~(LM_GEMM_A_MN_MAJOR | LM_GEMM_B_MN_MAJOR)) return LM_ERR_INVALID_ARG;
+    const bool a_mn = (flags & LM_GEMM_A_MN_MAJOR) != 0, b_mn = (flags & LM_GEMM_B_MN_MAJOR) != 0;
     if (K % 16 != 0 || N % 8 != 0) return LM_ERR_UNSUPPORTED_SHAPE;
+    // an MN-major operand's rows (one per K) must start on 16-byte boundaries
+    if ((a_mn && M % 16 != 0) || (b_mn && N % 16 != 0)) return LM_ERR_UNSUPPORTED_SHAPE;
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
         return LM_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(aux) || !aligned16(D2))
@@ -802,6 +827,8 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
     if (epi == LM_EPI_ACCUM_F32) a.amax_out = nullptr;
     a.amax_out = amax_out;
     a.err = err;
+    a.a_mn = a_mn ? 1 : 0;
+    a.b_mn = b_mn ? 1 : 0;
 
     CUtensorMap ta, tb;
     if (M > 128 || epi == kEpiSwigluFwd) {
@@ -815,11 +842,16 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
         // spanning M).
         a.stream_a = N <= M ? 1 : 0;
         a.group_m = a.stream_a ? 1 : a.num_mb;
-        a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, pair::TILE_M, pair::TILE_N);
+        a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, pair::TILE_M, pair::TILE_N, a.a_mn, a.b_mn);
         CUtensorMap td, tx;
-        if (!encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, 128, BK) ||
-            !encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, 128, BK))
-            return LM_ERR_CUDA;
+        // K-major: [rows x K] boxes of 128 rows x 128 K; MN-major: [K x cols]
+        // boxes of 128 K x 128 columns
+        const bool mok =
+            (a_mn ? encode_tmap_u8(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)M, BK, 128)
+                  : encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, 128, BK)) &&
+            (b_mn ? encode_tmap_u8(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)N, BK, 128)
+                  : encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, 128, BK));
+        if (!mok) return LM_ERR_CUDA;
         const bool dok = epi == LM_EPI_ACCUM_F32
                              ? encode_tmap_f32_sw128(&td, D, (uint64_t)M, (uint64_t)N, 32,
                                                      pair::EPI_COLS)
@@ -852,10 +884,13 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
     a.num_tiles = a.num_mb * a.num_nb;
     a.group_m = 16;
     a.stream_a = 0;
-    a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, one::BM, one::BN);
-    if (!encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, one::BM, BK) ||
-        !encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, one::BN, BK))
-        return LM_ERR_CUDA;
+    a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, one::BM, one::BN, a.a_mn, a.b_mn);
+    const bool mok =
+        (a_mn ? encode_tmap_u8(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)M, BK, one::BM)
+              : encode_tmap_u8(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)K, one::BM, BK)) &&
+        (b_mn ? encode_tmap_u8(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)N, BK, 128)
+              : encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, one::BN, BK));
+    if (!mok) return LM_ERR_CUDA;
     switch (epi) {
         case LM_EPI_NONE: return launch_one<LM_EPI_NONE>(ta, tb, a, s);
         case LM_EPI_RELU2_FWD: return launch_one<LM_EPI_RELU2_FWD>(ta, tb, a, s);
@@ -864,14 +899,23 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
     }
 }
 
+extern "C" lm_status lm_fp8_gemm_ex(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
+                                    lm_fp8_format fb, int64_t M, int64_t N, int64_t K,
+                                    uint32_t flags, const float* inv_scale_a,
+                                    const float* inv_scale_b, lm_epilogue epi, const void* aux,
+                                    void* D, float* amax_out, lm_stream_t stream) {
+    if (epi != LM_EPI_NONE && epi != LM_EPI_RELU2_FWD && epi != LM_EPI_RELU2_BWD &&
+        epi != LM_EPI_ACCUM_F32)
+        return LM_ERR_UNSUPPORTED_FORMAT;
+    return lm::gemm_dispatch(A, fa, B, fb, M, N, K, flags, inv_scale_a, inv_scale_b, (int)epi,
+                             aux, D, nullptr, amax_out, stream);
+}
+
 extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
                                  lm_fp8_format fb, int64_t M, int64_t N, int64_t K,
                                  const float* inv_scale_a, const float* inv_scale_b,
                                  lm_epilogue epi, const void* aux, void* D, float* amax_out,
                                  lm_stream_t stream) {
-    if (epi != LM_EPI_NONE && epi != LM_EPI_RELU2_FWD && epi != LM_EPI_RELU2_BWD &&
-        epi != LM_EPI_ACCUM_F32)
-        return LM_ERR_UNSUPPORTED_FORMAT;
-    return lm::gemm_dispatch(A, fa, B, fb, M, N, K, inv_scale_a, inv_scale_b, (int)epi, aux, D,
-                             nullptr, amax_out, stream);
+    return lm_fp8_gemm_ex(A, fa, B, fb, M, N, K, 0u, inv_scale_a, inv_scale_b, epi, aux, D,
+                          amax_out, stream);
 }

@@ -48,7 +48,7 @@ constexpr int kEpiSwigluFwd = 4;
 
 // lm_fp8_gemm with the internal epilogues and a second output.
 lm_status gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B, lm_fp8_format fb,
-                        int64_t M, int64_t N, int64_t K, const float* inv_scale_a,
+                        int64_t M, int64_t N, int64_t K, uint32_t flags, const float* inv_scale_a,
                         const float* inv_scale_b, int epi, const void* aux, void* D, void* D2,
                         float* amax_out, lm_stream_t stream);
 

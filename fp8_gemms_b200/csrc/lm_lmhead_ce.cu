@@ -29,7 +29,7 @@ constexpr int kCeThreads = 512;
 
 struct Ws {
     float* scales;  // {amax, scale, inv, 0} for X, W, dlogits
-    uint8_t *Wq, *WqT, *Xq, *XqT, *dLq, *dLqT;
+    uint8_t *Wq, *Xq, *dLq;
     uint16_t* logits;
     float* loss_rows;
 };
@@ -44,12 +44,9 @@ size_t layout(int64_t M, int64_t d, int64_t V, int64_t C, uint8_t* base, Ws* w) 
     Ws o;
     o.scales = reinterpret_cast<float*>(take(16 * sizeof(float)));
     o.Wq = take((size_t)V * d);
-    o.WqT = take((size_t)V * d);
     o.Xq = take((size_t)C * d);
-    o.XqT = take((size_t)C * d);
     o.logits = reinterpret_cast<uint16_t*>(take((size_t)C * V * 2));
     o.dLq = take((size_t)C * V);
-    o.dLqT = take((size_t)C * V);
     o.loss_rows = reinterpret_cast<float*>(take((size_t)M * sizeof(float)));
     if (w) *w = o;
     return off;
@@ -220,7 +217,7 @@ lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* labels, 
     if (cudaMemsetAsync(w.scales, 0, 16 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
     // W cast, and X's amax and scale over the whole tensor (no codes yet), with
     // one amax launch for both (slots zeroed above)
-    const CastItem in[2] = {{W, V, d, d, nullptr, SW, SW + 1, SW + 2, w.Wq, w.WqT},
+    const CastItem in[2] = {{W, V, d, d, nullptr, SW, SW + 1, SW + 2, w.Wq, nullptr},
                             {X, M, d, d, nullptr, SX, SX + 1, SX + 2, nullptr, nullptr}};
     LM_TRY(cast_set(in, 2, LM_FP8_E4M3, 0, true, s));
     const uint16_t* Xb = static_cast<const uint16_t*>(X);
@@ -228,7 +225,7 @@ lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* labels, 
     for (int64_t c0 = 0; c0 < M; c0 += chunk) {
         const int64_t rows = (M - c0) < chunk ? (M - c0) : chunk;
         LM_TRY(lm_fp8_amax_scale_cast(Xb + c0 * d, rows, d, d, LM_FP8_E4M3, 0, SX, SX, SX + 1,
-                                      SX + 2, w.Xq, w.XqT, stream));
+                                      SX + 2, w.Xq, nullptr, stream));
         LM_TRY(lm_fp8_gemm(w.Xq, LM_FP8_E4M3, w.Wq, LM_FP8_E4M3, rows, V, d, SX + 2, SW + 2,
                            LM_EPI_NONE, nullptr, w.logits, nullptr, stream));
         if (cudaMemsetAsync(SL, 0, 4 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
@@ -238,11 +235,14 @@ lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* labels, 
             reinterpret_cast<unsigned int*>(SL), err);
         if (launch_status() != LM_OK) return LM_ERR_CUDA;
         LM_TRY(lm_fp8_amax_scale_cast(w.logits, rows, V, V, LM_FP8_E5M2, 0, SL, SL, SL + 1,
-                                      SL + 2, w.dLq, w.dLqT, stream));
-        LM_TRY(lm_fp8_gemm(w.dLq, LM_FP8_E5M2, w.WqT, LM_FP8_E4M3, rows, d, V, SL + 2, SW + 2,
-                           LM_EPI_NONE, nullptr, dXb + c0 * d, nullptr, stream));
-        LM_TRY(lm_fp8_gemm(w.dLqT, LM_FP8_E5M2, w.XqT, LM_FP8_E4M3, V, d, rows, SL + 2, SX + 2,
-                           LM_EPI_ACCUM_F32, nullptr, dW, nullptr, stream));
+                                      SL + 2, w.dLq, nullptr, stream));
+        // dX = dL W (W [V x d] read MN-major); dW += dL^T X (both read MN-major)
+        LM_TRY(lm_fp8_gemm_ex(w.dLq, LM_FP8_E5M2, w.Wq, LM_FP8_E4M3, rows, d, V,
+                              LM_GEMM_B_MN_MAJOR, SL + 2, SW + 2, LM_EPI_NONE, nullptr,
+                              dXb + c0 * d, nullptr, stream));
+        LM_TRY(lm_fp8_gemm_ex(w.dLq, LM_FP8_E5M2, w.Xq, LM_FP8_E4M3, V, d, rows,
+                              LM_GEMM_A_MN_MAJOR | LM_GEMM_B_MN_MAJOR, SL + 2, SX + 2,
+                              LM_EPI_ACCUM_F32, nullptr, dW, nullptr, stream));
     }
     timing_mark(s, 'l');
     mean_loss_kernel<<<1, 1024, 0, s>>>(w.loss_rows, M, loss_out);

@@ -25,7 +25,7 @@ enum { S_X = 0, S_WU = 4, S_WD = 8, S_H = 12 };  // in lm_mlp_saved::scales
 enum { S_DY = 0, S_DH = 4 };                      // in the backward workspace
 
 struct BwdWorkspace {
-    uint8_t *dYq, *dYqT, *dHq, *dHqT;
+    uint8_t *dYq, *dHq;
     void* dH;
     float* scales;
 };
@@ -39,12 +39,10 @@ size_t bwd_layout(int64_t M, int64_t d, int64_t f, uint8_t* base, BwdWorkspace* 
         return p;
     };
     uint8_t* dYq = take(Md);
-    uint8_t* dYqT = take(Md);
     uint8_t* dH = take(Mf * 2);
     uint8_t* dHq = take(Mf);
-    uint8_t* dHqT = take(Mf);
     uint8_t* sc = take(8 * sizeof(float));
-    if (w) *w = BwdWorkspace{dYq, dYqT, dHq, dHqT, dH, reinterpret_cast<float*>(sc)};
+    if (w) *w = BwdWorkspace{dYq, dHq, dH, reinterpret_cast<float*>(sc)};
     return off;
 }
 
@@ -59,14 +57,10 @@ size_t saved_layout(int64_t M, int64_t d, int64_t f, uint8_t* base, lm_mlp_saved
     };
     lm_mlp_saved o;
     o.Xq = take(Md);
-    o.XqT = take(Md);
     o.Wuq = take(fd);
-    o.WuqT = take(fd);
     o.Wdq = take(fd);
-    o.WdqT = take(fd);
     o.H = take(Mf * 2);
     o.hq = take(Mf);
-    o.hqT = take(Mf);
     o.scales = reinterpret_cast<float*>(take(16 * sizeof(float)));
     if (s) *s = o;
     return off;
@@ -109,8 +103,7 @@ lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_dow
     if (flags & ~LM_MLP_REUSE_WEIGHT_CASTS) return LM_ERR_INVALID_ARG;
     const bool reuse = (flags & LM_MLP_REUSE_WEIGHT_CASTS) != 0;
     if (!X || !Y || !sv || (!reuse && (!W_up || !W_down))) return LM_ERR_INVALID_ARG;
-    if (!sv->Xq || !sv->XqT || !sv->Wuq || !sv->WuqT || !sv->Wdq || !sv->WdqT || !sv->H ||
-        !sv->hq || !sv->hqT || !sv->scales)
+    if (!sv->Xq || !sv->Wuq || !sv->Wdq || !sv->H || !sv->hq || !sv->scales)
         return LM_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     float* S = sv->scales;
@@ -122,17 +115,18 @@ lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_dow
         return LM_ERR_CUDA;
     }
     // X, W_up and W_down (or X alone): one amax launch and one cast launch;
-    // their amax slots were zeroed above
+    // their amax slots were zeroed above.  Row-major codes only: the
+    // backward reads them MN-major where it needs the transpose.
     const lm::CastItem in[3] = {
-        {X, M, d, d, nullptr, S + S_X, S + S_X + 1, S + S_X + 2, sv->Xq, sv->XqT},
-        {W_up, f, d, d, nullptr, S + S_WU, S + S_WU + 1, S + S_WU + 2, sv->Wuq, sv->WuqT},
-        {W_down, d, f, f, nullptr, S + S_WD, S + S_WD + 1, S + S_WD + 2, sv->Wdq, sv->WdqT}};
+        {X, M, d, d, nullptr, S + S_X, S + S_X + 1, S + S_X + 2, sv->Xq, nullptr},
+        {W_up, f, d, d, nullptr, S + S_WU, S + S_WU + 1, S + S_WU + 2, sv->Wuq, nullptr},
+        {W_down, d, f, f, nullptr, S + S_WD, S + S_WD + 1, S + S_WD + 2, sv->Wdq, nullptr}};
     LM_TRY(lm::cast_set(in, reuse ? 1 : 3, LM_FP8_E4M3, 0, true, s));
     // H = X W_up^T (bf16) and amax of h = bf16(relu(H)^2)
     LM_TRY(lm_fp8_gemm(sv->Xq, LM_FP8_E4M3, sv->Wuq, LM_FP8_E4M3, M, f, d, S + S_X + 2,
                        S + S_WU + 2, LM_EPI_RELU2_FWD, nullptr, sv->H, S + S_H, stream));
     LM_TRY(lm_fp8_amax_scale_cast(sv->H, M, f, f, LM_FP8_E4M3, 1, S + S_H, S + S_H, S + S_H + 1,
-                                  S + S_H + 2, sv->hq, sv->hqT, stream));
+                                  S + S_H + 2, sv->hq, nullptr, stream));
     // Y = h W_down^T
     LM_TRY(lm_fp8_gemm(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, S + S_H + 2,
                        S + S_WD + 2, LM_EPI_NONE, nullptr, Y, nullptr, stream));
@@ -164,21 +158,23 @@ lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* sv, int64_t M,
     float* G = w.scales;
     if (cudaMemsetAsync(G, 0, 8 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
     const lm::CastItem dy = {dY, M, d, d, nullptr, G + S_DY, G + S_DY + 1, G + S_DY + 2,
-                             w.dYq, w.dYqT};
+                             w.dYq, nullptr};
     LM_TRY(lm::cast_set(&dy, 1, LM_FP8_E5M2, 0, true, s));  // slot zeroed above
-    // dH = bf16(bf16(dY W_down) * 2 relu(H)), and its amax
-    LM_TRY(lm_fp8_gemm(w.dYq, LM_FP8_E5M2, sv->WdqT, LM_FP8_E4M3, M, f, d, G + S_DY + 2,
-                       S + S_WD + 2, LM_EPI_RELU2_BWD, sv->H, w.dH, G + S_DH, stream));
-    // dW_down = dY^T h (K = M)
-    LM_TRY(lm_fp8_gemm(w.dYqT, LM_FP8_E5M2, sv->hqT, LM_FP8_E4M3, d, f, M, G + S_DY + 2,
-                       S + S_H + 2, wgrad_epi, nullptr, dW_down, nullptr, stream));
+    constexpr uint32_t B_MN = LM_GEMM_B_MN_MAJOR, AB_MN = LM_GEMM_A_MN_MAJOR | LM_GEMM_B_MN_MAJOR;
+    // dH = bf16(bf16(dY W_down) * 2 relu(H)), and its amax; B = W_down [d x f]
+    // read MN-major as the [f x d] operand
+    LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->Wdq, LM_FP8_E4M3, M, f, d, B_MN, G + S_DY + 2,
+                          S + S_WD + 2, LM_EPI_RELU2_BWD, sv->H, w.dH, G + S_DH, stream));
+    // dW_down = dY^T h (K = M): dY [M x d] and h [M x f] read MN-major
+    LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->hq, LM_FP8_E4M3, d, f, M, AB_MN, G + S_DY + 2,
+                          S + S_H + 2, wgrad_epi, nullptr, dW_down, nullptr, stream));
     LM_TRY(lm_fp8_amax_scale_cast(w.dH, M, f, f, LM_FP8_E5M2, 0, G + S_DH, G + S_DH,
-                                  G + S_DH + 1, G + S_DH + 2, w.dHq, w.dHqT, stream));
-    // dX = dH W_up;  dW_up = dH^T X (K = M)
-    LM_TRY(lm_fp8_gemm(w.dHq, LM_FP8_E5M2, sv->WuqT, LM_FP8_E4M3, M, d, f, G + S_DH + 2,
-                       S + S_WU + 2, LM_EPI_NONE, nullptr, dX, nullptr, stream));
-    LM_TRY(lm_fp8_gemm(w.dHqT, LM_FP8_E5M2, sv->XqT, LM_FP8_E4M3, f, d, M, G + S_DH + 2,
-                       S + S_X + 2, wgrad_epi, nullptr, dW_up, nullptr, stream));
+                                  G + S_DH + 1, G + S_DH + 2, w.dHq, nullptr, stream));
+    // dX = dH W_up (W_up [f x d] read MN-major);  dW_up = dH^T X (K = M)
+    LM_TRY(lm_fp8_gemm_ex(w.dHq, LM_FP8_E5M2, sv->Wuq, LM_FP8_E4M3, M, d, f, B_MN, G + S_DH + 2,
+                          S + S_WU + 2, LM_EPI_NONE, nullptr, dX, nullptr, stream));
+    LM_TRY(lm_fp8_gemm_ex(w.dHq, LM_FP8_E5M2, sv->Xq, LM_FP8_E4M3, f, d, M, AB_MN, G + S_DH + 2,
+                          S + S_X + 2, wgrad_epi, nullptr, dW_up, nullptr, stream));
     return LM_OK;
 }
 

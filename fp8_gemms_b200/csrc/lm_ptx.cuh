@@ -160,29 +160,41 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // ------------------------------------------------- descriptors (sm_100)
-// Shared-memory matrix descriptor for a K-major operand tile stored in the
-// 128-byte swizzle layout that a TMA load with CU_TENSOR_MAP_SWIZZLE_128B
-// writes: row r of the tile at byte r*128, its 16-byte chunks XOR-permuted by
-// (r % 8).  Fields: start address >> 4 [0,14), leading byte offset >> 4
-// [16,30) (unused for swizzled K-major; 1), stride byte offset >> 4 [32,46)
-// = 1024 B between 8-row groups, descriptor version 1 at [46,48), layout
-// type SWIZZLE_128B = 2 at [61,64).  The tile base must be 1024-byte aligned.
-__device__ __forceinline__ uint64_t smem_desc_k128(uint32_t saddr) {
+// Shared-memory matrix descriptor for an operand tile stored in the 128-byte
+// swizzle layout that a TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes: row r
+// of the box at byte r*128, its 16-byte chunks XOR-permuted by (r % 8), 8-row
+// groups 1024 bytes apart.  Fields: start address >> 4 [0,14), leading byte
+// offset >> 4 [16,30), stride byte offset >> 4 [32,46), descriptor version 1
+// at [46,48), layout type SWIZZLE_128B = 2 at [61,64).  The tile base must be
+// 1024-byte aligned.
+//  - K-major tile (a row holds 128 bytes of K of one M/N index): the stride
+//    offset is the 1024 bytes between 8-row groups; the leading offset is
+//    unused (1).  The next 32 K of a row start 32 bytes further on.
+//  - MN-major tile (a row holds 128 M/N indices of one K): the stride offset
+//    is the 1024 bytes between groups of 8 K; the leading offset is the
+//    distance between blocks of 128 M/N indices (unused when the tile is 128
+//    wide).  The next 32 K start 32 rows = 4096 bytes further on.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
     d |= (uint64_t)(1024u >> 4) << 32;
     d |= (uint64_t)1u << 46;
     d |= (uint64_t)2u << 61;
     return d;
 }
+__device__ __forceinline__ uint64_t smem_desc_k128(uint32_t saddr) {
+    return smem_desc_sw128(saddr, 16u);
+}
 
-// Instruction descriptor, kind::f8f6f4, fp32 accumulator, both operands
-// K-major: D format F32 = 1 at [4,6), A format [7,10), B format [10,13)
-// (E4M3 = 0, E5M2 = 1), N >> 3 at [17,23), M >> 4 at [24,29).
-__host__ __device__ constexpr uint32_t idesc_f8(uint32_t fa, uint32_t fb, uint32_t m,
-                                                uint32_t n) {
-    return (1u << 4) | (fa << 7) | (fb << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
+// Instruction descriptor, kind::f8f6f4, fp32 accumulator: D format F32 = 1
+// at [4,6), A format [7,10), B format [10,13) (E4M3 = 0, E5M2 = 1), A major
+// at 15 and B major at 16 (0 = K-major, 1 = MN-major; MN-major is valid for
+// E4M3 and E5M2), N >> 3 at [17,23), M >> 4 at [24,29).
+__host__ __device__ constexpr uint32_t idesc_f8(uint32_t fa, uint32_t fb, uint32_t m, uint32_t n,
+                                                uint32_t a_mn = 0, uint32_t b_mn = 0) {
+    return (1u << 4) | (fa << 7) | (fb << 10) | (a_mn << 15) | (b_mn << 16) | ((n >> 3) << 17) |
+           ((m >> 4) << 24);
 }
 
 // ------------------------------------------------- clusters / CTA pairs

@@ -40,22 +40,18 @@ size_t saved_layout(int64_t M, int64_t d, int64_t f, uint8_t* base, lm_swiglu_sa
     };
     lm_swiglu_saved o;
     o.Xq = take(Md);
-    o.XqT = take(Md);
     o.Wguq = take(2 * fd);
-    o.WguqT = take(2 * fd);
     o.Wdq = take(fd);
-    o.WdqT = take(fd);
     o.GU = take(2 * Mf * 2);
     o.h = take(Mf * 2);
     o.hq = take(Mf);
-    o.hqT = take(Mf);
     o.scales = reinterpret_cast<float*>(take(16 * sizeof(float)));
     if (out) *out = o;
     return off;
 }
 
 struct BwdWs {
-    uint8_t *dYq, *dYqT, *dGUq, *dGUqT;
+    uint8_t *dYq, *dGUq;
     void *g, *dGU;
     float* scales;
 };
@@ -70,11 +66,9 @@ size_t bwd_layout(int64_t M, int64_t d, int64_t f, uint8_t* base, BwdWs* w) {
     };
     BwdWs o;
     o.dYq = take(Md);
-    o.dYqT = take(Md);
     o.g = take(Mf * 2);
     o.dGU = take(2 * Mf * 2);
     o.dGUq = take(2 * Mf);
-    o.dGUqT = take(2 * Mf);
     o.scales = reinterpret_cast<float*>(take(8 * sizeof(float)));
     if (w) *w = o;
     return off;
@@ -172,25 +166,25 @@ lm_status lm_swiglu_mlp_fwd(const void* X, const void* W_gu, const void* W_down,
                             lm_stream_t stream) {
     using namespace lm;
     if (!shape_ok(M, d, f)) return LM_ERR_UNSUPPORTED_SHAPE;
-    if (!X || !W_gu || !W_down || !Y || !sv || !sv->Xq || !sv->XqT || !sv->Wguq || !sv->WguqT ||
-        !sv->Wdq || !sv->WdqT || !sv->GU || !sv->h || !sv->hq || !sv->hqT || !sv->scales)
+    if (!X || !W_gu || !W_down || !Y || !sv || !sv->Xq || !sv->Wguq || !sv->Wdq || !sv->GU ||
+        !sv->h || !sv->hq || !sv->scales)
         return LM_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     float* S = sv->scales;
     if (cudaMemsetAsync(S, 0, 16 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
     // X, W_gu, W_down: one amax launch, one cast launch (slots zeroed above)
     const CastItem in[3] = {
-        {X, M, d, d, nullptr, S + S_X, S + S_X + 1, S + S_X + 2, sv->Xq, sv->XqT},
+        {X, M, d, d, nullptr, S + S_X, S + S_X + 1, S + S_X + 2, sv->Xq, nullptr},
         {W_gu, 2 * f, d, d, nullptr, S + S_WGU, S + S_WGU + 1, S + S_WGU + 2, sv->Wguq,
-         sv->WguqT},
-        {W_down, d, f, f, nullptr, S + S_WD, S + S_WD + 1, S + S_WD + 2, sv->Wdq, sv->WdqT}};
+         nullptr},
+        {W_down, d, f, f, nullptr, S + S_WD, S + S_WD + 1, S + S_WD + 2, sv->Wdq, nullptr}};
     LM_TRY(cast_set(in, 3, LM_FP8_E4M3, 0, true, s));
     if (M > 0)
-        LM_TRY(gemm_dispatch(sv->Xq, LM_FP8_E4M3, sv->Wguq, LM_FP8_E4M3, M, 2 * f, d, S + S_X + 2,
-                             S + S_WGU + 2, kEpiSwigluFwd, nullptr, sv->GU, sv->h, S + S_H,
-                             stream));
+        LM_TRY(gemm_dispatch(sv->Xq, LM_FP8_E4M3, sv->Wguq, LM_FP8_E4M3, M, 2 * f, d, 0u,
+                             S + S_X + 2, S + S_WGU + 2, kEpiSwigluFwd, nullptr, sv->GU, sv->h,
+                             S + S_H, stream));
     LM_TRY(lm_fp8_amax_scale_cast(sv->h, M, f, f, LM_FP8_E4M3, 0, S + S_H, S + S_H, S + S_H + 1,
-                                  S + S_H + 2, sv->hq, sv->hqT, stream));
+                                  S + S_H + 2, sv->hq, nullptr, stream));
     LM_TRY(lm_fp8_gemm(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, S + S_H + 2,
                        S + S_WD + 2, LM_EPI_NONE, nullptr, Y, nullptr, stream));
     return LM_OK;
@@ -211,13 +205,15 @@ lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* sv, int64_t M
     float* G = w.scales;
     if (cudaMemsetAsync(G, 0, 8 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
     const CastItem dy = {dY, M, d, d, nullptr, G + S_DY, G + S_DY + 1, G + S_DY + 2, w.dYq,
-                         w.dYqT};
+                         nullptr};
     LM_TRY(cast_set(&dy, 1, LM_FP8_E5M2, 0, true, s));  // slot zeroed above
     // g = dY W_down (plain bf16), dW_down = dY^T h
-    LM_TRY(lm_fp8_gemm(w.dYq, LM_FP8_E5M2, sv->WdqT, LM_FP8_E4M3, M, f, d, G + S_DY + 2,
-                       S + S_WD + 2, LM_EPI_NONE, nullptr, w.g, nullptr, stream));
-    LM_TRY(lm_fp8_gemm(w.dYqT, LM_FP8_E5M2, sv->hqT, LM_FP8_E4M3, d, f, M, G + S_DY + 2,
-                       S + S_H + 2, LM_EPI_NONE, nullptr, dW_down, nullptr, stream));
+    // (row-major codes read MN-major where the transpose is the operand)
+    constexpr uint32_t B_MN = LM_GEMM_B_MN_MAJOR, AB_MN = LM_GEMM_A_MN_MAJOR | LM_GEMM_B_MN_MAJOR;
+    LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->Wdq, LM_FP8_E4M3, M, f, d, B_MN, G + S_DY + 2,
+                          S + S_WD + 2, LM_EPI_NONE, nullptr, w.g, nullptr, stream));
+    LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->hq, LM_FP8_E4M3, d, f, M, AB_MN, G + S_DY + 2,
+                          S + S_H + 2, LM_EPI_NONE, nullptr, dW_down, nullptr, stream));
     if (M > 0) {
         int grid = sm_count() * 8;
         if (grid <= 0) return LM_ERR_CUDA;
@@ -228,12 +224,13 @@ lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* sv, int64_t M
         if (launch_status() != LM_OK) return LM_ERR_CUDA;
     }
     LM_TRY(lm_fp8_amax_scale_cast(w.dGU, M, 2 * f, 2 * f, LM_FP8_E5M2, 0, G + S_DGU, G + S_DGU,
-                                  G + S_DGU + 1, G + S_DGU + 2, w.dGUq, w.dGUqT, stream));
+                                  G + S_DGU + 1, G + S_DGU + 2, w.dGUq, nullptr, stream));
     // dX = dGU W_gu (K = 2f);  dW_gu = dGU^T X (K = M)
-    LM_TRY(lm_fp8_gemm(w.dGUq, LM_FP8_E5M2, sv->WguqT, LM_FP8_E4M3, M, d, 2 * f, G + S_DGU + 2,
-                       S + S_WGU + 2, LM_EPI_NONE, nullptr, dX, nullptr, stream));
-    LM_TRY(lm_fp8_gemm(w.dGUqT, LM_FP8_E5M2, sv->XqT, LM_FP8_E4M3, 2 * f, d, M, G + S_DGU + 2,
-                       S + S_X + 2, LM_EPI_NONE, nullptr, dW_gu, nullptr, stream));
+    LM_TRY(lm_fp8_gemm_ex(w.dGUq, LM_FP8_E5M2, sv->Wguq, LM_FP8_E4M3, M, d, 2 * f, B_MN,
+                          G + S_DGU + 2, S + S_WGU + 2, LM_EPI_NONE, nullptr, dX, nullptr, stream));
+    LM_TRY(lm_fp8_gemm_ex(w.dGUq, LM_FP8_E5M2, sv->Xq, LM_FP8_E4M3, 2 * f, d, M, AB_MN,
+                          G + S_DGU + 2, S + S_X + 2, LM_EPI_NONE, nullptr, dW_gu, nullptr,
+                          stream));
     return LM_OK;
 }
 

@@ -61,6 +61,8 @@ def main():
     p.add_argument("--fa", default="e4m3")
     p.add_argument("--fb", default="e4m3")
     p.add_argument("--epi", default="none", choices=list(EPI))
+    p.add_argument("--flags", type=int, default=0,
+                   help="operand storage: 1 = A MN-major, 2 = B MN-major, 3 = both")
     p.add_argument("--rows", type=int, default=16384)
     p.add_argument("--cols", type=int, default=3072)
     p.add_argument("--fmt", default="e4m3")
@@ -131,20 +133,21 @@ def main():
                    gbs=round(8 * n / avg / 1e6, 1), algorithmic_bytes=8 * n)
     elif a.op == "gemm":
         fa, fb, epi = FMT[a.fa], FMT[a.fb], EPI[a.epi]
-        A = random_codes(fa, a.M, a.K, gen)
-        B = random_codes(fb, a.N, a.K, gen)
+        A = random_codes(fa, *((a.K, a.M) if a.flags & 1 else (a.M, a.K)), gen)
+        B = random_codes(fb, *((a.K, a.N) if a.flags & 2 else (a.N, a.K)), gen)
         ia = torch.full((1,), 1e-2, device="cuda")
         ib = torch.full((1,), 1e-2, device="cuda")
         D = torch.empty(a.M, a.N, dtype=torch.bfloat16, device="cuda")
         aux = torch.randn(a.M, a.N, device="cuda", generator=gen).to(torch.bfloat16) \
             if epi == EPI_RELU2_BWD else None
         am = torch.zeros(1, device="cuda")
-        fn = lambda: _lib.lm_fp8_gemm(A, fa, B, fb, ia, ib, D, epi=epi, aux=aux, amax_out=am)
+        fn = lambda: _lib.lm_fp8_gemm_ex(A, fa, B, fb, ia, ib, D, flags=a.flags, epi=epi, aux=aux,
+                                         amax_out=am)
         ms = time_it(fn, a.iters, a.warmup, flush)
         flops = 2 * a.M * a.N * a.K
         byts = a.M * a.K + a.N * a.K + 2 * a.M * a.N * (2 if epi == EPI_RELU2_BWD else 1)
         avg = sum(ms) / len(ms)
-        out = dict(op="gemm", M=a.M, N=a.N, K=a.K, fa=a.fa, fb=a.fb, epi=a.epi,
+        out = dict(op="gemm", M=a.M, N=a.N, K=a.K, fa=a.fa, fb=a.fb, epi=a.epi, flags=a.flags,
                    avg_ms=round(avg, 4), min_ms=round(min(ms), 4),
                    tflops=round(flops / avg / 1e9, 1), algorithmic_bytes=byts)
     else:

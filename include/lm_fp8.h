@@ -133,6 +133,27 @@ LM_API lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8_t* 
                       const float* inv_scale_b, lm_epilogue epi, const void* aux, void* D,
                       float* amax_out, lm_stream_t stream);
 
+/* Operand storage flags of lm_fp8_gemm_ex. */
+#define LM_GEMM_A_MN_MAJOR 1u /* A stored as [K x M] row-major (M contiguous), i.e. A^T */
+#define LM_GEMM_B_MN_MAJOR 2u /* B stored as [K x N] row-major (N contiguous), i.e. B^T */
+
+/*
+ * lm_fp8_gemm with the storage of each operand chosen by `flags`: the same
+ * D = epilogue(A B^T s), where an MN-major operand is read as the transpose
+ * of the matrix stored.  This lets dgrad and wgrad consume the row-major codes
+ * of a cast directly: the tensor cores read 8-bit operands in either order
+ * from shared memory, so no transposed copy of the codes is needed
+ * (tcgen05.mma instruction descriptor, "transpose A/B" bits).
+ * Additional requirements: M % 16 == 0 with LM_GEMM_A_MN_MAJOR, N % 16 == 0
+ * with LM_GEMM_B_MN_MAJOR (each stored row starts on a 16-byte boundary);
+ * unknown flag bits return LM_ERR_INVALID_ARG.  flags == 0 is lm_fp8_gemm.
+ * The result is bit-identical to lm_fp8_gemm on the transposed copies.
+ */
+LM_API lm_status lm_fp8_gemm_ex(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
+                         lm_fp8_format fb, int64_t M, int64_t N, int64_t K, uint32_t flags,
+                         const float* inv_scale_a, const float* inv_scale_b, lm_epilogue epi,
+                         const void* aux, void* D, float* amax_out, lm_stream_t stream);
+
 /*
  * The producer of a GEMM input: RMSNorm, then the dynamic FP8 cast of its
  * output (the model's pre-norm; decomputer.nl, "Het trainen van een 3.8B
@@ -160,15 +181,11 @@ LM_API lm_status lm_rmsnorm_fp8_cast(const void* R, const void* weight, int64_t 
  * X [M x d], W_up [f x d], W_down [d x f]:
  */
 typedef struct lm_mlp_saved {
-    uint8_t* Xq;   /* [M x d] e4m3 */
-    uint8_t* XqT;  /* [d x M] e4m3, for wgrad of W_up */
-    uint8_t* Wuq;  /* [f x d] e4m3, forward B operand of the up GEMM */
-    uint8_t* WuqT; /* [d x f] e4m3, dgrad B operand */
-    uint8_t* Wdq;  /* [d x f] e4m3, forward B operand of the down GEMM */
-    uint8_t* WdqT; /* [f x d] e4m3, dgrad B operand */
+    uint8_t* Xq;   /* [M x d] e4m3; wgrad of W_up reads it MN-major */
+    uint8_t* Wuq;  /* [f x d] e4m3, B of the up GEMM; dgrad reads it MN-major */
+    uint8_t* Wdq;  /* [d x f] e4m3, B of the down GEMM; dgrad reads it MN-major */
     void* H;       /* [M x f] bf16 pre-activation X W_up^T */
-    uint8_t* hq;   /* [M x f] e4m3 codes of h = bf16(relu(H)^2) */
-    uint8_t* hqT;  /* [f x M] e4m3, for wgrad of W_down */
+    uint8_t* hq;   /* [M x f] e4m3 codes of h = bf16(relu(H)^2); wgrad reads it MN-major */
     float* scales; /* 16 device floats: {amax, scale, inv_scale, unused} for X, W_up, W_down, h */
 } lm_mlp_saved;
 
@@ -185,10 +202,12 @@ LM_API size_t lm_relu2_mlp_workspace_size(int64_t M, int64_t d, int64_t f);
 
 /*
  * relu^2 MLP forward, Y = relu(X W_up^T)^2 W_down^T, every GEMM in FP8:
- *   cast X, W_up, W_down to e4m3 (+ K-major transposes)
+ *   cast X, W_up, W_down to e4m3 (one amax launch, one cast launch)
  *   H = up GEMM with the RELU2_FWD epilogue (bf16 H + amax of h)
- *   cast h = bf16(relu(H)^2) to e4m3 (+ transpose) using that amax
+ *   cast h = bf16(relu(H)^2) to e4m3 using that amax
  *   Y = down GEMM (bf16)
+ * Only row-major codes are made: the backward's GEMMs read them MN-major
+ * (lm_fp8_gemm_ex), so no transposed copy is written or saved.
  * X: bf16 [M x d], W_up: bf16 [f x d], W_down: bf16 [d x f], Y: bf16 [M x d].
  * workspace may be NULL (ws_bytes 0).  Requirements: M, d, f multiples of 16.
  */
@@ -198,11 +217,13 @@ LM_API lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W
 
 /*
  * relu^2 MLP backward from the forward's saved tensors:
- *   cast dY to e5m2 (+ transpose)
+ *   cast dY to e5m2
  *   dH = dgrad of W_down with the RELU2_BWD epilogue: bf16(bf16(dY W_down) * 2 relu(H))
  *   dW_down = dY^T h   (wgrad, K = M)
- *   cast dH to e5m2 (+ transpose) using the epilogue's amax
+ *   cast dH to e5m2 using the epilogue's amax
  *   dX = dH W_up;  dW_up = dH^T X
+ * (W_down and W_up as dgrad B operands, and dY, h, dH, X as wgrad operands,
+ * are read MN-major from their row-major codes.)
  * dY: bf16 [M x d]; outputs bf16 dX [M x d], dW_up [f x d], dW_down [d x f].
  * workspace: device scratch of >= lm_relu2_mlp_workspace_size bytes,
  * 256-byte aligned.  Requirements as for the forward.
@@ -242,7 +263,7 @@ LM_API size_t lm_relu2_mlp_bwd_noalloc_max_bytes(void);
  * Gradient-accumulation forms of the MLP forward and backward (flags above).
  * With flags == 0 they are lm_relu2_mlp_fwd / lm_relu2_mlp_bwd.
  *  - LM_MLP_REUSE_WEIGHT_CASTS (fwd): skip the casts of W_up and W_down and
- *    use the codes, transposes and scales `saved` holds from an earlier
+ *    use the codes and scales `saved` holds from an earlier
  *    forward of the same weights (once per optimizer step is enough).
  *  - LM_MLP_ACCUMULATE_WGRAD (bwd): dW_up [f x d] and dW_down [d x f] are fp32;
  *    each wgrad GEMM adds fp32(acc * s) into them (LM_EPI_ACCUM_F32); dX stays
@@ -274,12 +295,12 @@ LM_API lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* saved, 
  * MLP; the saved GU holds G and U in the same interleaved column order.
  */
 typedef struct lm_swiglu_saved {
-    uint8_t *Xq, *XqT;     /* [M x d], [d x M] e4m3 */
-    uint8_t *Wguq, *WguqT; /* [2f x d], [d x 2f] e4m3, interleaved gate/up */
-    uint8_t *Wdq, *WdqT;   /* [d x f], [f x d] e4m3 */
+    uint8_t* Xq;           /* [M x d] e4m3 (read MN-major by the wgrad of W_gu) */
+    uint8_t* Wguq;         /* [2f x d] e4m3, interleaved gate/up */
+    uint8_t* Wdq;          /* [d x f] e4m3 */
     void* GU;              /* [M x 2f] bf16 pre-activations, interleaved */
     void* h;               /* [M x f] bf16 silu(G) U */
-    uint8_t *hq, *hqT;     /* [M x f], [f x M] e4m3 */
+    uint8_t* hq;           /* [M x f] e4m3 (read MN-major by the wgrad of W_down) */
     float* scales;         /* 16 floats: {amax, scale, inv_scale, 0} for X, W_gu, W_down, h */
 } lm_swiglu_saved;
 

@@ -78,16 +78,18 @@ def test_cast_host_checks_reject_before_launch(L):
 def test_mlp_sizes_and_carve(L):
     M, d, f = 256, 256, 1024
     r = lambda n: (n + 255) // 256 * 256
-    assert L.lm_relu2_mlp_saved_bytes(M, d, f) == (2 * r(M * d) + 4 * r(f * d) + r(2 * M * f)
-                                                   + 2 * r(M * f) + r(64))
-    assert L.lm_relu2_mlp_workspace_size(M, d, f) == (2 * r(M * d) + r(2 * M * f)
-                                                      + 2 * r(M * f) + r(32))
+    # row-major codes only (the backward reads them MN-major): X, W_up, W_down,
+    # H, h codes and the scales; scratch dY codes, dH, dH codes, scales
+    assert L.lm_relu2_mlp_saved_bytes(M, d, f) == (r(M * d) + 2 * r(f * d) + r(2 * M * f)
+                                                   + r(M * f) + r(64))
+    assert L.lm_relu2_mlp_workspace_size(M, d, f) == (r(M * d) + r(2 * M * f) + r(M * f)
+                                                      + r(32))
     assert L.lm_relu2_mlp_saved_bytes(M, d, 1000) == 0      # f not a multiple of 16
     s = L.MlpSaved()
     base = 0x100000
     n = L.lm_relu2_mlp_saved_bytes(M, d, f)
     assert L.lib.lm_relu2_mlp_saved_carve(base, n, M, d, f, ctypes.byref(s)) == 0
-    assert s.Xq == base and s.XqT == base + r(M * d) and s.scales == base + n - r(64)
+    assert s.Xq == base and s.Wuq == base + r(M * d) and s.scales == base + n - r(64)
     assert L.lib.lm_relu2_mlp_saved_carve(base, n - 1, M, d, f, ctypes.byref(s)) == 1
     assert L.lib.lm_relu2_mlp_saved_carve(base + 16, n, M, d, f, ctypes.byref(s)) == 2
 
@@ -124,6 +126,12 @@ def test_newer_entry_points_reject_before_launch(L):
     # the internal gated epilogue is not reachable through the public GEMM
     assert lib.lm_fp8_gemm(fake, 0, fake, 0, 256, 256, 64, fake, fake, 4, None, fake, None,
                            None) == 4
+    # operand-storage flags: unknown bits; MN-major rows not 16-byte aligned
+    gx = lib.lm_fp8_gemm_ex
+    assert gx(fake, 0, fake, 0, 256, 256, 64, 4, fake, fake, 0, None, fake, None, None) == 1
+    assert gx(fake, 0, fake, 0, 200, 256, 64, 1, fake, fake, 0, None, fake, None, None) == 3
+    assert gx(fake, 0, fake, 0, 256, 264, 64, 2, fake, fake, 0, None, fake, None, None) == 3
+    assert gx(fake, 0, fake, 0, 256, 264, 64, 1, fake, fake, 4, None, fake, None, None) == 4
     # no-alloc backward: shape beyond its array
     assert lib.lm_relu2_mlp_bwd_noalloc(None, C.byref(s), 16384, 3072, 12288, None, None, None,
                                         None) == 3

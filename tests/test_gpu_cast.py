@@ -67,6 +67,15 @@ def test_cast_heavy_tails_and_ties(orc, api):
     _check_cast(orc, api, x, E4M3)
 
 
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("relu2", [False, True])
+def test_cast_row_major_only_bit_exact(orc, api, shape, relu2):
+    """qT not requested: the TMA-fed kernel without its transpose stage (the
+    blocks' casts, whose codes the GEMMs read MN-major where needed)."""
+    x = synthetic.student_t3_bf16(shape, 44, int(relu2))
+    _check_cast(orc, api, x, E5M2 if relu2 else E4M3, relu2=relu2, want_qT=False)
+
+
 def test_cast_without_transpose_and_ragged_rows(orc, api):
     x = synthetic.normal_bf16((200, 96), 2.0, 43, 0)  # rows % 16 != 0: q only
     _check_cast(orc, api, x, E4M3, want_qT=False)

@@ -119,6 +119,71 @@ def test_gemm_persistent_many_tiles(lib, orc):
     run(lib, orc, 2048, 4096, 256)
 
 
+MN_CASES = [
+    # (M, N, K, flags): pair kernel (M > 128) and thin kernel (M <= 128), ragged
+    # tails in M, N and K where the 16-row rule of MN-major storage allows
+    (208, 336, 208, 1), (208, 336, 208, 2), (208, 336, 208, 3),
+    (128, 256, 128, 3),      # one tile, one k-block
+    (384, 768, 512, 1),
+    (2048, 4096, 256, 2),    # many tiles per cluster
+    (16, 16, 16, 3),         # thin kernel, smaller than a tile everywhere
+    (112, 528, 272, 2),      # thin kernel: B in two 128-wide MN blocks plus a ragged third tile
+    (96, 256, 8192, 1),      # thin kernel, long K (a wgrad's reduction length)
+]
+
+
+def mn_store(X, mn):
+    """The codes as the GPU reads them: X itself, or its transpose, contiguous."""
+    return from_u8(np.ascontiguousarray(X.T) if mn else X)
+
+
+@pytest.mark.parametrize("M,N,K,flags", MN_CASES)
+def test_gemm_mn_major_operands(lib, orc, M, N, K, flags):
+    """Operands stored MN-major (the transposes of A [M x K] / B [N x K]): the
+    oracle's result on the K-major codes, and bit-identical to the K-major run."""
+    A, B = codes(E5M2, (M, K), 21), codes(E4M3, (N, K), 22)
+    ia = torch.tensor([1e-4], device="cuda")
+    ib = torch.tensor([0.5], device="cuda")
+    D = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Dk = torch.empty_like(D)
+    am = torch.zeros(1, device="cuda")
+    amk = torch.zeros(1, device="cuda")
+    lib.lm_fp8_gemm_ex(mn_store(A, flags & 1), E5M2, mn_store(B, flags & 2), E4M3, ia, ib, D,
+                       flags=flags, amax_out=am)
+    lib.lm_fp8_gemm(from_u8(A), E5M2, from_u8(B), E4M3, ia, ib, Dk, amax_out=amk)
+    torch.cuda.synchronize()
+    assert lib.lm_get_error()[0] == 0
+    ref, _ = orc.gemm(A, E5M2, B, E4M3, np.float32(1e-4), np.float32(0.5))
+    assert_close(u16(D), ref, f"mn-major flags={flags} M={M} N={N} K={K}", ELEM_REL)
+    assert torch.equal(D.view(torch.int16), Dk.view(torch.int16))
+    assert torch.equal(am, amk)
+
+
+@pytest.mark.parametrize("epi", [EPI_RELU2_FWD, EPI_RELU2_BWD])
+@pytest.mark.parametrize("M,N,K", [(208, 336, 208), (64, 272, 96)])
+def test_gemm_mn_major_epilogues(lib, orc, epi, M, N, K):
+    A, B = codes(E4M3, (M, K), 23), codes(E4M3, (N, K), 24)
+    g = torch.Generator().manual_seed(25)
+    aux = u16(torch.randn(M, N, generator=g).to(torch.bfloat16)) if epi == EPI_RELU2_BWD else None
+    ia = torch.tensor([0.02], device="cuda")
+    ib = torch.tensor([0.5], device="cuda")
+    out = []
+    for flags in (0, 3):
+        D = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        am = torch.zeros(1, device="cuda")
+        lib.lm_fp8_gemm_ex(mn_store(A, flags & 1), E4M3, mn_store(B, flags & 2), E4M3, ia, ib, D,
+                           flags=flags, epi=epi, aux=None if aux is None else from_u16(aux),
+                           amax_out=am)
+        out.append((D, am))
+    torch.cuda.synchronize()
+    assert lib.lm_get_error()[0] == 0
+    assert torch.equal(out[0][0].view(torch.int16), out[1][0].view(torch.int16))
+    assert torch.equal(out[0][1], out[1][1])
+    ref, _ = orc.gemm(A, E4M3, B, E4M3, np.float32(0.02), np.float32(0.5), epi=epi, aux=aux)
+    assert_close(u16(out[1][0]), ref, f"mn-major epi={epi} M={M} N={N} K={K}",
+                 ELEM_REL_RELU2_BWD if epi == EPI_RELU2_BWD else ELEM_REL)
+
+
 def test_gemm_k_zero_and_empty(lib, orc):
     D = torch.full((32, 64), 1.0, dtype=torch.bfloat16, device="cuda")
     one = torch.ones(1, dtype=torch.float32, device="cuda")

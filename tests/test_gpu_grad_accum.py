@@ -46,6 +46,25 @@ def test_accumulating_gemm_twice(lib, orc, M, N, K):
     assert_close_f32(D.cpu().numpy(), ref, f"accum M={M} N={N} K={K}")
 
 
+@pytest.mark.parametrize("M,N,K", [(512, 336, 400), (96, 272, 160)])
+def test_accumulating_gemm_mn_major(lib, orc, M, N, K):
+    """The wgrad shape of the blocks: both operands MN-major (the row-major
+    codes of dY / X read as their transposes), accumulated in fp32."""
+    A, B = codes(E5M2, (M, K), 9), codes(E4M3, (N, K), 10)
+    D0 = np.random.default_rng(11).standard_normal((M, N)).astype(np.float32) * 1e-3
+    D = torch.from_numpy(D0.copy()).cuda()
+    ia = torch.tensor([1e-4], device="cuda")
+    ib = torch.tensor([0.05], device="cuda")
+    At = torch.from_numpy(np.ascontiguousarray(A.T)).cuda()
+    Bt = torch.from_numpy(np.ascontiguousarray(B.T)).cuda()
+    lib.lm_fp8_gemm_ex(At, E5M2, Bt, E4M3, ia, ib, D, flags=3, epi=lib.EPI_ACCUM_F32)
+    torch.cuda.synchronize()
+    assert lib.lm_get_error()[0] == 0
+    ref = D0.copy()
+    orc.gemm_accum_f32(A, E5M2, B, E4M3, np.float32(1e-4), np.float32(0.05), ref)
+    assert_close_f32(D.cpu().numpy(), ref, f"accum mn-major M={M} N={N} K={K}")
+
+
 def test_mlp_grad_accumulation_three_micro_batches(lib, orc):
     from fp8_gemms_b200 import api
     w = synthetic.TINY_MLP

@@ -40,6 +40,11 @@ def run_chain(api, w):
     return t, mlp, Y, dX, dWu, dWd
 
 
+def T(codes):
+    """Host transpose of a code matrix (the K-major operand the oracle takes)."""
+    return np.ascontiguousarray(codes.T)
+
+
 def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None):
     """rows: sample of output rows to check for the M x * GEMMs (None = all)."""
     sc = mlp.view("scales").cpu().numpy()
@@ -48,7 +53,6 @@ def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None):
         ref = orc.amax_scale_cast(synthetic.bits_u16(t[name]), E4M3)
         assert sc[si, 0] == ref["amax"] and sc[si, 1] == ref["scale"] and sc[si, 2] == ref["inv_scale"], name
         assert np.array_equal(u8(mlp.view(key)), ref["q"]), name
-        assert np.array_equal(u8(mlp.view(key + "T")), ref["qT"]), name + "T"
     Xq, Wuq, Wdq = u8(mlp.view("Xq")), u8(mlp.view("Wuq")), u8(mlp.view("Wdq"))
     H = u16(mlp.view("H"))
     # up GEMM (RELU2_FWD) from the GPU's codes and scales
@@ -59,9 +63,9 @@ def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None):
     # cast of h from the GPU's H and amax: bit-exact
     s_h, inv_h = orc.scale(sc[3, 0], E4M3)
     assert sc[3, 1] == s_h and sc[3, 2] == inv_h
-    hq_ref, hqT_ref = orc.cast(H, E4M3, s_h, relu2_input=True)
-    hq, hqT = u8(mlp.view("hq")), u8(mlp.view("hqT"))
-    assert np.array_equal(hq, hq_ref) and np.array_equal(hqT, hqT_ref)
+    hq_ref, _ = orc.cast(H, E4M3, s_h, relu2_input=True, want_qT=False)
+    hq = u8(mlp.view("hq"))
+    assert np.array_equal(hq, hq_ref)
     # down GEMM
     Yref, _ = orc.gemm(hq, E4M3, Wdq, E4M3, sc[3, 2], sc[2, 2], rows=rows)
     assert_close(u16(Y) if rows is None else u16(Y)[rows], Yref, "Y")
@@ -70,25 +74,27 @@ def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None):
     g = mlp.workspace_view("scales").cpu().numpy()
     ref = orc.amax_scale_cast(synthetic.bits_u16(t["dY"]), E5M2)
     assert g[0, 0] == ref["amax"] and g[0, 1] == ref["scale"] and g[0, 2] == ref["inv_scale"]
-    dYq, dYqT = u8(mlp.workspace_view("dYq")), u8(mlp.workspace_view("dYqT"))
-    assert np.array_equal(dYq, ref["q"]) and np.array_equal(dYqT, ref["qT"])
+    dYq = u8(mlp.workspace_view("dYq"))
+    assert np.array_equal(dYq, ref["q"])
+    # the backward's GEMMs read the row-major codes MN-major: the oracle gets
+    # the K-major operands, i.e. the host transposes of those codes
     dH = u16(mlp.workspace_view("dH"))
-    dHref, _ = orc.gemm(dYq, E5M2, u8(mlp.view("WdqT")), E4M3, g[0, 2], sc[2, 2],
+    dHref, _ = orc.gemm(dYq, E5M2, T(Wdq), E4M3, g[0, 2], sc[2, 2],
                         orc.EPI_RELU2_BWD, aux=H, rows=rows)
     assert_close(dH if rows is None else dH[rows], dHref, "dH", ELEM_REL_RELU2_BWD)
     assert g[1, 0] == orc.amax(dH)
     s_dh, inv_dh = orc.scale(g[1, 0], E5M2)
     assert g[1, 1] == s_dh and g[1, 2] == inv_dh
-    dHq_ref, dHqT_ref = orc.cast(dH, E5M2, s_dh)
-    dHq, dHqT = u8(mlp.workspace_view("dHq")), u8(mlp.workspace_view("dHqT"))
-    assert np.array_equal(dHq, dHq_ref) and np.array_equal(dHqT, dHqT_ref)
+    dHq_ref, _ = orc.cast(dH, E5M2, s_dh, want_qT=False)
+    dHq = u8(mlp.workspace_view("dHq"))
+    assert np.array_equal(dHq, dHq_ref)
     wrows = None if rows is None else np.arange(0, dWd.shape[0], max(1, dWd.shape[0] // 24))
-    ref_dWd, _ = orc.gemm(dYqT, E5M2, hqT, E4M3, g[0, 2], sc[3, 2], rows=wrows)
+    ref_dWd, _ = orc.gemm(T(dYq), E5M2, T(hq), E4M3, g[0, 2], sc[3, 2], rows=wrows)
     assert_close(u16(dWd) if wrows is None else u16(dWd)[wrows], ref_dWd, "dW_down")
-    ref_dX, _ = orc.gemm(dHq, E5M2, u8(mlp.view("WuqT")), E4M3, g[1, 2], sc[1, 2], rows=rows)
+    ref_dX, _ = orc.gemm(dHq, E5M2, T(Wuq), E4M3, g[1, 2], sc[1, 2], rows=rows)
     assert_close(u16(dX) if rows is None else u16(dX)[rows], ref_dX, "dX")
     urows = None if rows is None else np.arange(0, dWu.shape[0], max(1, dWu.shape[0] // 24))
-    ref_dWu, _ = orc.gemm(dHqT, E5M2, u8(mlp.view("XqT")), E4M3, g[1, 2], sc[0, 2], rows=urows)
+    ref_dWu, _ = orc.gemm(T(dHq), E5M2, T(Xq), E4M3, g[1, 2], sc[0, 2], rows=urows)
     assert_close(u16(dWu) if urows is None else u16(dWu)[urows], ref_dWu, "dW_up")
 
 

@@ -67,8 +67,8 @@ def check_stagewise(orc, mlp, X, Wgu, rows=None):
     # amax of h reported by the epilogue = max |GPU h|; the cast of h bit-exact
     assert sc[3, 0] == orc.amax(h)
     s_h, _ = orc.scale(sc[3, 0], E4M3)
-    hq, hqT = orc.cast(h, E4M3, s_h)
-    assert np.array_equal(u8(mlp.view("hq")), hq) and np.array_equal(u8(mlp.view("hqT")), hqT)
+    hq, _ = orc.cast(h, E4M3, s_h, want_qT=False)
+    assert np.array_equal(u8(mlp.view("hq")), hq)
 
 
 def test_swiglu_stagewise_ragged(orc):
