@@ -33,11 +33,14 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// h = bf16(relu(x)^2): the square of a bf16 value is exact in fp32, then
-// rounded once to bf16.  relu(NaN) stays NaN.
-__device__ __forceinline__ float relu2_bf16(float x) {
-    float r = x > 0.f ? x : (x != x ? x : 0.f);
-    return __bfloat162float(__float2bfloat16_rn(r * r));
+// Two packed bf16 x -> two packed h = bf16(relu(x)^2): a NaN-propagating max
+// with 0 (relu(NaN) stays NaN), then one bf16x2 multiply, which rounds the
+// exact square once to bf16.
+__device__ __forceinline__ uint32_t relu2_bf16x2(uint32_t w) {
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&w);
+    const __nv_bfloat162 r = __hmax2_nan(x, __float2bfloat162_rn(0.0f));
+    const __nv_bfloat162 h = __hmul2(r, r);
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // Two fp32 values -> two saturated RNE FP8 codes (lo in the low byte).
@@ -58,12 +61,8 @@ __device__ __forceinline__ uint2 convert8(uint4 v, float scale) {
     uint32_t p[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
-        if (RELU2) {
-            lo = relu2_bf16(lo);
-            hi = relu2_bf16(hi);
-        }
-        p[i] = cvt_pair<FMT>(__fmul_rn(lo, scale), __fmul_rn(hi, scale));
+        const uint32_t x = RELU2 ? relu2_bf16x2(w[i]) : w[i];
+        p[i] = cvt_pair<FMT>(__fmul_rn(bf16_lo(x), scale), __fmul_rn(bf16_hi(x), scale));
     }
     return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
 }
@@ -79,13 +78,10 @@ __device__ __forceinline__ uint32_t absmax8(uint4 v, uint32_t m) {
         m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
         return m;
     }
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        uint32_t lo = __float_as_uint(relu2_bf16(bf16_lo(w[i]))) >> 16;
-        uint32_t hi = __float_as_uint(relu2_bf16(bf16_hi(w[i]))) & 0xFFFF0000u;
-        m = __vmaxu2(m, (lo | hi) & 0x7FFF7FFFu);
-    }
+    m = __vmaxu2(m, relu2_bf16x2(v.x) & 0x7FFF7FFFu);
+    m = __vmaxu2(m, relu2_bf16x2(v.y) & 0x7FFF7FFFu);
+    m = __vmaxu2(m, relu2_bf16x2(v.z) & 0x7FFF7FFFu);
+    m = __vmaxu2(m, relu2_bf16x2(v.w) & 0x7FFF7FFFu);
     return m;
 }
 

@@ -68,6 +68,7 @@ def main():
     p.add_argument("--fmt", default="e4m3")
     p.add_argument("--relu2", action="store_true")
     p.add_argument("--amax-in", action="store_true")
+    p.add_argument("--no-qT", action="store_true", help="cast: row-major codes only")
     p.add_argument("--iters", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     a = p.parse_args()
@@ -154,17 +155,17 @@ def main():
         fmt = FMT[a.fmt]
         x = (torch.randn(a.rows, a.cols, device="cuda", generator=gen)).to(torch.bfloat16)
         q = torch.empty(a.rows, a.cols, dtype=torch.uint8, device="cuda")
-        qT = torch.empty(a.cols, a.rows, dtype=torch.uint8, device="cuda")
+        qT = None if a.no_qT else torch.empty(a.cols, a.rows, dtype=torch.uint8, device="cuda")
         sc = torch.zeros(4, device="cuda")
         amax_in = torch.full((1,), 4.0, device="cuda") if a.amax_in else None
         fn = lambda: _lib.lm_fp8_amax_scale_cast(x, fmt, sc[0:1], sc[1:2], sc[2:3], q, qT,
                                                  relu2_input=a.relu2, amax_in=amax_in)
         ms = time_it(fn, a.iters, a.warmup, flush)
         n = a.rows * a.cols
-        byts = n * (4 if a.amax_in else 6)
+        byts = n * ((2 if a.amax_in else 4) + (1 if a.no_qT else 2))
         avg = sum(ms) / len(ms)
         out = dict(op="cast", rows=a.rows, cols=a.cols, fmt=a.fmt, relu2=a.relu2,
-                   amax_in=a.amax_in, avg_ms=round(avg, 4), min_ms=round(min(ms), 4),
+                   amax_in=a.amax_in, qT=not a.no_qT, avg_ms=round(avg, 4), min_ms=round(min(ms), 4),
                    gbs=round(byts / avg / 1e6, 1), algorithmic_bytes=byts)
     if a.op == "mlp-accum":
         from . import api  # noqa: F811

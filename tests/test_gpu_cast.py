@@ -76,6 +76,50 @@ def test_cast_row_major_only_bit_exact(orc, api, shape, relu2):
     _check_cast(orc, api, x, E5M2 if relu2 else E4M3, relu2=relu2, want_qT=False)
 
 
+def _is_nan_code(c, fmt):
+    c = np.asarray(c) & 0x7F
+    return c == 0x7F if fmt == E4M3 else c > 0x7C
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+@pytest.mark.parametrize("amax", [1.0, 2.0 ** -20, 2.0 ** 40])
+@pytest.mark.parametrize("want_qT", [False, True])
+def test_cast_relu2_every_bf16_pattern(orc, api, fmt, amax, want_qT):
+    """h = bf16(relu(x)^2) then the scaled cast, over all 65,536 bf16 bit
+    patterns (zeros of both signs, subnormals, every rounding tie of a square,
+    overflow to infinity, infinities, NaNs) with the amax supplied: codes equal
+    the oracle's bit for bit; a NaN input gives a NaN code on both sides."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(4096, 16)
+    x = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    am = torch.tensor([amax], dtype=torch.float32, device="cuda")
+    sc = torch.zeros(4, device="cuda")
+    q = torch.empty(4096, 16, dtype=torch.uint8, device="cuda")
+    qT = torch.empty(16, 4096, dtype=torch.uint8, device="cuda") if want_qT else None
+    from fp8_gemms_b200 import _lib
+    _lib.lm_fp8_amax_scale_cast(x.cuda(), fmt, sc[0:1], sc[1:2], sc[2:3], q, qT,
+                                relu2_input=True, amax_in=am)
+    torch.cuda.synchronize()
+    assert _lib.lm_get_error()[0] == 0
+    s, inv = orc.scale(np.float32(amax), fmt)
+    assert f32(sc[1:2]) == s and f32(sc[2:3]) == inv
+    ref, refT = orc.cast(bits, fmt, s, relu2_input=True)
+    for got, want in [(u8(q), ref)] + ([(u8(qT), refT)] if want_qT else []):
+        nan = _is_nan_code(want, fmt)
+        assert np.array_equal(_is_nan_code(got, fmt), nan)
+        assert np.array_equal(got[~nan], want[~nan])
+
+
+def test_cast_relu2_amax_pass_over_finite_patterns(orc, api):
+    """The reduction pass of a relu^2 cast (no amax supplied) over every finite
+    bf16 pattern whose square stays finite: amax, scale and codes bit-exact."""
+    b = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    mag = b & 0x7FFF
+    b = b[mag < 0x5F00]  # |x| < 2^63: finite squares, no NaN or infinity
+    b = b[: (b.size // 16) * 16].reshape(-1, 16)
+    x = torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)
+    _check_cast(orc, api, x, E4M3, relu2=True, want_qT=b.shape[0] % 16 == 0)
+
+
 def test_cast_without_transpose_and_ragged_rows(orc, api):
     x = synthetic.normal_bf16((200, 96), 2.0, 43, 0)  # rows % 16 != 0: q only
     _check_cast(orc, api, x, E4M3, want_qT=False)
