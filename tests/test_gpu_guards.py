@@ -44,12 +44,31 @@ def test_gemm_writes_stay_inside_D(M, N, K, epi):
     assert intact(buf, nbytes)
 
 
+@pytest.mark.parametrize("M,N,K,epi", [(208, 336, 208, 0), (112, 528, 272, 3), (304, 1040, 96, 2)])
+def test_gemm_mn_major_writes_stay_inside_D(M, N, K, epi):
+    """Both operands stored MN-major (the transposes); ragged tiles in N and K."""
+    from fp8_gemms_b200 import _lib
+    At, Bt = codes((K, M), 3), codes((K, N), 4)
+    one = torch.full((1,), 0.01, device="cuda")
+    dt = torch.float32 if epi == 3 else torch.bfloat16
+    nbytes = M * N * (4 if epi == 3 else 2)
+    buf, D = guarded(nbytes, dt, (M, N))
+    if epi == 3:
+        D.zero_()
+    aux = torch.randn(M, N, device="cuda").to(torch.bfloat16) if epi == 2 else None
+    _lib.lm_fp8_gemm_ex(At, 0, Bt, 0, one, one, D, flags=3, epi=epi, aux=aux)
+    torch.cuda.synchronize()
+    assert _lib.lm_get_error()[0] == 0
+    assert intact(buf, nbytes)
+
+
+@pytest.mark.parametrize("transposed", [True, False])
 @pytest.mark.parametrize("rows,cols", [(272, 144), (16, 16), (1040, 48), (200, 96)])
-def test_cast_writes_stay_inside_q_and_qT(rows, cols):
+def test_cast_writes_stay_inside_q_and_qT(rows, cols, transposed):
     from fp8_gemms_b200 import _lib
     x = torch.randn(rows, cols, device="cuda").to(torch.bfloat16)
     bq, q = guarded(rows * cols, torch.uint8, (rows, cols))
-    want_qT = rows % 16 == 0
+    want_qT = transposed and rows % 16 == 0
     bt, qT = guarded(rows * cols, torch.uint8, (cols, rows)) if want_qT else (None, None)
     sc = torch.zeros(4, device="cuda")
     _lib.lm_fp8_amax_scale_cast(x, 0, sc[0:1], sc[1:2], sc[2:3], q, qT)
