@@ -8,13 +8,16 @@
 // bullet; "Appendix: De configuratie", loss).  Here the head's three GEMMs
 // run in FP8 with dynamic tensorwise scaling like every other linear:
 //
-//   once:      W -> e4m3 (+ transpose); amax/scale of X (whole tensor)
-//   per chunk: X_c -> e4m3 (+ transpose) at X's scale
+//   once:      W -> e4m3; amax/scale of X (whole tensor)
+//   per chunk: X_c -> e4m3 at X's scale
 //              logits_c = X_c W^T (bf16)
 //              CE: z = c tanh(l / c), row loss, dlogits (bf16, in place) + amax
-//              dlogits_c -> e5m2 (+ transpose), no reduction pass
-//              dX_c = dlogits_c W        (K = V)
-//              dW  += fp32(dlogits_c^T X_c)   (TMA reduce-add epilogue)
+//              dlogits_c -> e5m2, no reduction pass
+//              dX_c = dlogits_c W        (K = V; W's codes read MN-major)
+//              dW  += fp32(dlogits_c^T X_c)   (both read MN-major; TMA
+//                                              reduce-add epilogue)
+// Only row-major codes are written: the GEMMs that contract over a tensor's
+// rows read its codes MN-major.
 //   end:       mean loss = deterministic fp64 sum of the row losses / M
 #include <cuda_bf16.h>
 

@@ -1,13 +1,14 @@
 // lm_rmsnorm.cu -- the producer of the FP8 GEMM input: RMSNorm -> amax ->
-// dynamic e4m3 cast with its transposed copy.
+// dynamic e4m3 cast (row-major codes, and the transposed copy on request).
 //
 // The model normalises with RMSNorm (rms_norm_eps 1e-6; PyTorch's
 // F.rms_norm) before its linears (decomputer.nl, "Het trainen van een 3.8B
 // LLM tot 0.384 CORE voor $998", "Appendix: De configuratie"; section "Wat
 // niet werkte", Liger RMSNorm bullet).  Producing X's amax in the same pass
 // that writes X lets the cast skip its reduction pass: 8 bytes per element
-// move instead of 10 (norm 2+2, cast 2+2+1+1), and the cast re-reads X while
-// much of it is still in L2.
+// move instead of 10 (norm 2+2, cast 2+2+1+1 with the transposed copy; 7
+// instead of 9 without it), and the cast re-reads X while much of it is
+// still in L2.
 //
 // One warp per row: a first sweep sums squares in fp32, the second (the row
 // is then in L1) writes X = bf16(x * inv_rms * w) with 16-byte stores and
