@@ -29,7 +29,8 @@ EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
             "lm_selftest_bounded_wait", "lm_relu2_mlp_fwd_ex", "lm_relu2_mlp_bwd_ex",
             "lm_rmsnorm_fp8_cast", "lm_swiglu_mlp_saved_bytes", "lm_swiglu_mlp_saved_carve",
             "lm_swiglu_mlp_workspace_size", "lm_swiglu_mlp_fwd", "lm_swiglu_mlp_bwd",
-            "lm_fp8_lmhead_ce_workspace_size", "lm_fp8_lmhead_ce", "lm_fp8_gemm_ex"]
+            "lm_fp8_lmhead_ce_workspace_size", "lm_fp8_lmhead_ce", "lm_fp8_gemm_ex",
+            "lm_fp8_gemm_workspace_size"]
 
 
 class LmError(RuntimeError):
@@ -60,8 +61,10 @@ def _load():
     L.lm_fp8_gemm.argtypes = [P, i32, P, i32, i64, i64, i64, P, P, i32, P, P, P, P]
     L.lm_fp8_gemm.restype = st
     L.lm_fp8_gemm_ex.argtypes = [P, i32, P, i32, i64, i64, i64, ctypes.c_uint32, P, P, i32, P, P,
-                                 P, P]
+                                 P, P, ctypes.c_size_t, P]
     L.lm_fp8_gemm_ex.restype = st
+    L.lm_fp8_gemm_workspace_size.argtypes = []
+    L.lm_fp8_gemm_workspace_size.restype = ctypes.c_size_t
     L.lm_relu2_mlp_saved_bytes.argtypes = [i64, i64, i64]
     L.lm_relu2_mlp_saved_bytes.restype = ctypes.c_size_t
     L.lm_relu2_mlp_saved_carve.argtypes = [P, ctypes.c_size_t, i64, i64, i64,
@@ -91,7 +94,7 @@ def _load():
     L.lm_relu2_mlp_bwd_noalloc_max_bytes.argtypes = []
     L.lm_relu2_mlp_bwd_noalloc_max_bytes.restype = ctypes.c_size_t
     L.lm_relu2_mlp_fwd_ex.argtypes = [P, P, P, i64, i64, i64, P, ctypes.POINTER(MlpSaved),
-                                      ctypes.c_uint32, P]
+                                      P, ctypes.c_size_t, ctypes.c_uint32, P]
     L.lm_relu2_mlp_fwd_ex.restype = st
     L.lm_relu2_mlp_bwd_ex.argtypes = [P, ctypes.POINTER(MlpSaved), i64, i64, i64, P, P, P, P,
                                       ctypes.c_size_t, ctypes.c_uint32, P]
@@ -165,15 +168,25 @@ def lm_fp8_gemm(A, fa, B, fb, inv_scale_a, inv_scale_b, D, epi=EPI_NONE, aux=Non
                            _p(aux), _p(D), _p(amax_out), _stream(stream)), "lm_fp8_gemm")
 
 
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def lm_fp8_gemm_workspace_size():
+    return lib.lm_fp8_gemm_workspace_size()
+
+
 def lm_fp8_gemm_ex(A, fa, B, fb, inv_scale_a, inv_scale_b, D, flags=0, epi=EPI_NONE, aux=None,
-                   amax_out=None, stream=None):
+                   amax_out=None, workspace=None, stream=None):
     """lm_fp8_gemm with per-operand storage: with GEMM_A_MN_MAJOR, A is given as
-    its [K x M] transpose (row-major); with GEMM_B_MN_MAJOR, B as [K x N]."""
+    its [K x M] transpose (row-major); with GEMM_B_MN_MAJOR, B as [K x N].
+    workspace (a device buffer, or None) enables the split-K tail."""
     M, K = (A.shape[1], A.shape[0]) if flags & GEMM_A_MN_MAJOR else tuple(A.shape)
     N, K2 = (B.shape[1], B.shape[0]) if flags & GEMM_B_MN_MAJOR else tuple(B.shape)
     assert K == K2 and tuple(D.shape) == (M, N)
     _check(lib.lm_fp8_gemm_ex(_p(A), fa, _p(B), fb, M, N, K, flags, _p(inv_scale_a),
-                              _p(inv_scale_b), epi, _p(aux), _p(D), _p(amax_out), _stream(stream)),
+                              _p(inv_scale_b), epi, _p(aux), _p(D), _p(amax_out), _p(workspace),
+                              _nbytes(workspace), _stream(stream)),
            "lm_fp8_gemm_ex")
 
 
@@ -201,11 +214,12 @@ def lm_relu2_mlp_saved_carve(buf, M, d, f):
     return s
 
 
-def lm_relu2_mlp_fwd(X, W_up, W_down, Y, saved, stream=None):
+def lm_relu2_mlp_fwd(X, W_up, W_down, Y, saved, workspace=None, stream=None):
     M, d = X.shape
     f = W_up.shape[0]
     _check(lib.lm_relu2_mlp_fwd(_p(X), _p(W_up), _p(W_down), M, d, f, _p(Y),
-                                ctypes.byref(saved), None, 0, _stream(stream)),
+                                ctypes.byref(saved), _p(workspace), _nbytes(workspace),
+                                _stream(stream)),
            "lm_relu2_mlp_fwd")
 
 
@@ -218,11 +232,12 @@ def lm_relu2_mlp_bwd(dY, saved, dX, dW_up, dW_down, workspace, stream=None):
            "lm_relu2_mlp_bwd")
 
 
-def lm_relu2_mlp_fwd_ex(X, W_up, W_down, Y, saved, f, flags=0, stream=None):
+def lm_relu2_mlp_fwd_ex(X, W_up, W_down, Y, saved, f, flags=0, workspace=None, stream=None):
     """f: hidden size (W_up may be None when its cast is reused)."""
     M, d = X.shape
     _check(lib.lm_relu2_mlp_fwd_ex(_p(X), _p(W_up), _p(W_down), M, d, f, _p(Y),
-                                   ctypes.byref(saved), flags, _stream(stream)),
+                                   ctypes.byref(saved), _p(workspace), _nbytes(workspace), flags,
+                                   _stream(stream)),
            "lm_relu2_mlp_fwd_ex")
 
 

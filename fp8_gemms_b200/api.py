@@ -37,16 +37,22 @@ def cast(x, fmt, relu2_input=False, amax_in=None, want_q=True, want_qT=True, sca
     return q, qT, sc
 
 
+def gemm_workspace(device="cuda"):
+    """Scratch that lets a GEMM split its under-filled last wave of tiles."""
+    return torch.empty(_lib.lm_fp8_gemm_workspace_size(), dtype=torch.uint8, device=device)
+
+
 def gemm(A, fa, B, fb, inv_a, inv_b, epi=EPI_NONE, aux=None, amax_out=None, out=None,
-         flags=0, stream=None):
+         flags=0, workspace=None, stream=None):
     """bf16 D[M x N] = epi(A B^T inv_a inv_b) for FP8 codes A [M x K], B [N x K];
     with GEMM_A_MN_MAJOR / GEMM_B_MN_MAJOR in flags, A is given as [K x M] /
-    B as [K x N] (the row-major codes of the transpose)."""
+    B as [K x N] (the row-major codes of the transpose).  workspace: see
+    gemm_workspace (None: no split-K tail)."""
     M = A.shape[1] if flags & GEMM_A_MN_MAJOR else A.shape[0]
     N = B.shape[1] if flags & GEMM_B_MN_MAJOR else B.shape[0]
     D = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=_dev(A))
     _lib.lm_fp8_gemm_ex(A, fa, B, fb, inv_a, inv_b, D, flags=flags, epi=epi, aux=aux,
-                        amax_out=amax_out, stream=stream)
+                        amax_out=amax_out, workspace=workspace, stream=stream)
     return D
 
 
@@ -73,9 +79,11 @@ class Relu2Mlp:
             Y = torch.empty(self.M, self.d, dtype=torch.bfloat16, device=self.device)
         if reuse_weight_casts:
             _lib.lm_relu2_mlp_fwd_ex(X, None, None, Y, self.saved, self.f,
-                                     flags=MLP_REUSE_WEIGHT_CASTS, stream=stream)
+                                     flags=MLP_REUSE_WEIGHT_CASTS, workspace=self.workspace,
+                                     stream=stream)
         else:
-            _lib.lm_relu2_mlp_fwd(X, W_up, W_down, Y, self.saved, stream=stream)
+            _lib.lm_relu2_mlp_fwd(X, W_up, W_down, Y, self.saved, workspace=self.workspace,
+                                  stream=stream)
         return Y
 
     def backward_accumulate(self, dY, dW_up_f32, dW_down_f32, dX=None, stream=None):
@@ -114,11 +122,12 @@ class Relu2Mlp:
         return self.saved_buf[off:off + r * c].view(r, c)
 
     def workspace_view(self, name):
-        """Backward scratch: dYq, dH, dHq, scales (library layout: each buffer
-        rounded up to 256 bytes, in that order)."""
+        """Backward scratch: the GEMMs' split-K scratch, then dYq, dH, dHq,
+        scales (library layout: each buffer rounded up to 256 bytes)."""
         M, d, f = self.M, self.d, self.f
         r256 = lambda n: (n + 255) // 256 * 256
-        sizes = [("dYq", M * d), ("dH", M * f * 2), ("dHq", M * f), ("scales", 32)]
+        sizes = [("split", _lib.lm_fp8_gemm_workspace_size()), ("dYq", M * d),
+                 ("dH", M * f * 2), ("dHq", M * f), ("scales", 32)]
         off = 0
         for n, sz in sizes:
             if n == name:
@@ -228,8 +237,10 @@ def linear_fwd_bwd(X, W, dY, stream=None):
     Xq, _, _ = cast(X, E4M3, want_qT=False, scales=sc[0], stream=stream)
     Wq, _, _ = cast(W, E4M3, want_qT=False, scales=sc[1], stream=stream)
     dYq, _, _ = cast(dY, E5M2, want_qT=False, scales=sc[2], stream=stream)
-    Y = gemm(Xq, E4M3, Wq, E4M3, sc[0, 2:3], sc[1, 2:3], stream=stream)
-    dX = gemm(dYq, E5M2, Wq, E4M3, sc[2, 2:3], sc[1, 2:3], flags=GEMM_B_MN_MAJOR, stream=stream)
+    ws = gemm_workspace(X.device)
+    Y = gemm(Xq, E4M3, Wq, E4M3, sc[0, 2:3], sc[1, 2:3], workspace=ws, stream=stream)
+    dX = gemm(dYq, E5M2, Wq, E4M3, sc[2, 2:3], sc[1, 2:3], flags=GEMM_B_MN_MAJOR, workspace=ws,
+              stream=stream)
     dW = gemm(dYq, E5M2, Xq, E4M3, sc[2, 2:3], sc[0, 2:3],
-              flags=GEMM_A_MN_MAJOR | GEMM_B_MN_MAJOR, stream=stream)
+              flags=GEMM_A_MN_MAJOR | GEMM_B_MN_MAJOR, workspace=ws, stream=stream)
     return Y, dX, dW, dict(Xq=Xq, Wq=Wq, dYq=dYq, scales=sc)

@@ -39,11 +39,33 @@ constexpr int NUM_EPI_WARPS = 4;
 // codes recorded in the device error word when a bounded wait runs out
 enum : unsigned {
     W_EMPTY = 0x101, W_TEMPTY = 0x102, W_FULL = 0x103, W_DRAIN = 0x104, W_TFULL = 0x105,
-    W_LOADS = 0x106, W_AUX = 0x107
+    W_LOADS = 0x106, W_AUX = 0x107, W_SPLIT = 0x108, W_SPLIT_LOAD = 0x109
+};
+
+// Split-K tail.  Tiles go round-robin to the persistent clusters, so a last
+// wave of r < clusters tiles leaves the other clusters idle for a whole tile.
+// When 2r <= clusters, each of those r tiles is computed as two units over
+// the two halves of K, in the same round on two clusters: half 0 writes its
+// fp32 partial sums to a workspace and raises a flag per (CTA, warp); half 1
+// waits for the flag (bounded), copies the partial into its operand ring,
+// which is idle at that point (a split unit is always its cluster's last),
+// and adds it to its own sums before the epilogue.  Partial layout per
+// (tile, CTA rank, TMEM lane quarter): [chunk 8][float4 8][lane 32], so
+// both the writes and the reads are contiguous across a warp.
+constexpr size_t kSplitSlotFloat4 = 8 * 8 * 32;                   // one warp's partial
+constexpr size_t kSplitTileBytes = 2 * NUM_EPI_WARPS * kSplitSlotFloat4 * 16;  // 256 KB
+constexpr int kSplitMaxTiles = 64;
+
+struct WorkUnit {
+    int tile, kb0, kb1;
+    int half;  // -1: a whole tile; 0 / 1: first / second half of a split tile
 };
 
 struct GemmArgs {
     int M, N, num_mb, num_nb, num_kb, num_tiles, group_m;
+    int num_units, split_first;  // units: tiles [0, split_first), then split halves
+    float4* split_ws;            // partial sums of the split tiles
+    unsigned int* split_flags;   // [split tile][rank][quarter], zeroed before the launch
     int a_mn, b_mn;  // 1: the operand is stored MN-major ([K x M] / [K x N], M or N contiguous)
     int stream_a;  // 1: A is the streamed operand (evict-first loads), 0: B is
     const float* inv_a;
@@ -55,6 +77,12 @@ struct GemmArgs {
     unsigned int* err;
     uint32_t idesc;
 };
+
+__device__ __forceinline__ WorkUnit work_unit(int u, const GemmArgs& a) {
+    if (u < a.split_first) return {u, 0, a.num_kb, -1};
+    const int s = u - a.split_first, h = s & 1, kh = a.num_kb >> 1;
+    return {a.split_first + (s >> 1), h ? kh : 0, h ? a.num_kb : kh, h};
+}
 
 // Tile visiting order: groups of group_m row-blocks, column-blocks within a
 // group, so the tiles in flight at once share A and B panels in L2.
@@ -211,7 +239,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     uint64_t* tempty = tfull + 2;           // [2], leader only
     uint64_t* drain = tempty + 2;           // leader only
     uint64_t* auxbar = drain + 1;           // [4 warps][2 buffers]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + 2 * NUM_EPI_WARPS);
+    uint64_t* splitbar = auxbar + 2 * NUM_EPI_WARPS;  // [4 warps]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(splitbar + NUM_EPI_WARPS);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -229,6 +258,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         }
         mbar_init(drain, 1);
         for (int i = 0; i < 2 * NUM_EPI_WARPS; ++i) mbar_init(&auxbar[i], 1);
+        for (int i = 0; i < NUM_EPI_WARPS; ++i) mbar_init(&splitbar[i], 1);
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
@@ -259,12 +289,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0, issued = 0;
             bool ok = true;
-            for (int t = cluster; t < args.num_tiles && ok; t += nclusters) {
+            for (int u = cluster; u < args.num_units && ok; u += nclusters) {
+                const WorkUnit w = work_unit(u, args);
                 int mb, nb;
-                tile_coords(t, args.group_m, args.num_mb, args.num_nb, mb, nb);
+                tile_coords(w.tile, args.group_m, args.num_mb, args.num_nb, mb, nb);
                 const int arow = mb * TILE_M + (int)rank * 128;
                 const int brow = nb * TILE_N + (int)rank * 128;
-                for (int kb = 0; kb < args.num_kb; ++kb) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     // box coordinates (x innermost): K-major (k, m|n), MN-major (m|n, k)
                     const int ax = args.a_mn ? arow : kb * BK, ay = args.a_mn ? kb * BK : arow;
                     const int bx = args.b_mn ? brow : kb * BK, by = args.b_mn ? kb * BK : brow;
@@ -310,11 +341,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             // K-major row, or 32 rows of an MN-major tile
             const uint64_t a_step = args.a_mn ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
             const uint64_t b_step = args.b_mn ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
-            for (int t = cluster; t < args.num_tiles && ok; t += nclusters) {
+            for (int u = cluster; u < args.num_units && ok; u += nclusters) {
+                const WorkUnit w = work_unit(u, args);
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.err, W_TEMPTY)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TILE_N);
-                for (int kb = 0; kb < args.num_kb; ++kb) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait(&full[stage], phase, args.err, W_FULL)) {
                         ok = false;
                         break;
@@ -325,7 +357,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk)
                         mma_fp8_pair(d_tmem, ad + (uint64_t)kk * a_step, bd + (uint64_t)kk * b_step,
-                                     args.idesc, (kb | kk) != 0 ? 1u : 0u);
+                                     args.idesc, (kb != w.kb0 || kk != 0) ? 1u : 0u);
                     mma_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
                     if (++stage == STAGES) {
                         stage = 0;
@@ -356,14 +388,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         uint32_t ax_phase = 0;  // bit b: parity of the next wait on aux buffer b
         uint32_t n_stores = 0;
         bool ok = true;
-        for (int t = cluster; t < args.num_tiles && ok; t += nclusters) {
+        for (int u = cluster; u < args.num_units && ok; u += nclusters) {
+            const WorkUnit w = work_unit(u, args);
             int mb, nb;
-            tile_coords(t, args.group_m, args.num_mb, args.num_nb, mb, nb);
+            tile_coords(w.tile, args.group_m, args.num_mb, args.num_nb, mb, nb);
             const int grow = mb * TILE_M + (int)rank * 128 + quarter * 32;  // row of lane 0
             const int gcol = nb * TILE_N;
             const int left = args.N - gcol;
             const int n_chunks = left >= TILE_N ? TILE_N / EPI_COLS : (left + EPI_COLS - 1) / EPI_COLS;
-            if (EPI == LM_EPI_RELU2_BWD && lane == 0) {
+            // this warp's slot of a split tile's partial sums and flags
+            const size_t slot = w.half < 0 ? 0
+                                           : ((size_t)(w.tile - args.split_first) * 2 + rank) *
+                                                     NUM_EPI_WARPS + quarter;
+            if (EPI == LM_EPI_RELU2_BWD && lane == 0 && w.half != 0) {
                 // the first H box of this tile (no L2 prefetch of the next
                 // tile's H: measured, it raised DRAM reads by a third and cost
                 // 3.6% of this GEMM's time)
@@ -375,6 +412,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const uint32_t tbase =
                 tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * TILE_N);
+            if (w.half == 0) {
+                // first half of a split tile: publish the raw fp32 sums
+                float4* dst = args.split_ws + slot * kSplitSlotFloat4;
+                for (int c = 0; c < n_chunks; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tbase + (uint32_t)(c * EPI_COLS), r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[(c * 8 + i) * 32 + lane] =
+                            make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                        __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                }
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_gpu(args.split_flags + slot, 1u);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(tempty_leader + (uint32_t)(acc * 8));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+                continue;
+            }
+            // second half of a split tile: the first half's sums, copied into
+            // this warp's 32 KB of the operand ring (idle: this is the last unit)
+            const float4* part = nullptr;
+            if (w.half == 1) {
+                bool ready = true;
+                if (lane == 0) ready = flag_wait(args.split_flags + slot, 1u, args.err, W_SPLIT);
+                ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
+                if (ready) {
+                    uint8_t* buf = smem + wi * (int)(kSplitSlotFloat4 * 16);
+                    if (lane == 0) {
+                        const uint32_t bytes = (uint32_t)n_chunks * 8 * 32 * 16;
+                        mbar_arrive_expect_tx(&splitbar[wi], bytes);
+                        bulk_load_1d(smem_addr(buf), args.split_ws + slot * kSplitSlotFloat4, bytes,
+                                     &splitbar[wi]);
+                    }
+                    if (mbar_wait(&splitbar[wi], 0, args.err, W_SPLIT_LOAD))
+                        part = reinterpret_cast<const float4*>(buf);
+                    else  // error recorded; give the copy a second bounded wait before exit
+                        mbar_wait(&splitbar[wi], 0, args.err, W_SPLIT_LOAD);
+                }
+            }
             if (EPI == kEpiSwigluFwd) {
                 // gate columns [0,128) and up columns [128,256) of the tile: store
                 // G, U (bf16, interleaved as computed) and h = bf16(silu(G) U)
@@ -419,6 +500,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tbase + (uint32_t)(c * EPI_COLS), r);
                 tmem_ld_wait();
+                if (part) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 p = part[(c * 8 + i) * 32 + lane];
+                        r[4 * i] = __float_as_uint(__fadd_rn(p.x, __uint_as_float(r[4 * i])));
+                        r[4 * i + 1] = __float_as_uint(__fadd_rn(p.y, __uint_as_float(r[4 * i + 1])));
+                        r[4 * i + 2] = __float_as_uint(__fadd_rn(p.z, __uint_as_float(r[4 * i + 2])));
+                        r[4 * i + 3] = __float_as_uint(__fadd_rn(p.w, __uint_as_float(r[4 * i + 3])));
+                    }
+                }
                 uint32_t hw[16];  // saved H, two bf16 per word, columns 2i and 2i+1
                 if (EPI == LM_EPI_RELU2_BWD) {
                     const int b = c & 1;
@@ -748,8 +839,14 @@ lm_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
     if (!ensure_smem(pair::gemm_fp8_pair_kernel<EPI>, pair::SMEM_BYTES, done)) return LM_ERR_CUDA;
     const int sms = sm_count();
     if (sms < 2) return LM_ERR_CUDA;
-    const int clusters = a.num_tiles < sms / 2 ? a.num_tiles : sms / 2;
+    const int clusters = a.num_units < sms / 2 ? a.num_units : sms / 2;
     timing_mark(s, 'g');
+    if (a.split_flags && a.num_units > a.split_first &&
+        cudaMemsetAsync(a.split_flags, 0,
+                        (size_t)(a.num_units - a.split_first) / 2 * 2 * NUM_EPI_WARPS *
+                            sizeof(unsigned int),
+                        s) != cudaSuccess)
+        return LM_ERR_CUDA;
     pair::gemm_fp8_pair_kernel<EPI><<<2 * clusters, NUM_THREADS, pair::SMEM_BYTES, s>>>(ta, tb, td,
                                                                                       tx, td2, a);
     return launch_status();
@@ -771,11 +868,15 @@ lm_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArg
 }  // namespace
 }  // namespace lm
 
+size_t lm::gemm_split_workspace_bytes() {
+    return (size_t)kSplitMaxTiles * (kSplitTileBytes + 2 * NUM_EPI_WARPS * sizeof(unsigned int));
+}
+
 lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
                             lm_fp8_format fb, int64_t M, int64_t N, int64_t K, uint32_t flags,
                             const float* inv_scale_a, const float* inv_scale_b, int epi,
-                            const void* aux, void* D, void* D2, float* amax_out,
-                            lm_stream_t stream) {
+                            const void* aux, void* D, void* D2, float* amax_out, void* workspace,
+                            size_t ws_bytes, lm_stream_t stream) {
     using namespace lm;
     if ((fa != LM_FP8_E4M3 && fa != LM_FP8_E5M2) || (fb != LM_FP8_E4M3 && fb != LM_FP8_E5M2))
         return LM_ERR_UNSUPPORTED_FORMAT;
@@ -836,6 +937,25 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
         // spanning M).
         a.stream_a = N <= M ? 1 : 0;
         a.group_m = a.stream_a ? 1 : a.num_mb;
+        // split-K tail: with a workspace, a last wave of r tiles on C clusters
+        // with 2r <= C becomes 2r half-K units in the same round
+        a.num_units = a.num_tiles;
+        a.split_first = a.num_tiles;
+        a.split_ws = nullptr;
+        a.split_flags = nullptr;
+        const int sms = sm_count();
+        if (sms < 2) return LM_ERR_CUDA;
+        const int C = sms / 2;
+        const int rem = a.num_tiles % C;
+        if (workspace && epi != kEpiSwigluFwd && a.num_kb >= 2 && rem > 0 && 2 * rem <= C &&
+            rem <= kSplitMaxTiles && aligned16(workspace) &&
+            ws_bytes >= (size_t)rem * (kSplitTileBytes + 2 * NUM_EPI_WARPS * sizeof(unsigned int))) {
+            a.split_first = a.num_tiles - rem;
+            a.num_units = a.num_tiles + rem;
+            a.split_ws = static_cast<float4*>(workspace);
+            a.split_flags = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) +
+                                                            (size_t)rem * kSplitTileBytes);
+        }
         a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, pair::TILE_M, pair::TILE_N, a.a_mn, a.b_mn);
         CUtensorMap td, tx;
         // K-major: [rows x K] boxes of 128 rows x 128 K; MN-major: [K x cols]
@@ -876,6 +996,10 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
     a.num_mb = (int)((M + one::BM - 1) / one::BM);
     a.num_nb = (int)((N + one::BN - 1) / one::BN);
     a.num_tiles = a.num_mb * a.num_nb;
+    a.num_units = a.num_tiles;
+    a.split_first = a.num_tiles;
+    a.split_ws = nullptr;
+    a.split_flags = nullptr;
     a.group_m = 16;
     a.stream_a = 0;
     a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, one::BM, one::BN, a.a_mn, a.b_mn);
@@ -893,16 +1017,19 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
     }
 }
 
+extern "C" size_t lm_fp8_gemm_workspace_size(void) { return lm::gemm_split_workspace_bytes(); }
+
 extern "C" lm_status lm_fp8_gemm_ex(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
                                     lm_fp8_format fb, int64_t M, int64_t N, int64_t K,
                                     uint32_t flags, const float* inv_scale_a,
                                     const float* inv_scale_b, lm_epilogue epi, const void* aux,
-                                    void* D, float* amax_out, lm_stream_t stream) {
+                                    void* D, float* amax_out, void* workspace, size_t ws_bytes,
+                                    lm_stream_t stream) {
     if (epi != LM_EPI_NONE && epi != LM_EPI_RELU2_FWD && epi != LM_EPI_RELU2_BWD &&
         epi != LM_EPI_ACCUM_F32)
         return LM_ERR_UNSUPPORTED_FORMAT;
     return lm::gemm_dispatch(A, fa, B, fb, M, N, K, flags, inv_scale_a, inv_scale_b, (int)epi,
-                             aux, D, nullptr, amax_out, stream);
+                             aux, D, nullptr, amax_out, workspace, ws_bytes, stream);
 }
 
 extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
@@ -911,5 +1038,5 @@ extern "C" lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8
                                  lm_epilogue epi, const void* aux, void* D, float* amax_out,
                                  lm_stream_t stream) {
     return lm_fp8_gemm_ex(A, fa, B, fb, M, N, K, 0u, inv_scale_a, inv_scale_b, epi, aux, D,
-                          amax_out, stream);
+                          amax_out, nullptr, 0, stream);
 }

@@ -46,11 +46,14 @@ bool encode_tmap_bf16_plain(CUtensorMap* map, const void* base, uint64_t rows, u
 // h = bf16(silu(G) U) [M x N/2]; amax_out gets max |h|.
 constexpr int kEpiSwigluFwd = 4;
 
-// lm_fp8_gemm with the internal epilogues and a second output.
+// lm_fp8_gemm_ex with the internal epilogues and a second output.
 lm_status gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B, lm_fp8_format fb,
                         int64_t M, int64_t N, int64_t K, uint32_t flags, const float* inv_scale_a,
                         const float* inv_scale_b, int epi, const void* aux, void* D, void* D2,
-                        float* amax_out, lm_stream_t stream);
+                        float* amax_out, void* workspace, size_t ws_bytes, lm_stream_t stream);
+
+// Workspace bytes that let any GEMM split its last wave (lm_fp8_gemm_workspace_size).
+size_t gemm_split_workspace_bytes();
 
 // One tensor of lm::cast_set: the arguments of lm_fp8_amax_scale_cast.
 struct CastItem {

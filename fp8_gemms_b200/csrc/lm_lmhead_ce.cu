@@ -242,10 +242,10 @@ lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* labels, 
         // dX = dL W (W [V x d] read MN-major); dW += dL^T X (both read MN-major)
         LM_TRY(lm_fp8_gemm_ex(w.dLq, LM_FP8_E5M2, w.Wq, LM_FP8_E4M3, rows, d, V,
                               LM_GEMM_B_MN_MAJOR, SL + 2, SW + 2, LM_EPI_NONE, nullptr,
-                              dXb + c0 * d, nullptr, stream));
+                              dXb + c0 * d, nullptr, nullptr, 0, stream));
         LM_TRY(lm_fp8_gemm_ex(w.dLq, LM_FP8_E5M2, w.Xq, LM_FP8_E4M3, V, d, rows,
                               LM_GEMM_A_MN_MAJOR | LM_GEMM_B_MN_MAJOR, SL + 2, SX + 2,
-                              LM_EPI_ACCUM_F32, nullptr, dW, nullptr, stream));
+                              LM_EPI_ACCUM_F32, nullptr, dW, nullptr, nullptr, 0, stream));
     }
     timing_mark(s, 'l');
     mean_loss_kernel<<<1, 1024, 0, s>>>(w.loss_rows, M, loss_out);

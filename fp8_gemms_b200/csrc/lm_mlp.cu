@@ -25,6 +25,7 @@ enum { S_X = 0, S_WU = 4, S_WD = 8, S_H = 12 };  // in lm_mlp_saved::scales
 enum { S_DY = 0, S_DH = 4 };                      // in the backward workspace
 
 struct BwdWorkspace {
+    void* split;  // the GEMMs' split-K scratch (lm_fp8_gemm_workspace_size bytes)
     uint8_t *dYq, *dHq;
     void* dH;
     float* scales;
@@ -38,11 +39,12 @@ size_t bwd_layout(int64_t M, int64_t d, int64_t f, uint8_t* base, BwdWorkspace* 
         off += round_up(bytes);
         return p;
     };
+    uint8_t* split = take(lm::gemm_split_workspace_bytes());
     uint8_t* dYq = take(Md);
     uint8_t* dH = take(Mf * 2);
     uint8_t* dHq = take(Mf);
     uint8_t* sc = take(8 * sizeof(float));
-    if (w) *w = BwdWorkspace{dYq, dHq, dH, reinterpret_cast<float*>(sc)};
+    if (w) *w = BwdWorkspace{split, dYq, dHq, dH, reinterpret_cast<float*>(sc)};
     return off;
 }
 
@@ -97,15 +99,21 @@ size_t lm_relu2_mlp_workspace_size(int64_t M, int64_t d, int64_t f) {
 }
 
 lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_down, int64_t M,
-                              int64_t d, int64_t f, void* Y, lm_mlp_saved* sv, uint32_t flags,
-                              lm_stream_t stream) {
+                              int64_t d, int64_t f, void* Y, lm_mlp_saved* sv, void* workspace,
+                              size_t ws_bytes, uint32_t flags, lm_stream_t stream) {
     if (!mlp_shape_ok(M, d, f)) return LM_ERR_UNSUPPORTED_SHAPE;
     if (flags & ~LM_MLP_REUSE_WEIGHT_CASTS) return LM_ERR_INVALID_ARG;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+        return LM_ERR_ALIGNMENT;
     const bool reuse = (flags & LM_MLP_REUSE_WEIGHT_CASTS) != 0;
     if (!X || !Y || !sv || (!reuse && (!W_up || !W_down))) return LM_ERR_INVALID_ARG;
     if (!sv->Xq || !sv->Wuq || !sv->Wdq || !sv->H || !sv->hq || !sv->scales)
         return LM_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // the workspace, when given, holds the GEMMs' split-K scratch at its start
+    const size_t split_bytes = lm::gemm_split_workspace_bytes();
+    void* split = workspace && ws_bytes >= split_bytes ? workspace : nullptr;
+    const size_t sb = split ? split_bytes : 0;
     float* S = sv->scales;
     if (reuse) {  // keep the weights' scale blocks; reset X's and h's
         if (cudaMemsetAsync(S + S_X, 0, 4 * sizeof(float), s) != cudaSuccess ||
@@ -123,22 +131,21 @@ lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_dow
         {W_down, d, f, f, nullptr, S + S_WD, S + S_WD + 1, S + S_WD + 2, sv->Wdq, nullptr}};
     LM_TRY(lm::cast_set(in, reuse ? 1 : 3, LM_FP8_E4M3, 0, true, s));
     // H = X W_up^T (bf16) and amax of h = bf16(relu(H)^2)
-    LM_TRY(lm_fp8_gemm(sv->Xq, LM_FP8_E4M3, sv->Wuq, LM_FP8_E4M3, M, f, d, S + S_X + 2,
-                       S + S_WU + 2, LM_EPI_RELU2_FWD, nullptr, sv->H, S + S_H, stream));
+    LM_TRY(lm_fp8_gemm_ex(sv->Xq, LM_FP8_E4M3, sv->Wuq, LM_FP8_E4M3, M, f, d, 0u, S + S_X + 2,
+                          S + S_WU + 2, LM_EPI_RELU2_FWD, nullptr, sv->H, S + S_H, split, sb,
+                          stream));
     LM_TRY(lm_fp8_amax_scale_cast(sv->H, M, f, f, LM_FP8_E4M3, 1, S + S_H, S + S_H, S + S_H + 1,
                                   S + S_H + 2, sv->hq, nullptr, stream));
     // Y = h W_down^T
-    LM_TRY(lm_fp8_gemm(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, S + S_H + 2,
-                       S + S_WD + 2, LM_EPI_NONE, nullptr, Y, nullptr, stream));
+    LM_TRY(lm_fp8_gemm_ex(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, 0u, S + S_H + 2,
+                          S + S_WD + 2, LM_EPI_NONE, nullptr, Y, nullptr, split, sb, stream));
     return LM_OK;
 }
 
 lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W_down, int64_t M,
                            int64_t d, int64_t f, void* Y, lm_mlp_saved* sv, void* workspace,
                            size_t ws_bytes, lm_stream_t stream) {
-    (void)workspace;
-    (void)ws_bytes;
-    return lm_relu2_mlp_fwd_ex(X, W_up, W_down, M, d, f, Y, sv, 0u, stream);
+    return lm_relu2_mlp_fwd_ex(X, W_up, W_down, M, d, f, Y, sv, workspace, ws_bytes, 0u, stream);
 }
 
 lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* sv, int64_t M, int64_t d,
@@ -161,20 +168,22 @@ lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* sv, int64_t M,
                              w.dYq, nullptr};
     LM_TRY(lm::cast_set(&dy, 1, LM_FP8_E5M2, 0, true, s));  // slot zeroed above
     constexpr uint32_t B_MN = LM_GEMM_B_MN_MAJOR, AB_MN = LM_GEMM_A_MN_MAJOR | LM_GEMM_B_MN_MAJOR;
+    const size_t sb = lm::gemm_split_workspace_bytes();
     // dH = bf16(bf16(dY W_down) * 2 relu(H)), and its amax; B = W_down [d x f]
     // read MN-major as the [f x d] operand
     LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->Wdq, LM_FP8_E4M3, M, f, d, B_MN, G + S_DY + 2,
-                          S + S_WD + 2, LM_EPI_RELU2_BWD, sv->H, w.dH, G + S_DH, stream));
+                          S + S_WD + 2, LM_EPI_RELU2_BWD, sv->H, w.dH, G + S_DH, w.split, sb,
+                          stream));
     // dW_down = dY^T h (K = M): dY [M x d] and h [M x f] read MN-major
     LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->hq, LM_FP8_E4M3, d, f, M, AB_MN, G + S_DY + 2,
-                          S + S_H + 2, wgrad_epi, nullptr, dW_down, nullptr, stream));
+                          S + S_H + 2, wgrad_epi, nullptr, dW_down, nullptr, w.split, sb, stream));
     LM_TRY(lm_fp8_amax_scale_cast(w.dH, M, f, f, LM_FP8_E5M2, 0, G + S_DH, G + S_DH,
                                   G + S_DH + 1, G + S_DH + 2, w.dHq, nullptr, stream));
     // dX = dH W_up (W_up [f x d] read MN-major);  dW_up = dH^T X (K = M)
     LM_TRY(lm_fp8_gemm_ex(w.dHq, LM_FP8_E5M2, sv->Wuq, LM_FP8_E4M3, M, d, f, B_MN, G + S_DH + 2,
-                          S + S_WU + 2, LM_EPI_NONE, nullptr, dX, nullptr, stream));
+                          S + S_WU + 2, LM_EPI_NONE, nullptr, dX, nullptr, w.split, sb, stream));
     LM_TRY(lm_fp8_gemm_ex(w.dHq, LM_FP8_E5M2, sv->Xq, LM_FP8_E4M3, f, d, M, AB_MN, G + S_DH + 2,
-                          S + S_X + 2, wgrad_epi, nullptr, dW_up, nullptr, stream));
+                          S + S_X + 2, wgrad_epi, nullptr, dW_up, nullptr, w.split, sb, stream));
     return LM_OK;
 }
 

@@ -182,7 +182,7 @@ lm_status lm_swiglu_mlp_fwd(const void* X, const void* W_gu, const void* W_down,
     if (M > 0)
         LM_TRY(gemm_dispatch(sv->Xq, LM_FP8_E4M3, sv->Wguq, LM_FP8_E4M3, M, 2 * f, d, 0u,
                              S + S_X + 2, S + S_WGU + 2, kEpiSwigluFwd, nullptr, sv->GU, sv->h,
-                             S + S_H, stream));
+                             S + S_H, nullptr, 0, stream));
     LM_TRY(lm_fp8_amax_scale_cast(sv->h, M, f, f, LM_FP8_E4M3, 0, S + S_H, S + S_H, S + S_H + 1,
                                   S + S_H + 2, sv->hq, nullptr, stream));
     LM_TRY(lm_fp8_gemm(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, S + S_H + 2,
@@ -211,9 +211,9 @@ lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* sv, int64_t M
     // (row-major codes read MN-major where the transpose is the operand)
     constexpr uint32_t B_MN = LM_GEMM_B_MN_MAJOR, AB_MN = LM_GEMM_A_MN_MAJOR | LM_GEMM_B_MN_MAJOR;
     LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->Wdq, LM_FP8_E4M3, M, f, d, B_MN, G + S_DY + 2,
-                          S + S_WD + 2, LM_EPI_NONE, nullptr, w.g, nullptr, stream));
+                          S + S_WD + 2, LM_EPI_NONE, nullptr, w.g, nullptr, nullptr, 0, stream));
     LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->hq, LM_FP8_E4M3, d, f, M, AB_MN, G + S_DY + 2,
-                          S + S_H + 2, LM_EPI_NONE, nullptr, dW_down, nullptr, stream));
+                          S + S_H + 2, LM_EPI_NONE, nullptr, dW_down, nullptr, nullptr, 0, stream));
     if (M > 0) {
         int grid = sm_count() * 8;
         if (grid <= 0) return LM_ERR_CUDA;
@@ -227,10 +227,11 @@ lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* sv, int64_t M
                                   G + S_DGU + 1, G + S_DGU + 2, w.dGUq, nullptr, stream));
     // dX = dGU W_gu (K = 2f);  dW_gu = dGU^T X (K = M)
     LM_TRY(lm_fp8_gemm_ex(w.dGUq, LM_FP8_E5M2, sv->Wguq, LM_FP8_E4M3, M, d, 2 * f, B_MN,
-                          G + S_DGU + 2, S + S_WGU + 2, LM_EPI_NONE, nullptr, dX, nullptr, stream));
+                          G + S_DGU + 2, S + S_WGU + 2, LM_EPI_NONE, nullptr, dX, nullptr, nullptr,
+                          0, stream));
     LM_TRY(lm_fp8_gemm_ex(w.dGUq, LM_FP8_E5M2, sv->Xq, LM_FP8_E4M3, 2 * f, d, M, AB_MN,
                           G + S_DGU + 2, S + S_X + 2, LM_EPI_NONE, nullptr, dW_gu, nullptr,
-                          stream));
+                          nullptr, 0, stream));
     return LM_OK;
 }
 

@@ -63,6 +63,8 @@ def main():
     p.add_argument("--epi", default="none", choices=list(EPI))
     p.add_argument("--flags", type=int, default=0,
                    help="operand storage: 1 = A MN-major, 2 = B MN-major, 3 = both")
+    p.add_argument("--no-ws", action="store_true",
+                   help="gemm: no workspace, so no split-K tail")
     p.add_argument("--rows", type=int, default=16384)
     p.add_argument("--cols", type=int, default=3072)
     p.add_argument("--fmt", default="e4m3")
@@ -142,13 +144,16 @@ def main():
         aux = torch.randn(a.M, a.N, device="cuda", generator=gen).to(torch.bfloat16) \
             if epi == EPI_RELU2_BWD else None
         am = torch.zeros(1, device="cuda")
+        ws = None if a.no_ws else torch.empty(_lib.lm_fp8_gemm_workspace_size(),
+                                              dtype=torch.uint8, device="cuda")
         fn = lambda: _lib.lm_fp8_gemm_ex(A, fa, B, fb, ia, ib, D, flags=a.flags, epi=epi, aux=aux,
-                                         amax_out=am)
+                                         amax_out=am, workspace=ws)
         ms = time_it(fn, a.iters, a.warmup, flush)
         flops = 2 * a.M * a.N * a.K
         byts = a.M * a.K + a.N * a.K + 2 * a.M * a.N * (2 if epi == EPI_RELU2_BWD else 1)
         avg = sum(ms) / len(ms)
         out = dict(op="gemm", M=a.M, N=a.N, K=a.K, fa=a.fa, fb=a.fb, epi=a.epi, flags=a.flags,
+                   workspace=not a.no_ws,
                    avg_ms=round(avg, 4), min_ms=round(min(ms), 4),
                    tflops=round(flops / avg / 1e9, 1), algorithmic_bytes=byts)
     else:

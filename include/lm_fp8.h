@@ -146,13 +146,30 @@ LM_API lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8_t* 
  * (tcgen05.mma instruction descriptor, "transpose A/B" bits).
  * Additional requirements: M % 16 == 0 with LM_GEMM_A_MN_MAJOR, N % 16 == 0
  * with LM_GEMM_B_MN_MAJOR (each stored row starts on a 16-byte boundary);
- * unknown flag bits return LM_ERR_INVALID_ARG.  flags == 0 is lm_fp8_gemm.
- * The result is bit-identical to lm_fp8_gemm on the transposed copies.
+ * unknown flag bits return LM_ERR_INVALID_ARG.  With flags == 0 and no
+ * workspace this is lm_fp8_gemm.
+ *
+ * workspace (device, 16-byte aligned, >= lm_fp8_gemm_workspace_size() bytes,
+ * or NULL): scratch for a split-K tail.  The persistent grid gives tiles out
+ * round-robin; when the last wave holds at most half as many tiles as there
+ * are CTA pairs, each of those tiles is computed as two half-K units that run
+ * at once, the second adding the first's fp32 sums (exchanged through the
+ * workspace) before the epilogue.  The result then differs from the
+ * unsplit one only by fp32 summation order; it is the same from call to call.
+ * Calls that share a workspace must not overlap on the GPU.  With NULL
+ * (ws_bytes 0) no tile is split.
+ * Operands stored MN-major give bit-identical results to lm_fp8_gemm on the
+ * transposed copies (with the same workspace choice).
  */
 LM_API lm_status lm_fp8_gemm_ex(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
                          lm_fp8_format fb, int64_t M, int64_t N, int64_t K, uint32_t flags,
                          const float* inv_scale_a, const float* inv_scale_b, lm_epilogue epi,
-                         const void* aux, void* D, float* amax_out, lm_stream_t stream);
+                         const void* aux, void* D, float* amax_out, void* workspace,
+                         size_t ws_bytes, lm_stream_t stream);
+
+/* Workspace bytes that let lm_fp8_gemm_ex split the last wave of any shape
+ * (a fixed size: 64 tiles' fp32 sums and flags, about 16 MB). */
+LM_API size_t lm_fp8_gemm_workspace_size(void);
 
 /*
  * The producer of a GEMM input: RMSNorm, then the dynamic FP8 cast of its
@@ -197,7 +214,9 @@ LM_API size_t lm_relu2_mlp_saved_bytes(int64_t M, int64_t d, int64_t f);
 LM_API lm_status lm_relu2_mlp_saved_carve(void* base, size_t bytes, int64_t M, int64_t d, int64_t f,
                                    lm_mlp_saved* out);
 
-/* Bytes of scratch lm_relu2_mlp_bwd needs (lm_relu2_mlp_fwd needs none). */
+/* Bytes of scratch lm_relu2_mlp_bwd needs.  Its first
+ * lm_fp8_gemm_workspace_size() bytes are the GEMMs' split-K scratch, which is
+ * all lm_relu2_mlp_fwd uses of it (optionally). */
 LM_API size_t lm_relu2_mlp_workspace_size(int64_t M, int64_t d, int64_t f);
 
 /*
@@ -209,7 +228,10 @@ LM_API size_t lm_relu2_mlp_workspace_size(int64_t M, int64_t d, int64_t f);
  * Only row-major codes are made: the backward's GEMMs read them MN-major
  * (lm_fp8_gemm_ex), so no transposed copy is written or saved.
  * X: bf16 [M x d], W_up: bf16 [f x d], W_down: bf16 [d x f], Y: bf16 [M x d].
- * workspace may be NULL (ws_bytes 0).  Requirements: M, d, f multiples of 16.
+ * workspace: NULL (ws_bytes 0), or 256-byte-aligned device scratch of at least
+ * lm_fp8_gemm_workspace_size() bytes (e.g. the backward's workspace), which
+ * lets the GEMMs split an under-filled last wave (see lm_fp8_gemm_ex).
+ * Requirements: M, d, f multiples of 16.
  */
 LM_API lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W_down, int64_t M,
                            int64_t d, int64_t f, void* Y, lm_mlp_saved* saved, void* workspace,
@@ -271,7 +293,8 @@ LM_API size_t lm_relu2_mlp_bwd_noalloc_max_bytes(void);
  */
 LM_API lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_down,
                                      int64_t M, int64_t d, int64_t f, void* Y, lm_mlp_saved* saved,
-                                     uint32_t flags, lm_stream_t stream);
+                                     void* workspace, size_t ws_bytes, uint32_t flags,
+                                     lm_stream_t stream);
 LM_API lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* saved, int64_t M,
                                      int64_t d, int64_t f, void* dX, void* dW_up, void* dW_down,
                                      void* workspace, size_t ws_bytes, uint32_t flags,

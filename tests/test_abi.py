@@ -82,8 +82,12 @@ def test_mlp_sizes_and_carve(L):
     # H, h codes and the scales; scratch dY codes, dH, dH codes, scales
     assert L.lm_relu2_mlp_saved_bytes(M, d, f) == (r(M * d) + 2 * r(f * d) + r(2 * M * f)
                                                    + r(M * f) + r(64))
-    assert L.lm_relu2_mlp_workspace_size(M, d, f) == (r(M * d) + r(2 * M * f) + r(M * f)
-                                                      + r(32))
+    # scratch: the GEMMs' split-K scratch (64 tiles x 256 KB of fp32 sums plus a
+    # flag per CTA and warp), then dY codes, dH, dH codes, scales
+    split = 64 * (256 * 1024 + 2 * 4 * 4)
+    assert L.lib.lm_fp8_gemm_workspace_size() == split
+    assert L.lm_relu2_mlp_workspace_size(M, d, f) == (r(split) + r(M * d) + r(2 * M * f)
+                                                      + r(M * f) + r(32))
     assert L.lm_relu2_mlp_saved_bytes(M, d, 1000) == 0      # f not a multiple of 16
     s = L.MlpSaved()
     base = 0x100000
@@ -100,7 +104,11 @@ def test_newer_entry_points_reject_before_launch(L):
     lib = L.lib
     s = L.MlpSaved()
     # unknown flags
-    assert lib.lm_relu2_mlp_fwd_ex(fake, fake, fake, 256, 256, 1024, fake, C.byref(s), 4, None) == 1
+    assert lib.lm_relu2_mlp_fwd_ex(fake, fake, fake, 256, 256, 1024, fake, C.byref(s), None, 0, 4,
+                                   None) == 1
+    # a forward workspace must be 256-byte aligned
+    assert lib.lm_relu2_mlp_fwd_ex(fake, fake, fake, 256, 256, 1024, fake, C.byref(s), fake + 16,
+                                   1 << 30, 0, None) == 2
     assert lib.lm_relu2_mlp_bwd_ex(fake, C.byref(s), 256, 256, 1024, fake, fake, fake, fake,
                                    1 << 30, 1, None) == 1
     # rmsnorm: eps < 0, cols not a multiple of 16, misaligned weight
@@ -128,10 +136,10 @@ def test_newer_entry_points_reject_before_launch(L):
                            None) == 4
     # operand-storage flags: unknown bits; MN-major rows not 16-byte aligned
     gx = lib.lm_fp8_gemm_ex
-    assert gx(fake, 0, fake, 0, 256, 256, 64, 4, fake, fake, 0, None, fake, None, None) == 1
-    assert gx(fake, 0, fake, 0, 200, 256, 64, 1, fake, fake, 0, None, fake, None, None) == 3
-    assert gx(fake, 0, fake, 0, 256, 264, 64, 2, fake, fake, 0, None, fake, None, None) == 3
-    assert gx(fake, 0, fake, 0, 256, 264, 64, 1, fake, fake, 4, None, fake, None, None) == 4
+    assert gx(fake, 0, fake, 0, 256, 256, 64, 4, fake, fake, 0, None, fake, None, None, 0, None) == 1
+    assert gx(fake, 0, fake, 0, 200, 256, 64, 1, fake, fake, 0, None, fake, None, None, 0, None) == 3
+    assert gx(fake, 0, fake, 0, 256, 264, 64, 2, fake, fake, 0, None, fake, None, None, 0, None) == 3
+    assert gx(fake, 0, fake, 0, 256, 264, 64, 1, fake, fake, 4, None, fake, None, None, 0, None) == 4
     # no-alloc backward: shape beyond its array
     assert lib.lm_relu2_mlp_bwd_noalloc(None, C.byref(s), 16384, 3072, 12288, None, None, None,
                                         None) == 3
