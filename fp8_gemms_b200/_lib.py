@@ -108,7 +108,8 @@ def _load():
     L.lm_swiglu_mlp_saved_carve.restype = st
     L.lm_swiglu_mlp_workspace_size.argtypes = [i64, i64, i64]
     L.lm_swiglu_mlp_workspace_size.restype = ctypes.c_size_t
-    L.lm_swiglu_mlp_fwd.argtypes = [P, P, P, i64, i64, i64, P, ctypes.POINTER(SwigluSaved), P]
+    L.lm_swiglu_mlp_fwd.argtypes = [P, P, P, i64, i64, i64, P, ctypes.POINTER(SwigluSaved), P,
+                                    ctypes.c_size_t, P]
     L.lm_swiglu_mlp_fwd.restype = st
     L.lm_swiglu_mlp_bwd.argtypes = [P, ctypes.POINTER(SwigluSaved), i64, i64, i64, P, P, P, P,
                                     ctypes.c_size_t, P]
@@ -267,11 +268,12 @@ def lm_swiglu_mlp_saved_carve(buf, M, d, f):
     return s
 
 
-def lm_swiglu_mlp_fwd(X, W_gu, W_down, Y, saved, stream=None):
+def lm_swiglu_mlp_fwd(X, W_gu, W_down, Y, saved, workspace=None, stream=None):
     M, d = X.shape
     f = W_gu.shape[0] // 2
     _check(lib.lm_swiglu_mlp_fwd(_p(X), _p(W_gu), _p(W_down), M, d, f, _p(Y),
-                                 ctypes.byref(saved), _stream(stream)), "lm_swiglu_mlp_fwd")
+                                 ctypes.byref(saved), _p(workspace), _nbytes(workspace),
+                                 _stream(stream)), "lm_swiglu_mlp_fwd")
 
 
 def lm_swiglu_mlp_bwd(dY, saved, dX, dW_gu, dW_down, workspace, stream=None):

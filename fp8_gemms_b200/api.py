@@ -173,7 +173,8 @@ class SwigluMlp:
     def forward(self, X, W_gu, W_down, Y=None, stream=None):
         Y = Y if Y is not None else torch.empty(self.M, self.d, dtype=torch.bfloat16,
                                                 device=self.device)
-        _lib.lm_swiglu_mlp_fwd(X, W_gu, W_down, Y, self.saved, stream=stream)
+        _lib.lm_swiglu_mlp_fwd(X, W_gu, W_down, Y, self.saved, workspace=self.workspace,
+                               stream=stream)
         return Y
 
     def backward(self, dY, dX=None, dW_gu=None, dW_down=None, stream=None):

@@ -51,6 +51,7 @@ size_t saved_layout(int64_t M, int64_t d, int64_t f, uint8_t* base, lm_swiglu_sa
 }
 
 struct BwdWs {
+    void* split;  // the GEMMs' split-K scratch
     uint8_t *dYq, *dGUq;
     void *g, *dGU;
     float* scales;
@@ -65,6 +66,7 @@ size_t bwd_layout(int64_t M, int64_t d, int64_t f, uint8_t* base, BwdWs* w) {
         return p;
     };
     BwdWs o;
+    o.split = take(gemm_split_workspace_bytes());
     o.dYq = take(Md);
     o.g = take(Mf * 2);
     o.dGU = take(2 * Mf * 2);
@@ -162,10 +164,14 @@ size_t lm_swiglu_mlp_workspace_size(int64_t M, int64_t d, int64_t f) {
 }
 
 lm_status lm_swiglu_mlp_fwd(const void* X, const void* W_gu, const void* W_down, int64_t M,
-                            int64_t d, int64_t f, void* Y, lm_swiglu_saved* sv,
-                            lm_stream_t stream) {
+                            int64_t d, int64_t f, void* Y, lm_swiglu_saved* sv, void* workspace,
+                            size_t ws_bytes, lm_stream_t stream) {
     using namespace lm;
     if (!shape_ok(M, d, f)) return LM_ERR_UNSUPPORTED_SHAPE;
+    if (workspace && reinterpret_cast<uintptr_t>(workspace) % kAlign) return LM_ERR_ALIGNMENT;
+    // the workspace, when given, holds the GEMMs' split-K scratch at its start
+    void* split = workspace && ws_bytes >= gemm_split_workspace_bytes() ? workspace : nullptr;
+    const size_t sb = split ? gemm_split_workspace_bytes() : 0;
     if (!X || !W_gu || !W_down || !Y || !sv || !sv->Xq || !sv->Wguq || !sv->Wdq || !sv->GU ||
         !sv->h || !sv->hq || !sv->scales)
         return LM_ERR_INVALID_ARG;
@@ -185,8 +191,8 @@ lm_status lm_swiglu_mlp_fwd(const void* X, const void* W_gu, const void* W_down,
                              S + S_H, nullptr, 0, stream));
     LM_TRY(lm_fp8_amax_scale_cast(sv->h, M, f, f, LM_FP8_E4M3, 0, S + S_H, S + S_H, S + S_H + 1,
                                   S + S_H + 2, sv->hq, nullptr, stream));
-    LM_TRY(lm_fp8_gemm(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, S + S_H + 2,
-                       S + S_WD + 2, LM_EPI_NONE, nullptr, Y, nullptr, stream));
+    LM_TRY(lm_fp8_gemm_ex(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, 0u, S + S_H + 2,
+                          S + S_WD + 2, LM_EPI_NONE, nullptr, Y, nullptr, split, sb, stream));
     return LM_OK;
 }
 
@@ -210,10 +216,11 @@ lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* sv, int64_t M
     // g = dY W_down (plain bf16), dW_down = dY^T h
     // (row-major codes read MN-major where the transpose is the operand)
     constexpr uint32_t B_MN = LM_GEMM_B_MN_MAJOR, AB_MN = LM_GEMM_A_MN_MAJOR | LM_GEMM_B_MN_MAJOR;
+    const size_t sb = gemm_split_workspace_bytes();
     LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->Wdq, LM_FP8_E4M3, M, f, d, B_MN, G + S_DY + 2,
-                          S + S_WD + 2, LM_EPI_NONE, nullptr, w.g, nullptr, nullptr, 0, stream));
+                          S + S_WD + 2, LM_EPI_NONE, nullptr, w.g, nullptr, w.split, sb, stream));
     LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->hq, LM_FP8_E4M3, d, f, M, AB_MN, G + S_DY + 2,
-                          S + S_H + 2, LM_EPI_NONE, nullptr, dW_down, nullptr, nullptr, 0, stream));
+                          S + S_H + 2, LM_EPI_NONE, nullptr, dW_down, nullptr, w.split, sb, stream));
     if (M > 0) {
         int grid = sm_count() * 8;
         if (grid <= 0) return LM_ERR_CUDA;
@@ -227,11 +234,11 @@ lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* sv, int64_t M
                                   G + S_DGU + 1, G + S_DGU + 2, w.dGUq, nullptr, stream));
     // dX = dGU W_gu (K = 2f);  dW_gu = dGU^T X (K = M)
     LM_TRY(lm_fp8_gemm_ex(w.dGUq, LM_FP8_E5M2, sv->Wguq, LM_FP8_E4M3, M, d, 2 * f, B_MN,
-                          G + S_DGU + 2, S + S_WGU + 2, LM_EPI_NONE, nullptr, dX, nullptr, nullptr,
-                          0, stream));
+                          G + S_DGU + 2, S + S_WGU + 2, LM_EPI_NONE, nullptr, dX, nullptr, w.split,
+                          sb, stream));
     LM_TRY(lm_fp8_gemm_ex(w.dGUq, LM_FP8_E5M2, sv->Xq, LM_FP8_E4M3, 2 * f, d, M, AB_MN,
                           G + S_DGU + 2, S + S_X + 2, LM_EPI_NONE, nullptr, dW_gu, nullptr,
-                          nullptr, 0, stream));
+                          w.split, sb, stream));
     return LM_OK;
 }
 

@@ -333,7 +333,7 @@ LM_API lm_status lm_swiglu_mlp_saved_carve(void* base, size_t bytes, int64_t M, 
 LM_API size_t lm_swiglu_mlp_workspace_size(int64_t M, int64_t d, int64_t f);
 LM_API lm_status lm_swiglu_mlp_fwd(const void* X, const void* W_gu, const void* W_down,
                                    int64_t M, int64_t d, int64_t f, void* Y, lm_swiglu_saved* saved,
-                                   lm_stream_t stream);
+                                   void* workspace, size_t ws_bytes, lm_stream_t stream);
 LM_API lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* saved, int64_t M,
                                    int64_t d, int64_t f, void* dX, void* dW_gu, void* dW_down,
                                    void* workspace, size_t ws_bytes, lm_stream_t stream);

@@ -122,7 +122,8 @@ def test_newer_entry_points_reject_before_launch(L):
     # swiglu: f must be a multiple of 128
     assert L.lib.lm_swiglu_mlp_saved_bytes(256, 256, 200) == 0
     sw = L.SwigluSaved()
-    assert lib.lm_swiglu_mlp_fwd(fake, fake, fake, 256, 256, 200, fake, C.byref(sw), None) == 3
+    assert lib.lm_swiglu_mlp_fwd(fake, fake, fake, 256, 256, 200, fake, C.byref(sw), None, 0,
+                                 None) == 3
     # lm head: chunk not a multiple of 16, softcap <= 0, workspace too small
     assert lib.lm_fp8_lmhead_ce_workspace_size(64, 64, 128, 24) == 0
     n = lib.lm_fp8_lmhead_ce_workspace_size(64, 64, 128, 32)
