@@ -446,6 +446,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     uint8_t* buf = smem + wi * (int)(kSplitSlotFloat4 * 16);
                     if (lane == 0) {
                         const uint32_t bytes = (uint32_t)n_chunks * 8 * 32 * 16;
+                        fence_proxy_async_global();  // the acquired sums, then the bulk read
                         mbar_arrive_expect_tx(&splitbar[wi], bytes);
                         bulk_load_1d(smem_addr(buf), args.split_ws + slot * kSplitSlotFloat4, bytes,
                                      &splitbar[wi]);

@@ -295,6 +295,13 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                  : "memory");
 }
 
+// Order this thread's earlier generic-proxy view of global memory (e.g. data
+// another CTA published and this thread acquired) before its later
+// async-proxy (bulk copy) reads of it.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // 1-D bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
 // from this GPU's global memory into this CTA's shared memory, completing on
 // the mbarrier at `bar` (no multicast).
