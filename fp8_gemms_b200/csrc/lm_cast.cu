@@ -30,8 +30,6 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     return v;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // Two packed bf16 x -> two packed h = bf16(relu(x)^2): a NaN-propagating max
 // with 0 (relu(NaN) stays NaN), then one bf16x2 multiply, which rounds the
@@ -54,15 +52,32 @@ __device__ __forceinline__ uint32_t cvt_pair(float lo, float hi) {
     return r;
 }
 
+// Two packed bf16 -> two fp32 products fp32(v * scale), one packed f32x2
+// multiply (two IEEE round-to-nearest fp32 multiplies); scale2 = {scale, scale}.
+__device__ __forceinline__ void mul_bf16x2_f32(uint32_t w, uint64_t scale2, float& lo, float& hi) {
+    uint64_t x, r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(x), "l"(scale2));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+
+__device__ __forceinline__ uint64_t splat_f32x2(float s) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(s));
+    return r;
+}
+
 // 8 bf16 (16 bytes) -> 8 codes (8 bytes), code = fp8(fp32(v * scale)).
 template <int FMT, bool RELU2>
 __device__ __forceinline__ uint2 convert8(uint4 v, float scale) {
+    const uint64_t scale2 = splat_f32x2(scale);
     uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t p[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t x = RELU2 ? relu2_bf16x2(w[i]) : w[i];
-        p[i] = cvt_pair<FMT>(__fmul_rn(bf16_lo(x), scale), __fmul_rn(bf16_hi(x), scale));
+        float lo, hi;
+        mul_bf16x2_f32(RELU2 ? relu2_bf16x2(w[i]) : w[i], scale2, lo, hi);
+        p[i] = cvt_pair<FMT>(lo, hi);
     }
     return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
 }
