@@ -395,7 +395,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int grow = mb * TILE_M + (int)rank * 128 + quarter * 32;  // row of lane 0
             const int gcol = nb * TILE_N;
             const int left = args.N - gcol;
-            const int n_chunks = left >= TILE_N ? TILE_N / EPI_COLS : (left + EPI_COLS - 1) / EPI_COLS;
+            const int n_chunks =
+                left >= TILE_N ? TILE_N / EPI_COLS : (left + EPI_COLS - 1) / EPI_COLS;
             // this warp's slot of a split tile's partial sums and flags
             const size_t slot = w.half < 0 ? 0
                                            : ((size_t)(w.tile - args.split_first) * 2 + rank) *
@@ -421,9 +422,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
-                        dst[(c * 8 + i) * 32 + lane] =
-                            make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                        __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                        dst[(c * 8 + i) * 32 + lane] = make_float4(
+                            __uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                            __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
                 }
                 __threadfence();
                 __syncwarp();
@@ -457,7 +458,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         mbar_wait(&splitbar[wi], 0, args.err, W_SPLIT_LOAD);
                 }
             }
-            if (EPI == kEpiSwigluFwd) {
+            if constexpr (EPI == kEpiSwigluFwd) {
                 // gate columns [0,128) and up columns [128,256) of the tile: store
                 // G, U (bf16, interleaved as computed) and h = bf16(silu(G) U)
                 for (int c = 0; c < TILE_N / 2 / EPI_COLS; ++c) {
@@ -487,99 +488,96 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                                     gcol + c * EPI_COLS, grow, stream_policy, lane);
                     stage_box_store(sStore + wi * 2 * ACC_BOX_BYTES, n_stores, pu, &tmD,
                                     gcol + TILE_N / 2 + c * EPI_COLS, grow, stream_policy, lane);
-                    stage_box_store(sStore + wi * 2 * ACC_BOX_BYTES, n_stores, ph, &tmD2, hcol, grow,
-                                    stream_policy, lane);
+                    stage_box_store(sStore + wi * 2 * ACC_BOX_BYTES, n_stores, ph, &tmD2, hcol,
+                                    grow, stream_policy, lane);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote(tempty_leader + (uint32_t)(acc * 8));
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1u;
-                continue;
-            }
-            for (int c = 0; c < n_chunks; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tbase + (uint32_t)(c * EPI_COLS), r);
-                tmem_ld_wait();
-                if (part) {
+            } else {
+                for (int c = 0; c < n_chunks; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tbase + (uint32_t)(c * EPI_COLS), r);
+                    tmem_ld_wait();
+                    if (part) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 p = part[(c * 8 + i) * 32 + lane];
-                        r[4 * i] = __float_as_uint(__fadd_rn(p.x, __uint_as_float(r[4 * i])));
-                        r[4 * i + 1] = __float_as_uint(__fadd_rn(p.y, __uint_as_float(r[4 * i + 1])));
-                        r[4 * i + 2] = __float_as_uint(__fadd_rn(p.z, __uint_as_float(r[4 * i + 2])));
-                        r[4 * i + 3] = __float_as_uint(__fadd_rn(p.w, __uint_as_float(r[4 * i + 3])));
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 p = part[(c * 8 + i) * 32 + lane];
+                            const float q[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                r[4 * i + e] =
+                                    __float_as_uint(__fadd_rn(q[e], __uint_as_float(r[4 * i + e])));
+                        }
                     }
-                }
-                uint32_t hw[16];  // saved H, two bf16 per word, columns 2i and 2i+1
-                if (EPI == LM_EPI_RELU2_BWD) {
-                    const int b = c & 1;
-                    if (lane == 0 && c + 1 < n_chunks) {
+                    uint32_t hw[16];  // saved H, two bf16 per word, columns 2i and 2i+1
+                    if (EPI == LM_EPI_RELU2_BWD) {
+                        const int b = c & 1;
+                        if (lane == 0 && c + 1 < n_chunks) {
+                            fence_proxy_async_smem();
+                            mbar_arrive_expect_tx(&ax_bar[b ^ 1], BOX_BYTES);
+                            tma_load_2d_hint(smem_addr(ax_buf + (b ^ 1) * BOX_BYTES), &tmAux,
+                                             &ax_bar[b ^ 1], gcol + (c + 1) * EPI_COLS, grow,
+                                             stream_policy);
+                        }
+                        if (!mbar_wait(&ax_bar[b], (ax_phase >> b) & 1u, args.err, W_AUX)) {
+                            ok = false;
+                            break;
+                        }
+                        ax_phase ^= 1u << b;
+                        const uint8_t* src = ax_buf + b * BOX_BYTES;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint4 v = *reinterpret_cast<const uint4*>(src + sw64(lane, j));
+                            hw[4 * j] = v.x;
+                            hw[4 * j + 1] = v.y;
+                            hw[4 * j + 2] = v.z;
+                            hw[4 * j + 3] = v.w;
+                        }
+                    }
+                    if constexpr (EPI == LM_EPI_ACCUM_F32) {
+                        // fp32 partial -> 128B-swizzled 32 x 32 fp32 box -> TMA reduce-add
+                        uint8_t* dst =
+                            sStore + wi * 2 * ACC_BOX_BYTES + (n_stores & 1u) * ACC_BOX_BYTES;
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            *reinterpret_cast<float4*>(dst + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                                make_float4(__fmul_rn(__uint_as_float(r[4 * j]), s),
+                                            __fmul_rn(__uint_as_float(r[4 * j + 1]), s),
+                                            __fmul_rn(__uint_as_float(r[4 * j + 2]), s),
+                                            __fmul_rn(__uint_as_float(r[4 * j + 3]), s));
                         fence_proxy_async_smem();
-                        mbar_arrive_expect_tx(&ax_bar[b ^ 1], BOX_BYTES);
-                        tma_load_2d_hint(smem_addr(ax_buf + (b ^ 1) * BOX_BYTES), &tmAux,
-                                         &ax_bar[b ^ 1], gcol + (c + 1) * EPI_COLS, grow,
-                                         stream_policy);
-                    }
-                    if (!mbar_wait(&ax_bar[b], (ax_phase >> b) & 1u, args.err, W_AUX)) {
-                        ok = false;
-                        break;
-                    }
-                    ax_phase ^= 1u << b;
-                    const uint8_t* src = ax_buf + b * BOX_BYTES;
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_reduce_add_2d(&tmD, smem_addr(dst), gcol + c * EPI_COLS, grow);
+                            bulk_commit_group();
+                        }
+                        ++n_stores;
+                    } else {
+                        uint32_t packed[16];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint4 v = *reinterpret_cast<const uint4*>(src + sw64(lane, j));
-                        hw[4 * j] = v.x;
-                        hw[4 * j + 1] = v.y;
-                        hw[4 * j + 2] = v.z;
-                        hw[4 * j + 3] = v.w;
+                        for (int i = 0; i < 16; ++i)
+                            packed[i] = epi_pair<EPI>(r[2 * i], r[2 * i + 1], s,
+                                                      EPI == LM_EPI_RELU2_BWD ? hw[i] : 0u, amax2);
+                        // staging buffer n_stores & 1: the store that last used it must
+                        // have finished reading shared memory
+                        uint8_t* dst = st_buf + (n_stores & 1u) * BOX_BYTES;
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4*>(dst + sw64(lane, j)) =
+                                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                                           packed[4 * j + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d_hint(&tmD, smem_addr(dst), gcol + c * EPI_COLS, grow,
+                                              stream_policy);
+                            bulk_commit_group();
+                        }
+                        ++n_stores;
                     }
                 }
-                if (EPI == LM_EPI_ACCUM_F32) {
-                    // fp32 partial -> 128B-swizzled 32 x 32 fp32 box -> TMA reduce-add
-                    uint8_t* dst = sStore + wi * 2 * ACC_BOX_BYTES + (n_stores & 1u) * ACC_BOX_BYTES;
-                    if (lane == 0) bulk_wait_group_read<1>();
-                    __syncwarp();
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<float4*>(dst + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                            make_float4(__fmul_rn(__uint_as_float(r[4 * j]), s),
-                                        __fmul_rn(__uint_as_float(r[4 * j + 1]), s),
-                                        __fmul_rn(__uint_as_float(r[4 * j + 2]), s),
-                                        __fmul_rn(__uint_as_float(r[4 * j + 3]), s));
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_reduce_add_2d(&tmD, smem_addr(dst), gcol + c * EPI_COLS, grow);
-                        bulk_commit_group();
-                    }
-                    ++n_stores;
-                    continue;
-                }
-                uint32_t packed[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    packed[i] = epi_pair<EPI>(r[2 * i], r[2 * i + 1], s,
-                                              EPI == LM_EPI_RELU2_BWD ? hw[i] : 0u, amax2);
-                // staging buffer n_stores & 1: the store that last used it must
-                // have finished reading shared memory
-                uint8_t* dst = st_buf + (n_stores & 1u) * BOX_BYTES;
-                if (lane == 0) bulk_wait_group_read<1>();
-                __syncwarp();
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    *reinterpret_cast<uint4*>(dst + sw64(lane, j)) =
-                        make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
-                                   packed[4 * j + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d_hint(&tmD, smem_addr(dst), gcol + c * EPI_COLS, grow,
-                                      stream_policy);
-                    bulk_commit_group();
-                }
-                ++n_stores;
             }
             tc_fence_before();
             __syncwarp();
@@ -764,7 +762,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tmem_ld_wait();
                 if (!row_ok) continue;
                 const int64_t off = (int64_t)row * args.N + col0;
-                if (EPI == LM_EPI_ACCUM_F32) {
+                if constexpr (EPI == LM_EPI_ACCUM_F32) {
                     // each element has one owner thread: a plain read-modify-write
                     float* Df = static_cast<float*>(args.D) + off;
 #pragma unroll
@@ -777,27 +775,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         d4.w = __fadd_rn(d4.w, __fmul_rn(__uint_as_float(r[4 * v + 3]), s));
                         *reinterpret_cast<float4*>(Df + v * 4) = d4;
                     }
-                    continue;
-                }
+                } else {
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    if (col0 + v * 8 >= args.N) break;
-                    uint32_t hb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-                    if (EPI == LM_EPI_RELU2_BWD) {
-                        const uint4 a4 = *reinterpret_cast<const uint4*>(args.aux + off + v * 8);
-                        const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w};
+                    for (int v = 0; v < 4; ++v) {
+                        if (col0 + v * 8 >= args.N) break;
+                        uint32_t hb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                        if (EPI == LM_EPI_RELU2_BWD) {
+                            const uint4 a4 =
+                                *reinterpret_cast<const uint4*>(args.aux + off + v * 8);
+                            const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            hb[2 * i] = aw[i] & 0xFFFFu;
-                            hb[2 * i + 1] = aw[i] >> 16;
+                            for (int i = 0; i < 4; ++i) {
+                                hb[2 * i] = aw[i] & 0xFFFFu;
+                                hb[2 * i + 1] = aw[i] >> 16;
+                            }
                         }
-                    }
-                    uint32_t ob[8];
+                        uint32_t ob[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) ob[i] = epi_value<EPI>(r[v * 8 + i], s, hb[i], amax);
-                    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(args.D) + off + v * 8) =
-                        make_uint4(ob[0] | (ob[1] << 16), ob[2] | (ob[3] << 16),
-                                   ob[4] | (ob[5] << 16), ob[6] | (ob[7] << 16));
+                        for (int i = 0; i < 8; ++i)
+                            ob[i] = epi_value<EPI>(r[v * 8 + i], s, hb[i], amax);
+                        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(args.D) + off + v * 8) =
+                            make_uint4(ob[0] | (ob[1] << 16), ob[2] | (ob[3] << 16),
+                                       ob[4] | (ob[5] << 16), ob[6] | (ob[7] << 16));
+                    }
                 }
             }
             tc_fence_before();
@@ -950,7 +950,8 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
         const int rem = a.num_tiles % C;
         if (workspace && epi != kEpiSwigluFwd && a.num_kb >= 2 && rem > 0 && 2 * rem <= C &&
             rem <= kSplitMaxTiles && aligned16(workspace) &&
-            ws_bytes >= (size_t)rem * (kSplitTileBytes + 2 * NUM_EPI_WARPS * sizeof(unsigned int))) {
+            ws_bytes >=
+                (size_t)rem * (kSplitTileBytes + 2 * NUM_EPI_WARPS * sizeof(unsigned int))) {
             a.split_first = a.num_tiles - rem;
             a.num_units = a.num_tiles + rem;
             a.split_ws = static_cast<float4*>(workspace);

@@ -167,6 +167,118 @@ __global__ void __launch_bounds__(kCeThreads)
     }
 }
 
+// ---------------------------------------------------------------------
+// The same computation with the softcap written through r = sigmoid(-2y),
+// y = l / c: then tanh(y) = 1 - 2r, z = c - 2cr, exp(z - c) = exp(-2cr) and
+// the softcap's derivative 1 - tanh(y)^2 = 4r(1 - r).  Every term exp(z - c)
+// is at most 1, so the row's log-sum-exp needs no running maximum:
+// lse = c + log(sum exp(-2cr)).  Per logit and pass that is three hardware
+// transcendentals (two base-2 exponentials and a reciprocal) instead of a
+// division, tanhf and expf.  Used for softcaps up to kFastCeMaxCap, where
+// exp(-2c) stays a normal fp32 number (no term can flush to zero).
+constexpr float kFastCeMaxCap = 40.0f;
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// r = 1 / (exp(2 l / c) + 1); k2 = 2 log2(e) / c
+__device__ __forceinline__ float softcap_r(float l, float k2) {
+    return rcp_approx(__fadd_rn(ex2_approx(__fmul_rn(l, k2)), 1.0f));
+}
+
+__global__ void __launch_bounds__(kCeThreads)
+    softcap_ce_fast_kernel(uint16_t* __restrict__ logits, const int32_t* __restrict__ labels,
+                           int V, float c, float inv_count, float* __restrict__ loss_rows,
+                           unsigned int* __restrict__ amax_bits, unsigned int* err) {
+    const int64_t row = blockIdx.x;
+    uint4* lv = reinterpret_cast<uint4*>(logits + row * (int64_t)V);
+    const int nv = V >> 3;
+    int label = labels[row];
+    const bool label_ok = (unsigned)label < (unsigned)V;  // never read outside the row
+    if (!label_ok) {
+        if (threadIdx.x == 0) atomicCAS(err, 0u, 0x401u);
+        label = -1;  // no target: loss = lse, no one-hot term
+    }
+    const float log2e = 1.4426950408889634f;
+    const float k2 = __fdiv_rn(2.0f * log2e, c);  // exp(2y) = 2^(l k2)
+    const float kz = -2.0f * log2e * c;           // exp(z - c) = 2^(kz r)
+    float sum = 0.f;
+    for (int v = threadIdx.x; v < nv; v += kCeThreads) {
+        const uint4 x = lv[v];
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float r0 = softcap_r(__uint_as_float(w[i] << 16), k2);
+            const float r1 = softcap_r(__uint_as_float(w[i] & 0xFFFF0000u), k2);
+            sum = __fadd_rn(sum, ex2_approx(__fmul_rn(kz, r0)));
+            sum = __fadd_rn(sum, ex2_approx(__fmul_rn(kz, r1)));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, o));
+    __shared__ float ws[kCeThreads / 32];
+    __shared__ float s_inv_sum;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) ws[warp] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float S = 0.f;
+        for (int i = 0; i < kCeThreads / 32; ++i) S = __fadd_rn(S, ws[i]);
+        const float lse = __fadd_rn(c, logf(S));
+        float zl = 0.0f;
+        if (label_ok) {
+            const float l = __uint_as_float((uint32_t)logits[row * (int64_t)V + label] << 16);
+            zl = __fsub_rn(c, __fmul_rn(2.0f * c, softcap_r(l, k2)));
+        }
+        loss_rows[row] = __fsub_rn(lse, zl);
+        s_inv_sum = __fdiv_rn(1.0f, S);
+    }
+    __syncthreads();
+    const float inv_sum = s_inv_sum;
+    const float g4 = 4.0f * inv_count;  // (1 - t^2) = 4 r (1 - r), times 1/M
+    uint32_t m2 = 0;
+    for (int v = threadIdx.x; v < nv; v += kCeThreads) {
+        const uint4 x = lv[v];
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float g[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float l = __uint_as_float(h ? (w[i] & 0xFFFF0000u) : (w[i] << 16));
+                const float r = softcap_r(l, k2);
+                float p = __fmul_rn(ex2_approx(__fmul_rn(kz, r)), inv_sum);  // exp(z - lse)
+                if (8 * v + 2 * i + h == label) p = __fsub_rn(p, 1.0f);
+                g[h] = __fmul_rn(__fmul_rn(p, __fmul_rn(r, __fsub_rn(1.0f, r))), g4);
+            }
+            const __nv_bfloat162 b = __floats2bfloat162_rn(g[0], g[1]);
+            o[i] = *reinterpret_cast<const uint32_t*>(&b);
+            m2 = __vmaxu2(m2, o[i] & 0x7FFF7FFFu);
+        }
+        lv[v] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    uint32_t mm = max(m2 & 0xFFFFu, m2 >> 16);
+    mm = __reduce_max_sync(0xFFFFFFFFu, mm);
+    __shared__ uint32_t wm[kCeThreads / 32];
+    if (lane == 0) wm[warp] = mm;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int i = 0; i < kCeThreads / 32; ++i) b = max(b, wm[i]);
+        if (b) atomicMax(amax_bits, b << 16);
+    }
+}
+
 // mean of the row losses: fixed-order fp64 sum in one block (deterministic)
 __global__ void __launch_bounds__(1024) mean_loss_kernel(const float* __restrict__ rows, int64_t n,
                                                          float* __restrict__ out) {
@@ -233,9 +345,14 @@ lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* labels, 
                            LM_EPI_NONE, nullptr, w.logits, nullptr, stream));
         if (cudaMemsetAsync(SL, 0, 4 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
         timing_mark(s, 'e');
-        softcap_ce_kernel<<<(unsigned)rows, kCeThreads, 0, s>>>(
-            w.logits, labels + c0, (int)V, softcap, (float)(1.0 / (double)M), w.loss_rows + c0,
-            reinterpret_cast<unsigned int*>(SL), err);
+        if (softcap <= kFastCeMaxCap)
+            softcap_ce_fast_kernel<<<(unsigned)rows, kCeThreads, 0, s>>>(
+                w.logits, labels + c0, (int)V, softcap, (float)(1.0 / (double)M),
+                w.loss_rows + c0, reinterpret_cast<unsigned int*>(SL), err);
+        else
+            softcap_ce_kernel<<<(unsigned)rows, kCeThreads, 0, s>>>(
+                w.logits, labels + c0, (int)V, softcap, (float)(1.0 / (double)M),
+                w.loss_rows + c0, reinterpret_cast<unsigned int*>(SL), err);
         if (launch_status() != LM_OK) return LM_ERR_CUDA;
         LM_TRY(lm_fp8_amax_scale_cast(w.logits, rows, V, V, LM_FP8_E5M2, 0, SL, SL, SL + 1,
                                       SL + 2, w.dLq, nullptr, stream));

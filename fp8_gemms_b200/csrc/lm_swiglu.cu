@@ -220,7 +220,8 @@ lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* sv, int64_t M
     LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->Wdq, LM_FP8_E4M3, M, f, d, B_MN, G + S_DY + 2,
                           S + S_WD + 2, LM_EPI_NONE, nullptr, w.g, nullptr, w.split, sb, stream));
     LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->hq, LM_FP8_E4M3, d, f, M, AB_MN, G + S_DY + 2,
-                          S + S_H + 2, LM_EPI_NONE, nullptr, dW_down, nullptr, w.split, sb, stream));
+                          S + S_H + 2, LM_EPI_NONE, nullptr, dW_down, nullptr, w.split, sb,
+                          stream));
     if (M > 0) {
         int grid = sm_count() * 8;
         if (grid <= 0) return LM_ERR_CUDA;

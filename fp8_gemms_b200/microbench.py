@@ -116,10 +116,22 @@ def main():
         ms = time_it(fn, a.iters, a.warmup, flush)
         avg = sum(ms) / len(ms)
         flops = 3 * 2 * M * d * V
+        # one more call with the library's per-launch events: time per launch kind
+        timer = _lib.KernelTimer(16 * ((M + a.chunk - 1) // a.chunk) + 16)
+        flush.fill_(1)
+        end = torch.cuda.Event(enable_timing=True)
+        with timer:
+            fn()
+        end.record()
+        end.synchronize()
+        by_kind = {}
+        for kd, ms_k in zip(timer.kinds, timer.durations_ms(end)):
+            by_kind[kd] = round(by_kind.get(kd, 0.0) + ms_k, 4)
         out = dict(op="lmhead-ce", M=M, d=d, V=V, chunk=a.chunk, avg_ms=round(avg, 4),
                    tokens_per_s=round(M / avg * 1e3), tflops=round(flops / avg / 1e9, 1),
                    workspace_bytes=head.workspace.numel(), full_logits_bytes=2 * M * V,
-                   loss=round(float(head.loss.item()), 5))
+                   loss=round(float(head.loss.item()), 5),
+                   ms_by_launch_kind=by_kind)
     elif a.op == "rmsnorm-cast":
         R = torch.randn(a.rows, a.cols, device="cuda", generator=gen).to(torch.bfloat16)
         w = torch.randn(a.cols, device="cuda", generator=gen).to(torch.bfloat16)

@@ -48,6 +48,28 @@ def test_lmhead_ce_matches_oracle(orc, M, d, V, chunk):
     assert_close_f32(dW.cpu().numpy(), ref_dW, "dW")
 
 
+@pytest.mark.parametrize("softcap", [5.0, 50.0])
+def test_lmhead_ce_softcaps(orc, softcap):
+    """Softcaps up to 40 take the sigmoid-form kernel (hardware exp2 and
+    reciprocal, no running maximum); larger ones the tanhf / expf kernel."""
+    M, d, V, chunk = 192, 256, 2048, 64
+    X, W, labels = inputs(M, d, V, 12)
+    X = X * 4  # larger logits: the softcap saturates for many of them
+    from fp8_gemms_b200 import _lib, api
+    head = api.LmHeadCE(M, d, V, chunk)
+    dW = torch.zeros(V, d, dtype=torch.float32, device="cuda")
+    loss, dX, dW = head(X.cuda(), W.cuda(), labels.cuda(), dW=dW, softcap=softcap)
+    torch.cuda.synchronize()
+    assert _lib.lm_get_error()[0] == 0
+    ref_loss, ref_dX, ref_dW, ref_rows = orc.lmhead_ce(synthetic.bits_u16(X), synthetic.bits_u16(W),
+                                                       labels.numpy(), chunk, softcap=softcap)
+    assert abs(float(loss.item()) - ref_loss) <= 1e-3 * abs(ref_loss)
+    rows = head.row_losses().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(rows - ref_rows) <= 1e-3 * np.abs(ref_rows) + 1e-4)
+    assert_close(u16(dX), ref_dX, f"dX softcap={softcap}")
+    assert_close_f32(dW.cpu().numpy(), ref_dW, f"dW softcap={softcap}")
+
+
 def test_lmhead_ce_accumulates_into_dW(orc):
     M, d, V = 128, 128, 256
     X, W, labels = inputs(M, d, V, 9)
