@@ -7,6 +7,14 @@ iterations).  Also the small, self-contained command to run under ncu.
     python -m fp8_gemms_b200.microbench mlp-compare --M 16384
         (the non-gated relu^2 block, f = 4d, against the gated SwiGLU block,
         f = 2.75d, both fwd + bwd in FP8: ms per step and tokens per second)
+    python -m fp8_gemms_b200.microbench scaled-mm
+        (library calibration: torch._scaled_mm, i.e. cuBLASLt FP8, against this
+        library's GEMM on the six GEMM shapes of the relu^2 MLP step, M = 16384)
+    python -m fp8_gemms_b200.microbench torch-composition --M 16384
+        (the same relu^2 MLP step composed the way the pages' training code
+        composes it -- per-tensor amax and cast in PyTorch, transposed copies,
+        one torch._scaled_mm (cuBLASLt) per GEMM, unfused relu^2 / relu^2' --
+        against this library's two calls, on the same GPU and inputs)
     python -m fp8_gemms_b200.microbench mlp-accum --M 16384 --micro 7
         (one optimizer step of gradient accumulation: the weights are cast by the
         first micro-batch's forward and reused by the others; every backward adds
@@ -49,7 +57,7 @@ def time_it(fn, iters, warmup, flush):
 def main():
     p = argparse.ArgumentParser()
     p.add_argument("op", choices=["gemm", "cast", "mlp-accum", "rmsnorm-cast", "mlp-compare",
-                                  "lmhead-ce"])
+                                  "lmhead-ce", "scaled-mm", "torch-composition"])
     p.add_argument("--V", type=int, default=50304)
     p.add_argument("--chunk", type=int, default=4096)
     p.add_argument("--micro", type=int, default=7)
@@ -78,6 +86,96 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     if a.op == "mlp-accum":
         pass
+    elif a.op == "scaled-mm":
+        # (name, M, N, K, A format, B format, operand storage in the step)
+        shapes = [("up", 16384, 12288, 3072, E4M3, E4M3, 0),
+                  ("down", 16384, 3072, 12288, E4M3, E4M3, 0),
+                  ("dgrad-down", 16384, 12288, 3072, E5M2, E4M3, 2),
+                  ("wgrad-down", 3072, 12288, 16384, E5M2, E4M3, 3),
+                  ("dgrad-up", 16384, 3072, 12288, E5M2, E4M3, 2),
+                  ("wgrad-up", 12288, 3072, 16384, E5M2, E4M3, 3)]
+        ws = torch.empty(_lib.lm_fp8_gemm_workspace_size(), dtype=torch.uint8, device="cuda")
+        one = torch.ones((), device="cuda")
+        res = []
+        for name, M, N, K, fa, fb, flags in shapes:
+            A = random_codes(fa, M, K, gen)          # [M x K]
+            B = random_codes(fb, N, K, gen)          # [N x K]
+            At = A.t().contiguous() if flags & 1 else A
+            Bt = B.t().contiguous() if flags & 2 else B
+            ia = torch.full((1,), 1e-2, device="cuda")
+            D = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+            ours = lambda: _lib.lm_fp8_gemm_ex(At, fa, Bt, fb, ia, ia, D, flags=flags,
+                                               workspace=ws)
+            Af, Bf = A.view(TDT[fa]), B.view(TDT[fb])
+            lib_mm = lambda: torch._scaled_mm(Af, Bf.t(), scale_a=one, scale_b=one,
+                                              out_dtype=torch.bfloat16)
+            t_ours = sum(time_it(ours, a.iters, a.warmup, flush)) / a.iters
+            t_lib = sum(time_it(lib_mm, a.iters, a.warmup, flush)) / a.iters
+            fl = 2 * M * N * K
+            res.append(dict(gemm=name, M=M, N=N, K=K, ours_ms=round(t_ours, 4),
+                            scaled_mm_ms=round(t_lib, 4),
+                            ours_tflops=round(fl / t_ours / 1e9, 1),
+                            scaled_mm_tflops=round(fl / t_lib / 1e9, 1)))
+        tot_o = sum(r["ours_ms"] for r in res)
+        tot_l = sum(r["scaled_mm_ms"] for r in res)
+        out = dict(op="scaled-mm", gemms=res, ours_total_ms=round(tot_o, 4),
+                   scaled_mm_total_ms=round(tot_l, 4),
+                   ours_over_scaled_mm_speed=round(tot_l / tot_o, 4))
+    elif a.op == "torch-composition":
+        from . import api
+        M, d, f = a.M, a.d, a.f
+        bf = torch.bfloat16
+        X = torch.randn(M, d, device="cuda", generator=gen).to(bf)
+        Wu = (torch.randn(f, d, device="cuda", generator=gen) * 0.02).to(bf)
+        Wd = (torch.randn(d, f, device="cuda", generator=gen) * 0.02).to(bf)
+        dY = (torch.randn(M, d, device="cuda", generator=gen) * 1e-3).to(bf)
+        fmax = {torch.float8_e4m3fn: 448.0, torch.float8_e5m2: 57344.0}
+
+        def tcast(x, dt):
+            # amax -> scale -> saturating RNE cast, and the inverse scale
+            amax = x.abs().amax().float().clamp_min(1e-12)
+            sc = fmax[dt] / amax
+            q = (x.float() * sc).clamp(-fmax[dt], fmax[dt]).to(dt)
+            return q, (1.0 / sc).reshape(())
+
+        def mm(aq, ia, bq_nk, ib):
+            # D [M x N] = A [M x K] B[N x K]^T; cuBLASLt wants B column-major
+            return torch._scaled_mm(aq, bq_nk.t(), scale_a=ia, scale_b=ib, out_dtype=bf)
+
+        e4, e5 = torch.float8_e4m3fn, torch.float8_e5m2
+
+        def torch_step():
+            Xq, iX = tcast(X, e4)
+            Wuq, iWu = tcast(Wu, e4)
+            Wdq, iWd = tcast(Wd, e4)
+            H = mm(Xq, iX, Wuq, iWu)
+            h = torch.relu(H).square()
+            hq, ih = tcast(h, e4)
+            Yt = mm(hq, ih, Wdq, iWd)                                # Y
+            dYq, idY = tcast(dY, e5)
+            g = mm(dYq, idY, Wdq.t().contiguous(), iWd)              # dY W_down
+            dH = g * (2 * torch.relu(H))
+            dHq, idH = tcast(dH, e5)
+            dWd = mm(dYq.t().contiguous(), idY, hq.t().contiguous(), ih)   # dY^T h
+            dX = mm(dHq, idH, Wuq.t().contiguous(), iWu)                   # dH W_up
+            dWu = mm(dHq.t().contiguous(), idH, Xq.t().contiguous(), iX)   # dH^T X
+            return Yt, dX, dWu, dWd  # returned, so a compiler cannot drop the work
+
+        mlp = api.Relu2Mlp(M, d, f)
+        Y = torch.empty(M, d, dtype=bf, device="cuda")
+        ours_step = lambda: (mlp.forward(X, Wu, Wd, Y=Y), mlp.backward(dY))
+        t_ref = sum(time_it(torch_step, a.iters, a.warmup, flush)) / a.iters
+        # the same composition under torch.compile, as the pages ran it
+        compiled = torch.compile(torch_step)
+        t_cmp = sum(time_it(compiled, a.iters, a.warmup, flush)) / a.iters
+        t_ours = sum(time_it(ours_step, a.iters, a.warmup, flush)) / a.iters
+        flops = 6 * 2 * M * d * f
+        out = dict(op="torch-composition", M=M, d=d, f=f,
+                   eager_ms=round(t_ref, 4), eager_tflops=round(flops / t_ref / 1e9, 1),
+                   compiled_ms=round(t_cmp, 4), compiled_tflops=round(flops / t_cmp / 1e9, 1),
+                   ours_ms=round(t_ours, 4), ours_tflops=round(flops / t_ours / 1e9, 1),
+                   speedup_vs_eager=round(t_ref / t_ours, 3),
+                   speedup_vs_compiled=round(t_cmp / t_ours, 3))
     elif a.op == "mlp-compare":
         from . import api
         M, d = a.M, a.d
@@ -182,7 +280,8 @@ def main():
         byts = n * ((2 if a.amax_in else 4) + (1 if a.no_qT else 2))
         avg = sum(ms) / len(ms)
         out = dict(op="cast", rows=a.rows, cols=a.cols, fmt=a.fmt, relu2=a.relu2,
-                   amax_in=a.amax_in, qT=not a.no_qT, avg_ms=round(avg, 4), min_ms=round(min(ms), 4),
+                   amax_in=a.amax_in, qT=not a.no_qT, avg_ms=round(avg, 4),
+                   min_ms=round(min(ms), 4),
                    gbs=round(byts / avg / 1e6, 1), algorithmic_bytes=byts)
     if a.op == "mlp-accum":
         from . import api  # noqa: F811
