@@ -1,5 +1,6 @@
 // lm_cast.cu -- dynamic tensorwise FP8 scaling: amax reduction, scale, and
-// the saturating round-to-nearest-even cast with its K-major transposed copy.
+// the saturating round-to-nearest-even cast (row-major codes, and on request
+// the transposed copy).
 //
 // Method: one fp32 scale per tensor per cast, computed from that tensor's
 // current amax (decomputer.nl, "Het trainen van een 3.8B LLM tot 0.384 CORE
@@ -7,9 +8,14 @@
 // tensorwise scaling on all three GEMMs).  e4m3 (max 448) for activations and
 // weights, e5m2 (max 57344) for gradients.
 //
-// Both kernels are HBM-bound: 16-byte vector loads of bf16, codes written
-// with 8-byte (row-major) and 16-byte (transposed) stores; the transpose goes
-// through a 32 KB shared-memory tile and 4x4 byte permutes.
+// The passes are HBM-bound and take up to three tensors per launch:
+//  - amax: 16-byte loads, eight in flight per thread, packed bf16 maxima;
+//  - cast: a persistent TMA-fed kernel (tensor maps per tensor) whose
+//    consumer warps convert 8 bf16 at a time (packed f32x2 scaling, paired
+//    satfinite conversions) and store the row-major codes; the optional
+//    transpose is built in shared memory and stored by TMA;
+//  - a plain per-tile kernel for the row-major codes of tensors whose row
+//    count is not a multiple of 16.
 #include <cuda_bf16.h>
 
 #include "lm_internal.h"

@@ -7,7 +7,10 @@
 // "Niet-gated MLPs": two matmuls instead of three).  All six GEMMs (forward,
 // dgrad and wgrad of both linears) run in FP8 with dynamic tensorwise scaling
 // (same page, section "Vroege experimenten" item 4).  Each tensor is
-// quantised once per call; the backward reuses the forward's codes and scales.
+// quantised once per call, to row-major codes only; the backward reuses the
+// forward's codes and scales, reading them MN-major where a GEMM contracts
+// over their rows.  The workspace's first lm_fp8_gemm_workspace_size() bytes
+// let the GEMMs split an under-filled last wave of tiles.
 #include "lm_internal.h"
 
 namespace {

@@ -1,9 +1,9 @@
 // lm_mlp_noalloc.cu -- the relu^2 MLP backward for callers that cannot
 // allocate device memory.
 //
-// lm_relu2_mlp_bwd needs a caller-provided scratch workspace (the e5m2 codes
-// of dY and dH, the bf16 dH and two scale blocks).  Some
-// callers have no way to provide one: code that runs while a stream is being
+// lm_relu2_mlp_bwd needs a caller-provided scratch workspace (the GEMMs'
+// split-K scratch, the e5m2 codes of dY and dH, the bf16 dH and two scale
+// blocks).  Some callers have no way to provide one: code that runs while a stream is being
 // captured into a CUDA graph (cudaMalloc is not allowed there), plugins whose
 // host framework owns the whole device memory pool and forbids allocation in
 // its execute callback, and latency-critical loops that cannot afford the
