@@ -246,7 +246,7 @@ def run_gpu(args):
     # uploads its inputs from pinned host memory and downloads its results.
     # Three streams (copy-in, compute, copy-out) and two device buffer sets
     # let step k's compute overlap step k+1's upload and step k-1's download.
-    Ke = min(K, 50)  # long enough that the pipeline's fill and drain are a small share
+    Ke = min(K, 100)  # long enough that the pipeline's fill and drain are a small share
     in_names, out_names = ("X", "W_up", "W_down", "dY"), ("Y", "dX", "dW_up", "dW_down")
     pinned_in = {k: host[k].pin_memory() for k in in_names}
     pinned_out = [{k: torch.empty(dev[k].shape, dtype=torch.bfloat16).pin_memory()
