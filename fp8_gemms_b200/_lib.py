@@ -16,6 +16,7 @@ E4M3, E5M2 = 0, 1
 EPI_NONE, EPI_RELU2_FWD, EPI_RELU2_BWD, EPI_ACCUM_F32 = 0, 1, 2, 3
 GEMM_A_MN_MAJOR, GEMM_B_MN_MAJOR = 1, 2
 MLP_REUSE_WEIGHT_CASTS, MLP_ACCUMULATE_WGRAD = 1, 2
+LINEAR_REUSE_WEIGHT_CAST, LINEAR_ACCUMULATE_WGRAD = 1, 2
 
 STATUS = {0: "LM_OK", 1: "LM_ERR_INVALID_ARG", 2: "LM_ERR_ALIGNMENT",
           3: "LM_ERR_UNSUPPORTED_SHAPE", 4: "LM_ERR_UNSUPPORTED_FORMAT", 5: "LM_ERR_CUDA",
@@ -30,7 +31,9 @@ EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
             "lm_rmsnorm_fp8_cast", "lm_swiglu_mlp_saved_bytes", "lm_swiglu_mlp_saved_carve",
             "lm_swiglu_mlp_workspace_size", "lm_swiglu_mlp_fwd", "lm_swiglu_mlp_bwd",
             "lm_fp8_lmhead_ce_workspace_size", "lm_fp8_lmhead_ce", "lm_fp8_gemm_ex",
-            "lm_fp8_gemm_workspace_size"]
+            "lm_fp8_gemm_workspace_size", "lm_fp8_linear_saved_bytes",
+            "lm_fp8_linear_saved_carve", "lm_fp8_linear_workspace_size", "lm_fp8_linear_fwd",
+            "lm_fp8_linear_bwd"]
 
 
 class LmError(RuntimeError):
@@ -43,6 +46,11 @@ class MlpSaved(ctypes.Structure):
     """Mirror of lm_mlp_saved."""
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("Xq", "Wuq", "Wdq", "H", "hq", "scales")]
+
+
+class LinearSaved(ctypes.Structure):
+    """Mirror of lm_linear_saved."""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("Xq", "Wq", "scales")]
 
 
 class SwigluSaved(ctypes.Structure):
@@ -121,6 +129,18 @@ def _load():
     L.lm_fp8_lmhead_ce.restype = st
     L.lm_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
     L.lm_selftest_bounded_wait.restype = st
+    for fn in ("lm_fp8_linear_saved_bytes", "lm_fp8_linear_workspace_size"):
+        getattr(L, fn).argtypes = [i64, i64, i64]
+        getattr(L, fn).restype = ctypes.c_size_t
+    L.lm_fp8_linear_saved_carve.argtypes = [P, ctypes.c_size_t, i64, i64, i64,
+                                            ctypes.POINTER(LinearSaved)]
+    L.lm_fp8_linear_saved_carve.restype = st
+    L.lm_fp8_linear_fwd.argtypes = [P, P, i64, i64, i64, P, ctypes.POINTER(LinearSaved), P,
+                                    ctypes.c_size_t, ctypes.c_uint32, P]
+    L.lm_fp8_linear_fwd.restype = st
+    L.lm_fp8_linear_bwd.argtypes = [P, ctypes.POINTER(LinearSaved), i64, i64, i64, P, P, P,
+                                    ctypes.c_size_t, ctypes.c_uint32, P]
+    L.lm_fp8_linear_bwd.restype = st
     return L
 
 
@@ -259,6 +279,39 @@ def lm_relu2_mlp_bwd_noalloc(dY, saved, dX, dW_up, dW_down, stream=None):
     _check(lib.lm_relu2_mlp_bwd_noalloc(_p(dY), ctypes.byref(saved), M, d, f, _p(dX), _p(dW_up),
                                         _p(dW_down), _stream(stream)),
            "lm_relu2_mlp_bwd_noalloc")
+
+
+def lm_fp8_linear_saved_bytes(M, K, N):
+    return lib.lm_fp8_linear_saved_bytes(M, K, N)
+
+
+def lm_fp8_linear_workspace_size(M, K, N):
+    return lib.lm_fp8_linear_workspace_size(M, K, N)
+
+
+def lm_fp8_linear_saved_carve(buf, M, K, N):
+    s = LinearSaved()
+    _check(lib.lm_fp8_linear_saved_carve(_p(buf), _nbytes(buf), M, K, N, ctypes.byref(s)),
+           "lm_fp8_linear_saved_carve")
+    return s
+
+
+def lm_fp8_linear_fwd(X, W, Y, saved, N, flags=0, workspace=None, stream=None):
+    """X [M x K] -> Y [M x N]; N is given because W may be None when its cast
+    is reused (LINEAR_REUSE_WEIGHT_CAST)."""
+    M, K = X.shape
+    _check(lib.lm_fp8_linear_fwd(_p(X), _p(W), M, K, N, _p(Y), ctypes.byref(saved),
+                                 _p(workspace), _nbytes(workspace), flags, _stream(stream)),
+           "lm_fp8_linear_fwd")
+
+
+def lm_fp8_linear_bwd(dY, saved, K, dX, dW, workspace, flags=0, stream=None):
+    """dY [M x N]; dX [M x K] (or None: no dgrad); dW [N x K] bf16, or fp32
+    with LINEAR_ACCUMULATE_WGRAD."""
+    M, N = dY.shape
+    _check(lib.lm_fp8_linear_bwd(_p(dY), ctypes.byref(saved), M, K, N, _p(dX), _p(dW),
+                                 _p(workspace), _nbytes(workspace), flags, _stream(stream)),
+           "lm_fp8_linear_bwd")
 
 
 def lm_swiglu_mlp_saved_carve(buf, M, d, f):

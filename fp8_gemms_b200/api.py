@@ -10,8 +10,9 @@ import torch
 
 from . import _lib
 from ._lib import (E4M3, E5M2, EPI_ACCUM_F32, EPI_NONE, EPI_RELU2_BWD,  # noqa: F401
-                   EPI_RELU2_FWD, GEMM_A_MN_MAJOR, GEMM_B_MN_MAJOR, MLP_ACCUMULATE_WGRAD,
-                   MLP_REUSE_WEIGHT_CASTS, LmError)
+                   EPI_RELU2_FWD, GEMM_A_MN_MAJOR, GEMM_B_MN_MAJOR, LINEAR_ACCUMULATE_WGRAD,
+                   LINEAR_REUSE_WEIGHT_CAST, MLP_ACCUMULATE_WGRAD, MLP_REUSE_WEIGHT_CASTS,
+                   LmError)
 
 
 def _dev(t):
@@ -229,19 +230,90 @@ class LmHeadCE:
         return self.workspace[-tail:][:n].view(torch.float32)
 
 
+class Linear:
+    """Buffers of one plain FP8 linear Y = X W^T with X [M x K], W [N x K]:
+    the forward's saved codes and scales (one device allocation carved by the
+    library) and the backward's workspace.  forward()/backward() are single
+    C-ABI calls."""
+
+    def __init__(self, M, K, N, device="cuda"):
+        self.M, self.K, self.N = M, K, N
+        nbytes = _lib.lm_fp8_linear_saved_bytes(M, K, N)
+        if nbytes == 0:
+            raise LmError(3, "lm_fp8_linear_saved_bytes")
+        self.saved_buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.saved = _lib.lm_fp8_linear_saved_carve(self.saved_buf, M, K, N)
+        self.workspace = torch.empty(_lib.lm_fp8_linear_workspace_size(M, K, N),
+                                     dtype=torch.uint8, device=device)
+        self.device = device
+
+    def forward(self, X, W, Y=None, stream=None, reuse_weight_cast=False):
+        if Y is None:
+            Y = torch.empty(self.M, self.N, dtype=torch.bfloat16, device=self.device)
+        _lib.lm_fp8_linear_fwd(X, None if reuse_weight_cast else W, Y, self.saved, self.N,
+                               flags=LINEAR_REUSE_WEIGHT_CAST if reuse_weight_cast else 0,
+                               workspace=self.workspace, stream=stream)
+        return Y
+
+    def backward(self, dY, dX=None, dW=None, need_dX=True, stream=None):
+        """Returns (dX, dW); dX is None when need_dX is False (no dgrad)."""
+        dev = self.device
+        if need_dX and dX is None:
+            dX = torch.empty(self.M, self.K, dtype=torch.bfloat16, device=dev)
+        if dW is None:
+            dW = torch.empty(self.N, self.K, dtype=torch.bfloat16, device=dev)
+        _lib.lm_fp8_linear_bwd(dY, self.saved, self.K, dX if need_dX else None, dW,
+                               self.workspace, stream=stream)
+        return (dX if need_dX else None), dW
+
+    def backward_accumulate(self, dY, dW_f32, dX=None, need_dX=True, stream=None):
+        """Backward that adds this call's weight gradient into the fp32
+        accumulator dW_f32 [N x K]; returns dX (None when need_dX is False)."""
+        assert dW_f32.dtype == torch.float32
+        if need_dX and dX is None:
+            dX = torch.empty(self.M, self.K, dtype=torch.bfloat16, device=self.device)
+        _lib.lm_fp8_linear_bwd(dY, self.saved, self.K, dX if need_dX else None, dW_f32,
+                               self.workspace, flags=LINEAR_ACCUMULATE_WGRAD, stream=stream)
+        return dX if need_dX else None
+
+    # views of the saved and scratch buffers (for inspection and stagewise checks)
+    def view(self, name):
+        M, K, N = self.M, self.K, self.N
+        base = self.saved_buf.data_ptr()
+        off = getattr(self.saved, name) - base
+        if name == "scales":
+            return self.saved_buf[off:off + 32].view(torch.float32).view(2, 4)
+        r, c = {"Xq": (M, K), "Wq": (N, K)}[name]
+        return self.saved_buf[off:off + r * c].view(r, c)
+
+    def workspace_view(self, name):
+        """Backward scratch (library layout, each part rounded up to 256
+        bytes): the GEMMs' split-K scratch, dY's codes, dY's scale block."""
+        r256 = lambda n: (n + 255) // 256 * 256
+        off = r256(_lib.lm_fp8_gemm_workspace_size())
+        n = self.M * self.N
+        if name == "dYq":
+            return self.workspace[off:off + n].view(self.M, self.N)
+        if name == "scales":
+            off += r256(n)
+            return self.workspace[off:off + 16].view(torch.float32)
+        raise KeyError(name)
+
+
 def linear_fwd_bwd(X, W, dY, stream=None):
-    """Plain linear Y = X W^T with its dgrad and wgrad, all in FP8: X, W cast
-    to e4m3 and dY to e5m2 (row-major codes only), then Y = Xq Wq^T,
-    dX = dYq W (Wq read MN-major), dW = dY^T X (dYq and Xq read MN-major).
-    Returns (Y, dX, dW, intermediates)."""
-    sc = new_scales(X.device, 3)
-    Xq, _, _ = cast(X, E4M3, want_qT=False, scales=sc[0], stream=stream)
-    Wq, _, _ = cast(W, E4M3, want_qT=False, scales=sc[1], stream=stream)
-    dYq, _, _ = cast(dY, E5M2, want_qT=False, scales=sc[2], stream=stream)
-    ws = gemm_workspace(X.device)
-    Y = gemm(Xq, E4M3, Wq, E4M3, sc[0, 2:3], sc[1, 2:3], workspace=ws, stream=stream)
-    dX = gemm(dYq, E5M2, Wq, E4M3, sc[2, 2:3], sc[1, 2:3], flags=GEMM_B_MN_MAJOR, workspace=ws,
-              stream=stream)
-    dW = gemm(dYq, E5M2, Xq, E4M3, sc[2, 2:3], sc[0, 2:3],
-              flags=GEMM_A_MN_MAJOR | GEMM_B_MN_MAJOR, workspace=ws, stream=stream)
-    return Y, dX, dW, dict(Xq=Xq, Wq=Wq, dYq=dYq, scales=sc)
+    """Plain linear Y = X W^T with its dgrad and wgrad, all in FP8, through
+    lm_fp8_linear_fwd and lm_fp8_linear_bwd: X, W cast to e4m3 and dY to e5m2
+    (row-major codes only), then Y = Xq Wq^T, dX = dYq W (Wq read MN-major),
+    dW = dY^T X (dYq and Xq read MN-major).
+    Returns (Y, dX, dW, intermediates): the codes Xq, Wq, dYq and a [3 x 4]
+    host array of the {amax, scale, inv_scale, 0} blocks of X, W and dY."""
+    M, K = X.shape
+    N = W.shape[0]
+    lin = Linear(M, K, N, device=X.device)
+    Y = lin.forward(X, W, stream=stream)
+    dX, dW = lin.backward(dY, stream=stream)
+    if stream is not None:
+        stream.synchronize()
+    sc = torch.cat([lin.view("scales"), lin.workspace_view("scales").view(1, 4)]).cpu().numpy()
+    return Y, dX, dW, dict(Xq=lin.view("Xq"), Wq=lin.view("Wq"), dYq=lin.workspace_view("dYq"),
+                           scales=sc)

@@ -15,6 +15,14 @@ iterations).  Also the small, self-contained command to run under ncu.
         composes it -- per-tensor amax and cast in PyTorch, transposed copies,
         one torch._scaled_mm (cuBLASLt) per GEMM, unfused relu^2 / relu^2' --
         against this library's two calls, on the same GPU and inputs)
+    python -m fp8_gemms_b200.microbench linears --workload attn-head
+        (the attention projections Q, K, V, O and the LM head at M = 8192, each
+        fwd + dgrad + wgrad through lm_fp8_linear_fwd / _bwd: per linear, and
+        the whole set eagerly and replayed from a CUDA graph)
+    python -m fp8_gemms_b200.microbench linears --workload stack
+        (the per-step linear GEMM set of a 28-layer d = 3072 stack at M = 16384:
+        per layer Q, K, V, O and the relu^2 MLP, fwd + dgrad + wgrad, each
+        layer with its own weights and t3-distributed activations)
     python -m fp8_gemms_b200.microbench mlp-accum --M 16384 --micro 7
         (one optimizer step of gradient accumulation: the weights are cast by the
         first micro-batch's forward and reused by the others; every backward adds
@@ -54,10 +62,106 @@ def time_it(fn, iters, warmup, flush):
     return ms
 
 
+def _draw(shape, dist, gen):
+    """Seeded device draw: N(0, sigma) or Student-t with 3 degrees of freedom
+    (Z / sqrt(chi2_3 / 3)), rounded to bf16."""
+    if dist == "t3":
+        z = torch.randn(*shape, device="cuda", generator=gen)
+        chi = torch.zeros_like(z)
+        for _ in range(3):
+            n = torch.randn(*shape, device="cuda", generator=gen)
+            chi.addcmul_(n, n)
+        return (z / torch.sqrt(chi / 3.0)).to(torch.bfloat16)
+    return (torch.randn(*shape, device="cuda", generator=gen) * dist).to(torch.bfloat16)
+
+
+def linears(a, gen, flush):
+    from . import api, synthetic
+    if a.workload == "attn-head":
+        M, layers, x_dist = 8192, 1, 1.0
+        shapes = synthetic.ATTN_LINEARS + [("lm_head", synthetic.VOCAB_PADDED,
+                                            synthetic.D_MODEL)]
+        mlp_dims = None
+    else:
+        M, layers, x_dist = 16384, a.layers, "t3"
+        shapes = synthetic.ATTN_LINEARS
+        mlp_dims = (synthetic.D_MODEL, synthetic.D_FF)
+    lins = {(n, k): api.Linear(M, k, n) for _, n, k in shapes}
+    outs = {(n, k): (torch.empty(M, n, dtype=torch.bfloat16, device="cuda"),
+                     torch.empty(M, k, dtype=torch.bfloat16, device="cuda"),
+                     torch.empty(n, k, dtype=torch.bfloat16, device="cuda"))
+            for _, n, k in shapes}
+    data = []   # per layer: [(name, n, k, X, W, dY)], and the MLP's tensors
+    for _ in range(layers):
+        lay = [(name, n, k, _draw((M, k), x_dist, gen), _draw((n, k), 0.02, gen),
+                _draw((M, n), 1e-3, gen)) for name, n, k in shapes]
+        mt = None
+        if mlp_dims:
+            d, f = mlp_dims
+            mt = (_draw((M, d), x_dist, gen), _draw((f, d), 0.02, gen),
+                  _draw((d, f), 0.02, gen), _draw((M, d), 1e-3, gen))
+        data.append((lay, mt))
+    mlp = api.Relu2Mlp(M, *mlp_dims) if mlp_dims else None
+    if mlp:
+        d, f = mlp_dims
+        mY = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+        mdX = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+        mdWu = torch.empty(f, d, dtype=torch.bfloat16, device="cuda")
+        mdWd = torch.empty(d, f, dtype=torch.bfloat16, device="cuda")
+
+    def run_linear(name, n, k, X, W, dY):
+        lin, (Y, dX, dW) = lins[(n, k)], outs[(n, k)]
+        lin.forward(X, W, Y=Y)
+        lin.backward(dY, dX=dX, dW=dW)
+
+    def step():
+        for lay, mt in data:
+            for item in lay:
+                run_linear(*item)
+            if mt:
+                mlp.forward(mt[0], mt[1], mt[2], Y=mY)
+                mlp.backward(mt[3], dX=mdX, dW_up=mdWu, dW_down=mdWd)
+
+    flops_lin = {name: 6 * M * n * k for name, n, k in shapes}
+    flops = layers * (sum(flops_lin.values()) +
+                      (12 * M * mlp_dims[0] * mlp_dims[1] if mlp_dims else 0))
+    res = dict(op="linears", workload=a.workload, M=M, layers=layers,
+               tflop_per_step=round(flops / 1e12, 4))
+    per = []
+    for item in data[0][0]:
+        ms = time_it(lambda: run_linear(*item), a.iters, a.warmup, flush)
+        t = sum(ms) / len(ms)
+        per.append(dict(linear=item[0], N=item[1], K=item[2], ms=round(t, 4),
+                        tflops=round(flops_lin[item[0]] / t / 1e9, 1)))
+    res["per_linear_layer0"] = per
+    iters = max(2, a.iters // (4 if layers > 1 else 1))
+    ms = time_it(step, iters, a.warmup, flush)
+    t = sum(ms) / len(ms)
+    res.update(eager_ms=round(t, 4), eager_tflops=round(flops / t / 1e9, 1))
+    if layers == 1:
+        # replayed from a CUDA graph: no host launch overhead between the kernels
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                step()
+        torch.cuda.current_stream().wait_stream(s)
+        ms = time_it(g.replay, a.iters, a.warmup, flush)
+        t = sum(ms) / len(ms)
+        res.update(graph_ms=round(t, 4), graph_tflops=round(flops / t / 1e9, 1))
+        del g
+    res["pct_of_4500_tflops"] = round(100 * flops / (min(
+        res.get("graph_ms", 1e30), res["eager_ms"]) * 1e9) / 4500.0, 1)
+    return res
+
+
 def main():
     p = argparse.ArgumentParser()
     p.add_argument("op", choices=["gemm", "cast", "mlp-accum", "rmsnorm-cast", "mlp-compare",
-                                  "lmhead-ce", "scaled-mm", "torch-composition"])
+                                  "lmhead-ce", "scaled-mm", "torch-composition", "linears"])
+    p.add_argument("--workload", default="attn-head", choices=["attn-head", "stack"])
+    p.add_argument("--layers", type=int, default=28)
     p.add_argument("--V", type=int, default=50304)
     p.add_argument("--chunk", type=int, default=4096)
     p.add_argument("--micro", type=int, default=7)
@@ -86,6 +190,8 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     if a.op == "mlp-accum":
         pass
+    elif a.op == "linears":
+        out = linears(a, gen, flush)
     elif a.op == "scaled-mm":
         # (name, M, N, K, A format, B format, operand storage in the step)
         shapes = [("up", 16384, 12288, 3072, E4M3, E4M3, 0),

@@ -301,6 +301,59 @@ LM_API lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* saved, 
                                      lm_stream_t stream);
 
 /*
+ * Plain FP8 linear layer, Y = X W^T, with its dgrad and wgrad (the attention
+ * projections and the LM head of the model; decomputer.nl, "Het trainen van
+ * een 3.8B LLM tot 0.384 CORE voor $998", section "Vroege experimenten" item
+ * 4: all three GEMMs of a linear in FP8 with dynamic tensorwise scaling):
+ *   forward:  cast X, W to e4m3 (one amax launch, one cast launch);  Y = Xq Wq^T
+ *   backward: cast dY to e5m2;  dX = dYq Wq;  dW = dYq^T Xq   (K of the wgrad = M)
+ * Only row-major codes are made; the dgrad reads Wq and the wgrad reads dYq
+ * and Xq MN-major (lm_fp8_gemm_ex), so no transposed copy is written.
+ * X: bf16 [M x K]; W: bf16 [N x K]; Y, dY: bf16 [M x N]; dX: bf16 [M x K];
+ * dW: bf16 [N x K], or an fp32 accumulator with LM_LINEAR_ACCUMULATE_WGRAD.
+ * Requirements: M, K, N multiples of 16 (M may be 0).
+ */
+typedef struct lm_linear_saved {
+    uint8_t* Xq;   /* [M x K] e4m3 codes of X; the wgrad reads them MN-major */
+    uint8_t* Wq;   /* [N x K] e4m3 codes of W; the dgrad reads them MN-major */
+    float* scales; /* 8 device floats: {amax, scale, inv_scale, unused} for X, then W */
+} lm_linear_saved;
+
+#define LM_LINEAR_REUSE_WEIGHT_CAST 1u /* fwd: W's codes and scale block in `saved` are
+                                          current; W's cast is skipped (W may be NULL) */
+#define LM_LINEAR_ACCUMULATE_WGRAD 2u  /* bwd: dW is an fp32 [N x K] accumulator; this
+                                          call's weight gradient is added to it */
+
+/* Bytes of every buffer of lm_linear_saved (each 256-byte aligned); 0 for an
+ * unsupported shape. */
+LM_API size_t lm_fp8_linear_saved_bytes(int64_t M, int64_t K, int64_t N);
+
+/* Host-only pointer arithmetic: carve a caller-allocated, 256-byte-aligned
+ * device buffer `base` of `bytes` (>= lm_fp8_linear_saved_bytes) into `out`. */
+LM_API lm_status lm_fp8_linear_saved_carve(void* base, size_t bytes, int64_t M, int64_t K,
+                                           int64_t N, lm_linear_saved* out);
+
+/* Bytes of scratch lm_fp8_linear_bwd needs: the GEMMs' split-K scratch
+ * (lm_fp8_gemm_workspace_size bytes, all the forward uses of it), then dY's
+ * codes and scale block; 0 for an unsupported shape. */
+LM_API size_t lm_fp8_linear_workspace_size(int64_t M, int64_t K, int64_t N);
+
+/* Forward.  workspace: NULL (ws_bytes 0) or 256-byte-aligned scratch of at least
+ * lm_fp8_gemm_workspace_size() bytes, which lets the GEMM split an under-filled
+ * last wave.  flags: 0 or LM_LINEAR_REUSE_WEIGHT_CAST; other bits return
+ * LM_ERR_INVALID_ARG. */
+LM_API lm_status lm_fp8_linear_fwd(const void* X, const void* W, int64_t M, int64_t K,
+                                   int64_t N, void* Y, lm_linear_saved* saved, void* workspace,
+                                   size_t ws_bytes, uint32_t flags, lm_stream_t stream);
+
+/* Backward from the forward's saved codes.  dX may be NULL (no dgrad, e.g. for a
+ * layer whose input needs no gradient).  workspace: >= lm_fp8_linear_workspace_size
+ * bytes, 256-byte aligned.  flags: 0 or LM_LINEAR_ACCUMULATE_WGRAD. */
+LM_API lm_status lm_fp8_linear_bwd(const void* dY, const lm_linear_saved* saved, int64_t M,
+                                   int64_t K, int64_t N, void* dX, void* dW, void* workspace,
+                                   size_t ws_bytes, uint32_t flags, lm_stream_t stream);
+
+/*
  * Gated (SwiGLU) MLP, the comparison workload of the non-gated relu^2 MLP
  * (decomputer.nl, "Het trainen van een 3.8B LLM tot 0.384 CORE voor $998",
  * section "Doorvoer (Throughput) verhogen", bullet "Niet-gated MLPs": three

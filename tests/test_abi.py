@@ -144,3 +144,34 @@ def test_newer_entry_points_reject_before_launch(L):
     # no-alloc backward: shape beyond its array
     assert lib.lm_relu2_mlp_bwd_noalloc(None, C.byref(s), 16384, 3072, 12288, None, None, None,
                                         None) == 3
+
+
+def test_linear_sizes_carve_and_checks(L):
+    import ctypes as C
+    M, K, N = 256, 192, 320
+    r = lambda n: (n + 255) // 256 * 256
+    # saved: X codes, W codes, two scale blocks; scratch: split-K region, dY codes, one block
+    assert L.lm_fp8_linear_saved_bytes(M, K, N) == r(M * K) + r(N * K) + r(32)
+    split = L.lib.lm_fp8_gemm_workspace_size()
+    assert L.lm_fp8_linear_workspace_size(M, K, N) == r(split) + r(M * N) + r(16)
+    assert L.lm_fp8_linear_saved_bytes(M, K, 200) == 0      # N not a multiple of 16
+    assert L.lm_fp8_linear_workspace_size(24, K, N) == 0    # M not a multiple of 16
+    assert L.lm_fp8_linear_saved_bytes(0, K, N) == r(N * K) + r(32)
+    s = L.LinearSaved()
+    base, n = 0x100000, L.lm_fp8_linear_saved_bytes(M, K, N)
+    assert L.lib.lm_fp8_linear_saved_carve(base, n, M, K, N, C.byref(s)) == 0
+    assert s.Xq == base and s.Wq == base + r(M * K) and s.scales == base + n - r(32)
+    assert L.lib.lm_fp8_linear_saved_carve(base, n - 1, M, K, N, C.byref(s)) == 1
+    assert L.lib.lm_fp8_linear_saved_carve(base + 16, n, M, K, N, C.byref(s)) == 2
+    fake = 0x10000
+    fwd, bwd = L.lib.lm_fp8_linear_fwd, L.lib.lm_fp8_linear_bwd
+    ws = L.lm_fp8_linear_workspace_size(M, K, N)
+    assert fwd(fake, fake, M, K, 200, fake, C.byref(s), None, 0, 0, None) == 3
+    assert fwd(fake, fake, M, K, N, fake, C.byref(s), None, 0, 4, None) == 1    # unknown flag
+    assert fwd(fake, fake, M, K, N, fake, C.byref(s), fake + 16, ws, 0, None) == 2
+    assert fwd(fake, None, M, K, N, fake, C.byref(s), None, 0, 0, None) == 1    # W needed
+    assert fwd(None, fake, M, K, N, fake, C.byref(s), None, 0, 0, None) == 1
+    assert bwd(fake, C.byref(s), M, K, N, fake, fake, fake, ws - 1, 0, None) == 1
+    assert bwd(fake, C.byref(s), M, K, N, fake, fake, fake + 16, ws, 0, None) == 2
+    assert bwd(fake, C.byref(s), M, K, N, fake, fake, fake, ws, 1, None) == 1   # fwd's flag
+    assert bwd(fake, C.byref(s), M, K, N, fake, None, fake, ws, 0, None) == 1   # dW needed

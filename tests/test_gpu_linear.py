@@ -1,7 +1,8 @@
-"""GPU parity of the plain FP8 linear (forward, dgrad, wgrad) at the
-attention-projection and LM-head shapes: X [M x K] and W [N x K] cast to e4m3,
-dY [M x N] to e5m2 (each with its K-major transposed copy), then
-Y = Xq Wq^T, dX = dYq (Wq^T)^T, dW = (dYq^T)(Xq^T)^T, all through the C ABI.
+"""GPU parity of the plain FP8 linear (lm_fp8_linear_fwd / lm_fp8_linear_bwd:
+forward, dgrad, wgrad) at the attention-projection and LM-head shapes: X [M x K]
+and W [N x K] cast to e4m3, dY [M x N] to e5m2 (row-major codes only), then
+Y = Xq Wq^T, dX = dYq Wq, dW = dYq^T Xq, the last two reading the codes
+MN-major.
 
 Casts are checked bit-exact over whole tensors; GEMM outputs elementwise
 within the stated tolerance, on all rows for small M and on sampled rows at
@@ -11,7 +12,7 @@ import pytest
 import torch
 
 from fp8_gemms_b200 import synthetic
-from gpu_util import assert_close, f32, u8, u16
+from gpu_util import assert_close, assert_close_f32, f32, u8, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +31,7 @@ def check_linear(orc, api, X, W, dY, rows=None, wrows=None):
     torch.cuda.synchronize()
     from fp8_gemms_b200 import _lib
     assert _lib.lm_get_error()[0] == 0
-    sc = q["scales"].cpu().numpy()
+    sc = q["scales"]
     for i, (t, fmt, key) in enumerate([(X, E4M3, "Xq"), (W, E4M3, "Wq"), (dY, E5M2, "dYq")]):
         ref = orc.amax_scale_cast(synthetic.bits_u16(t), fmt)
         assert sc[i, 0] == ref["amax"] and sc[i, 1] == ref["scale"] and sc[i, 2] == ref["inv_scale"]
@@ -56,6 +57,90 @@ def test_linear_shapes_small_batch(orc, api, name, n_out, n_in):
     w = synthetic.LinearWorkload("small", 512, [(name, n_out, n_in)])
     t = w.tensors(0)
     check_linear(orc, api, t["X"], t["W"], t["dY"])
+
+
+def test_linear_ragged_shape(orc, api):
+    """Every dimension off the 256-wide tile: M = 272, K = 208, N = 336."""
+    w = synthetic.LinearWorkload("ragged", 272, [("r", 336, 208)])
+    t = w.tensors(0)
+    check_linear(orc, api, t["X"], t["W"], t["dY"])
+
+
+def _lin_inputs(M, K, N, seed=0):
+    t = synthetic.LinearWorkload("lin", M, [("l", N, K)], seed=seed).tensors(0)
+    return t["X"].cuda(), t["W"].cuda(), t["dY"].cuda()
+
+
+def test_linear_reused_weight_cast_and_skipped_dgrad(api):
+    """The forward with LM_LINEAR_REUSE_WEIGHT_CAST uses W's codes and scale
+    from the previous forward (they equal a fresh cast's); the backward with
+    dX = NULL computes the same dW and leaves the dgrad out."""
+    from fp8_gemms_b200 import _lib
+    M, K, N = 512, 256, 384
+    X, W, dY = _lin_inputs(M, K, N, seed=5)
+    lin = api.Linear(M, K, N)
+    lin.forward(X, W)
+    w_scale, w_codes = lin.view("scales")[1].clone(), lin.view("Wq").clone()
+    X2 = torch.roll(X, 7, dims=0).contiguous()
+    Y2 = lin.forward(X2, None, reuse_weight_cast=True)
+    fresh = api.Linear(M, K, N)
+    Y3 = fresh.forward(X2, W)
+    torch.cuda.synchronize()
+    assert _lib.lm_get_error()[0] == 0
+    assert torch.equal(Y2.view(torch.int16), Y3.view(torch.int16))
+    assert torch.equal(lin.view("scales")[1], w_scale) and torch.equal(lin.view("Wq"), w_codes)
+    assert torch.equal(lin.view("scales"), fresh.view("scales"))
+    dX, dW = lin.backward(dY)
+    dX_none, dW2 = lin.backward(dY, need_dX=False)
+    torch.cuda.synchronize()
+    assert dX_none is None and dX is not None
+    assert torch.equal(dW.view(torch.int16), dW2.view(torch.int16))
+
+
+def test_linear_accumulating_wgrad(orc, api):
+    """LM_LINEAR_ACCUMULATE_WGRAD over two calls: dW (fp32) += dYq^T Xq s each
+    time, against the oracle's fp32-accumulating GEMM on the saved codes."""
+    M, K, N = 384, 256, 320
+    D0 = np.random.default_rng(6).standard_normal((N, K)).astype(np.float32) * 1e-3
+    dW = torch.from_numpy(D0.copy()).cuda()
+    ref = D0.copy()
+    lin = api.Linear(M, K, N)
+    for seed in (7, 8):
+        X, W, dY = _lin_inputs(M, K, N, seed=seed)
+        lin.forward(X, W)
+        dX = lin.backward_accumulate(dY, dW)
+        torch.cuda.synchronize()
+        sx = lin.view("scales").cpu().numpy()
+        sg = lin.workspace_view("scales").cpu().numpy()
+        Xq, dYq = u8(lin.view("Xq")), u8(lin.workspace_view("dYq"))
+        orc.gemm_accum_f32(np.ascontiguousarray(dYq.T), E5M2, np.ascontiguousarray(Xq.T), E4M3,
+                           sg[2], sx[0, 2], ref)
+        ref_dX, _ = orc.gemm(dYq, E5M2, np.ascontiguousarray(u8(lin.view("Wq")).T), E4M3,
+                             sg[2], sx[1, 2])
+        assert_close(u16(dX), ref_dX, "dX")
+    from fp8_gemms_b200 import _lib
+    assert _lib.lm_get_error()[0] == 0
+    assert_close_f32(dW.cpu().numpy(), ref, "accumulated dW")
+
+
+def test_linear_empty_batch(orc, api):
+    """M = 0: nothing to multiply; W is still cast (its scale block is exact),
+    Y and dX are empty and dW is zero."""
+    K, N = 256, 128
+    _, W, _ = _lin_inputs(16, K, N, seed=9)
+    lin = api.Linear(0, K, N)
+    X = torch.empty(0, K, dtype=torch.bfloat16, device="cuda")
+    Y = lin.forward(X, W)
+    dX, dW = lin.backward(torch.empty(0, N, dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    from fp8_gemms_b200 import _lib
+    assert _lib.lm_get_error()[0] == 0
+    assert Y.shape == (0, N) and dX.shape == (0, K)
+    assert not bool(dW.view(torch.int16).any())
+    ref = orc.amax_scale_cast(synthetic.bits_u16(W.cpu()), E4M3)
+    sc = lin.view("scales").cpu().numpy()
+    assert sc[1, 0] == ref["amax"] and sc[1, 1] == ref["scale"] and sc[1, 2] == ref["inv_scale"]
+    assert np.array_equal(u8(lin.view("Wq")), ref["q"])
 
 
 def test_linear_student_t_activations(orc, api):
