@@ -33,7 +33,7 @@ EXPORTED = ["lm_fp8_amax_scale_cast", "lm_fp8_gemm", "lm_relu2_mlp_saved_bytes",
             "lm_fp8_lmhead_ce_workspace_size", "lm_fp8_lmhead_ce", "lm_fp8_gemm_ex",
             "lm_fp8_gemm_workspace_size", "lm_fp8_linear_saved_bytes",
             "lm_fp8_linear_saved_carve", "lm_fp8_linear_workspace_size", "lm_fp8_linear_fwd",
-            "lm_fp8_linear_bwd"]
+            "lm_fp8_linear_bwd", "lm_fp8_gemm_split_plan"]
 
 
 class LmError(RuntimeError):
@@ -129,6 +129,9 @@ def _load():
     L.lm_fp8_lmhead_ce.restype = st
     L.lm_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
     L.lm_selftest_bounded_wait.restype = st
+    L.lm_fp8_gemm_split_plan.argtypes = [i64, i64, i64, i32, ctypes.POINTER(ctypes.c_int),
+                                         ctypes.POINTER(ctypes.c_int)]
+    L.lm_fp8_gemm_split_plan.restype = st
     for fn in ("lm_fp8_linear_saved_bytes", "lm_fp8_linear_workspace_size"):
         getattr(L, fn).argtypes = [i64, i64, i64]
         getattr(L, fn).restype = ctypes.c_size_t
@@ -195,6 +198,15 @@ def _nbytes(t):
 
 def lm_fp8_gemm_workspace_size():
     return lib.lm_fp8_gemm_workspace_size()
+
+
+def lm_fp8_gemm_split_plan(M, N, K, sm_count):
+    """(parts, tail_tiles): the split-K tail lm_fp8_gemm_ex uses for this shape
+    on a GPU of sm_count multiprocessors (host arithmetic only)."""
+    parts, tail = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib.lm_fp8_gemm_split_plan(M, N, K, sm_count, ctypes.byref(parts), ctypes.byref(tail)),
+           "lm_fp8_gemm_split_plan")
+    return parts.value, tail.value
 
 
 def lm_fp8_gemm_ex(A, fa, B, fb, inv_scale_a, inv_scale_b, D, flags=0, epi=EPI_NONE, aux=None,

@@ -44,28 +44,37 @@ enum : unsigned {
 
 // Split-K tail.  Tiles go round-robin to the persistent clusters, so a last
 // wave of r < clusters tiles leaves the other clusters idle for a whole tile.
-// When 2r <= clusters, each of those r tiles is computed as two units over
-// the two halves of K, in the same round on two clusters: half 0 writes its
-// fp32 partial sums to a workspace and raises a flag per (CTA, warp); half 1
-// waits for the flag (bounded), copies the partial into its operand ring,
-// which is idle at that point (a split unit is always its cluster's last),
-// and adds it to its own sums before the epilogue.  Partial layout per
-// (tile, CTA rank, TMEM lane quarter): [chunk 8][float4 8][lane 32], so
-// both the writes and the reads are contiguous across a warp.
+// Each of those r tiles can instead run as S units over S consecutive ranges
+// of K.  A round of C clusters holds P = C / S such tiles, whose S parts sit
+// on consecutive clusters of that round (the rest of the round's clusters get
+// no unit).  Parts 0..S-2 write their fp32 partial sums to a workspace slot and
+// raise a flag per (CTA, warp); part S-1, on the highest of the tile's
+// clusters, waits for those flags (bounded) and adds the partials to its own
+// sums before the epilogue.  With S = 2 in the grid's last round the partial
+// is bulk-copied into the operand ring, idle there (the unit is its cluster's
+// last); otherwise it is read from global memory.  Partial layout per (tile,
+// part, CTA rank, TMEM lane quarter): [chunk 8][float4 8][lane 32], so both
+// the writes and the reads are contiguous across a warp.
 constexpr size_t kSplitSlotFloat4 = 8 * 8 * 32;                   // one warp's partial
 constexpr size_t kSplitTileBytes = 2 * NUM_EPI_WARPS * kSplitSlotFloat4 * 16;  // 256 KB
-constexpr int kSplitMaxTiles = 64;
+constexpr int kSplitMaxSlots = 128;  // partial tiles the workspace holds
+constexpr int kSplitMaxParts = 8;
 
 struct WorkUnit {
-    int tile, kb0, kb1;
-    int half;  // -1: a whole tile; 0 / 1: first / second half of a split tile
+    int tile;  // -1: no work (a cluster left idle in a round of split tiles)
+    int kb0, kb1;
+    int part;  // -1: a whole tile; else part 0..S-1 of a split tile (S-1 finishes it)
 };
 
 struct GemmArgs {
     int M, N, num_mb, num_nb, num_kb, num_tiles, group_m;
-    int num_units, split_first;  // units: tiles [0, split_first), then split halves
+    int num_units, split_first;  // units: tiles [0, split_first), then rounds of split parts
+    int split_parts;             // S (>= 2 when some tiles are split)
+    int split_round;             // units per round (C, the clusters of a full grid)
+    int split_per_round;         // P = C / S split tiles per round
+    int split_slots;             // partial tiles in the workspace: split tiles x (S - 1)
     float4* split_ws;            // partial sums of the split tiles
-    unsigned int* split_flags;   // [split tile][rank][quarter], zeroed before the launch
+    unsigned int* split_flags;   // [slot][rank][quarter], zeroed before the launch
     int a_mn, b_mn;  // 1: the operand is stored MN-major ([K x M] / [K x N], M or N contiguous)
     int stream_a;  // 1: A is the streamed operand (evict-first loads), 0: B is
     const float* inv_a;
@@ -78,10 +87,23 @@ struct GemmArgs {
     uint32_t idesc;
 };
 
+// MULTI = false: no split, or halves in one round (units split_first + 2t and
+// split_first + 2t + 1 are the halves of tile split_first + t).  MULTI = true:
+// S parts, P tiles per round of split_round units.
+template <bool MULTI>
 __device__ __forceinline__ WorkUnit work_unit(int u, const GemmArgs& a) {
     if (u < a.split_first) return {u, 0, a.num_kb, -1};
-    const int s = u - a.split_first, h = s & 1, kh = a.num_kb >> 1;
-    return {a.split_first + (s >> 1), h ? kh : 0, h ? a.num_kb : kh, h};
+    if constexpr (!MULTI) {
+        const int s = u - a.split_first, h = s & 1, kh = a.num_kb >> 1;
+        return {a.split_first + (s >> 1), h ? kh : 0, h ? a.num_kb : kh, h};
+    } else {
+        const int s = u - a.split_first, S = a.split_parts;
+        const int round = s / a.split_round, pos = s - round * a.split_round;
+        const int t = pos / S, part = pos - t * S;
+        const int tile = a.split_first + round * a.split_per_round + t;
+        if (t >= a.split_per_round || tile >= a.num_tiles) return {-1, 0, 0, -1};
+        return {tile, part * a.num_kb / S, (part + 1) * a.num_kb / S, part};
+    }
 }
 
 // Tile visiting order: groups of group_m row-blocks, column-blocks within a
@@ -218,7 +240,11 @@ __device__ __forceinline__ uint32_t sw64(int r, int j) {
     return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
 }
 
-template <int EPI>
+// MULTI: the instantiation launched when the split tail has three or more
+// parts (the last part reads the others' sums from global memory).  The
+// instantiations for no split or halves leave that code out, which keeps the
+// epilogue loop of the common case as lean as it was measured.
+template <int EPI, bool MULTI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_fp8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB,
@@ -290,7 +316,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             uint32_t phase = 0, issued = 0;
             bool ok = true;
             for (int u = cluster; u < args.num_units && ok; u += nclusters) {
-                const WorkUnit w = work_unit(u, args);
+                const WorkUnit w = work_unit<MULTI>(u, args);
+                if (MULTI && w.tile < 0) continue;
                 int mb, nb;
                 tile_coords(w.tile, args.group_m, args.num_mb, args.num_nb, mb, nb);
                 const int arow = mb * TILE_M + (int)rank * 128;
@@ -342,7 +369,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const uint64_t a_step = args.a_mn ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
             const uint64_t b_step = args.b_mn ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
             for (int u = cluster; u < args.num_units && ok; u += nclusters) {
-                const WorkUnit w = work_unit(u, args);
+                const WorkUnit w = work_unit<MULTI>(u, args);
+                if (MULTI && w.tile < 0) continue;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.err, W_TEMPTY)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TILE_N);
@@ -389,7 +417,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         uint32_t n_stores = 0;
         bool ok = true;
         for (int u = cluster; u < args.num_units && ok; u += nclusters) {
-            const WorkUnit w = work_unit(u, args);
+            const WorkUnit w = work_unit<MULTI>(u, args);
+            if (MULTI && w.tile < 0) continue;
             int mb, nb;
             tile_coords(w.tile, args.group_m, args.num_mb, args.num_nb, mb, nb);
             const int grow = mb * TILE_M + (int)rank * 128 + quarter * 32;  // row of lane 0
@@ -397,11 +426,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int left = args.N - gcol;
             const int n_chunks =
                 left >= TILE_N ? TILE_N / EPI_COLS : (left + EPI_COLS - 1) / EPI_COLS;
-            // this warp's slot of a split tile's partial sums and flags
-            const size_t slot = w.half < 0 ? 0
-                                           : ((size_t)(w.tile - args.split_first) * 2 + rank) *
-                                                     NUM_EPI_WARPS + quarter;
-            if (EPI == LM_EPI_RELU2_BWD && lane == 0 && w.half != 0) {
+            // this warp's slot of a split tile's partial sums and flags: part p
+            // of the tile (p < S-1) writes slot_of(p); the last part reads them
+            const int S = MULTI ? args.split_parts : 2;
+            const bool finishes = w.part < 0 || w.part == S - 1;
+            auto slot_of = [&](int p) {
+                return (((size_t)(w.tile - args.split_first) * (size_t)(S - 1) + (size_t)p) * 2 +
+                        rank) * NUM_EPI_WARPS + quarter;
+            };
+            if (EPI == LM_EPI_RELU2_BWD && lane == 0 && finishes) {
                 // the first H box of this tile (no L2 prefetch of the next
                 // tile's H: measured, it raised DRAM reads by a third and cost
                 // 3.6% of this GEMM's time)
@@ -413,9 +446,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const uint32_t tbase =
                 tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * TILE_N);
-            if (w.half == 0) {
-                // first half of a split tile: publish the raw fp32 sums
-                float4* dst = args.split_ws + slot * kSplitSlotFloat4;
+            if (!finishes) {
+                // an earlier part of a split tile: publish the raw fp32 sums
+                float4* dst = args.split_ws + slot_of(w.part) * kSplitSlotFloat4;
                 for (int c = 0; c < n_chunks; ++c) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(tbase + (uint32_t)(c * EPI_COLS), r);
@@ -428,7 +461,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
                 __threadfence();
                 __syncwarp();
-                if (lane == 0) st_release_gpu(args.split_flags + slot, 1u);
+                if (lane == 0) st_release_gpu(args.split_flags + slot_of(w.part), 1u);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_remote(tempty_leader + (uint32_t)(acc * 8));
@@ -436,26 +469,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 if (acc == 0) acc_phase ^= 1u;
                 continue;
             }
-            // second half of a split tile: the first half's sums, copied into
-            // this warp's 32 KB of the operand ring (idle: this is the last unit)
-            const float4* part = nullptr;
-            if (w.half == 1) {
+            // the last part of a split tile: the other parts' sums.  With two
+            // parts in the grid's last round, the first part's sums are copied
+            // into this warp's 32 KB of the operand ring (idle: no unit follows
+            // on this cluster); otherwise they are read from global memory.
+            const float4* part = nullptr;   // in shared memory
+            const float4* gpart = nullptr;  // in global memory, slot_of(0) .. slot_of(S-2)
+            if (w.part > 0 && finishes) {
                 bool ready = true;
-                if (lane == 0) ready = flag_wait(args.split_flags + slot, 1u, args.err, W_SPLIT);
+                if (lane == 0)
+                    for (int p = 0; p < S - 1 && ready; ++p)
+                        ready = flag_wait(args.split_flags + slot_of(p), 1u, args.err, W_SPLIT);
                 ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
-                if (ready) {
+                if (ready && (!MULTI || (S == 2 && u + nclusters >= args.num_units))) {
                     uint8_t* buf = smem + wi * (int)(kSplitSlotFloat4 * 16);
                     if (lane == 0) {
                         const uint32_t bytes = (uint32_t)n_chunks * 8 * 32 * 16;
                         fence_proxy_async_global();  // the acquired sums, then the bulk read
                         mbar_arrive_expect_tx(&splitbar[wi], bytes);
-                        bulk_load_1d(smem_addr(buf), args.split_ws + slot * kSplitSlotFloat4, bytes,
-                                     &splitbar[wi]);
+                        bulk_load_1d(smem_addr(buf), args.split_ws + slot_of(0) * kSplitSlotFloat4,
+                                     bytes, &splitbar[wi]);
                     }
                     if (mbar_wait(&splitbar[wi], 0, args.err, W_SPLIT_LOAD))
                         part = reinterpret_cast<const float4*>(buf);
                     else  // error recorded; give the copy a second bounded wait before exit
                         mbar_wait(&splitbar[wi], 0, args.err, W_SPLIT_LOAD);
+                } else if (ready) {
+                    if constexpr (MULTI) {
+                        __syncwarp();  // lane 0's acquire of the flags, then every lane's reads
+                        __threadfence();
+                        gpart = args.split_ws + slot_of(0) * kSplitSlotFloat4;
+                    }
                 }
             }
             if constexpr (EPI == kEpiSwigluFwd) {
@@ -505,6 +549,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                             for (int e = 0; e < 4; ++e)
                                 r[4 * i + e] =
                                     __float_as_uint(__fadd_rn(q[e], __uint_as_float(r[4 * i + e])));
+                        }
+                    } else if (MULTI && gpart) {
+                        // parts 0..S-2 in order; a part's slots are 2 ranks x 4 warps apart
+#pragma unroll 1
+                        for (int p = 0; p < S - 1; ++p) {
+                            const float4* src = gpart +
+                                                (size_t)p * 2 * NUM_EPI_WARPS * kSplitSlotFloat4 +
+                                                (size_t)(c * 8) * 32 + lane;
+                            float4 v[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) v[i] = __ldcg(src + i * 32);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float q[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    r[4 * i + e] = __float_as_uint(
+                                        __fadd_rn(q[e], __uint_as_float(r[4 * i + e])));
+                            }
                         }
                     }
                     uint32_t hw[16];  // saved H, two bf16 per word, columns 2i and 2i+1
@@ -832,25 +895,41 @@ bool ensure_smem(F* kernel, int bytes, bool (&done)[64]) {
     return true;
 }
 
-template <int EPI>
-lm_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
-                      const CUtensorMap& tx, const CUtensorMap& td2, const GemmArgs& a,
-                      cudaStream_t s) {
+template <int EPI, bool MULTI>
+lm_status launch_pair_as(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                         const CUtensorMap& tx, const CUtensorMap& td2, const GemmArgs& a,
+                         cudaStream_t s) {
     static bool done[64] = {};
-    if (!ensure_smem(pair::gemm_fp8_pair_kernel<EPI>, pair::SMEM_BYTES, done)) return LM_ERR_CUDA;
+    if (!ensure_smem(pair::gemm_fp8_pair_kernel<EPI, MULTI>, pair::SMEM_BYTES, done))
+        return LM_ERR_CUDA;
     const int sms = sm_count();
     if (sms < 2) return LM_ERR_CUDA;
     const int clusters = a.num_units < sms / 2 ? a.num_units : sms / 2;
     timing_mark(s, 'g');
-    if (a.split_flags && a.num_units > a.split_first &&
+    if (a.split_flags && a.split_slots > 0 &&
         cudaMemsetAsync(a.split_flags, 0,
-                        (size_t)(a.num_units - a.split_first) / 2 * 2 * NUM_EPI_WARPS *
-                            sizeof(unsigned int),
+                        (size_t)a.split_slots * 2 * NUM_EPI_WARPS * sizeof(unsigned int),
                         s) != cudaSuccess)
         return LM_ERR_CUDA;
-    pair::gemm_fp8_pair_kernel<EPI><<<2 * clusters, NUM_THREADS, pair::SMEM_BYTES, s>>>(ta, tb, td,
-                                                                                      tx, td2, a);
+    pair::gemm_fp8_pair_kernel<EPI, MULTI>
+        <<<2 * clusters, NUM_THREADS, pair::SMEM_BYTES, s>>>(ta, tb, td, tx, td2, a);
     return launch_status();
+}
+
+// No split or halves in one round: the lean instantiation; three or more parts
+// (never for the gated epilogue): the one that reads partials from global memory.
+template <int EPI>
+lm_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                      const CUtensorMap& tx, const CUtensorMap& td2, const GemmArgs& a,
+                      cudaStream_t s) {
+    if constexpr (EPI == kEpiSwigluFwd) {
+        return launch_pair_as<EPI, false>(ta, tb, td, tx, td2, a, s);
+    } else {
+        const bool halves_in_one_round =
+            a.split_parts <= 2 && a.num_units - a.split_first <= a.split_round;
+        if (!halves_in_one_round) return launch_pair_as<EPI, true>(ta, tb, td, tx, td2, a, s);
+        return launch_pair_as<EPI, false>(ta, tb, td, tx, td2, a, s);
+    }
 }
 
 template <int EPI>
@@ -870,7 +949,71 @@ lm_status launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArg
 }  // namespace lm
 
 size_t lm::gemm_split_workspace_bytes() {
-    return (size_t)kSplitMaxTiles * (kSplitTileBytes + 2 * NUM_EPI_WARPS * sizeof(unsigned int));
+    return (size_t)kSplitMaxSlots * (kSplitTileBytes + 2 * NUM_EPI_WARPS * sizeof(unsigned int));
+}
+
+namespace lm {
+namespace {
+
+// Modelled time of the last wave's rem tiles run as S parts each, in units of
+// one k-block of one tile: the rounds they take, each as long as one part's
+// k-blocks plus the last part's reads of the other S - 1 partial sums.  Each
+// read costs about 14 k-block times (5.6 us for 128 KB per CTA, read in 4 KB
+// steps per warp): measured on B200 with the 48-tile wgrad of a 1024-row
+// linear, where three parts over two rounds ran 15 us slower than no split.
+double split_tail_cost(int rem, int num_kb, int C, int S) {
+    const int per_round = C / S;
+    const int rounds = (rem + per_round - 1) / per_round;
+    return rounds * ((double)num_kb / S + 14.0 * (S - 1));
+}
+
+// Parts per tile for the last wave of a CTA-pair GEMM with num_tiles tiles of
+// num_kb k-blocks on C clusters (1: no split).
+//  - A last wave of rem <= C / 2 tiles is halved, as long as each half gets a
+//    k-block; more parts only when the model above is 25% faster than halves.
+//  - A fuller last wave takes the fastest S of the model when that is at least
+//    10% faster than leaving the wave unsplit.
+// S is at most kSplitMaxParts, each part gets two k-blocks or more when S > 2,
+// and the partials fit the workspace (rem * (S - 1) <= kSplitMaxSlots).
+int split_parts_for(int num_tiles, int num_kb, int C) {
+    if (C < 2) return 1;
+    const int rem = num_tiles % C;
+    if (rem == 0 || num_kb < 2) return 1;
+    const bool halves = 2 * rem <= C && rem <= kSplitMaxSlots;
+    const double bound = halves ? 0.75 * split_tail_cost(rem, num_kb, C, 2) : 0.9 * num_kb;
+    int best = halves ? 2 : 1;
+    double best_cost = 1e300;
+    for (int S = halves ? 3 : 2; S <= kSplitMaxParts; ++S) {
+        if (C / S < 1 || num_kb < 2 * S || (int64_t)rem * (S - 1) > kSplitMaxSlots) continue;
+        const double c = split_tail_cost(rem, num_kb, C, S);
+        if (c <= bound && c < best_cost) {
+            best = S;
+            best_cost = c;
+        }
+    }
+    return best;
+}
+
+}  // namespace
+}  // namespace lm
+
+extern "C" lm_status lm_fp8_gemm_split_plan(int64_t M, int64_t N, int64_t K, int sm_count,
+                                            int* parts, int* tail_tiles) {
+    if (!parts || !tail_tiles || M < 0 || N < 0 || K < 0 || sm_count < 2)
+        return LM_ERR_INVALID_ARG;
+    *parts = 1;
+    *tail_tiles = 0;
+    if (M <= 128 || N == 0 || K == 0) return LM_OK;  // the single-CTA kernel: never split
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    const int64_t num_kb = (K + lm::BK - 1) / lm::BK;
+    if (tiles >= (int64_t(1) << 31) || num_kb >= (int64_t(1) << 31)) return LM_ERR_UNSUPPORTED_SHAPE;
+    const int C = sm_count / 2;
+    const int S = lm::split_parts_for((int)tiles, (int)num_kb, C);
+    if (S > 1) {
+        *parts = S;
+        *tail_tiles = (int)(tiles % C);
+    }
+    return LM_OK;
 }
 
 lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
@@ -938,25 +1081,38 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
         // spanning M).
         a.stream_a = N <= M ? 1 : 0;
         a.group_m = a.stream_a ? 1 : a.num_mb;
-        // split-K tail: with a workspace, a last wave of r tiles on C clusters
-        // with 2r <= C becomes 2r half-K units in the same round
+        // split-K tail: with a workspace, the last wave's rem tiles may run as
+        // S parts each over ranges of K, P = C / S tiles per round of C units
         a.num_units = a.num_tiles;
         a.split_first = a.num_tiles;
+        a.split_parts = 1;
+        a.split_round = 1;
+        a.split_per_round = 1;
+        a.split_slots = 0;
         a.split_ws = nullptr;
         a.split_flags = nullptr;
         const int sms = sm_count();
         if (sms < 2) return LM_ERR_CUDA;
         const int C = sms / 2;
         const int rem = a.num_tiles % C;
-        if (workspace && epi != kEpiSwigluFwd && a.num_kb >= 2 && rem > 0 && 2 * rem <= C &&
-            rem <= kSplitMaxTiles && aligned16(workspace) &&
-            ws_bytes >=
-                (size_t)rem * (kSplitTileBytes + 2 * NUM_EPI_WARPS * sizeof(unsigned int))) {
+        const int S = workspace && epi != kEpiSwigluFwd && aligned16(workspace)
+                          ? split_parts_for(a.num_tiles, a.num_kb, C)
+                          : 1;
+        const size_t slots = (size_t)rem * (size_t)(S - 1);
+        if (S > 1 &&
+            ws_bytes >= slots * (kSplitTileBytes + 2 * NUM_EPI_WARPS * sizeof(unsigned int))) {
+            const int P = C / S;
+            const int rounds = (rem + P - 1) / P;
             a.split_first = a.num_tiles - rem;
-            a.num_units = a.num_tiles + rem;
+            a.split_parts = S;
+            a.split_round = C;
+            a.split_per_round = P;
+            a.split_slots = (int)slots;
+            // full rounds, then the last round's tiles (no idle units at the end)
+            a.num_units = a.split_first + (rounds - 1) * C + (rem - (rounds - 1) * P) * S;
             a.split_ws = static_cast<float4*>(workspace);
             a.split_flags = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) +
-                                                            (size_t)rem * kSplitTileBytes);
+                                                            slots * kSplitTileBytes);
         }
         a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, pair::TILE_M, pair::TILE_N, a.a_mn, a.b_mn);
         CUtensorMap td, tx;
@@ -1000,6 +1156,10 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
     a.num_tiles = a.num_mb * a.num_nb;
     a.num_units = a.num_tiles;
     a.split_first = a.num_tiles;
+    a.split_parts = 1;
+    a.split_round = 1;
+    a.split_per_round = 1;
+    a.split_slots = 0;
     a.split_ws = nullptr;
     a.split_flags = nullptr;
     a.group_m = 16;

@@ -151,13 +151,14 @@ LM_API lm_status lm_fp8_gemm(const uint8_t* A, lm_fp8_format fa, const uint8_t* 
  *
  * workspace (device, 16-byte aligned, >= lm_fp8_gemm_workspace_size() bytes,
  * or NULL): scratch for a split-K tail.  The persistent grid gives tiles out
- * round-robin; when the last wave holds at most half as many tiles as there
- * are CTA pairs, each of those tiles is computed as two half-K units that run
- * at once, the second adding the first's fp32 sums (exchanged through the
- * workspace) before the epilogue.  The result then differs from the
- * unsplit one only by fp32 summation order; it is the same from call to call.
- * Calls that share a workspace must not overlap on the GPU.  With NULL
- * (ws_bytes 0) no tile is split.
+ * round-robin, so a last wave with fewer tiles than CTA pairs leaves pairs
+ * idle.  Each tile of that wave may instead be computed as S units over S
+ * ranges of K (lm_fp8_gemm_split_plan gives S for a shape): the last unit of
+ * a tile adds the others' fp32 sums, exchanged through the workspace, before
+ * the epilogue.  The result then differs from the unsplit one only by fp32
+ * summation order; it is the same from call to call.  Calls that share a
+ * workspace must not overlap on the GPU.  With NULL (ws_bytes 0) no tile is
+ * split.
  * Operands stored MN-major give bit-identical results to lm_fp8_gemm on the
  * transposed copies (with the same workspace choice).
  */
@@ -168,8 +169,20 @@ LM_API lm_status lm_fp8_gemm_ex(const uint8_t* A, lm_fp8_format fa, const uint8_
                          size_t ws_bytes, lm_stream_t stream);
 
 /* Workspace bytes that let lm_fp8_gemm_ex split the last wave of any shape
- * (a fixed size: 64 tiles' fp32 sums and flags, about 16 MB). */
+ * (a fixed size: 128 partial tiles' fp32 sums and flags, about 32 MB). */
 LM_API size_t lm_fp8_gemm_workspace_size(void);
+
+/* The split-K tail lm_fp8_gemm_ex (with a workspace) uses for an M x N x K
+ * GEMM on a GPU of sm_count multiprocessors.  Host arithmetic only; nothing
+ * is launched and no GPU is needed.  *parts: the K ranges each tile of the
+ * last wave runs as (1: no split); *tail_tiles: how many tiles are split.
+ *  - A last wave of at most half as many tiles as CTA pairs is halved.
+ *  - Otherwise the wave's tiles are split only when a time model of the tail
+ *    says that more parts are clearly faster.
+ *  - Shapes with M <= 128 (a single-CTA kernel) are never split.
+ * Returns LM_ERR_INVALID_ARG for null outputs, negative sizes or sm_count < 2. */
+LM_API lm_status lm_fp8_gemm_split_plan(int64_t M, int64_t N, int64_t K, int sm_count,
+                                        int* parts, int* tail_tiles);
 
 /*
  * The producer of a GEMM input: RMSNorm, then the dynamic FP8 cast of its

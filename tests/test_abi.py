@@ -82,9 +82,9 @@ def test_mlp_sizes_and_carve(L):
     # H, h codes and the scales; scratch dY codes, dH, dH codes, scales
     assert L.lm_relu2_mlp_saved_bytes(M, d, f) == (r(M * d) + 2 * r(f * d) + r(2 * M * f)
                                                    + r(M * f) + r(64))
-    # scratch: the GEMMs' split-K scratch (64 tiles x 256 KB of fp32 sums plus a
-    # flag per CTA and warp), then dY codes, dH, dH codes, scales
-    split = 64 * (256 * 1024 + 2 * 4 * 4)
+    # scratch: the GEMMs' split-K scratch (128 partial tiles x 256 KB of fp32 sums
+    # plus a flag per CTA and warp), then dY codes, dH, dH codes, scales
+    split = 128 * (256 * 1024 + 2 * 4 * 4)
     assert L.lib.lm_fp8_gemm_workspace_size() == split
     assert L.lm_relu2_mlp_workspace_size(M, d, f) == (r(split) + r(M * d) + r(2 * M * f)
                                                       + r(M * f) + r(32))
@@ -175,3 +175,57 @@ def test_linear_sizes_carve_and_checks(L):
     assert bwd(fake, C.byref(s), M, K, N, fake, fake, fake + 16, ws, 0, None) == 2
     assert bwd(fake, C.byref(s), M, K, N, fake, fake, fake, ws, 1, None) == 1   # fwd's flag
     assert bwd(fake, C.byref(s), M, K, N, fake, None, fake, ws, 0, None) == 1   # dW needed
+
+
+def test_split_plan_on_a_148_sm_gpu(L):
+    """The split-K tail plan (host arithmetic).  With 148 SMs there are C = 74
+    CTA pairs; the last wave holds rem = tiles mod 74 tiles of 256 x 256."""
+    plan = lambda M, N, K: L.lm_fp8_gemm_split_plan(M, N, K, 148)
+    # relu^2 MLP, M = 16384: N = 3072 GEMMs have 768 tiles, rem 28 <= 37: halves
+    assert plan(16384, 3072, 12288) == (2, 28)
+    # N = 12288 GEMMs: 3072 tiles, rem 38 > 37, K = 3072 too short to gain: unsplit
+    assert plan(16384, 12288, 3072) == (1, 0)
+    # wgrads: 576 tiles, rem 58; more parts would need 2+ rounds each: unsplit
+    assert plan(3072, 12288, 16384) == (1, 0) and plan(12288, 3072, 16384) == (1, 0)
+    # K / V wgrad: 48 tiles, all in the last wave; three parts would take two
+    # rounds and two partial reads each, measured slower: unsplit
+    assert plan(1024, 3072, 8192) == (1, 0) and plan(1024, 3072, 16384) == (1, 0)
+    # deep K pays for more parts: 44 tiles, K = 32768, three parts in two rounds
+    assert plan(256 * 44, 256, 32768) == (3, 44)
+    # LM head dgrad (K = 50304): 384 tiles, rem 14; five parts in one round
+    assert plan(8192, 3072, 50304) == (5, 14)
+    # a chunk's dgrad in the fused LM head: 192 tiles, rem 44: three parts
+    assert plan(4096, 3072, 50304) == (3, 44)
+    # short K with a small tail keeps halves (8 k-blocks: more parts do not pay)
+    assert plan(8192, 3072, 1024) == (2, 14)
+    # a single k-block is never split; M <= 128 takes the single-CTA kernel
+    assert plan(512, 512, 128) == (1, 0) and plan(128, 4096, 4096) == (1, 0)
+    # no last wave to fill
+    assert plan(256 * 74, 256, 4096) == (1, 0)
+    import ctypes as C
+    p, t = C.c_int(), C.c_int()
+    assert L.lib.lm_fp8_gemm_split_plan(256, 256, 256, 1, C.byref(p), C.byref(t)) == 1
+    assert L.lib.lm_fp8_gemm_split_plan(-1, 256, 256, 148, C.byref(p), C.byref(t)) == 1
+    assert L.lib.lm_fp8_gemm_split_plan(256, 256, 256, 148, None, C.byref(t)) == 1
+
+
+def test_split_plan_invariants_over_shapes(L):
+    """For every plan: parts in [1, 8]; a split tail has two k-blocks per part
+    (one for halves) and its partials fit the workspace's 128 tiles."""
+    for sms in (148, 132, 16):
+        C = sms // 2
+        for M in (256, 768, 4096, 16384, 40960):
+            for N in (256, 1024, 3072, 12288, 50304):
+                for K in (128, 256, 1024, 3072, 12288, 50304):
+                    S, rem = L.lm_fp8_gemm_split_plan(M, N, K, sms)
+                    tiles = -(-M // 256) * -(-N // 256)
+                    kb = -(-K // 128)
+                    assert 1 <= S <= 8
+                    if S == 1:
+                        assert rem == 0
+                        continue
+                    assert rem == tiles % C and rem > 0
+                    assert kb >= (2 if S == 2 else 2 * S)
+                    assert rem * (S - 1) <= 128
+                    if 2 * rem <= C:
+                        assert S >= 2   # a tail of at most half the pairs is always split
