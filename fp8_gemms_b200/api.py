@@ -5,6 +5,10 @@ libfp8lm.so does every step of the computation.
     mlp = api.Relu2Mlp(M, d, f)          # caller-owned saved tensors + workspace
     Y = mlp.forward(X, W_up, W_down)
     dX, dW_up, dW_down = mlp.backward(dY)
+
+    lin = api.Linear(M, K, N)            # a plain linear Y = X W^T (attention, LM head)
+    Y = lin.forward(X, W)
+    dX, dW = lin.backward(dY)
 """
 import torch
 
