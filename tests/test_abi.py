@@ -229,3 +229,37 @@ def test_split_plan_invariants_over_shapes(L):
                     assert rem * (S - 1) <= 128
                     if 2 * rem <= C:
                         assert S >= 2   # a tail of at most half the pairs is always split
+
+
+def test_plain_c_program_uses_the_boundary(L, tmp_path):
+    """The header is plain C99, and a C program links against the library and
+    calls its host-only entry points (no torch, no GPU)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not found")
+    src = tmp_path / "use_abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "lm_fp8.h"
+int main(void) {
+    int parts = 0, tail = 0;
+    if (lm_fp8_gemm_split_plan(16384, 3072, 12288, 148, &parts, &tail) != LM_OK) return 1;
+    lm_linear_saved s;
+    if (lm_fp8_linear_saved_carve((void*)0x100000, lm_fp8_linear_saved_bytes(256, 192, 320),
+                                  256, 192, 320, &s) != LM_OK) return 2;
+    printf("%d|%d|%d|%zu|%s\n", parts, tail, (int)((char*)s.Wq - (char*)s.Xq),
+           lm_fp8_gemm_workspace_size(), lm_status_string(LM_ERR_ALIGNMENT));
+    return 0;
+}
+""")
+    exe = tmp_path / "use_abi"
+    libdir = os.path.dirname(L.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-L", libdir, "-lfp8lm",
+                    "-Wl,-rpath," + libdir, "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True,
+                         text=True).stdout.strip().split("|")
+    assert out[:3] == ["2", "28", str(256 * 192)]
+    assert int(out[3]) == L.lib.lm_fp8_gemm_workspace_size()
+    assert out[4].startswith("LM_ERR_ALIGNMENT")
