@@ -175,7 +175,9 @@ lm_status lm_get_error(lm_stream_t stream, uint32_t* where_out) {
         return LM_ERR_CUDA;
     if (where_out) *where_out = v;
     if (!v) return LM_OK;
-    return (v & 0xF00u) == 0x400u ? LM_ERR_INVALID_ARG : LM_ERR_TIMEOUT;
+    if ((v & 0xF00u) == 0x400u) return LM_ERR_INVALID_ARG;
+    if ((v & 0xF00u) == 0x500u) return LM_ERR_NONFINITE;
+    return LM_ERR_TIMEOUT;
 }
 
 const char* lm_status_string(lm_status s) {
@@ -187,7 +189,7 @@ const char* lm_status_string(lm_status s) {
         case LM_ERR_UNSUPPORTED_FORMAT: return "LM_ERR_UNSUPPORTED_FORMAT: unsupported format pair or epilogue";
         case LM_ERR_CUDA: return "LM_ERR_CUDA: CUDA call or kernel launch failed";
         case LM_ERR_TIMEOUT: return "LM_ERR_TIMEOUT: a device-side bounded wait ran out";
-        case LM_ERR_NONFINITE: return "LM_ERR_NONFINITE: non-finite amax";
+        case LM_ERR_NONFINITE: return "LM_ERR_NONFINITE: a cast met a NaN or infinite amax";
     }
     return "unknown lm_status";
 }

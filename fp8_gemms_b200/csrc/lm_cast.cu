@@ -172,8 +172,13 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const AmaxSet set) {
     }
 }
 
+// The scales of a tensor from its amax.  A NaN or infinite amax (the tensor
+// holds a NaN or an infinity) still yields the scales the formula gives -- a
+// NaN or zero scale -- and records kErrNonfiniteAmax in the error word, which
+// lm_get_error reports as LM_ERR_NONFINITE.
 __device__ __forceinline__ void write_scales(float amax, float fmax, float* amax_out,
-                                             float* scale_out, float* inv_out, float* scale_reg) {
+                                             float* scale_out, float* inv_out, float* scale_reg,
+                                             unsigned int* err) {
     const float a = amax < 1e-12f ? 1e-12f : amax;
     const float scale = __fdiv_rn(fmax, a);
     *scale_reg = scale;
@@ -181,13 +186,14 @@ __device__ __forceinline__ void write_scales(float amax, float fmax, float* amax
         *amax_out = amax;
         *scale_out = scale;
         *inv_out = __fdiv_rn(1.0f, scale);
+        if (!(amax <= 3.40282347e38f)) atomicCAS(err, 0u, kErrNonfiniteAmax);
     }
 }
 
 __global__ void scales_only_kernel(const float* amax_src, float fmax, float* amax_out,
-                                   float* scale_out, float* inv_out) {
+                                   float* scale_out, float* inv_out, unsigned int* err) {
     float s;
-    write_scales(*amax_src, fmax, amax_out, scale_out, inv_out, &s);
+    write_scales(*amax_src, fmax, amax_out, scale_out, inv_out, &s, err);
 }
 
 // Pass 2: scale, cast and transpose one 256 x 128 tile per block.  Tiles are
@@ -197,11 +203,11 @@ template <int FMT, bool RELU2>
 __global__ void __launch_bounds__(kThreads) cast_kernel(
     const uint16_t* __restrict__ x, int rows, int cols, int64_t ld, const float* amax_src,
     float* amax_out, float* scale_out, float* inv_out, uint8_t* __restrict__ q,
-    uint8_t* __restrict__ qT, int tiles_c, int num_tiles) {
+    uint8_t* __restrict__ qT, int tiles_c, int num_tiles, unsigned int* err) {
     __shared__ __align__(16) uint32_t tile[kCastRows][kCastCols / 4];
     const float fmax = FMT == LM_FP8_E4M3 ? 448.0f : 57344.0f;
     float scale;
-    write_scales(*amax_src, fmax, amax_out, scale_out, inv_out, &scale);
+    write_scales(*amax_src, fmax, amax_out, scale_out, inv_out, &scale, err);
 
     const int t = num_tiles - 1 - (int)blockIdx.x;
     const int r0 = (t / tiles_c) * kCastRows;
@@ -341,7 +347,7 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
     for (int j = 0; j < kMaxSet; ++j)
         if (j < set.n)
             write_scales(*set.amax_src[j], fmax, set.amax_out[j], set.scale_out[j], set.inv_out[j],
-                         &sc[j]);
+                         &sc[j], err);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -531,10 +537,12 @@ lm_status launch_cast_rows(const CastItem& it, const float* amax_src, cudaStream
     const int rows = (int)it.rows, cols = (int)it.cols;
     const int tiles_c = (cols + kCastCols - 1) / kCastCols;
     const int n = ((rows + kCastRows - 1) / kCastRows) * tiles_c;
+    unsigned int* err = device_error_word();
+    if (!err) return LM_ERR_CUDA;
     timing_mark(s, 'c');
     cast_kernel<FMT, RELU2><<<n, kThreads, 0, s>>>(static_cast<const uint16_t*>(it.x), rows, cols,
                                                   it.ld, amax_src, it.amax_out, it.scale_out,
-                                                  it.inv_scale_out, it.q, it.qT, tiles_c, n);
+                                                  it.inv_scale_out, it.q, it.qT, tiles_c, n, err);
     return launch_status();
 }
 
@@ -631,9 +639,11 @@ lm_status lm::cast_set(const CastItem* items, int n, lm_fp8_format fmt, int relu
     for (int j = 0; j < n; ++j) {
         const CastItem& it = items[j];
         if (it.rows == 0 || it.cols == 0 || (!it.q && !it.qT)) {
+            unsigned int* err = device_error_word();
+            if (!err) return LM_ERR_CUDA;
             timing_mark(s, 's');
             scales_only_kernel<<<1, 1, 0, s>>>(src[j], fmax, it.amax_out, it.scale_out,
-                                               it.inv_scale_out);
+                                               it.inv_scale_out, err);
             if (launch_status() != LM_OK) return LM_ERR_CUDA;
         }
     }

@@ -14,6 +14,11 @@ namespace lm {
 // code of the bounded wait that ran out).  nullptr if CUDA is unusable.
 unsigned int* device_error_word();
 
+// Device error codes: 0x1xx-0x3xx a bounded wait ran out (LM_ERR_TIMEOUT),
+// 0x4xx invalid device-side data (LM_ERR_INVALID_ARG), 0x5xx a non-finite
+// value where the method needs a finite one (LM_ERR_NONFINITE).
+constexpr unsigned int kErrNonfiniteAmax = 0x501u;  // a cast met a NaN or infinite amax
+
 // Multiprocessor count of the current device (cached per device).
 int sm_count();
 

@@ -58,7 +58,7 @@ typedef enum {
     LM_ERR_UNSUPPORTED_FORMAT = 4, /* e5m2 x e5m2, or an unknown format/epilogue */
     LM_ERR_CUDA = 5,               /* a CUDA runtime/driver call or launch failed */
     LM_ERR_TIMEOUT = 6,            /* a device-side bounded wait ran out */
-    LM_ERR_NONFINITE = 7           /* reserved: non-finite amax reported by a check */
+    LM_ERR_NONFINITE = 7           /* a cast met a NaN or infinite amax (lm_get_error) */
 } lm_status;
 
 typedef enum { LM_FP8_E4M3 = 0, LM_FP8_E5M2 = 1 } lm_fp8_format;
@@ -432,12 +432,15 @@ LM_API lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* l
                                   size_t ws_bytes, lm_stream_t stream);
 
 /* Synchronises `stream`, then returns and clears the current device's error
- * word: LM_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
- * LM_ERR_INVALID_ARG if a kernel met invalid device-side data (code 0x401: a
- * label outside [0, V) in lm_fp8_lmhead_ce, treated as having no target),
- * LM_ERR_CUDA if the synchronisation itself failed, else LM_OK.  If
- * where_out is non-NULL it receives the code of the wait that ran out (0 if
- * none). */
+ * word (the first code recorded since the last call wins):
+ *  - LM_ERR_TIMEOUT if a kernel's bounded wait ran out;
+ *  - LM_ERR_INVALID_ARG if a kernel met invalid device-side data (code 0x401:
+ *    a label outside [0, V) in lm_fp8_lmhead_ce, treated as having no target);
+ *  - LM_ERR_NONFINITE if a cast's amax was NaN or infinite (code 0x501: the
+ *    tensor held a NaN or an infinity; its scales and codes follow the formulas
+ *    and are NaN or zero, and everything computed from them is meaningless);
+ *  - LM_ERR_CUDA if the synchronisation itself failed; else LM_OK.
+ * If where_out is non-NULL it receives the code (0 if none). */
 LM_API lm_status lm_get_error(lm_stream_t stream, uint32_t* where_out);
 
 /*

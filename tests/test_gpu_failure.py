@@ -31,3 +31,43 @@ def test_selftest_rejects_bad_limits():
     from fp8_gemms_b200 import _lib
     assert _lib.STATUS[_lib.lib.lm_selftest_bounded_wait(0, None)] == "LM_ERR_INVALID_ARG"
     assert _lib.STATUS[_lib.lib.lm_selftest_bounded_wait(6000, None)] == "LM_ERR_INVALID_ARG"
+
+
+@pytest.mark.parametrize("bad", [float("nan"), float("inf"), float("-inf")])
+@pytest.mark.parametrize("path", ["tma", "ragged_rows", "scales_only"])
+def test_nonfinite_amax_is_reported(bad, path):
+    """A tensor holding a NaN or an infinity has a non-finite amax.  Each cast
+    path then records code 0x501, and lm_get_error returns LM_ERR_NONFINITE
+    once (the word is cleared).  The same tensor made finite reports LM_OK."""
+    import math
+    from fp8_gemms_b200 import _lib
+    rows = 200 if path == "ragged_rows" else 64   # rows % 16 != 0: the per-tile kernel
+    x = torch.randn(rows, 128, device="cuda").to(torch.bfloat16)
+    x[3, 17] = bad
+    sc = torch.zeros(4, device="cuda")
+    q = None if path == "scales_only" else torch.empty(rows, 128, dtype=torch.uint8,
+                                                        device="cuda")
+    _lib.lm_fp8_amax_scale_cast(x, _lib.E4M3, sc[0:1], sc[1:2], sc[2:3], q, None)
+    st, where = _lib.lm_get_error()
+    assert _lib.STATUS[st] == "LM_ERR_NONFINITE" and where == 0x501
+    assert _lib.lm_get_error() == (0, 0)
+    amax = float(sc[0])
+    assert math.isnan(amax) if math.isnan(bad) else amax == math.inf
+    x[3, 17] = 0.0
+    _lib.lm_fp8_amax_scale_cast(x, _lib.E4M3, sc[0:1], sc[1:2], sc[2:3], q, None)
+    assert _lib.lm_get_error() == (0, 0)
+    assert math.isfinite(float(sc[0])) and float(sc[1]) > 0
+
+
+def test_nonfinite_input_to_the_mlp_is_reported():
+    """A NaN in X reaches the forward's cast of X: the block reports
+    LM_ERR_NONFINITE rather than returning codes silently derived from it."""
+    from fp8_gemms_b200 import _lib, api, synthetic
+    w = synthetic.TINY_MLP
+    t = {k: v.cuda() for k, v in w.tensors().items()}
+    t["X"][5, 9] = float("nan")
+    mlp = api.Relu2Mlp(w.M, w.d, w.f)
+    mlp.forward(t["X"], t["W_up"], t["W_down"])
+    st, where = _lib.lm_get_error()
+    assert _lib.STATUS[st] == "LM_ERR_NONFINITE" and where == 0x501
+    assert _lib.lm_get_error() == (0, 0)
