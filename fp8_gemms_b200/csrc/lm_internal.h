@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <initializer_list>
+
 #include "lm_fp8.h"
 
 namespace lm {
@@ -82,6 +84,15 @@ lm_status cast_set(const CastItem* items, int n, lm_fp8_format fmt, int relu2_in
 void timing_mark(cudaStream_t s, char kind);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Every pointer 16-byte aligned (a null pointer counts as aligned).  The
+// composite entry points check all their tensors with it before the first
+// launch, so a misaligned output is refused with nothing enqueued.
+inline bool all_aligned16(std::initializer_list<const void*> ps) {
+    for (const void* p : ps)
+        if (!aligned16(p)) return false;
+    return true;
+}
 
 inline lm_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? LM_OK : LM_ERR_CUDA;

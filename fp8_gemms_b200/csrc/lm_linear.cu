@@ -97,6 +97,7 @@ lm_status lm_fp8_linear_fwd(const void* X, const void* W, int64_t M, int64_t K, 
     // with M == 0 there is no X or Y to touch (W is still cast)
     if (!sv || (M > 0 && (!X || !Y)) || (!reuse && !W)) return LM_ERR_INVALID_ARG;
     if (!sv->Xq || !sv->Wq || !sv->scales) return LM_ERR_INVALID_ARG;
+    if (!lm::all_aligned16({X, W, Y, sv->Xq, sv->Wq})) return LM_ERR_ALIGNMENT;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t split_bytes = lm::gemm_split_workspace_bytes();
     void* split = workspace && ws_bytes >= split_bytes ? workspace : nullptr;
@@ -124,6 +125,7 @@ lm_status lm_fp8_linear_bwd(const void* dY, const lm_linear_saved* sv, int64_t M
     if (ws_bytes < bwd_layout(M, N, nullptr, nullptr, nullptr, nullptr))
         return LM_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return LM_ERR_ALIGNMENT;
+    if (!lm::all_aligned16({dY, dX, dW, sv->Xq, sv->Wq})) return LM_ERR_ALIGNMENT;
     void* split;
     uint8_t* dYq;
     float* G;

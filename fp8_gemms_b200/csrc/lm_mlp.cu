@@ -112,6 +112,8 @@ lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_dow
     if (!X || !Y || !sv || (!reuse && (!W_up || !W_down))) return LM_ERR_INVALID_ARG;
     if (!sv->Xq || !sv->Wuq || !sv->Wdq || !sv->H || !sv->hq || !sv->scales)
         return LM_ERR_INVALID_ARG;
+    if (!lm::all_aligned16({X, W_up, W_down, Y, sv->Xq, sv->Wuq, sv->Wdq, sv->H, sv->hq}))
+        return LM_ERR_ALIGNMENT;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // the workspace, when given, holds the GEMMs' split-K scratch at its start
     const size_t split_bytes = lm::gemm_split_workspace_bytes();
@@ -159,6 +161,10 @@ lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* sv, int64_t M,
     if (!dY || !sv || !dX || !dW_up || !dW_down || !workspace) return LM_ERR_INVALID_ARG;
     if (ws_bytes < bwd_layout(M, d, f, nullptr, nullptr)) return LM_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return LM_ERR_ALIGNMENT;
+    if (!sv->Xq || !sv->Wuq || !sv->Wdq || !sv->H || !sv->hq || !sv->scales)
+        return LM_ERR_INVALID_ARG;
+    if (!lm::all_aligned16({dY, dX, dW_up, dW_down, sv->Xq, sv->Wuq, sv->Wdq, sv->H, sv->hq}))
+        return LM_ERR_ALIGNMENT;
     const lm_epilogue wgrad_epi =
         (flags & LM_MLP_ACCUMULATE_WGRAD) ? LM_EPI_ACCUM_F32 : LM_EPI_NONE;
     BwdWorkspace w;

@@ -175,6 +175,8 @@ lm_status lm_swiglu_mlp_fwd(const void* X, const void* W_gu, const void* W_down,
     if (!X || !W_gu || !W_down || !Y || !sv || !sv->Xq || !sv->Wguq || !sv->Wdq || !sv->GU ||
         !sv->h || !sv->hq || !sv->scales)
         return LM_ERR_INVALID_ARG;
+    if (!all_aligned16({X, W_gu, W_down, Y, sv->Xq, sv->Wguq, sv->Wdq, sv->GU, sv->h, sv->hq}))
+        return LM_ERR_ALIGNMENT;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     float* S = sv->scales;
     if (cudaMemsetAsync(S, 0, 16 * sizeof(float), s) != cudaSuccess) return LM_ERR_CUDA;
@@ -204,6 +206,11 @@ lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* sv, int64_t M
     if (!dY || !sv || !dX || !dW_gu || !dW_down || !workspace) return LM_ERR_INVALID_ARG;
     if (ws_bytes < bwd_layout(M, d, f, nullptr, nullptr)) return LM_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return LM_ERR_ALIGNMENT;
+    if (!sv->Xq || !sv->Wguq || !sv->Wdq || !sv->GU || !sv->h || !sv->hq || !sv->scales)
+        return LM_ERR_INVALID_ARG;
+    if (!all_aligned16({dY, dX, dW_gu, dW_down, sv->Xq, sv->Wguq, sv->Wdq, sv->GU, sv->h,
+                        sv->hq}))
+        return LM_ERR_ALIGNMENT;
     BwdWs w;
     bwd_layout(M, d, f, static_cast<uint8_t*>(workspace), &w);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

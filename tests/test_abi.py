@@ -263,3 +263,39 @@ int main(void) {
     assert out[:3] == ["2", "28", str(256 * 192)]
     assert int(out[3]) == L.lib.lm_fp8_gemm_workspace_size()
     assert out[4].startswith("LM_ERR_ALIGNMENT")
+
+
+def test_composite_entry_points_refuse_misaligned_tensors_before_any_launch(L):
+    """A misaligned output of a composite call is refused before its first
+    launch: the status is LM_ERR_ALIGNMENT, not the LM_ERR_CUDA that reaching a
+    CUDA call would give on a host without a GPU."""
+    import ctypes as C
+    fake, bad = 0x100000, 0x100008           # 16-byte aligned / 8 bytes off
+    mlp = L.MlpSaved(*([fake] * 6))
+    sw = L.SwigluSaved(*([fake] * 7))
+    lin = L.LinearSaved(fake, fake, fake)
+    ws = 1 << 31
+    lib = L.lib
+    M, d, f = 256, 256, 1024
+    # relu^2 MLP: misaligned Y (forward), dX (backward), a saved tensor (both)
+    assert lib.lm_relu2_mlp_fwd(fake, fake, fake, M, d, f, bad, C.byref(mlp), None, 0, None) == 2
+    assert lib.lm_relu2_mlp_bwd(fake, C.byref(mlp), M, d, f, bad, fake, fake, fake, ws, None) == 2
+    mlp_bad = L.MlpSaved(fake, fake, fake, bad, fake, fake)       # H
+    assert lib.lm_relu2_mlp_fwd(fake, fake, fake, M, d, f, fake, C.byref(mlp_bad), None, 0,
+                                None) == 2
+    assert lib.lm_relu2_mlp_bwd(fake, C.byref(mlp_bad), M, d, f, fake, fake, fake, fake, ws,
+                                None) == 2
+    # gated MLP (f a multiple of 128)
+    assert lib.lm_swiglu_mlp_fwd(fake, fake, fake, M, d, f, bad, C.byref(sw), None, 0, None) == 2
+    assert lib.lm_swiglu_mlp_bwd(fake, C.byref(sw), M, d, f, fake, bad, fake, fake, ws, None) == 2
+    # plain linear: misaligned Y, dW, saved codes
+    K, N = 192, 320
+    assert lib.lm_fp8_linear_fwd(fake, fake, M, K, N, bad, C.byref(lin), None, 0, 0, None) == 2
+    assert lib.lm_fp8_linear_bwd(fake, C.byref(lin), M, K, N, fake, bad, fake, ws, 0, None) == 2
+    lin_bad = L.LinearSaved(fake, bad, fake)
+    assert lib.lm_fp8_linear_fwd(fake, fake, M, K, N, fake, C.byref(lin_bad), None, 0, 0,
+                                 None) == 2
+    # a missing saved buffer is an argument error, in the backward too
+    sw_null = L.SwigluSaved(fake, fake, fake, None, fake, fake, fake)
+    assert lib.lm_swiglu_mlp_bwd(fake, C.byref(sw_null), M, d, f, fake, fake, fake, fake, ws,
+                                 None) == 1
