@@ -68,9 +68,9 @@ def lib():
         L.orc_gemm_accum_f32.restype = None
         L.orc_rmsnorm.argtypes = [P, P, i64, i64, ctypes.c_double, P]
         L.orc_rmsnorm.restype = None
-        L.orc_swiglu_h.argtypes = [P, i64, i64, P]
+        L.orc_swiglu_h.argtypes = [P, P, i64, i64, P]
         L.orc_swiglu_h.restype = ctypes.c_float
-        L.orc_swiglu_bwd.argtypes = [P, P, i64, i64, P]
+        L.orc_swiglu_bwd.argtypes = [P, P, P, i64, i64, P, P]
         L.orc_swiglu_bwd.restype = ctypes.c_float
         L.orc_swiglu_f64.argtypes = [P, P, P, P, P, i64, i64, i64, P, P, P, P, P]
         L.orc_swiglu_f64.restype = None
@@ -78,6 +78,8 @@ def lib():
         L.orc_softcap_ce.restype = None
         L.orc_mlp_f64.argtypes = [P, P, P, P, i64, i64, i64, P, P, P, P]
         L.orc_mlp_f64.restype = None
+        L.orc_lmhead_ce_f64.argtypes = [P, P, P, i64, i64, i64, ctypes.c_double, P, P, P]
+        L.orc_lmhead_ce_f64.restype = None
         _lib = L
     return _lib
 
@@ -305,64 +307,76 @@ def mlp_f64(X, W_up, W_down, dY=None):
 
 
 # ------------------------------------------------ gated (SwiGLU) variant
-def interleave_gate_up(Wg, Wu):
-    """Rows of W_gate and W_up (each f x d) interleaved in blocks of 128:
-    [Wg[0:128]; Wu[0:128]; Wg[128:256]; Wu[128:256]; ...] (f % 128 == 0)."""
-    f, d = Wg.shape
-    assert f % 128 == 0 and Wu.shape == (f, d)
-    out = np.empty((2 * f, d), Wg.dtype)
-    for b in range(f // 128):
-        out[256 * b:256 * b + 128] = Wg[128 * b:128 * b + 128]
-        out[256 * b + 128:256 * b + 256] = Wu[128 * b:128 * b + 128]
+def amax_scale_cast_joint(tensors, fmt, amax_in=None):
+    """Several tensors quantised as ONE tensor: one amax over all of them, one
+    scale, then each tensor's codes (+ transposes) at that scale.  The gated
+    block's gate and up weights form one fused weight, and its dG and dU one
+    gradient, so each pair shares a tensorwise scale."""
+    a = max(amax(t) for t in tensors) if amax_in is None else np.float32(amax_in)
+    s, inv = scale(a, fmt)
+    out = dict(amax=np.float32(a), scale=s, inv_scale=inv, q=[], qT=[])
+    for t in tensors:
+        q, qT = cast(t, fmt, s)
+        out["q"].append(q)
+        out["qT"].append(qT)
     return out
 
 
-def deinterleave_gate_up(Wgu):
-    f = Wgu.shape[0] // 2
-    Wg = np.concatenate([Wgu[256 * b:256 * b + 128] for b in range(f // 128)])
-    Wu = np.concatenate([Wgu[256 * b + 128:256 * b + 256] for b in range(f // 128)])
-    return Wg, Wu
-
-
-def swiglu_h(GU):
-    GU = _c(GU, np.uint16)
-    M, f2 = GU.shape
-    h = np.zeros((M, f2 // 2), np.uint16)
-    a = lib().orc_swiglu_h(_ptr(GU), M, f2 // 2, _ptr(h))
+def swiglu_h(G, U):
+    """h = bf16(silu(G) U) from bf16 G, U [M x f]; returns (h, amax of h)."""
+    G = _c(G, np.uint16)
+    U = _c(U, np.uint16)
+    assert G.shape == U.shape
+    M, f = G.shape
+    h = np.zeros((M, f), np.uint16)
+    a = lib().orc_swiglu_h(_ptr(G), _ptr(U), M, f, _ptr(h))
     return h, np.float32(a)
 
 
-def swiglu_bwd(g, GU):
+def swiglu_bwd(g, G, U):
+    """dG = bf16(g U silu'(G)), dU = bf16(g silu(G)); returns (dG, dU, amax over both)."""
     g = _c(g, np.uint16)
-    GU = _c(GU, np.uint16)
+    G = _c(G, np.uint16)
+    U = _c(U, np.uint16)
+    assert g.shape == G.shape == U.shape
     M, f = g.shape
-    dGU = np.zeros((M, 2 * f), np.uint16)
-    a = lib().orc_swiglu_bwd(_ptr(g), _ptr(GU), M, f, _ptr(dGU))
-    return dGU, np.float32(a)
+    dG = np.zeros((M, f), np.uint16)
+    dU = np.zeros((M, f), np.uint16)
+    a = lib().orc_swiglu_bwd(_ptr(g), _ptr(G), _ptr(U), M, f, _ptr(dG), _ptr(dU))
+    return dG, dU, np.float32(a)
 
 
-def swiglu_fwd(X, W_gu, W_down):
-    """Gated MLP forward in FP8: W_gu is the interleaved [2f x d] gate/up weight."""
+def swiglu_fwd(X, W_gate, W_up, W_down):
+    """Gated MLP forward in FP8 (bf16 bits in): G = Xq Wgq^T, U = Xq Wuq^T,
+    h = silu(G) U, Y = hq Wdq^T.  W_gate and W_up share one scale."""
     cx = amax_scale_cast(X, E4M3)
-    cgu = amax_scale_cast(W_gu, E4M3)
+    cw = amax_scale_cast_joint([W_gate, W_up], E4M3)
     cd = amax_scale_cast(W_down, E4M3)
-    GU, _ = gemm(cx["q"], E4M3, cgu["q"], E4M3, cx["inv_scale"], cgu["inv_scale"])
-    h, amax_h = swiglu_h(GU)
+    G, _ = gemm(cx["q"], E4M3, cw["q"][0], E4M3, cx["inv_scale"], cw["inv_scale"])
+    U, _ = gemm(cx["q"], E4M3, cw["q"][1], E4M3, cx["inv_scale"], cw["inv_scale"])
+    h, amax_h = swiglu_h(G, U)
     ch = amax_scale_cast(h, E4M3, amax_in=amax_h)
     Y, _ = gemm(ch["q"], E4M3, cd["q"], E4M3, ch["inv_scale"], cd["inv_scale"])
-    return dict(Y=Y, X=cx, W_gu=cgu, W_down=cd, GU=GU, h_bf16=h, h=ch)
+    return dict(Y=Y, X=cx, W_gu=cw, W_down=cd, G=G, U=U, h_bf16=h, h=ch)
 
 
 def swiglu_bwd_chain(dY, saved):
+    """Gated MLP backward in FP8: g = dYq Wd (plain dgrad), dG and dU from g,
+    cast to e5m2 with one shared scale; dX = dGq Wgq + dUq Wuq as one GEMM over
+    the concatenated reduction [G | U]; dW_gate = dGq^T Xq, dW_up = dUq^T Xq,
+    dW_down = dYq^T hq."""
     cg = amax_scale_cast(dY, E5M2)
-    cx, cgu, cd, ch = saved["X"], saved["W_gu"], saved["W_down"], saved["h"]
+    cx, cw, cd, ch = saved["X"], saved["W_gu"], saved["W_down"], saved["h"]
     g, _ = gemm(cg["q"], E5M2, cd["qT"], E4M3, cg["inv_scale"], cd["inv_scale"])
     dW_down, _ = gemm(cg["qT"], E5M2, ch["qT"], E4M3, cg["inv_scale"], ch["inv_scale"])
-    dGU, amax_d = swiglu_bwd(g, saved["GU"])
-    cdg = amax_scale_cast(dGU, E5M2, amax_in=amax_d)
-    dX, _ = gemm(cdg["q"], E5M2, cgu["qT"], E4M3, cdg["inv_scale"], cgu["inv_scale"])
-    dW_gu, _ = gemm(cdg["qT"], E5M2, cx["qT"], E4M3, cdg["inv_scale"], cx["inv_scale"])
-    return dict(dX=dX, dW_gu=dW_gu, dW_down=dW_down, dY=cg, g=g, dGU=dGU, dgu=cdg)
+    dG, dU, amax_d = swiglu_bwd(g, saved["G"], saved["U"])
+    cdg = amax_scale_cast_joint([dG, dU], E5M2, amax_in=amax_d)
+    dX, _ = gemm(np.hstack(cdg["q"]), E5M2, np.hstack(cw["qT"]), E4M3, cdg["inv_scale"],
+                 cw["inv_scale"])
+    dW_gate, _ = gemm(cdg["qT"][0], E5M2, cx["qT"], E4M3, cdg["inv_scale"], cx["inv_scale"])
+    dW_up, _ = gemm(cdg["qT"][1], E5M2, cx["qT"], E4M3, cdg["inv_scale"], cx["inv_scale"])
+    return dict(dX=dX, dW_gate=dW_gate, dW_up=dW_up, dW_down=dW_down, dY=cg, g=g, dG=dG,
+                dU=dU, dgu=cdg)
 
 
 def swiglu_f64(X, Wg, Wu, Wd, dY=None):
@@ -392,6 +406,23 @@ def softcap_ce(logits, labels, softcap=15.0, inv_count=None, want_grad=True):
     lib().orc_softcap_ce(_ptr(logits), _ptr(labels), rows, V, float(softcap), float(inv),
                          _ptr(dl), _ptr(loss))
     return loss, dl
+
+
+def lmhead_ce_f64(X, W, labels, softcap=15.0, want_grad=True):
+    """Unquantised, unchunked fp64 LM head + softcapped CE (float64 arrays in):
+    mean loss, dX [M x d], dW [V x d] of loss = mean(lse(z) - z[label]),
+    z = c tanh(X W^T / c)."""
+    X = _c(X, np.float64)
+    W = _c(W, np.float64)
+    labels = _c(np.asarray(labels, dtype=np.int32), np.int32)
+    M, d = X.shape
+    V = W.shape[0]
+    loss = np.zeros(1, np.float64)
+    dX = np.zeros((M, d)) if want_grad else None
+    dW = np.zeros((V, d)) if want_grad else None
+    lib().orc_lmhead_ce_f64(_ptr(X), _ptr(W), _ptr(labels), M, d, V, float(softcap), _ptr(loss),
+                            _ptr(dX), _ptr(dW))
+    return float(loss[0]), dX, dW
 
 
 def lmhead_ce(X, W, labels, chunk, softcap=15.0):

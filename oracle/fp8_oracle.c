@@ -321,45 +321,43 @@ void orc_rmsnorm(const uint16_t* R, const uint16_t* w, int64_t rows, int64_t col
 /* ------------------------------------------ gated (SwiGLU) MLP variant */
 /* The comparison workload of the "Niet-gated MLPs" bullet (decomputer.nl,
  * section "Doorvoer (Throughput) verhogen"): h = silu(G) * U with
- * G = X W_gate^T, U = X W_up^T, silu(x) = x / (1 + exp(-x)).
- * Layout used by the GEMM path: gate and up are interleaved in blocks of 128
- * columns, GU[:, 256 b + j] = G[:, 128 b + j] and GU[:, 256 b + 128 + j] =
- * U[:, 128 b + j] (j < 128); the same order holds for the interleaved weight
- * rows and for dGU.  Readings: h and dG, dU are each rounded once to bf16
- * from the exact (fp64) value of the product. */
+ * G = X W_gate^T, U = X W_up^T, silu(x) = x / (1 + exp(-x)).  G, U, h, dG and
+ * dU are separate row-major [M x f] tensors here.  Readings: h and dG, dU are
+ * each rounded once to bf16 from the exact (fp64) value of the product. */
 static double silu(double x) { return x / (1.0 + exp(-x)); }
 static double dsilu(double x) {
     double sg = 1.0 / (1.0 + exp(-x));
     return sg * (1.0 + x * (1.0 - sg));
 }
 
-/* h [M x f] from GU [M x 2f] (bf16 bits), amax of h returned. */
-float orc_swiglu_h(const uint16_t* GU, int64_t M, int64_t f, uint16_t* h) {
+/* h [M x f] from G and U [M x f] (bf16 bits); returns the amax of h. */
+float orc_swiglu_h(const uint16_t* G, const uint16_t* U, int64_t M, int64_t f, uint16_t* h) {
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t j = 0; j < f; ++j) {
-            int64_t b = j / 128, o = j % 128;
-            double g = orc_bf16_to_double(GU[m * 2 * f + 256 * b + o]);
-            double u = orc_bf16_to_double(GU[m * 2 * f + 256 * b + 128 + o]);
+            double g = orc_bf16_to_double(G[m * f + j]);
+            double u = orc_bf16_to_double(U[m * f + j]);
             h[m * f + j] = orc_bf16_from_double(silu(g) * u);
         }
     return orc_amax(h, M, f, f, 0);
 }
 
-/* dGU [M x 2f] from g = dh [M x f] and GU: dG = g U silu'(G), dU = g silu(G). */
-float orc_swiglu_bwd(const uint16_t* g_, const uint16_t* GU, int64_t M, int64_t f,
-                     uint16_t* dGU) {
+/* dG = g U silu'(G) and dU = g silu(G) [M x f] from g = dh and G, U [M x f];
+ * returns the amax over both (they form one tensor for the next cast). */
+float orc_swiglu_bwd(const uint16_t* g_, const uint16_t* G, const uint16_t* U, int64_t M,
+                     int64_t f, uint16_t* dG, uint16_t* dU) {
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t j = 0; j < f; ++j) {
-            int64_t b = j / 128, o = j % 128;
-            int64_t ig = m * 2 * f + 256 * b + o, iu = ig + 128;
-            double g = orc_bf16_to_double(g_[m * f + j]);
-            double G = orc_bf16_to_double(GU[ig]), U = orc_bf16_to_double(GU[iu]);
-            dGU[ig] = orc_bf16_from_double(g * U * dsilu(G));
-            dGU[iu] = orc_bf16_from_double(g * silu(G));
+            int64_t i = m * f + j;
+            double g = orc_bf16_to_double(g_[i]);
+            double gv = orc_bf16_to_double(G[i]), uv = orc_bf16_to_double(U[i]);
+            dG[i] = orc_bf16_from_double(g * uv * dsilu(gv));
+            dU[i] = orc_bf16_from_double(g * silu(gv));
         }
-    return orc_amax(dGU, M, 2 * f, 2 * f, 0);
+    float a = orc_amax(dG, M, f, f, 0), b = orc_amax(dU, M, f, f, 0);
+    if (a != a || b != b) return a != a ? a : b; /* a NaN amax propagates */
+    return a > b ? a : b;
 }
 
 /* ----------------------------- softcapped cross-entropy of the LM head */
@@ -394,6 +392,54 @@ void orc_softcap_ce(const uint16_t* logits, const int32_t* labels, int64_t rows,
                 dlogits[r * V + v] = orc_bf16_from_double(p * (1.0 - (z / c) * (z / c)) * inv_count);
             }
     }
+}
+
+/* Plain fp64 LM head with the softcapped cross-entropy, no quantisation and
+ * no chunking: the sanity reference for the FP8 chunked head, and the
+ * function whose gradient is pinned by finite differences of its loss.
+ *   l = X W^T [M x V],  z = c tanh(l / c),  loss = mean_r (lse_r - z[r, label_r])
+ *   dl = (softmax(z) - onehot) (1 - (z / c)^2) / M
+ *   dX = dl W [M x d],  dW = dl^T X [V x d]
+ * X: M x d, W: V x d (row-major doubles).  dX and dW may be NULL. */
+void orc_lmhead_ce_f64(const double* X, const double* W, const int32_t* labels, int64_t M,
+                       int64_t d, int64_t V, double c, double* loss_out, double* dX,
+                       double* dW) {
+    double* dl = (double*)calloc((size_t)(M * V > 0 ? M * V : 1), sizeof(double));
+    double total = 0.0;
+    for (int64_t r = 0; r < M; ++r) {
+        double* z = dl + r * V; /* holds z first, then dl */
+        double m = -INFINITY;
+        for (int64_t v = 0; v < V; ++v) {
+            double l = 0.0;
+            for (int64_t k = 0; k < d; ++k) l += X[r * d + k] * W[v * d + k];
+            z[v] = c * tanh(l / c);
+            if (z[v] > m) m = z[v];
+        }
+        double sum = 0.0;
+        for (int64_t v = 0; v < V; ++v) sum += exp(z[v] - m);
+        double lse = m + log(sum);
+        total += lse - z[labels[r]];
+        for (int64_t v = 0; v < V; ++v) {
+            double p = exp(z[v] - lse) - (v == labels[r] ? 1.0 : 0.0);
+            z[v] = p * (1.0 - (z[v] / c) * (z[v] / c)) / (double)M;
+        }
+    }
+    *loss_out = total / (double)M;
+    if (dX)
+        for (int64_t r = 0; r < M; ++r)
+            for (int64_t k = 0; k < d; ++k) {
+                double acc = 0.0;
+                for (int64_t v = 0; v < V; ++v) acc += dl[r * V + v] * W[v * d + k];
+                dX[r * d + k] = acc;
+            }
+    if (dW)
+        for (int64_t v = 0; v < V; ++v)
+            for (int64_t k = 0; k < d; ++k) {
+                double acc = 0.0;
+                for (int64_t r = 0; r < M; ++r) acc += dl[r * V + v] * X[r * d + k];
+                dW[v * d + k] = acc;
+            }
+    free(dl);
 }
 
 /* ---------------------------------------------- unquantised fp64 MLP chain */

@@ -13,6 +13,31 @@ pytestmark = pytest.mark.gpu
 E4M3, E5M2 = 0, 1
 
 
+# The library's gated block keeps gate and up side by side in one tensor,
+# alternating in blocks of 128 (rows of the fused weight W_gu [2f x d], columns
+# of the pre-activation GU [M x 2f]).  The oracle takes them separately; these
+# helpers move between the two layouts on the test side.
+def interleave_rows(Wg, Wu):
+    f = Wg.shape[0]
+    out = np.empty((2 * f,) + Wg.shape[1:], Wg.dtype)
+    for b in range(f // 128):
+        out[256 * b:256 * b + 128] = Wg[128 * b:128 * b + 128]
+        out[256 * b + 128:256 * b + 256] = Wu[128 * b:128 * b + 128]
+    return out
+
+
+def split_rows(Wgu):
+    f = Wgu.shape[0] // 2
+    Wg = np.concatenate([Wgu[256 * b:256 * b + 128] for b in range(f // 128)])
+    Wu = np.concatenate([Wgu[256 * b + 128:256 * b + 256] for b in range(f // 128)])
+    return Wg, Wu
+
+
+def split_cols(GU):
+    Gt, Ut = split_rows(np.ascontiguousarray(GU.T))
+    return np.ascontiguousarray(Gt.T), np.ascontiguousarray(Ut.T)
+
+
 def make(M, d, f, seed):
     X = synthetic.normal_bf16((M, d), 1.0, seed, 0)
     Wg = synthetic.normal_bf16((f, d), 0.02, seed, 1)
@@ -38,12 +63,14 @@ def test_swiglu_end_to_end_small(orc):
     X, Wg, Wu, Wd, dY = make(M, d, f, 80)
     mlp, Wgu, Y, dX, dWgu, dWd = run_gpu(M, d, f, X, Wg, Wu, Wd, dY)
     b = synthetic.bits_u16
-    fwd = orc.swiglu_fwd(b(X), orc.interleave_gate_up(b(Wg), b(Wu)), b(Wd))
+    fwd = orc.swiglu_fwd(b(X), b(Wg), b(Wu), b(Wd))
     bwd = orc.swiglu_bwd_chain(b(dY), fwd)
-    assert np.array_equal(u16(Wgu), orc.interleave_gate_up(b(Wg), b(Wu)))
+    assert np.array_equal(u16(Wgu), interleave_rows(b(Wg), b(Wu)))
     assert_close(u16(Y), fwd["Y"], "Y")
     assert_close(u16(dX), bwd["dX"], "dX")
-    assert_close(u16(dWgu), bwd["dW_gu"], "dW_gu")
+    dWg, dWu = split_rows(u16(dWgu))
+    assert_close(dWg, bwd["dW_gate"], "dW_gate")
+    assert_close(dWu, bwd["dW_up"], "dW_up")
     assert_close(u16(dWd), bwd["dW_down"], "dW_down")
 
 
@@ -52,15 +79,22 @@ def check_stagewise(orc, mlp, X, Wgu, rows=None):
     Xq, Wguq = u8(mlp.view("Xq")), u8(mlp.view("Wguq"))
     ref = orc.amax_scale_cast(synthetic.bits_u16(X), E4M3)
     assert np.array_equal(Xq, ref["q"]) and sc[0, 0] == ref["amax"]
-    refw = orc.amax_scale_cast(u16(Wgu), E4M3)
-    assert np.array_equal(Wguq, refw["q"]) and sc[1, 1] == refw["scale"]
-    GU = u16(mlp.view("GU"))
-    GUref, _ = orc.gemm(Xq, E4M3, Wguq, E4M3, sc[0, 2], sc[1, 2], rows=rows)
-    assert_close(GU if rows is None else GU[rows], GUref, "GU")
+    # the gate and up weights share one scale: their joint cast, bit-exact
+    Wg, Wu = split_rows(u16(Wgu))
+    refw = orc.amax_scale_cast_joint([Wg, Wu], E4M3)
+    Wgq, Wuq = split_rows(Wguq)
+    assert sc[1, 0] == refw["amax"] and sc[1, 1] == refw["scale"]
+    assert np.array_equal(Wgq, refw["q"][0]) and np.array_equal(Wuq, refw["q"][1])
+    G, U = split_cols(u16(mlp.view("GU")))
+    Gref, _ = orc.gemm(Xq, E4M3, Wgq, E4M3, sc[0, 2], sc[1, 2], rows=rows)
+    Uref, _ = orc.gemm(Xq, E4M3, Wuq, E4M3, sc[0, 2], sc[1, 2], rows=rows)
+    sel = (lambda a: a) if rows is None else (lambda a: a[rows])
+    assert_close(sel(G), Gref, "G")
+    assert_close(sel(U), Uref, "U")
     h = u16(mlp.view("h"))
-    # h from the GPU's own G|U: within one bf16 step of bf16(silu(G) U)
-    href, _ = orc.swiglu_h(GU if rows is None else GU[rows])
-    hv = (h if rows is None else h[rows]).astype(np.uint32) << 16
+    # h from the GPU's own G and U: within one bf16 step of bf16(silu(G) U)
+    href, _ = orc.swiglu_h(sel(G), sel(U))
+    hv = sel(h).astype(np.uint32) << 16
     rv = href.astype(np.uint32) << 16
     g, r = hv.view(np.float32).astype(np.float64), rv.view(np.float32).astype(np.float64)
     assert np.all(np.abs(g - r) <= 2.0 ** -7 * np.abs(r) + 1e-30)
@@ -84,7 +118,7 @@ def test_swiglu_thin_batch(orc):
     X, Wg, Wu, Wd, dY = make(M, d, f, 82)
     mlp, Wgu, Y, dX, dWgu, dWd = run_gpu(M, d, f, X, Wg, Wu, Wd, dY)
     b = synthetic.bits_u16
-    fwd = orc.swiglu_fwd(b(X), orc.interleave_gate_up(b(Wg), b(Wu)), b(Wd))
+    fwd = orc.swiglu_fwd(b(X), b(Wg), b(Wu), b(Wd))
     bwd = orc.swiglu_bwd_chain(b(dY), fwd)
     assert_close(u16(Y), fwd["Y"], "Y")
     assert_close(u16(dX), bwd["dX"], "dX")

@@ -131,16 +131,28 @@ def test_relu2_epilogues_match_elementwise_definitions(orc):
     assert amax_dh == np.float32(ref.float().abs().max().item())
 
 
-def test_relu2_derivative_by_finite_differences(orc):
-    """d/dx relu(x)^2 = 2 relu(x), away from the kink."""
+def test_relu2_backward_epilogue_is_the_derivative_of_relu2(orc):
+    """With the dgrad GEMM's value g = 1 exactly (one-hot codes of 1.0, unit
+    scales), the oracle's relu^2 backward epilogue returns d/dH relu(H)^2 at
+    every saved H: central differences of relu(x)^2 in fp64 at the same
+    points (away from the kink), to 1e-6."""
     rng = np.random.default_rng(17)
-    for x in rng.uniform(-3, 3, 200):
-        if abs(x) < 1e-3:
-            continue
-        eps = 1e-6
-        f = lambda t: max(t, 0.0) ** 2
-        fd = (f(x + eps) - f(x - eps)) / (2 * eps)
-        assert abs(fd - 2 * max(x, 0.0)) < 1e-6
+    M, N, K = 4, 64, 16
+    H = synthetic.bits_u16(torch.tensor(rng.uniform(-3, 3, (M, N)), dtype=torch.float32)
+                           .to(torch.bfloat16))
+    Hv = (H.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.min(np.abs(Hv)) > 1e-3
+    A = np.zeros((M, K), np.uint8)
+    B = np.zeros((N, K), np.uint8)
+    A[:, 0] = orc.fp8_encode(1.0, E5M2)
+    B[:, 0] = orc.fp8_encode(1.0, E4M3)
+    dH, _ = orc.gemm(A, E5M2, B, E4M3, np.float32(1.0), np.float32(1.0),
+                     epi=orc.EPI_RELU2_BWD, aux=H)
+    got = (dH.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    eps = 1e-6
+    f = lambda t: np.maximum(t, 0.0) ** 2
+    fd = (f(Hv + eps) - f(Hv - eps)) / (2 * eps)
+    assert np.all(np.abs(got - fd) <= 1e-6 * np.maximum(1.0, np.abs(fd)))
 
 
 def test_f64_chain_backward_by_finite_differences(orc):

@@ -45,9 +45,20 @@ def test_unit_rms_and_scale_invariance(orc):
     assert np.array_equal(orc.rmsnorm(R4, eps=0.0), orc.rmsnorm(Rb, eps=0.0))
 
 
-def test_fused_producer_is_norm_then_cast(orc):
-    R = synthetic.student_t3_bf16((48, 128), 62, 0)
-    w = synthetic.normal_bf16((128,), 1.0, 62, 1)
-    out = orc.rmsnorm_fp8_cast(synthetic.bits_u16(R), synthetic.bits_u16(w))
-    ref = orc.amax_scale_cast(out["X"], orc.E4M3)
-    assert out["amax"] == ref["amax"] and np.array_equal(out["q"], ref["q"])
+def test_fused_producer_closed_forms(orc):
+    """RMSNorm then the e4m3 cast, on rows whose outcome is known in closed
+    form: constant rows normalise to +-1, so amax = 1, scale = 448 and every
+    code is +-448 (0x7E / 0xFE); a one-hot row with weight 0.5 (d = 256)
+    becomes -8 at its one entry, so amax = 8, scale = 56 and the codes are
+    0xFE there and 0 elsewhere."""
+    R = np.zeros((3, 256), np.float32)
+    R[0], R[1], R[2] = 3.0, -0.25, 50.0
+    out = orc.rmsnorm_fp8_cast(bits(R), eps=0.0)
+    assert out["amax"] == 1.0 and out["scale"] == 448.0 and out["inv_scale"] == np.float32(1 / 448)
+    assert np.all(out["q"][0] == 0x7E) and np.all(out["q"][1] == 0xFE) and np.all(out["q"][2] == 0x7E)
+    R1 = np.zeros((1, 256), np.float32)
+    R1[0, 7] = -2.0
+    out = orc.rmsnorm_fp8_cast(bits(R1), bits(np.full(256, 0.5, np.float32)), eps=0.0)
+    assert out["amax"] == 8.0 and out["scale"] == 56.0
+    assert out["q"][0, 7] == 0xFE and np.count_nonzero(out["q"]) == 1
+    assert out["qT"][7, 0] == 0xFE

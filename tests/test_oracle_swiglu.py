@@ -1,6 +1,7 @@
 """Pins of the oracle's gated (SwiGLU) MLP variant: silu and its derivative
-by closed forms and identities, the fp64 chain's backward by finite
-differences, the gate/up interleaving, and the FP8 chain against fp64."""
+by closed forms and identities, dG and dU by finite differences of silu(G) U,
+the fp64 chain's backward by finite differences of its forward, the shared
+scale of the gate/up weight, and the FP8 chain against fp64."""
 import numpy as np
 import torch
 
@@ -20,28 +21,34 @@ def round_bf16(x):
     return np.ldexp(np.rint(m * 256.0), e - 8)
 
 
-def gu_of(G, U):
-    """Interleave G, U ([M x f] each) into the GU layout (blocks of 128)."""
-    M, f = G.shape
-    GU = np.empty((M, 2 * f), G.dtype)
-    for b in range(f // 128):
-        GU[:, 256 * b:256 * b + 128] = G[:, 128 * b:128 * b + 128]
-        GU[:, 256 * b + 128:256 * b + 256] = U[:, 128 * b:128 * b + 128]
-    return GU
-
-
 def test_silu_closed_forms_and_odd_identity(orc):
     G = np.zeros((2, 128), np.float32)
     G[0, :] = np.linspace(-6, 6, 128)
     U = np.ones((2, 128), np.float32)
-    h, _ = orc.swiglu_h(gu_of(bits(G), bits(U)))
+    h, amax_h = orc.swiglu_h(bits(G), bits(U))
     hv = vals(h)
     assert np.all(hv[1] == 0.0)                                   # silu(0) = 0
     g = vals(bits(G[0]))
     exact = g / (1.0 + np.exp(-g))
     assert np.array_equal(hv[0], round_bf16(exact))               # one rounding of x*sigma(x)
-    hn, _ = orc.swiglu_h(gu_of(bits(-G), bits(U)))
+    assert amax_h == np.float32(np.abs(hv).max())
+    hn, _ = orc.swiglu_h(bits(-G), bits(U))
     assert np.allclose(hv[0] - vals(hn)[0], g, atol=2 * 2.0 ** -8 * np.abs(g).max())
+
+
+def test_h_is_linear_in_u(orc):
+    """h = silu(G) U: doubling U doubles h exactly (a power-of-two scale), and a
+    negative U flips its sign; G and U are not interchangeable."""
+    rng = np.random.default_rng(35)
+    G = bits(rng.standard_normal((4, 64)) * 2)
+    U = bits(rng.standard_normal((4, 64)))
+    h, _ = orc.swiglu_h(G, U)
+    h2, _ = orc.swiglu_h(G, bits(vals(U) * 2.0))
+    hn, _ = orc.swiglu_h(G, bits(-vals(U)))
+    assert np.array_equal(vals(h2), 2.0 * vals(h))
+    assert np.array_equal(vals(hn), -vals(h))
+    hs, _ = orc.swiglu_h(U, G)
+    assert not np.array_equal(hs, h)
 
 
 def test_silu_derivative_at_zero_and_far_out(orc):
@@ -50,11 +57,28 @@ def test_silu_derivative_at_zero_and_far_out(orc):
     G[0, 1], G[0, 2] = 30.0, -30.0
     U = np.full((1, f), 3.0, np.float32)
     g = np.ones((1, f), np.float32)
-    dGU, _ = orc.swiglu_bwd(bits(g), gu_of(bits(G), bits(U)))
-    d = vals(dGU)
-    assert d[0, 0] == 1.5 and d[0, 128] == 0.0                    # silu'(0) = 1/2, silu(0) = 0
-    assert d[0, 1] == 3.0 and d[0, 129] == 30.0                   # silu'(30) ~ 1, silu(30) ~ 30
-    assert abs(d[0, 2]) < 1e-9 and abs(d[0, 130]) < 1e-9         # silu'(-30), silu(-30) ~ 0
+    dG, dU, amax_d = orc.swiglu_bwd(bits(g), bits(G), bits(U))
+    dg, du = vals(dG), vals(dU)
+    assert dg[0, 0] == 1.5 and du[0, 0] == 0.0                    # silu'(0) = 1/2, silu(0) = 0
+    assert dg[0, 1] == 3.0 and du[0, 1] == 30.0                   # silu'(30) ~ 1, silu(30) ~ 30
+    assert abs(dg[0, 2]) < 1e-9 and abs(du[0, 2]) < 1e-9         # silu'(-30), silu(-30) ~ 0
+    assert amax_d == np.float32(30.0)                             # the amax spans dG and dU
+
+
+def test_swiglu_bwd_by_finite_differences_of_h(orc):
+    """dG and dU are the partial derivatives of silu(G) U times g: central
+    differences of the fp64 silu(G) U at each point, within bf16 rounding."""
+    rng = np.random.default_rng(36)
+    G = vals(bits(rng.standard_normal((3, 40)) * 3))
+    U = vals(bits(rng.standard_normal((3, 40))))
+    g = vals(bits(rng.standard_normal((3, 40))))
+    dG, dU, _ = orc.swiglu_bwd(bits(g), bits(G), bits(U))
+    h = lambda a, b: a / (1.0 + np.exp(-a)) * b
+    eps = 1e-6
+    fdG = g * (h(G + eps, U) - h(G - eps, U)) / (2 * eps)
+    fdU = g * (h(G, U + eps) - h(G, U - eps)) / (2 * eps)
+    assert np.all(np.abs(vals(dG) - fdG) <= 2.0 ** -8 * np.abs(fdG) + 1e-8)
+    assert np.all(np.abs(vals(dU) - fdU) <= 2.0 ** -8 * np.abs(fdU) + 1e-8)
 
 
 def test_swiglu_f64_backward_by_finite_differences(orc):
@@ -78,13 +102,16 @@ def test_swiglu_f64_backward_by_finite_differences(orc):
             assert abs(fd - out[key][idx]) <= 1e-6 * max(1.0, abs(fd)), (key, idx)
 
 
-def test_interleave_round_trip(orc):
-    Wg = np.arange(256 * 3).reshape(256, 3)
-    Wu = -np.arange(256 * 3).reshape(256, 3)
-    Wgu = orc.interleave_gate_up(Wg, Wu)
-    assert np.array_equal(Wgu[0:128], Wg[0:128]) and np.array_equal(Wgu[128:256], Wu[0:128])
-    g2, u2 = orc.deinterleave_gate_up(Wgu)
-    assert np.array_equal(g2, Wg) and np.array_equal(u2, Wu)
+def test_joint_cast_shares_one_scale(orc):
+    """Gate and up weights are quantised as one tensor: the amax is the larger
+    of the two, and each is cast at that one scale."""
+    Wg = synthetic.normal_bf16((128, 64), 0.02, 34, 0)
+    Wu = synthetic.normal_bf16((128, 64), 0.5, 34, 1)
+    b = synthetic.bits_u16
+    j = orc.amax_scale_cast_joint([b(Wg), b(Wu)], orc.E4M3)
+    both = orc.amax_scale_cast(np.vstack([b(Wg), b(Wu)]), orc.E4M3)
+    assert j["amax"] == both["amax"] == orc.amax(b(Wu))
+    assert np.array_equal(np.vstack(j["q"]), both["q"])
 
 
 def test_fp8_swiglu_chain_within_fp8_error_of_f64(orc):
@@ -95,12 +122,13 @@ def test_fp8_swiglu_chain_within_fp8_error_of_f64(orc):
     Wd = synthetic.normal_bf16((d, f), 0.05, 33, 3)
     dY = synthetic.normal_bf16((M, d), 1e-3, 33, 4)
     b = lambda t: synthetic.bits_u16(t)
-    fwd = orc.swiglu_fwd(b(X), orc.interleave_gate_up(b(Wg), b(Wu)), b(Wd))
+    fwd = orc.swiglu_fwd(b(X), b(Wg), b(Wu), b(Wd))
     bwd = orc.swiglu_bwd_chain(b(dY), fwd)
     ref = orc.swiglu_f64(*(t.double().numpy() for t in (X, Wg, Wu, Wd, dY)))
-    dWg, dWu = orc.deinterleave_gate_up(bwd["dW_gu"])
     rel = lambda got, r: np.linalg.norm(vals(got) - r) / np.linalg.norm(r)
     assert rel(fwd["Y"], ref["Y"]) < 0.1
     assert rel(bwd["dX"], ref["dX"]) < 0.15
-    assert rel(dWg, ref["dWg"]) < 0.15 and rel(dWu, ref["dWu"]) < 0.15
+    assert rel(bwd["dW_gate"], ref["dWg"]) < 0.15 and rel(bwd["dW_up"], ref["dWu"]) < 0.15
     assert rel(bwd["dW_down"], ref["dWd"]) < 0.15
+    # a swapped gate/up pair is far outside that error
+    assert rel(bwd["dW_up"], ref["dWg"]) > 0.5
