@@ -233,6 +233,32 @@ class LmHeadCE:
         tail = (n + 255) // 256 * 256
         return self.workspace[-tail:][:n].view(torch.float32)
 
+    def view(self, name):
+        """Workspace views after a call (library layout, each part rounded up
+        to 256 bytes): "scales" [3 x 4] {amax, scale, inv_scale, 0} of X, W and
+        the last chunk's dlogits; "Wq" [V x d]; and the last chunk's "Xq"
+        [C x d], "dlogits" (bf16, written over its logits) [C x V] and "dLq"
+        [C x V], where C is that chunk's row count."""
+        M, d, V, C = self.M, self.d, self.V, self.chunk
+        r256 = lambda n: (n + 255) // 256 * 256
+        rows = M - (M - 1) // C * C if M else 0
+        off = {"scales": 0}
+        off["Wq"] = r256(64)
+        off["Xq"] = off["Wq"] + r256(V * d)
+        off["dlogits"] = off["Xq"] + r256(C * d)
+        off["dLq"] = off["dlogits"] + r256(C * V * 2)
+        o = off[name]
+        ws = self.workspace
+        if name == "scales":
+            return ws[o:o + 48].view(torch.float32).view(3, 4)
+        if name == "Wq":
+            return ws[o:o + V * d].view(V, d)
+        if name == "Xq":
+            return ws[o:o + rows * d].view(rows, d)
+        if name == "dlogits":
+            return ws[o:o + rows * V * 2].view(torch.bfloat16).view(rows, V)
+        return ws[o:o + rows * V].view(rows, V)
+
 
 class Linear:
     """Buffers of one plain FP8 linear Y = X W^T with X [M x K], W [N x K]:

@@ -3,12 +3,11 @@
 //
 // lm_relu2_mlp_bwd needs a caller-provided scratch workspace (the GEMMs'
 // split-K scratch, the e5m2 codes of dY and dH, the bf16 dH and two scale
-// blocks).  Some callers have no way to provide one: code that runs while a stream is being
-// captured into a CUDA graph (cudaMalloc is not allowed there), plugins whose
-// host framework owns the whole device memory pool and forbids allocation in
-// its execute callback, and latency-critical loops that cannot afford the
-// device-wide synchronisation cudaMalloc/cudaFree may cause.  For them this
-// file keeps the workspace in a fixed device array that the library owns.
+// blocks).  Some callers have no way to provide one: plugins whose host
+// framework owns the whole device memory pool and forbids allocation in its
+// execute callback, and latency-critical loops that cannot afford the
+// device-wide synchronisation that cudaMalloc/cudaFree may cause.  For them
+// this file keeps the workspace in a fixed device array that the library owns.
 //
 // Limits and sharing:
 //  - the array holds kScratchBytes (64 MiB); shapes whose workspace
@@ -20,8 +19,10 @@
 //    overlaps on the GPU (different streams, no ordering between them) race
 //    and corrupt each other's results.  Calls on one stream are safe;
 //  - the array keeps whatever the previous call left in it; the backward
-//    zeroes the only part that must start at zero (its amax accumulators) on
-//    every call.
+//    zeroes what must start at zero (its amax accumulators and the split-K
+//    flags) on every call.
+#include <atomic>
+
 #include "lm_internal.h"
 
 namespace {
@@ -33,19 +34,21 @@ constexpr size_t kScratchBytes = size_t(64) << 20;
 static __device__ __align__(256) unsigned char g_mlp_bwd_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {};
+// Device address of the array per device, looked up on the first call made
+// with that device current.  Host threads may race on the first lookup; each
+// stores the same address, and the atomics keep that well defined.  The
+// address is not valid after cudaDeviceReset on that device.
+std::atomic<void*> g_scratch_ptr[kMaxDevices];
 
-// Device address of the scratch on the current device, looked up once per
-// device (with that device current) and cached.  nullptr on failure.
+// Device address of the scratch on the current device.  nullptr on failure.
 void* scratch_address() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_mlp_bwd_scratch) != cudaSuccess || !p) return nullptr;
-        g_scratch_ptr[dev] = p;
-    }
-    return g_scratch_ptr[dev];
+    void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    if (cudaGetSymbolAddress(&p, g_mlp_bwd_scratch) != cudaSuccess || !p) return nullptr;
+    g_scratch_ptr[dev].store(p, std::memory_order_release);
+    return p;
 }
 
 }  // namespace

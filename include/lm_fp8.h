@@ -270,16 +270,20 @@ LM_API lm_status lm_relu2_mlp_bwd(const void* dY, const lm_mlp_saved* saved, int
 /*
  * relu^2 MLP backward that allocates nothing (no counterpart on the pages:
  * the method itself says nothing about memory ownership).  For callers that
- * cannot hand the library a workspace -- code running during CUDA graph
- * capture, where cudaMalloc is not allowed; plugins whose host framework owns
- * all device memory and forbids allocation in its execute callback; loops that
+ * cannot hand the library a workspace: plugins whose host framework owns all
+ * device memory and forbids allocation in its execute callback, and loops that
  * cannot absorb the device-wide synchronisation of cudaMalloc/cudaFree.
  * Computes exactly what lm_relu2_mlp_bwd computes, using as its workspace a
  * 64 MiB device array owned by the library (lm_relu2_mlp_bwd_noalloc_max_bytes).
- *  - Shapes whose lm_relu2_mlp_workspace_size exceeds that size return
- *    LM_ERR_UNSUPPORTED_SHAPE with nothing enqueued.
+ *  - A shape fits when lm_relu2_mlp_workspace_size(M, d, f) is at most that
+ *    size: the GEMMs' split-K scratch (lm_fp8_gemm_workspace_size, about
+ *    32 MiB) plus M*d + 3*M*f bytes, each part rounded up to 256 bytes.  At
+ *    the model's d = 3072, f = 12288 that is M <= 832 tokens (M = 512 fits,
+ *    M = 1024 does not); the 256 x 256 x 1024 block fits.  Larger shapes
+ *    return LM_ERR_UNSUPPORTED_SHAPE with nothing enqueued.
  *  - The first call on a device looks up the array's device address with that
  *    device current; make that first call before any stream capture begins.
+ *    The looked-up address is not valid after cudaDeviceReset on that device.
  *    Every GPU that loads the array keeps it until the process exits.
  *  - All calls on a device share the array, which keeps the previous call's
  *    contents (the backward re-zeroes what must start at zero).  Calls whose

@@ -59,6 +59,15 @@ def assert_close(got_bits, ref_bits, what="", elem_rel=ELEM_REL):
         assert np.linalg.norm(g - r) / nr <= NORM_REL, f"{what}: normwise {np.linalg.norm(g - r) / nr:.3e}"
 
 
+def cast_ref(orc, bits, fmt, relu2_input=False, amax_in=None):
+    """The oracle's dynamic cast of a whole tensor, row-major codes only:
+    dict(amax, scale, inv_scale, q)."""
+    a = orc.amax(bits, relu2_input) if amax_in is None else np.float32(amax_in)
+    s, inv = orc.scale(a, fmt)
+    q, _ = orc.cast(bits, fmt, s, relu2_input, want_qT=False)
+    return dict(amax=a, scale=s, inv_scale=inv, q=q)
+
+
 def bf16_neighbours(bits):
     """The bf16 values one ulp below and above each value (bits, same shape)."""
     b = np.asarray(bits, np.uint16).astype(np.int32)

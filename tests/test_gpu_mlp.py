@@ -14,7 +14,7 @@ import pytest
 import torch
 
 from fp8_gemms_b200 import synthetic
-from gpu_util import ELEM_REL_RELU2_BWD, assert_close, f32, u8, u16
+from gpu_util import ELEM_REL_RELU2_BWD, assert_close, cast_ref, f32, u8, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -45,12 +45,14 @@ def T(codes):
     return np.ascontiguousarray(codes.T)
 
 
-def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None):
-    """rows: sample of output rows to check for the M x * GEMMs (None = all)."""
+def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None, wd_rows=None, wu_rows=None):
+    """rows: sample of output rows to check for the M x * GEMMs (None = all);
+    wd_rows / wu_rows: rows of dW_down / dW_up to check (default: all when rows
+    is None, else 24 evenly spaced rows)."""
     sc = mlp.view("scales").cpu().numpy()
     # casts of the inputs: bit-exact
     for name, key, si in [("X", "Xq", 0), ("W_up", "Wuq", 1), ("W_down", "Wdq", 2)]:
-        ref = orc.amax_scale_cast(synthetic.bits_u16(t[name]), E4M3)
+        ref = cast_ref(orc, synthetic.bits_u16(t[name]), E4M3)
         assert sc[si, 0] == ref["amax"] and sc[si, 1] == ref["scale"] and sc[si, 2] == ref["inv_scale"], name
         assert np.array_equal(u8(mlp.view(key)), ref["q"]), name
     Xq, Wuq, Wdq = u8(mlp.view("Xq")), u8(mlp.view("Wuq")), u8(mlp.view("Wdq"))
@@ -72,7 +74,7 @@ def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None):
     if dX is None:
         return
     g = mlp.workspace_view("scales").cpu().numpy()
-    ref = orc.amax_scale_cast(synthetic.bits_u16(t["dY"]), E5M2)
+    ref = cast_ref(orc, synthetic.bits_u16(t["dY"]), E5M2)
     assert g[0, 0] == ref["amax"] and g[0, 1] == ref["scale"] and g[0, 2] == ref["inv_scale"]
     dYq = u8(mlp.workspace_view("dYq"))
     assert np.array_equal(dYq, ref["q"])
@@ -88,12 +90,16 @@ def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None):
     dHq_ref, _ = orc.cast(dH, E5M2, s_dh, want_qT=False)
     dHq = u8(mlp.workspace_view("dHq"))
     assert np.array_equal(dHq, dHq_ref)
-    wrows = None if rows is None else np.arange(0, dWd.shape[0], max(1, dWd.shape[0] // 24))
+    wrows = wd_rows
+    if wrows is None and rows is not None:
+        wrows = np.arange(0, dWd.shape[0], max(1, dWd.shape[0] // 24))
     ref_dWd, _ = orc.gemm(T(dYq), E5M2, T(hq), E4M3, g[0, 2], sc[3, 2], rows=wrows)
     assert_close(u16(dWd) if wrows is None else u16(dWd)[wrows], ref_dWd, "dW_down")
     ref_dX, _ = orc.gemm(dHq, E5M2, T(Wuq), E4M3, g[1, 2], sc[1, 2], rows=rows)
     assert_close(u16(dX) if rows is None else u16(dX)[rows], ref_dX, "dX")
-    urows = None if rows is None else np.arange(0, dWu.shape[0], max(1, dWu.shape[0] // 24))
+    urows = wu_rows
+    if urows is None and rows is not None:
+        urows = np.arange(0, dWu.shape[0], max(1, dWu.shape[0] // 24))
     ref_dWu, _ = orc.gemm(T(dHq), E5M2, T(Xq), E4M3, g[1, 2], sc[0, 2], rows=urows)
     assert_close(u16(dWu) if urows is None else u16(dWu)[urows], ref_dWu, "dW_up")
 
@@ -153,3 +159,14 @@ def test_full_size_mlp_sampled(orc, api):
     rows = np.concatenate([np.arange(0, 16), np.arange(w.M - 16, w.M),
                            np.random.default_rng(0).choice(w.M, 16, replace=False)])
     check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=np.sort(rows))
+
+
+@pytest.mark.slow
+def test_full_size_mlp_forward_only_sampled(orc, api):
+    """The 3.8B-shape forward alone (X [16384 x 3072] = 16 sequences x 1024
+    tokens): up GEMM with the relu^2 epilogue and its amax, the cast of h,
+    the down GEMM; casts bit-exact over whole tensors, GEMMs on sampled rows."""
+    w = synthetic.MLP_FWD
+    t, mlp, Y, *_ = run_chain(api, w)
+    rows = np.sort(np.random.default_rng(2).choice(w.M, 32, replace=False))
+    check_stagewise(orc, mlp, t, Y, None, None, None, rows=rows)

@@ -1,15 +1,17 @@
 """The allocation-free relu^2 MLP backward (lm_relu2_mlp_bwd_noalloc).
 
-It exists for callers that cannot allocate device memory -- during CUDA graph
-capture, inside a host framework that owns the memory pool, or where the
-synchronisation of cudaMalloc is unaffordable -- and keeps its workspace in a
-fixed array owned by the library.  It must produce what the allocating
-backward (lm_relu2_mlp_bwd) produces, on consecutive calls that reuse that
-array, and must reject shapes whose workspace does not fit.
+It exists for callers that cannot allocate device memory -- plugins inside a
+host framework that owns the memory pool, or loops that cannot afford the
+synchronisation of cudaMalloc -- and keeps its workspace in a fixed array
+owned by the library.  It runs the same kernels with the same split plan as
+the allocating backward (lm_relu2_mlp_bwd), so its outputs must be
+bit-identical to that backward's on the same inputs, on consecutive calls that
+reuse the array; and it must reject shapes whose workspace does not fit.
 
 This file is collected last on purpose and sets up everything it needs, so it
 passes alone in a fresh process as well as after the other tests.
 """
+import numpy as np
 import pytest
 import torch
 
@@ -19,7 +21,11 @@ from gpu_util import assert_close, u16
 pytestmark = pytest.mark.gpu
 
 
-def test_noalloc_backward_matches_allocating_backward_on_two_calls():
+def test_noalloc_backward_matches_allocating_backward_on_two_calls(orc):
+    """Two calls in a row through the C ABI.  The second uses dY / 4, so its
+    amax, scales and every code differ from the first's: state the first call
+    left in the shared array (amax accumulators, split-K flags, dH codes) would
+    show as a mismatch."""
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     from fp8_gemms_b200 import _lib, api
 
@@ -28,19 +34,25 @@ def test_noalloc_backward_matches_allocating_backward_on_two_calls():
     dev = {k: v.cuda() for k, v in t.items()}
     mlp = api.Relu2Mlp(w.M, w.d, w.f)
     mlp.forward(dev["X"], dev["W_up"], dev["W_down"])
-    ref_dX, ref_dWu, ref_dWd = mlp.backward(dev["dY"])      # caller-provided workspace
     torch.cuda.synchronize()
 
-    for call in range(2):                                    # the array is reused as-is
+    for call, dY in enumerate([dev["dY"], dev["dY"] * 0.25]):
+        ref_dX, ref_dWu, ref_dWd = mlp.backward(dY)          # caller-provided workspace
         dX = torch.full_like(ref_dX, float("nan"))
         dWu = torch.full_like(ref_dWu, float("nan"))
         dWd = torch.full_like(ref_dWd, float("nan"))
-        _lib.lm_relu2_mlp_bwd_noalloc(dev["dY"], mlp.saved, dX, dWu, dWd)
+        _lib.lm_relu2_mlp_bwd_noalloc(dY, mlp.saved, dX, dWu, dWd)
         torch.cuda.synchronize()
         assert _lib.lm_get_error()[0] == 0
-        assert_close(u16(dX), u16(ref_dX), f"dX, call {call}")
-        assert_close(u16(dWu), u16(ref_dWu), f"dW_up, call {call}")
-        assert_close(u16(dWd), u16(ref_dWd), f"dW_down, call {call}")
+        assert torch.equal(dX, ref_dX), f"dX, call {call}"
+        assert torch.equal(dWu, ref_dWu), f"dW_up, call {call}"
+        assert torch.equal(dWd, ref_dWd), f"dW_down, call {call}"
+        if call == 0:
+            b = {k: synthetic.bits_u16(v) for k, v in t.items()}
+            bwd = orc.mlp_bwd(b["dY"], orc.mlp_fwd(b["X"], b["W_up"], b["W_down"]))
+            assert_close(u16(dX), bwd["dX"], "dX vs oracle")
+            assert_close(u16(dWu), bwd["dW_up"], "dW_up vs oracle")
+            assert_close(u16(dWd), bwd["dW_down"], "dW_down vs oracle")
 
 
 def test_noalloc_backward_rejects_shapes_beyond_its_array():
@@ -49,7 +61,8 @@ def test_noalloc_backward_rejects_shapes_beyond_its_array():
 
     cap = _lib.lib.lm_relu2_mlp_bwd_noalloc_max_bytes()
     assert cap == 64 << 20
-    M, d, f = 16384, 3072, 12288                              # needs ~0.9 GB of workspace
+    assert _lib.lm_relu2_mlp_workspace_size(832, 3072, 12288) <= cap
+    M, d, f = 848, 3072, 12288                                # the first M that does not fit
     assert _lib.lm_relu2_mlp_workspace_size(M, d, f) > cap
     s = _lib.MlpSaved()
     status = _lib.lib.lm_relu2_mlp_bwd_noalloc(None, s, M, d, f, None, None, None, None)
