@@ -14,16 +14,21 @@ is no data-path collective and scaling is weak.
 
 Timing: CUDA events on the launching stream around each step, L2 flushed
 (a 256 MiB write) before every timed step, W untimed warm-up steps, max over
-ranks.  SM clocks are sampled with nvidia-smi during the timed region.
+ranks.  SM clocks and clock-event reasons are sampled in-process through NVML
+every few milliseconds; only samples taken inside the timed region count.
+
+Besides the headline (the fwd + bwd block at M = 16384), the same JSON line
+carries the other GEMM sets of the little-lm model under "configs", each timed
+the same way with its own oracle sample: the MLP forward alone (M = 16384),
+the attention projections + LM head (M = 8192) and the 28-layer stack's
+linear-layer set (M = 16384, t3 activations).
 """
 import argparse
 import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import threading
 import time
 
@@ -38,7 +43,7 @@ DENSE_FP8_PEAK_TFLOPS = 4500.0                 # public B200 dense FP8 figure
 PAGES_FP8_PEAK_TFLOPS = 4190.0                 # the dense FP8 peak the pages' MFU figure implies
 NOMINAL_FP8_OVER_BF16 = 2.0                    # 4.5 / 2.25 PFLOP/s dense
 WORKLOAD = "relu2 MLP fwd+dgrad+wgrad M=16384 d=3072 f=12288"
-LAUNCHES_PER_STEP = 12                         # kernels of ours per fwd+bwd: "acgcgacggcgg"
+LAUNCHES_PER_STEP = 11                         # kernels of ours per fwd+bwd: "acgcgacgggg"
 
 # DRAM traffic of one GEMM launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum), valid only for the kernel source it was taken on;
@@ -57,6 +62,10 @@ def parse_args():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=256)
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the other GEMM sets (MLP forward, attention + head, stack)")
+    p.add_argument("--config-steps", type=int, default=20)
+    p.add_argument("--stack-steps", type=int, default=3)
     return p.parse_args()
 
 
@@ -79,55 +88,87 @@ def read_peaks():
 
 
 # ----------------------------------------------------------------- clocks
-class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, gpu_id):
-        self.gpu = gpu_id  # nvidia-smi -i accepts an index or a GPU UUID
-        self.proc = None
-        self.out = None
+
+class ClockSampler:
+    """Samples the SM clock, power and clock-event reasons of one GPU through
+    NVML from a host thread every ~2 ms.  region() marks the timed region; the
+    summary uses only the samples taken inside it."""
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.samples = []   # (t, sm_mhz, power_w, reasons)
+        self.regions = []
+        self._stop = threading.Event()
+        self.h = None
+        self.max_mhz = None
 
     def __enter__(self):
-        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.gpu), "-lms", "50"], stdout=self.out, stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
-        time.sleep(0.15)
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.h = None
+        if self.h is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
         return self
 
-    def __exit__(self, *exc):
-        if self.proc:
-            self.proc.terminate()
+    def _run(self):
+        nv, h = self.nv, self.h
+        while not self._stop.is_set():
             try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.perf_counter(), sm, pw, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
-    def summary(self):
-        rows = []
-        try:
-            with open(self.out.name) as f:
-                for line in f:
-                    parts = [x.strip() for x in line.split(",")]
-                    if len(parts) == 9:
-                        rows.append(parts)
-        finally:
-            os.unlink(self.out.name)
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.h is not None:
+            self.thread.join(timeout=5)
+            try:
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
+
+    class _Region:
+        def __init__(self, owner):
+            self.owner = owner
+
+        def __enter__(self):
+            self.t0 = time.perf_counter()
+
+        def __exit__(self, *exc):
+            self.owner.regions.append((self.t0, time.perf_counter()))
+
+    def region(self):
+        return ClockSampler._Region(self)
+
+    def summary(self, region=0):
+        if self.h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"],
+                    "samples": 0, "source": "nvml"}
+        t0, t1 = self.regions[region]
+        rows = [r for r in self.samples if t0 <= r[0] <= t1]
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
-        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(pw) if pw else None}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"],
+                    "samples": 0, "source": "nvml"}
+        sm = [r[1] for r in rows]
+        reasons = sorted({n for r in rows for n, b in REASON_BITS.items() if r[3] & b})
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_p90_mhz":
+                sorted(sm)[int(0.9 * (len(sm) - 1))], "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(rows),
+                "region_s": round(t1 - t0, 4), "power_w_max": max(r[2] for r in rows),
+                "source": "nvml, in-process, ~2 ms period, samples inside the timed region only"}
 
 
 # ------------------------------------------------------------ GPU pieces
@@ -154,13 +195,16 @@ def job_tflops(world, steps, flops_per_step, total_ms):
     return world * steps * flops_per_step / (total_ms * 1e-3) / 1e12
 
 
-# algorithmic bytes of the casts of one step (X, W_up, W_down, h, dY, dH):
-# full cast (amax pass + cast pass) = 2 B amax read + 2 B read + 1 B codes per
-# element; a cast whose amax came from a GEMM epilogue = 2 B read + 1 B codes.
+# algorithmic bytes of the cast launches of one step: a full cast (amax pass +
+# cast pass) moves 2 B (amax read) + 2 B (read) + 1 B (codes) per element; a
+# cast whose amax came from a GEMM epilogue 2 + 1 B.  The launches: the amax
+# of X, W_up and W_down; the casts of X and W_up; the cast of h; the amax and
+# cast of dY.  W_down's codes (3 B/element after its amax) and dH's cast run
+# in side warps of the up GEMM and of the dW_down GEMM, inside those launches.
 # Only row-major codes are written: the backward's GEMMs read them MN-major.
 def cast_bytes():
     Md, fd, Mf = M_TOK * D_MODEL, D_FF * D_MODEL, M_TOK * D_FF
-    return [5 * Md, 5 * fd, 5 * fd, 3 * Mf, 5 * Md, 3 * Mf]
+    return [5 * Md, 5 * fd, 2 * fd, 3 * Mf, 5 * Md]
 
 
 def src_sha(path):
@@ -213,15 +257,16 @@ def run_gpu(args):
     timers = [lib.KernelTimer(2 * LAUNCHES_PER_STEP) for _ in range(K)]
     barrier()
     props = torch.cuda.get_device_properties(device)
-    smi_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
-    with ClockSampler(smi_id) as clk:
-        for k in range(K):
-            flush.fill_(k & 0xFF)
-            starts[k].record()
-            with timers[k]:
-                step()
-            ends[k].record()
-        barrier()
+    uuid = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else ""
+    with ClockSampler(uuid) as clk:
+        with clk.region():
+            for k in range(K):
+                flush.fill_(k & 0xFF)
+                starts[k].record()
+                with timers[k]:
+                    step()
+                ends[k].record()
+            barrier()
     clocks = clk.summary()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), world, device)
@@ -323,7 +368,11 @@ def run_gpu(args):
     clock_peak = (world * props.multi_processor_count * 16384 * clocks["sm_mhz"] * 1e6 / 1e12
                   if clocks.get("sm_mhz") else None)
     e2e_value = job_tflops(world, Ke, STEP_FLOPS, e2e_ms)
-    fp8_peak = peaks["bf16_sus"] * NOMINAL_FP8_OVER_BF16
+    # The timed region is well under a second, so the kernel is compared with
+    # the burst GEMM peak; the sustained (seconds-long, power-capped) one is
+    # reported beside it.
+    fp8_peak = peaks["bf16"] * NOMINAL_FP8_OVER_BF16
+    fp8_peak_sus = peaks["bf16_sus"] * NOMINAL_FP8_OVER_BF16
     achieved = GEMM_FLOPS / (gemm_avg_ms * 1e-3) / 1e12
     traffic = None
     gemm_src = os.path.join(ROOT, "fp8_gemms_b200", "csrc", "lm_gemm.cu")
@@ -331,6 +380,8 @@ def run_gpu(args):
         traffic = GEMM_TRAFFIC["bytes_per_launch"]
     cb = cast_bytes()
     cast_gbs = sum(cb) / (sum(cast_ms) * 1e-3) / 1e9
+    mhz = clocks.get("sm_mhz")
+    configs = run_configs(args, device, world, flush, host, dev, mlp, peaks, rank)
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -354,17 +405,23 @@ def run_gpu(args):
         "roofline": {"bound": "tensor", "kernel": "gemm_fp8_pair_kernel (tcgen05, CTA pairs)",
                      "achieved": round(achieved, 2), "peak": round(fp8_peak, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
-                     "peak_source": f"{peaks['src']} bf16 sustained {peaks['bf16_sus']} x "
-                                    f"nominal fp8/bf16 ratio {NOMINAL_FP8_OVER_BF16}",
+                     "peak_source": f"{peaks['src']} bf16 burst {peaks['bf16']} x nominal "
+                                    f"fp8/bf16 ratio {NOMINAL_FP8_OVER_BF16} (timed region "
+                                    f"under a second)",
+                     "peak_sustained": round(fp8_peak_sus, 1),
+                     "frac_of_sustained": round(achieved / fp8_peak_sus, 4),
                      "flops_per_launch": GEMM_FLOPS, "avg_launch_ms": round(gemm_avg_ms, 4),
+                     "avg_launch_kcycles": round(gemm_avg_ms * mhz, 1) if mhz else None,
                      "traffic": traffic},
         "cast_kernels": {"achieved_gbs": round(cast_gbs, 1), "peak_gbs": peaks["hbm"],
                          "frac": round(cast_gbs / peaks["hbm"], 4),
+                         "frac_of_8tbs": round(cast_gbs / 8000.0, 4),
                          "algorithmic_bytes_per_step": sum(cb),
                          "ms_per_step": round(sum(cast_ms), 4)},
         "gemm_ms_per_step": round(sum(gemm_ms), 4),
         "launch_sequence": kinds,
         "per_launch_ms": [round(a, 4) for a in avg],
+        "per_gemm_kcycles": [round(a * mhz, 1) for a in gemm_ms] if mhz else None,
         "lead_in_ms_per_step": round(statistics.mean(lead_ms), 4),
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "steps": Ke,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -379,6 +436,7 @@ def run_gpu(args):
                    "micro-batch of an optimizer step"},
         "gpu_launches": K * LAUNCHES_PER_STEP,
         "clocks": clocks,
+        "configs": configs,
     }
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(host, args.cpu_sample_tokens)
@@ -387,6 +445,193 @@ def run_gpu(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------- the other GEMM sets
+def time_steps(step, K, W, flush, cap):
+    """W warm-up steps, then K steps each preceded by an L2 flush and timed
+    with CUDA events.  One more step runs with the library's launch events,
+    for the split between GEMM launches and the rest; a host-side gap before
+    a launch counts towards that launch, so where the host issues launches
+    more slowly than the GPU runs them the split is of the instrumented
+    eager step, not of device time alone.  Returns (ms per step, GEMM ms,
+    other ms) of that step."""
+    import torch
+    from fp8_gemms_b200 import _lib as lib
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for k in range(K):
+        flush.fill_(k & 0xFF)
+        ev[k][0].record()
+        step()
+        ev[k][1].record()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    flush.fill_(0)
+    t = lib.KernelTimer(cap)
+    end = torch.cuda.Event(enable_timing=True)
+    with t:
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    d = t.durations_ms(end)
+    g = sum(x for x, kd in zip(d, t.kinds) if kd == "g")
+    return ms, g, sum(d) - g
+
+
+def time_graph(step, K, flush):
+    """The same step captured once into a CUDA graph and replayed K times (L2
+    flushed before each replay): device time without host launch gaps."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            step()
+    torch.cuda.current_stream().wait_stream(s)
+    g.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for k in range(K):
+        flush.fill_(k & 0xFF)
+        ev[k][0].record()
+        g.replay()
+        ev[k][1].record()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    del g
+    return ms
+
+
+def config_entry(name, flops, cast_bytes_total, ms, gemm_ms, other_ms, peaks, world):
+    """Throughput and roofline of one GEMM set: the roofline time is the
+    GEMMs' FLOPs at the dense FP8 peak plus the casts' algorithmic bytes at
+    HBM bandwidth (each kernel bound by the slower of the two, which is FLOPs
+    for every GEMM and bytes for every cast here)."""
+    t_nom = flops / 4.5e15 + cast_bytes_total / 8e12
+    t_meas = (flops / (peaks["bf16"] * NOMINAL_FP8_OVER_BF16 * 1e12) +
+              cast_bytes_total / (peaks["hbm"] * 1e9))
+    tflops = world * flops / (ms * 1e-3) / 1e12
+    return {"workload": name, "ms_per_step": round(ms, 4), "tflops": round(tflops, 2),
+            "flops_per_step": flops, "pct_of_dense_fp8_peak":
+            round(100.0 * tflops / (world * DENSE_FP8_PEAK_TFLOPS), 2),
+            "instrumented_step": {"gemm_ms": round(gemm_ms, 4), "other_ms": round(other_ms, 4)},
+            "cast_bytes_per_step": cast_bytes_total,
+            "roofline": {"ms_nominal": round(t_nom * 1e3, 4), "frac_nominal":
+                         round(t_nom * 1e3 / ms, 4), "ms_measured_peaks":
+                         round(t_meas * 1e3, 4), "frac_measured_peaks":
+                         round(t_meas * 1e3 / ms, 4),
+                         "how": "GEMM FLOPs at 4.5 PFLOP/s (nominal) or 2 x the measured "
+                                "bf16 burst (measured) + cast bytes at 8 TB/s or the "
+                                "measured copy bandwidth"}}
+
+
+def add_graph(entry, flops, graph_ms, world):
+    tf = world * flops / (graph_ms * 1e-3) / 1e12
+    entry["graph_replay"] = {"ms_per_step": round(graph_ms, 4), "tflops": round(tf, 2),
+                             "pct_of_dense_fp8_peak":
+                             round(100.0 * tf / (world * DENSE_FP8_PEAK_TFLOPS), 2)}
+
+
+def linear_cast_bytes(M, N, K):
+    return 5 * (M * K + N * K + M * N)   # full casts of X, W and dY
+
+
+def mlp_cast_bytes(M, d, f, backward=True):
+    b = 5 * M * d + 10 * f * d + 3 * M * f           # X, W_up, W_down, h
+    return b + (5 * M * d + 3 * M * f if backward else 0)   # dY, dH
+
+
+def run_configs(args, device, world, flush, host, dev, mlp, peaks, rank):
+    """Configs 2, 4 and 5 of the little-lm GEMM sets, each timed like the
+    headline, with the oracle's sample time on rank 0."""
+    import torch
+    from fp8_gemms_b200 import api, synthetic
+    if args.no_configs:
+        return None
+    out = {}
+    K = args.config_steps
+    # -- the MLP forward alone at M = 16384 (16 x 1024 tokens)
+    fl = 2 * GEMM_FLOPS
+    ms, g, o = time_steps(lambda: mlp.forward(dev["X"], dev["W_up"], dev["W_down"], Y=dev["Y"]),
+                          K, 3, flush, 16)
+    ms = max_over_ranks(ms, world, device)
+    out["mlp_fwd_M16384"] = config_entry(synthetic.MLP_FWD.name, fl,
+                                         mlp_cast_bytes(M_TOK, D_MODEL, D_FF, False), ms, g, o,
+                                         peaks, world)
+    # -- attention projections + LM head at M = 8192
+    w = synthetic.ATTN_HEAD
+    items = []
+    for i, (name, n, k) in enumerate(w.linears):
+        t = w.tensors(i, device=device)
+        lin = api.Linear(w.M, k, n, device=device)
+        bufs = (torch.empty(w.M, n, dtype=torch.bfloat16, device=device),
+                torch.empty(w.M, k, dtype=torch.bfloat16, device=device),
+                torch.empty(n, k, dtype=torch.bfloat16, device=device))
+        items.append((lin, t, bufs))
+
+    def step4():
+        for lin, t, (Y, dX, dW) in items:
+            lin.forward(t["X"], t["W"], Y=Y)
+            lin.backward(t["dY"], dX=dX, dW=dW)
+
+    ms, g, o = time_steps(step4, K, 3, flush, 64)
+    ms = max_over_ranks(ms, world, device)
+    cb = sum(linear_cast_bytes(w.M, n, k) for _, n, k in w.linears)
+    out["attn_lmhead_M8192"] = config_entry(w.name, w.flops, cb, ms, g, o, peaks, world)
+    add_graph(out["attn_lmhead_M8192"], w.flops,
+              max_over_ranks(time_graph(step4, K, flush), world, device), world)
+    del items
+    torch.cuda.empty_cache()
+    # -- the 28-layer stack: per layer Q, K, V, O and the relu^2 MLP, each layer
+    # with its own seeded weights and t3 activations (drawn on the device)
+    layers = []
+    for layer in range(synthetic.N_LAYERS):
+        lw, mw = synthetic.stack_layer(layer)
+        layers.append(([lw.tensors(i, device=device) for i in range(len(lw.linears))],
+                       mw.tensors(device=device)))
+    lins = {(n, k): api.Linear(M_TOK, k, n, device=device) for _, n, k in synthetic.ATTN_LINEARS}
+    lbuf = {(n, k): (torch.empty(M_TOK, n, dtype=torch.bfloat16, device=device),
+                     torch.empty(M_TOK, k, dtype=torch.bfloat16, device=device),
+                     torch.empty(n, k, dtype=torch.bfloat16, device=device))
+            for _, n, k in synthetic.ATTN_LINEARS}
+    shapes = [(n, k) for _, n, k in synthetic.ATTN_LINEARS]
+
+    def step5():
+        for lts, mt in layers:
+            for (n, k), t in zip(shapes, lts):
+                Y, dX, dW = lbuf[(n, k)]
+                lins[(n, k)].forward(t["X"], t["W"], Y=Y)
+                lins[(n, k)].backward(t["dY"], dX=dX, dW=dW)
+            mlp.forward(mt["X"], mt["W_up"], mt["W_down"], Y=dev["Y"])
+            mlp.backward(mt["dY"], dX=dev["dX"], dW_up=dev["dW_up"], dW_down=dev["dW_down"])
+
+    K5 = max(1, min(K, args.stack_steps))
+    ms, g, o = time_steps(step5, K5, 1, flush, 1200)
+    ms = max_over_ranks(ms, world, device)
+    per_layer_flops = (sum(6 * M_TOK * n * k for n, k in shapes) + 12 * M_TOK * D_MODEL * D_FF)
+    cb = synthetic.N_LAYERS * (sum(linear_cast_bytes(M_TOK, n, k) for n, k in shapes) +
+                               mlp_cast_bytes(M_TOK, D_MODEL, D_FF))
+    out["stack28_M16384_t3"] = config_entry(
+        "28-layer stack: Q, K, V, O + relu2 MLP per layer, fwd+dgrad+wgrad, M=16384, t3 "
+        "activations", synthetic.N_LAYERS * per_layer_flops, cb, ms, g, o, peaks, world)
+    out["stack28_M16384_t3"]["inputs"] = ("drawn on the device with the synthetic recipe "
+                                          "(per-layer seeds, CUDA generators)")
+    add_graph(out["stack28_M16384_t3"], synthetic.N_LAYERS * per_layer_flops,
+              max_over_ranks(time_graph(step5, K5, flush), world, device), world)
+    del layers, lins, lbuf
+    torch.cuda.empty_cache()
+    for v in out.values():
+        v["steps"] = K if v is not out["stack28_M16384_t3"] else K5
+    if rank == 0 and not args.no_cpu_baseline:
+        for key, o in oracle_config_samples(host).items():
+            out[key]["oracle"] = o
+    return out
 
 
 # --------------------------------------------------------------- oracle
@@ -410,6 +655,69 @@ def cpu_baseline(host, tokens):
             "sample": f"oracle relu2 MLP fwd+bwd on {tokens} of {M_TOK} tokens, full "
                       f"d={D_MODEL} f={D_FF} weights (casts of the full weights included); "
                       f"{dt:.1f} s"}
+
+
+def oracle_config_samples(host):
+    """The oracle, as it stands, on bounded samples of configs 2, 4 and 5 (host
+    cores; a baseline, not a target).  Each sample keeps the full weights and
+    takes the first T tokens of the activations; config 5 times one layer of
+    the stack and multiplies by 28 (labelled extrapolated)."""
+    import oracle
+    from fp8_gemms_b200 import synthetic
+    b = synthetic.bits_u16
+    threads = oracle.num_threads()
+    res = {}
+    T = 128
+    t0 = time.perf_counter()
+    oracle.mlp_fwd(b(host["X"][:T]), b(host["W_up"]), b(host["W_down"]))
+    dt = time.perf_counter() - t0
+    res["mlp_fwd_M16384"] = {"tflops": round(4 * T * D_MODEL * D_FF / dt / 1e12, 6),
+                             "seconds": round(dt, 3), "cores": threads, "kind": "oracle",
+                             "sample": f"relu2 MLP forward on {T} of {M_TOK} tokens, full "
+                                       "weights (their casts included)"}
+    T = 64
+    w = synthetic.ATTN_HEAD
+    dt, fl = 0.0, 0
+    for i, (name, n, k) in enumerate(w.linears):
+        seed, base = w.seed, 4 * i
+        X = synthetic.normal_bf16((T, k), 1.0, seed, base)
+        W = synthetic.normal_bf16((n, k), 0.02, seed, base + 1)
+        dY = synthetic.normal_bf16((T, n), 1e-3, seed, base + 2)
+        t0 = time.perf_counter()
+        oracle.linear_fwd_bwd(b(X), b(W), b(dY))
+        dt += time.perf_counter() - t0
+        fl += 6 * T * n * k
+    res["attn_lmhead_M8192"] = {"tflops": round(fl / dt / 1e12, 6), "seconds": round(dt, 3),
+                                "cores": threads, "kind": "oracle",
+                                "sample": f"Q, K, V, O and LM head fwd+dgrad+wgrad on {T} of "
+                                          f"{w.M} tokens, full weights"}
+    T = 32
+    lw, mw = synthetic.stack_layer(0)
+    dt, fl = 0.0, 0
+    for i, (name, n, k) in enumerate(lw.linears):
+        X = synthetic.student_t3_bf16((T, k), lw.seed, 4 * i)
+        W = synthetic.normal_bf16((n, k), 0.02, lw.seed, 4 * i + 1)
+        dY = synthetic.normal_bf16((T, n), 1e-3, lw.seed, 4 * i + 2)
+        t0 = time.perf_counter()
+        oracle.linear_fwd_bwd(b(X), b(W), b(dY))
+        dt += time.perf_counter() - t0
+        fl += 6 * T * n * k
+    X = synthetic.student_t3_bf16((T, D_MODEL), mw.seed, 0)
+    Wu = synthetic.normal_bf16((D_FF, D_MODEL), 0.02, mw.seed, 1)
+    Wd = synthetic.normal_bf16((D_MODEL, D_FF), 0.02, mw.seed, 2)
+    dY = synthetic.normal_bf16((T, D_MODEL), 1e-3, mw.seed, 3)
+    t0 = time.perf_counter()
+    oracle.mlp_bwd(b(dY), oracle.mlp_fwd(b(X), b(Wu), b(Wd)))
+    dt += time.perf_counter() - t0
+    fl += 12 * T * D_MODEL * D_FF
+    n = synthetic.N_LAYERS
+    res["stack28_M16384_t3"] = {"tflops": round(fl / dt / 1e12, 6),
+                                "seconds": round(dt * n, 3), "cores": threads,
+                                "kind": "oracle", "extrapolated": True,
+                                "sample": f"layer 0 (Q, K, V, O, relu2 MLP fwd+bwd) on {T} "
+                                          f"of {M_TOK} tokens, full weights; seconds = that "
+                                          f"layer's time x {n}"}
+    return res
 
 
 def run_reference(args):

@@ -18,6 +18,7 @@
 //    count is not a multiple of 16.
 #include <cuda_bf16.h>
 
+#include "lm_cast_math.cuh"
 #include "lm_internal.h"
 #include "lm_ptx.cuh"
 
@@ -27,66 +28,6 @@ namespace {
 constexpr int kCastRows = 256;  // tile rows (the qT segment written per column)
 constexpr int kCastCols = 128;  // tile columns (bytes of codes per smem row)
 constexpr int kThreads = 256;
-
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-
-// Two packed bf16 x -> two packed h = bf16(relu(x)^2): a NaN-propagating max
-// with 0 (relu(NaN) stays NaN), then one bf16x2 multiply, which rounds the
-// exact square once to bf16.
-__device__ __forceinline__ uint32_t relu2_bf16x2(uint32_t w) {
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&w);
-    const __nv_bfloat162 r = __hmax2_nan(x, __float2bfloat162_rn(0.0f));
-    const __nv_bfloat162 h = __hmul2(r, r);
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// Two fp32 values -> two saturated RNE FP8 codes (lo in the low byte).
-template <int FMT>
-__device__ __forceinline__ uint32_t cvt_pair(float lo, float hi) {
-    uint16_t r;
-    if (FMT == LM_FP8_E4M3)
-        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    else
-        asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
-// Two packed bf16 -> two fp32 products fp32(v * scale), one packed f32x2
-// multiply (two IEEE round-to-nearest fp32 multiplies); scale2 = {scale, scale}.
-__device__ __forceinline__ void mul_bf16x2_f32(uint32_t w, uint64_t scale2, float& lo, float& hi) {
-    uint64_t x, r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(w << 16), "r"(w & 0xFFFF0000u));
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(x), "l"(scale2));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
-}
-
-__device__ __forceinline__ uint64_t splat_f32x2(float s) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(s));
-    return r;
-}
-
-// 8 bf16 (16 bytes) -> 8 codes (8 bytes), code = fp8(fp32(v * scale)).
-template <int FMT, bool RELU2>
-__device__ __forceinline__ uint2 convert8(uint4 v, float scale) {
-    const uint64_t scale2 = splat_f32x2(scale);
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t p[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float lo, hi;
-        mul_bf16x2_f32(RELU2 ? relu2_bf16x2(w[i]) : w[i], scale2, lo, hi);
-        p[i] = cvt_pair<FMT>(lo, hi);
-    }
-    return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
-}
 
 // max over the 8 bf16 of v of |x| (or of h = bf16(relu(x)^2)), as bf16 bits.
 // Non-negative bf16 values order like their bits; NaN sorts above infinity.
@@ -179,8 +120,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const AmaxSet set) {
 __device__ __forceinline__ void write_scales(float amax, float fmax, float* amax_out,
                                              float* scale_out, float* inv_out, float* scale_reg,
                                              unsigned int* err) {
-    const float a = amax < 1e-12f ? 1e-12f : amax;
-    const float scale = __fdiv_rn(fmax, a);
+    const float scale = scale_from_amax(amax, fmax);
     *scale_reg = scale;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *amax_out = amax;
@@ -639,6 +579,7 @@ lm_status lm::cast_set(const CastItem* items, int n, lm_fp8_format fmt, int relu
     for (int j = 0; j < n; ++j) {
         const CastItem& it = items[j];
         if (it.rows == 0 || it.cols == 0 || (!it.q && !it.qT)) {
+            if (it.amax_only) continue;
             unsigned int* err = device_error_word();
             if (!err) return LM_ERR_CUDA;
             timing_mark(s, 's');

@@ -25,6 +25,7 @@
 // Every mbarrier wait is bounded (see lm_ptx.cuh).
 #include <cuda_bf16.h>
 
+#include "lm_cast_math.cuh"
 #include "lm_internal.h"
 #include "lm_ptx.cuh"
 
@@ -35,6 +36,9 @@ constexpr int BK = 128;     // K bytes (= FP8 elements) per pipeline stage
 constexpr int UMMA_K = 32;  // K per tcgen05.mma for 8-bit inputs
 constexpr int NUM_THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int NUM_EPI_WARPS = 4;
+// With a side cast: warps 6-9 cast another tensor beside the tiles.
+constexpr int SIDE_WARPS = 4;
+constexpr int NUM_THREADS_SIDE = NUM_THREADS + 32 * SIDE_WARPS;
 
 // codes recorded in the device error word when a bounded wait runs out
 enum : unsigned {
@@ -85,7 +89,53 @@ struct GemmArgs {
     float* amax_out;
     unsigned int* err;
     uint32_t idesc;
+    // side cast (kernels instantiated with SIDE only): side_nvec 16-byte
+    // vectors of bf16 at side_x -> 8-byte code vectors at side_q
+    const uint4* side_x;
+    uint2* side_q;
+    int64_t side_nvec;
+    int side_fmt;
+    const float* side_amax_in;
+    float *side_amax_out, *side_scale_out, *side_inv_out;
 };
+
+// The side cast's loop for one format: eight 16-byte loads in flight per
+// thread, each 8 bf16 -> 8 codes with the cast kernels' arithmetic.
+template <int FMT>
+__device__ __forceinline__ void side_cast_loop(const GemmArgs& a, int64_t t, int64_t nt,
+                                               float scale) {
+    const uint4* x = a.side_x;
+    uint2* q = a.side_q;
+    const int64_t n = a.side_nvec;
+    int64_t i = t;
+    for (; i + 7 * nt < n; i += 8 * nt) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = ld_stream_v4(x + i + u * nt);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) q[i + u * nt] = convert8<FMT, false>(v[u], scale);
+    }
+    for (; i < n; i += nt) q[i] = convert8<FMT, false>(ld_stream_v4(x + i), scale);
+}
+
+// The side cast, run by the side warps of every CTA (thread t of nt): the
+// scale from the already-reduced amax, the scale block (thread 0), the codes.
+// A NaN or infinite amax records kErrNonfiniteAmax, as the cast kernels do.
+__device__ __forceinline__ void side_cast_run(const GemmArgs& a, int64_t t, int64_t nt) {
+    const float amax = *a.side_amax_in;
+    const bool e4 = a.side_fmt == LM_FP8_E4M3;
+    const float scale = scale_from_amax(amax, e4 ? 448.0f : 57344.0f);
+    if (t == 0) {
+        *a.side_amax_out = amax;
+        *a.side_scale_out = scale;
+        *a.side_inv_out = __fdiv_rn(1.0f, scale);
+        if (!(amax <= 3.40282347e38f)) atomicCAS(a.err, 0u, kErrNonfiniteAmax);
+    }
+    if (e4)
+        side_cast_loop<LM_FP8_E4M3>(a, t, nt, scale);
+    else
+        side_cast_loop<LM_FP8_E5M2>(a, t, nt, scale);
+}
 
 // MULTI = false: no split, or halves in one round (units split_first + 2t and
 // split_first + 2t + 1 are the halves of tile split_first + t).  MULTI = true:
@@ -104,6 +154,16 @@ __device__ __forceinline__ WorkUnit work_unit(int u, const GemmArgs& a) {
         if (t >= a.split_per_round || tile >= a.num_tiles) return {-1, 0, 0, -1};
         return {tile, part * a.num_kb / S, (part + 1) * a.num_kb / S, part};
     }
+}
+
+// The i-th k-block a unit processes in round `round` of its cluster (the
+// round-th unit that cluster takes).  Even rounds walk the unit's K range
+// forward, odd rounds backward: the tiles of one round start on the K slices
+// the previous round read last, which are the ones still in L2.  Every
+// cluster of a round takes the same direction, so the tiles in flight at
+// once still read the same slices together.
+__device__ __forceinline__ int k_block(const WorkUnit& w, int i, int round) {
+    return (round & 1) ? w.kb1 - 1 - i : w.kb0 + i;
 }
 
 // Tile visiting order: groups of group_m row-blocks, column-blocks within a
@@ -226,6 +286,12 @@ constexpr int EPI_COLS = 32;                   // columns per epilogue chunk
 constexpr int BOX_BYTES = 32 * EPI_COLS * 2;   // one warp's 32 x 32 bf16 box
 constexpr int STORE_BYTES = NUM_EPI_WARPS * 2 * BOX_BYTES;
 constexpr int AUX_BYTES = NUM_EPI_WARPS * 2 * BOX_BYTES;
+// The relu^2 backward epilogue uses the store and aux areas together as a
+// ring of H_SLOTS boxes per warp: each saved-H box is loaded H_AHEAD chunks
+// before it is needed and its dH is staged in place for the TMA store.
+constexpr int H_SLOTS = 4;
+constexpr int H_AHEAD = H_SLOTS - 1;
+static_assert(NUM_EPI_WARPS * H_SLOTS * BOX_BYTES == STORE_BYTES + AUX_BYTES, "H ring layout");
 // the accumulating epilogue stages 32 x 32 fp32 boxes (4 KB, two per warp) in
 // the store and aux areas together (contiguous, 32 KB)
 constexpr int ACC_BOX_BYTES = 32 * EPI_COLS * 4;
@@ -244,8 +310,9 @@ __device__ __forceinline__ uint32_t sw64(int r, int j) {
 // parts (the last part reads the others' sums from global memory).  The
 // instantiations for no split or halves leave that code out, which keeps the
 // epilogue loop of the common case as lean as it was measured.
-template <int EPI, bool MULTI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+// SIDE: the instantiation with four more warps that run a side cast.
+template <int EPI, bool MULTI, bool SIDE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_SIDE : NUM_THREADS, 1)
     gemm_fp8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmD,
@@ -264,8 +331,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     uint64_t* tfull = empty + STAGES;       // [2], both CTAs
     uint64_t* tempty = tfull + 2;           // [2], leader only
     uint64_t* drain = tempty + 2;           // leader only
-    uint64_t* auxbar = drain + 1;           // [4 warps][2 buffers]
-    uint64_t* splitbar = auxbar + 2 * NUM_EPI_WARPS;  // [4 warps]
+    uint64_t* auxbar = drain + 1;           // [4 warps][H_SLOTS boxes]
+    uint64_t* splitbar = auxbar + H_SLOTS * NUM_EPI_WARPS;  // [4 warps]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(splitbar + NUM_EPI_WARPS);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -283,7 +350,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&tempty[a], 2 * NUM_EPI_WARPS);
         }
         mbar_init(drain, 1);
-        for (int i = 0; i < 2 * NUM_EPI_WARPS; ++i) mbar_init(&auxbar[i], 1);
+        for (int i = 0; i < H_SLOTS * NUM_EPI_WARPS; ++i) mbar_init(&auxbar[i], 1);
         for (int i = 0; i < NUM_EPI_WARPS; ++i) mbar_init(&splitbar[i], 1);
         fence_barrier_init();
     }
@@ -315,14 +382,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0, issued = 0;
             bool ok = true;
-            for (int u = cluster; u < args.num_units && ok; u += nclusters) {
+            for (int u = cluster, round = 0; u < args.num_units && ok;
+                 u += nclusters, ++round) {
                 const WorkUnit w = work_unit<MULTI>(u, args);
                 if (MULTI && w.tile < 0) continue;
                 int mb, nb;
                 tile_coords(w.tile, args.group_m, args.num_mb, args.num_nb, mb, nb);
                 const int arow = mb * TILE_M + (int)rank * 128;
                 const int brow = nb * TILE_N + (int)rank * 128;
-                for (int kb = w.kb0; kb < w.kb1; ++kb) {
+                for (int i = 0; i < w.kb1 - w.kb0; ++i) {
+                    const int kb = k_block(w, i, round);
                     // box coordinates (x innermost): K-major (k, m|n), MN-major (m|n, k)
                     const int ax = args.a_mn ? arow : kb * BK, ay = args.a_mn ? kb * BK : arow;
                     const int bx = args.b_mn ? brow : kb * BK, by = args.b_mn ? kb * BK : brow;
@@ -374,7 +443,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.err, W_TEMPTY)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TILE_N);
-                for (int kb = w.kb0; kb < w.kb1; ++kb) {
+                for (int i = 0; i < w.kb1 - w.kb0; ++i) {
                     if (!mbar_wait(&full[stage], phase, args.err, W_FULL)) {
                         ok = false;
                         break;
@@ -385,7 +454,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk)
                         mma_fp8_pair(d_tmem, ad + (uint64_t)kk * a_step, bd + (uint64_t)kk * b_step,
-                                     args.idesc, (kb != w.kb0 || kk != 0) ? 1u : 0u);
+                                     args.idesc, (i != 0 || kk != 0) ? 1u : 0u);
                     mma_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
                     if (++stage == STAGES) {
                         stage = 0;
@@ -400,20 +469,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             mma_commit_pair(drain, 0x1);  // all MMAs retired before teardown
             mbar_wait(drain, 0, args.err, W_DRAIN);
         }
+    } else if (SIDE && warp >= 2 + NUM_EPI_WARPS) {
+        // ------------------------------------------ side cast (both CTAs)
+        constexpr int kSideThreads = 32 * SIDE_WARPS;
+        side_cast_run(args, (int64_t)blockIdx.x * kSideThreads + (threadIdx.x - NUM_THREADS),
+                      (int64_t)gridDim.x * kSideThreads);
     } else {
         // ------------------------------------------- epilogue (both CTAs)
         const int wi = warp - 2;       // staging slot
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         uint8_t* st_buf = sStore + wi * 2 * BOX_BYTES;
-        uint8_t* ax_buf = sAux + wi * 2 * BOX_BYTES;
-        uint64_t* ax_bar = auxbar + wi * 2;
+        // relu^2 backward: this warp's ring of saved-H boxes (dH staged in place)
+        uint8_t* h_ring = sStore + wi * H_SLOTS * BOX_BYTES;
+        uint64_t* h_bar = auxbar + wi * H_SLOTS;
+        uint32_t h_issued = 0, h_used = 0;  // H boxes loaded / consumed by this warp
         const uint32_t tempty_leader = map_to_rank(smem_addr(tempty), 0);
         const uint64_t stream_policy = l2_policy_evict_first();  // D and H are touched once
         const float s = __fmul_rn(*args.inv_a, *args.inv_b);
         uint32_t amax2 = 0;  // two bf16-bit halves of the running max
         int acc = 0;
         uint32_t acc_phase = 0;
-        uint32_t ax_phase = 0;  // bit b: parity of the next wait on aux buffer b
         uint32_t n_stores = 0;
         bool ok = true;
         for (int u = cluster; u < args.num_units && ok; u += nclusters) {
@@ -434,13 +509,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 return (((size_t)(w.tile - args.split_first) * (size_t)(S - 1) + (size_t)p) * 2 +
                         rank) * NUM_EPI_WARPS + quarter;
             };
-            if (EPI == LM_EPI_RELU2_BWD && lane == 0 && finishes) {
-                // the first H box of this tile (no L2 prefetch of the next
-                // tile's H: measured, it raised DRAM reads by a third and cost
-                // 3.6% of this GEMM's time)
+            // relu^2 backward: load saved-H box j of this warp into ring slot
+            // j % H_SLOTS.  The dH store that last read that slot (box j -
+            // H_SLOTS) is at least the second most recent store, so waiting
+            // until at most one store is still reading shared memory frees it.
+            auto issue_h = [&](int chunk) {
+                const uint32_t slot = h_issued % H_SLOTS;
+                bulk_wait_group_read<1>();
                 fence_proxy_async_smem();
-                mbar_arrive_expect_tx(&ax_bar[0], BOX_BYTES);
-                tma_load_2d_hint(smem_addr(ax_buf), &tmAux, &ax_bar[0], gcol, grow, stream_policy);
+                mbar_arrive_expect_tx(&h_bar[slot], BOX_BYTES);
+                tma_load_2d_hint(smem_addr(h_ring + slot * BOX_BYTES), &tmAux, &h_bar[slot],
+                                 gcol + chunk * EPI_COLS, grow, stream_policy);
+            };
+            if constexpr (EPI == LM_EPI_RELU2_BWD) {
+                if (finishes) {
+                    // this tile's first H_AHEAD boxes arrive while its
+                    // accumulator is still being computed
+                    const int first = n_chunks < H_AHEAD ? n_chunks : H_AHEAD;
+                    for (int c = 0; c < first; ++c) {
+                        if (lane == 0) issue_h(c);
+                        ++h_issued;
+                    }
+                }
             }
             if (!mbar_wait(&tfull[acc], acc_phase, args.err, W_TFULL)) break;
             tc_fence_after();
@@ -570,32 +660,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                             }
                         }
                     }
-                    uint32_t hw[16];  // saved H, two bf16 per word, columns 2i and 2i+1
-                    if (EPI == LM_EPI_RELU2_BWD) {
-                        const int b = c & 1;
-                        if (lane == 0 && c + 1 < n_chunks) {
-                            fence_proxy_async_smem();
-                            mbar_arrive_expect_tx(&ax_bar[b ^ 1], BOX_BYTES);
-                            tma_load_2d_hint(smem_addr(ax_buf + (b ^ 1) * BOX_BYTES), &tmAux,
-                                             &ax_bar[b ^ 1], gcol + (c + 1) * EPI_COLS, grow,
-                                             stream_policy);
-                        }
-                        if (!mbar_wait(&ax_bar[b], (ax_phase >> b) & 1u, args.err, W_AUX)) {
+                    if constexpr (EPI == LM_EPI_RELU2_BWD) {
+                        // saved H of this chunk (two bf16 per word, columns
+                        // 2i and 2i+1) from its ring slot; dH goes back into
+                        // the same slot (each lane rewrites only its own row)
+                        // and is TMA-stored from there
+                        const uint32_t slot = h_used % H_SLOTS;
+                        uint8_t* box = h_ring + slot * BOX_BYTES;
+                        if (!mbar_wait(&h_bar[slot], (h_used / H_SLOTS) & 1u, args.err, W_AUX)) {
                             ok = false;
                             break;
                         }
-                        ax_phase ^= 1u << b;
-                        const uint8_t* src = ax_buf + b * BOX_BYTES;
+                        ++h_used;
+                        uint32_t hw[16];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            const uint4 v = *reinterpret_cast<const uint4*>(src + sw64(lane, j));
+                            const uint4 v = *reinterpret_cast<const uint4*>(box + sw64(lane, j));
                             hw[4 * j] = v.x;
                             hw[4 * j + 1] = v.y;
                             hw[4 * j + 2] = v.z;
                             hw[4 * j + 3] = v.w;
                         }
-                    }
-                    if constexpr (EPI == LM_EPI_ACCUM_F32) {
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            packed[i] = epi_pair<EPI>(r[2 * i], r[2 * i + 1], s, hw[i], amax2);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4*>(box + sw64(lane, j)) =
+                                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                                           packed[4 * j + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d_hint(&tmD, smem_addr(box), gcol + c * EPI_COLS, grow,
+                                              stream_policy);
+                            bulk_commit_group();
+                        }
+                        if (c + H_AHEAD < n_chunks) {
+                            if (lane == 0) issue_h(c + H_AHEAD);
+                            ++h_issued;
+                        }
+                    } else if constexpr (EPI == LM_EPI_ACCUM_F32) {
                         // fp32 partial -> 128B-swizzled 32 x 32 fp32 box -> TMA reduce-add
                         uint8_t* dst =
                             sStore + wi * 2 * ACC_BOX_BYTES + (n_stores & 1u) * ACC_BOX_BYTES;
@@ -619,8 +725,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         uint32_t packed[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
-                            packed[i] = epi_pair<EPI>(r[2 * i], r[2 * i + 1], s,
-                                                      EPI == LM_EPI_RELU2_BWD ? hw[i] : 0u, amax2);
+                            packed[i] = epi_pair<EPI>(r[2 * i], r[2 * i + 1], s, 0u, amax2);
                         // staging buffer n_stores & 1: the store that last used it must
                         // have finished reading shared memory
                         uint8_t* dst = st_buf + (n_stores & 1u) * BOX_BYTES;
@@ -648,6 +753,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
+        // H boxes still in flight (only after a wait ran out): let them land
+        // (bounded) before the shared memory is released
+        for (uint32_t j = h_used; j < h_issued; ++j)
+            mbar_wait(&h_bar[j % H_SLOTS], (j / H_SLOTS) & 1u, args.err, W_AUX);
         if (lane == 0) bulk_wait_group<0>();
         reduce_amax<EPI>(max(amax2 & 0xFFFFu, amax2 >> 16), args.amax_out, lane);
     }
@@ -895,12 +1004,12 @@ bool ensure_smem(F* kernel, int bytes, bool (&done)[64]) {
     return true;
 }
 
-template <int EPI, bool MULTI>
+template <int EPI, bool MULTI, bool SIDE>
 lm_status launch_pair_as(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                          const CUtensorMap& tx, const CUtensorMap& td2, const GemmArgs& a,
                          cudaStream_t s) {
     static bool done[64] = {};
-    if (!ensure_smem(pair::gemm_fp8_pair_kernel<EPI, MULTI>, pair::SMEM_BYTES, done))
+    if (!ensure_smem(pair::gemm_fp8_pair_kernel<EPI, MULTI, SIDE>, pair::SMEM_BYTES, done))
         return LM_ERR_CUDA;
     const int sms = sm_count();
     if (sms < 2) return LM_ERR_CUDA;
@@ -911,24 +1020,35 @@ lm_status launch_pair_as(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
                         (size_t)a.split_slots * 2 * NUM_EPI_WARPS * sizeof(unsigned int),
                         s) != cudaSuccess)
         return LM_ERR_CUDA;
-    pair::gemm_fp8_pair_kernel<EPI, MULTI>
-        <<<2 * clusters, NUM_THREADS, pair::SMEM_BYTES, s>>>(ta, tb, td, tx, td2, a);
+    pair::gemm_fp8_pair_kernel<EPI, MULTI, SIDE>
+        <<<2 * clusters, SIDE ? NUM_THREADS_SIDE : NUM_THREADS, pair::SMEM_BYTES, s>>>(
+            ta, tb, td, tx, td2, a);
     return launch_status();
 }
 
 // No split or halves in one round: the lean instantiation; three or more parts
 // (never for the gated epilogue): the one that reads partials from global memory.
+// With a side cast (a.side_nvec > 0; plain and relu^2-forward epilogues, no
+// multi-part tail) the instantiation with side warps; *side_done says whether
+// this launch carries it.
 template <int EPI>
 lm_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                       const CUtensorMap& tx, const CUtensorMap& td2, const GemmArgs& a,
-                      cudaStream_t s) {
+                      cudaStream_t s, bool* side_done) {
+    *side_done = false;
     if constexpr (EPI == kEpiSwigluFwd) {
-        return launch_pair_as<EPI, false>(ta, tb, td, tx, td2, a, s);
+        return launch_pair_as<EPI, false, false>(ta, tb, td, tx, td2, a, s);
     } else {
         const bool halves_in_one_round =
             a.split_parts <= 2 && a.num_units - a.split_first <= a.split_round;
-        if (!halves_in_one_round) return launch_pair_as<EPI, true>(ta, tb, td, tx, td2, a, s);
-        return launch_pair_as<EPI, false>(ta, tb, td, tx, td2, a, s);
+        if (!halves_in_one_round) return launch_pair_as<EPI, true, false>(ta, tb, td, tx, td2, a, s);
+        if constexpr (EPI == LM_EPI_NONE || EPI == LM_EPI_RELU2_FWD) {
+            if (a.side_nvec > 0) {
+                *side_done = true;
+                return launch_pair_as<EPI, false, true>(ta, tb, td, tx, td2, a, s);
+            }
+        }
+        return launch_pair_as<EPI, false, false>(ta, tb, td, tx, td2, a, s);
     }
 }
 
@@ -1016,12 +1136,35 @@ extern "C" lm_status lm_fp8_gemm_split_plan(int64_t M, int64_t N, int64_t K, int
     return LM_OK;
 }
 
+namespace lm {
+namespace {
+
+// The side cast as its own launch (when the GEMM launch cannot carry it).
+lm_status side_cast_alone(const SideCast& sc, cudaStream_t s) {
+    const CastItem it = {sc.x, sc.rows, sc.cols, sc.cols, sc.amax_in, sc.amax_out,
+                         sc.scale_out, sc.inv_scale_out, sc.q, nullptr};
+    return cast_set(&it, 1, sc.fmt, 0, true, s);
+}
+
+}  // namespace
+}  // namespace lm
+
 lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B,
                             lm_fp8_format fb, int64_t M, int64_t N, int64_t K, uint32_t flags,
                             const float* inv_scale_a, const float* inv_scale_b, int epi,
                             const void* aux, void* D, void* D2, float* amax_out, void* workspace,
-                            size_t ws_bytes, lm_stream_t stream) {
+                            size_t ws_bytes, lm_stream_t stream, const SideCast* side) {
     using namespace lm;
+    if (side) {
+        // checked like lm_fp8_amax_scale_cast's arguments, before any launch
+        if ((side->fmt != LM_FP8_E4M3 && side->fmt != LM_FP8_E5M2) || side->rows < 0 ||
+            side->cols < 0 || side->cols % 16 != 0 || !side->amax_in || !side->amax_out ||
+            !side->scale_out || !side->inv_scale_out ||
+            ((side->rows > 0 && side->cols > 0) && (!side->x || !side->q)))
+            return LM_ERR_INVALID_ARG;
+        if (!aligned16(side->x) || !aligned16(side->q)) return LM_ERR_ALIGNMENT;
+        if (side->rows == 0 || side->cols == 0) side = nullptr;  // nothing to cast
+    }
     if ((fa != LM_FP8_E4M3 && fa != LM_FP8_E5M2) || (fb != LM_FP8_E4M3 && fb != LM_FP8_E5M2))
         return LM_ERR_UNSUPPORTED_FORMAT;
     if (fa == LM_FP8_E5M2 && fb == LM_FP8_E5M2) return LM_ERR_UNSUPPORTED_FORMAT;
@@ -1029,7 +1172,8 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
         epi != LM_EPI_ACCUM_F32 && epi != kEpiSwigluFwd)
         return LM_ERR_UNSUPPORTED_FORMAT;
     if (M < 0 || N < 0 || K < 0) return LM_ERR_INVALID_ARG;
-    if (M == 0 || N == 0) return LM_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (M == 0 || N == 0) return side ? side_cast_alone(*side, s) : LM_OK;
     if (!D || !inv_scale_a || !inv_scale_b) return LM_ERR_INVALID_ARG;
     if (K > 0 && (!A || !B)) return LM_ERR_INVALID_ARG;
     if (epi == LM_EPI_RELU2_BWD && !aux) return LM_ERR_INVALID_ARG;
@@ -1044,12 +1188,11 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
     if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(aux) || !aligned16(D2))
         return LM_ERR_ALIGNMENT;
 
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (K == 0) {  // empty reduction: D = epi(0) = 0 (accumulating: D += 0), amax unchanged
-        if (epi == LM_EPI_ACCUM_F32) return LM_OK;
-        if (cudaMemsetAsync(D, 0, (size_t)M * (size_t)N * 2, s) != cudaSuccess)
+        if (epi != LM_EPI_ACCUM_F32 &&
+            cudaMemsetAsync(D, 0, (size_t)M * (size_t)N * 2, s) != cudaSuccess)
             return LM_ERR_CUDA;
-        return LM_OK;
+        return side ? side_cast_alone(*side, s) : LM_OK;
     }
     unsigned int* err = device_error_word();
     if (!err) return LM_ERR_CUDA;
@@ -1063,11 +1206,26 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
     a.aux = static_cast<const uint16_t*>(aux);
     a.D = D;
     a.D2 = D2;
-    if (epi == LM_EPI_ACCUM_F32) a.amax_out = nullptr;
-    a.amax_out = amax_out;
+    a.amax_out = epi == LM_EPI_ACCUM_F32 ? nullptr : amax_out;
     a.err = err;
     a.a_mn = a_mn ? 1 : 0;
     a.b_mn = b_mn ? 1 : 0;
+    a.side_x = nullptr;
+    a.side_q = nullptr;
+    a.side_nvec = 0;
+    a.side_fmt = 0;
+    a.side_amax_in = nullptr;
+    a.side_amax_out = a.side_scale_out = a.side_inv_out = nullptr;
+    if (side) {
+        a.side_x = static_cast<const uint4*>(side->x);
+        a.side_q = reinterpret_cast<uint2*>(side->q);
+        a.side_nvec = side->rows * side->cols / 8;
+        a.side_fmt = (int)side->fmt;
+        a.side_amax_in = side->amax_in;
+        a.side_amax_out = side->amax_out;
+        a.side_scale_out = side->scale_out;
+        a.side_inv_out = side->inv_scale_out;
+    }
 
     CUtensorMap ta, tb;
     if (M > 128 || epi == kEpiSwigluFwd) {
@@ -1140,16 +1298,25 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
         if (epi == kEpiSwigluFwd &&
             !encode_tmap_bf16_sw64(&td2, D2, (uint64_t)M, (uint64_t)(N / 2), 32, pair::EPI_COLS))
             return LM_ERR_CUDA;
+        bool side_done = false;
+        lm_status st;
         switch (epi) {
-            case LM_EPI_NONE: return launch_pair<LM_EPI_NONE>(ta, tb, td, tx, td2, a, s);
+            case LM_EPI_NONE:
+                st = launch_pair<LM_EPI_NONE>(ta, tb, td, tx, td2, a, s, &side_done);
+                break;
             case LM_EPI_RELU2_FWD:
-                return launch_pair<LM_EPI_RELU2_FWD>(ta, tb, td, tx, td2, a, s);
+                st = launch_pair<LM_EPI_RELU2_FWD>(ta, tb, td, tx, td2, a, s, &side_done);
+                break;
             case LM_EPI_RELU2_BWD:
-                return launch_pair<LM_EPI_RELU2_BWD>(ta, tb, td, tx, td2, a, s);
+                st = launch_pair<LM_EPI_RELU2_BWD>(ta, tb, td, tx, td2, a, s, &side_done);
+                break;
             case LM_EPI_ACCUM_F32:
-                return launch_pair<LM_EPI_ACCUM_F32>(ta, tb, td, tx, td2, a, s);
-            default: return launch_pair<kEpiSwigluFwd>(ta, tb, td, tx, td2, a, s);
+                st = launch_pair<LM_EPI_ACCUM_F32>(ta, tb, td, tx, td2, a, s, &side_done);
+                break;
+            default: st = launch_pair<kEpiSwigluFwd>(ta, tb, td, tx, td2, a, s, &side_done);
         }
+        if (st != LM_OK || side_done || !side) return st;
+        return side_cast_alone(*side, s);
     }
     a.num_mb = (int)((M + one::BM - 1) / one::BM);
     a.num_nb = (int)((N + one::BN - 1) / one::BN);
@@ -1171,12 +1338,15 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
         (b_mn ? encode_tmap_u8(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)N, BK, 128)
               : encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, one::BN, BK));
     if (!mok) return LM_ERR_CUDA;
+    lm_status st;
     switch (epi) {
-        case LM_EPI_NONE: return launch_one<LM_EPI_NONE>(ta, tb, a, s);
-        case LM_EPI_RELU2_FWD: return launch_one<LM_EPI_RELU2_FWD>(ta, tb, a, s);
-        case LM_EPI_RELU2_BWD: return launch_one<LM_EPI_RELU2_BWD>(ta, tb, a, s);
-        default: return launch_one<LM_EPI_ACCUM_F32>(ta, tb, a, s);
+        case LM_EPI_NONE: st = launch_one<LM_EPI_NONE>(ta, tb, a, s); break;
+        case LM_EPI_RELU2_FWD: st = launch_one<LM_EPI_RELU2_FWD>(ta, tb, a, s); break;
+        case LM_EPI_RELU2_BWD: st = launch_one<LM_EPI_RELU2_BWD>(ta, tb, a, s); break;
+        default: st = launch_one<LM_EPI_ACCUM_F32>(ta, tb, a, s);
     }
+    if (st != LM_OK || !side) return st;
+    return side_cast_alone(*side, s);
 }
 
 extern "C" size_t lm_fp8_gemm_workspace_size(void) { return lm::gemm_split_workspace_bytes(); }

@@ -53,11 +53,30 @@ bool encode_tmap_bf16_plain(CUtensorMap* map, const void* base, uint64_t rows, u
 // h = bf16(silu(G) U) [M x N/2]; amax_out gets max |h|.
 constexpr int kEpiSwigluFwd = 4;
 
-// lm_fp8_gemm_ex with the internal epilogues and a second output.
+// A cast that a GEMM launch runs in extra warps beside its tiles: a contiguous
+// bf16 tensor whose amax has already been reduced (by an earlier kernel on
+// the stream) is cast to row-major codes at the scale that amax gives, and
+// its {amax, scale, inv_scale} are written.  The GEMM must neither read the
+// codes nor write the input.  Where the GEMM launch cannot carry it (the
+// thin kernel, a multi-part split tail, an empty GEMM), gemm_dispatch runs
+// the cast as its own launch after the GEMM instead; the results are the same
+// bits either way.
+struct SideCast {
+    const void* x;  // bf16 [rows x cols], contiguous
+    int64_t rows, cols;
+    lm_fp8_format fmt;
+    const float* amax_in;
+    float *amax_out, *scale_out, *inv_scale_out;
+    uint8_t* q;  // [rows x cols] codes
+};
+
+// lm_fp8_gemm_ex with the internal epilogues, a second output and an
+// optional side cast.
 lm_status gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B, lm_fp8_format fb,
                         int64_t M, int64_t N, int64_t K, uint32_t flags, const float* inv_scale_a,
                         const float* inv_scale_b, int epi, const void* aux, void* D, void* D2,
-                        float* amax_out, void* workspace, size_t ws_bytes, lm_stream_t stream);
+                        float* amax_out, void* workspace, size_t ws_bytes, lm_stream_t stream,
+                        const SideCast* side = nullptr);
 
 // Workspace bytes that let any GEMM split its last wave (lm_fp8_gemm_workspace_size).
 size_t gemm_split_workspace_bytes();
@@ -69,6 +88,9 @@ struct CastItem {
     const float* amax_in;
     float *amax_out, *scale_out, *inv_scale_out;
     uint8_t *q, *qT;
+    // with q and qT NULL: reduce the amax only and leave the scales to a
+    // later side cast (no scales-only launch)
+    bool amax_only = false;
 };
 constexpr int kMaxCastSet = 3;
 

@@ -127,18 +127,23 @@ lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_dow
     } else if (cudaMemsetAsync(S, 0, 16 * sizeof(float), s) != cudaSuccess) {
         return LM_ERR_CUDA;
     }
-    // X, W_up and W_down (or X alone): one amax launch and one cast launch;
-    // their amax slots were zeroed above.  Row-major codes only: the
-    // backward reads them MN-major where it needs the transpose.
+    // X, W_up and W_down (or X alone): one amax launch for all three (their
+    // amax slots were zeroed above) and one cast launch for X and W_up.
+    // W_down is cast beside the up GEMM, which does not read it.  Row-major
+    // codes only: the backward reads them MN-major where it needs the
+    // transpose.
     const lm::CastItem in[3] = {
         {X, M, d, d, nullptr, S + S_X, S + S_X + 1, S + S_X + 2, sv->Xq, nullptr},
         {W_up, f, d, d, nullptr, S + S_WU, S + S_WU + 1, S + S_WU + 2, sv->Wuq, nullptr},
-        {W_down, d, f, f, nullptr, S + S_WD, S + S_WD + 1, S + S_WD + 2, sv->Wdq, nullptr}};
+        {W_down, d, f, f, nullptr, S + S_WD, S + S_WD + 1, S + S_WD + 2, nullptr, nullptr,
+         true}};
     LM_TRY(lm::cast_set(in, reuse ? 1 : 3, LM_FP8_E4M3, 0, true, s));
-    // H = X W_up^T (bf16) and amax of h = bf16(relu(H)^2)
-    LM_TRY(lm_fp8_gemm_ex(sv->Xq, LM_FP8_E4M3, sv->Wuq, LM_FP8_E4M3, M, f, d, 0u, S + S_X + 2,
-                          S + S_WU + 2, LM_EPI_RELU2_FWD, nullptr, sv->H, S + S_H, split, sb,
-                          stream));
+    const lm::SideCast wd = {W_down, d, f, LM_FP8_E4M3, S + S_WD, S + S_WD, S + S_WD + 1,
+                             S + S_WD + 2, sv->Wdq};
+    // H = X W_up^T (bf16) and amax of h = bf16(relu(H)^2); W_down's codes
+    LM_TRY(lm::gemm_dispatch(sv->Xq, LM_FP8_E4M3, sv->Wuq, LM_FP8_E4M3, M, f, d, 0u, S + S_X + 2,
+                             S + S_WU + 2, LM_EPI_RELU2_FWD, nullptr, sv->H, nullptr, S + S_H,
+                             split, sb, stream, reuse ? nullptr : &wd));
     LM_TRY(lm_fp8_amax_scale_cast(sv->H, M, f, f, LM_FP8_E4M3, 1, S + S_H, S + S_H, S + S_H + 1,
                                   S + S_H + 2, sv->hq, nullptr, stream));
     // Y = h W_down^T
@@ -183,11 +188,13 @@ lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* sv, int64_t M,
     LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->Wdq, LM_FP8_E4M3, M, f, d, B_MN, G + S_DY + 2,
                           S + S_WD + 2, LM_EPI_RELU2_BWD, sv->H, w.dH, G + S_DH, w.split, sb,
                           stream));
-    // dW_down = dY^T h (K = M): dY [M x d] and h [M x f] read MN-major
-    LM_TRY(lm_fp8_gemm_ex(w.dYq, LM_FP8_E5M2, sv->hq, LM_FP8_E4M3, d, f, M, AB_MN, G + S_DY + 2,
-                          S + S_H + 2, wgrad_epi, nullptr, dW_down, nullptr, w.split, sb, stream));
-    LM_TRY(lm_fp8_amax_scale_cast(w.dH, M, f, f, LM_FP8_E5M2, 0, G + S_DH, G + S_DH,
-                                  G + S_DH + 1, G + S_DH + 2, w.dHq, nullptr, stream));
+    // dW_down = dY^T h (K = M): dY [M x d] and h [M x f] read MN-major; the
+    // cast of dH (its amax came from the epilogue above) runs beside it
+    const lm::SideCast dh = {w.dH, M, f, LM_FP8_E5M2, G + S_DH, G + S_DH, G + S_DH + 1,
+                             G + S_DH + 2, w.dHq};
+    LM_TRY(lm::gemm_dispatch(w.dYq, LM_FP8_E5M2, sv->hq, LM_FP8_E4M3, d, f, M, AB_MN,
+                             G + S_DY + 2, S + S_H + 2, wgrad_epi, nullptr, dW_down, nullptr,
+                             nullptr, w.split, sb, stream, &dh));
     // dX = dH W_up (W_up [f x d] read MN-major);  dW_up = dH^T X (K = M)
     LM_TRY(lm_fp8_gemm_ex(w.dHq, LM_FP8_E5M2, sv->Wuq, LM_FP8_E4M3, M, d, f, B_MN, G + S_DH + 2,
                           S + S_WU + 2, LM_EPI_NONE, nullptr, dX, nullptr, w.split, sb, stream));

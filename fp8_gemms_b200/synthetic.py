@@ -8,6 +8,10 @@ Recipe:
   * every tensor has its own CPU ``torch.Generator`` seeded with
     ``seed * 1009 + index`` (index = position of the tensor in its workload),
     so any one tensor can be regenerated without drawing the others;
+  * the same recipe can draw on a CUDA device instead (``device=``), with a
+    CUDA generator seeded the same way: same distributions and seeds, other
+    values.  The benchmark uses it for workloads too large to draw on the host
+    in reasonable time (the 28-layer stack); the parity tests use host draws;
   * values are drawn in fp32 and rounded to bf16 (round to nearest even);
   * "N(0, s)" means standard deviation s; "t3" means a standard Student-t with
     3 degrees of freedom, Z / sqrt(chi2_3 / 3), not rescaled.
@@ -31,31 +35,32 @@ N_Q_HEADS, N_KV_HEADS, HEAD_DIM = 24, 8, 128
 VOCAB, VOCAB_PADDED = 50257, 50304
 
 
-def _gen(seed: int, index: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+def _gen(seed: int, index: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
     g.manual_seed(seed * 1009 + index)
     return g
 
 
-def normal_bf16(shape, std: float, seed: int, index: int) -> torch.Tensor:
-    x = torch.randn(*shape, generator=_gen(seed, index), dtype=torch.float32)
+def normal_bf16(shape, std: float, seed: int, index: int, device="cpu") -> torch.Tensor:
+    x = torch.randn(*shape, generator=_gen(seed, index, device), dtype=torch.float32,
+                    device=device)
     return (x * std).to(torch.bfloat16)
 
 
-def student_t3_bf16(shape, seed: int, index: int) -> torch.Tensor:
-    g = _gen(seed, index)
-    z = torch.randn(*shape, generator=g, dtype=torch.float32)
-    c = torch.randn(3, *shape, generator=g, dtype=torch.float32).square().sum(0)
+def student_t3_bf16(shape, seed: int, index: int, device="cpu") -> torch.Tensor:
+    g = _gen(seed, index, device)
+    z = torch.randn(*shape, generator=g, dtype=torch.float32, device=device)
+    c = torch.randn(3, *shape, generator=g, dtype=torch.float32, device=device).square().sum(0)
     return (z / torch.sqrt(c / 3.0)).to(torch.bfloat16)
 
 
-def draw(spec, seed: int, index: int) -> torch.Tensor:
+def draw(spec, seed: int, index: int, device="cpu") -> torch.Tensor:
     shape, dist = spec
     kind, param = dist
     if kind == "normal":
-        return normal_bf16(shape, param, seed, index)
+        return normal_bf16(shape, param, seed, index, device)
     if kind == "t3":
-        return student_t3_bf16(shape, seed, index)
+        return student_t3_bf16(shape, seed, index, device)
     raise ValueError(kind)
 
 
@@ -70,13 +75,13 @@ class MlpWorkload:
     x_dist: tuple = ("normal", 1.0)
     seed: int = 0
 
-    def tensors(self):
-        x = draw(((self.M, self.d), self.x_dist), self.seed, 0)
-        wu = draw(((self.f, self.d), ("normal", 0.02)), self.seed, 1)
-        wd = draw(((self.d, self.f), ("normal", 0.02)), self.seed, 2)
+    def tensors(self, device="cpu"):
+        x = draw(((self.M, self.d), self.x_dist), self.seed, 0, device)
+        wu = draw(((self.f, self.d), ("normal", 0.02)), self.seed, 1, device)
+        wd = draw(((self.d, self.f), ("normal", 0.02)), self.seed, 2, device)
         out = dict(X=x, W_up=wu, W_down=wd)
         if self.backward:
-            out["dY"] = draw(((self.M, self.d), ("normal", 1e-3)), self.seed, 3)
+            out["dY"] = draw(((self.M, self.d), ("normal", 1e-3)), self.seed, 3, device)
         return out
 
     @property
@@ -94,14 +99,14 @@ class LinearWorkload:
     x_dist: tuple = ("normal", 1.0)
     seed: int = 0
 
-    def tensors(self, i: int):
+    def tensors(self, i: int, device="cpu"):
         lname, n_out, n_in = self.linears[i]
         base = 4 * i
         return dict(
             name=lname,
-            X=draw(((self.M, n_in), self.x_dist), self.seed, base + 0),
-            W=draw(((n_out, n_in), ("normal", 0.02)), self.seed, base + 1),
-            dY=draw(((self.M, n_out), ("normal", 1e-3)), self.seed, base + 2),
+            X=draw(((self.M, n_in), self.x_dist), self.seed, base + 0, device),
+            W=draw(((n_out, n_in), ("normal", 0.02)), self.seed, base + 1, device),
+            dY=draw(((self.M, n_out), ("normal", 1e-3)), self.seed, base + 2, device),
         )
 
     @property

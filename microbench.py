@@ -1,40 +1,44 @@
 """Time one C-ABI call on synthetic data (CUDA events, L2 flushed between
 iterations).  Also the small, self-contained command to run under ncu.
 
-    python -m fp8_gemms_b200.microbench gemm --M 16384 --N 12288 --K 3072 --epi relu2_fwd
-    python -m fp8_gemms_b200.microbench cast --rows 16384 --cols 3072 --fmt e4m3
-    python -m fp8_gemms_b200.microbench cast --rows 16384 --cols 12288 --relu2 --amax-in
-    python -m fp8_gemms_b200.microbench mlp-compare --M 16384
+    python microbench.py gemm --M 16384 --N 12288 --K 3072 --epi relu2_fwd
+    python microbench.py cast --rows 16384 --cols 3072 --fmt e4m3
+    python microbench.py cast --rows 16384 --cols 12288 --relu2 --amax-in
+    python microbench.py mlp-compare --M 16384
         (the non-gated relu^2 block, f = 4d, against the gated SwiGLU block,
         f = 2.75d, both fwd + bwd in FP8: ms per step and tokens per second)
-    python -m fp8_gemms_b200.microbench scaled-mm
+    python microbench.py scaled-mm
         (library calibration: torch._scaled_mm, i.e. cuBLASLt FP8, against this
         library's GEMM on the six GEMM shapes of the relu^2 MLP step, M = 16384)
-    python -m fp8_gemms_b200.microbench torch-composition --M 16384
+    python microbench.py torch-composition --M 16384
         (the same relu^2 MLP step composed the way the pages' training code
         composes it -- per-tensor amax and cast in PyTorch, transposed copies,
         one torch._scaled_mm (cuBLASLt) per GEMM, unfused relu^2 / relu^2' --
         against this library's two calls, on the same GPU and inputs)
-    python -m fp8_gemms_b200.microbench linears --workload attn-head
+    python microbench.py linears --workload attn-head
         (the attention projections Q, K, V, O and the LM head at M = 8192, each
         fwd + dgrad + wgrad through lm_fp8_linear_fwd / _bwd: per linear, and
         the whole set eagerly and replayed from a CUDA graph)
-    python -m fp8_gemms_b200.microbench linears --workload stack
+    python microbench.py linears --workload stack
         (the per-step linear GEMM set of a 28-layer d = 3072 stack at M = 16384:
         per layer Q, K, V, O and the relu^2 MLP, fwd + dgrad + wgrad, each
         layer with its own weights and t3-distributed activations)
-    python -m fp8_gemms_b200.microbench mlp-accum --M 16384 --micro 7
+    python microbench.py mlp-accum --M 16384 --micro 7
         (one optimizer step of gradient accumulation: the weights are cast by the
         first micro-batch's forward and reused by the others; every backward adds
         its weight gradients into fp32 accumulators)
 """
 import argparse
 import json
+import os
+import sys
 
 import torch
 
-from . import _lib
-from ._lib import E4M3, E5M2, EPI_NONE, EPI_RELU2_BWD, EPI_RELU2_FWD
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+from fp8_gemms_b200 import _lib  # noqa: E402
+from fp8_gemms_b200._lib import E4M3, E5M2, EPI_NONE, EPI_RELU2_BWD, EPI_RELU2_FWD  # noqa: E402
 
 FMT = {"e4m3": E4M3, "e5m2": E5M2}
 EPI = {"none": EPI_NONE, "relu2_fwd": EPI_RELU2_FWD, "relu2_bwd": EPI_RELU2_BWD}
@@ -76,7 +80,7 @@ def _draw(shape, dist, gen):
 
 
 def linears(a, gen, flush):
-    from . import api, synthetic
+    from fp8_gemms_b200 import api, synthetic
     if a.workload == "attn-head":
         M, layers, x_dist = 8192, 1, 1.0
         shapes = synthetic.ATTN_LINEARS + [("lm_head", synthetic.VOCAB_PADDED,
@@ -228,7 +232,7 @@ def main():
                    scaled_mm_total_ms=round(tot_l, 4),
                    ours_over_scaled_mm_speed=round(tot_l / tot_o, 4))
     elif a.op == "torch-composition":
-        from . import api
+        from fp8_gemms_b200 import api
         M, d, f = a.M, a.d, a.f
         bf = torch.bfloat16
         X = torch.randn(M, d, device="cuda", generator=gen).to(bf)
@@ -283,7 +287,7 @@ def main():
                    speedup_vs_eager=round(t_ref / t_ours, 3),
                    speedup_vs_compiled=round(t_cmp / t_ours, 3))
     elif a.op == "mlp-compare":
-        from . import api
+        from fp8_gemms_b200 import api
         M, d = a.M, a.d
         res = {}
         for name, f in (("relu2", 4 * d), ("swiglu", (11 * d) // 4)):
@@ -308,7 +312,7 @@ def main():
                    relu2_over_swiglu_tokens=round(res["relu2"]["tokens_per_s"] /
                                                   res["swiglu"]["tokens_per_s"], 4))
     elif a.op == "lmhead-ce":
-        from . import api
+        from fp8_gemms_b200 import api
         M, d, V = a.M, a.d, a.V
         head = api.LmHeadCE(M, d, V, a.chunk)
         X = torch.randn(M, d, device="cuda", generator=gen).to(torch.bfloat16)
@@ -390,7 +394,7 @@ def main():
                    min_ms=round(min(ms), 4),
                    gbs=round(byts / avg / 1e6, 1), algorithmic_bytes=byts)
     if a.op == "mlp-accum":
-        from . import api  # noqa: F811
+        from fp8_gemms_b200 import api  # noqa: F811
         M, d, f = a.M, a.d, a.f
         mlp = api.Relu2Mlp(M, d, f)
         Wu = (torch.randn(f, d, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)

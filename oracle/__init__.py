@@ -230,6 +230,23 @@ def rmsnorm_fp8_cast(R, w=None, eps=1e-6, fmt=E4M3):
     return out
 
 
+# ---------------------------------------------------------- plain linear
+def linear_fwd_bwd(X, W, dY):
+    """Plain FP8 linear Y = X W^T with its dgrad and wgrad (the attention
+    projections and the LM head): X and W quantised to e4m3 and dY to e5m2,
+    each once with its own tensorwise scale (decomputer.nl, "Het trainen van
+    een 3.8B LLM tot 0.384 CORE voor $998", section "Vroege experimenten" item
+    4: all three GEMMs of a linear in FP8).
+      Y = Xq Wq^T,  dX = dYq Wq,  dW = dYq^T Xq   (bf16 bits out)."""
+    cx = amax_scale_cast(X, E4M3)
+    cw = amax_scale_cast(W, E4M3)
+    cg = amax_scale_cast(dY, E5M2)
+    Y, _ = gemm(cx["q"], E4M3, cw["q"], E4M3, cx["inv_scale"], cw["inv_scale"])
+    dX, _ = gemm(cg["q"], E5M2, cw["qT"], E4M3, cg["inv_scale"], cw["inv_scale"])
+    dW, _ = gemm(cg["qT"], E5M2, cx["qT"], E4M3, cg["inv_scale"], cx["inv_scale"])
+    return dict(Y=Y, dX=dX, dW=dW, X=cx, W=cw, dY=cg)
+
+
 # -------------------------------------------------------------- MLP chain
 def mlp_fwd(X, W_up, W_down):
     """relu^2 MLP forward with dynamic tensorwise FP8 scaling.

@@ -74,3 +74,29 @@ def test_reference_arm_under_two_ranks_only_rank0_prints():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
     assert len(lines) == 1 and json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_clock_summary_counts_only_samples_inside_the_timed_region():
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.ClockSampler("GPU-none")
+    c.h, c.max_mhz = object(), 1965
+    c.samples = [(0.5, 1965, 200.0, 0), (1.5, 1500, 900.0, 0x4), (2.5, 1400, 1000.0, 0x4 | 0x8),
+                 (3.5, 1965, 210.0, 0)]
+    c.regions = [(1.0, 3.0)]
+    s = c.summary()
+    assert s["samples"] == 2 and s["sm_mhz"] == 1450 and s["sm_min_mhz"] == 1400
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"] and s["power_w_max"] == 1000.0
+
+
+def test_config_roofline_arithmetic():
+    """Roofline time of a GEMM set = FLOPs at the dense FP8 peak + cast bytes
+    at HBM bandwidth; 4.5 TFLOP and 8 GB take 1 ms each at 4.5 PF and 8 TB/s."""
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = dict(hbm=8000.0, bf16=2250.0, bf16_sus=2000.0)
+    e = bench.config_entry("x", 4.5e12, 8e9, 4.0, 3.0, 1.0, peaks, 1)
+    assert abs(e["roofline"]["ms_nominal"] - 2.0) < 1e-9
+    assert abs(e["roofline"]["frac_nominal"] - 0.5) < 1e-9
+    assert abs(e["roofline"]["frac_measured_peaks"] - 0.5) < 1e-9
+    assert abs(e["tflops"] - 1125.0) < 1e-6 and abs(e["pct_of_dense_fp8_peak"] - 25.0) < 1e-9

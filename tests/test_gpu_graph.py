@@ -1,5 +1,5 @@
 """The library allocates nothing and never synchronises the host, so a whole
-relu^2 MLP step (forward + backward, 16 kernels) can be captured once into a
+relu^2 MLP step (forward + backward, eleven kernels) can be captured once into a
 CUDA graph and replayed; replays must reproduce eager results bit for bit."""
 import pytest
 import torch

@@ -45,6 +45,12 @@ def T(codes):
     return np.ascontiguousarray(codes.T)
 
 
+def Td(view):
+    """The same transpose of a device code matrix, made on the device (a copy
+    of bytes, no arithmetic) and brought to the host."""
+    return u8(view.t().contiguous())
+
+
 def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None, wd_rows=None, wu_rows=None):
     """rows: sample of output rows to check for the M x * GEMMs (None = all);
     wd_rows / wu_rows: rows of dW_down / dW_up to check (default: all when rows
@@ -81,7 +87,7 @@ def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None, wd_rows=None, wu_ro
     # the backward's GEMMs read the row-major codes MN-major: the oracle gets
     # the K-major operands, i.e. the host transposes of those codes
     dH = u16(mlp.workspace_view("dH"))
-    dHref, _ = orc.gemm(dYq, E5M2, T(Wdq), E4M3, g[0, 2], sc[2, 2],
+    dHref, _ = orc.gemm(dYq, E5M2, Td(mlp.view("Wdq")), E4M3, g[0, 2], sc[2, 2],
                         orc.EPI_RELU2_BWD, aux=H, rows=rows)
     assert_close(dH if rows is None else dH[rows], dHref, "dH", ELEM_REL_RELU2_BWD)
     assert g[1, 0] == orc.amax(dH)
@@ -93,14 +99,16 @@ def check_stagewise(orc, mlp, t, Y, dX, dWu, dWd, rows=None, wd_rows=None, wu_ro
     wrows = wd_rows
     if wrows is None and rows is not None:
         wrows = np.arange(0, dWd.shape[0], max(1, dWd.shape[0] // 24))
-    ref_dWd, _ = orc.gemm(T(dYq), E5M2, T(hq), E4M3, g[0, 2], sc[3, 2], rows=wrows)
+    ref_dWd, _ = orc.gemm(Td(mlp.workspace_view("dYq")), E5M2, Td(mlp.view("hq")), E4M3,
+                          g[0, 2], sc[3, 2], rows=wrows)
     assert_close(u16(dWd) if wrows is None else u16(dWd)[wrows], ref_dWd, "dW_down")
-    ref_dX, _ = orc.gemm(dHq, E5M2, T(Wuq), E4M3, g[1, 2], sc[1, 2], rows=rows)
+    ref_dX, _ = orc.gemm(dHq, E5M2, Td(mlp.view("Wuq")), E4M3, g[1, 2], sc[1, 2], rows=rows)
     assert_close(u16(dX) if rows is None else u16(dX)[rows], ref_dX, "dX")
     urows = wu_rows
     if urows is None and rows is not None:
         urows = np.arange(0, dWu.shape[0], max(1, dWu.shape[0] // 24))
-    ref_dWu, _ = orc.gemm(T(dHq), E5M2, T(Xq), E4M3, g[1, 2], sc[0, 2], rows=urows)
+    ref_dWu, _ = orc.gemm(Td(mlp.workspace_view("dHq")), E5M2, Td(mlp.view("Xq")), E4M3,
+                          g[1, 2], sc[0, 2], rows=urows)
     assert_close(u16(dWu) if urows is None else u16(dWu)[urows], ref_dWu, "dW_up")
 
 
@@ -128,6 +136,15 @@ def test_mlp_ragged_shapes(orc, api):
     """M, d, f multiples of 16 but not of any tile: every GEMM and cast has a
     ragged tail."""
     w = synthetic.MlpWorkload("ragged", 272, 208, 848, True)
+    t, mlp, Y, dX, dWu, dWd = run_chain(api, w)
+    check_stagewise(orc, mlp, t, Y, dX, dWu, dWd)
+
+
+def test_mlp_small_model_dim(orc, api):
+    """d = 128: the dW_down GEMM (M = d rows) runs on the single-CTA kernel,
+    which carries no side warps, so the cast of dH runs as its own launch
+    after it; the codes must be the same bits either way."""
+    w = synthetic.MlpWorkload("d128", 512, 128, 512, True, seed=6)
     t, mlp, Y, dX, dWu, dWd = run_chain(api, w)
     check_stagewise(orc, mlp, t, Y, dX, dWu, dWd)
 

@@ -26,7 +26,7 @@ import torch
 
 from fp8_gemms_b200 import synthetic
 from gpu_util import assert_close, cast_ref, u8, u16
-from test_gpu_mlp import check_stagewise
+from test_gpu_mlp import Td, check_stagewise
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -75,12 +75,11 @@ def check_linear_layer(orc, api, t, layer, i):
     check_casts_equal(orc, sc[2], dYq, synthetic.bits_u16(dY), E5M2, what + " dY")
     rows = block_rows(X.shape[0], layer, i)
     wrows = block_rows(W.shape[0], layer, 100 + i)
-    T = lambda a: np.ascontiguousarray(a.T)
     ref_Y, _ = orc.gemm(Xq, E4M3, Wq, E4M3, sc[0, 2], sc[1, 2], rows=rows)
     assert_close(u16(Y)[rows], ref_Y, what + " Y")
-    ref_dX, _ = orc.gemm(dYq, E5M2, T(Wq), E4M3, sc[2, 2], sc[1, 2], rows=rows)
+    ref_dX, _ = orc.gemm(dYq, E5M2, Td(q["Wq"]), E4M3, sc[2, 2], sc[1, 2], rows=rows)
     assert_close(u16(dX)[rows], ref_dX, what + " dX")
-    ref_dW, _ = orc.gemm(T(dYq), E5M2, T(Xq), E4M3, sc[2, 2], sc[0, 2], rows=wrows)
+    ref_dW, _ = orc.gemm(Td(q["dYq"]), E5M2, Td(q["Xq"]), E4M3, sc[2, 2], sc[0, 2], rows=wrows)
     assert_close(u16(dW)[wrows], ref_dW, what + " dW")
 
 

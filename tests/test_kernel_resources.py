@@ -65,10 +65,15 @@ def test_no_kernel_spills(reports):
 
 def test_gemm_register_budget(reports):
     pair = {k: v for k, v in reports["lm_gemm.cu"].items() if "gemm_fp8_pair_kernel" in k}
-    # four public epilogues x (lean, multi-part split) + the gated epilogue
-    assert len(pair) == 9
+    # four public epilogues x (lean, multi-part split) + the gated epilogue, and
+    # the side-cast instantiations of the plain and relu^2-forward epilogues
+    assert len(pair) == 11
+    assert sum(re.search(r"ILi\d+ELb[01]ELb1EE", k) is not None for k in pair) == 2
     for name, (regs, _, _) in pair.items():
-        assert regs <= 255, (name, regs)
+        # 192 threads: the 255-register cap; 320 threads (side warps): the
+        # register file split evenly, 65536 / 320 rounded down to 8
+        side = re.search(r"ILi\d+ELb[01]ELb1EE", name) is not None  # <EPI, MULTI, SIDE=true>
+        assert regs <= (200 if side else 255), (name, regs)
 
 
 def test_cast_keeps_two_ctas_per_sm(reports):

@@ -252,3 +252,21 @@ def test_grad_accum_chain_matches_sum_of_per_micro_batch_gradients(orc):
     # the fp32 accumulator of one micro-batch equals the bf16 chain's wgrad to bf16 rounding
     dWu_bf = bf16_vals(bwd["dW_up"])
     assert np.all(np.abs(singles[0][1] - dWu_bf) <= 2.0 ** -8 * np.abs(dWu_bf) + 1e-30)
+
+
+def test_fp8_linear_within_fp8_error_of_f64(orc):
+    """The plain FP8 linear (forward, dgrad, wgrad) approaches the exact
+    Y = X W^T, dX = dY W, dW = dY^T X within FP8 error; a transposed or
+    swapped operand lands far outside it."""
+    M, K, N = 96, 128, 80
+    X = synthetic.normal_bf16((M, K), 1.0, 47, 0)
+    W = synthetic.normal_bf16((N, K), 0.02, 47, 1)
+    dY = synthetic.normal_bf16((M, N), 1e-3, 47, 2)
+    out = orc.linear_fwd_bwd(*(synthetic.bits_u16(t) for t in (X, W, dY)))
+    x, w, g = (t.double().numpy() for t in (X, W, dY))
+    v = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    rel = lambda got, r: np.linalg.norm(v(got) - r) / np.linalg.norm(r)
+    assert rel(out["Y"], x @ w.T) < 0.08
+    assert rel(out["dX"], g @ w) < 0.15
+    assert rel(out["dW"], g.T @ x) < 0.15
+    assert rel(out["dW"], (g.T @ x)[::-1]) > 0.5
