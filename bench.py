@@ -478,6 +478,7 @@ def time_steps(step, K, W, flush, cap):
     end.record()
     torch.cuda.synchronize()
     d = t.durations_ms(end)
+    assert len(t.kinds) == len(d) == t.n and t.n < cap, (len(t.kinds), len(d), t.n, cap)
     g = sum(x for x, kd in zip(d, t.kinds) if kd == "g")
     return ms, g, sum(d) - g
 
@@ -612,7 +613,7 @@ def run_configs(args, device, world, flush, host, dev, mlp, peaks, rank):
             mlp.backward(mt["dY"], dX=dev["dX"], dW_up=dev["dW_up"], dW_down=dev["dW_down"])
 
     K5 = max(1, min(K, args.stack_steps))
-    ms, g, o = time_steps(step5, K5, 1, flush, 1200)
+    ms, g, o = time_steps(step5, K5, 1, flush, 1400)
     ms = max_over_ranks(ms, world, device)
     per_layer_flops = (sum(6 * M_TOK * n * k for n, k in shapes) + 12 * M_TOK * D_MODEL * D_FF)
     cb = synthetic.N_LAYERS * (sum(linear_cast_bytes(M_TOK, n, k) for n, k in shapes) +

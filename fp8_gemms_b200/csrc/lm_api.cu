@@ -43,7 +43,7 @@ struct TimingState {
     void* const* events = nullptr;
     int capacity = 0;
     int count = 0;
-    char kinds[512];
+    char kinds[4096];  // labels of the first 4096 recorded launches
 };
 thread_local TimingState t_timing;
 }  // namespace

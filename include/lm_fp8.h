@@ -458,7 +458,8 @@ LM_API lm_status lm_get_error(lm_stream_t stream, uint32_t* where_out);
  * lm_timing_kinds() copies one character per recorded launch ('a' amax
  * reduction, 'c' cast, 's' scales only, 'g' GEMM, 'n' RMSNorm, 'w'
  * SwiGLU backward elementwise, 'e' softcapped CE, 'l' mean loss) into out[0..cap) and
- * returns how many it wrote.  State is per host thread.
+ * returns how many it wrote; labels are kept for the first 4096 launches
+ * after an attach.  State is per host thread.
  */
 LM_API void lm_timing_attach(void* const* events, int capacity);
 LM_API int lm_timing_detach(void);
