@@ -71,3 +71,34 @@ def test_nonfinite_input_to_the_mlp_is_reported():
     st, where = _lib.lm_get_error()
     assert _lib.STATUS[st] == "LM_ERR_NONFINITE" and where == 0x501
     assert _lib.lm_get_error() == (0, 0)
+
+
+@pytest.mark.parametrize("where_bad", ["W_down", "saved H"])
+def test_nonfinite_tensor_cast_beside_a_gemm_is_reported(where_bad):
+    """W_down's codes are written by side warps of the up GEMM's launch, and
+    dH's by side warps of the dW_down GEMM's launch.  A NaN in W_down (its
+    amax is NaN), or an infinity in the saved H (dH = g 2 relu(H) is then
+    infinite while dY is finite), is reported from there, and the scales
+    follow the formula."""
+    from fp8_gemms_b200 import _lib, api, synthetic
+    w = synthetic.TINY_MLP
+    t = {k: v.cuda() for k, v in w.tensors().items()}
+    if where_bad == "W_down":
+        t["W_down"][3, 7] = float("nan")
+    mlp = api.Relu2Mlp(w.M, w.d, w.f)
+    mlp.forward(t["X"], t["W_up"], t["W_down"])
+    if where_bad == "saved H":
+        assert _lib.lm_get_error() == (0, 0)
+        mlp.view("H")[:, 5] = float("inf")       # one whole column: some g there is nonzero
+        mlp.backward(t["dY"])
+    st, where = _lib.lm_get_error()
+    assert _lib.STATUS[st] == "LM_ERR_NONFINITE" and where == 0x501
+    assert _lib.lm_get_error() == (0, 0)
+    if where_bad == "W_down":
+        sc = mlp.view("scales").cpu()
+        assert torch.isnan(sc[2, 0]) and torch.isnan(sc[2, 1])
+    else:
+        # dH is +-inf (or NaN where g is exactly 0): a non-finite amax, and the
+        # scale the formula gives (57344 / inf = 0, or NaN)
+        g = mlp.workspace_view("scales").cpu()
+        assert not torch.isfinite(g[1, 0]) and (g[1, 1] == 0.0 or torch.isnan(g[1, 1]))
