@@ -626,10 +626,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
                                     grow, stream_policy, lane);
                 }
             } else {
+                // chunk c + 1's TMEM load is issued as soon as chunk c's values
+                // are computed, so it overlaps chunk c's staging and store
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tbase, r);
                 for (int c = 0; c < n_chunks; ++c) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tbase + (uint32_t)(c * EPI_COLS), r);
-                    tmem_ld_wait();
+                    tmem_ld_wait(r);
                     if (part) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
@@ -685,6 +687,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             packed[i] = epi_pair<EPI>(r[2 * i], r[2 * i + 1], s, hw[i], amax2);
+                        if (c + 1 < n_chunks)
+                            tmem_ld_32x32b_x32(tbase + (uint32_t)((c + 1) * EPI_COLS), r);
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
                             *reinterpret_cast<uint4*>(box + sw64(lane, j)) =
@@ -714,6 +718,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
                                             __fmul_rn(__uint_as_float(r[4 * j + 1]), s),
                                             __fmul_rn(__uint_as_float(r[4 * j + 2]), s),
                                             __fmul_rn(__uint_as_float(r[4 * j + 3]), s));
+                        if (c + 1 < n_chunks)
+                            tmem_ld_32x32b_x32(tbase + (uint32_t)((c + 1) * EPI_COLS), r);
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
@@ -726,6 +732,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             packed[i] = epi_pair<EPI>(r[2 * i], r[2 * i + 1], s, 0u, amax2);
+                        if (c + 1 < n_chunks)
+                            tmem_ld_32x32b_x32(tbase + (uint32_t)((c + 1) * EPI_COLS), r);
                         // staging buffer n_stores & 1: the store that last used it must
                         // have finished reading shared memory
                         uint8_t* dst = st_buf + (n_stores & 1u) * BOX_BYTES;
