@@ -286,12 +286,13 @@ constexpr int EPI_COLS = 32;                   // columns per epilogue chunk
 constexpr int BOX_BYTES = 32 * EPI_COLS * 2;   // one warp's 32 x 32 bf16 box
 constexpr int STORE_BYTES = NUM_EPI_WARPS * 2 * BOX_BYTES;
 constexpr int AUX_BYTES = NUM_EPI_WARPS * 2 * BOX_BYTES;
-// The relu^2 backward epilogue uses the store and aux areas together as a
-// ring of H_SLOTS boxes per warp: each saved-H box is loaded H_AHEAD chunks
-// before it is needed and its dH is staged in place for the TMA store.
-constexpr int H_SLOTS = 4;
-constexpr int H_AHEAD = H_SLOTS - 1;
-static_assert(NUM_EPI_WARPS * H_SLOTS * BOX_BYTES == STORE_BYTES + AUX_BYTES, "H ring layout");
+// The plain and relu^2 epilogues stage their bf16 output in boxes of 32 rows
+// x 64 columns (two 32-column chunks, 4 KB, 128-byte swizzle), two per warp in
+// the store and aux areas together.  The relu^2 backward loads each saved-H
+// box into the same slot and writes dH over it in place.
+constexpr int WIDE_COLS = 2 * EPI_COLS;
+constexpr int WIDE_BYTES = 32 * WIDE_COLS * 2;
+static_assert(NUM_EPI_WARPS * 2 * WIDE_BYTES == STORE_BYTES + AUX_BYTES, "wide box layout");
 // the accumulating epilogue stages 32 x 32 fp32 boxes (4 KB, two per warp) in
 // the store and aux areas together (contiguous, 32 KB)
 constexpr int ACC_BOX_BYTES = 32 * EPI_COLS * 4;
@@ -299,11 +300,10 @@ static_assert(NUM_EPI_WARPS * 2 * ACC_BOX_BYTES == STORE_BYTES + AUX_BYTES, "sta
 constexpr uint32_t TMEM_COLS = 2 * TILE_N;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + AUX_BYTES + 1024 + 512;
 
-// Offset of 16-byte chunk j of row r in a 32-row x 64-byte box written or
-// read by a TMA with CU_TENSOR_MAP_SWIZZLE_64B: chunk bits [4,6) are XORed
-// with address bits [7,9), i.e. with (r >> 1) & 3.
-__device__ __forceinline__ uint32_t sw64(int r, int j) {
-    return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+// Offset of 16-byte chunk j (0..7) of row r in a 32-row x 128-byte box of a
+// TMA with CU_TENSOR_MAP_SWIZZLE_128B: chunk bits [4,7) XORed with r & 7.
+__device__ __forceinline__ uint32_t sw128(int r, int j) {
+    return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4));
 }
 
 // MULTI: the instantiation launched when the split tail has three or more
@@ -331,8 +331,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
     uint64_t* tfull = empty + STAGES;       // [2], both CTAs
     uint64_t* tempty = tfull + 2;           // [2], leader only
     uint64_t* drain = tempty + 2;           // leader only
-    uint64_t* auxbar = drain + 1;           // [4 warps][H_SLOTS boxes]
-    uint64_t* splitbar = auxbar + H_SLOTS * NUM_EPI_WARPS;  // [4 warps]
+    uint64_t* auxbar = drain + 1;           // [4 warps][2 boxes]
+    uint64_t* splitbar = auxbar + 2 * NUM_EPI_WARPS;  // [4 warps]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(splitbar + NUM_EPI_WARPS);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -350,7 +350,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
             mbar_init(&tempty[a], 2 * NUM_EPI_WARPS);
         }
         mbar_init(drain, 1);
-        for (int i = 0; i < H_SLOTS * NUM_EPI_WARPS; ++i) mbar_init(&auxbar[i], 1);
+        for (int i = 0; i < 2 * NUM_EPI_WARPS; ++i) mbar_init(&auxbar[i], 1);
         for (int i = 0; i < NUM_EPI_WARPS; ++i) mbar_init(&splitbar[i], 1);
         fence_barrier_init();
     }
@@ -478,11 +478,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
         // ------------------------------------------- epilogue (both CTAs)
         const int wi = warp - 2;       // staging slot
         const int quarter = warp & 3;  // TMEM lanes this warp may access
-        uint8_t* st_buf = sStore + wi * 2 * BOX_BYTES;
-        // relu^2 backward: this warp's ring of saved-H boxes (dH staged in place)
-        uint8_t* h_ring = sStore + wi * H_SLOTS * BOX_BYTES;
-        uint64_t* h_bar = auxbar + wi * H_SLOTS;
-        uint32_t h_issued = 0, h_used = 0;  // H boxes loaded / consumed by this warp
+        // this warp's two 64-column boxes (plain and relu^2 epilogues), and,
+        // for the relu^2 backward, one barrier per box for its saved-H load
+        uint8_t* wide = sStore + wi * 2 * WIDE_BYTES;
+        uint64_t* h_bar = auxbar + wi * 2;
+        uint32_t h_issued = 0, h_used = 0;  // saved-H boxes loaded / consumed by this warp
+        uint32_t n_wide = 0;                // 64-column boxes stored by this warp
         const uint32_t tempty_leader = map_to_rank(smem_addr(tempty), 0);
         const uint64_t stream_policy = l2_policy_evict_first();  // D and H are touched once
         const float s = __fmul_rn(*args.inv_a, *args.inv_b);
@@ -509,25 +510,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
                 return (((size_t)(w.tile - args.split_first) * (size_t)(S - 1) + (size_t)p) * 2 +
                         rank) * NUM_EPI_WARPS + quarter;
             };
-            // relu^2 backward: load saved-H box j of this warp into ring slot
-            // j % H_SLOTS.  The dH store that last read that slot (box j -
-            // H_SLOTS) is at least the second most recent store, so waiting
-            // until at most one store is still reading shared memory frees it.
-            auto issue_h = [&](int chunk) {
-                const uint32_t slot = h_issued % H_SLOTS;
-                bulk_wait_group_read<1>();
+            // relu^2 backward: load saved-H box j (64 columns) of this warp
+            // into slot j & 1, once every store that read that slot has
+            // finished reading it
+            const int n_pairs = (n_chunks + 1) / 2;
+            auto issue_h = [&](int pair) {
+                const uint32_t slot = h_issued & 1u;
+                bulk_wait_group_read<0>();
                 fence_proxy_async_smem();
-                mbar_arrive_expect_tx(&h_bar[slot], BOX_BYTES);
-                tma_load_2d_hint(smem_addr(h_ring + slot * BOX_BYTES), &tmAux, &h_bar[slot],
-                                 gcol + chunk * EPI_COLS, grow, stream_policy);
+                mbar_arrive_expect_tx(&h_bar[slot], WIDE_BYTES);
+                tma_load_2d_hint(smem_addr(wide + slot * WIDE_BYTES), &tmAux, &h_bar[slot],
+                                 gcol + pair * WIDE_COLS, grow, stream_policy);
             };
             if constexpr (EPI == LM_EPI_RELU2_BWD) {
                 if (finishes) {
-                    // this tile's first H_AHEAD boxes arrive while its
-                    // accumulator is still being computed
-                    const int first = n_chunks < H_AHEAD ? n_chunks : H_AHEAD;
-                    for (int c = 0; c < first; ++c) {
-                        if (lane == 0) issue_h(c);
+                    // this tile's first two boxes arrive while its accumulator
+                    // is still being computed
+                    for (int q = 0; q < 2 && q < n_pairs; ++q) {
+                        if (lane == 0) issue_h(q);
                         ++h_issued;
                     }
                 }
@@ -664,20 +664,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
                     }
                     if constexpr (EPI == LM_EPI_RELU2_BWD) {
                         // saved H of this chunk (two bf16 per word, columns
-                        // 2i and 2i+1) from its ring slot; dH goes back into
-                        // the same slot (each lane rewrites only its own row)
-                        // and is TMA-stored from there
-                        const uint32_t slot = h_used % H_SLOTS;
-                        uint8_t* box = h_ring + slot * BOX_BYTES;
-                        if (!mbar_wait(&h_bar[slot], (h_used / H_SLOTS) & 1u, args.err, W_AUX)) {
-                            ok = false;
-                            break;
+                        // 2i and 2i+1) from its half of the pair's box; dH
+                        // goes back over it (each lane rewrites only its own
+                        // row) and the box is TMA-stored after its second half
+                        const int half = c & 1;
+                        const uint32_t slot = h_used & 1u;
+                        uint8_t* box = wide + slot * WIDE_BYTES;
+                        if (half == 0) {
+                            if (c >= 2 && c / 2 + 1 < n_pairs) {
+                                // the next pair's box goes into the slot whose
+                                // store was issued last
+                                if (lane == 0) issue_h(c / 2 + 1);
+                                ++h_issued;
+                            }
+                            if (!mbar_wait(&h_bar[slot], (h_used >> 1) & 1u, args.err, W_AUX)) {
+                                ok = false;
+                                break;
+                            }
                         }
-                        ++h_used;
                         uint32_t hw[16];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            const uint4 v = *reinterpret_cast<const uint4*>(box + sw64(lane, j));
+                            const uint4 v =
+                                *reinterpret_cast<const uint4*>(box + sw128(lane, 4 * half + j));
                             hw[4 * j] = v.x;
                             hw[4 * j + 1] = v.y;
                             hw[4 * j + 2] = v.z;
@@ -691,19 +700,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
                             tmem_ld_32x32b_x32(tbase + (uint32_t)((c + 1) * EPI_COLS), r);
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
-                            *reinterpret_cast<uint4*>(box + sw64(lane, j)) =
+                            *reinterpret_cast<uint4*>(box + sw128(lane, 4 * half + j)) =
                                 make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
                                            packed[4 * j + 3]);
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d_hint(&tmD, smem_addr(box), gcol + c * EPI_COLS, grow,
-                                              stream_policy);
-                            bulk_commit_group();
-                        }
-                        if (c + H_AHEAD < n_chunks) {
-                            if (lane == 0) issue_h(c + H_AHEAD);
-                            ++h_issued;
+                        if (half == 1 || c + 1 == n_chunks) {
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_2d_hint(&tmD, smem_addr(box), gcol + (c & ~1) * EPI_COLS,
+                                                  grow, stream_policy);
+                                bulk_commit_group();
+                            }
+                            ++h_used;
                         }
                     } else if constexpr (EPI == LM_EPI_ACCUM_F32) {
                         // fp32 partial -> 128B-swizzled 32 x 32 fp32 box -> TMA reduce-add
@@ -734,24 +742,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
                             packed[i] = epi_pair<EPI>(r[2 * i], r[2 * i + 1], s, 0u, amax2);
                         if (c + 1 < n_chunks)
                             tmem_ld_32x32b_x32(tbase + (uint32_t)((c + 1) * EPI_COLS), r);
-                        // staging buffer n_stores & 1: the store that last used it must
-                        // have finished reading shared memory
-                        uint8_t* dst = st_buf + (n_stores & 1u) * BOX_BYTES;
-                        if (lane == 0) bulk_wait_group_read<1>();
-                        __syncwarp();
+                        // box n_wide & 1: before its first half is written, the
+                        // store that last used it must have finished reading
+                        const int half = c & 1;
+                        uint8_t* box = wide + (n_wide & 1u) * WIDE_BYTES;
+                        if (half == 0) {
+                            if (lane == 0) bulk_wait_group_read<1>();
+                            __syncwarp();
+                        }
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
-                            *reinterpret_cast<uint4*>(dst + sw64(lane, j)) =
+                            *reinterpret_cast<uint4*>(box + sw128(lane, 4 * half + j)) =
                                 make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
                                            packed[4 * j + 3]);
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d_hint(&tmD, smem_addr(dst), gcol + c * EPI_COLS, grow,
-                                              stream_policy);
-                            bulk_commit_group();
+                        if (half == 1 || c + 1 == n_chunks) {
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_2d_hint(&tmD, smem_addr(box), gcol + (c & ~1) * EPI_COLS,
+                                                  grow, stream_policy);
+                                bulk_commit_group();
+                            }
+                            ++n_wide;
                         }
-                        ++n_stores;
                     }
                 }
             }
@@ -764,7 +777,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
         // H boxes still in flight (only after a wait ran out): let them land
         // (bounded) before the shared memory is released
         for (uint32_t j = h_used; j < h_issued; ++j)
-            mbar_wait(&h_bar[j % H_SLOTS], (j / H_SLOTS) & 1u, args.err, W_AUX);
+            mbar_wait(&h_bar[j & 1u], (j >> 1) & 1u, args.err, W_AUX);
         if (lane == 0) bulk_wait_group<0>();
         reduce_amax<EPI>(max(amax2 & 0xFFFFu, amax2 >> 16), args.amax_out, lane);
     }
@@ -1290,14 +1303,17 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
             (b_mn ? encode_tmap_u8(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)N, BK, 128)
                   : encode_tmap_u8(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)K, 128, BK));
         if (!mok) return LM_ERR_CUDA;
-        const bool dok = epi == LM_EPI_ACCUM_F32
-                             ? encode_tmap_f32_sw128(&td, D, (uint64_t)M, (uint64_t)N, 32,
-                                                     pair::EPI_COLS)
-                             : encode_tmap_bf16_sw64(&td, D, (uint64_t)M, (uint64_t)N, 32,
-                                                     pair::EPI_COLS);
+        // D: fp32 32 x 32 boxes (accumulating), bf16 32 x 32 (gated), bf16 32 x 64
+        // (plain and relu^2); the saved H like D
+        const bool dok =
+            epi == LM_EPI_ACCUM_F32
+                ? encode_tmap_f32_sw128(&td, D, (uint64_t)M, (uint64_t)N, 32, pair::EPI_COLS)
+            : epi == kEpiSwigluFwd
+                ? encode_tmap_bf16_sw64(&td, D, (uint64_t)M, (uint64_t)N, 32, pair::EPI_COLS)
+                : encode_tmap_bf16_sw128(&td, D, (uint64_t)M, (uint64_t)N, 32, pair::WIDE_COLS);
         if (!dok) return LM_ERR_CUDA;
         if (epi == LM_EPI_RELU2_BWD) {
-            if (!encode_tmap_bf16_sw64(&tx, aux, (uint64_t)M, (uint64_t)N, 32, pair::EPI_COLS))
+            if (!encode_tmap_bf16_sw128(&tx, aux, (uint64_t)M, (uint64_t)N, 32, pair::WIDE_COLS))
                 return LM_ERR_CUDA;
         } else {
             tx = td;  // unused

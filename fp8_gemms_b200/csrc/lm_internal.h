@@ -36,6 +36,11 @@ bool encode_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 bool encode_tmap_bf16_sw64(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                            uint32_t box_rows, uint32_t box_cols);
 
+// The same with the 128-byte swizzle (box_cols * 2 must be 128): the plain and
+// relu^2 epilogues' 32 x 64 boxes.
+bool encode_tmap_bf16_sw128(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                            uint32_t box_rows, uint32_t box_cols);
+
 // 2-D fp32 tensor map for a row-major [rows x cols] matrix, box
 // [box_rows x box_cols] with the 128-byte swizzle (box_cols * 4 must be 128);
 // used for the accumulating epilogue's TMA reduce-adds.
