@@ -554,7 +554,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
                 if (lane == 0) st_release_gpu(args.split_flags + slot_of(w.part), 1u);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_remote(tempty_leader + (uint32_t)(acc * 8));
+                if (lane == 0) mbar_arrive_remote_relaxed(tempty_leader + (uint32_t)(acc * 8));
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
                 continue;
@@ -770,7 +770,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(tempty_leader + (uint32_t)(acc * 8));
+            if (lane == 0) mbar_arrive_remote_relaxed(tempty_leader + (uint32_t)(acc * 8));
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }

@@ -232,9 +232,16 @@ __device__ __forceinline__ void cluster_sync() {
                      : "memory");
 }
 
-// arrive on an mbarrier in another CTA of the cluster (shared::cluster address)
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+// Arrive on an mbarrier in another CTA of the cluster (shared::cluster
+// address), relaxed: the arrive orders none of this thread's earlier memory
+// operations.  The only use is the epilogue's "accumulator drained" signal,
+// which carries no data in generic memory: every TMEM read it covers has
+// completed (tcgen05.wait::ld) and is fenced by tcgen05.fence::before_thread_sync
+// before the arrive.  A release at cluster scope here also waited for the
+// tile's TMA stores to drain, about 2.5k cycles per tile, which held back the
+// MMAs of short-K tiles.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                  : "memory");
 }
 
