@@ -85,15 +85,19 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const AmaxSet set) {
     int64_t i = (int64_t)(b - b0) * kThreads + threadIdx.x;
     if (ld == cols) {
         const uint4* xv = reinterpret_cast<const uint4*>(x);
-        // eight independent 16-byte loads in flight per thread
-        for (; i + 7 * stride < nvec; i += 8 * stride) {
+        // eight independent 16-byte loads in flight per thread, the last batch
+        // predicated (a vector past the end counts as zeros), so that a small
+        // tensor's few vectors per thread are fetched together, not one
+        // dependent load after another
+        for (; i < nvec; i += 8 * stride) {
             uint4 v[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = ld_stream_v4(xv + i + u * stride);
+            for (int u = 0; u < 8; ++u)
+                v[u] = i + u * stride < nvec ? ld_stream_v4(xv + i + u * stride)
+                                             : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int u = 0; u < 8; ++u) m = absmax8<RELU2>(v[u], m);
         }
-        for (; i < nvec; i += stride) m = absmax8<RELU2>(ld_stream_v4(xv + i), m);
     } else {
         for (; i < nvec; i += stride) {
             const int64_t r = i / vpr, c = (i - r * vpr) << 3;
@@ -281,13 +285,6 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
         reinterpret_cast<uint64_t*>(sIn + STAGES * IN_BYTES + (TRANS ? CODE_BYTES : 0));
     uint64_t* empty = full + STAGES;
 
-    const float fmax = FMT == LM_FP8_E4M3 ? 448.0f : 57344.0f;
-    float sc[kMaxSet] = {0.f, 0.f, 0.f};
-#pragma unroll
-    for (int j = 0; j < kMaxSet; ++j)
-        if (j < set.n)
-            write_scales(*set.amax_src[j], fmax, set.amax_out[j], set.scale_out[j], set.inv_out[j],
-                         &sc[j], err);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -328,6 +325,14 @@ __global__ void __launch_bounds__(tmac::THREADS) cast_tma_kernel(
     }
 
     // ---------------------------------------------------- consumers
+    // the scales, while the producer's first loads are in flight
+    const float fmax = FMT == LM_FP8_E4M3 ? 448.0f : 57344.0f;
+    float sc[kMaxSet] = {0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < kMaxSet; ++j)
+        if (j < set.n)
+            write_scales(*set.amax_src[j], fmax, set.amax_out[j], set.scale_out[j], set.inv_out[j],
+                         &sc[j], err);
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
