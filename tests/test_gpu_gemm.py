@@ -81,6 +81,7 @@ SHAPES = [
     (2304, 256, 256),   # 9 row-blocks of 256: one raster group spans M
     (4608, 512, 128),   # 18 row-blocks: groups of 8 plus a ragged last group
     (300, 1032, 1040),  # ragged everywhere, many tiles
+    (260, 296, 144),    # last column tile: 40 columns, two 32-column chunks in one 64-column box
 ]
 
 
@@ -98,12 +99,17 @@ def test_gemm_e4m3_e5m2(lib, orc):
     run(lib, orc, 256, 512, 256, fa=E4M3, fb=E5M2, inv_b=1e-4)
 
 
-@pytest.mark.parametrize("M,N,K", [(384, 768, 512), (200, 328, 208)])
+# (2048, 4096, 256): 128 tiles, so some CTA pairs take two and the epilogue's
+# box slots carry over from one tile to the next
+RELU2_SHAPES = [(384, 768, 512), (200, 328, 208), (260, 296, 144), (2048, 4096, 256)]
+
+
+@pytest.mark.parametrize("M,N,K", RELU2_SHAPES)
 def test_gemm_relu2_fwd_epilogue(lib, orc, M, N, K):
     run(lib, orc, M, N, K, epi=EPI_RELU2_FWD)
 
 
-@pytest.mark.parametrize("M,N,K", [(384, 768, 512), (200, 328, 208)])
+@pytest.mark.parametrize("M,N,K", RELU2_SHAPES)
 def test_gemm_relu2_bwd_epilogue(lib, orc, M, N, K):
     run(lib, orc, M, N, K, fa=E5M2, epi=EPI_RELU2_BWD, inv_a=1e-4)
 
