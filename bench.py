@@ -43,7 +43,7 @@ DENSE_FP8_PEAK_TFLOPS = 4500.0                 # public B200 dense FP8 figure
 PAGES_FP8_PEAK_TFLOPS = 4190.0                 # the dense FP8 peak the pages' MFU figure implies
 NOMINAL_FP8_OVER_BF16 = 2.0                    # 4.5 / 2.25 PFLOP/s dense
 WORKLOAD = "relu2 MLP fwd+dgrad+wgrad M=16384 d=3072 f=12288"
-LAUNCHES_PER_STEP = 11                         # kernels of ours per fwd+bwd: "acgcgacgggg"
+LAUNCHES_PER_STEP = 10                         # kernels of ours per fwd+bwd: "acggacgggg"
 
 # DRAM traffic of one GEMM launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum), valid only for the kernel source it was taken on;
@@ -198,13 +198,13 @@ def job_tflops(world, steps, flops_per_step, total_ms):
 # algorithmic bytes of the cast launches of one step: a full cast (amax pass +
 # cast pass) moves 2 B (amax read) + 2 B (read) + 1 B (codes) per element; a
 # cast whose amax came from a GEMM epilogue 2 + 1 B.  The launches: the amax
-# of X, W_up and W_down; the casts of X and W_up; the cast of h; the amax and
-# cast of dY.  W_down's codes (3 B/element after its amax) and dH's cast run
-# in side warps of the up GEMM and of the dW_down GEMM, inside those launches.
+# of X, W_up and W_down; the casts of X and W_up; the amax and cast of dY.
+# W_down's codes, h's and dH's (3 B/element each after their amax) are cast
+# by side warps of the up, down and dW_down GEMMs, inside those launches.
 # Only row-major codes are written: the backward's GEMMs read them MN-major.
 def cast_bytes():
-    Md, fd, Mf = M_TOK * D_MODEL, D_FF * D_MODEL, M_TOK * D_FF
-    return [5 * Md, 5 * fd, 2 * fd, 3 * Mf, 5 * Md]
+    Md, fd = M_TOK * D_MODEL, D_FF * D_MODEL
+    return [5 * Md, 5 * fd, 2 * fd, 5 * Md]
 
 
 def src_sha(path):

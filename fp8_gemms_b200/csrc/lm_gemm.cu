@@ -43,7 +43,7 @@ constexpr int NUM_THREADS_SIDE = NUM_THREADS + 32 * SIDE_WARPS;
 // codes recorded in the device error word when a bounded wait runs out
 enum : unsigned {
     W_EMPTY = 0x101, W_TEMPTY = 0x102, W_FULL = 0x103, W_DRAIN = 0x104, W_TFULL = 0x105,
-    W_LOADS = 0x106, W_AUX = 0x107, W_SPLIT = 0x108, W_SPLIT_LOAD = 0x109
+    W_LOADS = 0x106, W_AUX = 0x107, W_SPLIT = 0x108, W_SPLIT_LOAD = 0x109, W_SIDE_READY = 0x10A
 };
 
 // Split-K tail.  Tiles go round-robin to the persistent clusters, so a last
@@ -97,6 +97,16 @@ struct GemmArgs {
     int side_fmt;
     const float* side_amax_in;
     float *side_amax_out, *side_scale_out, *side_inv_out;
+    // side cast that produces this GEMM's own A (side_ready != nullptr): the
+    // side warps cast A's bf16 source [M x K] (relu^2 first if side_relu2) in
+    // units of 256 rows x 128 columns, in the order the tiles consume them,
+    // and set bit kb % 32 of side_ready[mb * side_ready_words + kb / 32] once
+    // unit (mb, kb) is stored; the producer loads an A box only after its bit
+    // is set, and the epilogue takes A's scale from side_amax_in
+    unsigned int* side_ready;
+    int side_ready_words;
+    int side_relu2;
+    int side_cols;
 };
 
 // The side cast's loop for one format: eight 16-byte loads in flight per
@@ -118,6 +128,92 @@ __device__ __forceinline__ void side_cast_loop(const GemmArgs& a, int64_t t, int
     for (; i < n; i += nt) q[i] = convert8<FMT, false>(ld_stream_v4(x + i), scale);
 }
 
+// Unit i of a side cast that feeds A -> its row block mb and k-block kb.  With
+// one tile group per row block (group_m == 1) row block mb's first tile falls
+// in round (mb * num_nb) / C of the C clusters; the units go round by round,
+// k-block-major within a round over that round's row blocks, and an odd
+// round's k-blocks backward, as its tiles walk K.  Otherwise k-block-major
+// over all row blocks.  Any order is correct (the producer waits for each
+// unit); this one casts a unit shortly before its first tile needs it.
+__device__ __forceinline__ void side_unit(int64_t i, const GemmArgs& a, int C, int& mb, int& kb) {
+    const int nkb = a.num_kb, nmb = a.num_mb, nnb = a.num_nb;
+    if (a.group_m != 1) {
+        kb = (int)(i / nmb);
+        mb = (int)(i - (int64_t)kb * nmb);
+        return;
+    }
+    const int v = (int)(i / nkb);
+    const int r = (int)((int64_t)v * nnb / C);
+    const int first = (int)(((int64_t)r * C + nnb - 1) / nnb);
+    int next = (int)(((int64_t)(r + 1) * C + nnb - 1) / nnb);
+    if (next > nmb) next = nmb;
+    const int64_t local = i - (int64_t)first * nkb;
+    const int n = next - first;
+    kb = (int)(local / n);
+    mb = first + (int)(local - (int64_t)kb * n);
+    if (r & 1) kb = nkb - 1 - kb;
+}
+
+// A side cast that feeds A: the side warps of CTA `cta` (thread t of 128)
+// take units cta, cta + ncta, ...; 8 rows x 16 vectors of a unit per step,
+// eight steps in flight per thread.  The side warps meet at named barrier 1
+// after a unit's stores; thread 0 then fences and publishes the unit's bit.
+template <int FMT, bool RELU2>
+__device__ __forceinline__ void side_cast_units(const GemmArgs& a, int cta, int ncta, int t,
+                                                int C, float scale) {
+    const uint16_t* x = static_cast<const uint16_t*>(static_cast<const void*>(a.side_x));
+    uint8_t* q = reinterpret_cast<uint8_t*>(a.side_q);
+    const int64_t M = a.M, K = a.side_cols;
+    const int64_t total = (int64_t)a.num_mb * a.num_kb;
+    const int rr = t >> 4, v = t & 15;
+    for (int64_t i = cta; i < total; i += ncta) {
+        int mb, kb;
+        side_unit(i, a, C, mb, kb);
+        const int64_t col = (int64_t)kb * 128 + v * 8;
+        const int64_t row0 = (int64_t)mb * 256 + rr;
+#pragma unroll 1
+        for (int b = 0; b < 4; ++b) {
+            uint4 val[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t r = row0 + 8 * (8 * b + u);
+                val[u] = (r < M && col < K) ? ld_stream_v4(x + r * K + col)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t r = row0 + 8 * (8 * b + u);
+                if (r < M && col < K)
+                    *reinterpret_cast<uint2*>(q + r * K + col) = convert8<FMT, RELU2>(val[u], scale);
+            }
+        }
+        // every side thread's stores, then (thread 0) a fence and the bit
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * SIDE_WARPS) : "memory");
+        if (t == 0) {
+            __threadfence();
+            atomicOr(a.side_ready + (int64_t)mb * a.side_ready_words + (kb >> 5), 1u << (kb & 31));
+        }
+    }
+}
+
+// Wait until bit `bit` of *word is set (acquire), for at most kWaitLimitNs;
+// returns the word, or 0 after recording `where` in the error word.
+__device__ __forceinline__ uint32_t ready_wait(const unsigned int* word, uint32_t bit,
+                                               unsigned int* err, unsigned int where) {
+    uint32_t v = ld_acquire_gpu(word);
+    if (v & bit) return v;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        __nanosleep(64);
+        v = ld_acquire_gpu(word);
+        if (v & bit) return v;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            atomicCAS(err, 0u, where);
+            return 0u;
+        }
+    }
+}
+
 // The side cast, run by the side warps of every CTA (thread t of nt): the
 // scale from the already-reduced amax, the scale block (thread 0), the codes.
 // A NaN or infinite amax records kErrNonfiniteAmax, as the cast kernels do.
@@ -130,6 +226,20 @@ __device__ __forceinline__ void side_cast_run(const GemmArgs& a, int64_t t, int6
         *a.side_scale_out = scale;
         *a.side_inv_out = __fdiv_rn(1.0f, scale);
         if (!(amax <= 3.40282347e38f)) atomicCAS(a.err, 0u, kErrNonfiniteAmax);
+    }
+    if (a.side_ready) {
+        constexpr int kT = 32 * SIDE_WARPS;
+        const int cta = (int)(t / kT), ncta = (int)(nt / kT), lt = (int)(t - (int64_t)cta * kT);
+        const int C = ncta / 2;
+        if (e4 && a.side_relu2)
+            side_cast_units<LM_FP8_E4M3, true>(a, cta, ncta, lt, C, scale);
+        else if (e4)
+            side_cast_units<LM_FP8_E4M3, false>(a, cta, ncta, lt, C, scale);
+        else if (a.side_relu2)
+            side_cast_units<LM_FP8_E5M2, true>(a, cta, ncta, lt, C, scale);
+        else
+            side_cast_units<LM_FP8_E5M2, false>(a, cta, ncta, lt, C, scale);
+        return;
     }
     if (e4)
         side_cast_loop<LM_FP8_E4M3>(a, t, nt, scale);
@@ -382,6 +492,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
             int stage = 0;
             uint32_t phase = 0, issued = 0;
             bool ok = true;
+            uint32_t rword = 0;  // side cast feeding A: the last ready word read
+            int rkey = -1;       // and its index
             for (int u = cluster, round = 0; u < args.num_units && ok;
                  u += nclusters, ++round) {
                 const WorkUnit w = work_unit<MULTI>(u, args);
@@ -398,6 +510,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
                     if (!mbar_wait(&empty[stage], phase ^ 1u, args.err, W_EMPTY)) {
                         ok = false;
                         break;
+                    }
+                    if (args.side_ready) {
+                        // A's unit (mb, kb) is stored by the side warps
+                        const int key = mb * args.side_ready_words + (kb >> 5);
+                        const uint32_t bit = 1u << (kb & 31);
+                        if (key != rkey || !(rword & bit)) {
+                            rkey = key;
+                            rword = ready_wait(args.side_ready + key, bit, args.err, W_SIDE_READY);
+                            if (!(rword & bit)) {
+                                ok = false;
+                                break;
+                            }
+                            fence_proxy_async_global();  // the acquired codes, then the TMA read
+                        }
                     }
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
                     const uint32_t bar = full_leader + (uint32_t)(stage * 8);
@@ -486,7 +612,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
         uint32_t n_wide = 0;                // 64-column boxes stored by this warp
         const uint32_t tempty_leader = map_to_rank(smem_addr(tempty), 0);
         const uint64_t stream_policy = l2_policy_evict_first();  // D and H are touched once
-        const float s = __fmul_rn(*args.inv_a, *args.inv_b);
+        // A's scale: from its amax when the side warps are still writing the
+        // scale block (side cast feeding A), with the cast's own arithmetic
+        const float inv_a =
+            args.side_ready
+                ? __fdiv_rn(1.0f, scale_from_amax(*args.side_amax_in,
+                                                  args.side_fmt == LM_FP8_E4M3 ? 448.0f : 57344.0f))
+                : *args.inv_a;
+        const float s = __fmul_rn(inv_a, *args.inv_b);
         uint32_t amax2 = 0;  // two bf16-bit halves of the running max
         int acc = 0;
         uint32_t acc_phase = 0;
@@ -1036,10 +1169,21 @@ lm_status launch_pair_as(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
     if (sms < 2) return LM_ERR_CUDA;
     const int clusters = a.num_units < sms / 2 ? a.num_units : sms / 2;
     timing_mark(s, 'g');
-    if (a.split_flags && a.split_slots > 0 &&
-        cudaMemsetAsync(a.split_flags, 0,
-                        (size_t)a.split_slots * 2 * NUM_EPI_WARPS * sizeof(unsigned int),
-                        s) != cudaSuccess)
+    // the split tail's flags and, right after them, a fed A's ready bits:
+    // one memset
+    uint8_t* zero_at = nullptr;
+    size_t zero_bytes = 0;
+    if (a.split_flags && a.split_slots > 0) {
+        zero_at = reinterpret_cast<uint8_t*>(a.split_flags);
+        zero_bytes = (size_t)a.split_slots * 2 * NUM_EPI_WARPS * sizeof(unsigned int);
+    }
+    if (a.side_ready) {
+        uint8_t* r = reinterpret_cast<uint8_t*>(a.side_ready);
+        if (!zero_at) zero_at = r;
+        zero_bytes = (size_t)(r - zero_at) +
+                     (size_t)a.num_mb * (size_t)a.side_ready_words * sizeof(unsigned int);
+    }
+    if (zero_bytes && cudaMemsetAsync(zero_at, 0, zero_bytes, s) != cudaSuccess)
         return LM_ERR_CUDA;
     pair::gemm_fp8_pair_kernel<EPI, MULTI, SIDE>
         <<<2 * clusters, SIDE ? NUM_THREADS_SIDE : NUM_THREADS, pair::SMEM_BYTES, s>>>(
@@ -1164,7 +1308,7 @@ namespace {
 lm_status side_cast_alone(const SideCast& sc, cudaStream_t s) {
     const CastItem it = {sc.x, sc.rows, sc.cols, sc.cols, sc.amax_in, sc.amax_out,
                          sc.scale_out, sc.inv_scale_out, sc.q, nullptr};
-    return cast_set(&it, 1, sc.fmt, 0, true, s);
+    return cast_set(&it, 1, sc.fmt, sc.relu2 ? 1 : 0, true, s);
 }
 
 }  // namespace
@@ -1184,6 +1328,9 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
             ((side->rows > 0 && side->cols > 0) && (!side->x || !side->q)))
             return LM_ERR_INVALID_ARG;
         if (!aligned16(side->x) || !aligned16(side->q)) return LM_ERR_ALIGNMENT;
+        if (side->feeds_a && (side->q != A || side->rows != M || side->cols != K ||
+                              side->fmt != fa || (flags & LM_GEMM_A_MN_MAJOR)))
+            return LM_ERR_INVALID_ARG;
         if (side->rows == 0 || side->cols == 0) side = nullptr;  // nothing to cast
     }
     if ((fa != LM_FP8_E4M3 && fa != LM_FP8_E5M2) || (fb != LM_FP8_E4M3 && fb != LM_FP8_E5M2))
@@ -1237,6 +1384,10 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
     a.side_fmt = 0;
     a.side_amax_in = nullptr;
     a.side_amax_out = a.side_scale_out = a.side_inv_out = nullptr;
+    a.side_ready = nullptr;
+    a.side_ready_words = 0;
+    a.side_relu2 = 0;
+    a.side_cols = 0;
     if (side) {
         a.side_x = static_cast<const uint4*>(side->x);
         a.side_q = reinterpret_cast<uint2*>(side->q);
@@ -1246,6 +1397,8 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
         a.side_amax_out = side->amax_out;
         a.side_scale_out = side->scale_out;
         a.side_inv_out = side->inv_scale_out;
+        a.side_relu2 = side->relu2 ? 1 : 0;
+        a.side_cols = (int)side->cols;
     }
 
     CUtensorMap ta, tb;
@@ -1292,6 +1445,29 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
             a.split_ws = static_cast<float4*>(workspace);
             a.split_flags = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) +
                                                             slots * kSplitTileBytes);
+        }
+        if (side && side->feeds_a) {
+            // A cast by the side warps ahead of the tiles: only where the launch
+            // has side warps (no multi-part split) and the workspace holds the
+            // units' ready bits after the split tail's flags; otherwise A is
+            // cast by its own launch first
+            const bool side_warps = (epi == LM_EPI_NONE || epi == LM_EPI_RELU2_FWD) &&
+                                    a.split_parts <= 2 &&
+                                    a.num_units - a.split_first <= a.split_round;
+            const size_t used =
+                (size_t)a.split_slots * (kSplitTileBytes + 2 * NUM_EPI_WARPS * sizeof(unsigned int));
+            const int words = (a.num_kb + 31) / 32;
+            const size_t need = used + (size_t)a.num_mb * (size_t)words * sizeof(unsigned int);
+            if (side_warps && workspace && aligned16(workspace) && ws_bytes >= need) {
+                a.side_ready =
+                    reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + used);
+                a.side_ready_words = words;
+            } else {
+                const lm_status cs = side_cast_alone(*side, s);
+                if (cs != LM_OK) return cs;
+                side = nullptr;
+                a.side_nvec = 0;
+            }
         }
         a.idesc = idesc_f8((uint32_t)fa, (uint32_t)fb, pair::TILE_M, pair::TILE_N, a.a_mn, a.b_mn);
         CUtensorMap td, tx;
@@ -1341,6 +1517,11 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
         }
         if (st != LM_OK || side_done || !side) return st;
         return side_cast_alone(*side, s);
+    }
+    if (side && side->feeds_a) {  // the thin kernel has no side warps: A first
+        const lm_status cs = side_cast_alone(*side, s);
+        if (cs != LM_OK) return cs;
+        side = nullptr;
     }
     a.num_mb = (int)((M + one::BM - 1) / one::BM);
     a.num_nb = (int)((N + one::BN - 1) / one::BN);

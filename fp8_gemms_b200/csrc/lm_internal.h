@@ -73,6 +73,13 @@ struct SideCast {
     const float* amax_in;
     float *amax_out, *scale_out, *inv_scale_out;
     uint8_t* q;  // [rows x cols] codes
+    int relu2 = 0;    // cast h = bf16(relu(x)^2) instead of x
+    // The codes are the GEMM's own A ([M x K], K-major, format fa, q == A):
+    // the side warps cast it unit by unit ahead of the tiles that read it,
+    // and the inverse scale A is dequantised with comes from amax_in.
+    // Without a workspace to hold the units' ready bits, or where the
+    // launch has no side warps, the cast runs as its own launch first.
+    int feeds_a = 0;
 };
 
 // lm_fp8_gemm_ex with the internal epilogues, a second output and an

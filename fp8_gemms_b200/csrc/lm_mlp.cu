@@ -144,11 +144,17 @@ lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_dow
     LM_TRY(lm::gemm_dispatch(sv->Xq, LM_FP8_E4M3, sv->Wuq, LM_FP8_E4M3, M, f, d, 0u, S + S_X + 2,
                              S + S_WU + 2, LM_EPI_RELU2_FWD, nullptr, sv->H, nullptr, S + S_H,
                              split, sb, stream, reuse ? nullptr : &wd));
-    LM_TRY(lm_fp8_amax_scale_cast(sv->H, M, f, f, LM_FP8_E4M3, 1, S + S_H, S + S_H, S + S_H + 1,
-                                  S + S_H + 2, sv->hq, nullptr, stream));
-    // Y = h W_down^T
-    LM_TRY(lm_fp8_gemm_ex(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, 0u, S + S_H + 2,
-                          S + S_WD + 2, LM_EPI_NONE, nullptr, Y, nullptr, split, sb, stream));
+    // Y = h W_down^T, with h = bf16(relu(H)^2) cast to its codes (the amax came
+    // from the up GEMM's epilogue) by the down GEMM's side warps, unit by unit
+    // ahead of the tiles that read them (its own launch first where that
+    // cannot be done: no workspace, a thin M or a multi-part split tail)
+    lm::SideCast hc = {sv->H, M, f, LM_FP8_E4M3, S + S_H, S + S_H, S + S_H + 1, S + S_H + 2,
+                       sv->hq};
+    hc.relu2 = 1;
+    hc.feeds_a = 1;
+    LM_TRY(lm::gemm_dispatch(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, 0u, S + S_H + 2,
+                             S + S_WD + 2, LM_EPI_NONE, nullptr, Y, nullptr, nullptr, split, sb,
+                             stream, &hc));
     return LM_OK;
 }
 

@@ -187,3 +187,23 @@ def test_full_size_mlp_forward_only_sampled(orc, api):
     t, mlp, Y, *_ = run_chain(api, w)
     rows = np.sort(np.random.default_rng(2).choice(w.M, 32, replace=False))
     check_stagewise(orc, mlp, t, Y, None, None, None, rows=rows)
+
+
+@pytest.mark.parametrize("workspace", [True, False])
+@pytest.mark.parametrize("M,d,f", [(512, 256, 1024), (4096, 512, 2048), (1168, 256, 1040)])
+def test_mlp_forward_h_cast_in_down_gemm_or_own_launch(orc, api, M, d, f, workspace):
+    """With a workspace, h is cast by the down GEMM's side warps, unit by unit
+    ahead of the tiles that read it (several units per CTA, ragged last row
+    block and k-block at (1168, 1040)); without one, by its own launch before
+    the GEMM.  Either way: casts bit-exact, the GEMMs within tolerance."""
+    from fp8_gemms_b200 import _lib
+    w = synthetic.MlpWorkload("h cast placement", M, d, f, False, ("t3", None), 11)
+    t = w.tensors()
+    dev = {k: v.cuda() for k, v in t.items()}
+    mlp = api.Relu2Mlp(M, d, f)
+    Y = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    _lib.lm_relu2_mlp_fwd(dev["X"], dev["W_up"], dev["W_down"], Y, mlp.saved,
+                          workspace=mlp.workspace if workspace else None)
+    torch.cuda.synchronize()
+    assert _lib.lm_get_error()[0] == 0
+    check_stagewise(orc, mlp, t, Y, None, None, None)
