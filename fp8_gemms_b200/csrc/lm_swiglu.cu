@@ -191,10 +191,14 @@ lm_status lm_swiglu_mlp_fwd(const void* X, const void* W_gu, const void* W_down,
         LM_TRY(gemm_dispatch(sv->Xq, LM_FP8_E4M3, sv->Wguq, LM_FP8_E4M3, M, 2 * f, d, 0u,
                              S + S_X + 2, S + S_WGU + 2, kEpiSwigluFwd, nullptr, sv->GU, sv->h,
                              S + S_H, nullptr, 0, stream));
-    LM_TRY(lm_fp8_amax_scale_cast(sv->h, M, f, f, LM_FP8_E4M3, 0, S + S_H, S + S_H, S + S_H + 1,
-                                  S + S_H + 2, sv->hq, nullptr, stream));
-    LM_TRY(lm_fp8_gemm_ex(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, 0u, S + S_H + 2,
-                          S + S_WD + 2, LM_EPI_NONE, nullptr, Y, nullptr, split, sb, stream));
+    // Y = h W_down^T, h's codes cast (amax from the epilogue above) by the down
+    // GEMM's side warps unit by unit ahead of its tiles, or by their own launch
+    // first where that cannot be done
+    SideCast hc = {sv->h, M, f, LM_FP8_E4M3, S + S_H, S + S_H, S + S_H + 1, S + S_H + 2, sv->hq};
+    hc.feeds_a = 1;
+    LM_TRY(gemm_dispatch(sv->hq, LM_FP8_E4M3, sv->Wdq, LM_FP8_E4M3, M, d, f, 0u, S + S_H + 2,
+                         S + S_WD + 2, LM_EPI_NONE, nullptr, Y, nullptr, nullptr, split, sb,
+                         stream, &hc));
     return LM_OK;
 }
 
@@ -238,12 +242,14 @@ lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* sv, int64_t M
             static_cast<uint16_t*>(w.dGU), reinterpret_cast<unsigned int*>(G + S_DGU));
         if (launch_status() != LM_OK) return LM_ERR_CUDA;
     }
-    LM_TRY(lm_fp8_amax_scale_cast(w.dGU, M, 2 * f, 2 * f, LM_FP8_E5M2, 0, G + S_DGU, G + S_DGU,
-                                  G + S_DGU + 1, G + S_DGU + 2, w.dGUq, nullptr, stream));
-    // dX = dGU W_gu (K = 2f);  dW_gu = dGU^T X (K = M)
-    LM_TRY(lm_fp8_gemm_ex(w.dGUq, LM_FP8_E5M2, sv->Wguq, LM_FP8_E4M3, M, d, 2 * f, B_MN,
-                          G + S_DGU + 2, S + S_WGU + 2, LM_EPI_NONE, nullptr, dX, nullptr, w.split,
-                          sb, stream));
+    // dX = dGU W_gu (K = 2f), dGU's codes (amax from the elementwise kernel)
+    // cast by the GEMM's side warps ahead of its tiles;  dW_gu = dGU^T X (K = M)
+    SideCast gc = {w.dGU, M, 2 * f, LM_FP8_E5M2, G + S_DGU, G + S_DGU, G + S_DGU + 1,
+                   G + S_DGU + 2, w.dGUq};
+    gc.feeds_a = 1;
+    LM_TRY(gemm_dispatch(w.dGUq, LM_FP8_E5M2, sv->Wguq, LM_FP8_E4M3, M, d, 2 * f, B_MN,
+                         G + S_DGU + 2, S + S_WGU + 2, LM_EPI_NONE, nullptr, dX, nullptr, nullptr,
+                         w.split, sb, stream, &gc));
     LM_TRY(lm_fp8_gemm_ex(w.dGUq, LM_FP8_E5M2, sv->Xq, LM_FP8_E4M3, 2 * f, d, M, AB_MN,
                           G + S_DGU + 2, S + S_X + 2, LM_EPI_NONE, nullptr, dW_gu, nullptr,
                           w.split, sb, stream));
