@@ -35,6 +35,10 @@ struct Ws {
     uint8_t *Wq, *Xq, *dLq;
     uint16_t* logits;
     float* loss_rows;
+    // the dX GEMM's ready bits, one per 256-row x 128-column unit of the
+    // dlogits codes that its side warps cast ahead of its tiles
+    unsigned int* ready;
+    size_t ready_bytes;
 };
 
 size_t layout(int64_t M, int64_t d, int64_t V, int64_t C, uint8_t* base, Ws* w) {
@@ -50,7 +54,9 @@ size_t layout(int64_t M, int64_t d, int64_t V, int64_t C, uint8_t* base, Ws* w) 
     o.Xq = take((size_t)C * d);
     o.logits = reinterpret_cast<uint16_t*>(take((size_t)C * V * 2));
     o.dLq = take((size_t)C * V);
-    o.loss_rows = reinterpret_cast<float*>(take((size_t)M * sizeof(float)));
+    o.ready_bytes = (size_t)((C + 255) / 256) * (size_t)((((V + 127) / 128) + 31) / 32) * 4;
+    o.ready = reinterpret_cast<unsigned int*>(take(o.ready_bytes));
+    o.loss_rows = reinterpret_cast<float*>(take((size_t)M * sizeof(float)));  // the tail
     if (w) *w = o;
     return off;
 }
@@ -354,12 +360,15 @@ lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* labels, 
                 w.logits, labels + c0, (int)V, softcap, (float)(1.0 / (double)M),
                 w.loss_rows + c0, reinterpret_cast<unsigned int*>(SL), err);
         if (launch_status() != LM_OK) return LM_ERR_CUDA;
-        LM_TRY(lm_fp8_amax_scale_cast(w.logits, rows, V, V, LM_FP8_E5M2, 0, SL, SL, SL + 1,
-                                      SL + 2, w.dLq, nullptr, stream));
-        // dX = dL W (W [V x d] read MN-major); dW += dL^T X (both read MN-major)
-        LM_TRY(lm_fp8_gemm_ex(w.dLq, LM_FP8_E5M2, w.Wq, LM_FP8_E4M3, rows, d, V,
-                              LM_GEMM_B_MN_MAJOR, SL + 2, SW + 2, LM_EPI_NONE, nullptr,
-                              dXb + c0 * d, nullptr, nullptr, 0, stream));
+        // dX = dL W (W [V x d] read MN-major), dL's codes cast by the GEMM's side
+        // warps unit by unit ahead of its tiles (the workspace holds only their
+        // ready bits, so no split tail); dW += dL^T X (both read MN-major)
+        SideCast lc = {w.logits, rows, V, LM_FP8_E5M2, SL, SL, SL + 1, SL + 2, w.dLq};
+        lc.feeds_a = 1;
+        LM_TRY(gemm_dispatch(w.dLq, LM_FP8_E5M2, w.Wq, LM_FP8_E4M3, rows, d, V,
+                             LM_GEMM_B_MN_MAJOR, SL + 2, SW + 2, LM_EPI_NONE, nullptr,
+                             dXb + c0 * d, nullptr, nullptr, w.ready, w.ready_bytes, stream,
+                             &lc));
         LM_TRY(lm_fp8_gemm_ex(w.dLq, LM_FP8_E5M2, w.Xq, LM_FP8_E4M3, V, d, rows,
                               LM_GEMM_A_MN_MAJOR | LM_GEMM_B_MN_MAJOR, SL + 2, SX + 2,
                               LM_EPI_ACCUM_F32, nullptr, dW, nullptr, nullptr, 0, stream));
