@@ -178,10 +178,12 @@ __global__ void __launch_bounds__(kCeThreads)
 // y = l / c: then tanh(y) = 1 - 2r, z = c - 2cr, exp(z - c) = exp(-2cr) and
 // the softcap's derivative 1 - tanh(y)^2 = 4r(1 - r).  Every term exp(z - c)
 // is at most 1, so the row's log-sum-exp needs no running maximum:
-// lse = c + log(sum exp(-2cr)).  Per logit and pass that is three hardware
-// transcendentals (two base-2 exponentials and a reciprocal) instead of a
-// division, tanhf and expf.  Used for softcaps up to kFastCeMaxCap, where
-// exp(-2c) stays a normal fp32 number (no term can flush to zero).
+// lse = c + log(sum exp(-2cr)).  Per logit and pass that is two hardware
+// transcendentals (a base-2 exponential and a reciprocal) and one base-2
+// exponential on the FMA pipe (ex2_fma) instead of a division, tanhf and expf.  Used for softcaps up to kFastCeMaxCap, where
+// exp(-2c) stays a normal fp32 number (no term can flush to zero) and the
+// exponent of every exp(z - c) term lies in [-2 log2(e) kFastCeMaxCap, 0] =
+// [-115.4, 0], inside the range of ex2_fma.
 constexpr float kFastCeMaxCap = 40.0f;
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -194,6 +196,77 @@ __device__ __forceinline__ float rcp_approx(float x) {
     float y;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Two fp32 lanes in one 64-bit register, and the packed f32x2 arithmetic of
+// sm_100 on them: each lane is one IEEE round-to-nearest operation, exactly
+// the scalar __fadd_rn / __fsub_rn / __fmul_rn / __fmaf_rn, at half the
+// instructions.
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void up2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// 2^x for x in [-116, 0] on the FMA and integer pipes, two lanes at a time.
+// x = n + f with n = rint(x) and f in [-1/2, 1/2]: adding 1.5 * 2^23 + 127
+// leaves n + 127 in the sum's low bits, which shifted into the exponent field
+// are the bits of 2^n; 2^f from a degree-5 polynomial, a Remez minimax fit of
+// the relative error on [-1/2, 1/2] made for this kernel (at most 1.6e-7 with
+// these fp32 coefficients); 2^f 2^n is one exact multiply.  The
+// kernel's exp(z - c) terms, whose argument lies in [-2 log2(e) c, 0], use it
+// instead of ex2.approx, so that the transcendental pipe (left with the
+// softcap's ex2 and rcp) and the FMA pipe share the work.
+constexpr float kExp2C0 = 1.0000001192092896f, kExp2C1 = 0.6931469440460205f,
+                kExp2C2 = 0.24022120237350464f, kExp2C3 = 0.05550713092088699f,
+                kExp2C4 = 0.009675540961325169f, kExp2C5 = 0.0013276472454890609f;
+
+__device__ __forceinline__ uint64_t ex2_fma2(uint64_t x) {
+    const uint64_t magic = pk2(12583039.0f, 12583039.0f);  // 1.5 * 2^23 + 127
+    const uint64_t t = add2(x, magic);  // rint(x) + 127 in the low bits of each lane
+    const uint64_t f = sub2(x, sub2(t, magic));
+    uint64_t p = fma2(pk2(kExp2C5, kExp2C5), f, pk2(kExp2C4, kExp2C4));
+    p = fma2(p, f, pk2(kExp2C3, kExp2C3));
+    p = fma2(p, f, pk2(kExp2C2, kExp2C2));
+    p = fma2(p, f, pk2(kExp2C1, kExp2C1));
+    p = fma2(p, f, pk2(kExp2C0, kExp2C0));
+    float t0, t1;
+    up2(t, t0, t1);
+    return mul2(p, pk2(__int_as_float(__float_as_int(t0) << 23),
+                       __int_as_float(__float_as_int(t1) << 23)));
+}
+
+// r = 1 / (exp(2 l / c) + 1) for the two logits of a bf16 pair w (low half
+// first); k2 = {2 log2(e) / c} in both lanes
+__device__ __forceinline__ uint64_t softcap_r2(uint32_t w, uint64_t k2, uint64_t one) {
+    float e0, e1;
+    up2(mul2(pk2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)), k2), e0, e1);
+    float d0, d1;
+    up2(add2(pk2(ex2_approx(e0), ex2_approx(e1)), one), d0, d1);
+    return pk2(rcp_approx(d0), rcp_approx(d1));
 }
 
 // r = 1 / (exp(2 l / c) + 1); k2 = 2 log2(e) / c
@@ -217,18 +290,19 @@ __global__ void __launch_bounds__(kCeThreads)
     const float log2e = 1.4426950408889634f;
     const float k2 = __fdiv_rn(2.0f * log2e, c);  // exp(2y) = 2^(l k2)
     const float kz = -2.0f * log2e * c;           // exp(z - c) = 2^(kz r)
-    float sum = 0.f;
+    const uint64_t k2x2 = pk2(k2, k2), kzx2 = pk2(kz, kz), one2 = pk2(1.0f, 1.0f);
+    // each thread keeps two partial sums (even and odd logits), added at the end
+    uint64_t sum2 = pk2(0.f, 0.f);
     for (int v = threadIdx.x; v < nv; v += kCeThreads) {
         const uint4 x = lv[v];
         const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float r0 = softcap_r(__uint_as_float(w[i] << 16), k2);
-            const float r1 = softcap_r(__uint_as_float(w[i] & 0xFFFF0000u), k2);
-            sum = __fadd_rn(sum, ex2_approx(__fmul_rn(kz, r0)));
-            sum = __fadd_rn(sum, ex2_approx(__fmul_rn(kz, r1)));
-        }
+        for (int i = 0; i < 4; ++i)
+            sum2 = add2(sum2, ex2_fma2(mul2(kzx2, softcap_r2(w[i], k2x2, one2))));
     }
+    float s0, s1;
+    up2(sum2, s0, s1);
+    float sum = __fadd_rn(s0, s1);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, o));
     __shared__ float ws[kCeThreads / 32];
@@ -251,23 +325,28 @@ __global__ void __launch_bounds__(kCeThreads)
     __syncthreads();
     const float inv_sum = s_inv_sum;
     const float g4 = 4.0f * inv_count;  // (1 - t^2) = 4 r (1 - r), times 1/M
+    const uint64_t invx2 = pk2(inv_sum, inv_sum), g4x2 = pk2(g4, g4);
     uint32_t m2 = 0;
     for (int v = threadIdx.x; v < nv; v += kCeThreads) {
         const uint4 x = lv[v];
         const uint32_t w[4] = {x.x, x.y, x.z, x.w};
         uint32_t o[4];
+        const bool target_here = (unsigned)(label - 8 * v) < 8u;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            float g[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float l = __uint_as_float(h ? (w[i] & 0xFFFF0000u) : (w[i] << 16));
-                const float r = softcap_r(l, k2);
-                float p = __fmul_rn(ex2_approx(__fmul_rn(kz, r)), inv_sum);  // exp(z - lse)
-                if (8 * v + 2 * i + h == label) p = __fsub_rn(p, 1.0f);
-                g[h] = __fmul_rn(__fmul_rn(p, __fmul_rn(r, __fsub_rn(1.0f, r))), g4);
+            const uint64_t r = softcap_r2(w[i], k2x2, one2);
+            uint64_t p = mul2(ex2_fma2(mul2(kzx2, r)), invx2);  // exp(z - lse)
+            const int base = 8 * v + 2 * i;
+            if (target_here && (unsigned)(label - base) < 2u) {  // the target logit: p - 1
+                float p0, p1;
+                up2(p, p0, p1);
+                if (label == base) p0 = __fsub_rn(p0, 1.0f);
+                else p1 = __fsub_rn(p1, 1.0f);
+                p = pk2(p0, p1);
             }
-            const __nv_bfloat162 b = __floats2bfloat162_rn(g[0], g[1]);
+            float g0, g1;
+            up2(mul2(mul2(p, mul2(r, sub2(one2, r))), g4x2), g0, g1);
+            const __nv_bfloat162 b = __floats2bfloat162_rn(g0, g1);
             o[i] = *reinterpret_cast<const uint32_t*>(&b);
             m2 = __vmaxu2(m2, o[i] & 0x7FFF7FFFu);
         }
