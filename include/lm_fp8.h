@@ -243,7 +243,11 @@ LM_API size_t lm_relu2_mlp_workspace_size(int64_t M, int64_t d, int64_t f);
  * X: bf16 [M x d], W_up: bf16 [f x d], W_down: bf16 [d x f], Y: bf16 [M x d].
  * workspace: NULL (ws_bytes 0), or 256-byte-aligned device scratch of at least
  * lm_fp8_gemm_workspace_size() bytes (e.g. the backward's workspace), which
- * lets the GEMMs split an under-filled last wave (see lm_fp8_gemm_ex).
+ * lets the GEMMs split an under-filled last wave (see lm_fp8_gemm_ex).  With
+ * a workspace and M > 128, the cast of h runs inside the down GEMM's launch
+ * (extra warps cast it in 256 x 128 blocks just before the GEMM's tiles read
+ * them; the workspace also holds one ready bit per block); otherwise it is its
+ * own launch before the down GEMM.  The codes are the same either way.
  * Requirements: M, d, f multiples of 16.
  */
 LM_API lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W_down, int64_t M,
