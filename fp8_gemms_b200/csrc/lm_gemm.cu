@@ -128,6 +128,15 @@ __device__ __forceinline__ void side_cast_loop(const GemmArgs& a, int64_t t, int
     for (; i < n; i += nt) q[i] = convert8<FMT, false>(ld_stream_v4(x + i), scale);
 }
 
+// The side cast feeding A keeps num_mb * words ready words, then (8-byte
+// aligned) a 64-bit counter of claimed units; all of it zeroed per launch.
+__host__ __device__ __forceinline__ int64_t side_counter_word(int64_t num_mb, int64_t words) {
+    return (num_mb * words + 1) & ~int64_t(1);
+}
+__host__ __device__ __forceinline__ size_t side_ready_bytes(int64_t num_mb, int64_t words) {
+    return (size_t)(side_counter_word(num_mb, words) + 2) * sizeof(unsigned int);
+}
+
 // Unit i of a side cast that feeds A -> its row block mb and k-block kb.  With
 // one tile group per row block (group_m == 1) row block mb's first tile falls
 // in round (mb * num_nb) / C of the C clusters; the units go round by round,
@@ -154,19 +163,28 @@ __device__ __forceinline__ void side_unit(int64_t i, const GemmArgs& a, int C, i
     if (r & 1) kb = nkb - 1 - kb;
 }
 
-// A side cast that feeds A: the side warps of CTA `cta` (thread t of 128)
-// take units cta, cta + ncta, ...; 8 rows x 16 vectors of a unit per step,
-// eight steps in flight per thread.  The side warps meet at named barrier 1
-// after a unit's stores; thread 0 then fences and publishes the unit's bit.
+// A side cast that feeds A: the side warps of a CTA (thread t of 128) claim
+// the next unit from a counter after the ready words (thread 0, broadcast
+// through `slot` in shared memory), so units go out in the order above to
+// whichever CTAs are running: no CTA waits on another being resident.  8 rows
+// x 16 vectors of a unit per step, eight steps in flight per thread.  The side
+// warps meet at named barrier 1 after a unit's stores; thread 0 then fences
+// and publishes the unit's bit.
 template <int FMT, bool RELU2>
-__device__ __forceinline__ void side_cast_units(const GemmArgs& a, int cta, int ncta, int t,
-                                                int C, float scale) {
+__device__ __forceinline__ void side_cast_units(const GemmArgs& a, int t, int C, float scale,
+                                                volatile int64_t* slot) {
     const uint16_t* x = static_cast<const uint16_t*>(static_cast<const void*>(a.side_x));
     uint8_t* q = reinterpret_cast<uint8_t*>(a.side_q);
     const int64_t M = a.M, K = a.side_cols;
     const int64_t total = (int64_t)a.num_mb * a.num_kb;
+    unsigned long long* next = reinterpret_cast<unsigned long long*>(
+        a.side_ready + side_counter_word(a.num_mb, a.side_ready_words));
     const int rr = t >> 4, v = t & 15;
-    for (int64_t i = cta; i < total; i += ncta) {
+    for (;;) {
+        if (t == 0) *slot = (int64_t)atomicAdd(next, 1ull);
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * SIDE_WARPS) : "memory");
+        const int64_t i = *slot;  // read by every side thread before the next claim
+        if (i >= total) break;
         int mb, kb;
         side_unit(i, a, C, mb, kb);
         const int64_t col = (int64_t)kb * 128 + v * 8;
@@ -217,7 +235,8 @@ __device__ __forceinline__ uint32_t ready_wait(const unsigned int* word, uint32_
 // The side cast, run by the side warps of every CTA (thread t of nt): the
 // scale from the already-reduced amax, the scale block (thread 0), the codes.
 // A NaN or infinite amax records kErrNonfiniteAmax, as the cast kernels do.
-__device__ __forceinline__ void side_cast_run(const GemmArgs& a, int64_t t, int64_t nt) {
+__device__ __forceinline__ void side_cast_run(const GemmArgs& a, int64_t t, int64_t nt,
+                                              volatile int64_t* slot) {
     const float amax = *a.side_amax_in;
     const bool e4 = a.side_fmt == LM_FP8_E4M3;
     const float scale = scale_from_amax(amax, e4 ? 448.0f : 57344.0f);
@@ -232,13 +251,13 @@ __device__ __forceinline__ void side_cast_run(const GemmArgs& a, int64_t t, int6
         const int cta = (int)(t / kT), ncta = (int)(nt / kT), lt = (int)(t - (int64_t)cta * kT);
         const int C = ncta / 2;
         if (e4 && a.side_relu2)
-            side_cast_units<LM_FP8_E4M3, true>(a, cta, ncta, lt, C, scale);
+            side_cast_units<LM_FP8_E4M3, true>(a, lt, C, scale, slot);
         else if (e4)
-            side_cast_units<LM_FP8_E4M3, false>(a, cta, ncta, lt, C, scale);
+            side_cast_units<LM_FP8_E4M3, false>(a, lt, C, scale, slot);
         else if (a.side_relu2)
-            side_cast_units<LM_FP8_E5M2, true>(a, cta, ncta, lt, C, scale);
+            side_cast_units<LM_FP8_E5M2, true>(a, lt, C, scale, slot);
         else
-            side_cast_units<LM_FP8_E5M2, false>(a, cta, ncta, lt, C, scale);
+            side_cast_units<LM_FP8_E5M2, false>(a, lt, C, scale, slot);
         return;
     }
     if (e4)
@@ -599,7 +618,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SIDE ? NUM_THREADS_S
         // ------------------------------------------ side cast (both CTAs)
         constexpr int kSideThreads = 32 * SIDE_WARPS;
         side_cast_run(args, (int64_t)blockIdx.x * kSideThreads + (threadIdx.x - NUM_THREADS),
-                      (int64_t)gridDim.x * kSideThreads);
+                      (int64_t)gridDim.x * kSideThreads,
+                      reinterpret_cast<volatile int64_t*>(tmem_slot + 2));
     } else {
         // ------------------------------------------- epilogue (both CTAs)
         const int wi = warp - 2;       // staging slot
@@ -1181,7 +1201,7 @@ lm_status launch_pair_as(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
         uint8_t* r = reinterpret_cast<uint8_t*>(a.side_ready);
         if (!zero_at) zero_at = r;
         zero_bytes = (size_t)(r - zero_at) +
-                     (size_t)a.num_mb * (size_t)a.side_ready_words * sizeof(unsigned int);
+                     side_ready_bytes(a.num_mb, a.side_ready_words);
     }
     if (zero_bytes && cudaMemsetAsync(zero_at, 0, zero_bytes, s) != cudaSuccess)
         return LM_ERR_CUDA;
@@ -1457,7 +1477,7 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
             const size_t used =
                 (size_t)a.split_slots * (kSplitTileBytes + 2 * NUM_EPI_WARPS * sizeof(unsigned int));
             const int words = (a.num_kb + 31) / 32;
-            const size_t need = used + (size_t)a.num_mb * (size_t)words * sizeof(unsigned int);
+            const size_t need = used + side_ready_bytes(a.num_mb, words);
             if (side_warps && workspace && aligned16(workspace) && ws_bytes >= need) {
                 a.side_ready =
                     reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + used);

@@ -54,7 +54,10 @@ size_t layout(int64_t M, int64_t d, int64_t V, int64_t C, uint8_t* base, Ws* w) 
     o.Xq = take((size_t)C * d);
     o.logits = reinterpret_cast<uint16_t*>(take((size_t)C * V * 2));
     o.dLq = take((size_t)C * V);
-    o.ready_bytes = (size_t)((C + 255) / 256) * (size_t)((((V + 127) / 128) + 31) / 32) * 4;
+    // ready words of (C / 256) x (V / 128) units, then an 8-byte-aligned
+    // 64-bit counter (the GEMM's layout for a side cast feeding A)
+    const int64_t ready_words = ((C + 255) / 256) * ((((V + 127) / 128) + 31) / 32);
+    o.ready_bytes = (size_t)(((ready_words + 1) & ~int64_t(1)) + 2) * 4;
     o.ready = reinterpret_cast<unsigned int*>(take(o.ready_bytes));
     o.loss_rows = reinterpret_cast<float*>(take((size_t)M * sizeof(float)));  // the tail
     if (w) *w = o;
