@@ -23,6 +23,10 @@ iterations).  Also the small, self-contained command to run under ncu.
         (the per-step linear GEMM set of a 28-layer d = 3072 stack at M = 16384:
         per layer Q, K, V, O and the relu^2 MLP, fwd + dgrad + wgrad, each
         layer with its own weights and t3-distributed activations)
+    python microbench.py mlp-fwd --M 16384
+        (the relu^2 MLP forward alone: casts, the up GEMM, and the down GEMM
+        whose side warps cast h; with --warmup 1 --iters 1 the 4th GEMM launch
+        is the second forward's down GEMM, the one to capture under ncu)
     python microbench.py mlp-accum --M 16384 --micro 7
         (one optimizer step of gradient accumulation: the weights are cast by the
         first micro-batch's forward and reused by the others; every backward adds
@@ -162,8 +166,9 @@ def linears(a, gen, flush):
 
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("op", choices=["gemm", "cast", "mlp-accum", "rmsnorm-cast", "mlp-compare",
-                                  "lmhead-ce", "scaled-mm", "torch-composition", "linears"])
+    p.add_argument("op", choices=["gemm", "cast", "mlp-accum", "mlp-fwd", "rmsnorm-cast",
+                                  "mlp-compare", "lmhead-ce", "scaled-mm", "torch-composition",
+                                  "linears"])
     p.add_argument("--workload", default="attn-head", choices=["attn-head", "stack"])
     p.add_argument("--layers", type=int, default=28)
     p.add_argument("--V", type=int, default=50304)
@@ -194,6 +199,18 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     if a.op == "mlp-accum":
         pass
+    elif a.op == "mlp-fwd":
+        from fp8_gemms_b200 import api
+        M, d, f = a.M, a.d, a.f
+        mlp = api.Relu2Mlp(M, d, f)
+        X = torch.randn(M, d, device="cuda", generator=gen).to(torch.bfloat16)
+        Wu = (torch.randn(f, d, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)
+        Wd = (torch.randn(d, f, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)
+        Y = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+        ms = time_it(lambda: mlp.forward(X, Wu, Wd, Y=Y), a.iters, a.warmup, flush)
+        avg = sum(ms) / len(ms)
+        out = dict(op="mlp-fwd", M=M, d=d, f=f, avg_ms=round(avg, 4),
+                   tflops=round(2 * 2 * M * d * f / avg / 1e9, 1))
     elif a.op == "linears":
         out = linears(a, gen, flush)
     elif a.op == "scaled-mm":
