@@ -49,7 +49,7 @@ LAUNCHES_PER_STEP = 10                         # kernels of ours per fwd+bwd: "a
 # dram__bytes_write.sum), valid only for the kernel source it was taken on;
 # the summary and the command are in profiles/.
 GEMM_TRAFFIC = {
-    "source_sha256": "93fd0d3af89608b6746c2bdf2715e8174e20b66dbaab1ea799b8620890340ed4",
+    "source_sha256": "a9aaa2d5389fdca3657e531b4b9b3ced39f8c2d80d4cd714ea66b6ab6f9cbb9e",
     "bytes_per_launch": 493504981,  # mean of the step's six GEMMs, profiles/gemm_fp8_pair_relu2_mlp_shapes.md
 }
 

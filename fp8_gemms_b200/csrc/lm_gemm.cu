@@ -15,9 +15,16 @@
 // live in TMEM (2 x 256 fp32 columns per CTA, double-buffered so the
 // epilogue of one tile overlaps the main loop of the next).  The epilogue
 // warps of each CTA drain their own 128 rows: tcgen05.ld -> dequant scale ->
-// relu^2 / relu^2' -> bf16 -> 64B-swizzled shared staging -> TMA store, and
-// reduce the amax of what the next cast consumes.  No TMA load uses cluster
-// multicast; only the MMA-completion commits are multicast to the pair.
+// relu^2 / relu^2' -> bf16 -> 32 x 64 staging boxes (128-byte swizzle) -> TMA
+// store, and reduce the amax of what the next cast consumes.  No TMA load uses
+// cluster multicast; only the MMA-completion commits are multicast to the pair.
+//
+// Side casts: an instantiation with four more warps casts a bf16 tensor whose
+// amax an earlier kernel reduced, beside the tiles.  Either a tensor the GEMM
+// does not read (flat, no waits), or the GEMM's own A operand: then the side
+// warps cast it in 256 x 128 units in the order the tiles consume them and set
+// a ready bit per unit, and the TMA producer loads an A box only once its
+// unit's bit is set.
 //
 // Thin kernel (M <= 128): one CTA per 128 x 256 tile (cta_group::1), same
 // ring and TMEM double buffer, per-thread global stores.
