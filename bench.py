@@ -250,24 +250,37 @@ def run_gpu(args):
         raise RuntimeError(f"device error {st} at wait {where:#x}")
 
     # ---- timed region: K steps through the two C-ABI calls; the library
-    # records an event before each of its kernel launches (lm_timing_attach)
+    # records an event before each of its kernel launches (lm_timing_attach).
+    # A region whose clock record shows a hardware or thermal slowdown is
+    # measured once more (every rank takes the same decision), and the line
+    # names the reasons that the first one saw.
     K = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    timers = [lib.KernelTimer(2 * LAUNCHES_PER_STEP) for _ in range(K)]
-    barrier()
     props = torch.cuda.get_device_properties(device)
     uuid = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else ""
-    with ClockSampler(uuid) as clk:
-        with clk.region():
-            for k in range(K):
-                flush.fill_(k & 0xFF)
-                starts[k].record()
-                with timers[k]:
-                    step()
-                ends[k].record()
-            barrier()
-    clocks = clk.summary()
+    slow_reasons = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+    first_reasons = None
+    for attempt in range(2):
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        timers = [lib.KernelTimer(2 * LAUNCHES_PER_STEP) for _ in range(K)]
+        barrier()
+        with ClockSampler(uuid) as clk:
+            with clk.region():
+                for k in range(K):
+                    flush.fill_(k & 0xFF)
+                    starts[k].record()
+                    with timers[k]:
+                        step()
+                    ends[k].record()
+                barrier()
+        clocks = clk.summary()
+        slow = sorted(set(clocks.get("reasons") or []) & set(slow_reasons))
+        if attempt == 1 or max_over_ranks(1.0 if slow else 0.0, world, device) == 0.0:
+            break
+        first_reasons = slow or ["on another rank"]
+        time.sleep(2.0)
+    if first_reasons:
+        clocks["remeasured_after"] = first_reasons
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), world, device)
     st, where = lib.lm_get_error()
