@@ -190,12 +190,15 @@ def test_full_size_mlp_forward_only_sampled(orc, api):
 
 
 @pytest.mark.parametrize("workspace", [True, False])
-@pytest.mark.parametrize("M,d,f", [(512, 256, 1024), (4096, 512, 2048), (1168, 256, 1040)])
+@pytest.mark.parametrize("M,d,f", [(512, 256, 1024), (4096, 512, 2048), (1168, 256, 1040),
+                                   (512, 768, 1024)])
 def test_mlp_forward_h_cast_in_down_gemm_or_own_launch(orc, api, M, d, f, workspace):
     """With a workspace, h is cast by the down GEMM's side warps, unit by unit
     ahead of the tiles that read it (several units per CTA, ragged last row
-    block and k-block at (1168, 1040)); without one, by its own launch before
-    the GEMM.  Either way: casts bit-exact, the GEMMs within tolerance."""
+    block and k-block at (1168, 1040); at (512, 768) the down GEMM's N exceeds
+    its M, so its tiles sweep row blocks fastest and the units go k-block by
+    k-block over all row blocks); without one, by its own launch before the
+    GEMM.  Either way: casts bit-exact, the GEMMs within tolerance."""
     from fp8_gemms_b200 import _lib
     w = synthetic.MlpWorkload("h cast placement", M, d, f, False, ("t3", None), 11)
     t = w.tensors()
