@@ -14,8 +14,12 @@ is no data-path collective and scaling is weak.
 
 Timing: CUDA events on the launching stream around each step, L2 flushed
 (a 256 MiB write) before every timed step, W untimed warm-up steps, max over
-ranks.  SM clocks and clock-event reasons are sampled in-process through NVML
-every few milliseconds; only samples taken inside the timed region count.
+ranks.  Each timed loop starts behind a short device-side sleep, so the host
+is already ahead of the GPU when the first timed step starts and a host-side
+stall while it issues later steps does not leave the GPU idle inside one.
+SM clocks and clock-event reasons are sampled in-process through NVML every
+few milliseconds; only samples taken while the timed steps ran on the device
+count (the sampler watches the first start and the last end event).
 
 Besides the headline (the fwd + bwd block at M = 16384), the same JSON line
 carries the other GEMM sets of the little-lm model under "configs", each timed
@@ -95,13 +99,15 @@ REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slow
 class ClockSampler:
     """Samples the SM clock, power and clock-event reasons of one GPU through
     NVML from a host thread every ~2 ms.  region() marks the timed region; the
-    summary uses only the samples taken inside it."""
+    summary uses only the samples taken inside it.  The thread also polls the
+    region's watched CUDA events (Event.query is thread-safe)."""
 
     def __init__(self, uuid):
         self.uuid = uuid
         self.samples = []   # (t, sm_mhz, power_w, reasons)
         self.regions = []
         self._stop = threading.Event()
+        self._watch = None  # [start event, end event, t seen done, t seen done]
         self.h = None
         self.max_mhz = None
 
@@ -126,7 +132,15 @@ class ClockSampler:
                 sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
                 pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
                 rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.samples.append((time.perf_counter(), sm, pw, rs))
+                t = time.perf_counter()
+                self.samples.append((t, sm, pw, rs))
+                w = self._watch
+                if w is not None:
+                    if w[2] is None and w[0] is not None and w[0].query():
+                        w[2] = time.perf_counter()   # the samples after this one
+                    if w[2] is not None and w[3] is None and w[1] is not None \
+                            and w[1].query():
+                        w[3] = t
             except Exception:
                 pass
             time.sleep(0.002)
@@ -146,11 +160,35 @@ class ClockSampler:
 
         def __enter__(self):
             self.t0 = time.perf_counter()
+            self.owner._watch = [None, None, None, None]
+            return self
+
+        def watch_start(self, ev):
+            """ev: the first timed event, already recorded."""
+            self.owner._watch[0] = ev
+
+        def watch_end(self, ev):
+            """ev: the last timed event, already recorded."""
+            self.owner._watch[1] = ev
 
         def __exit__(self, *exc):
-            self.owner.regions.append((self.t0, time.perf_counter()))
+            o = self.owner
+            w = o._watch
+            if o.h is not None and w[1] is not None:
+                deadline = time.perf_counter() + 0.5
+                while w[3] is None and time.perf_counter() < deadline:
+                    time.sleep(0.002)
+            o._watch = None
+            t1 = time.perf_counter()
+            o.regions.append((w[2] if w[2] is not None else self.t0,
+                              w[3] if w[3] is not None else t1))
 
     def region(self):
+        """The timed region.  By default the host time inside the with-block;
+        once watch_start() and watch_end() have handed it the recorded CUDA
+        events that open and close the timed steps, the span from when the
+        sampler thread first saw the first complete to when it first saw the
+        second complete (2 ms resolution)."""
         return ClockSampler._Region(self)
 
     def summary(self, region=0):
@@ -168,7 +206,8 @@ class ClockSampler:
                 sorted(sm)[int(0.9 * (len(sm) - 1))], "sm_max_mhz": self.max_mhz,
                 "reasons": reasons, "samples": len(rows),
                 "region_s": round(t1 - t0, 4), "power_w_max": max(r[2] for r in rows),
-                "source": "nvml, in-process, ~2 ms period, samples inside the timed region only"}
+                "source": "nvml, in-process, ~2 ms period, samples taken while the timed "
+                          "steps ran on the device only"}
 
 
 # ------------------------------------------------------------ GPU pieces
@@ -188,6 +227,15 @@ def max_over_ranks(x, world, device):
     t = torch.tensor([float(x)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def host_ahead(torch, steps):
+    """Queues a device-side sleep of about a millisecond per step to come (at
+    most 50 ms) ahead of a timed loop: the host issues the loop's launches
+    while the GPU sleeps, so it is ahead when the first timed step starts and
+    a host-side stall while it issues later steps cannot leave the GPU idle
+    inside a timed step.  The sleep lies before the first timed event."""
+    torch.cuda._sleep(int(min(50, steps) * 2.0e6))   # ~2e6 SM cycles per ms
 
 
 def job_tflops(world, steps, flops_per_step, total_ms):
@@ -265,13 +313,17 @@ def run_gpu(args):
         timers = [lib.KernelTimer(2 * LAUNCHES_PER_STEP) for _ in range(K)]
         barrier()
         with ClockSampler(uuid) as clk:
-            with clk.region():
+            host_ahead(torch, K)
+            with clk.region() as reg:
                 for k in range(K):
                     flush.fill_(k & 0xFF)
                     starts[k].record()
+                    if k == 0:
+                        reg.watch_start(starts[0])
                     with timers[k]:
                         step()
                     ends[k].record()
+                reg.watch_end(ends[-1])
                 barrier()
         clocks = clk.summary()
         slow = sorted(set(clocks.get("reasons") or []) & set(slow_reasons))
@@ -361,6 +413,7 @@ def run_gpu(args):
     c_end = [torch.cuda.Event(enable_timing=True) for _ in range(Kc)]
     mlp.forward(dev["X"], dev["W_up"], dev["W_down"], Y=dev["Y"])  # casts of these weights
     barrier()
+    host_ahead(torch, Kc)
     for k in range(Kc):
         flush.fill_(k & 0xFF)
         c_start[k].record()
@@ -368,8 +421,9 @@ def run_gpu(args):
         mlp.backward(dev["dY"], dX=dev["dX"], dW_up=dev["dW_up"], dW_down=dev["dW_down"])
         c_end[k].record()
     barrier()
-    cached_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(c_start, c_end)), world,
-                               device)
+    cached_steps = [a.elapsed_time(b) for a, b in zip(c_start, c_end)]
+    cached_ms = max_over_ranks(sum(cached_steps), world, device)
+    cached_median = statistics.median(cached_steps)
     st, where = lib.lm_get_error()
     if st != 0:
         raise RuntimeError(f"device error {st} at wait {where:#x}")
@@ -436,6 +490,9 @@ def run_gpu(args):
         "per_launch_ms": [round(a, 4) for a in avg],
         "per_gemm_kcycles": [round(a * mhz, 1) for a in gemm_ms] if mhz else None,
         "lead_in_ms_per_step": round(statistics.mean(lead_ms), 4),
+        "step_ms_spread": {"min": round(min(step_ms), 4),
+                           "median": round(statistics.median(step_ms), 4),
+                           "max": round(max(step_ms), 4)},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "steps": Ke,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms / Ke, 4),
@@ -445,6 +502,7 @@ def run_gpu(args):
         "weight_casts_cached": {
             "value": round(job_tflops(world, Kc, STEP_FLOPS, cached_ms), 2), "unit": "TFLOP/s",
             "steps": Kc, "ms_per_step": round(cached_ms / Kc, 4),
+            "step_ms_median": round(cached_median, 4),
             "how": "forward reuses the W_up/W_down codes and scales, as after the first "
                    "micro-batch of an optimizer step"},
         "gpu_launches": K * LAUNCHES_PER_STEP,
@@ -476,6 +534,7 @@ def time_steps(step, K, W, flush, cap):
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
+    host_ahead(torch, K)
     for k in range(K):
         flush.fill_(k & 0xFF)
         ev[k][0].record()
@@ -511,6 +570,7 @@ def time_graph(step, K, flush):
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
+    host_ahead(torch, K)
     for k in range(K):
         flush.fill_(k & 0xFF)
         ev[k][0].record()
