@@ -55,6 +55,56 @@ def test_noalloc_backward_matches_allocating_backward_on_two_calls(orc):
             assert_close(u16(dWd), bwd["dW_down"], "dW_down vs oracle")
 
 
+def test_noalloc_backward_in_a_cuda_graph():
+    """The entry point is meant for graph capture: after one eager call (which
+    resolves the library array's address), the backward is captured once and
+    replayed; every replay must reproduce the eager outputs bit for bit, and a
+    replay after the inputs change must follow them."""
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from fp8_gemms_b200 import _lib, api
+
+    w = synthetic.TINY_MLP
+    dev = {k: v.cuda() for k, v in w.tensors().items()}
+    mlp = api.Relu2Mlp(w.M, w.d, w.f)
+    mlp.forward(dev["X"], dev["W_up"], dev["W_down"])
+    dY = dev["dY"].clone()
+    dX = torch.empty(w.M, w.d, dtype=torch.bfloat16, device="cuda")
+    dWu = torch.empty(w.f, w.d, dtype=torch.bfloat16, device="cuda")
+    dWd = torch.empty(w.d, w.f, dtype=torch.bfloat16, device="cuda")
+
+    def bwd():
+        _lib.lm_relu2_mlp_bwd_noalloc(dY, mlp.saved, dX, dWu, dWd)
+
+    bwd()                                        # eager warm-up before capture
+    torch.cuda.synchronize()
+    assert _lib.lm_get_error()[0] == 0
+    eager = [x.clone() for x in (dX, dWu, dWd)]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            bwd()
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):
+        for x in (dX, dWu, dWd):
+            x.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert _lib.lm_get_error()[0] == 0
+        for name, a, b in zip(("dX", "dW_up", "dW_down"), eager, (dX, dWu, dWd)):
+            assert torch.equal(a, b), name
+    # new upstream gradient, same buffers: the replay follows it
+    dY.mul_(0.25)
+    g.replay()
+    ref_dX, ref_dWu, ref_dWd = mlp.backward(dY)
+    torch.cuda.synchronize()
+    del g
+    assert torch.equal(dX, ref_dX)
+    assert torch.equal(dWu, ref_dWu)
+    assert torch.equal(dWd, ref_dWd)
+
+
 def test_noalloc_backward_rejects_shapes_beyond_its_array():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     from fp8_gemms_b200 import _lib
