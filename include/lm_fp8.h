@@ -234,7 +234,9 @@ LM_API size_t lm_relu2_mlp_workspace_size(int64_t M, int64_t d, int64_t f);
 
 /*
  * relu^2 MLP forward, Y = relu(X W_up^T)^2 W_down^T, every GEMM in FP8:
- *   cast X, W_up, W_down to e4m3 (one amax launch, one cast launch)
+ *   cast X, W_up, W_down to e4m3 (one amax launch for the three, one cast
+ *     launch for X and W_up; W_down's codes are written by extra warps of
+ *     the up GEMM's launch, which does not read them)
  *   H = up GEMM with the RELU2_FWD epilogue (bf16 H + amax of h)
  *   cast h = bf16(relu(H)^2) to e4m3 using that amax
  *   Y = down GEMM (bf16)
@@ -259,7 +261,8 @@ LM_API lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W
  *   cast dY to e5m2
  *   dH = dgrad of W_down with the RELU2_BWD epilogue: bf16(bf16(dY W_down) * 2 relu(H))
  *   dW_down = dY^T h   (wgrad, K = M)
- *   cast dH to e5m2 using the epilogue's amax
+ *   cast dH to e5m2 using the epilogue's amax (by extra warps of the dW_down
+ *     GEMM's launch, which does not read dH)
  *   dX = dH W_up;  dW_up = dH^T X
  * (W_down and W_up as dgrad B operands, and dY, h, dH, X as wgrad operands,
  * are read MN-major from their row-major codes.)
