@@ -1358,7 +1358,6 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
         if (side->feeds_a && (side->q != A || side->rows != M || side->cols != K ||
                               side->fmt != fa || (flags & LM_GEMM_A_MN_MAJOR)))
             return LM_ERR_INVALID_ARG;
-        if (side->rows == 0 || side->cols == 0) side = nullptr;  // nothing to cast
     }
     if ((fa != LM_FP8_E4M3 && fa != LM_FP8_E5M2) || (fb != LM_FP8_E4M3 && fb != LM_FP8_E5M2))
         return LM_ERR_UNSUPPORTED_FORMAT;
@@ -1388,6 +1387,10 @@ lm_status lm::gemm_dispatch(const uint8_t* A, lm_fp8_format fa, const uint8_t* B
             cudaMemsetAsync(D, 0, (size_t)M * (size_t)N * 2, s) != cudaSuccess)
             return LM_ERR_CUDA;
         return side ? side_cast_alone(*side, s) : LM_OK;
+    }
+    if (side && (side->rows == 0 || side->cols == 0)) {  // nothing to cast: its scales alone
+        if (lm_status st = side_cast_alone(*side, s)) return st;
+        side = nullptr;
     }
     unsigned int* err = device_error_word();
     if (!err) return LM_ERR_CUDA;

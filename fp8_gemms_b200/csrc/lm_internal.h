@@ -65,7 +65,8 @@ constexpr int kEpiSwigluFwd = 4;
 // codes nor write the input.  Where the GEMM launch cannot carry it (the
 // thin kernel, a multi-part split tail, an empty GEMM), gemm_dispatch runs
 // the cast as its own launch after the GEMM instead; the results are the same
-// bits either way.
+// bits either way.  An empty tensor (no rows or no columns) gets its scale
+// block alone, from amax_in, in a launch of its own.
 struct SideCast {
     const void* x;  // bf16 [rows x cols], contiguous
     int64_t rows, cols;

@@ -109,8 +109,9 @@ lm_status lm_relu2_mlp_fwd_ex(const void* X, const void* W_up, const void* W_dow
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
         return LM_ERR_ALIGNMENT;
     const bool reuse = (flags & LM_MLP_REUSE_WEIGHT_CASTS) != 0;
-    if (!X || !Y || !sv || (!reuse && (!W_up || !W_down))) return LM_ERR_INVALID_ARG;
-    if (!sv->Xq || !sv->Wuq || !sv->Wdq || !sv->H || !sv->hq || !sv->scales)
+    // tensors with M rows may be NULL when M == 0 (an empty micro-batch)
+    if (!sv || (M > 0 && (!X || !Y)) || (!reuse && (!W_up || !W_down))) return LM_ERR_INVALID_ARG;
+    if (!sv->Wuq || !sv->Wdq || !sv->scales || (M > 0 && (!sv->Xq || !sv->H || !sv->hq)))
         return LM_ERR_INVALID_ARG;
     if (!lm::all_aligned16({X, W_up, W_down, Y, sv->Xq, sv->Wuq, sv->Wdq, sv->H, sv->hq}))
         return LM_ERR_ALIGNMENT;
@@ -169,10 +170,13 @@ lm_status lm_relu2_mlp_bwd_ex(const void* dY, const lm_mlp_saved* sv, int64_t M,
                               size_t ws_bytes, uint32_t flags, lm_stream_t stream) {
     if (!mlp_shape_ok(M, d, f)) return LM_ERR_UNSUPPORTED_SHAPE;
     if (flags & ~LM_MLP_ACCUMULATE_WGRAD) return LM_ERR_INVALID_ARG;
-    if (!dY || !sv || !dX || !dW_up || !dW_down || !workspace) return LM_ERR_INVALID_ARG;
+    // tensors with M rows may be NULL when M == 0 (an empty micro-batch: the
+    // weight gradients are then zero, or left as they were when accumulating)
+    if (!sv || !dW_up || !dW_down || !workspace || (M > 0 && (!dY || !dX)))
+        return LM_ERR_INVALID_ARG;
     if (ws_bytes < bwd_layout(M, d, f, nullptr, nullptr)) return LM_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return LM_ERR_ALIGNMENT;
-    if (!sv->Xq || !sv->Wuq || !sv->Wdq || !sv->H || !sv->hq || !sv->scales)
+    if (!sv->Wuq || !sv->Wdq || !sv->scales || (M > 0 && (!sv->Xq || !sv->H || !sv->hq)))
         return LM_ERR_INVALID_ARG;
     if (!lm::all_aligned16({dY, dX, dW_up, dW_down, sv->Xq, sv->Wuq, sv->Wdq, sv->H, sv->hq}))
         return LM_ERR_ALIGNMENT;

@@ -250,7 +250,9 @@ LM_API size_t lm_relu2_mlp_workspace_size(int64_t M, int64_t d, int64_t f);
  * (extra warps cast it in 256 x 128 blocks just before the GEMM's tiles read
  * them; the workspace also holds one ready bit per block); otherwise it is its
  * own launch before the down GEMM.  The codes are the same either way.
- * Requirements: M, d, f multiples of 16.
+ * Requirements: M, d, f multiples of 16.  M may be 0 (an empty micro-batch):
+ * X and Y may then be NULL, the weights are still cast, and the scale blocks
+ * of X and h are those of amax 0.
  */
 LM_API lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W_down, int64_t M,
                            int64_t d, int64_t f, void* Y, lm_mlp_saved* saved, void* workspace,
@@ -268,7 +270,8 @@ LM_API lm_status lm_relu2_mlp_fwd(const void* X, const void* W_up, const void* W
  * are read MN-major from their row-major codes.)
  * dY: bf16 [M x d]; outputs bf16 dX [M x d], dW_up [f x d], dW_down [d x f].
  * workspace: device scratch of >= lm_relu2_mlp_workspace_size bytes,
- * 256-byte aligned.  Requirements as for the forward.
+ * 256-byte aligned.  Requirements as for the forward.  With M == 0, dY and dX
+ * may be NULL, and dW_up and dW_down are zero.
  */
 LM_API lm_status lm_relu2_mlp_bwd(const void* dY, const lm_mlp_saved* saved, int64_t M, int64_t d,
                            int64_t f, void* dX, void* dW_up, void* dW_down, void* workspace,

@@ -210,3 +210,32 @@ def test_mlp_forward_h_cast_in_down_gemm_or_own_launch(orc, api, M, d, f, worksp
     torch.cuda.synchronize()
     assert _lib.lm_get_error()[0] == 0
     check_stagewise(orc, mlp, t, Y, None, None, None)
+
+
+def test_mlp_empty_batch(orc, api):
+    """M = 0, an empty micro-batch: nothing to multiply.  Both weights are
+    still cast (W_down's codes by the launch that stands in for the up GEMM's
+    side warps), bit-exact against the oracle; Y and dX are empty; both weight
+    gradients are zero; h's scale block is that of amax 0.  Tensors with M
+    rows arrive as NULL pointers."""
+    from fp8_gemms_b200 import _lib
+    d, f = 256, 1024
+    t = synthetic.MlpWorkload("empty", 16, d, f, False, seed=5).tensors()
+    Wu, Wd = t["W_up"].cuda(), t["W_down"].cuda()
+    mlp = api.Relu2Mlp(0, d, f)
+    X = torch.empty(0, d, dtype=torch.bfloat16, device="cuda")
+    Y = mlp.forward(X, Wu, Wd)
+    dX, dWu, dWd = mlp.backward(torch.empty(0, d, dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    assert _lib.lm_get_error()[0] == 0
+    assert Y.shape == (0, d) and dX.shape == (0, d)
+    assert not bool(dWu.view(torch.int16).any()) and not bool(dWd.view(torch.int16).any())
+    sc = mlp.view("scales").cpu().numpy()
+    for row, name, W in ((1, "Wuq", t["W_up"]), (2, "Wdq", t["W_down"])):
+        ref = orc.amax_scale_cast(synthetic.bits_u16(W), E4M3)
+        assert sc[row, 0] == ref["amax"] and sc[row, 1] == ref["scale"], name
+        assert sc[row, 2] == ref["inv_scale"], name
+        assert np.array_equal(u8(mlp.view(name)), ref["q"]), name
+    s0, inv0 = orc.scale(np.float32(0.0), E4M3)
+    for row in (0, 3):                       # X and h: amax 0
+        assert sc[row, 0] == 0.0 and sc[row, 1] == s0 and sc[row, 2] == inv0
