@@ -234,12 +234,14 @@ def max_over_ranks(x, world, device):
 
 
 def host_ahead(torch, steps):
-    """Queues a device-side sleep of about a millisecond per step to come (at
-    most 50 ms) ahead of a timed loop: the host issues the loop's launches
-    while the GPU sleeps, so it is ahead when the first timed step starts and
-    a host-side stall while it issues later steps cannot leave the GPU idle
-    inside a timed step.  The sleep lies before the first timed event."""
-    torch.cuda._sleep(int(min(50, steps) * 2.0e6))   # ~2e6 SM cycles per ms
+    """Queues a device-side sleep of about half a millisecond per step to come
+    (at most 10 ms) ahead of a timed loop.  The host issues a step's launches
+    in well under that (bench.py reports host_issue_ms_per_step), so it is
+    several steps ahead when the first timed step starts and pulls further
+    ahead with every step; a host-side stall while it issues later steps then
+    cannot leave the GPU idle inside a timed step.  The sleep lies before the
+    first timed event."""
+    torch.cuda._sleep(int(min(10.0, 0.5 * steps) * 2.0e6))   # ~2e6 SM cycles per ms
 
 
 def job_tflops(world, steps, flops_per_step, total_ms):
@@ -319,6 +321,7 @@ def run_gpu(args):
         with ClockSampler(uuid) as clk:
             host_ahead(torch, K)
             with clk.region() as reg:
+                t_issue = time.perf_counter()
                 for k in range(K):
                     flush.fill_(k & 0xFF)
                     starts[k].record()
@@ -328,6 +331,7 @@ def run_gpu(args):
                         step()
                     ends[k].record()
                 reg.watch_end(ends[-1])
+                t_issue = time.perf_counter() - t_issue
                 barrier()
         clocks = clk.summary()
         slow = sorted(set(clocks.get("reasons") or []) & set(slow_reasons))
@@ -494,9 +498,11 @@ def run_gpu(args):
         "per_launch_ms": [round(a, 4) for a in avg],
         "per_gemm_kcycles": [round(a * mhz, 1) for a in gemm_ms] if mhz else None,
         "lead_in_ms_per_step": round(statistics.mean(lead_ms), 4),
+        "host_issue_ms_per_step": round(1e3 * t_issue / K, 4),
         "step_ms_spread": {"min": round(min(step_ms), 4),
                            "median": round(statistics.median(step_ms), 4),
-                           "max": round(max(step_ms), 4)},
+                           "max": round(max(step_ms), 4),
+                           "first": round(step_ms[0], 4), "last": round(step_ms[-1], 4)},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "steps": Ke,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms / Ke, 4),
