@@ -138,16 +138,22 @@ class ClockSampler:
                 rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
                 t = time.perf_counter()
                 self.samples.append((t, sm, pw, rs))
-                w = self._watch
-                if w is not None:
-                    if w[2] is None and w[0] is not None and w[0].query():
-                        w[2] = time.perf_counter()   # the samples after this one
-                    if w[2] is not None and w[3] is None and w[1] is not None \
-                            and w[1].query():
-                        w[3] = t
+                self._poll_watch(t)
             except Exception:
                 pass
             time.sleep(0.002)
+
+    def _poll_watch(self, t):
+        """After the sample taken at t: note when the watched start event is
+        first seen complete (the samples after this one count) and then when
+        the end event is (the sample at t is the last that counts)."""
+        w = self._watch
+        if w is None:
+            return
+        if w[2] is None and w[0] is not None and w[0].query():
+            w[2] = time.perf_counter()
+        if w[2] is not None and w[3] is None and w[1] is not None and w[1].query():
+            w[3] = t
 
     def __exit__(self, *exc):
         self._stop.set()

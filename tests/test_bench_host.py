@@ -89,6 +89,47 @@ def test_clock_summary_counts_only_samples_inside_the_timed_region():
     assert s["reasons"] == ["hw_slowdown", "sw_power_cap"] and s["power_w_max"] == 1000.0
 
 
+def test_clock_region_follows_the_watched_events():
+    """The region spans from when the first timed event is seen complete to
+    when the last one is: samples before the first step ran on the device or
+    after the last one finished do not count, whatever the host was doing."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Ev:
+        def __init__(self):
+            self.done = False
+
+        def query(self):
+            return self.done
+
+    c = bench.ClockSampler("GPU-none")
+    c.h, c.max_mhz = object(), 1965
+    start, end = Ev(), Ev()
+    with c.region() as reg:
+        c._poll_watch(0.1)                 # nothing armed yet
+        reg.watch_start(start)
+        c._poll_watch(0.2)                 # armed, not complete
+        assert c._watch[2] is None
+        start.done = True
+        c._poll_watch(0.3)
+        t_start = c._watch[2]              # host time just after that poll
+        assert t_start is not None
+        reg.watch_end(end)
+        c._poll_watch(0.4)
+        assert c._watch[3] is None
+        end.done = True
+        c._poll_watch(5.0)
+    assert c._watch is None
+    assert c.regions == [(t_start, 5.0)]
+    # without the watched events the region is the host time of the block
+    c2 = bench.ClockSampler("GPU-none")
+    with c2.region():
+        pass
+    (a, b), = c2.regions
+    assert a <= b
+
+
 def test_config_roofline_arithmetic():
     """Roofline time of a GEMM set = FLOPs at the dense FP8 peak + cast bytes
     at HBM bandwidth; 4.5 TFLOP and 8 GB take 1 ms each at 4.5 PF and 8 TB/s."""
