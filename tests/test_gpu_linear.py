@@ -175,3 +175,29 @@ def test_stack_layer_linears_full_size_sampled(orc, api, layer):
         t = lin.tensors(i)
         check_linear(orc, api, t["X"], t["W"], t["dY"], rows=_sample(lin.M),
                      wrows=_sample(t["W"].shape[0], seed=1))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("i", [0, 1, 4], ids=["q", "k", "lm_head"])
+def test_attention_and_head_linears_are_deterministic_over_repeats(api, i):
+    """Five fwd+dgrad+wgrad passes of the Q, K and LM-head linears at M = 8192
+    (split tails, MN-major operands), L2 flushed between them: Y, dX and dW
+    are bit-identical to the first pass's."""
+    from fp8_gemms_b200 import _lib
+    t = synthetic.ATTN_HEAD.tensors(i)
+    X, W, dY = t["X"].cuda(), t["W"].cuda(), t["dY"].cuda()
+    M, K = X.shape
+    lin = api.Linear(M, K, W.shape[0])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    first = None
+    for it in range(5):
+        flush.fill_(it)
+        Y = lin.forward(X, W)
+        dX, dW = lin.backward(dY)
+        torch.cuda.synchronize()
+        assert _lib.lm_get_error()[0] == 0
+        if first is None:
+            first = [Y.clone(), dX.clone(), dW.clone()]
+            continue
+        for name, a, b in zip(("Y", "dX", "dW"), first, (Y, dX, dW)):
+            assert torch.equal(a, b), f"{name} differs at repeat {it}"
