@@ -58,7 +58,7 @@ LAUNCHES_PER_STEP = 10                         # kernels of ours per fwd+bwd: "a
 # information is byte-identical to that source's.
 GEMM_TRAFFIC = {
     "source_sha256": "0e123c3b8a0053a031744441664db7012c4c4b211cd815114a45108732abcc4a",
-    "bytes_per_launch": 493504981,  # mean of the step's six GEMMs, profiles/gemm_fp8_pair_relu2_mlp_shapes.md
+    "bytes_per_launch": 493504981,  # mean over the step's six GEMM shapes, one capture each
 }
 
 
