@@ -368,9 +368,10 @@ def run_gpu(args):
 
     # ---- the same step with the weight casts cached: the forward reuses the
     # codes and scales of W_up and W_down (LM_MLP_REUSE_WEIGHT_CASTS), as every
-    # micro-batch after the first of an optimizer step does.  Timed right
-    # after the headline region, with its own warm-up and clock record, so
-    # that the two see a similar power state.
+    # micro-batch after the first of an optimizer step does.  Timed like the
+    # headline region, from a similar power state: the GPU idles for a second
+    # (the headline region starts after the process's set-up), then its own
+    # warm-up steps, then the timed steps with their own clock record.
     Kc = min(K, 50)
     c_start = [torch.cuda.Event(enable_timing=True) for _ in range(Kc)]
     c_end = [torch.cuda.Event(enable_timing=True) for _ in range(Kc)]
@@ -380,6 +381,8 @@ def run_gpu(args):
         mlp.forward(dev["X"], None, None, Y=dev["Y"], reuse_weight_casts=True)
         mlp.backward(dev["dY"], dX=dev["dX"], dW_up=dev["dW_up"], dW_down=dev["dW_down"])
 
+    barrier()
+    time.sleep(1.0)
     for _ in range(max(3, args.warmup)):
         cached_step()
     barrier()
