@@ -172,8 +172,9 @@ lm_status lm_swiglu_mlp_fwd(const void* X, const void* W_gu, const void* W_down,
     // the workspace, when given, holds the GEMMs' split-K scratch at its start
     void* split = workspace && ws_bytes >= gemm_split_workspace_bytes() ? workspace : nullptr;
     const size_t sb = split ? gemm_split_workspace_bytes() : 0;
-    if (!X || !W_gu || !W_down || !Y || !sv || !sv->Xq || !sv->Wguq || !sv->Wdq || !sv->GU ||
-        !sv->h || !sv->hq || !sv->scales)
+    // tensors with M rows may be NULL when M == 0 (an empty micro-batch)
+    if (!W_gu || !W_down || !sv || !sv->Wguq || !sv->Wdq || !sv->scales ||
+        (M > 0 && (!X || !Y || !sv->Xq || !sv->GU || !sv->h || !sv->hq)))
         return LM_ERR_INVALID_ARG;
     if (!all_aligned16({X, W_gu, W_down, Y, sv->Xq, sv->Wguq, sv->Wdq, sv->GU, sv->h, sv->hq}))
         return LM_ERR_ALIGNMENT;
@@ -207,10 +208,13 @@ lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* sv, int64_t M
                             size_t ws_bytes, lm_stream_t stream) {
     using namespace lm;
     if (!shape_ok(M, d, f)) return LM_ERR_UNSUPPORTED_SHAPE;
-    if (!dY || !sv || !dX || !dW_gu || !dW_down || !workspace) return LM_ERR_INVALID_ARG;
+    // tensors with M rows may be NULL when M == 0 (the weight gradients are then zero)
+    if (!sv || !dW_gu || !dW_down || !workspace || (M > 0 && (!dY || !dX)))
+        return LM_ERR_INVALID_ARG;
     if (ws_bytes < bwd_layout(M, d, f, nullptr, nullptr)) return LM_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return LM_ERR_ALIGNMENT;
-    if (!sv->Xq || !sv->Wguq || !sv->Wdq || !sv->GU || !sv->h || !sv->hq || !sv->scales)
+    if (!sv->Wguq || !sv->Wdq || !sv->scales ||
+        (M > 0 && (!sv->Xq || !sv->GU || !sv->h || !sv->hq)))
         return LM_ERR_INVALID_ARG;
     if (!all_aligned16({dY, dX, dW_gu, dW_down, sv->Xq, sv->Wguq, sv->Wdq, sv->GU, sv->h,
                         sv->hq}))

@@ -395,7 +395,9 @@ LM_API lm_status lm_fp8_linear_bwd(const void* dY, const lm_linear_saved* saved,
  * blocks of 128 (rows 256b..256b+127 = W_gate rows 128b.., the next 128 =
  * W_up rows 128b..); dW_gu comes back in the same order.  f % 128 == 0,
  * d % 16 == 0, M % 16 == 0.  Buffers, workspace and errors as for the relu^2
- * MLP; the saved GU holds G and U in the same interleaved column order.
+ * MLP, M = 0 included (an empty micro-batch: tensors with M rows may be NULL,
+ * the weights are still cast, the weight gradients are zero); the saved GU
+ * holds G and U in the same interleaved column order.
  */
 typedef struct lm_swiglu_saved {
     uint8_t* Xq;           /* [M x d] e4m3 (read MN-major by the wgrad of W_gu) */

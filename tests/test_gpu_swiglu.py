@@ -6,7 +6,7 @@ import pytest
 import torch
 
 from fp8_gemms_b200 import synthetic
-from gpu_util import ELEM_REL, assert_close, f32, u8, u16
+from gpu_util import ELEM_REL, assert_close, cast_ref, f32, u8, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -156,3 +156,23 @@ def test_swiglu_full_shape_is_deterministic_over_repeats():
             continue
         for name, a, b in zip(("Y", "dX", "dW_gu", "dW_down"), first, (Y, dX, dWgu, dWd)):
             assert torch.equal(a, b), f"{name} differs at repeat {it}"
+
+
+def test_swiglu_empty_batch(orc):
+    """M = 0: the weights are still cast, bit-exact against the oracle; Y and
+    dX are empty, dW_gu and dW_down are zero; tensors with M rows are NULL."""
+    from fp8_gemms_b200 import _lib, api
+    d, f = 256, 256
+    _, Wg, Wu, Wd, _ = make(16, d, f, 85)
+    Wgu = api.interleave_gate_up(Wg.cuda(), Wu.cuda())
+    mlp = api.SwigluMlp(0, d, f)
+    Y = mlp.forward(torch.empty(0, d, dtype=torch.bfloat16, device="cuda"), Wgu, Wd.cuda())
+    dX, dWgu, dWd = mlp.backward(torch.empty(0, d, dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    assert _lib.lm_get_error()[0] == 0
+    assert Y.shape == (0, d) and dX.shape == (0, d)
+    assert not bool(dWgu.view(torch.int16).any()) and not bool(dWd.view(torch.int16).any())
+    ref = cast_ref(orc, synthetic.bits_u16(Wgu.cpu()), 0)
+    assert np.array_equal(u8(mlp.view("Wguq")), ref["q"])
+    ref = cast_ref(orc, synthetic.bits_u16(Wd), 0)
+    assert np.array_equal(u8(mlp.view("Wdq")), ref["q"])
