@@ -404,7 +404,9 @@ lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* labels, 
                            lm_stream_t stream) {
     using namespace lm;
     if (!shapes_ok(M, d, V, chunk)) return LM_ERR_UNSUPPORTED_SHAPE;
-    if (!X || !W || !labels || !loss_out || !dX || !dW || !workspace) return LM_ERR_INVALID_ARG;
+    // X, labels and dX may be NULL when M == 0 (no tokens: loss 0, dW unchanged)
+    if (!W || !loss_out || !dW || !workspace || (M > 0 && (!X || !labels || !dX)))
+        return LM_ERR_INVALID_ARG;
     if (!(softcap > 0.f)) return LM_ERR_INVALID_ARG;
     if (ws_bytes < layout(M, d, V, chunk, nullptr, nullptr)) return LM_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return LM_ERR_ALIGNMENT;

@@ -439,7 +439,8 @@ LM_API lm_status lm_swiglu_mlp_bwd(const void* dY, const lm_swiglu_saved* saved,
  * X: bf16 [M x d]; W: bf16 [V x d]; labels: device int32 [M], each in [0, V);
  * loss_out: device fp32 scalar; dX: bf16 [M x d]; dW: fp32 [V x d] (added to);
  * chunk: tokens per chunk; workspace: >= lm_fp8_lmhead_ce_workspace_size bytes,
- * 256-byte aligned.  M, d, V, chunk multiples of 16.
+ * 256-byte aligned.  M, d, V, chunk multiples of 16.  M may be 0: X, labels
+ * and dX may then be NULL, W is still cast, the loss is 0 and dW is unchanged.
  */
 LM_API size_t lm_fp8_lmhead_ce_workspace_size(int64_t M, int64_t d, int64_t V, int64_t chunk);
 LM_API lm_status lm_fp8_lmhead_ce(const void* X, const void* W, const int32_t* labels, int64_t M,

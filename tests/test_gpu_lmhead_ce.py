@@ -87,6 +87,25 @@ def test_lmhead_ce_accumulates_into_dW(orc):
     assert torch.allclose(dW, 2 * once, rtol=1e-5, atol=1e-12)
 
 
+def test_lmhead_ce_empty_batch(orc):
+    """M = 0: no tokens.  W is still cast (bit-exact against the oracle), the
+    loss is 0, dW keeps what it held, and X, labels and dX arrive as NULL."""
+    from fp8_gemms_b200 import _lib, api
+    d, V = 64, 128
+    _, W, _ = inputs(16, d, V, 11)
+    head = api.LmHeadCE(0, d, V, 32)
+    head.loss.fill_(7.0)                     # the call must write the 0
+    dW = torch.full((V, d), 0.5, dtype=torch.float32, device="cuda")
+    loss, dX, _ = head(torch.empty(0, d, dtype=torch.bfloat16, device="cuda"), W.cuda(),
+                       torch.empty(0, dtype=torch.int32, device="cuda"), dW=dW)
+    torch.cuda.synchronize()
+    assert _lib.lm_get_error()[0] == 0
+    assert float(loss) == 0.0 and dX.shape == (0, d)
+    assert bool((dW == 0.5).all())
+    ref = cast_ref(orc, synthetic.bits_u16(W), 0)
+    assert np.array_equal(u8(head.view("Wq")), ref["q"])
+
+
 def test_invalid_label_is_reported_not_read(orc):
     from fp8_gemms_b200 import _lib
     M, d, V = 32, 64, 128
