@@ -268,3 +268,49 @@ def test_full_size_step_is_deterministic_over_repeats(api):
         names = ("Y", "dX", "dW_up", "dW_down", "hq", "dHq", "scales", "bwd scales")
         for name, a, b in zip(names, first, outs):
             assert torch.equal(a, b), f"{name} differs at repeat {it}"
+
+
+@pytest.mark.slow
+def test_mlp_forward_beyond_2_31_elements(orc, api):
+    """M = 196,608 tokens, so H and h hold 2.4e9 elements, more than 2^31: the
+    forward in bench.py's launch configuration (h cast by the down GEMM's side
+    warps), checked on rows on both sides of element 2^31 and at the end.
+    Whole-tensor amax of X and of h bit-exact; on the sampled rows X's and h's
+    codes bit-exact, H and Y within the GEMM bar."""
+    from fp8_gemms_b200 import _lib
+    M, d, f = 196608, 3072, 12288
+    assert M * f > 2 ** 31
+    X = synthetic.normal_bf16((M, d), 1.0, 7, 0, device="cuda")
+    Wu = synthetic.normal_bf16((f, d), 0.02, 7, 1).cuda()
+    Wd = synthetic.normal_bf16((d, f), 0.02, 7, 2).cuda()
+    mlp = api.Relu2Mlp(M, d, f)
+    Y = mlp.forward(X, Wu, Wd)
+    torch.cuda.synchronize()
+    assert _lib.lm_get_error()[0] == 0
+    edge = 2 ** 31 // f                       # the row holding element 2^31 of H
+    rows = np.array([0, 1, edge - 1, edge, edge + 1, M // 2, M - 2, M - 1])
+    sc = mlp.view("scales").cpu().numpy()
+    xb = synthetic.bits_u16(X.cpu())
+    s_x, inv_x = orc.scale(orc.amax(xb), E4M3)
+    assert sc[0, 0] == orc.amax(xb) and sc[0, 1] == s_x and sc[0, 2] == inv_x
+    Xq_rows = u8(mlp.view("Xq")[torch.as_tensor(rows, device="cuda")])
+    q_ref, _ = orc.cast(np.ascontiguousarray(xb[rows]), E4M3, s_x, want_qT=False)
+    assert np.array_equal(Xq_rows, q_ref)
+    del xb
+    for name, key, si in [("W_up", "Wuq", 1), ("W_down", "Wdq", 2)]:
+        ref = cast_ref(orc, synthetic.bits_u16((Wu if si == 1 else Wd).cpu()), E4M3)
+        assert sc[si, 0] == ref["amax"] and np.array_equal(u8(mlp.view(key)), ref["q"]), name
+    H = u16(mlp.view("H"))
+    Href, _ = orc.gemm(u8(mlp.view("Xq")), E4M3, u8(mlp.view("Wuq")), E4M3, sc[0, 2], sc[1, 2],
+                       orc.EPI_RELU2_FWD, rows=rows)
+    assert_close(H[rows], Href, "H")
+    assert sc[3, 0] == orc.amax(H, relu2_input=True)
+    s_h, inv_h = orc.scale(sc[3, 0], E4M3)
+    assert sc[3, 1] == s_h and sc[3, 2] == inv_h
+    hq_ref, _ = orc.cast(np.ascontiguousarray(H[rows]), E4M3, s_h, relu2_input=True,
+                         want_qT=False)
+    del H
+    hq = u8(mlp.view("hq"))
+    assert np.array_equal(hq[rows], hq_ref)
+    Yref, _ = orc.gemm(hq, E4M3, u8(mlp.view("Wdq")), E4M3, sc[3, 2], sc[2, 2], rows=rows)
+    assert_close(u16(Y)[rows], Yref, "Y")
