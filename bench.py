@@ -459,7 +459,6 @@ def run_gpu(args):
     last = (Ke - 1) % 2
     assert torch.equal(pinned_out[last]["dX"][:4].float(), dbuf[last]["dX"][:4].cpu().float())
 
-
     peaks = read_peaks()
     value = job_tflops(world, K, STEP_FLOPS, total_ms)
     # the tensor pipe's dense FP8 peak at the SM clock sampled during the timed
