@@ -465,4 +465,6 @@ def lmhead_ce(X, W, labels, chunk, softcap=15.0):
         cdl = amax_scale_cast(dl, E5M2)
         dX[c0:c1], _ = gemm(cdl["q"], E5M2, cw["qT"], E4M3, cdl["inv_scale"], cw["inv_scale"])
         gemm_accum_f32(cdl["qT"], E5M2, XqT, E4M3, cdl["inv_scale"], isx, dW)
-    return losses.mean(), dX, dW, losses
+    # no tokens: the mean over an empty batch is taken as 0 (a reading; the
+    # pages only ever average over a full micro-batch)
+    return (losses.mean() if M else 0.0), dX, dW, losses

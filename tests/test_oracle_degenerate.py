@@ -49,3 +49,13 @@ def test_no_tokens_give_empty_outputs_and_zero_weight_gradients(orc):
     assert bw["dX"].shape == (0, 32)
     assert bw["dW_up"].shape == (64, 32) and not (bw["dW_up"] & 0x7FFF).any()
     assert bw["dW_down"].shape == (32, 64) and not (bw["dW_down"] & 0x7FFF).any()
+
+
+def test_lm_head_with_no_tokens(orc):
+    """M = 0: dW is a sum over no tokens, so zero; dX has no rows; the mean
+    loss over no tokens is taken as 0 (the library's reading)."""
+    W = synthetic.bits_u16(synthetic.normal_bf16((48, 32), 0.02, 4, 1))
+    X = np.zeros((0, 32), np.uint16)
+    loss, dX, dW, rows = orc.lmhead_ce(X, W, np.zeros(0, np.int32), chunk=16)
+    assert loss == 0.0 and dX.shape == (0, 32) and rows.shape == (0,)
+    assert dW.shape == (48, 32) and not dW.any()
